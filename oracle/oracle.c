@@ -1,0 +1,438 @@
+/*
+ * oracle.c -- plain, slow CPU restatement of block-scaled weight quantization with a
+ * searched E4M3 block scale.
+ *
+ * TEST INFRASTRUCTURE ONLY. The test suite, the smoke check and the benchmark's CPU
+ * baseline are its only callers. It shares no code, header, table or constant with the
+ * CUDA library, and the library never calls it.
+ *
+ * Sources (page title, section):
+ *  - "Is Finer Better? The Limits of Microscaling Formats in LLMs", sec. 2.1
+ *    (Microscaling formats): s = Q_scale(xmax / C), q_i = Q_elem(x_i / s), x^ = s * q.
+ *    Appendix F.3: the smallest positive E4M3 value 2^-9 (subnormals included); a block
+ *    whose scale rounds to zero has every element rounded to zero.
+ *  - qwantize "Results", section "INT8 (FP8 E4M3 scales)": symmetric INT8 in [-127, 127],
+ *    the per-block amax stored as E4M3, effective scale amax_fp8 / 127 divided in float32;
+ *    the bounded search around the naive amax snap.
+ *  - qwantize "Results", sections "NVFP4 (FP8 E4M3 scales)" and "Correctness notes":
+ *    naive / SSE-optimal / H-optimal; FP4 decisions at the 0.75, 1.75, 3.5 boundaries;
+ *    section "Exotic Scales": the E2M1 codebook {0, 0.5, 1, 1.5, 2, 3, 4, 6} and the count
+ *    of 126 positive E4M3 values.
+ *  - "quantization_algorithms.txt", section 1 (Activation-weighted scale search): the
+ *    diagonal objective sum_ij h_j (w_ij - s Q(w_ij / s))^2 with h_j = E[x_j^2]; a
+ *    logarithmic grid of tile scales; section 2: nearest-E4M3 projection by binary search
+ *    in a sorted float32 table of the finite E4M3 values.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - every rounding onto a grid is round-to-nearest, ties to the even code, saturating at
+ *    the largest finite value; the division w / s is IEEE float32 (C float division);
+ *  - the block error of one candidate is accumulated in double, in element order, as
+ *    e += c_j * (d * d) with d = (double)w - (double)fl32(s * q);
+ *  - candidate ties go to the lowest candidate index (the smallest scale);
+ *  - a naive scale that rounds to E4M3 code 0 gives all-zero magnitudes (sign bits kept);
+ *    the search never picks code 0; a window around code 0 is [1, w].
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared oracle.c -lm
+ * (no fused multiply-add: every product and sum above is a separately rounded step).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ----------------------------------------------------------------------------------
+ * Number formats, decoded from their bit fields.
+ * ---------------------------------------------------------------------------------- */
+
+/* E4M3 ("FN": no infinities; S.1111.111 is NaN): 4 exponent bits with bias 7, 3 mantissa
+ * bits. Exponent field 0 encodes subnormals m/8 * 2^-6, otherwise (1 + m/8) * 2^(e-7). */
+double orc_e4m3_value(int code)
+{
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* E2M1: 2 exponent bits with bias 1, 1 mantissa bit. Exponent field 0 encodes m * 0.5. */
+double orc_e2m1_value(int code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? 0.5 * (double)m : ldexp(1.0 + (double)m / 2.0, e - 1);
+    return s ? -v : v;
+}
+
+/* Sorted tables of the non-negative grid values; the table index is the magnitude code
+ * (for E4M3 and E2M1 the codes of positive values increase with the value). */
+static float T_E4M3[127];   /* codes 0x00 .. 0x7E: 0, 2^-9, ..., 448 */
+static float T_E2M1[8];     /* codes 0 .. 7: 0, 0.5, ..., 6 */
+static float T_INT[128];    /* 0 .. 127 */
+
+__attribute__((constructor)) static void orc_init_tables(void)
+{
+    for (int c = 0; c < 127; ++c) T_E4M3[c] = (float)orc_e4m3_value(c);
+    for (int c = 0; c < 8; ++c) T_E2M1[c] = (float)orc_e2m1_value(c);
+    for (int c = 0; c < 128; ++c) T_INT[c] = (float)c;
+}
+
+/* Copies of the tables, for the self-tests. */
+void orc_e4m3_table(float *out127) { memcpy(out127, T_E4M3, sizeof T_E4M3); }
+void orc_e2m1_table(float *out8) { memcpy(out8, T_E2M1, sizeof T_E2M1); }
+
+/* Index of the table value nearest to z >= 0 (tab ascending, tab[0] == 0). Equidistant
+ * values go to the even index; z at or above the last value (and +inf) saturates to the
+ * last index; zero and NaN give 0. */
+static int nearest_rne(const float *tab, int n, float z)
+{
+    if (!(z > 0.0f)) return 0;
+    if (z >= tab[n - 1]) return n - 1;
+    int lo = 0, hi = n - 1;            /* tab[lo] <= z < tab[hi] */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (tab[mid] <= z) lo = mid; else hi = mid;
+    }
+    double dlo = (double)z - (double)tab[lo];
+    double dhi = (double)tab[hi] - (double)z;
+    if (dlo < dhi) return lo;
+    if (dhi < dlo) return hi;
+    return (lo % 2 == 0) ? lo : hi;
+}
+
+/* Round-to-nearest-even onto the non-negative E4M3 grid with saturation: the code. */
+int orc_e4m3_rne_code(float x) { return nearest_rne(T_E4M3, 127, x); }
+/* Round-to-nearest-even onto the E2M1 magnitudes with saturation at 6: the code 0..7. */
+int orc_e2m1_rne_code(float x) { return nearest_rne(T_E2M1, 8, x); }
+/* Round-to-nearest-even onto 0..127. */
+int orc_int127_rne(float x) { return nearest_rne(T_INT, 128, x); }
+
+/* ----------------------------------------------------------------------------------
+ * Element access.
+ * ---------------------------------------------------------------------------------- */
+
+enum { ORC_F32 = 0, ORC_BF16 = 1 };
+enum { ORC_NVFP4 = 0, ORC_INT8 = 1, ORC_E4M3 = 2 };
+enum { ORC_NAIVE = 0, ORC_SSE = 1, ORC_HOPT = 2 };
+
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+static float elem(const void *base, int dtype, int64_t ld, int64_t i, int64_t j)
+{
+    if (dtype == ORC_BF16) return bf16_to_float(((const uint16_t *)base)[i * ld + j]);
+    return ((const float *)base)[i * ld + j];
+}
+
+/* ----------------------------------------------------------------------------------
+ * h_j = E[x_j^2] over the rows of X ("quantization_algorithms.txt", section 1).
+ * The sum of squares is taken in double, then divided by R and rounded to float once.
+ * ---------------------------------------------------------------------------------- */
+void orc_act_sqsum(const void *X, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                   int64_t row0, int64_t row1, double *colsum)
+{
+    for (int64_t j = 0; j < cols; ++j) colsum[j] = 0.0;
+    for (int64_t r = row0; r < row1 && r < rows; ++r)
+        for (int64_t j = 0; j < cols; ++j) {
+            double x = (double)elem(X, dtype, ld, r, j);
+            colsum[j] += x * x;
+        }
+}
+
+void orc_act_sqmean(const void *X, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                    float *h)
+{
+    double *s = (double *)malloc(sizeof(double) * (size_t)(cols > 0 ? cols : 1));
+    orc_act_sqsum(X, dtype, rows, cols, ld, 0, rows, s);
+    for (int64_t j = 0; j < cols; ++j) h[j] = rows > 0 ? (float)(s[j] / (double)rows) : 0.0f;
+    free(s);
+}
+
+/* ----------------------------------------------------------------------------------
+ * One-dimensional blocks (NVFP4 and INT8): B contiguous weights of one row share one
+ * E4M3 scale byte.
+ * ---------------------------------------------------------------------------------- */
+
+/* The magnitude code of element w at candidate scale code c, and its dequantised value
+ * fl32(scale * q) (without sign). NVFP4: scale = E4M3(c), q = E2M1 nearest of
+ * fl32(|w| / scale). INT8: scale = fl32(E4M3(c) / 127), q = nearest integer in [0, 127]
+ * of fl32(|w| / scale). Scale code 0 (a naive snap to zero) gives q = 0. */
+static int project(int fmt, int c, float w, float *wq_abs)
+{
+    float a = fabsf(w);
+    if (c == 0) { *wq_abs = 0.0f; return 0; }
+    if (fmt == ORC_NVFP4) {
+        float s = T_E4M3[c];
+        float z = a / s;
+        int q = nearest_rne(T_E2M1, 8, z);
+        *wq_abs = s * T_E2M1[q];
+        return q;
+    } else {
+        float s = T_E4M3[c] / 127.0f;
+        float z = a / s;
+        int q = nearest_rne(T_INT, 128, z);
+        *wq_abs = (float)q * s;
+        return q;
+    }
+}
+
+/* Exported for the exhaustive projection self-tests. */
+int orc_project(int fmt, int c, float w, float *wq_abs) { return project(fmt, c, w, wq_abs); }
+
+void orc_project_many(int fmt, int c, const float *w, int64_t count, uint8_t *q, float *wq_abs)
+{
+    for (int64_t i = 0; i < count; ++i) q[i] = (uint8_t)project(fmt, c, w[i], &wq_abs[i]);
+}
+
+/* Block error at candidate c: sum_j c_j (w_j - wq_j)^2 in double, element order. */
+static double block_error(int fmt, int c, const float *w, const float *cw, int B)
+{
+    double e = 0.0;
+    for (int j = 0; j < B; ++j) {
+        float wq_abs;
+        project(fmt, c, w[j], &wq_abs);
+        float wq = copysignf(wq_abs, w[j]);
+        double d = (double)w[j] - (double)wq;
+        e += (double)cw[j] * (d * d);
+    }
+    return e;
+}
+
+/* Naive snap: NVFP4 E4M3(fl32(amax / 6)); INT8 E4M3(amax) (the stored amax). */
+static int naive_code(int fmt, float amax)
+{
+    if (fmt == ORC_NVFP4) return nearest_rne(T_E4M3, 127, amax / 6.0f);
+    return nearest_rne(T_E4M3, 127, amax);
+}
+
+int orc_naive_code(int fmt, float amax) { return naive_code(fmt, amax); }
+
+/*
+ * Quantize rows [row0, row1) of W [n, k] (leading dimension ld) in blocks of B along k.
+ * fmt: ORC_NVFP4 or ORC_INT8. mode: ORC_NAIVE, ORC_SSE or ORC_HOPT (h required).
+ * window < 0: every positive E4M3 scale code 1..126; otherwise codes [c0-window,
+ * c0+window] clipped to [1, 126], c0 the naive code.
+ * Outputs (row-major, all n rows addressable): codes -- NVFP4 [n][k/2] with element 2i in
+ * the low nibble, nibble = sign << 3 | E2M1 code; INT8 [n][k] two's complement.
+ * scales [n][k/B] E4M3 codes. Optional (may be NULL): best / second [n][k/B] -- the
+ * smallest and the second-smallest candidate error (second = +inf with one candidate;
+ * both NaN in naive mode), naive [n][k/B] the naive code.
+ * Returns 0, or -1 on bad arguments.
+ */
+int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
+                        const float *h, int fmt, int mode, int B, int window,
+                        int64_t row0, int64_t row1, uint8_t *codes, uint8_t *scales,
+                        double *best, double *second, int32_t *naive)
+{
+    if (B <= 0 || k % B != 0 || (fmt != ORC_NVFP4 && fmt != ORC_INT8)) return -1;
+    if (mode == ORC_HOPT && h == NULL) return -1;
+    int64_t kb = k / B;
+    float *w = (float *)malloc(sizeof(float) * (size_t)B);
+    float *cw = (float *)malloc(sizeof(float) * (size_t)B);
+    for (int64_t i = row0; i < row1 && i < n; ++i) {
+        for (int64_t b = 0; b < kb; ++b) {
+            int64_t j0 = b * B;
+            float amax = 0.0f;
+            for (int j = 0; j < B; ++j) {
+                w[j] = elem(W, dtype, ld, i, j0 + j);
+                cw[j] = (mode == ORC_HOPT) ? h[j0 + j] : 1.0f;
+                if (fabsf(w[j]) > amax) amax = fabsf(w[j]);
+            }
+            int c0 = naive_code(fmt, amax);
+            int cbest = c0;
+            double e1 = NAN, e2 = NAN;
+            if (mode != ORC_NAIVE) {
+                int lo = 1, hi = 126;
+                if (window >= 0) {
+                    lo = c0 - window < 1 ? 1 : c0 - window;
+                    hi = c0 + window > 126 ? 126 : c0 + window;
+                    if (c0 == 0) { lo = 1; hi = window < 1 ? 1 : window; }
+                }
+                e1 = INFINITY; e2 = INFINITY; cbest = lo;
+                for (int c = lo; c <= hi; ++c) {
+                    double e = block_error(fmt, c, w, cw, B);
+                    if (e < e1) { e2 = e1; e1 = e; cbest = c; }
+                    else if (e < e2) e2 = e;
+                }
+            }
+            scales[i * kb + b] = (uint8_t)cbest;
+            if (best) best[i * kb + b] = e1;
+            if (second) second[i * kb + b] = e2;
+            if (naive) naive[i * kb + b] = c0;
+            for (int j = 0; j < B; ++j) {
+                float wq_abs;
+                int q = project(fmt, cbest, w[j], &wq_abs);
+                int neg = signbit(w[j]) ? 1 : 0;
+                if (fmt == ORC_NVFP4) {
+                    uint8_t nib = (uint8_t)((neg << 3) | q);
+                    uint8_t *p = &codes[i * (k / 2) + (j0 + j) / 2];
+                    if (((j0 + j) & 1) == 0) *p = (uint8_t)((*p & 0xF0) | nib);
+                    else *p = (uint8_t)((*p & 0x0F) | (nib << 4));
+                } else {
+                    int v = neg ? -q : q;
+                    ((int8_t *)codes)[i * k + j0 + j] = (int8_t)v;
+                }
+            }
+        }
+    }
+    free(w);
+    free(cw);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------------------
+ * E4M3 elements on T x T tiles with one float32 scale per tile, searched on a
+ * logarithmic grid ("quantization_algorithms.txt", section 1).
+ * base = fl32(amax_tile / 448); grid g_p = fl32(2^(lo + (hi - lo) p / (P - 1))),
+ * p = 0..P-1 (computed in double, rounded once); candidate s_p = fl32(base * g_p).
+ * Naive mode: s = base. A tile whose scale is 0 gets zero magnitudes (sign bits kept);
+ * a candidate scale that underflows to 0 is skipped.
+ * ---------------------------------------------------------------------------------- */
+
+static int e4m3_elem_code(float a, float s, float *wq_abs)
+{
+    if (s == 0.0f) { *wq_abs = 0.0f; return 0; }
+    float z = a / s;
+    int q = nearest_rne(T_E4M3, 127, z);
+    *wq_abs = s * T_E4M3[q];
+    return q;
+}
+
+int orc_project_e4m3(float w, float s, float *wq_abs) { return e4m3_elem_code(fabsf(w), s, wq_abs); }
+
+void orc_project_e4m3_many(float s, const float *w, int64_t count, uint8_t *q, float *wq_abs)
+{
+    for (int64_t i = 0; i < count; ++i) q[i] = (uint8_t)e4m3_elem_code(fabsf(w[i]), s, &wq_abs[i]);
+}
+
+void orc_log_grid(int P, double lo, double hi, float *g)
+{
+    for (int p = 0; p < P; ++p)
+        g[p] = (float)exp2(lo + (hi - lo) * (double)p / (double)(P - 1));
+}
+
+/*
+ * Tiles of T rows x T columns; tile rows [trow0, trow1). codes [n][k] bytes
+ * (sign << 7 | E4M3 code), scales [n/T][k/T] float. best / second / grid_index optional:
+ * [n/T][k/T] (grid_index -1 in naive mode).
+ */
+int orc_quantize_tiles(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
+                       const float *h, int mode, int T, int P, double lo, double hi,
+                       int64_t trow0, int64_t trow1, uint8_t *codes, float *scales,
+                       double *best, double *second, int32_t *grid_index)
+{
+    if (T <= 0 || n % T != 0 || k % T != 0 || P < 2 || P > 4096) return -1;
+    if (mode == ORC_HOPT && h == NULL) return -1;
+    int64_t tn = n / T, tk = k / T;
+    float *g = (float *)malloc(sizeof(float) * (size_t)P);
+    orc_log_grid(P, lo, hi, g);
+    for (int64_t ti = trow0; ti < trow1 && ti < tn; ++ti) {
+        for (int64_t tj = 0; tj < tk; ++tj) {
+            int64_t i0 = ti * T, j0 = tj * T;
+            float amax = 0.0f;
+            for (int64_t i = 0; i < T; ++i)
+                for (int64_t j = 0; j < T; ++j) {
+                    float a = fabsf(elem(W, dtype, ld, i0 + i, j0 + j));
+                    if (a > amax) amax = a;
+                }
+            float base = amax / 448.0f;
+            float s = base;
+            int pbest = -1;
+            double e1 = NAN, e2 = NAN;
+            if (mode != ORC_NAIVE && base > 0.0f) {
+                e1 = INFINITY; e2 = INFINITY;
+                for (int p = 0; p < P; ++p) {
+                    float sp = base * g[p];
+                    if (sp == 0.0f) continue;
+                    double e = 0.0;
+                    for (int64_t i = 0; i < T; ++i)
+                        for (int64_t j = 0; j < T; ++j) {
+                            float w = elem(W, dtype, ld, i0 + i, j0 + j);
+                            float wq_abs;
+                            e4m3_elem_code(fabsf(w), sp, &wq_abs);
+                            float wq = copysignf(wq_abs, w);
+                            double d = (double)w - (double)wq;
+                            double c = (mode == ORC_HOPT) ? (double)h[j0 + j] : 1.0;
+                            e += c * (d * d);
+                        }
+                    if (e < e1) { e2 = e1; e1 = e; pbest = p; }
+                    else if (e < e2) e2 = e;
+                }
+                s = pbest >= 0 ? base * g[pbest] : 0.0f;
+            }
+            scales[ti * tk + tj] = s;
+            if (best) best[ti * tk + tj] = e1;
+            if (second) second[ti * tk + tj] = e2;
+            if (grid_index) grid_index[ti * tk + tj] = pbest;
+            for (int64_t i = 0; i < T; ++i)
+                for (int64_t j = 0; j < T; ++j) {
+                    float w = elem(W, dtype, ld, i0 + i, j0 + j);
+                    float wq_abs;
+                    int q = e4m3_elem_code(fabsf(w), s, &wq_abs);
+                    codes[(i0 + i) * k + j0 + j] = (uint8_t)((signbit(w) ? 0x80 : 0) | q);
+                }
+        }
+    }
+    free(g);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------------------
+ * Dequantisation and error metrics (qwantize "Results": weight error
+ * ||Q(W) - W||_F / ||W||_F; the h-weighted error is the diagonal objective itself).
+ * ---------------------------------------------------------------------------------- */
+
+/* W^ [n][k] float from codes and scales. fmt as above; B the block (tile edge for E4M3). */
+int orc_dequant(const uint8_t *codes, const void *scales, int fmt, int B, int64_t n,
+                int64_t k, float *out)
+{
+    if (B <= 0 || k % B != 0) return -1;
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < k; ++j) {
+            float v;
+            if (fmt == ORC_NVFP4) {
+                uint8_t byte = codes[i * (k / 2) + j / 2];
+                int nib = (j & 1) ? (byte >> 4) : (byte & 15);
+                float s = T_E4M3[((const uint8_t *)scales)[i * (k / B) + j / B]];
+                v = s * T_E2M1[nib & 7];
+                if (nib & 8) v = -v;
+            } else if (fmt == ORC_INT8) {
+                int q = ((const int8_t *)codes)[i * k + j];
+                float s = T_E4M3[((const uint8_t *)scales)[i * (k / B) + j / B]] / 127.0f;
+                v = (float)(q < 0 ? -q : q) * s;
+                if (q < 0) v = -v;
+            } else {
+                uint8_t c = codes[i * k + j];
+                float s = ((const float *)scales)[(i / B) * (k / B) + j / B];
+                v = s * T_E4M3[c & 0x7F];
+                if (c & 0x80) v = -v;
+            }
+            out[i * k + j] = v;
+        }
+    return 0;
+}
+
+/* sums[0] = sum (w - w^)^2, sums[1] = sum w^2, sums[2] = sum h_j (w - w^)^2,
+ * sums[3] = sum h_j w^2 (both 0 when h is NULL); doubles, row-major order. */
+void orc_error_sums(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
+                    const float *What, const float *h, double *sums)
+{
+    double s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < k; ++j) {
+            double w = (double)elem(W, dtype, ld, i, j);
+            double d = w - (double)What[i * k + j];
+            s0 += d * d;
+            s1 += w * w;
+            if (h) {
+                s2 += (double)h[j] * (d * d);
+                s3 += (double)h[j] * (w * w);
+            }
+        }
+    sums[0] = s0; sums[1] = s1; sums[2] = s2; sums[3] = s3;
+}

@@ -1,0 +1,52 @@
+"""Planted mistakes: each variant below copies the oracle's C source, injects one plausible
+bug (a dropped term, a wrong tie rule, a transposed index, ...), builds it on the CPU and
+runs the pin suite against it. Every variant must make the pins fail: this shows the pins
+are strong enough to catch that class of mistake."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+MUTANTS = {
+    "drop_h_weight": ("e += (double)cw[j] * (d * d);", "e += (d * d);"),
+    "ties_always_up": ("return (lo % 2 == 0) ? lo : hi;", "return hi;"),
+    "naive_divisor": ("return nearest_rne(T_E4M3, 127, amax / 6.0f);",
+                      "return nearest_rne(T_E4M3, 127, amax / 4.0f);"),
+    "candidate_ties_high": ("if (e < e1) { e2 = e1; e1 = e; cbest = c; }",
+                            "if (e <= e1) { e2 = e1; e1 = e; cbest = c; }"),
+    "int8_divisor": ("float s = T_E4M3[c] / 127.0f;\n        float z = a / s;",
+                     "float s = T_E4M3[c] / 128.0f;\n        float z = a / s;"),
+    "sign_dropped": ("int neg = signbit(w[j]) ? 1 : 0;", "int neg = 0;"),
+    "tile_h_by_row": ("double c = (mode == ORC_HOPT) ? (double)h[j0 + j] : 1.0;",
+                      "double c = (mode == ORC_HOPT) ? (double)h[i0 + i] : 1.0;"),
+    "window_short": ("hi = c0 + window > 126 ? 126 : c0 + window;",
+                     "hi = c0 + window > 126 ? 126 : c0 + window - 1;"),
+    "mean_over_r_minus_1": ("(float)(s[j] / (double)rows)", "(float)(s[j] / (double)(rows - 1))"),
+    "e2m1_exponent": ("ldexp(1.0 + (double)m / 2.0, e - 1)", "ldexp(1.0 + (double)m / 2.0, e)"),
+    "nibble_order": ("if (((j0 + j) & 1) == 0) *p", "if (((j0 + j) & 1) == 1) *p"),
+    "e4m3_subnormal": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
+    "dequant_not_rounded": ("float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - (double)wq;",
+                            "float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - 1.0000001 * (double)wq;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mut = tmp_path / "oracle_mut.c"
+    mut.write_text(src.replace(old, new))
+    so = tmp_path / "liboracle_mut.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-o",
+                    str(so), str(mut), "-lm"], check=True)
+    env = dict(os.environ, MXQ_ORACLE_LIB=str(so))
+    res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                          os.path.join(HERE, "test_oracle_pins.py")], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=600)
+    assert res.returncode != 0, f"pins did not catch planted mistake {name}:\n{res.stdout[-2000:]}"
