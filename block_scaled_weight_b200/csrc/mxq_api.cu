@@ -1,0 +1,300 @@
+// mxq_api.cu -- the extern "C" boundary of libmxq.so: host-side validation, workspace
+// queries and kernel launches. See include/mxq.h for the contract of every call.
+#include "../../include/mxq.h"
+#include "mxq_internal.h"
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+namespace mxq {
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+}  // namespace mxq
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+mxq_status fail(mxq_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+mxq_status fail(mxq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+mxq_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return MXQ_OK;
+  return fail(MXQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+int elsize(int32_t dt) { return dt == MXQ_BF16 ? 2 : 4; }
+
+mxq_status check_matrix(const void* X, int32_t dt, int64_t rows, int64_t cols, int64_t ld,
+                        const char* name) {
+  if (dt != MXQ_BF16 && dt != MXQ_F32) return fail(MXQ_ERR_DTYPE, "%s: dtype %d", name, dt);
+  if (rows < 0 || cols < 0) return fail(MXQ_ERR_SHAPE, "%s: negative shape", name);
+  if (ld < cols) return fail(MXQ_ERR_SHAPE, "%s: ld %lld < cols %lld", name, (long long)ld,
+                             (long long)cols);
+  if (rows == 0 || cols == 0) return MXQ_OK;
+  if (!X) return fail(MXQ_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(X, 16)) return fail(MXQ_ERR_ALIGN, "%s not 16-byte aligned", name);
+  if ((ld * elsize(dt)) % 16 != 0)
+    return fail(MXQ_ERR_ALIGN, "%s: ld * element size not a multiple of 16 bytes", name);
+  return MXQ_OK;
+}
+
+mxq_status check_params(const mxq_params* p, int64_t n, int64_t k) {
+  if (!p) return fail(MXQ_ERR_INVALID_ARG, "params is NULL");
+  if (p->mode < MXQ_NAIVE || p->mode > MXQ_HOPT) return fail(MXQ_ERR_INVALID_ARG, "mode %d", p->mode);
+  switch (p->fmt) {
+    case MXQ_FMT_NVFP4:
+      if (p->block != 16 && p->block != 32)
+        return fail(MXQ_ERR_UNSUPPORTED, "NVFP4 block %d (16 or 32)", p->block);
+      if (p->tile_rows != 1) return fail(MXQ_ERR_UNSUPPORTED, "NVFP4 tile_rows must be 1");
+      break;
+    case MXQ_FMT_INT8:
+      if (p->block != 32 && p->block != 64 && p->block != 128 && p->block != 256)
+        return fail(MXQ_ERR_UNSUPPORTED, "INT8 block %d (32, 64, 128 or 256)", p->block);
+      if (p->tile_rows != 1) return fail(MXQ_ERR_UNSUPPORTED, "INT8 tile_rows must be 1");
+      break;
+    case MXQ_FMT_E4M3:
+      if (p->block != 64 || p->tile_rows != 64)
+        return fail(MXQ_ERR_UNSUPPORTED, "E4M3 tiles are 64 x 64");
+      if (p->mode != MXQ_NAIVE) {
+        if (p->log_points < 2 || p->log_points > 256)
+          return fail(MXQ_ERR_INVALID_ARG, "log_points %d (2..256)", p->log_points);
+        if (!std::isfinite(p->log_lo_exp2) || !std::isfinite(p->log_hi_exp2) ||
+            !(p->log_lo_exp2 < p->log_hi_exp2) || std::fabs(p->log_lo_exp2) > 64 ||
+            std::fabs(p->log_hi_exp2) > 64)
+          return fail(MXQ_ERR_INVALID_ARG, "log grid exponents");
+      }
+      if (n % 64 != 0) return fail(MXQ_ERR_SHAPE, "n %% 64 != 0 for E4M3 tiles");
+      break;
+    default:
+      return fail(MXQ_ERR_INVALID_ARG, "fmt %d", p->fmt);
+  }
+  if (p->window < -1) return fail(MXQ_ERR_INVALID_ARG, "window %d", p->window);
+  if (k % p->block != 0) return fail(MXQ_ERR_SHAPE, "k %% block != 0");
+  return MXQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mxq_status_string(mxq_status s) {
+  switch (s) {
+    case MXQ_OK: return "ok";
+    case MXQ_ERR_INVALID_ARG: return "invalid argument";
+    case MXQ_ERR_SHAPE: return "bad shape";
+    case MXQ_ERR_DTYPE: return "unsupported dtype";
+    case MXQ_ERR_ALIGN: return "misaligned pointer or leading dimension";
+    case MXQ_ERR_UNSUPPORTED: return "unsupported combination";
+    case MXQ_ERR_CUDA: return "CUDA error";
+    case MXQ_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* mxq_last_error(void) { return g_err; }
+
+size_t mxq_act_sqmean_workspace(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0) return 0;
+  // the strip width only shapes the grid; the chunk count for bf16 is never smaller
+  const int ch = std::max(mxq::hpass_chunks(rows, cols, MXQ_BF16), mxq::hpass_chunks(rows, cols, MXQ_F32));
+  return (size_t)ch * (size_t)cols * sizeof(double);
+}
+
+static mxq_status act_common(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+                             int64_t ld, void* workspace, size_t ws, double** partial,
+                             int* chunks) {
+  mxq_status s = check_matrix(X, dtype, rows, cols, ld, "X");
+  if (s != MXQ_OK) return s;
+  const int vec = dtype == MXQ_BF16 ? 8 : 4;
+  if (cols % vec != 0) return fail(MXQ_ERR_SHAPE, "cols %% %d != 0", vec);
+  if (rows == 0 || cols == 0) return MXQ_OK;
+  const size_t need = mxq_act_sqmean_workspace(rows, cols);
+  if (!workspace || ws < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws, need);
+  if (!aligned(workspace, 8)) return fail(MXQ_ERR_ALIGN, "workspace not 8-byte aligned");
+  *partial = (double*)workspace;
+  *chunks = mxq::hpass_chunks(rows, cols, dtype);
+  return MXQ_OK;
+}
+
+mxq_status mxq_act_sqmean(const void* X, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                          float* h, void* workspace, size_t workspace_bytes, void* stream) {
+  double* partial = nullptr;
+  int chunks = 0;
+  mxq_status s = act_common(X, dtype, rows, cols, ld, workspace, workspace_bytes, &partial,
+                            &chunks);
+  if (s != MXQ_OK) return s;
+  if (cols == 0) return MXQ_OK;
+  if (!h) return fail(MXQ_ERR_INVALID_ARG, "h is NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rows == 0) return cuda_status(cudaMemsetAsync(h, 0, cols * sizeof(float), st), "memset h");
+  s = cuda_status(mxq::launch_hpass_partial(X, dtype, rows, cols, ld, chunks, partial, st),
+                  "h pass");
+  if (s != MXQ_OK) return s;
+  return cuda_status(mxq::launch_hpass_finalize(partial, chunks, cols, rows, nullptr, h, st),
+                     "h finalize");
+}
+
+mxq_status mxq_act_sqsum(const void* X, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                         double* colsum, void* workspace, size_t workspace_bytes, void* stream) {
+  double* partial = nullptr;
+  int chunks = 0;
+  mxq_status s = act_common(X, dtype, rows, cols, ld, workspace, workspace_bytes, &partial,
+                            &chunks);
+  if (s != MXQ_OK) return s;
+  if (cols == 0) return MXQ_OK;
+  if (!colsum) return fail(MXQ_ERR_INVALID_ARG, "colsum is NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rows == 0)
+    return cuda_status(cudaMemsetAsync(colsum, 0, cols * sizeof(double), st), "memset colsum");
+  s = cuda_status(mxq::launch_hpass_partial(X, dtype, rows, cols, ld, chunks, partial, st),
+                  "h pass");
+  if (s != MXQ_OK) return s;
+  return cuda_status(mxq::launch_hpass_finalize(partial, chunks, cols, 0, colsum, nullptr, st),
+                     "h partial combine");
+}
+
+mxq_status mxq_act_sqmean_finalize(const double* partials, int64_t parts, int64_t cols,
+                                   int64_t total_rows, float* h, void* stream) {
+  if (parts < 0 || cols < 0 || total_rows < 0) return fail(MXQ_ERR_SHAPE, "negative size");
+  if (cols == 0) return MXQ_OK;
+  if (!h || (parts > 0 && !partials)) return fail(MXQ_ERR_INVALID_ARG, "NULL pointer");
+  if (partials && !aligned(partials, 8)) return fail(MXQ_ERR_ALIGN, "partials not 8-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (parts == 0 || total_rows == 0)
+    return cuda_status(cudaMemsetAsync(h, 0, cols * sizeof(float), st), "memset h");
+  return cuda_status(mxq::launch_hpass_finalize(partials, parts, cols, total_rows, nullptr, h, st),
+                     "h finalize");
+}
+
+mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                        const float* h, const mxq_params* p, void* codes, void* scales,
+                        void* stream) {
+  mxq_status s = check_matrix(W, dtype, n, k, ld, "W");
+  if (s != MXQ_OK) return s;
+  s = check_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (n == 0 || k == 0) return MXQ_OK;
+  if (!codes || !scales) return fail(MXQ_ERR_INVALID_ARG, "codes or scales is NULL");
+  if (!aligned(codes, 16)) return fail(MXQ_ERR_ALIGN, "codes not 16-byte aligned");
+  if (p->fmt == MXQ_FMT_E4M3 && !aligned(scales, 4))
+    return fail(MXQ_ERR_ALIGN, "scales not 4-byte aligned");
+  if (p->mode == MXQ_HOPT) {
+    if (!h) return fail(MXQ_ERR_INVALID_ARG, "H-optimal needs h");
+    if (!aligned(h, 16)) return fail(MXQ_ERR_ALIGN, "h not 16-byte aligned");
+  }
+  mxq::QuantArgs a{};
+  a.W = W;
+  a.dtype = dtype;
+  a.n = n;
+  a.k = k;
+  a.ld = ld;
+  a.h = p->mode == MXQ_HOPT ? h : nullptr;
+  a.fmt = p->fmt;
+  a.mode = p->mode;
+  a.block = p->block;
+  a.window = p->window;
+  a.codes = codes;
+  a.scales = scales;
+  a.log_points = p->fmt == MXQ_FMT_E4M3 && p->mode != MXQ_NAIVE ? p->log_points : 0;
+  for (int i = 0; i < a.log_points; ++i) {
+    const double lo = p->log_lo_exp2, hi = p->log_hi_exp2;
+    a.log_grid[i] = (float)std::exp2(lo + (hi - lo) * (double)i / (double)(a.log_points - 1));
+  }
+  return cuda_status(mxq::launch_quantize(a, (cudaStream_t)stream), "quantize");
+}
+
+mxq_status mxq_project(const float* w, int64_t count, int32_t fmt, float scale, uint8_t* q,
+                       void* stream) {
+  if (count < 0) return fail(MXQ_ERR_SHAPE, "negative count");
+  if (fmt < MXQ_FMT_NVFP4 || fmt > MXQ_FMT_E4M3) return fail(MXQ_ERR_INVALID_ARG, "fmt %d", fmt);
+  if (count == 0) return MXQ_OK;
+  if (!w || !q) return fail(MXQ_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(w, 4)) return fail(MXQ_ERR_ALIGN, "w not 4-byte aligned");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return fail(MXQ_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (fmt != MXQ_FMT_E4M3) {
+    // NVFP4 and INT8 scales are E4M3 values: 4 significant bits, 2^-9 .. 448
+    int e = 0;
+    const float m = std::frexp(scale, &e);
+    const float m16 = m * 16.0f;
+    if (scale < 0.001953125f || scale > 448.0f || m16 != std::floor(m16))
+      return fail(MXQ_ERR_INVALID_ARG, "scale is not a positive E4M3 value");
+  }
+  return cuda_status(mxq::launch_project(w, count, fmt, scale, q, (cudaStream_t)stream),
+                     "project");
+}
+
+mxq_status mxq_dequant(const void* codes, const void* scales, const mxq_params* p, int64_t n,
+                       int64_t k, float* out, void* stream) {
+  if (n < 0 || k < 0) return fail(MXQ_ERR_SHAPE, "negative shape");
+  mxq_status s = check_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (n == 0 || k == 0) return MXQ_OK;
+  if (!codes || !scales || !out) return fail(MXQ_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(codes, 16) || !aligned(out, 16) || !aligned(scales, 4))
+    return fail(MXQ_ERR_ALIGN, "codes/out not 16-byte or scales not 4-byte aligned");
+  mxq::DecodeArgs d{codes, scales, p->fmt, p->block, n, k};
+  return cuda_status(mxq::launch_dequant(d, out, (cudaStream_t)stream), "dequant");
+}
+
+size_t mxq_error_workspace(int64_t n, int64_t k) {
+  if (n <= 0 || k <= 0) return 0;
+  return (size_t)mxq::error_partials(n, k) * 4 * sizeof(double);
+}
+
+mxq_status mxq_error(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                     const void* codes, const void* scales, const float* h,
+                     const mxq_params* p, double* sums, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  mxq_status s = check_matrix(W, dtype, n, k, ld, "W");
+  if (s != MXQ_OK) return s;
+  s = check_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (!sums) return fail(MXQ_ERR_INVALID_ARG, "sums is NULL");
+  if (!aligned(sums, 8)) return fail(MXQ_ERR_ALIGN, "sums not 8-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (n == 0 || k == 0) return cuda_status(cudaMemsetAsync(sums, 0, 4 * sizeof(double), st), "memset");
+  if (!codes || !scales) return fail(MXQ_ERR_INVALID_ARG, "codes or scales is NULL");
+  if (!aligned(codes, 16) || !aligned(scales, 4))
+    return fail(MXQ_ERR_ALIGN, "codes not 16-byte or scales not 4-byte aligned");
+  if (h && !aligned(h, 16)) return fail(MXQ_ERR_ALIGN, "h not 16-byte aligned");
+  const size_t need = mxq_error_workspace(n, k);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 8)) return fail(MXQ_ERR_ALIGN, "workspace not 8-byte aligned");
+  mxq::DecodeArgs d{codes, scales, p->fmt, p->block, n, k};
+  return cuda_status(mxq::launch_error(d, W, dtype, ld, h, (double*)workspace,
+                                       mxq::error_partials(n, k), sums, st),
+                     "error");
+}
+
+mxq_status mxq_metrics_from_sums(const double* s, mxq_metrics* out) {
+  if (!s || !out) return fail(MXQ_ERR_INVALID_ARG, "NULL pointer");
+  out->sse = s[0];
+  out->w_sq = s[1];
+  out->hsse = s[2];
+  out->hw_sq = s[3];
+  out->weight_rel = s[1] > 0 ? std::sqrt(s[0] / s[1]) : 0.0;
+  out->h_rel = s[3] > 0 ? std::sqrt(s[2] / s[3]) : 0.0;
+  return MXQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// mxq_internal.h -- launch plumbing shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxq {
+
+// ---- h pass -------------------------------------------------------------------------
+// The activation matrix is cut into column strips of kStripCols and into `chunks` row
+// chunks; one CTA per (strip, chunk) writes double column sums of squares into
+// partial[chunk][cols]. The chunk count depends only on (rows, cols), so the reduction
+// order (and the result) is the same on every run and every device.
+constexpr int kHpassThreads = 256;
+int hpass_chunks(int64_t rows, int64_t cols, int dtype);
+cudaError_t launch_hpass_partial(const void* X, int dtype, int64_t rows, int64_t cols,
+                                 int64_t ld, int chunks, double* partial, cudaStream_t st);
+// out[j] = sum_{p < parts} partial[p][j] (ascending p); if h != nullptr also
+// h[j] = fl32(out[j] / total_rows). Either output may be null.
+cudaError_t launch_hpass_finalize(const double* partial, int64_t parts, int64_t cols,
+                                  int64_t total_rows, double* colsum, float* h, cudaStream_t st);
+
+// ---- quantization ---------------------------------------------------------------------
+struct QuantArgs {
+  const void* W;
+  int dtype;
+  int64_t n, k, ld;
+  const float* h;      // null unless mode == HOPT
+  int fmt, mode, block, window;
+  void* codes;
+  void* scales;
+  int log_points;
+  float log_grid[256];  // E4M3 tiles: g_p
+};
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, uint8_t* q,
+                           cudaStream_t st);
+
+// ---- dequant / error ------------------------------------------------------------------
+struct DecodeArgs {
+  const void* codes;
+  const void* scales;
+  int fmt, block;
+  int64_t n, k;
+};
+cudaError_t launch_dequant(const DecodeArgs& d, float* out, cudaStream_t st);
+int error_partials(int64_t n, int64_t k);
+cudaError_t launch_error(const DecodeArgs& d, const void* W, int dtype, int64_t ld,
+                         const float* h, double* partial, int parts, double* sums,
+                         cudaStream_t st);
+
+int sm_count();
+
+}  // namespace mxq

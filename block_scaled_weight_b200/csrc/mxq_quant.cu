@@ -1,0 +1,637 @@
+// mxq_quant.cu -- fused per-block scale search + quantize (naive / sse / hopt).
+//
+// Definitions ("Is Finer Better? The Limits of Microscaling Formats in LLMs", sec. 2.1;
+// qwantize "Results", INT8 and NVFP4 sections; "quantization_algorithms.txt", sec. 1):
+//   naive  s0 = RNE_E4M3(amax / qmax)  (INT8: the stored amax RNE_E4M3(amax))
+//   sse    argmin_s  sum_j (w_j - fl32(s q_j))^2
+//   hopt   argmin_s  sum_j h_j (w_j - fl32(s q_j))^2,  q_j = RNE_grid(fl32(|w_j| / s))
+// Candidate ties go to the smallest scale.
+//
+// Exactness. The element decisions use exactly the IEEE float32 quotient:
+//  * NVFP4: an E4M3 scale has a significand of at most 4 bits, so |w| / s can never lie
+//    within 2^-29 (relative) of a float32 rounding boundary without being a float32
+//    itself. The quotient is formed as fma(a, r_hi, a * r_lo) with r_hi + r_lo = 1/s to
+//    ~2^-48 (host-computed split of the reciprocal), whose error (~2^-46) is far inside
+//    that gap: the result is the correctly rounded quotient, bit for bit.
+//  * INT8 and E4M3 tiles: __fdiv_rn, the IEEE-rounded division.
+// Candidate errors are accumulated in float32 (packed f32x2 math); with every term
+// non-negative the float32 sum is within gamma = (B + 8) 2^-24 (relative) plus a tiny
+// absolute underflow slack of the exact sum. Any candidate whose lower bound does not
+// exceed the winner's upper bound is re-scored in double exactly as the plain definition
+// orders it (element order, e += c_j * (d * d)), and the smallest double error (lowest
+// index on ties) wins. So NVFP4 and INT8 picks equal the definition's, ties included.
+// E4M3 tiles accumulate float32 terms (3 roundings each) in double: the tile error is
+// within 2e-7 relative, so any pick whose two best errors differ by more than 1e-6
+// relative is exact.
+#include "mxq_common.cuh"
+#include "mxq_internal.h"
+
+#include <cuda_fp16.h>
+
+#include <cmath>
+#include <cstring>
+
+namespace mxq {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// ---------------------------------------------------------------------------------------
+// Per-candidate constants for NVFP4: {s, r_hi, r_lo, s as fp16 bits}. Computed once on
+// the host (double arithmetic), passed by value and staged in shared memory.
+// ---------------------------------------------------------------------------------------
+struct Fp4Table {
+  float4 c[128];
+};
+
+struct Fp4Params {
+  const char* W;
+  int64_t n, k, ld_bytes;
+  const float* h;
+  int window;
+  uint8_t* codes;
+  uint8_t* scales;
+};
+
+template <int B, bool BF16>
+__device__ __forceinline__ void load_block(const char* p, float2 (&a)[B / 2], uint32_t& sgn) {
+  uint32_t wds[BF16 ? B / 2 : B];
+  if constexpr (BF16) {
+#pragma unroll
+    for (int v = 0; v < B / 8; ++v) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(p) + v);
+      wds[4 * v] = x.x; wds[4 * v + 1] = x.y; wds[4 * v + 2] = x.z; wds[4 * v + 3] = x.w;
+    }
+    sgn = 0;
+#pragma unroll
+    for (int i = 0; i < B / 2; ++i) {
+      sgn |= ((wds[i] >> 15) & 1u) << (2 * i);
+      sgn |= (wds[i] >> 31) << (2 * i + 1);
+      a[i] = make_float2(__uint_as_float((wds[i] << 16) & 0x7fffffffu),
+                         __uint_as_float(wds[i] & 0x7fff0000u));
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < B / 4; ++v) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(p) + v);
+      wds[4 * v] = x.x; wds[4 * v + 1] = x.y; wds[4 * v + 2] = x.z; wds[4 * v + 3] = x.w;
+    }
+    sgn = 0;
+#pragma unroll
+    for (int i = 0; i < B / 2; ++i) {
+      sgn |= (wds[2 * i] >> 31) << (2 * i);
+      sgn |= (wds[2 * i + 1] >> 31) << (2 * i + 1);
+      a[i] = make_float2(__uint_as_float(wds[2 * i] & 0x7fffffffu),
+                         __uint_as_float(wds[2 * i + 1] & 0x7fffffffu));
+    }
+  }
+}
+
+template <int B>
+__device__ __forceinline__ void load_h(const float* h, float2 (&c)[B / 2]) {
+#pragma unroll
+  for (int v = 0; v < B / 4; ++v) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(h) + v);
+    c[2 * v] = make_float2(x.x, x.y);
+    c[2 * v + 1] = make_float2(x.z, x.w);
+  }
+}
+
+template <int B>
+__device__ __forceinline__ float block_amax(const float2 (&a)[B / 2]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < B / 2; ++i) m = fmaxf(m, fmaxf(a[i].x, a[i].y));
+  return m;
+}
+
+// fl32(|w| / s) for an E4M3 scale s, from the split reciprocal (see the file header).
+__device__ __forceinline__ float2 fp4_quot(float2 a, float2 rhi, float2 rlo) {
+  return __ffma2_rn(a, rhi, __fmul2_rn(a, rlo));
+}
+
+// Float32 error of one candidate: sum_j c_j (s g_j - a_j)^2 (c_j = 1 for SSE).
+template <int B, bool HOPT>
+__device__ __forceinline__ float fp4_eval(const float2 (&a)[B / 2], const float2 (&na)[B / 2],
+                                          const float2 (&c)[B / 2], float4 t) {
+  const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
+  const uint16_t s_h = (uint16_t)__float_as_uint(t.w);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int p = 0; p < B / 2; ++p) {
+    const float2 x = fp4_quot(a[p], rhi, rlo);
+    const uint32_t g = e2m1x2_to_f16x2(e2m1x2_rn(x.x, x.y));
+    const float2 d = make_float2(fma_h_h_f(lo16(g), s_h, na[p].x), fma_h_h_f(hi16(g), s_h, na[p].y));
+    float2& acc = (p & 1) ? acc1 : acc0;
+    if constexpr (HOPT) {
+      acc = __ffma2_rn(__fmul2_rn(c[p], d), d, acc);
+    } else {
+      acc = __ffma2_rn(d, d, acc);
+    }
+  }
+  return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+}
+
+// Double error of one candidate, in the definition's order: e += c_j * (d * d),
+// d = (double)|w_j| - (double)fl32(s g_j).
+template <int B, bool HOPT>
+__device__ double fp4_exact(const float2 (&a)[B / 2], const float2 (&c)[B / 2], float4 t) {
+  const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
+  double e = 0.0;
+#pragma unroll
+  for (int p = 0; p < B / 2; ++p) {
+    const float2 x = fp4_quot(a[p], rhi, rlo);
+    const uint32_t g = e2m1x2_to_f16x2(e2m1x2_rn(x.x, x.y));
+    const float g0 = __half2float(__ushort_as_half(lo16(g)));
+    const float g1 = __half2float(__ushort_as_half(hi16(g)));
+    const double d0 = (double)a[p].x - (double)__fmul_rn(t.x, g0);
+    const double d1 = (double)a[p].y - (double)__fmul_rn(t.x, g1);
+    const double c0 = HOPT ? (double)c[p].x : 1.0;
+    const double c1 = HOPT ? (double)c[p].y : 1.0;
+    e = __dadd_rn(e, __dmul_rn(c0, __dmul_rn(d0, d0)));
+    e = __dadd_rn(e, __dmul_rn(c1, __dmul_rn(d1, d1)));
+  }
+  return e;
+}
+
+// Packed NVFP4 codes of one block at candidate table entry t (scale code != 0).
+template <int B>
+__device__ __forceinline__ void fp4_emit(const float2 (&a)[B / 2], uint32_t sgn, float4 t,
+                                         bool zero, uint8_t* dst) {
+  const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
+  uint32_t wds[B / 8];
+#pragma unroll
+  for (int i = 0; i < B / 8; ++i) wds[i] = 0;
+#pragma unroll
+  for (int p = 0; p < B / 2; ++p) {
+    uint32_t byte = 0;
+    if (!zero) {
+      const float2 x = fp4_quot(a[p], rhi, rlo);
+      byte = e2m1x2_rn(x.x, x.y);
+    }
+    byte |= ((sgn >> (2 * p)) & 1u) << 3;
+    byte |= ((sgn >> (2 * p + 1)) & 1u) << 7;
+    wds[p / 4] |= byte << (8 * (p % 4));
+  }
+  if constexpr (B == 16) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(wds[0], wds[1]);
+  } else {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+  }
+}
+
+// NVFP4, naive: one thread per block (HBM-bound).
+template <int B, bool BF16>
+__global__ void __launch_bounds__(kThreads)
+k_fp4_naive(Fp4Params P, Fp4Table T) {
+  __shared__ float4 tab[128];
+  for (int i = threadIdx.x; i < 128; i += kThreads) tab[i] = T.c[i];
+  __syncthreads();
+  const int64_t kb = P.k / B, nblocks = P.n * kb;
+  const int elsz = BF16 ? 2 : 4;
+  for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks;
+       b += (int64_t)gridDim.x * kThreads) {
+    const int64_t row = b / kb, jb = b - row * kb;
+    float2 a[B / 2];
+    uint32_t sgn;
+    load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
+    const int c0 = e4m3_rn_code(__fdiv_rn(block_amax<B>(a), 6.0f));
+    fp4_emit<B>(a, sgn, tab[c0], c0 == 0, P.codes + row * (P.k / 2) + jb * (B / 2));
+    P.scales[b] = (uint8_t)c0;
+  }
+}
+
+// NVFP4, SSE / H-optimal search: one thread per block walks every candidate.
+template <int B, bool BF16, bool HOPT>
+__global__ void __launch_bounds__(kThreads)
+k_fp4_search(Fp4Params P, Fp4Table T) {
+  __shared__ float4 tab[128];
+  for (int i = threadIdx.x; i < 128; i += kThreads) tab[i] = T.c[i];
+  __syncthreads();
+  const int64_t kb = P.k / B, nblocks = P.n * kb;
+  const int elsz = BF16 ? 2 : 4;
+  const float gam = (float)(B + 8) * 5.9604645e-8f;  // (B + 8) 2^-24
+  const float lo_f = 1.0f - gam, hi_f = 1.0f + 2.0f * gam;
+  const float slack = 7.3468396e-40f;                // 2^-130: underflow slack
+  for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks;
+       b += (int64_t)gridDim.x * kThreads) {
+    const int64_t row = b / kb, jb = b - row * kb;
+    float2 a[B / 2], na[B / 2], c[B / 2];
+    uint32_t sgn;
+    load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
+#pragma unroll
+    for (int p = 0; p < B / 2; ++p) na[p] = make_float2(-a[p].x, -a[p].y);
+    if constexpr (HOPT) load_h<B>(P.h + jb * B, c);
+    const int c0 = e4m3_rn_code(__fdiv_rn(block_amax<B>(a), 6.0f));
+    int lo = 1, hi = 126;
+    if (P.window >= 0) {
+      lo = max(1, c0 - P.window);
+      hi = min(126, c0 + P.window);
+      if (c0 == 0) { lo = 1; hi = max(1, P.window); }
+    }
+    float m1 = __int_as_float(0x7f800000), m2 = m1;
+    int i1 = lo;
+    for (int cc = lo; cc <= hi; ++cc) {
+      const float e = fp4_eval<B, HOPT>(a, na, c, tab[cc]);
+      if (e < m1) { m2 = m1; m1 = e; i1 = cc; }
+      else if (e < m2) m2 = e;
+    }
+    const float upper = fmaf(m1, hi_f, slack);
+    if (!(m2 * lo_f - slack > upper)) {
+      // A second candidate may tie or beat the float32 winner: re-score in double.
+      double best = __longlong_as_double(0x7ff0000000000000ll);
+      int bi = i1;
+      for (int cc = lo; cc <= hi; ++cc) {
+        const float e = fp4_eval<B, HOPT>(a, na, c, tab[cc]);
+        if (!(e * lo_f - slack > upper)) {
+          const double ed = fp4_exact<B, HOPT>(a, c, tab[cc]);
+          if (ed < best) { best = ed; bi = cc; }
+        }
+      }
+      i1 = bi;
+    }
+    fp4_emit<B>(a, sgn, tab[i1], false, P.codes + row * (P.k / 2) + jb * (B / 2));
+    P.scales[b] = (uint8_t)i1;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// INT8 with E4M3 stored amax: one warp per block, lanes own elements j = lane + 32 t.
+// ---------------------------------------------------------------------------------------
+struct Int8Params {
+  const char* W;
+  int64_t n, k, ld_bytes;
+  const float* h;
+  int B, window;
+  int8_t* codes;
+  uint8_t* scales;
+};
+
+template <int NE, bool BF16>
+__device__ __forceinline__ void load_lane_elems(const char* row, int lane, float (&a)[NE],
+                                                uint32_t& sgn) {
+  sgn = 0;
+#pragma unroll
+  for (int t = 0; t < NE; ++t) {
+    const int j = lane + 32 * t;
+    uint32_t bits;
+    if constexpr (BF16) bits = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(row) + j) << 16;
+    else bits = __float_as_uint(__ldg(reinterpret_cast<const float*>(row) + j));
+    sgn |= (bits >> 31) << t;
+    a[t] = __uint_as_float(bits & 0x7fffffffu);
+  }
+}
+
+__device__ __forceinline__ float int8_q(float a, float s_eff) {
+  return fminf(rintf(__fdiv_rn(a, s_eff)), 127.0f);
+}
+
+template <int NE, bool BF16, int MODE>
+__global__ void __launch_bounds__(kThreads)
+k_int8(Int8Params P) {
+  constexpr int B = 32 * NE;
+  __shared__ float sa[kThreads / 32][B];
+  __shared__ float sc[kThreads / 32][B];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t kb = P.k / B, nblocks = P.n * kb;
+  const int elsz = BF16 ? 2 : 4;
+  const float gam = (float)(NE + 16) * 5.9604645e-8f;
+  const float lo_f = 1.0f - gam, hi_f = 1.0f + 2.0f * gam;
+  const float slack = 7.3468396e-40f;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t b = gw; b < nblocks; b += nw) {
+    const int64_t row = b / kb, jb = b - row * kb;
+    const char* rp = P.W + row * P.ld_bytes + jb * B * elsz;
+    float a[NE], c[NE];
+    uint32_t sgn;
+    load_lane_elems<NE, BF16>(rp, lane, a, sgn);
+#pragma unroll
+    for (int t = 0; t < NE; ++t) c[t] = (MODE == 2) ? __ldg(P.h + jb * B + lane + 32 * t) : 1.0f;
+    float amax = 0.f;
+#pragma unroll
+    for (int t = 0; t < NE; ++t) amax = fmaxf(amax, a[t]);
+    amax = warp_max(amax);
+    const int c0 = e4m3_rn_code(amax);
+    int best = c0;
+    if (MODE != 0) {
+      int lo = max(1, c0 - P.window), hi = min(126, c0 + P.window);
+      if (P.window < 0) { lo = 1; hi = 126; }
+      else if (c0 == 0) { lo = 1; hi = max(1, P.window); }
+      float m1 = __int_as_float(0x7f800000), m2 = m1;
+      int i1 = lo;
+      for (int cc = lo; cc <= hi; ++cc) {
+        const float s_eff = __fdiv_rn(e4m3_pos(cc), 127.0f);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < NE; ++t) {
+          const float wq = __fmul_rn(int8_q(a[t], s_eff), s_eff);
+          const float d = __fsub_rn(a[t], wq);
+          if (t & 1) acc.y = fmaf(__fmul_rn(c[t], d), d, acc.y);
+          else acc.x = fmaf(__fmul_rn(c[t], d), d, acc.x);
+        }
+        const float e = warp_sum(acc.x + acc.y);
+        if (e < m1) { m2 = m1; m1 = e; i1 = cc; }
+        else if (e < m2) m2 = e;
+      }
+      const float upper = fmaf(m1, hi_f, slack);
+      if (!(m2 * lo_f - slack > upper)) {
+        // Rare: re-score the candidates in the band in double, element order, on lane 0.
+#pragma unroll
+        for (int t = 0; t < NE; ++t) {
+          sa[wid][lane + 32 * t] = a[t];
+          sc[wid][lane + 32 * t] = c[t];
+        }
+        __syncwarp();
+        double bestd = __longlong_as_double(0x7ff0000000000000ll);
+        int bi = i1;
+        for (int cc = lo; cc <= hi; ++cc) {
+          const float s_eff = __fdiv_rn(e4m3_pos(cc), 127.0f);
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int t = 0; t < NE; ++t) {
+            const float wq = __fmul_rn(int8_q(a[t], s_eff), s_eff);
+            const float d = __fsub_rn(a[t], wq);
+            if (t & 1) acc.y = fmaf(__fmul_rn(c[t], d), d, acc.y);
+            else acc.x = fmaf(__fmul_rn(c[t], d), d, acc.x);
+          }
+          const float e = warp_sum(acc.x + acc.y);
+          if (!(e * lo_f - slack > upper)) {
+            double ed = 0.0;
+            if (lane == 0) {
+              for (int j = 0; j < B; ++j) {
+                const float aj = sa[wid][j];
+                const float wq = __fmul_rn(int8_q(aj, s_eff), s_eff);
+                const double d = (double)aj - (double)wq;
+                const double cj = (MODE == 2) ? (double)sc[wid][j] : 1.0;
+                ed = __dadd_rn(ed, __dmul_rn(cj, __dmul_rn(d, d)));
+              }
+            }
+            ed = __shfl_sync(kFull, ed, 0);
+            if (ed < bestd) { bestd = ed; bi = cc; }
+          }
+        }
+        __syncwarp();
+        i1 = bi;
+      }
+      best = i1;
+    }
+    int8_t* out = P.codes + row * P.k + jb * B;
+    const float s_eff = best ? __fdiv_rn(e4m3_pos(best), 127.0f) : 0.0f;
+#pragma unroll
+    for (int t = 0; t < NE; ++t) {
+      const int q = best ? (int)int8_q(a[t], s_eff) : 0;
+      out[lane + 32 * t] = (int8_t)(((sgn >> t) & 1u) ? -q : q);
+    }
+    if (lane == 0) P.scales[b] = (uint8_t)best;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// E4M3 elements, one float32 scale per 64 x 64 tile searched on a logarithmic grid.
+// One CTA (256 threads) per tile; thread t owns row t/4, columns 16 (t%4) .. +16.
+// ---------------------------------------------------------------------------------------
+struct TileParams {
+  const char* W;
+  int64_t n, k, ld_bytes;
+  const float* h;
+  int points;
+  uint8_t* codes;
+  float* scales;
+};
+struct LogGrid {
+  float g[256];
+};
+
+constexpr int kTile = 64;
+constexpr int kTileChunk = 16;  // candidates per register pass
+
+__device__ __forceinline__ float e4m3_elem_wq(float a, float s, float& q_out) {
+  const float z = __fdiv_rn(a, s);
+  const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)e4m3x2_rn(z, 0.0f));
+  q_out = __half2float(__ushort_as_half(lo16(h2)));
+  return __fmul_rn(s, q_out);
+}
+
+template <bool BF16, int MODE>
+__global__ void __launch_bounds__(kThreads)
+k_e4m3_tile(TileParams P, LogGrid G) {
+  __shared__ float g[256];
+  __shared__ float red_max[kThreads / 32];
+  __shared__ double red[kThreads / 32][kTileChunk];
+  __shared__ double err[256];
+  __shared__ int pick;
+  for (int i = threadIdx.x; i < P.points; i += kThreads) g[i] = G.g[i];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int r = threadIdx.x >> 2, c0 = (threadIdx.x & 3) * 16;
+  const int64_t tn = P.n / kTile, tk = P.k / kTile, ntiles = tn * tk;
+  const int elsz = BF16 ? 2 : 4;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t ti = tile / tk, tj = tile - ti * tk;
+    const int64_t row = ti * kTile + r, col = tj * kTile + c0;
+    float2 a2[8];
+    uint32_t sgn;
+    load_block<16, BF16>(P.W + row * P.ld_bytes + col * elsz, a2, sgn);
+    float a[16], c[16];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) { a[2 * p] = a2[p].x; a[2 * p + 1] = a2[p].y; }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) c[j] = (MODE == 2) ? __ldg(P.h + col + j) : 1.0f;
+    float am = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) am = fmaxf(am, a[j]);
+    am = warp_max(am);
+    if (lane == 0) red_max[wid] = am;
+    __syncthreads();
+    am = red_max[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) am = fmaxf(am, red_max[w]);
+    const float base = __fdiv_rn(am, 448.0f);
+    float s = base;
+    if (MODE != 0 && base > 0.0f) {
+      for (int p0 = 0; p0 < P.points; p0 += kTileChunk) {
+        double part[kTileChunk];
+#pragma unroll
+        for (int u = 0; u < kTileChunk; ++u) {
+          part[u] = 0.0;
+          const int p = p0 + u;
+          if (p < P.points) {
+            const float sp = __fmul_rn(base, g[p]);
+            if (sp > 0.0f) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                float q;
+                const float d = __fsub_rn(a[j], e4m3_elem_wq(a[j], sp, q));
+                part[u] += (double)__fmul_rn(__fmul_rn(c[j], d), d);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kTileChunk; ++u) {
+          double v = warp_sum(part[u]);
+          if (lane == 0) red[wid][u] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < kTileChunk && p0 + (int)threadIdx.x < P.points) {
+          const int p = p0 + threadIdx.x;
+          double e = 0.0;
+#pragma unroll
+          for (int w = 0; w < kThreads / 32; ++w) e += red[w][threadIdx.x];
+          const float sp = __fmul_rn(base, g[p]);
+          err[p] = sp > 0.0f ? e : __longlong_as_double(0x7ff0000000000000ll);
+        }
+        __syncthreads();
+      }
+      if (wid == 0) {
+        double v = __longlong_as_double(0x7ff0000000000000ll);
+        int vi = 0x7fffffff;
+        for (int p = lane; p < P.points; p += 32) {
+          if (err[p] < v) { v = err[p]; vi = p; }
+        }
+        warp_argmin(v, vi);
+        if (lane == 0) pick = (v < __longlong_as_double(0x7ff0000000000000ll)) ? vi : -1;
+      }
+      __syncthreads();
+      s = pick >= 0 ? __fmul_rn(base, g[pick]) : 0.0f;
+    }
+    // emit 16 bytes per thread
+    uint32_t wds[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+      uint32_t pair = 0;
+      if (s > 0.0f) pair = e4m3x2_rn(__fdiv_rn(a[j], s), __fdiv_rn(a[j + 1], s)) & 0x7f7fu;
+      pair |= ((sgn >> j) & 1u) << 7;
+      pair |= ((sgn >> (j + 1)) & 1u) << 15;
+      wds[j / 4] |= pair << (8 * (j % 4));
+    }
+    *reinterpret_cast<uint4*>(P.codes + row * P.k + col) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+    if (threadIdx.x == 0) P.scales[tile] = s;
+    __syncthreads();
+  }
+}
+
+// Element projection at one fixed scale (verification entry point): the magnitude code
+// that the search kernels produce for |w| at that scale.
+__global__ void k_project(const float* __restrict__ w, int64_t count, int fmt, float scale,
+                          float rhi, float rlo, uint8_t* __restrict__ q) {
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < count;
+       i += (int64_t)gridDim.x * kThreads) {
+    const float a = fabsf(w[i]);
+    uint32_t code;
+    if (fmt == 0) {
+      const float2 x = fp4_quot(make_float2(a, 0.f), make_float2(rhi, rhi), make_float2(rlo, rlo));
+      code = e2m1x2_rn(x.x, 0.f) & 7u;
+    } else if (fmt == 1) {
+      code = (uint32_t)int8_q(a, __fdiv_rn(scale, 127.0f));
+    } else {
+      code = e4m3x2_rn(__fdiv_rn(a, scale), 0.f) & 0x7fu;
+    }
+    q[i] = (uint8_t)code;
+  }
+}
+
+Fp4Table make_fp4_table() {
+  Fp4Table t;
+  for (int c = 0; c < 128; ++c) {
+    double v;
+    if (c == 0 || c == 127) {
+      t.c[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    const int e = c >> 3, m = c & 7;
+    v = e == 0 ? (double)m / 8.0 * (1.0 / 64.0) : (1.0 + m / 8.0) * ldexp(1.0, e - 7);
+    const double r = 1.0 / v;
+    const float rhi = (float)r;
+    const float rlo = (float)(r - (double)rhi);
+    const __half sh = __double2half(v);  // exact: every E4M3 value is an fp16 value
+    const uint32_t sbits = (uint32_t)__half_as_ushort(sh);
+    float sfl;
+    memcpy(&sfl, &sbits, sizeof sfl);
+    t.c[c] = make_float4((float)v, rhi, rlo, sfl);
+  }
+  return t;
+}
+
+int grid_for(int64_t work_threads) {
+  const int64_t want = (work_threads + kThreads - 1) / kThreads;
+  const int64_t cap = (int64_t)sm_count() * 64;
+  return (int)(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+template <int B, bool BF16>
+cudaError_t fp4_dispatch(const QuantArgs& a, cudaStream_t st) {
+  static const Fp4Table T = make_fp4_table();
+  Fp4Params P{(const char*)a.W, a.n, a.k, a.ld * (BF16 ? 2 : 4), a.h, a.window,
+              (uint8_t*)a.codes, (uint8_t*)a.scales};
+  const int64_t nblocks = a.n * (a.k / B);
+  const int grid = grid_for(nblocks);
+  if (a.mode == 0) k_fp4_naive<B, BF16><<<grid, kThreads, 0, st>>>(P, T);
+  else if (a.mode == 1) k_fp4_search<B, BF16, false><<<grid, kThreads, 0, st>>>(P, T);
+  else k_fp4_search<B, BF16, true><<<grid, kThreads, 0, st>>>(P, T);
+  return cudaGetLastError();
+}
+
+template <int NE, bool BF16>
+cudaError_t int8_dispatch(const QuantArgs& a, cudaStream_t st) {
+  Int8Params P{(const char*)a.W, a.n, a.k, a.ld * (BF16 ? 2 : 4), a.h, a.block, a.window,
+               (int8_t*)a.codes, (uint8_t*)a.scales};
+  const int64_t nblocks = a.n * (a.k / a.block);
+  const int grid = grid_for(nblocks * 32);
+  if (a.mode == 0) k_int8<NE, BF16, 0><<<grid, kThreads, 0, st>>>(P);
+  else if (a.mode == 1) k_int8<NE, BF16, 1><<<grid, kThreads, 0, st>>>(P);
+  else k_int8<NE, BF16, 2><<<grid, kThreads, 0, st>>>(P);
+  return cudaGetLastError();
+}
+
+template <bool BF16>
+cudaError_t tile_dispatch(const QuantArgs& a, cudaStream_t st) {
+  TileParams P{(const char*)a.W, a.n, a.k, a.ld * (BF16 ? 2 : 4), a.h, a.log_points,
+               (uint8_t*)a.codes, (float*)a.scales};
+  LogGrid G;
+  for (int i = 0; i < 256; ++i) G.g[i] = i < a.log_points ? a.log_grid[i] : 0.f;
+  const int64_t ntiles = (a.n / kTile) * (a.k / kTile);
+  int64_t grid = ntiles;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  if (a.mode == 0) k_e4m3_tile<BF16, 0><<<(unsigned)grid, kThreads, 0, st>>>(P, G);
+  else if (a.mode == 1) k_e4m3_tile<BF16, 1><<<(unsigned)grid, kThreads, 0, st>>>(P, G);
+  else k_e4m3_tile<BF16, 2><<<(unsigned)grid, kThreads, 0, st>>>(P, G);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, uint8_t* q,
+                           cudaStream_t st) {
+  float rhi = 0.f, rlo = 0.f;
+  if (fmt == 0) {
+    const double r = 1.0 / (double)scale;
+    rhi = (float)r;
+    rlo = (float)(r - (double)rhi);
+  }
+  int64_t grid = (count + kThreads - 1) / kThreads;
+  if (grid > 4096) grid = 4096;
+  k_project<<<(unsigned)grid, kThreads, 0, st>>>(w, count, fmt, scale, rhi, rlo, q);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
+  const bool bf = a.dtype == 1;
+  if (a.fmt == 0) {
+    if (a.block == 16) return bf ? fp4_dispatch<16, true>(a, st) : fp4_dispatch<16, false>(a, st);
+    return bf ? fp4_dispatch<32, true>(a, st) : fp4_dispatch<32, false>(a, st);
+  }
+  if (a.fmt == 1) {
+    switch (a.block) {
+      case 32: return bf ? int8_dispatch<1, true>(a, st) : int8_dispatch<1, false>(a, st);
+      case 64: return bf ? int8_dispatch<2, true>(a, st) : int8_dispatch<2, false>(a, st);
+      case 128: return bf ? int8_dispatch<4, true>(a, st) : int8_dispatch<4, false>(a, st);
+      default: return bf ? int8_dispatch<8, true>(a, st) : int8_dispatch<8, false>(a, st);
+    }
+  }
+  return bf ? tile_dispatch<true>(a, st) : tile_dispatch<false>(a, st);
+}
+
+}  // namespace mxq

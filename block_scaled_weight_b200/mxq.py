@@ -1,0 +1,233 @@
+"""Thin ctypes binding of ``libmxq.so`` (declared in ``include/mxq.h``).
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream. The functions keep the C names;
+outputs that are not given are allocated with torch on the input's device.
+
+The binding never falls back to another implementation: if the shared library is
+missing it raises ``ImportError`` at import time (build it with
+``python -m block_scaled_weight_b200.build`` or ``__graft_entry__.build()``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmxq.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libmxq.so not built ({_LIB_PATH}); run block_scaled_weight_b200.build")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+MXQ_OK = 0
+STATUS = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_SHAPE", 3: "MXQ_ERR_DTYPE",
+          4: "MXQ_ERR_ALIGN", 5: "MXQ_ERR_UNSUPPORTED", 6: "MXQ_ERR_CUDA",
+          7: "MXQ_ERR_WORKSPACE"}
+F32, BF16 = 0, 1
+FMT = {"nvfp4": 0, "int8": 1, "e4m3": 2}
+MODE = {"naive": 0, "sse": 1, "hopt": 2}
+
+EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqsum",
+           "mxq_act_sqmean_finalize", "mxq_quantize", "mxq_project", "mxq_dequant", "mxq_error_workspace",
+           "mxq_error", "mxq_metrics_from_sums", "mxq_status_string", "mxq_last_error")
+
+
+class MxqParams(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("mode", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("tile_rows", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("log_points", ctypes.c_int32), ("log_lo_exp2", ctypes.c_float),
+                ("log_hi_exp2", ctypes.c_float)]
+
+
+class MxqMetrics(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_double) for n in ("sse", "w_sq", "hsse", "hw_sq", "weight_rel",
+                                               "h_rel")]
+
+
+_P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_sig = {
+    "mxq_act_sqmean_workspace": (_SZ, [_I64, _I64]),
+    "mxq_act_sqmean": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "mxq_act_sqsum": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "mxq_act_sqmean_finalize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
+    "mxq_quantize": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(MxqParams),
+                                    _P, _P, _P]),
+    "mxq_project": (ctypes.c_int, [_P, _I64, _I32, ctypes.c_float, _P, _P]),
+    "mxq_dequant": (ctypes.c_int, [_P, _P, ctypes.POINTER(MxqParams), _I64, _I64, _P, _P]),
+    "mxq_error_workspace": (_SZ, [_I64, _I64]),
+    "mxq_error": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
+                                 ctypes.POINTER(MxqParams), _P, _P, _SZ, _P]),
+    "mxq_metrics_from_sums": (ctypes.c_int, [_P, ctypes.POINTER(MxqMetrics)]),
+    "mxq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mxq_last_error": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class MxqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.mxq_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+def _check(status: int, where: str):
+    if status != MXQ_OK:
+        raise MxqError(status, where)
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def params(fmt="nvfp4", mode="hopt", block=16, *, window=-1, tile_rows=None, log_points=64,
+           log_lo_exp2=-2.0, log_hi_exp2=2.0) -> MxqParams:
+    f = FMT[fmt] if isinstance(fmt, str) else int(fmt)
+    m = MODE[mode] if isinstance(mode, str) else int(mode)
+    if tile_rows is None:
+        tile_rows = block if f == FMT["e4m3"] else 1
+    return MxqParams(f, m, block, tile_rows, window, log_points, log_lo_exp2, log_hi_exp2)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    return 99  # rejected by the library with MXQ_ERR_DTYPE
+
+
+def _ld(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride")
+    return t.stride(0)
+
+
+def mxq_act_sqmean_workspace(rows: int, cols: int) -> int:
+    return int(_lib.mxq_act_sqmean_workspace(rows, cols))
+
+
+def mxq_error_workspace(n: int, k: int) -> int:
+    return int(_lib.mxq_error_workspace(n, k))
+
+
+def _workspace(nbytes, device, ws):
+    if ws is not None:
+        return ws
+    return torch.empty(max(int(nbytes), 8), dtype=torch.uint8, device=device)
+
+
+def mxq_act_sqmean(X: torch.Tensor, h: torch.Tensor | None = None, *, workspace=None,
+                   stream=None) -> torch.Tensor:
+    """h_j = mean_r X[r, j]^2 (float32 [cols])."""
+    R, K = X.shape
+    if h is None:
+        h = torch.empty(K, dtype=torch.float32, device=X.device)
+    ws = _workspace(mxq_act_sqmean_workspace(R, K), X.device, workspace)
+    _check(_lib.mxq_act_sqmean(_ptr(X), _dtype(X), R, K, _ld(X), _ptr(h), _ptr(ws), ws.numel(),
+                               _stream(stream, X.device)), "mxq_act_sqmean")
+    return h
+
+
+def mxq_act_sqsum(X: torch.Tensor, colsum: torch.Tensor | None = None, *, workspace=None,
+                  stream=None) -> torch.Tensor:
+    """sum_r X[r, j]^2 over this shard's rows (float64 [cols])."""
+    R, K = X.shape
+    if colsum is None:
+        colsum = torch.empty(K, dtype=torch.float64, device=X.device)
+    ws = _workspace(mxq_act_sqmean_workspace(R, K), X.device, workspace)
+    _check(_lib.mxq_act_sqsum(_ptr(X), _dtype(X), R, K, _ld(X), _ptr(colsum), _ptr(ws),
+                              ws.numel(), _stream(stream, X.device)), "mxq_act_sqsum")
+    return colsum
+
+
+def mxq_act_sqmean_finalize(partials: torch.Tensor, total_rows: int,
+                            h: torch.Tensor | None = None, *, stream=None) -> torch.Tensor:
+    """h from gathered per-shard column sums ``partials`` [parts, cols] (float64)."""
+    parts, K = partials.shape
+    if h is None:
+        h = torch.empty(K, dtype=torch.float32, device=partials.device)
+    _check(_lib.mxq_act_sqmean_finalize(_ptr(partials.contiguous()), parts, K, int(total_rows),
+                                        _ptr(h), _stream(stream, partials.device)),
+           "mxq_act_sqmean_finalize")
+    return h
+
+
+def output_shapes(p: MxqParams, n: int, k: int):
+    """(codes shape, codes dtype, scales shape, scales dtype) for a quantization."""
+    if p.fmt == FMT["nvfp4"]:
+        return (n, k // 2), torch.uint8, (n, k // p.block), torch.uint8
+    if p.fmt == FMT["int8"]:
+        return (n, k), torch.int8, (n, k // p.block), torch.uint8
+    return (n, k), torch.uint8, (n // p.block, k // p.block), torch.float32
+
+
+def mxq_quantize(W: torch.Tensor, p: MxqParams, h: torch.Tensor | None = None, *, codes=None,
+                 scales=None, stream=None):
+    """(codes, scales) of W [n, k] under settings ``p`` (see ``params``)."""
+    n, k = W.shape
+    cs, cd, ss, sd = output_shapes(p, n, k)
+    if codes is None:
+        codes = torch.empty(cs, dtype=cd, device=W.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sd, device=W.device)
+    _check(_lib.mxq_quantize(_ptr(W), _dtype(W), n, k, _ld(W), _ptr(h), ctypes.byref(p),
+                             _ptr(codes), _ptr(scales), _stream(stream, W.device)),
+           "mxq_quantize")
+    return codes, scales
+
+
+def mxq_project(w: torch.Tensor, fmt: str, scale: float, *, q=None, stream=None) -> torch.Tensor:
+    """Magnitude codes of float32 ``w`` at one fixed scale (the search's element step)."""
+    w = w.contiguous()
+    if q is None:
+        q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    _check(_lib.mxq_project(_ptr(w), w.numel(), FMT[fmt], float(scale), _ptr(q),
+                            _stream(stream, w.device)), "mxq_project")
+    return q
+
+
+def mxq_dequant(codes: torch.Tensor, scales: torch.Tensor, p: MxqParams, n: int, k: int, *,
+                out=None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(n, k, dtype=torch.float32, device=codes.device)
+    _check(_lib.mxq_dequant(_ptr(codes), _ptr(scales), ctypes.byref(p), n, k, _ptr(out),
+                            _stream(stream, codes.device)), "mxq_dequant")
+    return out
+
+
+def mxq_error(W: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, p: MxqParams,
+              h: torch.Tensor | None = None, *, sums=None, workspace=None,
+              stream=None) -> torch.Tensor:
+    """Device float64 [4]: sum d^2, sum w^2, sum h d^2, sum h w^2."""
+    n, k = W.shape
+    if sums is None:
+        sums = torch.empty(4, dtype=torch.float64, device=W.device)
+    ws = _workspace(mxq_error_workspace(n, k), W.device, workspace)
+    _check(_lib.mxq_error(_ptr(W), _dtype(W), n, k, _ld(W), _ptr(codes), _ptr(scales), _ptr(h),
+                          ctypes.byref(p), _ptr(sums), _ptr(ws), ws.numel(),
+                          _stream(stream, W.device)), "mxq_error")
+    return sums
+
+
+def mxq_metrics_from_sums(sums) -> dict:
+    """Metrics from four host doubles (a CPU tensor, a list or a numpy array)."""
+    arr = (ctypes.c_double * 4)(*[float(x) for x in list(sums)])
+    m = MxqMetrics()
+    _check(_lib.mxq_metrics_from_sums(ctypes.cast(arr, ctypes.c_void_p), ctypes.byref(m)),
+           "mxq_metrics_from_sums")
+    return {name: getattr(m, name) for name, _ in MxqMetrics._fields_}

@@ -1,0 +1,210 @@
+/*
+ * mxq.h -- block-scaled post-training weight quantization with a searched E4M3 block
+ * scale, on NVIDIA B200 (sm_100a).
+ *
+ * For every block of B contiguous input-dimension weights of W [n, k] (or every 64 x 64
+ * tile, for E4M3 elements) the library picks one scale and emits the quantized codes:
+ *
+ *   naive    the amax snap s0 = RNE_E4M3(amax / qmax)
+ *            ("Is Finer Better? The Limits of Microscaling Formats in LLMs", sec. 2.1:
+ *            s = Q_scale(xmax / C), q = Q_elem(x / s), x^ = s * q);
+ *   sse      the candidate scale minimising sum_j (w_j - s q_j)^2;
+ *   hopt     the candidate scale minimising sum_j h_j (w_j - s q_j)^2 with
+ *            h_j = E[x_j^2] over calibration activations ("quantization_algorithms.txt",
+ *            sec. 1, the diagonal approximation of the output-error objective);
+ *
+ * over candidates on the E4M3 scale grid (all 126 positive finite values, or a window of
+ * codes around the naive snap; qwantize "Results", sections "INT8 (FP8 E4M3 scales)" and
+ * "NVFP4 (FP8 E4M3 scales)"), or, for E4M3 elements, on a logarithmic grid of float32 tile
+ * scales ("quantization_algorithms.txt", sec. 1).
+ *
+ * Element grids: NVFP4 E2M1 {0, 0.5, 1, 1.5, 2, 3, 4, 6} (qmax 6); symmetric INT8
+ * [-127, 127] with effective scale fl32(amax_e4m3 / 127) (qwantize "Results", INT8
+ * section); E4M3 elements (max 448). Every rounding onto a grid is round-to-nearest with
+ * ties to the even code and saturation; the quotient w / s is the IEEE float32 quotient.
+ * Candidate ties go to the smallest scale.
+ *
+ * Conventions for every call below:
+ *  - Pointers named as device pointers are device memory (any allocator) owned by the
+ *    caller; the library allocates nothing. Workspace sizes come from the *_workspace
+ *    queries.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *    stream) unless stated otherwise. Results are valid after the stream synchronises.
+ *  - Arguments are validated on the host before any launch; a rejected call launches
+ *    nothing and returns a status. A CUDA launch failure returns MXQ_ERR_CUDA and
+ *    mxq_last_error() (per host thread) describes it. No exception crosses the boundary.
+ *  - Calls are reentrant: the library keeps no mutable state besides the per-thread
+ *    error text.
+ *  - Empty problems (n, k or rows == 0) return MXQ_OK without launching.
+ *  - Weights and activations may not contain NaN or infinities (the result is then
+ *    unspecified, but no launch faults).
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MXQ_API __attribute__((visibility("default")))
+#else
+#define MXQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXQ_OK = 0,
+    MXQ_ERR_INVALID_ARG = 1,   /* null pointer, bad enum or parameter value */
+    MXQ_ERR_SHAPE = 2,         /* negative size, k % block != 0, ld < cols, ... */
+    MXQ_ERR_DTYPE = 3,         /* unsupported input element type */
+    MXQ_ERR_ALIGN = 4,         /* pointer or leading dimension not 16-byte aligned */
+    MXQ_ERR_UNSUPPORTED = 5,   /* valid but not implemented combination */
+    MXQ_ERR_CUDA = 6,          /* a CUDA call failed; see mxq_last_error() */
+    MXQ_ERR_WORKSPACE = 7      /* workspace missing or smaller than the query's answer */
+} mxq_status;
+
+typedef enum { MXQ_F32 = 0, MXQ_BF16 = 1 } mxq_dtype;
+typedef enum { MXQ_FMT_NVFP4 = 0, MXQ_FMT_INT8 = 1, MXQ_FMT_E4M3 = 2 } mxq_fmt;
+typedef enum { MXQ_NAIVE = 0, MXQ_SSE = 1, MXQ_HOPT = 2 } mxq_mode;
+
+/* Quantizer settings.
+ *  fmt        MXQ_FMT_NVFP4: E2M1 elements, one E4M3 scale per block of `block` (16 or 32)
+ *             contiguous weights along k.
+ *             MXQ_FMT_INT8: int8 elements in [-127, 127], one E4M3 byte (the stored amax)
+ *             per block of `block` (32, 64, 128 or 256) weights; effective scale
+ *             fl32(E4M3 / 127).
+ *             MXQ_FMT_E4M3: E4M3 elements, one float32 scale per `block` x `block` tile
+ *             (block = tile_rows = 64).
+ *  mode       MXQ_NAIVE, MXQ_SSE or MXQ_HOPT.
+ *  block      see fmt.
+ *  tile_rows  1 for NVFP4 and INT8; 64 (= block) for E4M3 tiles.
+ *  window     NVFP4 / INT8 search: -1 = all 126 positive finite E4M3 scales (codes
+ *             0x01..0x7E); w >= 0 = codes [c0 - w, c0 + w] clipped to [1, 126] around the
+ *             naive code c0 ([1, max(w, 1)] when c0 is 0). Ignored for E4M3 tiles.
+ *  log_points E4M3 tiles: P grid points g_p = fl32(2^(lo + (hi - lo) p / (P - 1))),
+ *             candidate s_p = fl32(fl32(amax_tile / 448) * g_p); 2 <= P <= 256.
+ *  log_lo_exp2, log_hi_exp2  lo and hi (finite, lo < hi); the pages' grid is -2, 2.
+ */
+typedef struct mxq_params {
+    int32_t fmt;
+    int32_t mode;
+    int32_t block;
+    int32_t tile_rows;
+    int32_t window;
+    int32_t log_points;
+    float log_lo_exp2;
+    float log_hi_exp2;
+} mxq_params;
+
+/* Weight error metrics from the four sums that mxq_error produces. */
+typedef struct mxq_metrics {
+    double sse;         /* sum (w - w^)^2 */
+    double w_sq;        /* sum w^2 */
+    double hsse;        /* sum h_j (w - w^)^2   (0 without h) */
+    double hw_sq;       /* sum h_j w^2          (0 without h) */
+    double weight_rel;  /* sqrt(sse / w_sq): ||Q(W) - W||_F / ||W||_F (qwantize "Results") */
+    double h_rel;       /* sqrt(hsse / hw_sq)   (0 without h) */
+} mxq_metrics;
+
+/* ------------------------------------------------------------------------------------
+ * h pass: h_j = E_r[x_rj^2] = (1/R) sum_r x_rj^2 over the rows of the calibration
+ * activations X ("quantization_algorithms.txt", sec. 1: h_j = E[x_j^2]).
+ *
+ *  X          device, [rows, cols] row-major with leading dimension ld (elements);
+ *             16-byte aligned; dtype MXQ_BF16 or MXQ_F32.
+ *  cols       multiple of 8 (bf16) or 4 (f32); ld >= cols with ld * elsize % 16 == 0.
+ *  h          device float [cols], written as fl32(sum / rows) (the sum is exact to within
+ *             ~2e-6 relative: float32 over at most 32 rows, then double).
+ *  workspace  device, at least mxq_act_sqmean_workspace(rows, cols) bytes, 8-byte aligned.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API size_t mxq_act_sqmean_workspace(int64_t rows, int64_t cols);
+MXQ_API mxq_status mxq_act_sqmean(const void* X, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                          float* h, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The two halves of mxq_act_sqmean, for row-sharded activations (one shard per GPU):
+ *  mxq_act_sqsum writes colsum[j] = sum over this shard's rows of x_rj^2 (device double
+ *  [cols]); workspace as for mxq_act_sqmean. After the shards' colsum vectors are gathered
+ *  into device memory partials [parts, cols] (row-major), mxq_act_sqmean_finalize writes
+ *  h[j] = fl32((sum_p partials[p][j]) / total_rows), summing p in ascending order. */
+MXQ_API mxq_status mxq_act_sqsum(const void* X, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                         double* colsum, void* workspace, size_t workspace_bytes, void* stream);
+MXQ_API mxq_status mxq_act_sqmean_finalize(const double* partials, int64_t parts, int64_t cols,
+                                   int64_t total_rows, float* h, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Scale search and quantization (naive / sse / hopt), fused in one kernel per format.
+ *
+ *  W       device, [n, k] row-major, leading dimension ld (elements), 16-byte aligned,
+ *          ld * elsize % 16 == 0; dtype MXQ_BF16 or MXQ_F32.
+ *  h       device float [k], 16-byte aligned; required for MXQ_HOPT, ignored otherwise.
+ *  p       host pointer to the settings.
+ *  codes   device, dense row-major:
+ *            NVFP4 uint8 [n, k/2]: element 2i in the low nibble, nibble = sign << 3 | e2m1
+ *            INT8  int8  [n, k]:   two's complement in [-127, 127]
+ *            E4M3  uint8 [n, k]:   sign << 7 | e4m3 code
+ *          The sign bit of a zero magnitude is the weight's sign bit (INT8 has no -0).
+ *  scales  device, dense row-major:
+ *            NVFP4, INT8: uint8 E4M3 codes [n, k/block]; code 0 only from a naive snap
+ *            that rounds to zero (then every magnitude is 0);
+ *            E4M3: float [n/64, k/64] tile scales (0 for an all-zero tile).
+ *  Shapes: k % block == 0; for E4M3 tiles n % 64 == 0 and k % 64 == 0.
+ *  Result: identical to the plain definition evaluated with IEEE float32 quotients and
+ *  float32 dequantised values, candidate errors accumulated in double in element order,
+ *  ties to the smallest scale (NVFP4 and INT8: exactly, including ties; E4M3 tiles:
+ *  exactly wherever the two best tile errors differ by more than 1e-6 relative).
+ * ------------------------------------------------------------------------------------ */
+MXQ_API mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                        const float* h, const mxq_params* p, void* codes, void* scales,
+                        void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Element projection at one fixed scale -- the per-element step of the search above,
+ * exposed so that it can be verified exhaustively.
+ *
+ *  w      device float [count], 4-byte aligned (only |w| is used).
+ *  fmt    MXQ_FMT_NVFP4: q = RNE_E2M1(fl32(|w| / scale)) code 0..7, scale an E4M3 value;
+ *         MXQ_FMT_INT8:  q = min(127, RNE_int(fl32(|w| / fl32(scale / 127)))), scale the
+ *                        stored E4M3 amax;
+ *         MXQ_FMT_E4M3:  q = RNE_E4M3(fl32(|w| / scale)) code 0..126, any float scale > 0.
+ *  q      device uint8 [count]: the magnitude codes.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API mxq_status mxq_project(const float* w, int64_t count, int32_t fmt, float scale,
+                               uint8_t* q, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Dequantisation: out [n, k] float (device, dense) = s * q with the layouts above
+ * (NVFP4: E4M3(scale) * E2M1(code); INT8: code * fl32(E4M3(scale) / 127), the product
+ * rounded to float; E4M3: tile scale * E4M3(code), rounded to float).
+ * ------------------------------------------------------------------------------------ */
+MXQ_API mxq_status mxq_dequant(const void* codes, const void* scales, const mxq_params* p, int64_t n,
+                       int64_t k, float* out, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Weight error (qwantize "Results": ||Q(W) - W||_F / ||W||_F) and the h-weighted error
+ * (the diagonal objective, "quantization_algorithms.txt", sec. 1), without materialising
+ * the dequantised matrix.
+ *
+ *  sums       device double [4]: sum (w - w^)^2, sum w^2, sum h_j (w - w^)^2,
+ *             sum h_j w^2 (the last two 0 when h is NULL). Deterministic (fixed-order
+ *             combine).
+ *  workspace  device, at least mxq_error_workspace(n, k) bytes, 8-byte aligned.
+ * mxq_metrics_from_sums (host, synchronous) turns four host doubles into mxq_metrics.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API size_t mxq_error_workspace(int64_t n, int64_t k);
+MXQ_API mxq_status mxq_error(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                     const void* codes, const void* scales, const float* h,
+                     const mxq_params* p, double* sums, void* workspace,
+                     size_t workspace_bytes, void* stream);
+MXQ_API mxq_status mxq_metrics_from_sums(const double* host_sums, mxq_metrics* out);
+
+/* Human-readable text for a status; the last failure's detail on this host thread. */
+MXQ_API const char* mxq_status_string(mxq_status s);
+MXQ_API const char* mxq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXQ_H */
