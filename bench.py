@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled weight quantization hot path on B200.
+
+One step = the whole path over one batch of synthetic input:
+  1. h pass        h_j = E_r[x_rj^2] over X [R, K] (bf16)        -- mxq_act_sqmean
+  2. search        NVFP4 (E2M1) block 16, H-optimal over all 126 E4M3 scales
+                   on W [N, K] (bf16), codes + scales            -- mxq_quantize
+  3. metrics       weight error and h-weighted error sums         -- mxq_error
+Default workload: the "full calibration" shape of the qwantize results page
+(W 2560x9728, X 244449x9728, both bf16), synthetic data.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+With N > 1 (launched by torch.distributed.run, one rank per GPU) every rank owns its own
+X and W of that shape (weak scaling); the h pass becomes per-rank column sums, one NCCL
+all-gather of those sums and a fixed-order finalize, so every rank quantizes with the
+global h. ``--impl reference`` times the CPU oracle (bounded sample) instead.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "G weights/s quantized (H-opt NVFP4 blk16) + h-pass GB/s; % of roofline"
+UNIT = "G weights/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+# Plain-ALU peak of the search kernel: 148 SMs x 4 sub-partitions x 32 FP32 lanes x
+# 1965 MHz (max SM clock) = lane-operations per second, an FMA counted as one operation.
+ALU_PEAK_TOPS = 148 * 128 * 1.965e9 / 1e12
+# Algorithmic op count of the H-optimal search per weight: C candidates x 6 (quotient,
+# projection, dequantise, subtract, h-multiply, square-accumulate) + 4 (amax, naive
+# quotient, final projection, pack).
+OPS_PER_WEIGHT_HOPT = lambda C: C * 6 + 4  # noqa: E731
+# Oracle samples: the cpu_baseline leg (about 10-30 s of CPU work) and each step of the
+# reference arm (well under a second, so that a long --steps run stays short).
+CPU_X_ROWS, CPU_W_ROWS = 32768, 512
+REF_X_ROWS, REF_W_ROWS = 2048, 8
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
+    ap.add_argument("--workload", default="nvfp4_full_calib")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--x-rows", type=int, default=0,
+                    help="use only this many activation rows (profiling captures)")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, rec["source"])
+        if source_sha(src) != rec["source_sha"]:
+            return None
+        return rec["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, max clock, throttle reasons) every 10 ms while active."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # NVML unavailable: report no clocks
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def workload_desc(wl, block):
+    (_, n, k), (r, _) = wl.weights[0], wl.x_shapes[0]
+    return (f"{wl.name}: W {n}x{k} bf16, X {r}x{k} bf16, NVFP4 E2M1 block {block}, "
+            f"H-optimal over all 126 E4M3 scales, then weight/h-weighted error sums")
+
+
+# ---------------------------------------------------------------------------------------
+# oracle (CPU) timing: the cpu_baseline leg and the reference arm
+# ---------------------------------------------------------------------------------------
+
+def oracle_step_sample(X_bits, W_bits, h_np, n_threads, R_full, N_full):
+    """Time the oracle on a bounded sample (X_bits: the first rows of X, W_bits: the first
+    rows of W, bf16 bits) and scale each part to the full workload (R_full rows of X,
+    N_full rows of W). Returns (seconds for a full step, measured seconds per part)."""
+    from oracle import oracle as orc
+    x_rows, K = X_bits.shape
+    w_rows = W_bits.shape[0]
+    t0 = time.perf_counter()
+    orc.act_sqmean(X_bits, n_threads=n_threads)
+    t1 = time.perf_counter()
+    r = orc.quantize(W_bits, "nvfp4", "hopt", 16, h=h_np, n_threads=n_threads)
+    What = orc.dequant(r.codes, r.scales, "nvfp4", 16, w_rows, K)
+    orc.error_sums(W_bits, What, h_np)
+    t2 = time.perf_counter()
+    full = (t1 - t0) * (R_full / x_rows) + (t2 - t1) * (N_full / w_rows)
+    return full, {"h_s": t1 - t0, "quant_s": t2 - t1}
+
+
+def bits_of(t):
+    import numpy as np
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def reference_arm(args):
+    """The CPU oracle, as it stands, timed on the host cores: each step is a bounded sample
+    of the workload, its time scaled to the full workload."""
+    rank, world, _ = dist_env()
+    if world > 1 and rank != 0:
+        return
+    from block_scaled_weight_b200 import synth
+    from oracle import oracle as orc
+    wl = synth.WORKLOADS[args.workload]
+    (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
+    x_rows, w_rows = REF_X_ROWS, REF_W_ROWS
+    X = bits_of(synth.workload_activations(wl, 0, rows=x_rows))
+    W = bits_of(synth.workload_weight(wl, 0, rows=w_rows))
+    h = orc.act_sqmean(X)
+    nt = os.cpu_count() or 1
+    times = []
+    for i in range(args.warmup + args.steps):
+        full, _ = oracle_step_sample(X, W, h, nt, R, n)
+        if i >= args.warmup:
+            times.append(full)
+    full_step = statistics.mean(times)
+    value = n * k / full_step / 1e9
+    sample = (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows (H-opt "
+              f"search + error) per step, {nt} threads; times scaled to the full workload")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(wl, 16)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nt, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+
+def gpu_arm(args):
+    import torch.distributed as dist
+    from block_scaled_weight_b200 import mxq, synth
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    wl = synth.WORKLOADS[args.workload]
+    (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
+    if args.x_rows:
+        R = min(R, args.x_rows)
+    block = 16
+    # inputs: every rank draws its own shard (weak scaling)
+    X = torch.empty(R, k, dtype=torch.bfloat16, device=dev)
+    synth.activations(R, k, wl.seed + 1000 * rank, device=dev, n_outlier=wl.x_outliers,
+                      outlier_factor=wl.x_outlier_factor, out=X)
+    W = synth.gaussian_weight(n, k, wl.seed + 1000 * rank, device=dev)
+    p = mxq.params("nvfp4", "hopt", block)
+    h = torch.empty(k, dtype=torch.float32, device=dev)
+    colsum = torch.empty(k, dtype=torch.float64, device=dev)
+    parts = torch.empty(world, k, dtype=torch.float64, device=dev)
+    ws = torch.empty(mxq.mxq_act_sqmean_workspace(R, k), dtype=torch.uint8, device=dev)
+    codes = torch.empty(n, k // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(n, k // block, dtype=torch.uint8, device=dev)
+    sums = torch.empty(4, dtype=torch.float64, device=dev)
+    ews = torch.empty(mxq.mxq_error_workspace(n, k), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 5 if world == 1 else 5  # hpass partial + finalize, search, error x2
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        if world == 1:
+            mxq.mxq_act_sqmean(X, h, workspace=ws)
+        else:
+            mxq.mxq_act_sqsum(X, colsum, workspace=ws)
+            dist.all_gather_into_tensor(parts, colsum)
+            mxq.mxq_act_sqmean_finalize(parts, R * world, h)
+        if ev is not None:
+            ev[1].record(stream)
+        mxq.mxq_quantize(W, p, h, codes=codes, scales=scales)
+        if ev is not None:
+            ev[2].record(stream)
+        mxq.mxq_error(W, codes, scales, p, h, sums=sums, workspace=ews)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    k_h = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    k_q = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    k_e = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    t = torch.tensor([ms_total, k_h, k_q, k_e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, k_h, k_q, k_e = t.tolist()
+    ms_step = ms_total / args.steps
+    weights = n * k
+    value = world * weights / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API, host buffers -----------------------------
+    X_host = torch.empty(R, k, dtype=torch.bfloat16, pin_memory=True)
+    X_host.copy_(X)
+    W_host = torch.empty(n, k, dtype=torch.bfloat16, pin_memory=True)
+    W_host.copy_(W)
+    codes_host = torch.empty_like(codes, device="cpu").pin_memory()
+    scales_host = torch.empty_like(scales, device="cpu").pin_memory()
+    sums_host = torch.empty(4, dtype=torch.float64, pin_memory=True)
+    h2d = X_host.numel() * 2 + W_host.numel() * 2
+    d2h = codes_host.numel() + scales_host.numel() + 8 * 4
+
+    def e2e_step():
+        X.copy_(X_host, non_blocking=True)
+        W.copy_(W_host, non_blocking=True)
+        step()
+        codes_host.copy_(codes, non_blocking=True)
+        scales_host.copy_(scales, non_blocking=True)
+        sums_host.copy_(sums, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t2 = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_ms = t2.item() / args.e2e_steps
+    e2e_value = world * weights / (e2e_ms * 1e-3) / 1e9
+    metrics = mxq.mxq_metrics_from_sums(sums_host)
+
+    # ---- roofline ------------------------------------------------------------------------
+    hbm, hbm_kind = measured_peaks()
+    x_bytes = R * k * 2 + 4 * k
+    h_gbs = x_bytes / (k_h * 1e-3) / 1e9
+    ops = OPS_PER_WEIGHT_HOPT(126) * weights
+    q_tops = ops / (k_q * 1e-3) / 1e12
+    e_bytes = weights * 2 + weights // 2 + weights // block + 4 * k
+    e_gbs = e_bytes / (k_e * 1e-3) / 1e9
+    kernels = {
+        "act_sqmean": {"ms": k_h, "bound": "hbm", "achieved": h_gbs, "peak": hbm, "unit": "GB/s",
+                       "frac": h_gbs / hbm, "algorithmic_bytes": x_bytes,
+                       "traffic": traffic_for("act_sqmean")},
+        "quantize": {"ms": k_q, "bound": "alu", "achieved": q_tops, "peak": ALU_PEAK_TOPS,
+                     "unit": "T lane-op/s", "frac": q_tops / ALU_PEAK_TOPS,
+                     "algorithmic_ops": ops, "traffic": traffic_for("quantize")},
+        "error": {"ms": k_e, "bound": "hbm", "achieved": e_gbs, "peak": hbm, "unit": "GB/s",
+                  "frac": e_gbs / hbm, "algorithmic_bytes": e_bytes,
+                  "traffic": traffic_for("error")},
+    }
+    dom = max(kernels, key=lambda kk: kernels[kk]["ms"])
+    dk = kernels[dom]
+    roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"],
+                "peak": dk["peak"], "unit": dk["unit"], "frac": dk["frac"],
+                "traffic": dk["traffic"],
+                "peak_source": ("MEASURED_PEAKS.json hbm_gbs (" + hbm_kind + ")")
+                if dk["bound"] == "hbm" else "148 SM x 128 FP32 lanes x 1965 MHz"}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(wl, block), "weights_per_gpu": weights,
+                       "x_rows_per_gpu": R,
+                       "parallelism": f"dp{world}" + (" (rows of X and W per rank; one "
+                                                      "all-gather of column sums)" if world > 1 else ""),
+                       "l2": "inputs larger than L2: X (%.2f GB) is streamed every step"
+                             % (R * k * 2 / 1e9)},
+            "h_pass_gbs": h_gbs, "h_pass_frac_of_hbm": h_gbs / hbm,
+            "roofline": roofline, "kernels": kernels,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary(),
+            "result": {"weight_rel": metrics["weight_rel"], "h_rel": metrics["h_rel"]}}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        x_rows, w_rows = CPU_X_ROWS, CPU_W_ROWS
+        Xb = bits_of(X[:x_rows].cpu())
+        Wb = bits_of(W[:w_rows].cpu())
+        from oracle import oracle as orc
+        nt = os.cpu_count() or 1
+        h_np = orc.act_sqmean(Xb, n_threads=nt)
+        full, d = oracle_step_sample(Xb, Wb, h_np, nt, R, n)
+        line["cpu_baseline"] = {
+            "value": weights / full / 1e9, "unit": UNIT, "cores": nt, "kind": "oracle",
+            "sample": (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows "
+                       f"(H-opt search + error), {nt} threads; times scaled to the full "
+                       f"workload ({d['h_s']:.1f} s + {d['quant_s']:.1f} s measured)")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

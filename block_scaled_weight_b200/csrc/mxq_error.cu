@@ -2,16 +2,19 @@
 //
 // Dequantised value (the microscaling reconstruction x^ = s q, "Is Finer Better? The
 // Limits of Microscaling Formats in LLMs", sec. 2.1):
-//   NVFP4  E4M3(scale) * E2M1(code)                (exact in float32)
-//   INT8   fl32(|q| * fl32(E4M3(scale) / 127)), signed
-//   E4M3   fl32(tile scale * E4M3(code)), signed
+//   NVFP4  E4M3(scale) * E2M1(code)                (exact in float32 and in fp16)
+//   INT8   fl32(q * fl32(E4M3(scale) / 127))
+//   E4M3   fl32(tile scale * E4M3(code))
 // Metrics (qwantize "Results": weight error ||Q(W) - W||_F / ||W||_F; the h-weighted
 // error of "quantization_algorithms.txt", sec. 1): the four sums sum d^2, sum w^2,
-// sum h d^2, sum h w^2. HBM-bound: each thread decodes 16 consecutive elements of a row;
-// float32 partials over those 16, double from there on; the per-CTA partials are summed
-// in a fixed order by a second one-CTA kernel (deterministic).
+// sum h d^2, sum h w^2. HBM-bound: each thread decodes 16 consecutive elements of a row
+// with the hardware E2M1 / E4M3 conversions; float32 partials over those 16 (packed f32x2
+// math), double from there on; the per-CTA partials are combined by a one-CTA kernel in a
+// fixed order (deterministic).
 #include "mxq_common.cuh"
 #include "mxq_internal.h"
+
+#include <cuda_fp16.h>
 
 namespace mxq {
 
@@ -20,67 +23,69 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxErrCtas = 148 * 8;
 
-__device__ __forceinline__ float e2m1_mag(uint32_t nib) {
-  // 0, 0.5, 1, 1.5, 2, 3, 4, 6 from the code bits: e = nib >> 1, m = nib & 1.
-  const uint32_t e = (nib >> 1) & 3u, m = nib & 1u;
-  return e == 0 ? 0.5f * (float)m : __uint_as_float(((126u + e) << 23) | (m << 22));
+__device__ __forceinline__ float2 h2f2(uint32_t h2) {
+  return make_float2(__half2float(__ushort_as_half(lo16(h2))),
+                     __half2float(__ushort_as_half(hi16(h2))));
 }
 
-// Decode the 16 elements starting at (row, col) into v[16].
+// Decoded (w^) values of the 16 elements starting at (row, col), as 8 float pairs.
+template <int FMT>
 __device__ __forceinline__ void decode16(const DecodeArgs& d, int64_t row, int64_t col,
-                                         float (&v)[16]) {
-  if (d.fmt == 0) {
+                                         float2 (&v)[8]) {
+  if constexpr (FMT == 0) {
     const uint8_t* cp = (const uint8_t*)d.codes + row * (d.k / 2) + col / 2;
     const uint2 cw = *reinterpret_cast<const uint2*>(cp);
     const float s = e4m3_pos(((const uint8_t*)d.scales)[row * (d.k / d.block) + col / d.block]);
+    const float2 s2 = make_float2(s, s);
     const uint32_t w2[2] = {cw.x, cw.y};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const uint32_t nib = (w2[j / 8] >> (4 * (j % 8))) & 15u;
-      const float m = __fmul_rn(s, e2m1_mag(nib & 7u));
-      v[j] = (nib & 8u) ? -m : m;
+    for (int p = 0; p < 8; ++p) {
+      const uint32_t byte = (w2[p / 4] >> (8 * (p % 4))) & 0xffu;
+      v[p] = __fmul2_rn(h2f2(e2m1x2_to_f16x2(byte)), s2);     // exact products
     }
-  } else if (d.fmt == 1) {
+  } else if constexpr (FMT == 1) {
     const int8_t* cp = (const int8_t*)d.codes + row * d.k + col;
     const uint4 cw = *reinterpret_cast<const uint4*>(cp);
     const int sc = ((const uint8_t*)d.scales)[row * (d.k / d.block) + col / d.block];
     const float s = __fdiv_rn(e4m3_pos(sc), 127.0f);
+    const float2 s2 = make_float2(s, s);
     const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int q = (int)(int8_t)((w4[j / 4] >> (8 * (j % 4))) & 0xffu);
-      const float m = __fmul_rn((float)(q < 0 ? -q : q), s);
-      v[j] = q < 0 ? -m : m;
+    for (int p = 0; p < 8; ++p) {
+      const uint32_t wd = w4[p / 2] >> (16 * (p % 2));
+      const float q0 = (float)(int8_t)(wd & 0xffu), q1 = (float)(int8_t)((wd >> 8) & 0xffu);
+      v[p] = __fmul2_rn(make_float2(q0, q1), s2);
     }
   } else {
     const uint8_t* cp = (const uint8_t*)d.codes + row * d.k + col;
     const uint4 cw = *reinterpret_cast<const uint4*>(cp);
     const float s = ((const float*)d.scales)[(row / d.block) * (d.k / d.block) + col / d.block];
+    const float2 s2 = make_float2(s, s);
     const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const uint32_t c = (w4[j / 4] >> (8 * (j % 4))) & 0xffu;
-      const float m = __fmul_rn(s, e4m3_pos((int)(c & 0x7fu)));
-      v[j] = (c & 0x80u) ? -m : m;
+    for (int p = 0; p < 8; ++p) {
+      const uint16_t pair = (uint16_t)(w4[p / 2] >> (16 * (p % 2)));
+      v[p] = __fmul2_rn(h2f2(e4m3x2_to_f16x2(pair)), s2);
     }
   }
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 k_dequant(DecodeArgs d, float* __restrict__ out) {
   const int64_t units = d.n * (d.k / 16);
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units;
        u += (int64_t)gridDim.x * kThreads) {
     const int64_t row = u / (d.k / 16), col = (u - row * (d.k / 16)) * 16;
-    float v[16];
-    decode16(d, row, col, v);
+    float2 v[8];
+    decode16<FMT>(d, row, col, v);
     float4* o = reinterpret_cast<float4*>(out + row * d.k + col);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    for (int i = 0; i < 4; ++i) o[i] = make_float4(v[2 * i].x, v[2 * i].y, v[2 * i + 1].x, v[2 * i + 1].y);
   }
 }
 
-template <bool BF16>
+template <int FMT, bool BF16, bool HAS_H>
 __global__ void __launch_bounds__(kThreads)
 k_error(DecodeArgs d, const char* __restrict__ W, int64_t ld_bytes, const float* __restrict__ h,
         double* __restrict__ partial) {
@@ -90,43 +95,43 @@ k_error(DecodeArgs d, const char* __restrict__ W, int64_t ld_bytes, const float*
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units;
        u += (int64_t)gridDim.x * kThreads) {
     const int64_t row = u / (d.k / 16), col = (u - row * (d.k / 16)) * 16;
-    float v[16], w[16], hh[16];
-    decode16(d, row, col, v);
+    float2 v[8], w[8];
+    decode16<FMT>(d, row, col, v);
     const char* wp = W + row * ld_bytes + col * (BF16 ? 2 : 4);
     if constexpr (BF16) {
       const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(wp));
       const uint4 x1 = __ldg(reinterpret_cast<const uint4*>(wp) + 1);
       const uint32_t wd[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { w[2 * i] = bf16lo(wd[i]); w[2 * i + 1] = bf16hi(wd[i]); }
+      for (int p = 0; p < 8; ++p) w[p] = make_float2(bf16lo(wd[p]), bf16hi(wd[p]));
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float4 x = __ldg(reinterpret_cast<const float4*>(wp) + i);
-        w[4 * i] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
+        w[2 * i] = make_float2(x.x, x.y);
+        w[2 * i + 1] = make_float2(x.z, x.w);
       }
     }
-    if (h) {
+    float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(h + col) + i);
-        hh[4 * i] = x.x; hh[4 * i + 1] = x.y; hh[4 * i + 2] = x.z; hh[4 * i + 3] = x.w;
+    for (int p = 0; p < 8; ++p) {
+      const float2 dd = __fadd2_rn(w[p], make_float2(-v[p].x, -v[p].y));
+      const float2 d2 = __fmul2_rn(dd, dd), w2 = __fmul2_rn(w[p], w[p]);
+      s0 = __fadd2_rn(s0, d2);
+      s1 = __fadd2_rn(s1, w2);
+      if constexpr (HAS_H) {
+        const float4 hv = __ldg(reinterpret_cast<const float4*>(h + col) + p / 2);
+        const float2 hh = (p & 1) ? make_float2(hv.z, hv.w) : make_float2(hv.x, hv.y);
+        s2 = __ffma2_rn(hh, d2, s2);
+        s3 = __ffma2_rn(hh, w2, s3);
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) hh[j] = 0.0f;
     }
-    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float dj = __fsub_rn(w[j], v[j]);
-      const float d2 = __fmul_rn(dj, dj), w2 = __fmul_rn(w[j], w[j]);
-      s0 += d2;
-      s1 += w2;
-      s2 = fmaf(hh[j], d2, s2);
-      s3 = fmaf(hh[j], w2, s3);
+    acc[0] += (double)s0.x + (double)s0.y;
+    acc[1] += (double)s1.x + (double)s1.y;
+    if constexpr (HAS_H) {
+      acc[2] += (double)s2.x + (double)s2.y;
+      acc[3] += (double)s3.x + (double)s3.y;
     }
-    acc[0] += (double)s0; acc[1] += (double)s1; acc[2] += (double)s2; acc[3] += (double)s3;
   }
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
@@ -143,12 +148,48 @@ k_error(DecodeArgs d, const char* __restrict__ W, int64_t ld_bytes, const float*
   }
 }
 
-__global__ void k_error_final(const double* __restrict__ partial, int parts, double* sums) {
-  if (threadIdx.x < 4) {
-    double s = 0.0;
-    for (int p = 0; p < parts; ++p) s += partial[p * 4 + threadIdx.x];
-    sums[threadIdx.x] = s;
+// One CTA: thread t sums partials t, t + 256, ... in order; then a fixed-shape tree.
+__global__ void __launch_bounds__(kThreads)
+k_error_final(const double* __restrict__ partial, int parts, double* sums) {
+  __shared__ double red[4][kThreads];
+  double s[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int p = threadIdx.x; p < parts; p += kThreads)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[i] += partial[p * 4 + i];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) red[i][threadIdx.x] = s[i];
+  __syncthreads();
+  for (int half = kThreads / 2; half > 0; half >>= 1) {
+    if ((int)threadIdx.x < half)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) red[i][threadIdx.x] += red[i][threadIdx.x + half];
+    __syncthreads();
   }
+  if (threadIdx.x < 4) sums[threadIdx.x] = red[threadIdx.x][0];
+}
+
+template <int FMT>
+cudaError_t dequant_fmt(const DecodeArgs& d, float* out, cudaStream_t st) {
+  const int64_t units = d.n * (d.k / 16);
+  int64_t grid = (units + kThreads - 1) / kThreads;
+  const int64_t cap = (int64_t)sm_count() * 16;
+  if (grid > cap) grid = cap;
+  k_dequant<FMT><<<(unsigned)grid, kThreads, 0, st>>>(d, out);
+  return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t error_fmt(const DecodeArgs& d, const void* W, int dtype, int64_t ld, const float* h,
+                      double* partial, int parts, cudaStream_t st) {
+  const char* Wc = (const char*)W;
+  if (dtype == 1) {
+    if (h) k_error<FMT, true, true><<<parts, kThreads, 0, st>>>(d, Wc, ld * 2, h, partial);
+    else k_error<FMT, true, false><<<parts, kThreads, 0, st>>>(d, Wc, ld * 2, h, partial);
+  } else {
+    if (h) k_error<FMT, false, true><<<parts, kThreads, 0, st>>>(d, Wc, ld * 4, h, partial);
+    else k_error<FMT, false, false><<<parts, kThreads, 0, st>>>(d, Wc, ld * 4, h, partial);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -161,24 +202,20 @@ int error_partials(int64_t n, int64_t k) {
 }
 
 cudaError_t launch_dequant(const DecodeArgs& d, float* out, cudaStream_t st) {
-  const int64_t units = d.n * (d.k / 16);
-  int64_t grid = (units + kThreads - 1) / kThreads;
-  const int64_t cap = (int64_t)sm_count() * 16;
-  if (grid > cap) grid = cap;
-  k_dequant<<<(unsigned)grid, kThreads, 0, st>>>(d, out);
-  return cudaGetLastError();
+  if (d.fmt == 0) return dequant_fmt<0>(d, out, st);
+  if (d.fmt == 1) return dequant_fmt<1>(d, out, st);
+  return dequant_fmt<2>(d, out, st);
 }
 
 cudaError_t launch_error(const DecodeArgs& d, const void* W, int dtype, int64_t ld,
                          const float* h, double* partial, int parts, double* sums,
                          cudaStream_t st) {
-  if (dtype == 1)
-    k_error<true><<<parts, kThreads, 0, st>>>(d, (const char*)W, ld * 2, h, partial);
-  else
-    k_error<false><<<parts, kThreads, 0, st>>>(d, (const char*)W, ld * 4, h, partial);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (d.fmt == 0) e = error_fmt<0>(d, W, dtype, ld, h, partial, parts, st);
+  else if (d.fmt == 1) e = error_fmt<1>(d, W, dtype, ld, h, partial, parts, st);
+  else e = error_fmt<2>(d, W, dtype, ld, h, partial, parts, st);
   if (e != cudaSuccess) return e;
-  k_error_final<<<1, 32, 0, st>>>(partial, parts, sums);
+  k_error_final<<<1, kThreads, 0, st>>>(partial, parts, sums);
   return cudaGetLastError();
 }
 

@@ -4,7 +4,8 @@
 // HBM-bound: every byte of X is read once. Each warp owns a strip of 32 x 16-byte
 // columns (256 bf16 or 128 f32 columns) and one of 8 interleaved row phases of a row
 // chunk; each lane keeps its 8 (or 4) columns' running sums. Loads are 128-bit,
-// non-caching in L1, four rows in flight per lane. Squares accumulate in float32 (packed
+// non-caching in L1, eight rows in flight per lane; the grid is one wave of resident
+// CTAs (strips x row chunks <= 148 SMs x 3). Squares accumulate in float32 (packed
 // f32x2 FMA) for at most 32 rows, then fold into double, so the column sum carries at
 // most ~32 float roundings (relative error <= 2e-6); the 8 row phases and the row chunks
 // are combined in double in a fixed order, which makes the result deterministic.
@@ -16,7 +17,9 @@ namespace mxq {
 namespace {
 
 constexpr int kWarps = kHpassThreads / 32;
-constexpr int kTargetCtas = 148 * 8;   // one wave of 8 resident 256-thread CTAs per SM
+constexpr int kRowsPerStep = 8;
+constexpr int kCtasPerSm = 3;          // resident 256-thread CTAs per SM (launch bounds)
+constexpr int kTargetCtas = 148 * kCtasPerSm;   // one wave on a 148-SM B200
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
@@ -45,7 +48,7 @@ __device__ __forceinline__ void acc_sq(const uint4& v, float2* acc) {
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kHpassThreads)
+__global__ void __launch_bounds__(kHpassThreads, kCtasPerSm)
 k_hpass_partial(const char* __restrict__ X, int64_t rows, int64_t cols, int64_t ld_bytes,
                 int64_t rows_per_chunk, double* __restrict__ partial) {
   constexpr int VEC = BF16 ? 8 : 4;       // elements per 16-byte load
@@ -78,17 +81,14 @@ k_hpass_partial(const char* __restrict__ X, int64_t rows, int64_t cols, int64_t 
     };
     int64_t r = r0 + warp;
     int it = 0;
-    // Four rows per step (r, r+8, r+16, r+24): four 16-byte loads in flight per lane.
-    for (; r + 3 * kWarps < r1; r += 4 * kWarps) {
-      const uint4 v0 = ld_stream(base + r * ld_bytes);
-      const uint4 v1 = ld_stream(base + (r + kWarps) * ld_bytes);
-      const uint4 v2 = ld_stream(base + (r + 2 * kWarps) * ld_bytes);
-      const uint4 v3 = ld_stream(base + (r + 3 * kWarps) * ld_bytes);
-      acc_sq<BF16>(v0, acc);
-      acc_sq<BF16>(v1, acc);
-      acc_sq<BF16>(v2, acc);
-      acc_sq<BF16>(v3, acc);
-      if (++it == 8) {  // 32 rows per float accumulator
+    // Eight rows per step (r, r+8, ..., r+56): eight 16-byte loads in flight per lane.
+    for (; r + 7 * kWarps < r1; r += kRowsPerStep * kWarps) {
+      uint4 v[kRowsPerStep];
+#pragma unroll
+      for (int u = 0; u < kRowsPerStep; ++u) v[u] = ld_stream(base + (r + u * kWarps) * ld_bytes);
+#pragma unroll
+      for (int u = 0; u < kRowsPerStep; ++u) acc_sq<BF16>(v[u], acc);
+      if (++it == 32 / kRowsPerStep) {  // at most 32 rows per float accumulator
         flush();
         it = 0;
       }
@@ -129,7 +129,7 @@ int strip_cols(int dtype) { return dtype == 1 ? 256 : 128; }
 int hpass_chunks(int64_t rows, int64_t cols, int dtype) {
   if (rows <= 0 || cols <= 0) return 1;
   const int64_t strips = (cols + strip_cols(dtype) - 1) / strip_cols(dtype);
-  int64_t chunks = (kTargetCtas + strips - 1) / strips;
+  int64_t chunks = kTargetCtas / strips;   // strips x chunks <= one wave
   const int64_t by_rows = (rows + 255) / 256;  // at least ~256 rows per chunk
   if (chunks > by_rows) chunks = by_rows;
   if (chunks < 1) chunks = 1;

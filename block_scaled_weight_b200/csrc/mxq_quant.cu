@@ -43,6 +43,7 @@ constexpr int kThreads = 256;
 // ---------------------------------------------------------------------------------------
 struct Fp4Table {
   float4 c[128];
+  float2 sig[8];  // split reciprocals 8/S of the normal significands S = 8..15
 };
 
 struct Fp4Params {
@@ -111,18 +112,34 @@ __device__ __forceinline__ float2 fp4_quot(float2 a, float2 rhi, float2 rlo) {
   return __ffma2_rn(a, rhi, __fmul2_rn(a, rlo));
 }
 
-// Float32 error of one candidate: sum_j c_j (s g_j - a_j)^2 (c_j = 1 for SSE).
+// a - s * g for a pair of elements at one candidate: the E2M1 codes of the exact float32
+// quotients x, decoded to halves, and one mixed-precision FMA each with the negated fp16
+// scale (s g is exact; a single rounding of the difference). The E2M1 byte never leaves
+// a .b8 register.
+__device__ __forceinline__ float2 fp4_pair_diff(float2 a, float2 x, uint32_t s_neg_h) {
+  float d0, d1;
+  asm("{\n\t.reg .b8 q;\n\t.reg .b32 g;\n\t.reg .b16 g0, g1, sn, sx;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q, %3, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 g, q;\n\t"
+      "mov.b32 {g0, g1}, g;\n\t"
+      "mov.b32 {sn, sx}, %6;\n\t"
+      "fma.rn.f32.f16 %0, g0, sn, %4;\n\t"
+      "fma.rn.f32.f16 %1, g1, sn, %5;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(x.x), "f"(x.y), "f"(a.x), "f"(a.y), "r"(s_neg_h));
+  return make_float2(d0, d1);
+}
+
+// Float32 error of one candidate: sum_j c_j (a_j - s g_j)^2 (c_j = 1 for SSE).
 template <int B, bool HOPT>
-__device__ __forceinline__ float fp4_eval(const float2 (&a)[B / 2], const float2 (&na)[B / 2],
-                                          const float2 (&c)[B / 2], float4 t) {
+__device__ __forceinline__ float fp4_eval(const float2 (&a)[B / 2], const float2 (&c)[B / 2],
+                                          float4 t) {
   const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
-  const uint16_t s_h = (uint16_t)__float_as_uint(t.w);
+  const uint32_t s_neg_h = __float_as_uint(t.w) ^ 0x8000u;
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int p = 0; p < B / 2; ++p) {
-    const float2 x = fp4_quot(a[p], rhi, rlo);
-    const uint32_t g = e2m1x2_to_f16x2(e2m1x2_rn(x.x, x.y));
-    const float2 d = make_float2(fma_h_h_f(lo16(g), s_h, na[p].x), fma_h_h_f(hi16(g), s_h, na[p].y));
+    const float2 d = fp4_pair_diff(a[p], fp4_quot(a[p], rhi, rlo), s_neg_h);
     float2& acc = (p & 1) ? acc1 : acc0;
     if constexpr (HOPT) {
       acc = __ffma2_rn(__fmul2_rn(c[p], d), d, acc);
@@ -202,12 +219,48 @@ k_fp4_naive(Fp4Params P, Fp4Table T) {
   }
 }
 
-// NVFP4, SSE / H-optimal search: one thread per block walks every candidate.
+// Float32 error of one candidate from precomputed exact quotients x (pairs):
+// sum_j c_j (a_j - s g_j)^2 with g = RNE_E2M1(x).
+template <int B, bool HOPT>
+__device__ __forceinline__ float fp4_eval_x(const float2 (&a)[B / 2], const float2 (&c)[B / 2],
+                                            const float2 (&xs)[B / 2], float2 pow2,
+                                            uint32_t s_neg_h) {
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int p = 0; p < B / 2; ++p) {
+    const float2 d = fp4_pair_diff(a[p], __fmul2_rn(xs[p], pow2), s_neg_h);
+    float2& acc = (p & 1) ? acc1 : acc0;
+    if constexpr (HOPT) {
+      acc = __ffma2_rn(__fmul2_rn(c[p], d), d, acc);
+    } else {
+      acc = __ffma2_rn(d, d, acc);
+    }
+  }
+  return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+}
+
+// Running (min, second min, arg min) over candidates visited in any order; equal errors
+// keep the smaller code and push the tie into the second slot (so the block is flagged).
+__device__ __forceinline__ void track(float e, int cc, float& m1, float& m2, int& i1) {
+  if (e < m1 || (e == m1 && cc < i1)) {
+    m2 = m1;
+    m1 = e;
+    i1 = cc;
+  } else if (e < m2) {
+    m2 = e;
+  }
+}
+
+// NVFP4, SSE / H-optimal search: one thread per block walks every candidate, grouped by
+// significand. Blocks whose float32 winner is not separated from the runner-up by the
+// error bound are flagged (bit 7 of the scale byte) for k_fp4_fixup.
 template <int B, bool BF16, bool HOPT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, B == 16 ? 3 : 2)
 k_fp4_search(Fp4Params P, Fp4Table T) {
   __shared__ float4 tab[128];
+  __shared__ float2 sig[8];
   for (int i = threadIdx.x; i < 128; i += kThreads) tab[i] = T.c[i];
+  for (int i = threadIdx.x; i < 8; i += kThreads) sig[i] = T.sig[i];
   __syncthreads();
   const int64_t kb = P.k / B, nblocks = P.n * kb;
   const int elsz = BF16 ? 2 : 4;
@@ -217,11 +270,9 @@ k_fp4_search(Fp4Params P, Fp4Table T) {
   for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks;
        b += (int64_t)gridDim.x * kThreads) {
     const int64_t row = b / kb, jb = b - row * kb;
-    float2 a[B / 2], na[B / 2], c[B / 2];
+    float2 a[B / 2], c[B / 2];
     uint32_t sgn;
     load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
-#pragma unroll
-    for (int p = 0; p < B / 2; ++p) na[p] = make_float2(-a[p].x, -a[p].y);
     if constexpr (HOPT) load_h<B>(P.h + jb * B, c);
     const int c0 = e4m3_rn_code(__fdiv_rn(block_amax<B>(a), 6.0f));
     int lo = 1, hi = 126;
@@ -232,27 +283,114 @@ k_fp4_search(Fp4Params P, Fp4Table T) {
     }
     float m1 = __int_as_float(0x7f800000), m2 = m1;
     int i1 = lo;
-    for (int cc = lo; cc <= hi; ++cc) {
-      const float e = fp4_eval<B, HOPT>(a, na, c, tab[cc]);
-      if (e < m1) { m2 = m1; m1 = e; i1 = cc; }
-      else if (e < m2) m2 = e;
+    // subnormal scales (codes 1..7): the split-reciprocal quotient per candidate
+    for (int cc = lo; cc <= min(hi, 7); ++cc) {
+      const float4 t = tab[cc];
+      const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
+      float2 xs[B / 2];
+#pragma unroll
+      for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
+      track(fp4_eval_x<B, HOPT>(a, c, xs, make_float2(1.f, 1.f), __float_as_uint(t.w) ^ 0x8000u),
+            cc, m1, m2, i1);
+    }
+    // Normal scales, grouped by mantissa field m: codes (e << 3) | m, e = 1..15. Their
+    // quotients are fl32(|w| 8/S) 2^(7-e) (S = 8 + m): exact power-of-two rescalings of
+    // one split-reciprocal quotient per significand (the result is a normal float
+    // whenever it can reach an E2M1 decision boundary).
+    for (int m = 0; m < 8; ++m) {
+      const int e_lo = max(1, (lo - m + 7) >> 3);
+      const int e_hi = min(m == 7 ? 14 : 15, (hi - m) >> 3);
+      if (e_lo > e_hi) continue;
+      const float2 r = sig[m];
+      const float2 rhi = make_float2(r.x, r.x), rlo = make_float2(r.y, r.y);
+      float2 xs[B / 2];
+#pragma unroll
+      for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
+      for (int e = e_lo; e <= e_hi; ++e) {
+        const int cc = (e << 3) | m;
+        const float pw = __int_as_float((134 - e) << 23);  // 2^(7 - e)
+        track(fp4_eval_x<B, HOPT>(a, c, xs, make_float2(pw, pw),
+                                  __float_as_uint(tab[cc].w) ^ 0x8000u),
+              cc, m1, m2, i1);
+      }
     }
     const float upper = fmaf(m1, hi_f, slack);
     if (!(m2 * lo_f - slack > upper)) {
-      // A second candidate may tie or beat the float32 winner: re-score in double.
+      // A second candidate may tie or beat the float32 winner: flag the block (bit 7 of
+      // the scale byte) for the exact pass, k_fp4_fixup.
+      P.scales[b] = (uint8_t)(0x80 | i1);
+    } else {
+      fp4_emit<B>(a, sgn, tab[i1], false, P.codes + row * (P.k / 2) + jb * (B / 2));
+      P.scales[b] = (uint8_t)i1;
+    }
+  }
+}
+
+// Exact pass over the blocks the search flagged. Each warp scans 32 scale bytes at a time;
+// every flagged block is handled by the whole warp: lanes evaluate candidates lo + lane +
+// 32 t in float32, the warp minimum bounds the band, candidates inside it are re-scored in
+// double in the definition's order, and the warp arg-min (lowest code on equal doubles)
+// is emitted.
+template <int B, bool BF16, bool HOPT>
+__global__ void __launch_bounds__(kThreads)
+k_fp4_fixup(Fp4Params P, Fp4Table T) {
+  __shared__ float4 tab[128];
+  for (int i = threadIdx.x; i < 128; i += kThreads) tab[i] = T.c[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t kb = P.k / B, nblocks = P.n * kb;
+  const int elsz = BF16 ? 2 : 4;
+  const float gam = (float)(B + 8) * 5.9604645e-8f;
+  const float lo_f = 1.0f - gam, hi_f = 1.0f + 2.0f * gam;
+  const float slack = 7.3468396e-40f;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t base = gw * 32; base < nblocks; base += nw * 32) {
+    const int64_t mine = base + lane;
+    const bool flagged = mine < nblocks && (P.scales[mine] & 0x80);
+    unsigned todo = __ballot_sync(kFull, flagged);
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int64_t b = base + src;
+      const int64_t row = b / kb, jb = b - row * kb;
+      float2 a[B / 2], c[B / 2];
+      uint32_t sgn;
+      load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
+      if constexpr (HOPT) load_h<B>(P.h + jb * B, c);
+      const int c0 = e4m3_rn_code(__fdiv_rn(block_amax<B>(a), 6.0f));
+      int lo = 1, hi = 126;
+      if (P.window >= 0) {
+        lo = max(1, c0 - P.window);
+        hi = min(126, c0 + P.window);
+        if (c0 == 0) { lo = 1; hi = max(1, P.window); }
+      }
+      float ef[4];
+      float mloc = __int_as_float(0x7f800000);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int cc = lo + lane + 32 * t;
+        ef[t] = cc <= hi ? fp4_eval<B, HOPT>(a, c, tab[cc]) : __int_as_float(0x7f800000);
+        mloc = fminf(mloc, ef[t]);
+      }
+      const float m1 = warp_min(mloc);
+      const float upper = fmaf(m1, hi_f, slack);
       double best = __longlong_as_double(0x7ff0000000000000ll);
-      int bi = i1;
-      for (int cc = lo; cc <= hi; ++cc) {
-        const float e = fp4_eval<B, HOPT>(a, na, c, tab[cc]);
-        if (!(e * lo_f - slack > upper)) {
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int cc = lo + lane + 32 * t;
+        if (cc <= hi && !(ef[t] * lo_f - slack > upper)) {
           const double ed = fp4_exact<B, HOPT>(a, c, tab[cc]);
-          if (ed < best) { best = ed; bi = cc; }
+          if (ed < best || (ed == best && cc < bi)) { best = ed; bi = cc; }
         }
       }
-      i1 = bi;
+      warp_argmin(best, bi);
+      if (lane == 0) {
+        fp4_emit<B>(a, sgn, tab[bi], false, P.codes + row * (P.k / 2) + jb * (B / 2));
+        P.scales[b] = (uint8_t)bi;
+      }
     }
-    fp4_emit<B>(a, sgn, tab[i1], false, P.codes + row * (P.k / 2) + jb * (B / 2));
-    P.scales[b] = (uint8_t)i1;
   }
 }
 
@@ -551,6 +689,11 @@ Fp4Table make_fp4_table() {
     memcpy(&sfl, &sbits, sizeof sfl);
     t.c[c] = make_float4((float)v, rhi, rlo, sfl);
   }
+  for (int m = 0; m < 8; ++m) {
+    const double q = 8.0 / (8.0 + m);
+    const float qh = (float)q;
+    t.sig[m] = make_float2(qh, (float)(q - (double)qh));
+  }
   return t;
 }
 
@@ -567,9 +710,18 @@ cudaError_t fp4_dispatch(const QuantArgs& a, cudaStream_t st) {
               (uint8_t*)a.codes, (uint8_t*)a.scales};
   const int64_t nblocks = a.n * (a.k / B);
   const int grid = grid_for(nblocks);
-  if (a.mode == 0) k_fp4_naive<B, BF16><<<grid, kThreads, 0, st>>>(P, T);
-  else if (a.mode == 1) k_fp4_search<B, BF16, false><<<grid, kThreads, 0, st>>>(P, T);
+  if (a.mode == 0) {
+    k_fp4_naive<B, BF16><<<grid, kThreads, 0, st>>>(P, T);
+    return cudaGetLastError();
+  }
+  if (a.mode == 1) k_fp4_search<B, BF16, false><<<grid, kThreads, 0, st>>>(P, T);
   else k_fp4_search<B, BF16, true><<<grid, kThreads, 0, st>>>(P, T);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t fwant = (nblocks + 32 * 8 - 1) / (32 * 8);   // one 32-block tile per warp
+  const int fgrid = (int)(fwant < (int64_t)sm_count() * 8 ? fwant : (int64_t)sm_count() * 8);
+  if (a.mode == 1) k_fp4_fixup<B, BF16, false><<<fgrid, kThreads, 0, st>>>(P, T);
+  else k_fp4_fixup<B, BF16, true><<<fgrid, kThreads, 0, st>>>(P, T);
   return cudaGetLastError();
 }
 
