@@ -46,7 +46,7 @@ ALU_PEAK_TOPS = 148 * 128 * 1.965e9 / 1e12
 OPS_PER_WEIGHT_HOPT = lambda C: C * 6 + 4  # noqa: E731
 # Oracle samples: the cpu_baseline leg (about 10-30 s of CPU work) and each step of the
 # reference arm (well under a second, so that a long --steps run stays short).
-CPU_X_ROWS, CPU_W_ROWS = 32768, 512
+CPU_X_ROWS, CPU_W_ROWS = 32768, 1024
 REF_X_ROWS, REF_W_ROWS = 2048, 8
 
 

@@ -1,0 +1,156 @@
+"""Full-size parity: every workload at its full shape on the GPU (the launch shapes the
+benchmark times), checked against the oracle on seeded samples of rows (the oracle computes
+those outputs one block at a time) and, for h, on the whole activation matrix.
+
+The oracle receives only its own inputs: h for the quantizer comparisons is the oracle's h
+(uploaded to the GPU), so the search is compared in isolation; the h pass is compared on its
+own; and one end-to-end check runs each side on its own h.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import near_tie_mask, oracle_view
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+DEV = "cuda"
+NT = os.cpu_count() or 1
+
+
+@pytest.fixture(scope="module")
+def mxq():
+    from block_scaled_weight_b200.build import build
+    build()
+    from block_scaled_weight_b200 import mxq as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def synth():
+    from block_scaled_weight_b200 import synth as s
+    return s
+
+
+def sampled_parity(mxq, orc, W, fmt, block, mode, h_np, window, rows, tag):
+    """Quantize all of W on the GPU; compare `rows` with the oracle; return near-tie count."""
+    p = mxq.params(fmt, mode, block, window=window)
+    hd = None if h_np is None else torch.from_numpy(h_np).to(DEV)
+    codes, scales = mxq.mxq_quantize(W, p, hd)
+    torch.cuda.synchronize()
+    Ws = oracle_view(W[torch.as_tensor(rows, device=W.device)])
+    r = orc.quantize(Ws, fmt, mode, block, h=h_np, window=window, n_threads=NT)
+    if fmt == "e4m3":
+        raise AssertionError("use tile_parity for e4m3")
+    g_codes = codes[torch.as_tensor(rows, device=W.device)].cpu().numpy().view(np.uint8)
+    g_scales = scales[torch.as_tensor(rows, device=W.device)].cpu().numpy()
+    bad = g_scales != r.scales
+    near = near_tie_mask(r.best, r.second)
+    assert not bad.any(), f"{tag}: {bad.sum()} of {bad.size} sampled blocks differ " \
+                          f"({(bad & near).sum()} in near ties)"
+    assert np.array_equal(g_codes, r.codes.view(np.uint8)), f"{tag}: codes differ"
+    return int(near.sum()), int(near.size)
+
+
+def test_nvfp4_full_calibration(mxq, orc, synth):
+    wl = synth.WORKLOADS["nvfp4_full_calib"]
+    (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
+    X = synth.workload_activations(wl, 0, device=DEV)               # 4.76 GB
+    h_gpu = mxq.mxq_act_sqmean(X)
+    torch.cuda.synchronize()
+    Xh = oracle_view(X)
+    del X
+    torch.cuda.empty_cache()
+    h_orc = orc.act_sqmean(Xh, n_threads=NT)
+    del Xh
+    np.testing.assert_allclose(h_gpu.cpu().numpy(), h_orc, rtol=1e-5)
+    W = synth.workload_weight(wl, 0, device=DEV)
+    rows = synth.sample_rows(n, 48, wl.seed).numpy()
+    for block in (16, 32):
+        for mode in ("naive", "sse", "hopt"):
+            near, tot = sampled_parity(mxq, orc, W, "nvfp4", block, mode,
+                                       h_orc if mode == "hopt" else None, -1, rows,
+                                       f"nvfp4 bs{block} {mode}")
+            print(f"nvfp4 bs{block} {mode}: {tot} sampled blocks bit-exact, {near} near ties")
+    # end to end: each side on its own h; picks may differ only where the h difference
+    # (<= ~2e-6 relative) can move a block whose two best errors are within 1e-5
+    p = mxq.params("nvfp4", "hopt", 16)
+    codes, scales = mxq.mxq_quantize(W, p, h_gpu)
+    r = orc.quantize(oracle_view(W[torch.as_tensor(rows, device=DEV)]), "nvfp4", "hopt", 16,
+                     h=h_orc, n_threads=NT)
+    g = scales[torch.as_tensor(rows, device=DEV)].cpu().numpy()
+    bad = g != r.scales
+    assert not (bad & ~near_tie_mask(r.best, r.second, rel=1e-5)).any()
+
+
+@pytest.mark.parametrize("block", [32, 64, 128, 256])
+def test_int8_e4m3_scales(mxq, orc, synth, block):
+    wl = synth.WORKLOADS["int8_e4m3scale"]
+    (_, n, k), _ = wl.weights[0], wl.x_shapes[0]
+    X = synth.workload_activations(wl, 0, device=DEV)
+    h_gpu = mxq.mxq_act_sqmean(X)
+    h_orc = orc.act_sqmean(oracle_view(X), n_threads=NT)
+    np.testing.assert_allclose(h_gpu.cpu().numpy(), h_orc, rtol=1e-5)
+    W = synth.workload_weight(wl, 0, device=DEV)
+    rows = synth.sample_rows(n, 24, wl.seed + block).numpy()
+    for mode in ("naive", "sse", "hopt"):
+        near, tot = sampled_parity(mxq, orc, W, "int8", block, mode,
+                                   h_orc if mode == "hopt" else None, 8, rows,
+                                   f"int8 bs{block} {mode}")
+        print(f"int8 bs{block} {mode}: {tot} sampled blocks bit-exact, {near} near ties")
+
+
+def test_e4m3_tiles_full(mxq, orc, synth):
+    wl = synth.WORKLOADS["e4m3_tiles"]
+    (_, n, k), _ = wl.weights[0], wl.x_shapes[0]
+    X = synth.workload_activations(wl, 0, device=DEV)
+    h_gpu = mxq.mxq_act_sqmean(X)
+    h_orc = orc.act_sqmean(oracle_view(X), n_threads=NT)
+    np.testing.assert_allclose(h_gpu.cpu().numpy(), h_orc, rtol=1e-5)
+    W = synth.workload_weight(wl, 0, device=DEV)
+    p = mxq.params("e4m3", "hopt", 64)
+    codes, scales = mxq.mxq_quantize(W, p, torch.from_numpy(h_orc).to(DEV))
+    torch.cuda.synchronize()
+    tile_rows = synth.sample_rows(n // 64, 2, wl.seed).numpy()
+    for tr in tile_rows:
+        Wt = oracle_view(W[tr * 64:(tr + 1) * 64])
+        r = orc.quantize(Wt, "e4m3", "hopt", 64, h=h_orc, n_threads=NT)
+        gs = scales[tr].cpu().numpy()
+        near = near_tie_mask(r.best, r.second)[0]
+        bad = gs != r.scales[0]
+        assert not (bad & ~near).any(), f"tile row {tr}: {(bad & ~near).sum()} tiles differ"
+        gc = codes[tr * 64:(tr + 1) * 64].cpu().numpy()
+        for tj in np.nonzero(~bad)[0]:
+            assert np.array_equal(gc[:, tj * 64:(tj + 1) * 64], r.codes[:, tj * 64:(tj + 1) * 64])
+        print(f"e4m3 tile row {tr}: {gs.size} tiles, {near.sum()} near ties, "
+              f"{bad.sum()} differing (all near ties)")
+
+
+def test_decoder_layer_back_to_back(mxq, orc, synth):
+    wl = synth.WORKLOADS["decoder_layer"]
+    hs = {}
+    for xi, (R, k) in enumerate(wl.x_shapes):
+        X = synth.workload_activations(wl, xi, device=DEV)
+        h_gpu = mxq.mxq_act_sqmean(X)
+        h_orc = orc.act_sqmean(oracle_view(X), n_threads=NT)
+        np.testing.assert_allclose(h_gpu.cpu().numpy(), h_orc, rtol=1e-5)
+        hs[k] = h_orc
+        del X
+        torch.cuda.empty_cache()
+    p = mxq.params("nvfp4", "hopt", 16)
+    outs = []
+    Ws = [synth.workload_weight(wl, i, device=DEV) for i in range(len(wl.weights))]
+    stream = torch.cuda.current_stream()
+    for W in Ws:                                            # back to back on one stream
+        outs.append(mxq.mxq_quantize(W, p, torch.from_numpy(hs[W.shape[1]]).to(DEV),
+                                     stream=stream))
+    torch.cuda.synchronize()
+    for i, (W, (codes, scales)) in enumerate(zip(Ws, outs)):
+        name, n, k = wl.weights[i]
+        rows = synth.sample_rows(n, 4, wl.seed + i).numpy()
+        r = orc.quantize(oracle_view(W[torch.as_tensor(rows, device=DEV)]), "nvfp4", "hopt", 16,
+                         h=hs[k], n_threads=NT)
+        ri = torch.as_tensor(rows, device=DEV)
+        assert np.array_equal(scales[ri].cpu().numpy(), r.scales), name
+        assert np.array_equal(codes[ri].cpu().numpy(), r.codes), name
