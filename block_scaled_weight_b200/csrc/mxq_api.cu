@@ -92,6 +92,13 @@ mxq_status check_params(const mxq_params* p, int64_t n, int64_t k) {
 
 }  // namespace
 
+void mxq::set_error_text(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+}
+
 extern "C" {
 
 const char* mxq_status_string(mxq_status s) {

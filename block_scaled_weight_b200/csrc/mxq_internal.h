@@ -50,5 +50,7 @@ cudaError_t launch_error(const DecodeArgs& d, const void* W, int dtype, int64_t 
                          cudaStream_t st);
 
 int sm_count();
+// Sets the per-thread text that mxq_last_error() returns.
+void set_error_text(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
 
 }  // namespace mxq

@@ -28,7 +28,8 @@ F32, BF16 = 0, 1
 FMT = {"nvfp4": 0, "int8": 1, "e4m3": 2}
 MODE = {"naive": 0, "sse": 1, "hopt": 2}
 
-EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqsum",
+EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc",
+           "mxq_act_sqsum",
            "mxq_act_sqmean_finalize", "mxq_quantize", "mxq_project", "mxq_dequant", "mxq_error_workspace",
            "mxq_error", "mxq_metrics_from_sums", "mxq_status_string", "mxq_last_error")
 
@@ -49,6 +50,7 @@ _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_
 _sig = {
     "mxq_act_sqmean_workspace": (_SZ, [_I64, _I64]),
     "mxq_act_sqmean": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "mxq_act_sqmean_noalloc": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P]),
     "mxq_act_sqsum": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mxq_act_sqmean_finalize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
     "mxq_quantize": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(MxqParams),
@@ -140,6 +142,19 @@ def mxq_act_sqmean(X: torch.Tensor, h: torch.Tensor | None = None, *, workspace=
     ws = _workspace(mxq_act_sqmean_workspace(R, K), X.device, workspace)
     _check(_lib.mxq_act_sqmean(_ptr(X), _dtype(X), R, K, _ld(X), _ptr(h), _ptr(ws), ws.numel(),
                                _stream(stream, X.device)), "mxq_act_sqmean")
+    return h
+
+
+def mxq_act_sqmean_noalloc(X: torch.Tensor, h: torch.Tensor | None = None, *,
+                           stream=None) -> torch.Tensor:
+    """h_j = mean_r X[r, j]^2 without a workspace: the library's static 1 MiB device scratch
+    is used instead (for callers that must not allocate device memory; widths up to 131072
+    columns). Calls that overlap on the GPU share that scratch and must be ordered."""
+    R, K = X.shape
+    if h is None:
+        h = torch.empty(K, dtype=torch.float32, device=X.device)
+    _check(_lib.mxq_act_sqmean_noalloc(_ptr(X), _dtype(X), R, K, _ld(X), _ptr(h),
+                                       _stream(stream, X.device)), "mxq_act_sqmean_noalloc")
     return h
 
 

@@ -124,6 +124,20 @@ MXQ_API size_t mxq_act_sqmean_workspace(int64_t rows, int64_t cols);
 MXQ_API mxq_status mxq_act_sqmean(const void* X, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
                           float* h, void* workspace, size_t workspace_bytes, void* stream);
 
+/* mxq_act_sqmean without a workspace argument, for callers that cannot allocate device
+ * memory (their device memory belongs to another allocator or a fixed arena, or they must
+ * not call cudaMalloc after start-up because it can synchronise the device). The pages
+ * have no counterpart: this is an interface variant, not part of the method.
+ * The scratch is a 1 MiB static device array inside the library, present on every GPU that
+ * loads it until the process exits; it covers every width up to 131072 columns (wider X is
+ * rejected with MXQ_ERR_SHAPE, launching nothing). No cudaMalloc, cudaFree or other
+ * allocation happens. All calls share the array: calls that overlap on the GPU race, so
+ * order them (e.g. one stream). The first call on each device, with that device current,
+ * looks up the array's device address; make it before any stream capture begins.
+ * Arguments and result as for mxq_act_sqmean. */
+MXQ_API mxq_status mxq_act_sqmean_noalloc(const void* X, int32_t dtype, int64_t rows,
+                                          int64_t cols, int64_t ld, float* h, void* stream);
+
 /* The two halves of mxq_act_sqmean, for row-sharded activations (one shard per GPU):
  *  mxq_act_sqsum writes colsum[j] = sum over this shard's rows of x_rj^2 (device double
  *  [cols]); workspace as for mxq_act_sqmean. After the shards' colsum vectors are gathered
