@@ -239,6 +239,13 @@ __device__ __forceinline__ float fp4_eval_x(const float2 (&a)[B / 2], const floa
   return (acc0.x + acc0.y) + (acc1.x + acc1.y);
 }
 
+// Float32 error of the two bound elements (at, with weights ct) at one candidate.
+__device__ __forceinline__ float fp4_lb(float2 at, float2 ct, float2 x, uint32_t s_neg_h) {
+  const float2 d = fp4_pair_diff(at, x, s_neg_h);
+  const float2 v = __fmul2_rn(__fmul2_rn(ct, d), d);
+  return v.x + v.y;
+}
+
 // Running (min, second min, arg min) over candidates visited in any order; equal errors
 // keep the smaller code and push the tie into the second slot (so the block is flagged).
 __device__ __forceinline__ void track(float e, int cc, float& m1, float& m2, int& i1) {
@@ -283,15 +290,77 @@ k_fp4_search(Fp4Params P, Fp4Table T) {
     }
     float m1 = __int_as_float(0x7f800000), m2 = m1;
     int i1 = lo;
-    // subnormal scales (codes 1..7): the split-reciprocal quotient per candidate
-    for (int cc = lo; cc <= min(hi, 7); ++cc) {
-      const float4 t = tab[cc];
+    // Seed: the naive code (clipped to the candidate range), evaluated in full.
+    const int cs = min(max(c0, lo), hi);
+    {
+      const float4 t = tab[cs];
       const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
       float2 xs[B / 2];
 #pragma unroll
       for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
       track(fp4_eval_x<B, HOPT>(a, c, xs, make_float2(1.f, 1.f), __float_as_uint(t.w) ^ 0x8000u),
-            cc, m1, m2, i1);
+            cs, m1, m2, i1);
+    }
+    // Lower bounds. A candidate's error is at least the error of any subset of elements;
+    // the subset here is the two elements with the largest c w^2 (t1, t2). A candidate
+    // whose bound, minus its float32 rounding margin, exceeds the current winner's upper
+    // bound can neither win nor tie, nor fall in the band that decides flagging: it is
+    // skipped without a full evaluation.
+    //
+    // Range cuts, from single elements j (T: the seed's upper bound, which only shrinks):
+    //  * for s < a_j / 6, element j maps to 6 s, so the error is at least
+    //    c_j (a_j - 6 s)^2, growing as s shrinks: every s below
+    //    max_j (a_j - sqrt(T / c_j)) / 6 is out;
+    //  * for s >= 4 a_j, element j's quotient is at most 0.25 and it maps to 0,
+    //    contributing exactly c_j a_j^2: every s >= min {4 a_j : c_j a_j^2 > T} is out.
+    // The candidate range shrinks to the codes in between. The margins (1e-5 relative)
+    // cover the float32 roundings of the approximate reciprocal square root and products.
+    float upper = fmaf(m1, hi_f, slack);
+    float2 at, ct;
+    float s_cut = 0.f, s_hi = __int_as_float(0x7f800000);
+    {
+      const float sqt = sqrtf(upper) * 1.00001f;
+      float v1 = -1.f, a1 = 0.f, c1 = 0.f, v2 = -1.f, a2 = 0.f, c2 = 0.f;
+      auto visit = [&](float aj, float cj) {
+        const float v = cj * aj * aj;
+        if (v > v1) { v2 = v1; a2 = a1; c2 = c1; v1 = v; a1 = aj; c1 = cj; }
+        else if (v > v2) { v2 = v; a2 = aj; c2 = cj; }
+        if (cj > 0.f) {
+          s_cut = fmaxf(s_cut, (aj - sqt * rsqrtf(cj)) * (1.0f / 6.0f) * 0.99999f);
+          if (v * 0.99999f - slack > upper) s_hi = fminf(s_hi, 4.0f * aj);
+        }
+      };
+#pragma unroll
+      for (int p = 0; p < B / 2; ++p) {
+        visit(a[p].x, HOPT ? c[p].x : 1.f);
+        visit(a[p].y, HOPT ? c[p].y : 1.f);
+      }
+      at = make_float2(a1, a2);
+      ct = make_float2(c1, c2);
+    }
+    if (s_cut > 0.f) {
+      int cl = e4m3_rn_code(s_cut);
+      if (e4m3_pos(cl) < s_cut) ++cl;                 // smallest code with value >= s_cut
+      lo = max(lo, cl);
+    }
+    if (s_hi < 1e30f) {
+      int ch = e4m3_rn_code(s_hi);
+      if (!(e4m3_pos(ch) < s_hi)) --ch;               // largest code with value < s_hi
+      hi = min(hi, ch);
+    }
+    const float lb_f = 1.0f - 8.0f * 5.9604645e-8f;
+    // subnormal scales (codes 1..7): the split-reciprocal quotient per candidate
+    for (int cc = lo; cc <= min(hi, 7); ++cc) {
+      if (cc == cs) continue;
+      const float4 t = tab[cc];
+      const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
+      const uint32_t sn = __float_as_uint(t.w) ^ 0x8000u;
+      if (fp4_lb(at, ct, fp4_quot(at, rhi, rlo), sn) * lb_f - slack > upper) continue;
+      float2 xs[B / 2];
+#pragma unroll
+      for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
+      track(fp4_eval_x<B, HOPT>(a, c, xs, make_float2(1.f, 1.f), sn), cc, m1, m2, i1);
+      upper = fmaf(m1, hi_f, slack);
     }
     // Normal scales, grouped by mantissa field m: codes (e << 3) | m, e = 1..15. Their
     // quotients are fl32(|w| 8/S) 2^(7-e) (S = 8 + m): exact power-of-two rescalings of
@@ -303,18 +372,26 @@ k_fp4_search(Fp4Params P, Fp4Table T) {
       if (e_lo > e_hi) continue;
       const float2 r = sig[m];
       const float2 rhi = make_float2(r.x, r.x), rlo = make_float2(r.y, r.y);
+      const float2 xt = fp4_quot(at, rhi, rlo);
       float2 xs[B / 2];
-#pragma unroll
-      for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
+      bool have_xs = false;
       for (int e = e_lo; e <= e_hi; ++e) {
         const int cc = (e << 3) | m;
+        if (cc == cs) continue;
+        const float4 t = tab[cc];
         const float pw = __int_as_float((134 - e) << 23);  // 2^(7 - e)
-        track(fp4_eval_x<B, HOPT>(a, c, xs, make_float2(pw, pw),
-                                  __float_as_uint(tab[cc].w) ^ 0x8000u),
-              cc, m1, m2, i1);
+        const float2 pw2 = make_float2(pw, pw);
+        const uint32_t sn = __float_as_uint(t.w) ^ 0x8000u;
+        if (fp4_lb(at, ct, __fmul2_rn(xt, pw2), sn) * lb_f - slack > upper) continue;
+        if (!have_xs) {
+#pragma unroll
+          for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
+          have_xs = true;
+        }
+        track(fp4_eval_x<B, HOPT>(a, c, xs, pw2, sn), cc, m1, m2, i1);
+        upper = fmaf(m1, hi_f, slack);
       }
     }
-    const float upper = fmaf(m1, hi_f, slack);
     if (!(m2 * lo_f - slack > upper)) {
       // A second candidate may tie or beat the float32 winner: flag the block (bit 7 of
       // the scale byte) for the exact pass, k_fp4_fixup.
