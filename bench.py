@@ -228,6 +228,7 @@ def reference_arm(args):
 def gpu_arm(args):
     import torch.distributed as dist
     from block_scaled_weight_b200 import mxq, synth
+    from block_scaled_weight_b200.dist import distributed_h
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -248,14 +249,15 @@ def gpu_arm(args):
     p = mxq.params("nvfp4", "hopt", block)
     h = torch.empty(k, dtype=torch.float32, device=dev)
     colsum = torch.empty(k, dtype=torch.float64, device=dev)
-    parts = torch.empty(world, k, dtype=torch.float64, device=dev)
     ws = torch.empty(mxq.mxq_act_sqmean_workspace(R, k), dtype=torch.uint8, device=dev)
     codes = torch.empty(n, k // 2, dtype=torch.uint8, device=dev)
     scales = torch.empty(n, k // block, dtype=torch.uint8, device=dev)
     sums = torch.empty(4, dtype=torch.float64, device=dev)
     ews = torch.empty(mxq.mxq_error_workspace(n, k), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 5 if world == 1 else 5  # hpass partial + finalize, search, error x2
+    # our kernels per step: h pass (2; 3 with the sharded finalize), search + exact fixup (2),
+    # error sums + combine (2)
+    launches_per_step = 6 if world == 1 else 7
 
     def step(ev=None):
         if ev is not None:
@@ -263,9 +265,9 @@ def gpu_arm(args):
         if world == 1:
             mxq.mxq_act_sqmean(X, h, workspace=ws)
         else:
-            mxq.mxq_act_sqsum(X, colsum, workspace=ws)
-            dist.all_gather_into_tensor(parts, colsum)
-            mxq.mxq_act_sqmean_finalize(parts, R * world, h)
+            # per-rank column sums -> rank-ordered all-gather -> fixed-order finalize
+            distributed_h(X, lambda x: mxq.mxq_act_sqsum(x, colsum, workspace=ws),
+                          lambda p, r: mxq.mxq_act_sqmean_finalize(p, r, h), R * world)
         if ev is not None:
             ev[1].record(stream)
         mxq.mxq_quantize(W, p, h, codes=codes, scales=scales)
