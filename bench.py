@@ -19,6 +19,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -37,13 +38,10 @@ UNIT = "G weights/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
 # Plain-ALU peak of the search kernel: 148 SMs x 4 sub-partitions x 32 FP32 lanes x
 # 1965 MHz (max SM clock) = lane-operations per second, an FMA counted as one operation.
 ALU_PEAK_TOPS = 148 * 128 * 1.965e9 / 1e12
-# Algorithmic op count of the H-optimal search per weight: C candidates x 6 (quotient,
-# projection, dequantise, subtract, h-multiply, square-accumulate) + 4 (amax, naive
-# quotient, final projection, pack).
-OPS_PER_WEIGHT_HOPT = lambda C: C * 6 + 4  # noqa: E731
 # Oracle samples: the cpu_baseline leg (about 10-30 s of CPU work) and each step of the
 # reference arm (well under a second, so that a long --steps run stays short).
 CPU_X_ROWS, CPU_W_ROWS = 32768, 1024
@@ -59,6 +57,8 @@ def parse():
     ap.add_argument("--workload", default="nvfp4_full_calib")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", type=int, default=0, help="block size (default: the workload's)")
+    ap.add_argument("--mode", default="", choices=["", "naive", "sse", "hopt"])
     ap.add_argument("--x-rows", type=int, default=0,
                     help="use only this many activation rows (profiling captures)")
     return ap.parse_args()
@@ -152,28 +152,36 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def workload_desc(wl, block):
-    (_, n, k), (r, _) = wl.weights[0], wl.x_shapes[0]
-    return (f"{wl.name}: W {n}x{k} bf16, X {r}x{k} bf16, NVFP4 E2M1 block {block}, "
-            f"H-optimal over all 126 E4M3 scales, then weight/h-weighted error sums")
+def workload_desc(wl, fmt, block, mode, window, x_rows=None):
+    """One-line description of what a step computes (both arms print the same)."""
+    x_rows = x_rows or [r for r, _ in wl.x_shapes]
+    dt = "bf16" if wl.w_dtype == torch.bfloat16 else "f32"
+    shapes = ", ".join(f"{nm} {n}x{k}" for nm, n, k in wl.weights)
+    xsh = ", ".join(f"{r}x{k}" for r, (_, k) in zip(x_rows, wl.x_shapes))
+    grid = ("64-point log grid" if fmt == "e4m3" else
+            "all 126 E4M3 scales" if window < 0 else f"E4M3 scales within +-{window} codes")
+    return (f"{wl.name}: W {shapes} {dt}; X {xsh} {dt}; {fmt} block {block}, {mode}, "
+            f"{grid}; then weight/h-weighted error sums")
 
 
 # ---------------------------------------------------------------------------------------
 # oracle (CPU) timing: the cpu_baseline leg and the reference arm
 # ---------------------------------------------------------------------------------------
 
-def oracle_step_sample(X_bits, W_bits, h_np, n_threads, R_full, N_full):
+def oracle_step_sample(X_bits, W_bits, h_np, n_threads, R_full, N_full, q):
     """Time the oracle on a bounded sample (X_bits: the first rows of X, W_bits: the first
-    rows of W, bf16 bits) and scale each part to the full workload (R_full rows of X,
-    N_full rows of W). Returns (seconds for a full step, measured seconds per part)."""
+    rows of W, bf16 bits; q = (fmt, block, mode, window)) and scale each part to the full
+    workload (R_full rows of X, N_full rows of W, in units of the sample's row widths).
+    Returns (seconds for a full step, measured seconds per part)."""
     from oracle import oracle as orc
+    fmt, block, mode, window = q
     x_rows, K = X_bits.shape
     w_rows = W_bits.shape[0]
     t0 = time.perf_counter()
     orc.act_sqmean(X_bits, n_threads=n_threads)
     t1 = time.perf_counter()
-    r = orc.quantize(W_bits, "nvfp4", "hopt", 16, h=h_np, n_threads=n_threads)
-    What = orc.dequant(r.codes, r.scales, "nvfp4", 16, w_rows, K)
+    r = orc.quantize(W_bits, fmt, mode, block, h=h_np, window=window, n_threads=n_threads)
+    What = orc.dequant(r.codes, r.scales, fmt, block, w_rows, K)
     orc.error_sums(W_bits, What, h_np)
     t2 = time.perf_counter()
     full = (t1 - t0) * (R_full / x_rows) + (t2 - t1) * (N_full / w_rows)
@@ -181,39 +189,49 @@ def oracle_step_sample(X_bits, W_bits, h_np, n_threads, R_full, N_full):
 
 
 def bits_of(t):
+    """Host copy for the oracle: bf16 as its raw 16-bit patterns, float32 as is."""
     import numpy as np
+    if t.dtype == torch.float32:
+        return t.contiguous().numpy()
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
 def reference_arm(args):
     """The CPU oracle, as it stands, timed on the host cores: each step is a bounded sample
-    of the workload, its time scaled to the full workload."""
+    of the workload (the first X and W matrices), its time scaled to the full workload."""
     rank, world, _ = dist_env()
     if world > 1 and rank != 0:
         return
     from block_scaled_weight_b200 import synth
     from oracle import oracle as orc
     wl = synth.WORKLOADS[args.workload]
+    q = quantizer_for(wl, args)
     (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
-    x_rows, w_rows = REF_X_ROWS, REF_W_ROWS
+    x_rows = min(REF_X_ROWS, R)
+    w_rows = min(max(REF_W_ROWS, q[1] if q[0] == "e4m3" else 1), n)
     X = bits_of(synth.workload_activations(wl, 0, rows=x_rows))
     W = bits_of(synth.workload_weight(wl, 0, rows=w_rows))
     h = orc.act_sqmean(X)
     nt = os.cpu_count() or 1
+    weights = sum(nn * kk for _, nn, kk in wl.weights)
+    R_full = sum(r * kk for r, kk in wl.x_shapes) / k
     times = []
     for i in range(args.warmup + args.steps):
-        full, _ = oracle_step_sample(X, W, h, nt, R, n)
+        full, _ = oracle_step_sample(X, W, h, nt, R_full, weights / k, q)
         if i >= args.warmup:
             times.append(full)
     full_step = statistics.mean(times)
-    value = n * k / full_step / 1e9
-    sample = (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows (H-opt "
+    value = weights / full_step / 1e9
+    sample = (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows ({q[2]} "
               f"search + error) per step, {nt} threads; times scaled to the full workload")
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+    headline = args.workload == "nvfp4_full_calib" and q[:3] == ("nvfp4", 16, "hopt")
+    metric = METRIC if headline else \
+        f"G weights/s quantized ({q[2]} {q[0]} blk{q[1]}) + h-pass GB/s; % of roofline"
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(wl, 16)},
+            "config": {"workload": workload_desc(wl, *q)},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": nt, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -224,6 +242,30 @@ def reference_arm(args):
 # ---------------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------------
+
+def quantizer_for(wl, args):
+    """(fmt, block, mode, window) the bench times for a workload."""
+    block = args.block or wl.blocks[0]
+    mode = args.mode or ("hopt" if "hopt" in wl.modes else wl.modes[-1])
+    return wl.fmt, block, mode, wl.window
+
+
+def ops_per_weight(fmt, mode, window):
+    """Algorithmic lane-operations per weight of a scale search: C candidates x 6 (quotient,
+    projection, dequantise, subtract, h-multiply, square-accumulate; 5 without h) + 4
+    (amax, naive quotient, final projection, pack)."""
+    C = 64 if fmt == "e4m3" else (126 if window < 0 else 2 * window + 1)
+    return C * (6 if mode == "hopt" else 5) + 4
+
+
+def code_bytes(fmt, block):
+    """Bytes of codes + scales per weight."""
+    if fmt == "nvfp4":
+        return 0.5 + 1.0 / block
+    if fmt == "int8":
+        return 1.0 + 1.0 / block
+    return 1.0 + 4.0 / (block * block)
+
 
 def gpu_arm(args):
     import torch.distributed as dist
@@ -237,49 +279,66 @@ def gpu_arm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     wl = synth.WORKLOADS[args.workload]
-    (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
-    if args.x_rows:
-        R = min(R, args.x_rows)
-    block = 16
+    fmt, block, mode, window = quantizer_for(wl, args)
+    p = mxq.params(fmt, mode, block, window=window)
     # inputs: every rank draws its own shard (weak scaling)
-    X = torch.empty(R, k, dtype=torch.bfloat16, device=dev)
-    synth.activations(R, k, wl.seed + 1000 * rank, device=dev, n_outlier=wl.x_outliers,
-                      outlier_factor=wl.x_outlier_factor, out=X)
-    W = synth.gaussian_weight(n, k, wl.seed + 1000 * rank, device=dev)
-    p = mxq.params("nvfp4", "hopt", block)
-    h = torch.empty(k, dtype=torch.float32, device=dev)
-    colsum = torch.empty(k, dtype=torch.float64, device=dev)
-    ws = torch.empty(mxq.mxq_act_sqmean_workspace(R, k), dtype=torch.uint8, device=dev)
-    codes = torch.empty(n, k // 2, dtype=torch.uint8, device=dev)
-    scales = torch.empty(n, k // block, dtype=torch.uint8, device=dev)
-    sums = torch.empty(4, dtype=torch.float64, device=dev)
-    ews = torch.empty(mxq.mxq_error_workspace(n, k), dtype=torch.uint8, device=dev)
+    wl_r = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
+    # activations and their h, one per activation width
+    Xs, hs, wss, cols = [], [], [], []
+    for xi, (R, k) in enumerate(wl.x_shapes):
+        R = min(R, args.x_rows) if args.x_rows else R
+        X = torch.empty(R, k, dtype=wl.w_dtype, device=dev)
+        synth.workload_activations(wl_r, xi, device=dev, rows=R, out=X)
+        Xs.append(X)
+        hs.append(torch.empty(k, dtype=torch.float32, device=dev))
+        wss.append(torch.empty(mxq.mxq_act_sqmean_workspace(R, k), dtype=torch.uint8, device=dev))
+        cols.append(torch.empty(k, dtype=torch.float64, device=dev))
+    # weights and their outputs (codes, scales, error sums, error workspace, which h)
+    Ws, outs = [], []
+    for wi, (_, n, k) in enumerate(wl.weights):
+        Ws.append(synth.workload_weight(wl_r, wi, device=dev))
+        cs, cd, ss, sd = mxq.output_shapes(p, n, k)
+        outs.append((torch.empty(cs, dtype=cd, device=dev), torch.empty(ss, dtype=sd, device=dev),
+                     torch.empty(4, dtype=torch.float64, device=dev),
+                     torch.empty(mxq.mxq_error_workspace(n, k), dtype=torch.uint8, device=dev),
+                     synth.x_index_for_weight(wl, wi)))
     stream = torch.cuda.current_stream(dev)
-    # our kernels per step: h pass (2; 3 with the sharded finalize), search + exact fixup (2),
-    # error sums + combine (2)
-    launches_per_step = 6 if world == 1 else 7
+    # our kernels per step: h pass (2 per activation matrix; 3 with the sharded finalize),
+    # search (+ exact fixup for NVFP4 searches), error sums + combine (2) per weight
+    fixup = 1 if fmt == "nvfp4" and mode != "naive" else 0
+    launches_per_step = len(Xs) * (2 if world == 1 else 3) + len(Ws) * (1 + fixup + 2)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        if world == 1:
-            mxq.mxq_act_sqmean(X, h, workspace=ws)
-        else:
-            # per-rank column sums -> rank-ordered all-gather -> fixed-order finalize
-            distributed_h(X, lambda x: mxq.mxq_act_sqsum(x, colsum, workspace=ws),
-                          lambda p, r: mxq.mxq_act_sqmean_finalize(p, r, h), R * world)
+        for X, h, ws, colsum in zip(Xs, hs, wss, cols):
+            if world == 1:
+                mxq.mxq_act_sqmean(X, h, workspace=ws)
+            else:
+                # per-rank column sums -> rank-ordered all-gather -> fixed-order finalize
+                distributed_h(X, lambda x, c=colsum, w=ws: mxq.mxq_act_sqsum(x, c, workspace=w),
+                              lambda pp, r, hh=h: mxq.mxq_act_sqmean_finalize(pp, r, hh),
+                              X.shape[0] * world)
         if ev is not None:
             ev[1].record(stream)
-        mxq.mxq_quantize(W, p, h, codes=codes, scales=scales)
+        for W, (codes, scales, _, _, xi) in zip(Ws, outs):
+            mxq.mxq_quantize(W, p, hs[xi], codes=codes, scales=scales)
         if ev is not None:
             ev[2].record(stream)
-        mxq.mxq_error(W, codes, scales, p, h, sums=sums, workspace=ews)
+        for W, (codes, scales, sums, ews, xi) in zip(Ws, outs):
+            mxq.mxq_error(W, codes, scales, p, hs[xi], sums=sums, workspace=ews)
         if ev is not None:
             ev[3].record(stream)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
+
+    # Inputs smaller than a few L2s would be served from L2 on the next step: flush L2
+    # between steps (a write of twice its size) and time the steps alone.
+    in_bytes = sum(t.numel() * t.element_size() for t in Xs + Ws)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) \
+        if in_bytes < 4 * L2_BYTES else None
 
     for _ in range(args.warmup):
         step()
@@ -293,11 +352,14 @@ def gpu_arm(args):
     with sampler:
         t_start.record(stream)
         for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
-    ms_total = t_start.elapsed_time(t_end)
+    ms_total = t_start.elapsed_time(t_end) if flush is None else \
+        sum(e[0].elapsed_time(e[3]) for e in evs)
     k_h = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     k_q = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     k_e = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
@@ -306,27 +368,26 @@ def gpu_arm(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_total, k_h, k_q, k_e = t.tolist()
     ms_step = ms_total / args.steps
-    weights = n * k
+    weights = sum(W.numel() for W in Ws)
     value = world * weights / (ms_step * 1e-3) / 1e9
 
     # ---- end to end through the public API, host buffers -----------------------------
-    X_host = torch.empty(R, k, dtype=torch.bfloat16, pin_memory=True)
-    X_host.copy_(X)
-    W_host = torch.empty(n, k, dtype=torch.bfloat16, pin_memory=True)
-    W_host.copy_(W)
-    codes_host = torch.empty_like(codes, device="cpu").pin_memory()
-    scales_host = torch.empty_like(scales, device="cpu").pin_memory()
-    sums_host = torch.empty(4, dtype=torch.float64, pin_memory=True)
-    h2d = X_host.numel() * 2 + W_host.numel() * 2
-    d2h = codes_host.numel() + scales_host.numel() + 8 * 4
+    Xh = [torch.empty(X.shape, dtype=X.dtype, pin_memory=True) for X in Xs]
+    Wh = [torch.empty(W.shape, dtype=W.dtype, pin_memory=True) for W in Ws]
+    for th, td in zip(Xh + Wh, Xs + Ws):
+        th.copy_(td)
+    oh = [tuple(torch.empty(td.shape, dtype=td.dtype, pin_memory=True) for td in o[:3])
+          for o in outs]
+    h2d = sum(th.numel() * th.element_size() for th in Xh + Wh)
+    d2h = sum(th.numel() * th.element_size() for o in oh for th in o)
 
     def e2e_step():
-        X.copy_(X_host, non_blocking=True)
-        W.copy_(W_host, non_blocking=True)
+        for td, th in zip(Xs + Ws, Xh + Wh):
+            td.copy_(th, non_blocking=True)
         step()
-        codes_host.copy_(codes, non_blocking=True)
-        scales_host.copy_(scales, non_blocking=True)
-        sums_host.copy_(sums, non_blocking=True)
+        for o, ho in zip(outs, oh):
+            for td, th in zip(o[:3], ho):
+                th.copy_(td, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -344,27 +405,36 @@ def gpu_arm(args):
         dist.all_reduce(t2, op=dist.ReduceOp.MAX)
     e2e_ms = t2.item() / args.e2e_steps
     e2e_value = world * weights / (e2e_ms * 1e-3) / 1e9
-    metrics = mxq.mxq_metrics_from_sums(sums_host)
+    metrics = mxq.mxq_metrics_from_sums(oh[0][2])
 
     # ---- roofline ------------------------------------------------------------------------
     hbm, hbm_kind = measured_peaks()
-    x_bytes = R * k * 2 + 4 * k
+    headline = (args.workload == "nvfp4_full_calib" and (fmt, block, mode) ==
+                ("nvfp4", 16, "hopt") and not args.x_rows)
+    x_bytes = sum(X.numel() * X.element_size() + 4 * X.shape[1] for X in Xs)
+    w_bytes = sum(W.numel() * W.element_size() for W in Ws)
     h_gbs = x_bytes / (k_h * 1e-3) / 1e9
-    ops = OPS_PER_WEIGHT_HOPT(126) * weights
-    q_tops = ops / (k_q * 1e-3) / 1e12
-    e_bytes = weights * 2 + weights // 2 + weights // block + 4 * k
+    kernels = {"act_sqmean": {"ms": k_h, "bound": "hbm", "achieved": h_gbs, "peak": hbm,
+                              "unit": "GB/s", "frac": h_gbs / hbm, "algorithmic_bytes": x_bytes,
+                              "traffic": traffic_for("act_sqmean") if headline else None}}
+    if mode == "naive":
+        q_bytes = w_bytes + weights * code_bytes(fmt, block)
+        q_gbs = q_bytes / (k_q * 1e-3) / 1e9
+        kernels["quantize"] = {"ms": k_q, "bound": "hbm", "achieved": q_gbs, "peak": hbm,
+                               "unit": "GB/s", "frac": q_gbs / hbm, "algorithmic_bytes": q_bytes,
+                               "traffic": None}
+    else:
+        ops = ops_per_weight(fmt, mode, window) * weights
+        q_tops = ops / (k_q * 1e-3) / 1e12
+        kernels["quantize"] = {"ms": k_q, "bound": "alu", "achieved": q_tops,
+                               "peak": ALU_PEAK_TOPS, "unit": "T lane-op/s",
+                               "frac": q_tops / ALU_PEAK_TOPS, "algorithmic_ops": ops,
+                               "traffic": traffic_for("quantize") if headline else None}
+    e_bytes = w_bytes + weights * code_bytes(fmt, block) + sum(4 * W.shape[1] for W in Ws)
     e_gbs = e_bytes / (k_e * 1e-3) / 1e9
-    kernels = {
-        "act_sqmean": {"ms": k_h, "bound": "hbm", "achieved": h_gbs, "peak": hbm, "unit": "GB/s",
-                       "frac": h_gbs / hbm, "algorithmic_bytes": x_bytes,
-                       "traffic": traffic_for("act_sqmean")},
-        "quantize": {"ms": k_q, "bound": "alu", "achieved": q_tops, "peak": ALU_PEAK_TOPS,
-                     "unit": "T lane-op/s", "frac": q_tops / ALU_PEAK_TOPS,
-                     "algorithmic_ops": ops, "traffic": traffic_for("quantize")},
-        "error": {"ms": k_e, "bound": "hbm", "achieved": e_gbs, "peak": hbm, "unit": "GB/s",
-                  "frac": e_gbs / hbm, "algorithmic_bytes": e_bytes,
-                  "traffic": traffic_for("error")},
-    }
+    kernels["error"] = {"ms": k_e, "bound": "hbm", "achieved": e_gbs, "peak": hbm, "unit": "GB/s",
+                        "frac": e_gbs / hbm, "algorithmic_bytes": e_bytes,
+                        "traffic": traffic_for("error") if headline else None}
     dom = max(kernels, key=lambda kk: kernels[kk]["ms"])
     dk = kernels[dom]
     roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"],
@@ -372,17 +442,24 @@ def gpu_arm(args):
                 "traffic": dk["traffic"],
                 "peak_source": ("MEASURED_PEAKS.json hbm_gbs (" + hbm_kind + ")")
                 if dk["bound"] == "hbm" else "148 SM x 128 FP32 lanes x 1965 MHz"}
-
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+    metric = METRIC if headline else \
+        f"G weights/s quantized ({mode} {fmt} blk{block}) + h-pass GB/s; % of roofline"
+    line = {"metric": metric, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": workload_desc(wl, block), "weights_per_gpu": weights,
-                       "x_rows_per_gpu": R,
+            "config": {"workload": workload_desc(wl, fmt, block, mode, window,
+                                                 [X.shape[0] for X in Xs]),
+                       "weights_per_gpu": weights,
+                       "x_rows_per_gpu": Xs[0].shape[0] if len(Xs) == 1 else
+                       [X.shape[0] for X in Xs],
                        "parallelism": f"dp{world}" + (" (rows of X and W per rank; one "
                                                       "all-gather of column sums)" if world > 1 else ""),
-                       "l2": "inputs larger than L2: X (%.2f GB) is streamed every step"
-                             % (R * k * 2 / 1e9)},
+                       "l2": ("inputs larger than L2: X (%.2f GB) is streamed every step"
+                              % (sum(X.numel() * X.element_size() for X in Xs) / 1e9))
+                       if flush is None else
+                       ("L2 flushed between steps (a %d MB write, outside the step's events); "
+                        "inputs %.0f MB" % (2 * L2_BYTES >> 20, in_bytes / 1e6))},
             "h_pass_gbs": h_gbs, "h_pass_frac_of_hbm": h_gbs / hbm,
             "roofline": roofline, "kernels": kernels,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -392,17 +469,22 @@ def gpu_arm(args):
             "result": {"weight_rel": metrics["weight_rel"], "h_rel": metrics["h_rel"]}}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        x_rows, w_rows = CPU_X_ROWS, CPU_W_ROWS
-        Xb = bits_of(X[:x_rows].cpu())
-        Wb = bits_of(W[:w_rows].cpu())
+        X0, W0 = Xs[0], Ws[0]
+        R0, n0 = X0.shape[0], W0.shape[0]
+        x_rows = min(CPU_X_ROWS, R0)
+        w_rows = min(CPU_W_ROWS // (8 if fmt == "e4m3" else 1), n0)
+        Xb = bits_of(X0[:x_rows].cpu())
+        Wb = bits_of(W0[:w_rows].cpu())
         from oracle import oracle as orc
         nt = os.cpu_count() or 1
         h_np = orc.act_sqmean(Xb, n_threads=nt)
-        full, d = oracle_step_sample(Xb, Wb, h_np, nt, R, n)
+        # the sample's per-row times scaled to every X row and every W row of the step
+        full, d = oracle_step_sample(Xb, Wb, h_np, nt, sum(X.numel() for X in Xs) / X0.shape[1],
+                                     weights / W0.shape[1], (fmt, block, mode, window))
         line["cpu_baseline"] = {
             "value": weights / full / 1e9, "unit": UNIT, "cores": nt, "kind": "oracle",
-            "sample": (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows "
-                       f"(H-opt search + error), {nt} threads; times scaled to the full "
+            "sample": (f"oracle on {x_rows} of {R0} X rows (h) and {w_rows} of {n0} W rows "
+                       f"({mode} search + error), {nt} threads; times scaled to the full "
                        f"workload ({d['h_s']:.1f} s + {d['quant_s']:.1f} s measured)")}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -13,16 +13,18 @@
 //    itself. The quotient is formed as fma(a, r_hi, a * r_lo) with r_hi + r_lo = 1/s to
 //    ~2^-48 (host-computed split of the reciprocal), whose error (~2^-46) is far inside
 //    that gap: the result is the correctly rounded quotient, bit for bit.
-//  * INT8 and E4M3 tiles: __fdiv_rn, the IEEE-rounded division.
+//  * INT8 and E4M3 tiles rank candidates with the product |w| * fl32(1/s) instead, and
+//    widen their error brackets by the largest change that a code differing from the
+//    IEEE quotient's can make (see the INT8 and tile sections); emitted codes and exact
+//    re-scores use __fdiv_rn, the IEEE-rounded division.
 // Candidate errors are accumulated in float32 (packed f32x2 math); with every term
-// non-negative the float32 sum is within gamma = (B + 8) 2^-24 (relative) plus a tiny
-// absolute underflow slack of the exact sum. Any candidate whose lower bound does not
-// exceed the winner's upper bound is re-scored in double exactly as the plain definition
-// orders it (element order, e += c_j * (d * d)), and the smallest double error (lowest
-// index on ties) wins. So NVFP4 and INT8 picks equal the definition's, ties included.
-// E4M3 tiles accumulate float32 terms (3 roundings each) in double: the tile error is
-// within 2e-7 relative, so any pick whose two best errors differ by more than 1e-6
-// relative is exact.
+// non-negative the float32 sum is within gamma (relative) plus a tiny absolute underflow
+// slack of the exact sum. Any candidate whose lower bound does not exceed the winner's
+// upper bound is re-scored in double exactly as the plain definition orders it (element
+// order, e += c_j * (d * d)), and the smallest double error (lowest index on ties) wins.
+// So NVFP4 and INT8 picks equal the definition's, ties included. E4M3 tiles re-score in
+// double in a fixed parallel order: picks equal the definition's wherever the two best
+// tile errors differ by more than ~1e-12 relative.
 #include "mxq_common.cuh"
 #include "mxq_internal.h"
 
@@ -472,140 +474,252 @@ k_fp4_fixup(Fp4Params P, Fp4Table T) {
 }
 
 // ---------------------------------------------------------------------------------------
-// INT8 with E4M3 stored amax: one warp per block, lanes own elements j = lane + 32 t.
+// INT8 with E4M3 stored amax. G = B / 32 lanes per block, each lane owns 32 consecutive
+// elements; a warp holds 32 / G blocks of one column block in consecutive rows, so every
+// group reads the same 32 h values per lane.
+//
+// Ranking without a division. Per candidate the lanes form x = fl(|w| * r) with
+// r = fl32(1/s) and q~ = RNE(min(x, 127)) (rounding by adding 2^23, which for
+// 0 <= x < 2^23 leaves an integer, ties to even), then fl32(q~ s) as one fma
+// (q~ + 2^23) s - 2^23 s, exact because 2^23 s is. x is within 2.0001 u |w|/s of
+// the real quotient (u = 2^-24) and the definition's fl32(|w|/s) within u |w|/s, so q~
+// can differ from the definition's q (by one) only when |w|/s lies within 2.0001 u |w|/s
+// of a half-integer k + 1/2; the two dequantised values then sit on either side of |w|
+// at distance ~s/2 and their squared errors differ by at most 10 u s |w| (4 u s |w| from
+// the real identity, 6 u s |w| from the float32 rounding of q s). So every candidate's
+// float32 error brackets the definition's double error within gamma (float32 rounding,
+// at most 24 roundings deep) plus delta = 16 u s sum_j c_j |w_j|. A block whose winner
+// is not separated from every other candidate by these brackets is flagged (scale byte
+// bit 7) and re-scored exactly by k_int8_fixup.
 // ---------------------------------------------------------------------------------------
 struct Int8Params {
   const char* W;
   int64_t n, k, ld_bytes;
   const float* h;
-  int B, window;
+  int window;
   int8_t* codes;
   uint8_t* scales;
 };
 
-template <int NE, bool BF16>
-__device__ __forceinline__ void load_lane_elems(const char* row, int lane, float (&a)[NE],
-                                                uint32_t& sgn) {
-  sgn = 0;
+// Per candidate code: {s = fl32(E4M3 / 127), -fl32(1/s), -2^23 s, 0}; host-computed.
+struct Int8Table {
+  float4 c[128];
+};
+
+// Float32 error of one candidate over a lane's 32 elements, from the negated magnitudes
+// na = -|w| (d = fl32(q s) - |w| has the magnitude of the definition's difference).
+template <bool HOPT>
+__device__ __forceinline__ float int8_eval(const float2 (&na)[16], const float2 (&c)[16],
+                                           float4 t) {
+  const float2 nr = make_float2(t.y, t.y), s2 = make_float2(t.x, t.x);
+  const float2 nms = make_float2(t.z, t.z), mag = make_float2(8388608.f, 8388608.f);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int t = 0; t < NE; ++t) {
-    const int j = lane + 32 * t;
-    uint32_t bits;
-    if constexpr (BF16) bits = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(row) + j) << 16;
-    else bits = __float_as_uint(__ldg(reinterpret_cast<const float*>(row) + j));
-    sgn |= (bits >> 31) << t;
-    a[t] = __uint_as_float(bits & 0x7fffffffu);
+  for (int p = 0; p < 16; ++p) {
+    const float2 x = __fmul2_rn(na[p], nr);
+    const float2 xt = __fadd2_rn(make_float2(fminf(x.x, 127.f), fminf(x.y, 127.f)), mag);
+    const float2 d = __fadd2_rn(__ffma2_rn(xt, s2, nms), na[p]);
+    float2& acc = (p & 1) ? acc1 : acc0;
+    if constexpr (HOPT) acc = __ffma2_rn(__fmul2_rn(c[p], d), d, acc);
+    else acc = __ffma2_rn(d, d, acc);
+  }
+  return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+}
+
+// The definition's code magnitude: min(RNE(fl32(|w| / s)), 127).
+__device__ __forceinline__ int int8_code(float a, float s) {
+  return (int)fminf(rintf(__fdiv_rn(a, s)), 127.0f);
+}
+
+__device__ __forceinline__ void int8_window(int c0, int window, int& lo, int& hi) {
+  lo = 1;
+  hi = 126;
+  if (window >= 0) {
+    lo = max(1, c0 - window);
+    hi = min(126, c0 + window);
+    if (c0 == 0) hi = max(1, window);
   }
 }
 
-__device__ __forceinline__ float int8_q(float a, float s_eff) {
-  return fminf(rintf(__fdiv_rn(a, s_eff)), 127.0f);
-}
-
-template <int NE, bool BF16, int MODE>
-__global__ void __launch_bounds__(kThreads)
-k_int8(Int8Params P) {
-  constexpr int B = 32 * NE;
-  __shared__ float sa[kThreads / 32][B];
-  __shared__ float sc[kThreads / 32][B];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t kb = P.k / B, nblocks = P.n * kb;
+template <int B, bool BF16, int MODE>
+__global__ void __launch_bounds__(kThreads, 2)
+k_int8_search(Int8Params P, Int8Table T) {
+  constexpr int G = B / 32, RPW = 32 / G;
+  __shared__ float4 tab[128];
+  for (int i = threadIdx.x; i < 128; i += kThreads) tab[i] = T.c[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, sub = lane % G, grp = lane / G;
+  const int64_t kb = P.k / B, items = (P.n + RPW - 1) / RPW * kb;
   const int elsz = BF16 ? 2 : 4;
-  const float gam = (float)(NE + 16) * 5.9604645e-8f;
+  const float gam = 40.0f * 5.9604645e-8f;
   const float lo_f = 1.0f - gam, hi_f = 1.0f + 2.0f * gam;
   const float slack = 7.3468396e-40f;
+  const float kdel = 16.0f * 5.9604645e-8f;
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
-  for (int64_t b = gw; b < nblocks; b += nw) {
-    const int64_t row = b / kb, jb = b - row * kb;
-    const char* rp = P.W + row * P.ld_bytes + jb * B * elsz;
-    float a[NE], c[NE];
-    uint32_t sgn;
-    load_lane_elems<NE, BF16>(rp, lane, a, sgn);
+  for (int64_t it = gw; it < items; it += nw) {
+    const int64_t rg = it / kb, jb = it - rg * kb;
+    const int64_t row = rg * RPW + grp;
+    const bool valid = row < P.n;
+    const int64_t col = jb * B + sub * 32;
+    float2 a[16], c[16];
+    uint32_t sgn = 0;
+    if (valid) {
+      load_block<32, BF16>(P.W + row * P.ld_bytes + col * elsz, a, sgn);
+    } else {
 #pragma unroll
-    for (int t = 0; t < NE; ++t) c[t] = (MODE == 2) ? __ldg(P.h + jb * B + lane + 32 * t) : 1.0f;
-    float amax = 0.f;
+      for (int p = 0; p < 16; ++p) a[p] = make_float2(0.f, 0.f);
+    }
+    if constexpr (MODE == 2) load_h<32>(P.h + col, c);
+    float amax = block_amax<32>(a);
 #pragma unroll
-    for (int t = 0; t < NE; ++t) amax = fmaxf(amax, a[t]);
-    amax = warp_max(amax);
+    for (int o = 1; o < G; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
     const int c0 = e4m3_rn_code(amax);
     int best = c0;
-    if (MODE != 0) {
-      int lo = max(1, c0 - P.window), hi = min(126, c0 + P.window);
-      if (P.window < 0) { lo = 1; hi = 126; }
-      else if (c0 == 0) { lo = 1; hi = max(1, P.window); }
-      float m1 = __int_as_float(0x7f800000), m2 = m1;
-      int i1 = lo;
-      for (int cc = lo; cc <= hi; ++cc) {
-        const float s_eff = __fdiv_rn(e4m3_pos(cc), 127.0f);
-        float2 acc = make_float2(0.f, 0.f);
+    bool flag = false;
+    if constexpr (MODE != 0) {
+      int lo, hi;
+      int8_window(c0, P.window, lo, hi);
+      float Q = 0.f;
 #pragma unroll
-        for (int t = 0; t < NE; ++t) {
-          const float wq = __fmul_rn(int8_q(a[t], s_eff), s_eff);
-          const float d = __fsub_rn(a[t], wq);
-          if (t & 1) acc.y = fmaf(__fmul_rn(c[t], d), d, acc.y);
-          else acc.x = fmaf(__fmul_rn(c[t], d), d, acc.x);
-        }
-        const float e = warp_sum(acc.x + acc.y);
-        if (e < m1) { m2 = m1; m1 = e; i1 = cc; }
-        else if (e < m2) m2 = e;
+      for (int p = 0; p < 16; ++p) {
+        Q = (MODE == 2) ? fmaf(c[p].x, a[p].x, fmaf(c[p].y, a[p].y, Q)) : Q + (a[p].x + a[p].y);
+        a[p] = make_float2(-a[p].x, -a[p].y);
       }
-      const float upper = fmaf(m1, hi_f, slack);
-      if (!(m2 * lo_f - slack > upper)) {
-        // Rare: re-score the candidates in the band in double, element order, on lane 0.
 #pragma unroll
-        for (int t = 0; t < NE; ++t) {
-          sa[wid][lane + 32 * t] = a[t];
-          sc[wid][lane + 32 * t] = c[t];
-        }
-        __syncwarp();
-        double bestd = __longlong_as_double(0x7ff0000000000000ll);
-        int bi = i1;
-        for (int cc = lo; cc <= hi; ++cc) {
-          const float s_eff = __fdiv_rn(e4m3_pos(cc), 127.0f);
-          float2 acc = make_float2(0.f, 0.f);
+      for (int o = 1; o < G; o <<= 1) Q += __shfl_xor_sync(kFull, Q, o);
+      const int span = P.window < 0 ? 126 : 2 * P.window + 1;
+      const float inf = __int_as_float(0x7f800000);
+      float m1 = inf, hi1 = inf, l1 = inf, l2 = inf;
+      int i1 = lo, j1 = -1;
+      for (int t = 0; t < span; ++t) {
+        const int cc = lo + t;
+        const float4 tb = tab[min(cc, 126)];
+        float e = int8_eval<MODE == 2>(a, c, tb);
 #pragma unroll
-          for (int t = 0; t < NE; ++t) {
-            const float wq = __fmul_rn(int8_q(a[t], s_eff), s_eff);
-            const float d = __fsub_rn(a[t], wq);
-            if (t & 1) acc.y = fmaf(__fmul_rn(c[t], d), d, acc.y);
-            else acc.x = fmaf(__fmul_rn(c[t], d), d, acc.x);
-          }
-          const float e = warp_sum(acc.x + acc.y);
-          if (!(e * lo_f - slack > upper)) {
-            double ed = 0.0;
-            if (lane == 0) {
-              for (int j = 0; j < B; ++j) {
-                const float aj = sa[wid][j];
-                const float wq = __fmul_rn(int8_q(aj, s_eff), s_eff);
-                const double d = (double)aj - (double)wq;
-                const double cj = (MODE == 2) ? (double)sc[wid][j] : 1.0;
-                ed = __dadd_rn(ed, __dmul_rn(cj, __dmul_rn(d, d)));
-              }
-            }
-            ed = __shfl_sync(kFull, ed, 0);
-            if (ed < bestd) { bestd = ed; bi = cc; }
-          }
+        for (int o = 1; o < G; o <<= 1) e += __shfl_xor_sync(kFull, e, o);
+        if (cc <= hi) {
+          const float del = fmaf(kdel * tb.x, Q, slack);
+          const float elo = fmaf(e, lo_f, -del);
+          if (e < m1) { m1 = e; i1 = cc; hi1 = fmaf(e, hi_f, del); }
+          if (elo < l1) { l2 = l1; l1 = elo; j1 = cc; }
+          else if (elo < l2) l2 = elo;
         }
-        __syncwarp();
-        i1 = bi;
       }
+      flag = !((j1 == i1 ? l2 : l1) > hi1);
       best = i1;
-    }
-    int8_t* out = P.codes + row * P.k + jb * B;
-    const float s_eff = best ? __fdiv_rn(e4m3_pos(best), 127.0f) : 0.0f;
 #pragma unroll
-    for (int t = 0; t < NE; ++t) {
-      const int q = best ? (int)int8_q(a[t], s_eff) : 0;
-      out[lane + 32 * t] = (int8_t)(((sgn >> t) & 1u) ? -q : q);
+      for (int p = 0; p < 16; ++p) a[p] = make_float2(-a[p].x, -a[p].y);
     }
-    if (lane == 0) P.scales[b] = (uint8_t)best;
+    if (valid) {
+      const float s = tab[best].x;
+      uint32_t pk[8];
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        int q0 = best ? int8_code(a[p].x, s) : 0, q1 = best ? int8_code(a[p].y, s) : 0;
+        if ((sgn >> (2 * p)) & 1u) q0 = -q0;
+        if ((sgn >> (2 * p + 1)) & 1u) q1 = -q1;
+        const uint32_t v = ((uint32_t)q0 & 0xffu) | (((uint32_t)q1 & 0xffu) << 8);
+        if (p & 1) pk[p >> 1] |= v << 16;
+        else pk[p >> 1] = v;
+      }
+      uint4* out = reinterpret_cast<uint4*>(P.codes + row * P.k + col);
+      out[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      out[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      if (sub == 0) P.scales[row * kb + jb] = (uint8_t)(best | (flag ? 0x80 : 0));
+    }
+  }
+}
+
+// Exact pass over the INT8 blocks the search flagged. Each warp scans 32 scale bytes at a
+// time; a flagged block is staged in the warp's shared memory, lane l scores candidates
+// lo + l + 32 t in double in the definition's order (e += c_j * (d * d) over j), the warp
+// arg-min (lowest code on equal doubles) wins, and the warp rewrites the block's codes.
+template <int B, bool BF16, bool HOPT>
+__global__ void __launch_bounds__(kThreads)
+k_int8_fixup(Int8Params P, Int8Table T) {
+  constexpr int NE = B / 32;
+  __shared__ float tab[128];
+  __shared__ float sa[kThreads / 32][B];
+  __shared__ float sc[kThreads / 32][HOPT ? B : 1];
+  for (int i = threadIdx.x; i < 128; i += kThreads) tab[i] = T.c[i].x;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t kb = P.k / B, nblocks = P.n * kb;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t base = gw * 32; base < nblocks; base += nw * 32) {
+    const int64_t mine = base + lane;
+    const bool flagged = mine < nblocks && (P.scales[mine] & 0x80);
+    unsigned todo = __ballot_sync(kFull, flagged);
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int64_t b = base + src;
+      const int64_t row = b / kb, jb = b - row * kb;
+      const char* rp = P.W + row * P.ld_bytes + jb * B * (BF16 ? 2 : 4);
+      uint32_t sgn = 0;
+      float amax = 0.f;
+#pragma unroll
+      for (int t = 0; t < NE; ++t) {
+        const int j = lane + 32 * t;
+        uint32_t bits;
+        if constexpr (BF16) bits = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(rp) + j) << 16;
+        else bits = __float_as_uint(__ldg(reinterpret_cast<const float*>(rp) + j));
+        sgn |= (bits >> 31) << t;
+        const float a = __uint_as_float(bits & 0x7fffffffu);
+        sa[wid][j] = a;
+        if constexpr (HOPT) sc[wid][j] = __ldg(P.h + jb * B + j);
+        amax = fmaxf(amax, a);
+      }
+      __syncwarp();
+      int lo, hi;
+      int8_window(e4m3_rn_code(warp_max(amax)), P.window, lo, hi);
+      double best = __longlong_as_double(0x7ff0000000000000ll);
+      int bi = 0x7fffffff;
+      for (int cc = lo + lane; cc <= hi; cc += 32) {
+        const float s = tab[cc];
+        double e = 0.0;
+        for (int j = 0; j < B; ++j) {
+          const float a = sa[wid][j];
+          const float wq = __fmul_rn((float)int8_code(a, s), s);
+          const double d = (double)a - (double)wq;
+          const double cj = HOPT ? (double)sc[wid][j] : 1.0;
+          e = __dadd_rn(e, __dmul_rn(cj, __dmul_rn(d, d)));
+        }
+        if (e < best) { best = e; bi = cc; }
+      }
+      warp_argmin(best, bi);
+      if (bi > 126) bi = lo;  // every candidate NaN (non-finite input): keep the first
+      const float s = tab[bi];
+      int8_t* out = P.codes + row * P.k + jb * B;
+#pragma unroll
+      for (int t = 0; t < NE; ++t) {
+        const int j = lane + 32 * t;
+        const int q = int8_code(sa[wid][j], s);
+        out[j] = (int8_t)(((sgn >> t) & 1u) ? -q : q);
+      }
+      if (lane == 0) P.scales[b] = (uint8_t)bi;
+      __syncwarp();
+    }
   }
 }
 
 // ---------------------------------------------------------------------------------------
 // E4M3 elements, one float32 scale per 64 x 64 tile searched on a logarithmic grid.
 // One CTA (256 threads) per tile; thread t owns row t/4, columns 16 (t%4) .. +16.
+//
+// Ranking without a division: per candidate s the threads form x = fl(|w| * fl32(1/s))
+// and its E4M3 code, in float32 with packed f32x2 math. x lies within 2.0001 u |w|/s of
+// the real quotient (u = 2^-24) and the definition's fl32(|w|/s) within u |w|/s, so the
+// two codes can differ only when |w|/s is that close to a rounding midpoint m of E4M3;
+// the neighbouring values v1 < m < v2 then give squared errors that differ by
+// 2 s^2 (v2 - v1) |w/s - m| <= 8 u w^2 (spacing at most twice the value), plus at most
+// 2 u w^2 from rounding s v in float32. So each candidate's float32 error brackets the
+// definition's within gamma (float32 rounding) plus delta = 17 u sum_j c_j w_j^2. Every
+// candidate whose bracket meets the winner's is re-scored in double as the definition
+// writes it (d = |w| - fl32(s v) in double, e += c (d d)), in a fixed parallel order, and
+// the smallest double error wins (lowest grid index on equal values).
 // ---------------------------------------------------------------------------------------
 struct TileParams {
   const char* W;
@@ -622,101 +736,182 @@ struct LogGrid {
 constexpr int kTile = 64;
 constexpr int kTileChunk = 16;  // candidates per register pass
 
-__device__ __forceinline__ float e4m3_elem_wq(float a, float s, float& q_out) {
-  const float z = __fdiv_rn(a, s);
-  const uint32_t h2 = e4m3x2_to_f16x2((uint16_t)e4m3x2_rn(z, 0.0f));
-  q_out = __half2float(__ushort_as_half(lo16(h2)));
-  return __fmul_rn(s, q_out);
+// E4M3 values of the codes of two non-negative floats (RNE, saturating), as float32.
+__device__ __forceinline__ float2 e4m3x2_round_values(float x0, float x1) {
+  float v0, v1;
+  asm("{\n\t.reg .b16 q, h0, h1;\n\t.reg .b32 v;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 q, %3, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 v, q;\n\t"
+      "mov.b32 {h0, h1}, v;\n\t"
+      "cvt.f32.f16 %0, h0;\n\t"
+      "cvt.f32.f16 %1, h1;\n\t}"
+      : "=f"(v0), "=f"(v1)
+      : "f"(x0), "f"(x1));
+  return make_float2(v0, v1);
+}
+
+// Float32 error of one candidate over a thread's 16 elements; na = -|w|,
+// t = {s, -fl32(1/s)}.
+template <bool HOPT>
+__device__ __forceinline__ float tile_eval(const float2 (&na)[8], const float2 (&c)[8],
+                                           float2 t) {
+  const float2 nr = make_float2(t.y, t.y), s2 = make_float2(t.x, t.x);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const float2 x = __fmul2_rn(na[p], nr);
+    const float2 v = e4m3x2_round_values(x.x, x.y);
+    const float2 d = __fadd2_rn(__fmul2_rn(v, s2), na[p]);
+    float2& acc = (p & 1) ? acc1 : acc0;
+    if constexpr (HOPT) acc = __ffma2_rn(__fmul2_rn(c[p], d), d, acc);
+    else acc = __ffma2_rn(d, d, acc);
+  }
+  return (acc0.x + acc0.y) + (acc1.x + acc1.y);
+}
+
+// The definition's dequantised magnitude fl32(s * E4M3(RNE(fl32(a / s)))).
+__device__ __forceinline__ float e4m3_elem_wq(float a, float s) {
+  const float2 v = e4m3x2_round_values(__fdiv_rn(a, s), 0.0f);
+  return __fmul_rn(s, v.x);
 }
 
 template <bool BF16, int MODE>
 __global__ void __launch_bounds__(kThreads)
 k_e4m3_tile(TileParams P, LogGrid G) {
+  constexpr int kWarps = kThreads / 32;
   __shared__ float g[256];
-  __shared__ float red_max[kThreads / 32];
-  __shared__ double red[kThreads / 32][kTileChunk];
-  __shared__ double err[256];
-  __shared__ int pick;
+  __shared__ float2 cand[256];
+  __shared__ float errf[256];
+  __shared__ unsigned char band[256];
+  __shared__ float red[kWarps][kTileChunk];
+  __shared__ double redd[kWarps];
+  __shared__ float red_max[kWarps], red_a[kWarps];
+  __shared__ int pick, nband;
   for (int i = threadIdx.x; i < P.points; i += kThreads) g[i] = G.g[i];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int r = threadIdx.x >> 2, c0 = (threadIdx.x & 3) * 16;
   const int64_t tn = P.n / kTile, tk = P.k / kTile, ntiles = tn * tk;
   const int elsz = BF16 ? 2 : 4;
+  const float inf = __int_as_float(0x7f800000);
+  const float gam = 40.0f * 5.9604645e-8f;
+  const float lo_f = 1.0f - gam, hi_f = 1.0f + 2.0f * gam;
+  const float slack = 7.3468396e-40f;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const int64_t ti = tile / tk, tj = tile - ti * tk;
     const int64_t row = ti * kTile + r, col = tj * kTile + c0;
-    float2 a2[8];
+    float2 na[8], c[8];
     uint32_t sgn;
-    load_block<16, BF16>(P.W + row * P.ld_bytes + col * elsz, a2, sgn);
-    float a[16], c[16];
+    load_block<16, BF16>(P.W + row * P.ld_bytes + col * elsz, na, sgn);
+    if constexpr (MODE == 2) load_h<16>(P.h + col, c);
+    else {
 #pragma unroll
-    for (int p = 0; p < 8; ++p) { a[2 * p] = a2[p].x; a[2 * p + 1] = a2[p].y; }
+      for (int p = 0; p < 8; ++p) c[p] = make_float2(1.f, 1.f);
+    }
+    float am = block_amax<16>(na), aw = 0.f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) c[j] = (MODE == 2) ? __ldg(P.h + col + j) : 1.0f;
-    float am = 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) am = fmaxf(am, a[j]);
+    for (int p = 0; p < 8; ++p) {
+      aw = fmaf(c[p].x * na[p].x, na[p].x, fmaf(c[p].y * na[p].y, na[p].y, aw));
+      na[p] = make_float2(-na[p].x, -na[p].y);
+    }
     am = warp_max(am);
-    if (lane == 0) red_max[wid] = am;
+    aw = warp_sum(aw);
+    if (lane == 0) { red_max[wid] = am; red_a[wid] = aw; }
     __syncthreads();
     am = red_max[0];
+    aw = red_a[0];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) am = fmaxf(am, red_max[w]);
+    for (int w = 1; w < kWarps; ++w) { am = fmaxf(am, red_max[w]); aw += red_a[w]; }
     const float base = __fdiv_rn(am, 448.0f);
     float s = base;
     if (MODE != 0 && base > 0.0f) {
+      // A candidate below 2^-100 would push 1/s, x or s v out of the normal float32
+      // range the bracket assumes: it gets the bracket [0, inf) (always re-scored).
+      for (int p = threadIdx.x; p < P.points; p += kThreads) {
+        const float sp = __fmul_rn(base, g[p]);
+        const bool fast = sp >= 0x1p-100f;
+        cand[p] = make_float2(sp, fast ? -__frcp_rn(sp) : 0.0f);
+        band[p] = sp > 0.0f && !fast;
+      }
+      __syncthreads();
       for (int p0 = 0; p0 < P.points; p0 += kTileChunk) {
-        double part[kTileChunk];
+        float part[kTileChunk];
 #pragma unroll
         for (int u = 0; u < kTileChunk; ++u) {
-          part[u] = 0.0;
           const int p = p0 + u;
-          if (p < P.points) {
-            const float sp = __fmul_rn(base, g[p]);
-            if (sp > 0.0f) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                float q;
-                const float d = __fsub_rn(a[j], e4m3_elem_wq(a[j], sp, q));
-                part[u] += (double)__fmul_rn(__fmul_rn(c[j], d), d);
-              }
-            }
-          }
+          part[u] = 0.f;
+          if (p < P.points && cand[p].y != 0.0f) part[u] = tile_eval<MODE == 2>(na, c, cand[p]);
         }
 #pragma unroll
         for (int u = 0; u < kTileChunk; ++u) {
-          double v = warp_sum(part[u]);
+          const float v = warp_sum(part[u]);
           if (lane == 0) red[wid][u] = v;
         }
         __syncthreads();
         if (threadIdx.x < kTileChunk && p0 + (int)threadIdx.x < P.points) {
           const int p = p0 + threadIdx.x;
-          double e = 0.0;
+          float e = red[0][threadIdx.x];
 #pragma unroll
-          for (int w = 0; w < kThreads / 32; ++w) e += red[w][threadIdx.x];
-          const float sp = __fmul_rn(base, g[p]);
-          err[p] = sp > 0.0f ? e : __longlong_as_double(0x7ff0000000000000ll);
+          for (int w = 1; w < kWarps; ++w) e += red[w][threadIdx.x];
+          errf[p] = cand[p].y != 0.0f ? e : inf;
         }
         __syncthreads();
       }
       if (wid == 0) {
-        double v = __longlong_as_double(0x7ff0000000000000ll);
+        float v = inf;
         int vi = 0x7fffffff;
-        for (int p = lane; p < P.points; p += 32) {
-          if (err[p] < v) { v = err[p]; vi = p; }
-        }
+        for (int p = lane; p < P.points; p += 32)
+          if (errf[p] < v) { v = errf[p]; vi = p; }
         warp_argmin(v, vi);
-        if (lane == 0) pick = (v < __longlong_as_double(0x7ff0000000000000ll)) ? vi : -1;
+        const float del = fmaf(17.0f * 5.9604645e-8f, aw, slack);
+        const float hi1 = fmaf(v, hi_f, del);
+        int cnt = 0;
+        for (int p = lane; p < P.points; p += 32) {
+          const bool in = band[p] || (p != vi && errf[p] < inf &&
+                                       !(fmaf(errf[p], lo_f, -del) > hi1));
+          band[p] = in;
+          cnt += in;
+        }
+        cnt = __reduce_add_sync(kFull, cnt);
+        if (lane == 0) { pick = v < inf ? vi : -1; nband = cnt; }
       }
       __syncthreads();
-      s = pick >= 0 ? __fmul_rn(base, g[pick]) : 0.0f;
+      if (nband > 0) {
+        // Re-score the winner and every candidate in its band in double.
+        const int first = pick;
+        double bestd = __longlong_as_double(0x7ff0000000000000ll);
+        int bi = first;
+        for (int p = 0; p < P.points; ++p) {
+          if (p != first && !band[p]) continue;
+          const float sp = cand[p].x;
+          double e = 0.0;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const double d0 = (double)(-na[q].x) - (double)e4m3_elem_wq(-na[q].x, sp);
+            const double d1 = (double)(-na[q].y) - (double)e4m3_elem_wq(-na[q].y, sp);
+            e += (double)c[q].x * (d0 * d0);
+            e += (double)c[q].y * (d1 * d1);
+          }
+          e = warp_sum(e);
+          if (lane == 0) redd[wid] = e;
+          __syncthreads();
+          e = redd[0];
+#pragma unroll
+          for (int w = 1; w < kWarps; ++w) e += redd[w];
+          if (e < bestd || (e == bestd && p < bi)) { bestd = e; bi = p; }
+          __syncthreads();
+        }
+        if (threadIdx.x == 0) pick = bi;
+        __syncthreads();
+      }
+      s = pick >= 0 ? cand[pick].x : 0.0f;
     }
     // emit 16 bytes per thread
     uint32_t wds[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int j = 0; j < 16; j += 2) {
+      const float a0 = -na[j / 2].x, a1 = -na[j / 2].y;
       uint32_t pair = 0;
-      if (s > 0.0f) pair = e4m3x2_rn(__fdiv_rn(a[j], s), __fdiv_rn(a[j + 1], s)) & 0x7f7fu;
+      if (s > 0.0f) pair = e4m3x2_rn(__fdiv_rn(a0, s), __fdiv_rn(a1, s)) & 0x7f7fu;
       pair |= ((sgn >> j) & 1u) << 7;
       pair |= ((sgn >> (j + 1)) & 1u) << 15;
       wds[j / 4] |= pair << (8 * (j % 4));
@@ -739,7 +934,7 @@ __global__ void k_project(const float* __restrict__ w, int64_t count, int fmt, f
       const float2 x = fp4_quot(make_float2(a, 0.f), make_float2(rhi, rhi), make_float2(rlo, rlo));
       code = e2m1x2_rn(x.x, 0.f) & 7u;
     } else if (fmt == 1) {
-      code = (uint32_t)int8_q(a, __fdiv_rn(scale, 127.0f));
+      code = (uint32_t)int8_code(a, __fdiv_rn(scale, 127.0f));
     } else {
       code = e4m3x2_rn(__fdiv_rn(a, scale), 0.f) & 0x7fu;
     }
@@ -802,15 +997,47 @@ cudaError_t fp4_dispatch(const QuantArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int NE, bool BF16>
+Int8Table make_int8_table() {
+  Int8Table t;
+  for (int c = 0; c < 128; ++c) {
+    if (c == 0 || c == 127) {
+      t.c[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    const int e = c >> 3, m = c & 7;
+    const float v = (float)(e == 0 ? (double)m / 8.0 * (1.0 / 64.0)
+                                   : (1.0 + m / 8.0) * ldexp(1.0, e - 7));  // exact
+    volatile float s = v / 127.0f;  // IEEE float32 division, as on the device
+    const float sf = s;
+    volatile float r = 1.0f / sf;
+    t.c[c] = make_float4(sf, -(float)r, -8388608.0f * sf, 0.f);
+  }
+  return t;
+}
+
+template <int B, bool BF16>
 cudaError_t int8_dispatch(const QuantArgs& a, cudaStream_t st) {
-  Int8Params P{(const char*)a.W, a.n, a.k, a.ld * (BF16 ? 2 : 4), a.h, a.block, a.window,
+  static const Int8Table T = make_int8_table();
+  Int8Params P{(const char*)a.W, a.n, a.k, a.ld * (BF16 ? 2 : 4), a.h, a.window,
                (int8_t*)a.codes, (uint8_t*)a.scales};
-  const int64_t nblocks = a.n * (a.k / a.block);
-  const int grid = grid_for(nblocks * 32);
-  if (a.mode == 0) k_int8<NE, BF16, 0><<<grid, kThreads, 0, st>>>(P);
-  else if (a.mode == 1) k_int8<NE, BF16, 1><<<grid, kThreads, 0, st>>>(P);
-  else k_int8<NE, BF16, 2><<<grid, kThreads, 0, st>>>(P);
+  constexpr int RPW = 32 / (B / 32);
+  const int64_t items = (a.n + RPW - 1) / RPW * (a.k / B);
+  const int64_t want = (items * 32 + kThreads - 1) / kThreads;
+  const int64_t cap = (int64_t)sm_count() * 2;
+  const int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
+  if (a.mode == 0) {
+    k_int8_search<B, BF16, 0><<<grid, kThreads, 0, st>>>(P, T);
+    return cudaGetLastError();
+  }
+  if (a.mode == 1) k_int8_search<B, BF16, 1><<<grid, kThreads, 0, st>>>(P, T);
+  else k_int8_search<B, BF16, 2><<<grid, kThreads, 0, st>>>(P, T);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t nblocks = a.n * (a.k / B);
+  const int64_t fwant = (nblocks + 32 * 8 - 1) / (32 * 8);
+  const int fgrid = (int)(fwant < (int64_t)sm_count() * 8 ? fwant : (int64_t)sm_count() * 8);
+  if (a.mode == 1) k_int8_fixup<B, BF16, false><<<fgrid, kThreads, 0, st>>>(P, T);
+  else k_int8_fixup<B, BF16, true><<<fgrid, kThreads, 0, st>>>(P, T);
   return cudaGetLastError();
 }
 
@@ -854,10 +1081,10 @@ cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
   }
   if (a.fmt == 1) {
     switch (a.block) {
-      case 32: return bf ? int8_dispatch<1, true>(a, st) : int8_dispatch<1, false>(a, st);
-      case 64: return bf ? int8_dispatch<2, true>(a, st) : int8_dispatch<2, false>(a, st);
-      case 128: return bf ? int8_dispatch<4, true>(a, st) : int8_dispatch<4, false>(a, st);
-      default: return bf ? int8_dispatch<8, true>(a, st) : int8_dispatch<8, false>(a, st);
+      case 32: return bf ? int8_dispatch<32, true>(a, st) : int8_dispatch<32, false>(a, st);
+      case 64: return bf ? int8_dispatch<64, true>(a, st) : int8_dispatch<64, false>(a, st);
+      case 128: return bf ? int8_dispatch<128, true>(a, st) : int8_dispatch<128, false>(a, st);
+      default: return bf ? int8_dispatch<256, true>(a, st) : int8_dispatch<256, false>(a, st);
     }
   }
   return bf ? tile_dispatch<true>(a, st) : tile_dispatch<false>(a, st);
