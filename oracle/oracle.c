@@ -18,6 +18,13 @@
  *    naive / SSE-optimal / H-optimal; FP4 decisions at the 0.75, 1.75, 3.5 boundaries;
  *    section "Exotic Scales": the E2M1 codebook {0, 0.5, 1, 1.5, 2, 3, 4, 6} and the count
  *    of 126 positive E4M3 values.
+ *  - qwantize "Results", section "MXFP4 (UE8M0 power-of-2 scales)": E2M1 elements with a
+ *    power-of-two block scale; sections "GPTQ Quantization" (the NVINT4 rows) and "Larger
+ *    blocks": INT4 elements, symmetric 0..7, with an E4M3 block scale; section "Exotic
+ *    Scales": the unsigned 8-bit scale formats UE4M4 (4 exponent bits, bias 7, 4 mantissa
+ *    bits, max 496) and UE5M3 (5 exponent bits, bias 15, 3 mantissa bits, max 122880),
+ *    every code finite, 255 positive values each.
+ *  - "Is Finer Better? ...", sec. 2.1: the OCP microscaling scale E8M0, 2^-127 .. 2^127.
  *  - "quantization_algorithms.txt", section 1 (Activation-weighted scale search): the
  *    diagonal objective sum_ij h_j (w_ij - s Q(w_ij / s))^2 with h_j = E[x_j^2]; a
  *    logarithmic grid of tile scales; section 2: nearest-E4M3 projection by binary search
@@ -30,7 +37,13 @@
  *    e += c_j * (d * d) with d = (double)w - (double)fl32(s * q);
  *  - candidate ties go to the lowest candidate index (the smallest scale);
  *  - a naive scale that rounds to E4M3 code 0 gives all-zero magnitudes (sign bits kept);
- *    the search never picks code 0; a window around code 0 is [1, w].
+ *    the search never picks code 0; a window around code 0 is [1, w]. The same holds for
+ *    the other scale formats whose code 0 is zero (UE4M4, UE5M3);
+ *  - the naive UE8M0 (MXFP4) scale is the OCP rule 2^(floor(log2 amax) - 2), 2 being the
+ *    largest E2M1 exponent, clamped to the E8M0 range (code 0 for amax = 0); the naive
+ *    scale of every other grid is the grid's nearest value to amax / qmax (qmax = 6 for
+ *    E2M1, 7 for INT4, 1 for the INT8 stored amax);
+ *  - INT4 codes are two's-complement nibbles in [-7, 7], element 2i in the low nibble.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fPIC -shared oracle.c -lm
  * (no fused multiply-add: every product and sum above is a separately rounded step).
@@ -64,17 +77,72 @@ double orc_e2m1_value(int code)
     return s ? -v : v;
 }
 
+/* UE4M4 (unsigned, every code finite): 4 exponent bits with bias 7, 4 mantissa bits.
+ * Exponent field 0 encodes m/16 * 2^-6, otherwise (1 + m/16) * 2^(e-7). */
+double orc_ue4m4_value(int code)
+{
+    int e = (code >> 4) & 15, m = code & 15;
+    if (e == 0) return ldexp((double)m / 16.0, -6);
+    return ldexp(1.0 + (double)m / 16.0, e - 7);
+}
+
+/* UE5M3 (unsigned, every code finite): 5 exponent bits with bias 15, 3 mantissa bits.
+ * Exponent field 0 encodes m/8 * 2^-14, otherwise (1 + m/8) * 2^(e-15). */
+double orc_ue5m3_value(int code)
+{
+    int e = (code >> 3) & 31, m = code & 7;
+    if (e == 0) return ldexp((double)m / 8.0, -14);
+    return ldexp(1.0 + (double)m / 8.0, e - 15);
+}
+
+/* UE8M0: the power of two 2^(code - 127); code 255 is NaN. */
+double orc_ue8m0_value(int code)
+{
+    if ((code & 255) == 255) return NAN;
+    return ldexp(1.0, (code & 255) - 127);
+}
+
 /* Sorted tables of the non-negative grid values; the table index is the magnitude code
- * (for E4M3 and E2M1 the codes of positive values increase with the value). */
+ * (for every format here the codes of positive values increase with the value). */
 static float T_E4M3[127];   /* codes 0x00 .. 0x7E: 0, 2^-9, ..., 448 */
 static float T_E2M1[8];     /* codes 0 .. 7: 0, 0.5, ..., 6 */
-static float T_INT[128];    /* 0 .. 127 */
+static float T_INT[128];    /* 0 .. 127 (its first 8 entries are the INT4 magnitudes) */
+static float T_UE4M4[256];  /* 0, 2^-10, ..., 496 */
+static float T_UE5M3[256];  /* 0, 2^-17, ..., 122880 */
+static float T_UE8M0[255];  /* 2^-127, ..., 2^127 */
 
 __attribute__((constructor)) static void orc_init_tables(void)
 {
     for (int c = 0; c < 127; ++c) T_E4M3[c] = (float)orc_e4m3_value(c);
     for (int c = 0; c < 8; ++c) T_E2M1[c] = (float)orc_e2m1_value(c);
     for (int c = 0; c < 128; ++c) T_INT[c] = (float)c;
+    for (int c = 0; c < 256; ++c) T_UE4M4[c] = (float)orc_ue4m4_value(c);
+    for (int c = 0; c < 256; ++c) T_UE5M3[c] = (float)orc_ue5m3_value(c);
+    for (int c = 0; c < 255; ++c) T_UE8M0[c] = (float)orc_ue8m0_value(c);
+}
+
+/* The block-scale grids: table, number of codes, first candidate code of a search. */
+enum { ORC_S_E4M3 = 0, ORC_S_UE4M4 = 1, ORC_S_UE5M3 = 2, ORC_S_UE8M0 = 3 };
+typedef struct { const float *tab; int n; int first; } scale_grid;
+
+static int grid_of(int sfmt, scale_grid *g)
+{
+    switch (sfmt) {
+    case ORC_S_E4M3: *g = (scale_grid){T_E4M3, 127, 1}; return 0;
+    case ORC_S_UE4M4: *g = (scale_grid){T_UE4M4, 256, 1}; return 0;
+    case ORC_S_UE5M3: *g = (scale_grid){T_UE5M3, 256, 1}; return 0;
+    case ORC_S_UE8M0: *g = (scale_grid){T_UE8M0, 255, 0}; return 0;
+    default: return -1;
+    }
+}
+
+/* Copy of a scale grid's table (out holds 256 floats); returns the number of codes. */
+int orc_scale_table(int sfmt, float *out)
+{
+    scale_grid g;
+    if (grid_of(sfmt, &g)) return -1;
+    memcpy(out, g.tab, sizeof(float) * (size_t)g.n);
+    return g.n;
 }
 
 /* Copies of the tables, for the self-tests. */
@@ -112,7 +180,7 @@ int orc_int127_rne(float x) { return nearest_rne(T_INT, 128, x); }
  * ---------------------------------------------------------------------------------- */
 
 enum { ORC_F32 = 0, ORC_BF16 = 1 };
-enum { ORC_NVFP4 = 0, ORC_INT8 = 1, ORC_E4M3 = 2 };
+enum { ORC_NVFP4 = 0, ORC_INT8 = 1, ORC_E4M3 = 2, ORC_INT4 = 3 };
 enum { ORC_NAIVE = 0, ORC_SSE = 1, ORC_HOPT = 2 };
 
 static float bf16_to_float(uint16_t b)
@@ -158,19 +226,29 @@ void orc_act_sqmean(const void *X, int dtype, int64_t rows, int64_t cols, int64_
  * E4M3 scale byte.
  * ---------------------------------------------------------------------------------- */
 
-/* The magnitude code of element w at candidate scale code c, and its dequantised value
- * fl32(scale * q) (without sign). NVFP4: scale = E4M3(c), q = E2M1 nearest of
- * fl32(|w| / scale). INT8: scale = fl32(E4M3(c) / 127), q = nearest integer in [0, 127]
- * of fl32(|w| / scale). Scale code 0 (a naive snap to zero) gives q = 0. */
-static int project(int fmt, int c, float w, float *wq_abs)
+/* The magnitude code of element w at candidate scale code c of grid sfmt, and its
+ * dequantised value fl32(scale * q) (without sign). NVFP4 (E2M1 elements): scale = the
+ * grid value, q = E2M1 nearest of fl32(|w| / scale). INT4: q = nearest integer in [0, 7]
+ * of fl32(|w| / scale). INT8 (E4M3 grid only): scale = fl32(E4M3(c) / 127), q = nearest
+ * integer in [0, 127] of fl32(|w| / scale). A zero scale (a naive snap to zero) gives
+ * q = 0. */
+static int project(int fmt, int sfmt, int c, float w, float *wq_abs)
 {
     float a = fabsf(w);
-    if (c == 0) { *wq_abs = 0.0f; return 0; }
+    scale_grid g;
+    if (grid_of(sfmt, &g)) { *wq_abs = NAN; return 0; }
+    if (g.tab[c] == 0.0f) { *wq_abs = 0.0f; return 0; }
     if (fmt == ORC_NVFP4) {
-        float s = T_E4M3[c];
+        float s = g.tab[c];
         float z = a / s;
         int q = nearest_rne(T_E2M1, 8, z);
         *wq_abs = s * T_E2M1[q];
+        return q;
+    } else if (fmt == ORC_INT4) {
+        float s = g.tab[c];
+        float z = a / s;
+        int q = nearest_rne(T_INT, 8, z);
+        *wq_abs = (float)q * s;
         return q;
     } else {
         float s = T_E4M3[c] / 127.0f;
@@ -182,20 +260,24 @@ static int project(int fmt, int c, float w, float *wq_abs)
 }
 
 /* Exported for the exhaustive projection self-tests. */
-int orc_project(int fmt, int c, float w, float *wq_abs) { return project(fmt, c, w, wq_abs); }
-
-void orc_project_many(int fmt, int c, const float *w, int64_t count, uint8_t *q, float *wq_abs)
+int orc_project(int fmt, int sfmt, int c, float w, float *wq_abs)
 {
-    for (int64_t i = 0; i < count; ++i) q[i] = (uint8_t)project(fmt, c, w[i], &wq_abs[i]);
+    return project(fmt, sfmt, c, w, wq_abs);
+}
+
+void orc_project_many(int fmt, int sfmt, int c, const float *w, int64_t count, uint8_t *q,
+                      float *wq_abs)
+{
+    for (int64_t i = 0; i < count; ++i) q[i] = (uint8_t)project(fmt, sfmt, c, w[i], &wq_abs[i]);
 }
 
 /* Block error at candidate c: sum_j c_j (w_j - wq_j)^2 in double, element order. */
-static double block_error(int fmt, int c, const float *w, const float *cw, int B)
+static double block_error(int fmt, int sfmt, int c, const float *w, const float *cw, int B)
 {
     double e = 0.0;
     for (int j = 0; j < B; ++j) {
         float wq_abs;
-        project(fmt, c, w[j], &wq_abs);
+        project(fmt, sfmt, c, w[j], &wq_abs);
         float wq = copysignf(wq_abs, w[j]);
         double d = (double)w[j] - (double)wq;
         e += (double)cw[j] * (d * d);
@@ -203,34 +285,55 @@ static double block_error(int fmt, int c, const float *w, const float *cw, int B
     return e;
 }
 
-/* Naive snap: NVFP4 E4M3(fl32(amax / 6)); INT8 E4M3(amax) (the stored amax). */
-static int naive_code(int fmt, float amax)
+/* Naive snap. NVFP4 on E4M3: E4M3(fl32(amax / 6)); INT8: E4M3(amax) (the stored amax);
+ * UE8M0: 2^(floor(log2 amax) - 2) (OCP), clamped to codes 0 .. 254; every other grid:
+ * its nearest value to fl32(amax / qmax), qmax = 6 (E2M1) or 7 (INT4). */
+static int naive_code(int fmt, int sfmt, float amax)
 {
-    if (fmt == ORC_NVFP4) return nearest_rne(T_E4M3, 127, amax / 6.0f);
-    return nearest_rne(T_E4M3, 127, amax);
+    scale_grid g;
+    if (fmt == ORC_INT8) return nearest_rne(T_E4M3, 127, amax);
+    if (fmt == ORC_NVFP4 && sfmt == ORC_S_E4M3) return nearest_rne(T_E4M3, 127, amax / 6.0f);
+    if (sfmt == ORC_S_UE8M0) {
+        if (!(amax > 0.0f)) return 0;
+        int ex;
+        frexp((double)amax, &ex);           /* amax = f 2^ex, 0.5 <= f < 1 */
+        int c = (ex - 1) - 2 + 127;
+        return c < 0 ? 0 : (c > 254 ? 254 : c);
+    }
+    if (grid_of(sfmt, &g)) return -1;
+    float qmax = (fmt == ORC_NVFP4) ? 6.0f : 7.0f;
+    return nearest_rne(g.tab, g.n, amax / qmax);
 }
 
-int orc_naive_code(int fmt, float amax) { return naive_code(fmt, amax); }
+int orc_naive_code(int fmt, int sfmt, float amax) { return naive_code(fmt, sfmt, amax); }
 
 /*
  * Quantize rows [row0, row1) of W [n, k] (leading dimension ld) in blocks of B along k.
- * fmt: ORC_NVFP4 or ORC_INT8. mode: ORC_NAIVE, ORC_SSE or ORC_HOPT (h required).
- * window < 0: every positive E4M3 scale code 1..126; otherwise codes [c0-window,
- * c0+window] clipped to [1, 126], c0 the naive code.
+ * fmt: ORC_NVFP4 (E2M1 elements), ORC_INT4 or ORC_INT8; sfmt: the scale grid
+ * (ORC_S_E4M3 for all three; UE4M4, UE5M3 or UE8M0 for E2M1 elements; UE4M4 or UE5M3 for
+ * INT4). mode: ORC_NAIVE, ORC_SSE or ORC_HOPT (h required).
+ * window < 0: every candidate code of the grid (E4M3 1..126, UE4M4 / UE5M3 1..255, UE8M0
+ * 0..254); otherwise codes [c0-window, c0+window] clipped to that range, c0 the naive code.
  * Outputs (row-major, all n rows addressable): codes -- NVFP4 [n][k/2] with element 2i in
- * the low nibble, nibble = sign << 3 | E2M1 code; INT8 [n][k] two's complement.
- * scales [n][k/B] E4M3 codes. Optional (may be NULL): best / second [n][k/B] -- the
+ * the low nibble, nibble = sign << 3 | E2M1 code; INT4 [n][k/2], same nibble order, the
+ * nibble the two's complement of the signed code; INT8 [n][k] two's complement.
+ * scales [n][k/B] scale codes. Optional (may be NULL): best / second [n][k/B] -- the
  * smallest and the second-smallest candidate error (second = +inf with one candidate;
  * both NaN in naive mode), naive [n][k/B] the naive code.
  * Returns 0, or -1 on bad arguments.
  */
 int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
-                        const float *h, int fmt, int mode, int B, int window,
+                        const float *h, int fmt, int sfmt, int mode, int B, int window,
                         int64_t row0, int64_t row1, uint8_t *codes, uint8_t *scales,
                         double *best, double *second, int32_t *naive)
 {
-    if (B <= 0 || k % B != 0 || (fmt != ORC_NVFP4 && fmt != ORC_INT8)) return -1;
+    scale_grid g;
+    if (B <= 0 || k % B != 0 || grid_of(sfmt, &g)) return -1;
+    if (fmt != ORC_NVFP4 && fmt != ORC_INT8 && fmt != ORC_INT4) return -1;
+    if (fmt == ORC_INT8 && sfmt != ORC_S_E4M3) return -1;
+    if (fmt == ORC_INT4 && sfmt == ORC_S_UE8M0) return -1;
     if (mode == ORC_HOPT && h == NULL) return -1;
+    const int cmax = g.n - 1;
     int64_t kb = k / B;
     float *w = (float *)malloc(sizeof(float) * (size_t)B);
     float *cw = (float *)malloc(sizeof(float) * (size_t)B);
@@ -243,19 +346,19 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
                 cw[j] = (mode == ORC_HOPT) ? h[j0 + j] : 1.0f;
                 if (fabsf(w[j]) > amax) amax = fabsf(w[j]);
             }
-            int c0 = naive_code(fmt, amax);
+            int c0 = naive_code(fmt, sfmt, amax);
             int cbest = c0;
             double e1 = NAN, e2 = NAN;
             if (mode != ORC_NAIVE) {
-                int lo = 1, hi = 126;
+                int lo = g.first, hi = cmax;
                 if (window >= 0) {
-                    lo = c0 - window < 1 ? 1 : c0 - window;
-                    hi = c0 + window > 126 ? 126 : c0 + window;
-                    if (c0 == 0) { lo = 1; hi = window < 1 ? 1 : window; }
+                    lo = c0 - window < g.first ? g.first : c0 - window;
+                    hi = c0 + window > cmax ? cmax : c0 + window;
+                    if (g.tab[c0] == 0.0f) { lo = 1; hi = window < 1 ? 1 : window; }
                 }
                 e1 = INFINITY; e2 = INFINITY; cbest = lo;
                 for (int c = lo; c <= hi; ++c) {
-                    double e = block_error(fmt, c, w, cw, B);
+                    double e = block_error(fmt, sfmt, c, w, cw, B);
                     if (e < e1) { e2 = e1; e1 = e; cbest = c; }
                     else if (e < e2) e2 = e;
                 }
@@ -266,10 +369,11 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
             if (naive) naive[i * kb + b] = c0;
             for (int j = 0; j < B; ++j) {
                 float wq_abs;
-                int q = project(fmt, cbest, w[j], &wq_abs);
+                int q = project(fmt, sfmt, cbest, w[j], &wq_abs);
                 int neg = signbit(w[j]) ? 1 : 0;
-                if (fmt == ORC_NVFP4) {
-                    uint8_t nib = (uint8_t)((neg << 3) | q);
+                if (fmt == ORC_NVFP4 || fmt == ORC_INT4) {
+                    uint8_t nib = (fmt == ORC_NVFP4) ? (uint8_t)((neg << 3) | q)
+                                                     : (uint8_t)((neg ? -q : q) & 15);
                     uint8_t *p = &codes[i * (k / 2) + (j0 + j) / 2];
                     if (((j0 + j) & 1) == 0) *p = (uint8_t)((*p & 0xF0) | nib);
                     else *p = (uint8_t)((*p & 0x0F) | (nib << 4));
@@ -387,20 +491,29 @@ int orc_quantize_tiles(const void *W, int dtype, int64_t n, int64_t k, int64_t l
  * ||Q(W) - W||_F / ||W||_F; the h-weighted error is the diagonal objective itself).
  * ---------------------------------------------------------------------------------- */
 
-/* W^ [n][k] float from codes and scales. fmt as above; B the block (tile edge for E4M3). */
-int orc_dequant(const uint8_t *codes, const void *scales, int fmt, int B, int64_t n,
+/* W^ [n][k] float from codes and scales. fmt / sfmt as above; B the block (tile edge for
+ * E4M3 elements, whose scales are floats). */
+int orc_dequant(const uint8_t *codes, const void *scales, int fmt, int sfmt, int B, int64_t n,
                 int64_t k, float *out)
 {
-    if (B <= 0 || k % B != 0) return -1;
+    scale_grid g;
+    if (B <= 0 || k % B != 0 || grid_of(sfmt, &g)) return -1;
     for (int64_t i = 0; i < n; ++i)
         for (int64_t j = 0; j < k; ++j) {
             float v;
-            if (fmt == ORC_NVFP4) {
+            if (fmt == ORC_NVFP4 || fmt == ORC_INT4) {
                 uint8_t byte = codes[i * (k / 2) + j / 2];
                 int nib = (j & 1) ? (byte >> 4) : (byte & 15);
-                float s = T_E4M3[((const uint8_t *)scales)[i * (k / B) + j / B]];
-                v = s * T_E2M1[nib & 7];
-                if (nib & 8) v = -v;
+                int sc = ((const uint8_t *)scales)[i * (k / B) + j / B];
+                float s = sc < g.n ? g.tab[sc] : NAN;
+                if (fmt == ORC_NVFP4) {
+                    v = s * T_E2M1[nib & 7];
+                    if (nib & 8) v = -v;
+                } else {
+                    int q = (nib & 8) ? 16 - nib : nib;       /* magnitude of the signed nibble */
+                    v = (float)q * s;
+                    if (nib & 8) v = -v;
+                }
             } else if (fmt == ORC_INT8) {
                 int q = ((const int8_t *)codes)[i * k + j];
                 float s = T_E4M3[((const uint8_t *)scales)[i * (k / B) + j / B]] / 127.0f;

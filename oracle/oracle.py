@@ -25,9 +25,11 @@ _lib = None
 _lock = threading.Lock()
 
 F32, BF16 = 0, 1
-NVFP4, INT8, E4M3 = 0, 1, 2
+NVFP4, INT8, E4M3, INT4 = 0, 1, 2, 3
 NAIVE, SSE, HOPT = 0, 1, 2
-FMTS = {"nvfp4": NVFP4, "int8": INT8, "e4m3": E4M3}
+FMTS = {"nvfp4": NVFP4, "int8": INT8, "e4m3": E4M3, "int4": INT4}
+# block-scale grids (sfmt): "mxfp4" is E2M1 elements ("nvfp4") on the "ue8m0" grid
+SFMTS = {"e4m3": 0, "ue4m4": 1, "ue5m3": 2, "ue8m0": 3}
 MODES = {"naive": NAIVE, "sse": SSE, "hopt": HOPT}
 
 _P = ctypes.c_void_p
@@ -50,31 +52,36 @@ def lib():
             L.orc_e4m3_value.argtypes = [_I]
             L.orc_e2m1_value.restype = _D
             L.orc_e2m1_value.argtypes = [_I]
+            for f in ("orc_ue4m4_value", "orc_ue5m3_value", "orc_ue8m0_value"):
+                getattr(L, f).restype = _D
+                getattr(L, f).argtypes = [_I]
+            L.orc_scale_table.restype = _I
+            L.orc_scale_table.argtypes = [_I, _P]
             L.orc_e4m3_table.argtypes = [_P]
             L.orc_e2m1_table.argtypes = [_P]
             for f in ("orc_e4m3_rne_code", "orc_e2m1_rne_code", "orc_int127_rne"):
                 getattr(L, f).restype = _I
                 getattr(L, f).argtypes = [ctypes.c_float]
             L.orc_project.restype = _I
-            L.orc_project.argtypes = [_I, _I, ctypes.c_float, ctypes.POINTER(ctypes.c_float)]
+            L.orc_project.argtypes = [_I, _I, _I, ctypes.c_float, ctypes.POINTER(ctypes.c_float)]
             L.orc_project_e4m3.restype = _I
             L.orc_project_e4m3.argtypes = [ctypes.c_float, ctypes.c_float,
                                            ctypes.POINTER(ctypes.c_float)]
-            L.orc_project_many.argtypes = [_I, _I, _P, _I64, _P, _P]
+            L.orc_project_many.argtypes = [_I, _I, _I, _P, _I64, _P, _P]
             L.orc_project_e4m3_many.argtypes = [ctypes.c_float, _P, _I64, _P, _P]
             L.orc_naive_code.restype = _I
-            L.orc_naive_code.argtypes = [_I, ctypes.c_float]
+            L.orc_naive_code.argtypes = [_I, _I, ctypes.c_float]
             L.orc_act_sqsum.argtypes = [_P, _I, _I64, _I64, _I64, _I64, _I64, _P]
             L.orc_act_sqmean.argtypes = [_P, _I, _I64, _I64, _I64, _P]
             L.orc_quantize_blocks.restype = _I
-            L.orc_quantize_blocks.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I,
+            L.orc_quantize_blocks.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I, _I,
                                               _I64, _I64, _P, _P, _P, _P, _P]
             L.orc_log_grid.argtypes = [_I, _D, _D, _P]
             L.orc_quantize_tiles.restype = _I
             L.orc_quantize_tiles.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _D, _D,
                                              _I64, _I64, _P, _P, _P, _P, _P]
             L.orc_dequant.restype = _I
-            L.orc_dequant.argtypes = [_P, _P, _I, _I, _I64, _I64, _P]
+            L.orc_dequant.argtypes = [_P, _P, _I, _I, _I, _I64, _I64, _P]
             L.orc_error_sums.argtypes = [_P, _I, _I64, _I64, _I64, _P, _P, _P]
             _lib = L
     return _lib
@@ -122,14 +129,28 @@ def e2m1_value(code: int) -> float:
     return lib().orc_e2m1_value(int(code))
 
 
-def naive_code(fmt: str, amax: float) -> int:
-    return lib().orc_naive_code(FMTS[fmt], float(amax))
+def scale_value(sfmt: str, code: int) -> float:
+    """Value of a scale code, decoded from its bit fields (E4M3, UE4M4, UE5M3, UE8M0)."""
+    if sfmt == "e4m3":
+        return e4m3_value(code)
+    return getattr(lib(), f"orc_{sfmt}_value")(int(code))
 
 
-def project(fmt: str, code: int, w: float):
-    """(magnitude code, |w^|) of one element at scale code ``code`` (NVFP4 / INT8)."""
+def scale_table(sfmt: str) -> np.ndarray:
+    """The sorted table of a scale grid, indexed by code."""
+    t = np.zeros(256, np.float32)
+    n = lib().orc_scale_table(SFMTS[sfmt], _ptr(t))
+    return t[:n].copy()
+
+
+def naive_code(fmt: str, amax: float, sfmt: str = "e4m3") -> int:
+    return lib().orc_naive_code(FMTS[fmt], SFMTS[sfmt], float(amax))
+
+
+def project(fmt: str, code: int, w: float, sfmt: str = "e4m3"):
+    """(magnitude code, |w^|) of one element at scale code ``code`` (NVFP4 / INT4 / INT8)."""
     out = ctypes.c_float()
-    q = lib().orc_project(FMTS[fmt], int(code), float(w), ctypes.byref(out))
+    q = lib().orc_project(FMTS[fmt], SFMTS[sfmt], int(code), float(w), ctypes.byref(out))
     return q, out.value
 
 
@@ -139,12 +160,13 @@ def project_e4m3(w: float, s: float):
     return q, out.value
 
 
-def project_many(fmt: str, code: int, w):
+def project_many(fmt: str, code: int, w, sfmt: str = "e4m3"):
     """Vector form of :func:`project`: (codes uint8, |w^| float32) for float32 ``w``."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     q = np.zeros(w.shape, np.uint8)
     wq = np.zeros(w.shape, np.float32)
-    lib().orc_project_many(FMTS[fmt], int(code), _ptr(w), w.size, _ptr(q), _ptr(wq))
+    lib().orc_project_many(FMTS[fmt], SFMTS[sfmt], int(code), _ptr(w), w.size, _ptr(q),
+                           _ptr(wq))
     return q, wq
 
 
@@ -206,9 +228,10 @@ class Result(dict):
 
 
 def quantize(W, fmt: str, mode: str, block: int, *, h=None, window: int = -1,
-             rows=None, n_threads=1, points=64, lo=-2.0, hi=2.0) -> Result:
+             rows=None, n_threads=1, points=64, lo=-2.0, hi=2.0, sfmt: str = "e4m3") -> Result:
     """Quantize W [n, k] (float32 or bf16 bits). ``rows``: optional (row0, row1) --
-    only those rows (tile rows for E4M3) are computed; other outputs stay zero/NaN."""
+    only those rows (tile rows for E4M3) are computed; other outputs stay zero/NaN.
+    ``sfmt``: the block-scale grid of NVFP4 / INT4 elements."""
     W, dt = _as_input(W)
     n, k = W.shape
     f, m = FMTS[fmt], MODES[mode]
@@ -238,7 +261,7 @@ def quantize(W, fmt: str, mode: str, block: int, *, h=None, window: int = -1,
         _run_ranges(run, r0, r1, nt)
         return Result(codes=codes, scales=scales, best=best, second=second, naive=gidx)
     kb = k // block
-    codes = np.zeros((n, k // 2) if f == NVFP4 else (n, k), np.uint8)
+    codes = np.zeros((n, k // 2) if f in (NVFP4, INT4) else (n, k), np.uint8)
     scales = np.zeros((n, kb), np.uint8)
     best = np.full((n, kb), np.nan)
     second = np.full((n, kb), np.nan)
@@ -246,9 +269,9 @@ def quantize(W, fmt: str, mode: str, block: int, *, h=None, window: int = -1,
     r0, r1 = (0, n) if rows is None else rows
 
     def run(a, b):
-        rc = lib().orc_quantize_blocks(_ptr(W), dt, n, k, k, _ptr(hp), f, m, block, window, a, b,
-                                       _ptr(codes), _ptr(scales), _ptr(best), _ptr(second),
-                                       _ptr(naive))
+        rc = lib().orc_quantize_blocks(_ptr(W), dt, n, k, k, _ptr(hp), f, SFMTS[sfmt], m, block,
+                                       window, a, b, _ptr(codes), _ptr(scales), _ptr(best),
+                                       _ptr(second), _ptr(naive))
         if rc != 0:
             raise ValueError("oracle rejected the arguments")
     _run_ranges(run, r0, r1, nt)
@@ -264,11 +287,13 @@ def _run_ranges(fn, r0, r1, nt):
         list(ex.map(lambda i: fn(int(bounds[i]), int(bounds[i + 1])), range(len(bounds) - 1)))
 
 
-def dequant(codes, scales, fmt: str, block: int, n: int, k: int) -> np.ndarray:
+def dequant(codes, scales, fmt: str, block: int, n: int, k: int,
+            sfmt: str = "e4m3") -> np.ndarray:
     codes = np.ascontiguousarray(codes)
     scales = np.ascontiguousarray(scales)
     out = np.zeros((n, k), np.float32)
-    rc = lib().orc_dequant(_ptr(codes), _ptr(scales), FMTS[fmt], block, n, k, _ptr(out))
+    rc = lib().orc_dequant(_ptr(codes), _ptr(scales), FMTS[fmt], SFMTS[sfmt], block, n, k,
+                           _ptr(out))
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out

@@ -24,12 +24,24 @@ MUTANTS = {
     "sign_dropped": ("int neg = signbit(w[j]) ? 1 : 0;", "int neg = 0;"),
     "tile_h_by_row": ("double c = (mode == ORC_HOPT) ? (double)h[j0 + j] : 1.0;",
                       "double c = (mode == ORC_HOPT) ? (double)h[i0 + i] : 1.0;"),
-    "window_short": ("hi = c0 + window > 126 ? 126 : c0 + window;",
-                     "hi = c0 + window > 126 ? 126 : c0 + window - 1;"),
+    "window_short": ("hi = c0 + window > cmax ? cmax : c0 + window;",
+                     "hi = c0 + window > cmax ? cmax : c0 + window - 1;"),
     "mean_over_r_minus_1": ("(float)(s[j] / (double)rows)", "(float)(s[j] / (double)(rows - 1))"),
     "e2m1_exponent": ("ldexp(1.0 + (double)m / 2.0, e - 1)", "ldexp(1.0 + (double)m / 2.0, e)"),
     "nibble_order": ("if (((j0 + j) & 1) == 0) *p", "if (((j0 + j) & 1) == 1) *p"),
     "e4m3_subnormal": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
+    "ue4m4_bias": ("return ldexp(1.0 + (double)m / 16.0, e - 7);",
+                   "return ldexp(1.0 + (double)m / 16.0, e - 8);"),
+    "ue5m3_subnormal": ("if (e == 0) return ldexp((double)m / 8.0, -14);",
+                        "if (e == 0) return ldexp((double)m / 8.0, -15);"),
+    "ue8m0_naive_round_up": ("int c = (ex - 1) - 2 + 127;", "int c = ex - 2 + 127;"),
+    "int4_saturates_at_6": ("int q = nearest_rne(T_INT, 8, z);", "int q = nearest_rne(T_INT, 7, z);"),
+    "int4_naive_divisor": ("float qmax = (fmt == ORC_NVFP4) ? 6.0f : 7.0f;",
+                           "float qmax = (fmt == ORC_NVFP4) ? 6.0f : 6.0f;"),
+    "int4_sign_magnitude": (": (uint8_t)((neg ? -q : q) & 15);", ": (uint8_t)((neg << 3) | q);"),
+    "ue8m0_skips_code_0": ("case ORC_S_UE8M0: *g = (scale_grid){T_UE8M0, 255, 0}; return 0;",
+                           "case ORC_S_UE8M0: *g = (scale_grid){T_UE8M0, 255, 1}; return 0;"),
+    "int4_dequant_magnitude": ("int q = (nib & 8) ? 16 - nib : nib;", "int q = nib & 7;"),
     "dequant_not_rounded": ("float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - (double)wq;",
                             "float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - 1.0000001 * (double)wq;"),
 }
@@ -47,6 +59,7 @@ def test_planted_mistake_is_caught(name, tmp_path):
                     str(so), str(mut), "-lm"], check=True)
     env = dict(os.environ, MXQ_ORACLE_LIB=str(so))
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                          os.path.join(HERE, "test_oracle_pins.py")], cwd=ROOT, env=env,
+                          os.path.join(HERE, "test_oracle_pins.py"),
+                          os.path.join(HERE, "test_oracle_pins_scales.py")], cwd=ROOT, env=env,
                          capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"pins did not catch planted mistake {name}:\n{res.stdout[-2000:]}"

@@ -190,7 +190,8 @@ def test_worked_examples(orc, case):
         assert got.hex() == case["codes"].replace(" ", "")
         return
     h = parse_floats(case["h"]) if "h" in case else None
-    r = orc.quantize(w, fmt, mode, B, h=h)
+    sfmt = case.get("sfmt", "e4m3")
+    r = orc.quantize(w, fmt, mode, B, h=h, sfmt=sfmt)
     assert int(r.scales[0, 0]) == int(case["scale"], 16)
     if "codes" in case:
         assert bytes(r.codes[0]).hex() == case["codes"].replace(" ", "")
@@ -199,7 +200,7 @@ def test_worked_examples(orc, case):
     if "second" in case:
         assert r.second[0, 0] == float(case["second"])
     if "sse" in case:
-        What = orc.dequant(r.codes, r.scales, fmt, B, 1, w.shape[1])
+        What = orc.dequant(r.codes, r.scales, fmt, B, 1, w.shape[1], sfmt=sfmt)
         m = orc.metrics(orc.error_sums(w, What))
         assert m["sse"] == float(case["sse"])
         if "weight_rel" in case:
