@@ -19,6 +19,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import collections
 import dataclasses
 import hashlib
 import json
@@ -45,6 +46,8 @@ ALU_PEAK_TOPS = 148 * 128 * 1.965e9 / 1e12
 # Oracle samples: the cpu_baseline leg (about 10-30 s of CPU work) and each step of the
 # reference arm (well under a second, so that a long --steps run stays short).
 CPU_X_ROWS, CPU_W_ROWS = 32768, 1024
+Quantizer = collections.namedtuple("Quantizer", "fmt block mode window sfmt")
+HEADLINE_Q = Quantizer("nvfp4", 16, "hopt", -1, "e4m3")
 REF_X_ROWS, REF_W_ROWS = 2048, 8
 
 
@@ -59,6 +62,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block", type=int, default=0, help="block size (default: the workload's)")
     ap.add_argument("--mode", default="", choices=["", "naive", "sse", "hopt"])
+    ap.add_argument("--fmt", default="", choices=["", "nvfp4", "int4", "int8", "e4m3"],
+                    help="element format (default: the workload's)")
+    ap.add_argument("--scale-fmt", default="", choices=["", "e4m3", "ue4m4", "ue5m3", "ue8m0"],
+                    help="block-scale grid of nvfp4 / int4 elements (ue8m0 = MXFP4)")
     ap.add_argument("--x-rows", type=int, default=0,
                     help="use only this many activation rows (profiling captures)")
     return ap.parse_args()
@@ -152,15 +159,27 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def workload_desc(wl, fmt, block, mode, window, x_rows=None):
+def quant_name(q):
+    """Short name of a quantizer: the element format, or MXFP4 / NVINT4 / E2M1-on-UE4M4 ..."""
+    if q.fmt == "nvfp4":
+        return {"e4m3": "nvfp4", "ue8m0": "mxfp4"}.get(q.sfmt, f"e2m1-{q.sfmt}")
+    if q.fmt == "int4":
+        return "nvint4" if q.sfmt == "e4m3" else f"int4-{q.sfmt}"
+    return q.fmt
+
+
+def workload_desc(wl, q, x_rows=None):
     """One-line description of what a step computes (both arms print the same)."""
+    fmt, block, mode, window = q.fmt, q.block, q.mode, q.window
     x_rows = x_rows or [r for r, _ in wl.x_shapes]
     dt = "bf16" if wl.w_dtype == torch.bfloat16 else "f32"
     shapes = ", ".join(f"{nm} {n}x{k}" for nm, n, k in wl.weights)
     xsh = ", ".join(f"{r}x{k}" for r, (_, k) in zip(x_rows, wl.x_shapes))
+    sg = q.sfmt.upper()
+    ncand = {"e4m3": 126, "ue4m4": 255, "ue5m3": 255, "ue8m0": 255}[q.sfmt]
     grid = ("64-point log grid" if fmt == "e4m3" else
-            "all 126 E4M3 scales" if window < 0 else f"E4M3 scales within +-{window} codes")
-    return (f"{wl.name}: W {shapes} {dt}; X {xsh} {dt}; {fmt} block {block}, {mode}, "
+            f"all {ncand} {sg} scales" if window < 0 else f"{sg} scales within +-{window} codes")
+    return (f"{wl.name}: W {shapes} {dt}; X {xsh} {dt}; {quant_name(q)} block {block}, {mode}, "
             f"{grid}; then weight/h-weighted error sums")
 
 
@@ -170,18 +189,19 @@ def workload_desc(wl, fmt, block, mode, window, x_rows=None):
 
 def oracle_step_sample(X_bits, W_bits, h_np, n_threads, R_full, N_full, q):
     """Time the oracle on a bounded sample (X_bits: the first rows of X, W_bits: the first
-    rows of W, bf16 bits; q = (fmt, block, mode, window)) and scale each part to the full
+    rows of W, bf16 bits; q the quantizer) and scale each part to the full
     workload (R_full rows of X, N_full rows of W, in units of the sample's row widths).
     Returns (seconds for a full step, measured seconds per part)."""
     from oracle import oracle as orc
-    fmt, block, mode, window = q
+    fmt, block, mode, window = q.fmt, q.block, q.mode, q.window
     x_rows, K = X_bits.shape
     w_rows = W_bits.shape[0]
     t0 = time.perf_counter()
     orc.act_sqmean(X_bits, n_threads=n_threads)
     t1 = time.perf_counter()
-    r = orc.quantize(W_bits, fmt, mode, block, h=h_np, window=window, n_threads=n_threads)
-    What = orc.dequant(r.codes, r.scales, fmt, block, w_rows, K)
+    r = orc.quantize(W_bits, fmt, mode, block, h=h_np, window=window, n_threads=n_threads,
+                     sfmt=q.sfmt)
+    What = orc.dequant(r.codes, r.scales, fmt, block, w_rows, K, sfmt=q.sfmt)
     orc.error_sums(W_bits, What, h_np)
     t2 = time.perf_counter()
     full = (t1 - t0) * (R_full / x_rows) + (t2 - t1) * (N_full / w_rows)
@@ -208,7 +228,7 @@ def reference_arm(args):
     q = quantizer_for(wl, args)
     (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
     x_rows = min(REF_X_ROWS, R)
-    w_rows = min(max(REF_W_ROWS, q[1] if q[0] == "e4m3" else 1), n)
+    w_rows = min(max(REF_W_ROWS, q.block if q.fmt == "e4m3" else 1), n)
     X = bits_of(synth.workload_activations(wl, 0, rows=x_rows))
     W = bits_of(synth.workload_weight(wl, 0, rows=w_rows))
     h = orc.act_sqmean(X)
@@ -222,16 +242,15 @@ def reference_arm(args):
             times.append(full)
     full_step = statistics.mean(times)
     value = weights / full_step / 1e9
-    sample = (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows ({q[2]} "
+    sample = (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows ({q.mode} "
               f"search + error) per step, {nt} threads; times scaled to the full workload")
-    headline = args.workload == "nvfp4_full_calib" and q[:3] == ("nvfp4", 16, "hopt")
-    metric = METRIC if headline else \
-        f"G weights/s quantized ({q[2]} {q[0]} blk{q[1]}) + h-pass GB/s; % of roofline"
+    headline = args.workload == "nvfp4_full_calib" and q == HEADLINE_Q
+    metric = METRIC if headline else metric_for(q)
     line = {"impl": "reference", "metric": metric, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(wl, *q)},
+            "config": {"workload": workload_desc(wl, q)},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": nt, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -244,23 +263,29 @@ def reference_arm(args):
 # ---------------------------------------------------------------------------------------
 
 def quantizer_for(wl, args):
-    """(fmt, block, mode, window) the bench times for a workload."""
+    """The quantizer the bench times for a workload (its own, or the command line's)."""
     block = args.block or wl.blocks[0]
     mode = args.mode or ("hopt" if "hopt" in wl.modes else wl.modes[-1])
-    return wl.fmt, block, mode, wl.window
+    return Quantizer(args.fmt or wl.fmt, block, mode, wl.window, args.scale_fmt or "e4m3")
 
 
-def ops_per_weight(fmt, mode, window):
+def metric_for(q):
+    return (f"G weights/s quantized ({q.mode} {quant_name(q)} blk{q.block}) + h-pass GB/s; "
+            f"% of roofline")
+
+
+def ops_per_weight(fmt, mode, window, sfmt="e4m3"):
     """Algorithmic lane-operations per weight of a scale search: C candidates x 6 (quotient,
     projection, dequantise, subtract, h-multiply, square-accumulate; 5 without h) + 4
     (amax, naive quotient, final projection, pack)."""
-    C = 64 if fmt == "e4m3" else (126 if window < 0 else 2 * window + 1)
+    full = 126 if sfmt == "e4m3" else 255
+    C = 64 if fmt == "e4m3" else (full if window < 0 else 2 * window + 1)
     return C * (6 if mode == "hopt" else 5) + 4
 
 
 def code_bytes(fmt, block):
     """Bytes of codes + scales per weight."""
-    if fmt == "nvfp4":
+    if fmt in ("nvfp4", "int4"):
         return 0.5 + 1.0 / block
     if fmt == "int8":
         return 1.0 + 1.0 / block
@@ -279,8 +304,9 @@ def gpu_arm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     wl = synth.WORKLOADS[args.workload]
-    fmt, block, mode, window = quantizer_for(wl, args)
-    p = mxq.params(fmt, mode, block, window=window)
+    q = quantizer_for(wl, args)
+    fmt, block, mode, window = q.fmt, q.block, q.mode, q.window
+    p = mxq.params(fmt, mode, block, window=window, scale_fmt=q.sfmt)
     # inputs: every rank draws its own shard (weak scaling)
     wl_r = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
     # activations and their h, one per activation width
@@ -409,8 +435,7 @@ def gpu_arm(args):
 
     # ---- roofline ------------------------------------------------------------------------
     hbm, hbm_kind = measured_peaks()
-    headline = (args.workload == "nvfp4_full_calib" and (fmt, block, mode) ==
-                ("nvfp4", 16, "hopt") and not args.x_rows)
+    headline = args.workload == "nvfp4_full_calib" and q == HEADLINE_Q and not args.x_rows
     x_bytes = sum(X.numel() * X.element_size() + 4 * X.shape[1] for X in Xs)
     w_bytes = sum(W.numel() * W.element_size() for W in Ws)
     h_gbs = x_bytes / (k_h * 1e-3) / 1e9
@@ -424,7 +449,7 @@ def gpu_arm(args):
                                "unit": "GB/s", "frac": q_gbs / hbm, "algorithmic_bytes": q_bytes,
                                "traffic": None}
     else:
-        ops = ops_per_weight(fmt, mode, window) * weights
+        ops = ops_per_weight(fmt, mode, window, q.sfmt) * weights
         q_tops = ops / (k_q * 1e-3) / 1e12
         kernels["quantize"] = {"ms": k_q, "bound": "alu", "achieved": q_tops,
                                "peak": ALU_PEAK_TOPS, "unit": "T lane-op/s",
@@ -442,14 +467,13 @@ def gpu_arm(args):
                 "traffic": dk["traffic"],
                 "peak_source": ("MEASURED_PEAKS.json hbm_gbs (" + hbm_kind + ")")
                 if dk["bound"] == "hbm" else "148 SM x 128 FP32 lanes x 1965 MHz"}
-    metric = METRIC if headline else \
-        f"G weights/s quantized ({mode} {fmt} blk{block}) + h-pass GB/s; % of roofline"
+    metric = METRIC if (args.workload == "nvfp4_full_calib" and q == HEADLINE_Q) \
+        else metric_for(q)
     line = {"metric": metric, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": workload_desc(wl, fmt, block, mode, window,
-                                                 [X.shape[0] for X in Xs]),
+            "config": {"workload": workload_desc(wl, q, [X.shape[0] for X in Xs]),
                        "weights_per_gpu": weights,
                        "x_rows_per_gpu": Xs[0].shape[0] if len(Xs) == 1 else
                        [X.shape[0] for X in Xs],
@@ -480,7 +504,7 @@ def gpu_arm(args):
         h_np = orc.act_sqmean(Xb, n_threads=nt)
         # the sample's per-row times scaled to every X row and every W row of the step
         full, d = oracle_step_sample(Xb, Wb, h_np, nt, sum(X.numel() for X in Xs) / X0.shape[1],
-                                     weights / W0.shape[1], (fmt, block, mode, window))
+                                     weights / W0.shape[1], q)
         line["cpu_baseline"] = {
             "value": weights / full / 1e9, "unit": UNIT, "cores": nt, "kind": "oracle",
             "sample": (f"oracle on {x_rows} of {R0} X rows (h) and {w_rows} of {n0} W rows "

@@ -1,6 +1,7 @@
 // mxq_api.cu -- the extern "C" boundary of libmxq.so: host-side validation, workspace
 // queries and kernel launches. See include/mxq.h for the contract of every call.
 #include "../../include/mxq.h"
+#include "mxq_grids.h"
 #include "mxq_internal.h"
 
 #include <algorithm>
@@ -60,14 +61,22 @@ mxq_status check_params(const mxq_params* p, int64_t n, int64_t k) {
   if (p->mode < MXQ_NAIVE || p->mode > MXQ_HOPT) return fail(MXQ_ERR_INVALID_ARG, "mode %d", p->mode);
   switch (p->fmt) {
     case MXQ_FMT_NVFP4:
+    case MXQ_FMT_INT4:
       if (p->block != 16 && p->block != 32)
-        return fail(MXQ_ERR_UNSUPPORTED, "NVFP4 block %d (16 or 32)", p->block);
-      if (p->tile_rows != 1) return fail(MXQ_ERR_UNSUPPORTED, "NVFP4 tile_rows must be 1");
+        return fail(MXQ_ERR_UNSUPPORTED, "%s block %d (16 or 32)",
+                    p->fmt == MXQ_FMT_NVFP4 ? "NVFP4" : "INT4", p->block);
+      if (p->tile_rows != 1) return fail(MXQ_ERR_UNSUPPORTED, "NVFP4 / INT4 tile_rows must be 1");
+      if (!mxq::grid_known(p->scale_fmt))
+        return fail(MXQ_ERR_INVALID_ARG, "scale_fmt %d", p->scale_fmt);
+      if (p->fmt == MXQ_FMT_INT4 && p->scale_fmt == MXQ_SCALE_UE8M0)
+        return fail(MXQ_ERR_UNSUPPORTED, "UE8M0 scales are for E2M1 elements (MXFP4)");
       break;
     case MXQ_FMT_INT8:
       if (p->block != 32 && p->block != 64 && p->block != 128 && p->block != 256)
         return fail(MXQ_ERR_UNSUPPORTED, "INT8 block %d (32, 64, 128 or 256)", p->block);
       if (p->tile_rows != 1) return fail(MXQ_ERR_UNSUPPORTED, "INT8 tile_rows must be 1");
+      if (p->scale_fmt != MXQ_SCALE_E4M3)
+        return fail(MXQ_ERR_UNSUPPORTED, "INT8 stores its amax as E4M3 (scale_fmt 0)");
       break;
     case MXQ_FMT_E4M3:
       if (p->block != 64 || p->tile_rows != 64)
@@ -81,6 +90,8 @@ mxq_status check_params(const mxq_params* p, int64_t n, int64_t k) {
           return fail(MXQ_ERR_INVALID_ARG, "log grid exponents");
       }
       if (n % 64 != 0) return fail(MXQ_ERR_SHAPE, "n %% 64 != 0 for E4M3 tiles");
+      if (p->scale_fmt != MXQ_SCALE_E4M3)
+        return fail(MXQ_ERR_UNSUPPORTED, "E4M3 tiles have float scales (scale_fmt 0)");
       break;
     default:
       return fail(MXQ_ERR_INVALID_ARG, "fmt %d", p->fmt);
@@ -218,6 +229,7 @@ mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int6
   a.mode = p->mode;
   a.block = p->block;
   a.window = p->window;
+  a.scale_fmt = p->scale_fmt;
   a.codes = codes;
   a.scales = scales;
   a.log_points = p->fmt == MXQ_FMT_E4M3 && p->mode != MXQ_NAIVE ? p->log_points : 0;
@@ -228,23 +240,21 @@ mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int6
   return cuda_status(mxq::launch_quantize(a, (cudaStream_t)stream), "quantize");
 }
 
-mxq_status mxq_project(const float* w, int64_t count, int32_t fmt, float scale, uint8_t* q,
-                       void* stream) {
+mxq_status mxq_project(const float* w, int64_t count, int32_t fmt, int32_t scale_fmt,
+                       float scale, uint8_t* q, void* stream) {
   if (count < 0) return fail(MXQ_ERR_SHAPE, "negative count");
-  if (fmt < MXQ_FMT_NVFP4 || fmt > MXQ_FMT_E4M3) return fail(MXQ_ERR_INVALID_ARG, "fmt %d", fmt);
+  if (fmt < MXQ_FMT_NVFP4 || fmt > MXQ_FMT_INT4) return fail(MXQ_ERR_INVALID_ARG, "fmt %d", fmt);
+  if (fmt != MXQ_FMT_E4M3 && !mxq::grid_known(scale_fmt))
+    return fail(MXQ_ERR_INVALID_ARG, "scale_fmt %d", scale_fmt);
+  if (fmt == MXQ_FMT_INT8 && scale_fmt != MXQ_SCALE_E4M3)
+    return fail(MXQ_ERR_UNSUPPORTED, "INT8 stores its amax as E4M3 (scale_fmt 0)");
   if (count == 0) return MXQ_OK;
   if (!w || !q) return fail(MXQ_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(w, 4)) return fail(MXQ_ERR_ALIGN, "w not 4-byte aligned");
   if (!(scale > 0.0f) || !std::isfinite(scale))
     return fail(MXQ_ERR_INVALID_ARG, "scale must be positive and finite");
-  if (fmt != MXQ_FMT_E4M3) {
-    // NVFP4 and INT8 scales are E4M3 values: 4 significant bits, 2^-9 .. 448
-    int e = 0;
-    const float m = std::frexp(scale, &e);
-    const float m16 = m * 16.0f;
-    if (scale < 0.001953125f || scale > 448.0f || m16 != std::floor(m16))
-      return fail(MXQ_ERR_INVALID_ARG, "scale is not a positive E4M3 value");
-  }
+  if (fmt != MXQ_FMT_E4M3 && !mxq::grid_has_value(scale_fmt, scale))
+    return fail(MXQ_ERR_INVALID_ARG, "scale is not a positive value of scale grid %d", scale_fmt);
   return cuda_status(mxq::launch_project(w, count, fmt, scale, q, (cudaStream_t)stream),
                      "project");
 }
@@ -258,7 +268,7 @@ mxq_status mxq_dequant(const void* codes, const void* scales, const mxq_params* 
   if (!codes || !scales || !out) return fail(MXQ_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(codes, 16) || !aligned(out, 16) || !aligned(scales, 4))
     return fail(MXQ_ERR_ALIGN, "codes/out not 16-byte or scales not 4-byte aligned");
-  mxq::DecodeArgs d{codes, scales, p->fmt, p->block, n, k};
+  mxq::DecodeArgs d{codes, scales, p->fmt, p->block, p->scale_fmt, n, k};
   return cuda_status(mxq::launch_dequant(d, out, (cudaStream_t)stream), "dequant");
 }
 
@@ -287,7 +297,7 @@ mxq_status mxq_error(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t
   if (!workspace || workspace_bytes < need)
     return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
   if (!aligned(workspace, 8)) return fail(MXQ_ERR_ALIGN, "workspace not 8-byte aligned");
-  mxq::DecodeArgs d{codes, scales, p->fmt, p->block, n, k};
+  mxq::DecodeArgs d{codes, scales, p->fmt, p->block, p->scale_fmt, n, k};
   return cuda_status(mxq::launch_error(d, W, dtype, ld, h, (double*)workspace,
                                        mxq::error_partials(n, k), sums, st),
                      "error");

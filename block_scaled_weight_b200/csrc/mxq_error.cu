@@ -3,6 +3,8 @@
 // Dequantised value (the microscaling reconstruction x^ = s q, "Is Finer Better? The
 // Limits of Microscaling Formats in LLMs", sec. 2.1):
 //   NVFP4  E4M3(scale) * E2M1(code)                (exact in float32 and in fp16)
+//   E2M1 on the UE4M4 / UE5M3 / UE8M0 grids: grid(scale) * E2M1(code)   (exact)
+//   INT4   grid(scale) * code, code the signed nibble (exact)
 //   INT8   fl32(q * fl32(E4M3(scale) / 127))
 //   E4M3   fl32(tile scale * E4M3(code))
 // Metrics (qwantize "Results": weight error ||Q(W) - W||_F / ||W||_F; the h-weighted
@@ -12,6 +14,7 @@
 // math), double from there on; the per-CTA partials are combined by a one-CTA kernel in a
 // fixed order (deterministic).
 #include "mxq_common.cuh"
+#include "mxq_grids.h"
 #include "mxq_internal.h"
 
 #include <cuda_fp16.h>
@@ -23,16 +26,62 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxErrCtas = 148 * 8;
 
+// Decoder variants: 0 E2M1 on E4M3 scales, 1 INT8, 2 E4M3 tiles, 3 INT4 on a scale table,
+// 4 E2M1 on a scale table.
+enum { kDecFp4 = 0, kDecInt8 = 1, kDecTile = 2, kDecInt4 = 3, kDecFp4Tab = 4 };
+
+// Scale-code values of a grid (NaN for the codes it does not define); staged in shared
+// memory by the kernels that decode through a table.
+struct ScaleTab {
+  float v[256];
+};
+
+ScaleTab make_scale_tab(int sfmt) {
+  ScaleTab t;
+  const GridInfo g = grid_info(sfmt);
+  for (int c = 0; c < 256; ++c) t.v[c] = c < g.ncodes ? (float)grid_value(sfmt, c) : __builtin_nanf("");
+  return t;
+}
+
+const ScaleTab& scale_tab(int sfmt) {
+  static const ScaleTab tabs[4] = {make_scale_tab(0), make_scale_tab(1), make_scale_tab(2),
+                                   make_scale_tab(3)};
+  return tabs[sfmt];
+}
+
+int decoder_of(const DecodeArgs& d) {
+  if (d.fmt == 3) return kDecInt4;
+  if (d.fmt == 0 && d.scale_fmt != kScaleE4M3) return kDecFp4Tab;
+  return d.fmt;
+}
+
 __device__ __forceinline__ float2 h2f2(uint32_t h2) {
   return make_float2(__half2float(__ushort_as_half(lo16(h2))),
                      __half2float(__ushort_as_half(hi16(h2))));
 }
 
 // Decoded (w^) values of the 16 elements starting at (row, col), as 8 float pairs.
+// stab: the scale table in shared memory (decoders 3 and 4).
 template <int FMT>
 __device__ __forceinline__ void decode16(const DecodeArgs& d, int64_t row, int64_t col,
-                                         float2 (&v)[8]) {
-  if constexpr (FMT == 0) {
+                                         float2 (&v)[8], const float* stab) {
+  if constexpr (FMT == kDecFp4Tab || FMT == kDecInt4) {
+    const uint8_t* cp = (const uint8_t*)d.codes + row * (d.k / 2) + col / 2;
+    const uint2 cw = *reinterpret_cast<const uint2*>(cp);
+    const float s = stab[((const uint8_t*)d.scales)[row * (d.k / d.block) + col / d.block]];
+    const float2 s2 = make_float2(s, s);
+    const uint32_t w2[2] = {cw.x, cw.y};
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const uint32_t byte = (w2[p / 4] >> (8 * (p % 4))) & 0xffu;
+      if constexpr (FMT == kDecFp4Tab) {
+        v[p] = __fmul2_rn(h2f2(e2m1x2_to_f16x2(byte)), s2);   // exact products
+      } else {
+        const int q0 = (int)(byte << 28) >> 28, q1 = (int)(byte << 24) >> 28;  // sign-extend
+        v[p] = __fmul2_rn(make_float2((float)q0, (float)q1), s2);
+      }
+    }
+  } else if constexpr (FMT == 0) {
     const uint8_t* cp = (const uint8_t*)d.codes + row * (d.k / 2) + col / 2;
     const uint2 cw = *reinterpret_cast<const uint2*>(cp);
     const float s = e4m3_pos(((const uint8_t*)d.scales)[row * (d.k / d.block) + col / d.block]);
@@ -72,13 +121,18 @@ __device__ __forceinline__ void decode16(const DecodeArgs& d, int64_t row, int64
 
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
-k_dequant(DecodeArgs d, float* __restrict__ out) {
+k_dequant(DecodeArgs d, ScaleTab T, float* __restrict__ out) {
+  __shared__ float stab[256];
+  if constexpr (FMT == kDecFp4Tab || FMT == kDecInt4) {
+    for (int i = threadIdx.x; i < 256; i += kThreads) stab[i] = T.v[i];
+    __syncthreads();
+  }
   const int64_t units = d.n * (d.k / 16);
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units;
        u += (int64_t)gridDim.x * kThreads) {
     const int64_t row = u / (d.k / 16), col = (u - row * (d.k / 16)) * 16;
     float2 v[8];
-    decode16<FMT>(d, row, col, v);
+    decode16<FMT>(d, row, col, v, stab);
     float4* o = reinterpret_cast<float4*>(out + row * d.k + col);
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[i] = make_float4(v[2 * i].x, v[2 * i].y, v[2 * i + 1].x, v[2 * i + 1].y);
@@ -87,16 +141,21 @@ k_dequant(DecodeArgs d, float* __restrict__ out) {
 
 template <int FMT, bool BF16, bool HAS_H>
 __global__ void __launch_bounds__(kThreads)
-k_error(DecodeArgs d, const char* __restrict__ W, int64_t ld_bytes, const float* __restrict__ h,
-        double* __restrict__ partial) {
+k_error(DecodeArgs d, ScaleTab T, const char* __restrict__ W, int64_t ld_bytes,
+        const float* __restrict__ h, double* __restrict__ partial) {
   __shared__ double red[kThreads / 32][4];
+  __shared__ float stab[256];
+  if constexpr (FMT == kDecFp4Tab || FMT == kDecInt4) {
+    for (int i = threadIdx.x; i < 256; i += kThreads) stab[i] = T.v[i];
+    __syncthreads();
+  }
   const int64_t units = d.n * (d.k / 16);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < units;
        u += (int64_t)gridDim.x * kThreads) {
     const int64_t row = u / (d.k / 16), col = (u - row * (d.k / 16)) * 16;
     float2 v[8], w[8];
-    decode16<FMT>(d, row, col, v);
+    decode16<FMT>(d, row, col, v, stab);
     const char* wp = W + row * ld_bytes + col * (BF16 ? 2 : 4);
     if constexpr (BF16) {
       const uint4 x0 = __ldg(reinterpret_cast<const uint4*>(wp));
@@ -174,7 +233,7 @@ cudaError_t dequant_fmt(const DecodeArgs& d, float* out, cudaStream_t st) {
   int64_t grid = (units + kThreads - 1) / kThreads;
   const int64_t cap = (int64_t)sm_count() * 16;
   if (grid > cap) grid = cap;
-  k_dequant<FMT><<<(unsigned)grid, kThreads, 0, st>>>(d, out);
+  k_dequant<FMT><<<(unsigned)grid, kThreads, 0, st>>>(d, scale_tab(d.scale_fmt), out);
   return cudaGetLastError();
 }
 
@@ -182,12 +241,13 @@ template <int FMT>
 cudaError_t error_fmt(const DecodeArgs& d, const void* W, int dtype, int64_t ld, const float* h,
                       double* partial, int parts, cudaStream_t st) {
   const char* Wc = (const char*)W;
+  const ScaleTab& T = scale_tab(d.scale_fmt);
   if (dtype == 1) {
-    if (h) k_error<FMT, true, true><<<parts, kThreads, 0, st>>>(d, Wc, ld * 2, h, partial);
-    else k_error<FMT, true, false><<<parts, kThreads, 0, st>>>(d, Wc, ld * 2, h, partial);
+    if (h) k_error<FMT, true, true><<<parts, kThreads, 0, st>>>(d, T, Wc, ld * 2, h, partial);
+    else k_error<FMT, true, false><<<parts, kThreads, 0, st>>>(d, T, Wc, ld * 2, h, partial);
   } else {
-    if (h) k_error<FMT, false, true><<<parts, kThreads, 0, st>>>(d, Wc, ld * 4, h, partial);
-    else k_error<FMT, false, false><<<parts, kThreads, 0, st>>>(d, Wc, ld * 4, h, partial);
+    if (h) k_error<FMT, false, true><<<parts, kThreads, 0, st>>>(d, T, Wc, ld * 4, h, partial);
+    else k_error<FMT, false, false><<<parts, kThreads, 0, st>>>(d, T, Wc, ld * 4, h, partial);
   }
   return cudaGetLastError();
 }
@@ -202,18 +262,26 @@ int error_partials(int64_t n, int64_t k) {
 }
 
 cudaError_t launch_dequant(const DecodeArgs& d, float* out, cudaStream_t st) {
-  if (d.fmt == 0) return dequant_fmt<0>(d, out, st);
-  if (d.fmt == 1) return dequant_fmt<1>(d, out, st);
-  return dequant_fmt<2>(d, out, st);
+  switch (decoder_of(d)) {
+    case kDecFp4: return dequant_fmt<kDecFp4>(d, out, st);
+    case kDecInt8: return dequant_fmt<kDecInt8>(d, out, st);
+    case kDecInt4: return dequant_fmt<kDecInt4>(d, out, st);
+    case kDecFp4Tab: return dequant_fmt<kDecFp4Tab>(d, out, st);
+    default: return dequant_fmt<kDecTile>(d, out, st);
+  }
 }
 
 cudaError_t launch_error(const DecodeArgs& d, const void* W, int dtype, int64_t ld,
                          const float* h, double* partial, int parts, double* sums,
                          cudaStream_t st) {
   cudaError_t e;
-  if (d.fmt == 0) e = error_fmt<0>(d, W, dtype, ld, h, partial, parts, st);
-  else if (d.fmt == 1) e = error_fmt<1>(d, W, dtype, ld, h, partial, parts, st);
-  else e = error_fmt<2>(d, W, dtype, ld, h, partial, parts, st);
+  switch (decoder_of(d)) {
+    case kDecFp4: e = error_fmt<kDecFp4>(d, W, dtype, ld, h, partial, parts, st); break;
+    case kDecInt8: e = error_fmt<kDecInt8>(d, W, dtype, ld, h, partial, parts, st); break;
+    case kDecInt4: e = error_fmt<kDecInt4>(d, W, dtype, ld, h, partial, parts, st); break;
+    case kDecFp4Tab: e = error_fmt<kDecFp4Tab>(d, W, dtype, ld, h, partial, parts, st); break;
+    default: e = error_fmt<kDecTile>(d, W, dtype, ld, h, partial, parts, st); break;
+  }
   if (e != cudaSuccess) return e;
   k_error_final<<<1, kThreads, 0, st>>>(partial, parts, sums);
   return cudaGetLastError();

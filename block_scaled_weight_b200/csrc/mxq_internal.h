@@ -27,12 +27,15 @@ struct QuantArgs {
   int64_t n, k, ld;
   const float* h;      // null unless mode == HOPT
   int fmt, mode, block, window;
+  int scale_fmt;       // block-scale grid of NVFP4 / INT4 elements (mxq_grids.h)
   void* codes;
   void* scales;
   int log_points;
   float log_grid[256];  // E4M3 tiles: g_p
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
+// E2M1 on a scale grid other than E4M3, and INT4 on any grid (mxq_quant_grid.cu).
+cudaError_t launch_quantize_grid(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, uint8_t* q,
                            cudaStream_t st);
 
@@ -41,6 +44,7 @@ struct DecodeArgs {
   const void* codes;
   const void* scales;
   int fmt, block;
+  int scale_fmt;  // NVFP4 / INT4: the block-scale grid
   int64_t n, k;
 };
 cudaError_t launch_dequant(const DecodeArgs& d, float* out, cudaStream_t st);

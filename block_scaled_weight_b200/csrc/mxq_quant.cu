@@ -25,6 +25,7 @@
 // So NVFP4 and INT8 picks equal the definition's, ties included. E4M3 tiles re-score in
 // double in a fixed parallel order: picks equal the definition's wherever the two best
 // tile errors differ by more than ~1e-12 relative.
+#include "mxq_block.cuh"
 #include "mxq_common.cuh"
 #include "mxq_internal.h"
 
@@ -56,58 +57,6 @@ struct Fp4Params {
   uint8_t* codes;
   uint8_t* scales;
 };
-
-template <int B, bool BF16>
-__device__ __forceinline__ void load_block(const char* p, float2 (&a)[B / 2], uint32_t& sgn) {
-  uint32_t wds[BF16 ? B / 2 : B];
-  if constexpr (BF16) {
-#pragma unroll
-    for (int v = 0; v < B / 8; ++v) {
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(p) + v);
-      wds[4 * v] = x.x; wds[4 * v + 1] = x.y; wds[4 * v + 2] = x.z; wds[4 * v + 3] = x.w;
-    }
-    sgn = 0;
-#pragma unroll
-    for (int i = 0; i < B / 2; ++i) {
-      sgn |= ((wds[i] >> 15) & 1u) << (2 * i);
-      sgn |= (wds[i] >> 31) << (2 * i + 1);
-      a[i] = make_float2(__uint_as_float((wds[i] << 16) & 0x7fffffffu),
-                         __uint_as_float(wds[i] & 0x7fff0000u));
-    }
-  } else {
-#pragma unroll
-    for (int v = 0; v < B / 4; ++v) {
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(p) + v);
-      wds[4 * v] = x.x; wds[4 * v + 1] = x.y; wds[4 * v + 2] = x.z; wds[4 * v + 3] = x.w;
-    }
-    sgn = 0;
-#pragma unroll
-    for (int i = 0; i < B / 2; ++i) {
-      sgn |= (wds[2 * i] >> 31) << (2 * i);
-      sgn |= (wds[2 * i + 1] >> 31) << (2 * i + 1);
-      a[i] = make_float2(__uint_as_float(wds[2 * i] & 0x7fffffffu),
-                         __uint_as_float(wds[2 * i + 1] & 0x7fffffffu));
-    }
-  }
-}
-
-template <int B>
-__device__ __forceinline__ void load_h(const float* h, float2 (&c)[B / 2]) {
-#pragma unroll
-  for (int v = 0; v < B / 4; ++v) {
-    const float4 x = __ldg(reinterpret_cast<const float4*>(h) + v);
-    c[2 * v] = make_float2(x.x, x.y);
-    c[2 * v + 1] = make_float2(x.z, x.w);
-  }
-}
-
-template <int B>
-__device__ __forceinline__ float block_amax(const float2 (&a)[B / 2]) {
-  float m = 0.f;
-#pragma unroll
-  for (int i = 0; i < B / 2; ++i) m = fmaxf(m, fmaxf(a[i].x, a[i].y));
-  return m;
-}
 
 // fl32(|w| / s) for an E4M3 scale s, from the split reciprocal (see the file header).
 __device__ __forceinline__ float2 fp4_quot(float2 a, float2 rhi, float2 rlo) {
@@ -248,17 +197,6 @@ __device__ __forceinline__ float fp4_lb(float2 at, float2 ct, float2 x, uint32_t
   return v.x + v.y;
 }
 
-// Running (min, second min, arg min) over candidates visited in any order; equal errors
-// keep the smaller code and push the tie into the second slot (so the block is flagged).
-__device__ __forceinline__ void track(float e, int cc, float& m1, float& m2, int& i1) {
-  if (e < m1 || (e == m1 && cc < i1)) {
-    m2 = m1;
-    m1 = e;
-    i1 = cc;
-  } else if (e < m2) {
-    m2 = e;
-  }
-}
 
 // NVFP4, SSE / H-optimal search: one thread per block walks every candidate, grouped by
 // significand. Blocks whose float32 winner is not separated from the runner-up by the
@@ -930,9 +868,10 @@ __global__ void k_project(const float* __restrict__ w, int64_t count, int fmt, f
        i += (int64_t)gridDim.x * kThreads) {
     const float a = fabsf(w[i]);
     uint32_t code;
-    if (fmt == 0) {
+    if (fmt == 0 || fmt == 3) {
+      // the split-reciprocal quotient of the search kernels (exact for every scale grid)
       const float2 x = fp4_quot(make_float2(a, 0.f), make_float2(rhi, rhi), make_float2(rlo, rlo));
-      code = e2m1x2_rn(x.x, 0.f) & 7u;
+      code = fmt == 0 ? (e2m1x2_rn(x.x, 0.f) & 7u) : (uint32_t)fminf(rintf(x.x), 7.0f);
     } else if (fmt == 1) {
       code = (uint32_t)int8_code(a, __fdiv_rn(scale, 127.0f));
     } else {
@@ -1062,7 +1001,7 @@ cudaError_t tile_dispatch(const QuantArgs& a, cudaStream_t st) {
 cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, uint8_t* q,
                            cudaStream_t st) {
   float rhi = 0.f, rlo = 0.f;
-  if (fmt == 0) {
+  if (fmt == 0 || fmt == 3) {
     const double r = 1.0 / (double)scale;
     rhi = (float)r;
     rlo = (float)(r - (double)rhi);
@@ -1075,6 +1014,7 @@ cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, 
 
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {
   const bool bf = a.dtype == 1;
+  if (a.fmt == 3 || (a.fmt == 0 && a.scale_fmt != 0)) return launch_quantize_grid(a, st);
   if (a.fmt == 0) {
     if (a.block == 16) return bf ? fp4_dispatch<16, true>(a, st) : fp4_dispatch<16, false>(a, st);
     return bf ? fp4_dispatch<32, true>(a, st) : fp4_dispatch<32, false>(a, st);

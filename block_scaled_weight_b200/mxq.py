@@ -25,8 +25,10 @@ STATUS = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_SHAPE", 3: "MXQ_ERR
           4: "MXQ_ERR_ALIGN", 5: "MXQ_ERR_UNSUPPORTED", 6: "MXQ_ERR_CUDA",
           7: "MXQ_ERR_WORKSPACE"}
 F32, BF16 = 0, 1
-FMT = {"nvfp4": 0, "int8": 1, "e4m3": 2}
+FMT = {"nvfp4": 0, "int8": 1, "e4m3": 2, "int4": 3}
 MODE = {"naive": 0, "sse": 1, "hopt": 2}
+# block-scale grids; MXFP4 is fmt "nvfp4" (E2M1 elements) with scale_fmt "ue8m0"
+SCALE = {"e4m3": 0, "ue4m4": 1, "ue5m3": 2, "ue8m0": 3}
 
 EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc",
            "mxq_act_sqsum",
@@ -38,7 +40,7 @@ class MxqParams(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("mode", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("tile_rows", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("log_points", ctypes.c_int32), ("log_lo_exp2", ctypes.c_float),
-                ("log_hi_exp2", ctypes.c_float)]
+                ("log_hi_exp2", ctypes.c_float), ("scale_fmt", ctypes.c_int32)]
 
 
 class MxqMetrics(ctypes.Structure):
@@ -55,7 +57,7 @@ _sig = {
     "mxq_act_sqmean_finalize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
     "mxq_quantize": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(MxqParams),
                                     _P, _P, _P]),
-    "mxq_project": (ctypes.c_int, [_P, _I64, _I32, ctypes.c_float, _P, _P]),
+    "mxq_project": (ctypes.c_int, [_P, _I64, _I32, _I32, ctypes.c_float, _P, _P]),
     "mxq_dequant": (ctypes.c_int, [_P, _P, ctypes.POINTER(MxqParams), _I64, _I64, _P, _P]),
     "mxq_error_workspace": (_SZ, [_I64, _I64]),
     "mxq_error": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
@@ -87,12 +89,13 @@ def lib_path() -> str:
 
 
 def params(fmt="nvfp4", mode="hopt", block=16, *, window=-1, tile_rows=None, log_points=64,
-           log_lo_exp2=-2.0, log_hi_exp2=2.0) -> MxqParams:
+           log_lo_exp2=-2.0, log_hi_exp2=2.0, scale_fmt="e4m3") -> MxqParams:
     f = FMT[fmt] if isinstance(fmt, str) else int(fmt)
+    sf = SCALE[scale_fmt] if isinstance(scale_fmt, str) else int(scale_fmt)
     m = MODE[mode] if isinstance(mode, str) else int(mode)
     if tile_rows is None:
         tile_rows = block if f == FMT["e4m3"] else 1
-    return MxqParams(f, m, block, tile_rows, window, log_points, log_lo_exp2, log_hi_exp2)
+    return MxqParams(f, m, block, tile_rows, window, log_points, log_lo_exp2, log_hi_exp2, sf)
 
 
 def _ptr(t):
@@ -184,7 +187,7 @@ def mxq_act_sqmean_finalize(partials: torch.Tensor, total_rows: int,
 
 def output_shapes(p: MxqParams, n: int, k: int):
     """(codes shape, codes dtype, scales shape, scales dtype) for a quantization."""
-    if p.fmt == FMT["nvfp4"]:
+    if p.fmt in (FMT["nvfp4"], FMT["int4"]):
         return (n, k // 2), torch.uint8, (n, k // p.block), torch.uint8
     if p.fmt == FMT["int8"]:
         return (n, k), torch.int8, (n, k // p.block), torch.uint8
@@ -206,13 +209,15 @@ def mxq_quantize(W: torch.Tensor, p: MxqParams, h: torch.Tensor | None = None, *
     return codes, scales
 
 
-def mxq_project(w: torch.Tensor, fmt: str, scale: float, *, q=None, stream=None) -> torch.Tensor:
-    """Magnitude codes of float32 ``w`` at one fixed scale (the search's element step)."""
+def mxq_project(w: torch.Tensor, fmt: str, scale: float, *, scale_fmt="e4m3", q=None,
+                stream=None) -> torch.Tensor:
+    """Magnitude codes of float32 ``w`` at one fixed scale (the search's element step);
+    ``scale`` is a value of the grid ``scale_fmt`` (NVFP4 / INT4 / INT8)."""
     w = w.contiguous()
     if q is None:
         q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
-    _check(_lib.mxq_project(_ptr(w), w.numel(), FMT[fmt], float(scale), _ptr(q),
-                            _stream(stream, w.device)), "mxq_project")
+    _check(_lib.mxq_project(_ptr(w), w.numel(), FMT[fmt], SCALE[scale_fmt], float(scale),
+                            _ptr(q), _stream(stream, w.device)), "mxq_project")
     return q
 
 

@@ -15,10 +15,13 @@
  *
  * over candidates on the E4M3 scale grid (all 126 positive finite values, or a window of
  * codes around the naive snap; qwantize "Results", sections "INT8 (FP8 E4M3 scales)" and
- * "NVFP4 (FP8 E4M3 scales)"), or, for E4M3 elements, on a logarithmic grid of float32 tile
- * scales ("quantization_algorithms.txt", sec. 1).
+ * "NVFP4 (FP8 E4M3 scales)"), on another 8-bit scale grid (UE8M0 powers of two -- MXFP4 --,
+ * UE4M4 or UE5M3; qwantize "Results", sections "MXFP4 (UE8M0 power-of-2 scales)" and
+ * "Exotic Scales"), or, for E4M3 elements, on a logarithmic grid of float32 tile scales
+ * ("quantization_algorithms.txt", sec. 1).
  *
- * Element grids: NVFP4 E2M1 {0, 0.5, 1, 1.5, 2, 3, 4, 6} (qmax 6); symmetric INT8
+ * Element grids: E2M1 {0, 0.5, 1, 1.5, 2, 3, 4, 6} (qmax 6); symmetric INT4 [-7, 7]
+ * (qmax 7; the NVINT4 rows of qwantize "Results", "GPTQ Quantization"); symmetric INT8
  * [-127, 127] with effective scale fl32(amax_e4m3 / 127) (qwantize "Results", INT8
  * section); E4M3 elements (max 448). Every rounding onto a grid is round-to-nearest with
  * ties to the even code and saturation; the quotient w / s is the IEEE float32 quotient.
@@ -67,12 +70,24 @@ typedef enum {
 } mxq_status;
 
 typedef enum { MXQ_F32 = 0, MXQ_BF16 = 1 } mxq_dtype;
-typedef enum { MXQ_FMT_NVFP4 = 0, MXQ_FMT_INT8 = 1, MXQ_FMT_E4M3 = 2 } mxq_fmt;
+typedef enum { MXQ_FMT_NVFP4 = 0, MXQ_FMT_INT8 = 1, MXQ_FMT_E4M3 = 2, MXQ_FMT_INT4 = 3 } mxq_fmt;
 typedef enum { MXQ_NAIVE = 0, MXQ_SSE = 1, MXQ_HOPT = 2 } mxq_mode;
+/* 8-bit block-scale grids (code -> value; every listed code finite):
+ *  MXQ_SCALE_E4M3   codes 0..126: 0, m/8 2^-6 (e = 0), (1 + m/8) 2^(e-7); candidates 1..126
+ *  MXQ_SCALE_UE4M4  codes 0..255: 0, m/16 2^-6 (e = 0), (1 + m/16) 2^(e-7) (max 496);
+ *                   candidates 1..255
+ *  MXQ_SCALE_UE5M3  codes 0..255: 0, m/8 2^-14 (e = 0), (1 + m/8) 2^(e-15) (max 122880);
+ *                   candidates 1..255
+ *  MXQ_SCALE_UE8M0  codes 0..254: 2^(code - 127) (OCP E8M0; 255 is NaN); candidates 0..254 */
+typedef enum { MXQ_SCALE_E4M3 = 0, MXQ_SCALE_UE4M4 = 1, MXQ_SCALE_UE5M3 = 2,
+               MXQ_SCALE_UE8M0 = 3 } mxq_scale_fmt;
 
 /* Quantizer settings.
- *  fmt        MXQ_FMT_NVFP4: E2M1 elements, one E4M3 scale per block of `block` (16 or 32)
- *             contiguous weights along k.
+ *  fmt        MXQ_FMT_NVFP4: E2M1 elements, one scale byte (grid `scale_fmt`) per block of
+ *             `block` (16 or 32) contiguous weights along k. With MXQ_SCALE_UE8M0 this is
+ *             MXFP4.
+ *             MXQ_FMT_INT4: int4 elements in [-7, 7], one scale byte (grid `scale_fmt`:
+ *             E4M3 -- NVINT4 --, UE4M4 or UE5M3) per block of `block` (16 or 32) weights.
  *             MXQ_FMT_INT8: int8 elements in [-127, 127], one E4M3 byte (the stored amax)
  *             per block of `block` (32, 64, 128 or 256) weights; effective scale
  *             fl32(E4M3 / 127).
@@ -81,12 +96,18 @@ typedef enum { MXQ_NAIVE = 0, MXQ_SSE = 1, MXQ_HOPT = 2 } mxq_mode;
  *  mode       MXQ_NAIVE, MXQ_SSE or MXQ_HOPT.
  *  block      see fmt.
  *  tile_rows  1 for NVFP4 and INT8; 64 (= block) for E4M3 tiles.
- *  window     NVFP4 / INT8 search: -1 = all 126 positive finite E4M3 scales (codes
- *             0x01..0x7E); w >= 0 = codes [c0 - w, c0 + w] clipped to [1, 126] around the
- *             naive code c0 ([1, max(w, 1)] when c0 is 0). Ignored for E4M3 tiles.
+ *  window     NVFP4 / INT4 / INT8 search: -1 = every candidate code of the scale grid
+ *             (E4M3: the 126 positive finite values 0x01..0x7E); w >= 0 = codes
+ *             [c0 - w, c0 + w] clipped to the candidate codes around the naive code c0
+ *             ([1, max(w, 1)] when c0 is a zero scale). Ignored for E4M3 tiles.
  *  log_points E4M3 tiles: P grid points g_p = fl32(2^(lo + (hi - lo) p / (P - 1))),
  *             candidate s_p = fl32(fl32(amax_tile / 448) * g_p); 2 <= P <= 256.
  *  log_lo_exp2, log_hi_exp2  lo and hi (finite, lo < hi); the pages' grid is -2, 2.
+ *  scale_fmt  the block-scale grid (mxq_scale_fmt) of NVFP4 and INT4 elements; INT8 and
+ *             E4M3 tiles need MXQ_SCALE_E4M3 (0); UE8M0 only with NVFP4 elements.
+ *             Naive scale: UE8M0 2^(floor(log2 amax) - 2) (the OCP rule, 2 = the largest
+ *             E2M1 exponent), clamped to codes 0..254 (0 for amax = 0); every other grid
+ *             its nearest value (RNE, saturating) to fl32(amax / qmax).
  */
 typedef struct mxq_params {
     int32_t fmt;
@@ -97,6 +118,7 @@ typedef struct mxq_params {
     int32_t log_points;
     float log_lo_exp2;
     float log_hi_exp2;
+    int32_t scale_fmt;
 } mxq_params;
 
 /* Weight error metrics from the four sums that mxq_error produces. */
@@ -157,17 +179,20 @@ MXQ_API mxq_status mxq_act_sqmean_finalize(const double* partials, int64_t parts
  *  p       host pointer to the settings.
  *  codes   device, dense row-major:
  *            NVFP4 uint8 [n, k/2]: element 2i in the low nibble, nibble = sign << 3 | e2m1
+ *            INT4  uint8 [n, k/2]: element 2i in the low nibble, nibble = the signed code
+ *                  in two's complement (-7 .. 7)
  *            INT8  int8  [n, k]:   two's complement in [-127, 127]
  *            E4M3  uint8 [n, k]:   sign << 7 | e4m3 code
  *          The sign bit of a zero magnitude is the weight's sign bit (INT8 has no -0).
  *  scales  device, dense row-major:
- *            NVFP4, INT8: uint8 E4M3 codes [n, k/block]; code 0 only from a naive snap
- *            that rounds to zero (then every magnitude is 0);
+ *            NVFP4, INT4, INT8: uint8 scale codes [n, k/block] of the scale grid; a zero
+ *            scale (code 0 of E4M3 / UE4M4 / UE5M3) only from a naive snap that rounds
+ *            to zero (then every magnitude is 0);
  *            E4M3: float [n/64, k/64] tile scales (0 for an all-zero tile).
  *  Shapes: k % block == 0; for E4M3 tiles n % 64 == 0 and k % 64 == 0.
  *  Result: identical to the plain definition evaluated with IEEE float32 quotients and
  *  float32 dequantised values, candidate errors accumulated in double in element order,
- *  ties to the smallest scale (NVFP4 and INT8: exactly, including ties; E4M3 tiles:
+ *  ties to the smallest scale (NVFP4, INT4 and INT8: exactly, including ties; E4M3 tiles:
  *  exactly wherever the two best tile errors differ by more than 1e-6 relative).
  * ------------------------------------------------------------------------------------ */
 MXQ_API mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
@@ -178,20 +203,25 @@ MXQ_API mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t
  * Element projection at one fixed scale -- the per-element step of the search above,
  * exposed so that it can be verified exhaustively.
  *
- *  w      device float [count], 4-byte aligned (only |w| is used).
- *  fmt    MXQ_FMT_NVFP4: q = RNE_E2M1(fl32(|w| / scale)) code 0..7, scale an E4M3 value;
- *         MXQ_FMT_INT8:  q = min(127, RNE_int(fl32(|w| / fl32(scale / 127)))), scale the
- *                        stored E4M3 amax;
- *         MXQ_FMT_E4M3:  q = RNE_E4M3(fl32(|w| / scale)) code 0..126, any float scale > 0.
- *  q      device uint8 [count]: the magnitude codes.
+ *  w          device float [count], 4-byte aligned (only |w| is used).
+ *  fmt        MXQ_FMT_NVFP4: q = RNE_E2M1(fl32(|w| / scale)) code 0..7;
+ *             MXQ_FMT_INT4:  q = min(7, RNE_int(fl32(|w| / scale)));
+ *             MXQ_FMT_INT8:  q = min(127, RNE_int(fl32(|w| / fl32(scale / 127)))), scale
+ *                            the stored E4M3 amax;
+ *             MXQ_FMT_E4M3:  q = RNE_E4M3(fl32(|w| / scale)) code 0..126, any float
+ *                            scale > 0.
+ *  scale_fmt  NVFP4 / INT4: the grid that `scale` must be a positive value of
+ *             (mxq_scale_fmt); INT8: MXQ_SCALE_E4M3; ignored for E4M3 elements.
+ *  q          device uint8 [count]: the magnitude codes.
  * ------------------------------------------------------------------------------------ */
-MXQ_API mxq_status mxq_project(const float* w, int64_t count, int32_t fmt, float scale,
-                               uint8_t* q, void* stream);
+MXQ_API mxq_status mxq_project(const float* w, int64_t count, int32_t fmt, int32_t scale_fmt,
+                               float scale, uint8_t* q, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * Dequantisation: out [n, k] float (device, dense) = s * q with the layouts above
- * (NVFP4: E4M3(scale) * E2M1(code); INT8: code * fl32(E4M3(scale) / 127), the product
- * rounded to float; E4M3: tile scale * E4M3(code), rounded to float).
+ * (NVFP4: grid(scale) * E2M1(code); INT4: grid(scale) * code; INT8: code *
+ * fl32(E4M3(scale) / 127), the product rounded to float; E4M3: tile scale * E4M3(code),
+ * rounded to float). A UE8M0 scale byte 255 (NaN) decodes to NaN.
  * ------------------------------------------------------------------------------------ */
 MXQ_API mxq_status mxq_dequant(const void* codes, const void* scales, const mxq_params* p, int64_t n,
                        int64_t k, float* out, void* stream);

@@ -89,6 +89,11 @@ def test_quantize_rejections(mxq):
     assert q(mxq, fmt="e4m3", mode="hopt", block=64, log_points=1) == S["MXQ_ERR_INVALID_ARG"]
     assert q(mxq, fmt="e4m3", mode="hopt", block=64, log_lo_exp2=3.0) == S["MXQ_ERR_INVALID_ARG"]
     assert q(mxq, fmt="nvfp4", mode="sse", block=16, window=-2) == S["MXQ_ERR_INVALID_ARG"]
+    assert q(mxq, fmt="int4", mode="sse", block=64) == S["MXQ_ERR_UNSUPPORTED"]
+    assert q(mxq, fmt="int4", mode="sse", block=16, scale_fmt="ue8m0") == S["MXQ_ERR_UNSUPPORTED"]
+    assert q(mxq, fmt="nvfp4", mode="sse", block=16, scale_fmt=7) == S["MXQ_ERR_INVALID_ARG"]
+    assert q(mxq, fmt="int8", mode="sse", block=32, scale_fmt="ue4m4") == S["MXQ_ERR_UNSUPPORTED"]
+    assert q(mxq, fmt="e4m3", mode="sse", block=64, scale_fmt="ue5m3") == S["MXQ_ERR_UNSUPPORTED"]
     p = mxq.params("nvfp4", "sse", 16)
     p.mode = 9
     assert mxq._lib.mxq_quantize(FAKE, 1, 64, 256, 256, FAKE, ctypes.byref(p), FAKE, FAKE,
@@ -129,11 +134,17 @@ def test_act_sqmean_rejections(mxq):
 def test_project_and_error_rejections(mxq):
     S = {v: k for k, v in mxq.STATUS.items()}
     pr = mxq._lib.mxq_project
-    assert pr(FAKE, 16, 0, 0.3, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]   # not an E4M3 value
-    assert pr(FAKE, 16, 0, 500.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
-    assert pr(FAKE, 16, 2, -1.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
-    assert pr(FAKE, 16, 5, 1.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
-    assert pr(FAKE + 2, 16, 0, 1.0, FAKE, None) == S["MXQ_ERR_ALIGN"]
+    assert pr(FAKE, 16, 0, 0, 0.3, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]  # not an E4M3 value
+    assert pr(FAKE, 16, 0, 0, 500.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert pr(FAKE, 16, 2, 0, -1.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert pr(FAKE, 16, 5, 0, 1.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert pr(FAKE + 2, 16, 0, 0, 1.0, FAKE, None) == S["MXQ_ERR_ALIGN"]
+    assert pr(FAKE, 16, 0, 3, 3.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]  # not a power of 2
+    assert pr(FAKE, 16, 0, 1, 0.1, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]  # not a UE4M4 value
+    assert pr(FAKE, 16, 0, 2, 122880.0 * 2, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert pr(FAKE, 16, 3, 9, 1.0, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]  # unknown grid
+    assert pr(FAKE, 16, 1, 1, 1.0, FAKE, None) == S["MXQ_ERR_UNSUPPORTED"]  # INT8 on UE4M4
+    assert pr(FAKE, 0, 0, 3, 2.0 ** -127, FAKE, None) == 0               # empty: no launch
     p = mxq.params("nvfp4", "sse", 16)
     e = mxq._lib.mxq_error
     need = mxq.mxq_error_workspace(64, 256)
