@@ -390,6 +390,119 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
 }
 
 /* ----------------------------------------------------------------------------------
+ * Block-Hessian objective ("quantization_algorithms.txt", section 1: the scale minimising
+ * || X_b (W_b - s Q(W_b / s))^T ||_F^2 over the block's calibration inputs X_b; the
+ * diagonal h_j = E[x_j^2] is its cheap approximation). For one row's block of B weights
+ * the objective is R * d^T G d with G = X_b^T X_b / R, the block's B x B Gram matrix.
+ * G is kept in float32 as fl32(sum_r x_ri x_rj / R) (the sum in double, rows ascending,
+ * then divided and rounded once, exactly as h), so diag(G) is h bit for bit.
+ * ---------------------------------------------------------------------------------- */
+
+/* G[b][i][j] for every column block b = 0 .. cols/B - 1 (row-major [cols/B][B][B]). */
+int orc_block_gram(const void *X, int dtype, int64_t rows, int64_t cols, int64_t ld, int B,
+                   float *G)
+{
+    if (B <= 0 || cols % B != 0) return -1;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)B * (size_t)B);
+    for (int64_t b = 0; b < cols / B; ++b) {
+        for (int t = 0; t < B * B; ++t) acc[t] = 0.0;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int i = 0; i < B; ++i) {
+                double xi = (double)elem(X, dtype, ld, r, b * B + i);
+                for (int j = 0; j < B; ++j)
+                    acc[i * B + j] += xi * (double)elem(X, dtype, ld, r, b * B + j);
+            }
+        for (int t = 0; t < B * B; ++t)
+            G[b * B * B + t] = rows > 0 ? (float)(acc[t] / (double)rows) : 0.0f;
+    }
+    free(acc);
+    return 0;
+}
+
+/* d^T G d of one block at candidate c, in double, in the order
+ * e += G_ij * (d_i * d_j) for i ascending, j ascending (d_i = w_i - fl32(s q_i)). */
+static double block_error_gram(int fmt, int sfmt, int c, const float *w, const float *Gb, int B)
+{
+    double *d = (double *)malloc(sizeof(double) * (size_t)B);
+    for (int j = 0; j < B; ++j) {
+        float wq_abs;
+        project(fmt, sfmt, c, w[j], &wq_abs);
+        d[j] = (double)w[j] - (double)copysignf(wq_abs, w[j]);
+    }
+    double e = 0.0;
+    for (int i = 0; i < B; ++i)
+        for (int j = 0; j < B; ++j)
+            e += (double)Gb[i * B + j] * (d[i] * d[j]);
+    free(d);
+    return e;
+}
+
+/*
+ * Block-Hessian H-optimal search: as orc_quantize_blocks in SSE / H mode, with the
+ * candidate error d^T G_b d (G from orc_block_gram, [k/B][B][B] float). Same outputs,
+ * candidates, window and tie rule.
+ */
+int orc_quantize_blocks_gram(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
+                             const float *G, int fmt, int sfmt, int B, int window,
+                             int64_t row0, int64_t row1, uint8_t *codes, uint8_t *scales,
+                             double *best, double *second, int32_t *naive)
+{
+    scale_grid g;
+    if (B <= 0 || k % B != 0 || grid_of(sfmt, &g) || G == NULL) return -1;
+    if (fmt != ORC_NVFP4 && fmt != ORC_INT8 && fmt != ORC_INT4) return -1;
+    if (fmt == ORC_INT8 && sfmt != ORC_S_E4M3) return -1;
+    if (fmt == ORC_INT4 && sfmt == ORC_S_UE8M0) return -1;
+    const int cmax = g.n - 1;
+    int64_t kb = k / B;
+    float *w = (float *)malloc(sizeof(float) * (size_t)B);
+    for (int64_t i = row0; i < row1 && i < n; ++i) {
+        for (int64_t b = 0; b < kb; ++b) {
+            int64_t j0 = b * B;
+            const float *Gb = G + b * B * B;
+            float amax = 0.0f;
+            for (int j = 0; j < B; ++j) {
+                w[j] = elem(W, dtype, ld, i, j0 + j);
+                if (fabsf(w[j]) > amax) amax = fabsf(w[j]);
+            }
+            int c0 = naive_code(fmt, sfmt, amax);
+            int lo = g.first, hi = cmax;
+            if (window >= 0) {
+                lo = c0 - window < g.first ? g.first : c0 - window;
+                hi = c0 + window > cmax ? cmax : c0 + window;
+                if (g.tab[c0] == 0.0f) { lo = 1; hi = window < 1 ? 1 : window; }
+            }
+            double e1 = INFINITY, e2 = INFINITY;
+            int cbest = lo;
+            for (int c = lo; c <= hi; ++c) {
+                double e = block_error_gram(fmt, sfmt, c, w, Gb, B);
+                if (e < e1) { e2 = e1; e1 = e; cbest = c; }
+                else if (e < e2) e2 = e;
+            }
+            scales[i * kb + b] = (uint8_t)cbest;
+            if (best) best[i * kb + b] = e1;
+            if (second) second[i * kb + b] = e2;
+            if (naive) naive[i * kb + b] = c0;
+            for (int j = 0; j < B; ++j) {
+                float wq_abs;
+                int q = project(fmt, sfmt, cbest, w[j], &wq_abs);
+                int neg = signbit(w[j]) ? 1 : 0;
+                if (fmt == ORC_INT8) {
+                    ((int8_t *)codes)[i * k + j0 + j] = (int8_t)(neg ? -q : q);
+                } else {
+                    uint8_t nib = (fmt == ORC_NVFP4) ? (uint8_t)((neg << 3) | q)
+                                                     : (uint8_t)((neg ? -q : q) & 15);
+                    uint8_t *p = &codes[i * (k / 2) + (j0 + j) / 2];
+                    p[0] = ((j0 + j) & 1) ? (uint8_t)((p[0] & 0x0F) | (nib << 4))
+                                          : (uint8_t)((p[0] & 0xF0) | nib);
+                }
+            }
+        }
+    }
+    free(w);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------------------
  * E4M3 elements on T x T tiles with one float32 scale per tile, searched on a
  * logarithmic grid ("quantization_algorithms.txt", section 1).
  * base = fl32(amax_tile / 448); grid g_p = fl32(2^(lo + (hi - lo) p / (P - 1))),

@@ -76,6 +76,11 @@ def lib():
             L.orc_quantize_blocks.restype = _I
             L.orc_quantize_blocks.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I, _I,
                                               _I64, _I64, _P, _P, _P, _P, _P]
+            L.orc_block_gram.restype = _I
+            L.orc_block_gram.argtypes = [_P, _I, _I64, _I64, _I64, _I, _P]
+            L.orc_quantize_blocks_gram.restype = _I
+            L.orc_quantize_blocks_gram.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I,
+                                                   _I64, _I64, _P, _P, _P, _P, _P]
             L.orc_log_grid.argtypes = [_I, _D, _D, _P]
             L.orc_quantize_tiles.restype = _I
             L.orc_quantize_tiles.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _D, _D,
@@ -275,6 +280,43 @@ def quantize(W, fmt: str, mode: str, block: int, *, h=None, window: int = -1,
         if rc != 0:
             raise ValueError("oracle rejected the arguments")
     _run_ranges(run, r0, r1, nt)
+    return Result(codes=codes, scales=scales, best=best, second=second, naive=naive)
+
+
+def block_gram(X, B: int) -> np.ndarray:
+    """G[b] = fl32(X_b^T X_b / R) for every column block b: float32 [cols/B, B, B]."""
+    X, dt = _as_input(X)
+    R, K = X.shape
+    G = np.zeros((K // B, B, B), np.float32)
+    if lib().orc_block_gram(_ptr(X), dt, R, K, K, B, _ptr(G)) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return G
+
+
+def quantize_gram(W, fmt: str, block: int, G, *, window: int = -1, rows=None, n_threads=1,
+                  sfmt: str = "e4m3") -> Result:
+    """Block-Hessian H-optimal search of W [n, k] with the Gram blocks G [k/B, B, B]."""
+    W, dt = _as_input(W)
+    n, k = W.shape
+    G = np.ascontiguousarray(G, dtype=np.float32)
+    if G.shape != (k // block, block, block):
+        raise ValueError("G must be [k/B, B, B]")
+    f = FMTS[fmt]
+    kb = k // block
+    codes = np.zeros((n, k // 2) if f in (NVFP4, INT4) else (n, k), np.uint8)
+    scales = np.zeros((n, kb), np.uint8)
+    best = np.full((n, kb), np.nan)
+    second = np.full((n, kb), np.nan)
+    naive = np.full((n, kb), -1, np.int32)
+    r0, r1 = (0, n) if rows is None else rows
+
+    def run(a, b):
+        rc = lib().orc_quantize_blocks_gram(_ptr(W), dt, n, k, k, _ptr(G), f, SFMTS[sfmt],
+                                            block, window, a, b, _ptr(codes), _ptr(scales),
+                                            _ptr(best), _ptr(second), _ptr(naive))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+    _run_ranges(run, r0, r1, _threads(n_threads))
     return Result(codes=codes, scales=scales, best=best, second=second, naive=naive)
 
 

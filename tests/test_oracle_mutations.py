@@ -42,6 +42,14 @@ MUTANTS = {
     "ue8m0_skips_code_0": ("case ORC_S_UE8M0: *g = (scale_grid){T_UE8M0, 255, 0}; return 0;",
                            "case ORC_S_UE8M0: *g = (scale_grid){T_UE8M0, 255, 1}; return 0;"),
     "int4_dequant_magnitude": ("int q = (nib & 8) ? 16 - nib : nib;", "int q = nib & 7;"),
+    "gram_not_a_mean": ("G[b * B * B + t] = rows > 0 ? (float)(acc[t] / (double)rows) : 0.0f;",
+                        "G[b * B * B + t] = rows > 0 ? (float)(acc[t]) : 0.0f;"),
+    "gram_wrong_columns": ("acc[i * B + j] += xi * (double)elem(X, dtype, ld, r, b * B + j);",
+                           "acc[i * B + j] += xi * (double)elem(X, dtype, ld, r, j);"),
+    "gram_diagonal_only": ("            e += (double)Gb[i * B + j] * (d[i] * d[j]);",
+                           "            e += (i == j) ? (double)Gb[i * B + j] * (d[i] * d[j]) : 0.0;"),
+    "gram_unsigned_difference": ("d[j] = (double)w[j] - (double)copysignf(wq_abs, w[j]);",
+                                 "d[j] = (double)fabsf(w[j]) - (double)wq_abs;"),
     "dequant_not_rounded": ("float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - (double)wq;",
                             "float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - 1.0000001 * (double)wq;"),
 }
@@ -60,6 +68,7 @@ def test_planted_mistake_is_caught(name, tmp_path):
     env = dict(os.environ, MXQ_ORACLE_LIB=str(so))
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                           os.path.join(HERE, "test_oracle_pins.py"),
-                          os.path.join(HERE, "test_oracle_pins_scales.py")], cwd=ROOT, env=env,
+                          os.path.join(HERE, "test_oracle_pins_scales.py"),
+                          os.path.join(HERE, "test_oracle_pins_gram.py")], cwd=ROOT, env=env,
                          capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"pins did not catch planted mistake {name}:\n{res.stdout[-2000:]}"
