@@ -307,6 +307,49 @@ static int naive_code(int fmt, int sfmt, float amax)
 
 int orc_naive_code(int fmt, int sfmt, float amax) { return naive_code(fmt, sfmt, amax); }
 
+/* Candidate codes of one block: every candidate of the grid, or the window of codes
+ * [c0 - window, c0 + window] clipped to them ([1, max(window, 1)] for a zero naive scale). */
+static void candidate_range(const scale_grid *g, int c0, int window, int *lo, int *hi)
+{
+    const int cmax = g->n - 1;
+    *lo = g->first;
+    *hi = cmax;
+    if (window >= 0) {
+        *lo = c0 - window < g->first ? g->first : c0 - window;
+        *hi = c0 + window > cmax ? cmax : c0 + window;
+        if (g->tab[c0] == 0.0f) { *lo = 1; *hi = window < 1 ? 1 : window; }
+    }
+}
+
+/* Running smallest and second-smallest candidate error; equal errors keep the earlier
+ * (lower) code. */
+static void keep_best(double e, int c, double *e1, double *e2, int *cbest)
+{
+    if (e < *e1) { *e2 = *e1; *e1 = e; *cbest = c; }
+    else if (e < *e2) *e2 = e;
+}
+
+/* Codes of row i's block starting at column j0 at scale code c (layouts as below). */
+static void emit_block(int fmt, int sfmt, int c, const float *w, int B, uint8_t *codes,
+                       int64_t i, int64_t j0, int64_t k)
+{
+    for (int j = 0; j < B; ++j) {
+        float wq_abs;
+        int q = project(fmt, sfmt, c, w[j], &wq_abs);
+        int neg = signbit(w[j]) ? 1 : 0;
+        if (fmt == ORC_NVFP4 || fmt == ORC_INT4) {
+            uint8_t nib = (fmt == ORC_NVFP4) ? (uint8_t)((neg << 3) | q)
+                                             : (uint8_t)((neg ? -q : q) & 15);
+            uint8_t *p = &codes[i * (k / 2) + (j0 + j) / 2];
+            if (((j0 + j) & 1) == 0) *p = (uint8_t)((*p & 0xF0) | nib);
+            else *p = (uint8_t)((*p & 0x0F) | (nib << 4));
+        } else {
+            int v = neg ? -q : q;
+            ((int8_t *)codes)[i * k + j0 + j] = (int8_t)v;
+        }
+    }
+}
+
 /*
  * Quantize rows [row0, row1) of W [n, k] (leading dimension ld) in blocks of B along k.
  * fmt: ORC_NVFP4 (E2M1 elements), ORC_INT4 or ORC_INT8; sfmt: the scale grid
@@ -333,7 +376,6 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
     if (fmt == ORC_INT8 && sfmt != ORC_S_E4M3) return -1;
     if (fmt == ORC_INT4 && sfmt == ORC_S_UE8M0) return -1;
     if (mode == ORC_HOPT && h == NULL) return -1;
-    const int cmax = g.n - 1;
     int64_t kb = k / B;
     float *w = (float *)malloc(sizeof(float) * (size_t)B);
     float *cw = (float *)malloc(sizeof(float) * (size_t)B);
@@ -350,38 +392,17 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
             int cbest = c0;
             double e1 = NAN, e2 = NAN;
             if (mode != ORC_NAIVE) {
-                int lo = g.first, hi = cmax;
-                if (window >= 0) {
-                    lo = c0 - window < g.first ? g.first : c0 - window;
-                    hi = c0 + window > cmax ? cmax : c0 + window;
-                    if (g.tab[c0] == 0.0f) { lo = 1; hi = window < 1 ? 1 : window; }
-                }
+                int lo, hi;
+                candidate_range(&g, c0, window, &lo, &hi);
                 e1 = INFINITY; e2 = INFINITY; cbest = lo;
-                for (int c = lo; c <= hi; ++c) {
-                    double e = block_error(fmt, sfmt, c, w, cw, B);
-                    if (e < e1) { e2 = e1; e1 = e; cbest = c; }
-                    else if (e < e2) e2 = e;
-                }
+                for (int c = lo; c <= hi; ++c)
+                    keep_best(block_error(fmt, sfmt, c, w, cw, B), c, &e1, &e2, &cbest);
             }
             scales[i * kb + b] = (uint8_t)cbest;
             if (best) best[i * kb + b] = e1;
             if (second) second[i * kb + b] = e2;
             if (naive) naive[i * kb + b] = c0;
-            for (int j = 0; j < B; ++j) {
-                float wq_abs;
-                int q = project(fmt, sfmt, cbest, w[j], &wq_abs);
-                int neg = signbit(w[j]) ? 1 : 0;
-                if (fmt == ORC_NVFP4 || fmt == ORC_INT4) {
-                    uint8_t nib = (fmt == ORC_NVFP4) ? (uint8_t)((neg << 3) | q)
-                                                     : (uint8_t)((neg ? -q : q) & 15);
-                    uint8_t *p = &codes[i * (k / 2) + (j0 + j) / 2];
-                    if (((j0 + j) & 1) == 0) *p = (uint8_t)((*p & 0xF0) | nib);
-                    else *p = (uint8_t)((*p & 0x0F) | (nib << 4));
-                } else {
-                    int v = neg ? -q : q;
-                    ((int8_t *)codes)[i * k + j0 + j] = (int8_t)v;
-                }
-            }
+            emit_block(fmt, sfmt, cbest, w, B, codes, i, j0, k);
         }
     }
     free(w);
@@ -452,7 +473,6 @@ int orc_quantize_blocks_gram(const void *W, int dtype, int64_t n, int64_t k, int
     if (fmt != ORC_NVFP4 && fmt != ORC_INT8 && fmt != ORC_INT4) return -1;
     if (fmt == ORC_INT8 && sfmt != ORC_S_E4M3) return -1;
     if (fmt == ORC_INT4 && sfmt == ORC_S_UE8M0) return -1;
-    const int cmax = g.n - 1;
     int64_t kb = k / B;
     float *w = (float *)malloc(sizeof(float) * (size_t)B);
     for (int64_t i = row0; i < row1 && i < n; ++i) {
@@ -465,37 +485,17 @@ int orc_quantize_blocks_gram(const void *W, int dtype, int64_t n, int64_t k, int
                 if (fabsf(w[j]) > amax) amax = fabsf(w[j]);
             }
             int c0 = naive_code(fmt, sfmt, amax);
-            int lo = g.first, hi = cmax;
-            if (window >= 0) {
-                lo = c0 - window < g.first ? g.first : c0 - window;
-                hi = c0 + window > cmax ? cmax : c0 + window;
-                if (g.tab[c0] == 0.0f) { lo = 1; hi = window < 1 ? 1 : window; }
-            }
+            int lo, hi, cbest;
+            candidate_range(&g, c0, window, &lo, &hi);
             double e1 = INFINITY, e2 = INFINITY;
-            int cbest = lo;
-            for (int c = lo; c <= hi; ++c) {
-                double e = block_error_gram(fmt, sfmt, c, w, Gb, B);
-                if (e < e1) { e2 = e1; e1 = e; cbest = c; }
-                else if (e < e2) e2 = e;
-            }
+            cbest = lo;
+            for (int c = lo; c <= hi; ++c)
+                keep_best(block_error_gram(fmt, sfmt, c, w, Gb, B), c, &e1, &e2, &cbest);
             scales[i * kb + b] = (uint8_t)cbest;
             if (best) best[i * kb + b] = e1;
             if (second) second[i * kb + b] = e2;
             if (naive) naive[i * kb + b] = c0;
-            for (int j = 0; j < B; ++j) {
-                float wq_abs;
-                int q = project(fmt, sfmt, cbest, w[j], &wq_abs);
-                int neg = signbit(w[j]) ? 1 : 0;
-                if (fmt == ORC_INT8) {
-                    ((int8_t *)codes)[i * k + j0 + j] = (int8_t)(neg ? -q : q);
-                } else {
-                    uint8_t nib = (fmt == ORC_NVFP4) ? (uint8_t)((neg << 3) | q)
-                                                     : (uint8_t)((neg ? -q : q) & 15);
-                    uint8_t *p = &codes[i * (k / 2) + (j0 + j) / 2];
-                    p[0] = ((j0 + j) & 1) ? (uint8_t)((p[0] & 0x0F) | (nib << 4))
-                                          : (uint8_t)((p[0] & 0xF0) | nib);
-                }
-            }
+            emit_block(fmt, sfmt, cbest, w, B, codes, i, j0, k);
         }
     }
     free(w);

@@ -17,15 +17,15 @@ MUTANTS = {
     "ties_always_up": ("return (lo % 2 == 0) ? lo : hi;", "return hi;"),
     "naive_divisor": ("return nearest_rne(T_E4M3, 127, amax / 6.0f);",
                       "return nearest_rne(T_E4M3, 127, amax / 4.0f);"),
-    "candidate_ties_high": ("if (e < e1) { e2 = e1; e1 = e; cbest = c; }",
-                            "if (e <= e1) { e2 = e1; e1 = e; cbest = c; }"),
+    "candidate_ties_high": ("if (e < *e1) { *e2 = *e1; *e1 = e; *cbest = c; }",
+                            "if (e <= *e1) { *e2 = *e1; *e1 = e; *cbest = c; }"),
     "int8_divisor": ("float s = T_E4M3[c] / 127.0f;\n        float z = a / s;",
                      "float s = T_E4M3[c] / 128.0f;\n        float z = a / s;"),
     "sign_dropped": ("int neg = signbit(w[j]) ? 1 : 0;", "int neg = 0;"),
     "tile_h_by_row": ("double c = (mode == ORC_HOPT) ? (double)h[j0 + j] : 1.0;",
                       "double c = (mode == ORC_HOPT) ? (double)h[i0 + i] : 1.0;"),
-    "window_short": ("hi = c0 + window > cmax ? cmax : c0 + window;",
-                     "hi = c0 + window > cmax ? cmax : c0 + window - 1;"),
+    "window_short": ("*hi = c0 + window > cmax ? cmax : c0 + window;",
+                     "*hi = c0 + window > cmax ? cmax : c0 + window - 1;"),
     "mean_over_r_minus_1": ("(float)(s[j] / (double)rows)", "(float)(s[j] / (double)(rows - 1))"),
     "e2m1_exponent": ("ldexp(1.0 + (double)m / 2.0, e - 1)", "ldexp(1.0 + (double)m / 2.0, e)"),
     "nibble_order": ("if (((j0 + j) & 1) == 0) *p", "if (((j0 + j) & 1) == 1) *p"),
