@@ -643,6 +643,24 @@ int orc_dequant(const uint8_t *codes, const void *scales, int fmt, int sfmt, int
     return 0;
 }
 
+/* Block-scale bytes [n][kb] rearranged into the tile layout that sm_100 block-scaled tensor
+ * core instructions read (not on the pages; an interface requirement of the hardware):
+ * 128-row x 4-column tiles of 512 bytes, tiles ordered by row tile then column tile; inside
+ * a tile, row m and column c sit at byte (m % 32) * 16 + (m / 32) * 4 + c. Rows are padded to
+ * a multiple of 128 and columns to a multiple of 4 with zero bytes. out: ceil(n/128) * 128 *
+ * ceil(kb/4) * 4 bytes. */
+void orc_swizzle_scales(const uint8_t *in, int64_t n, int64_t kb, uint8_t *out)
+{
+    int64_t rt = (n + 127) / 128, ct = (kb + 3) / 4;
+    memset(out, 0, (size_t)(rt * 128 * ct * 4));
+    for (int64_t m = 0; m < n; ++m)
+        for (int64_t c = 0; c < kb; ++c) {
+            int64_t tile = (m / 128) * ct + c / 4;
+            int64_t mm = m % 128, cc = c % 4;
+            out[tile * 512 + (mm % 32) * 16 + (mm / 32) * 4 + cc] = in[m * kb + c];
+        }
+}
+
 /* sums[0] = sum (w - w^)^2, sums[1] = sum w^2, sums[2] = sum h_j (w - w^)^2,
  * sums[3] = sum h_j w^2 (both 0 when h is NULL); doubles, row-major order. */
 void orc_error_sums(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,

@@ -81,6 +81,7 @@ def lib():
             L.orc_quantize_blocks_gram.restype = _I
             L.orc_quantize_blocks_gram.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I,
                                                    _I64, _I64, _P, _P, _P, _P, _P]
+            L.orc_swizzle_scales.argtypes = [_P, _I64, _I64, _P]
             L.orc_log_grid.argtypes = [_I, _D, _D, _P]
             L.orc_quantize_tiles.restype = _I
             L.orc_quantize_tiles.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _D, _D,
@@ -338,6 +339,15 @@ def dequant(codes, scales, fmt: str, block: int, n: int, k: int,
                            _ptr(out))
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def swizzle_scales(scales) -> np.ndarray:
+    """Scale bytes [n, kb] in the 128 x 4 tile layout of sm_100 block-scaled MMA (flat)."""
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    n, kb = scales.shape
+    out = np.zeros(((n + 127) // 128) * 128 * ((kb + 3) // 4) * 4, np.uint8)
+    lib().orc_swizzle_scales(_ptr(scales), n, kb, _ptr(out))
     return out
 
 

@@ -246,3 +246,20 @@ def test_zero_block_takes_first_candidate(orc):
         assert np.all(r.codes == 0)
     rn = orc.quantize(W, "nvfp4", "naive", 16, sfmt="ue8m0")
     assert rn.scales.tolist() == [[0, 0]]
+
+
+def test_swizzled_scale_layout(orc):
+    """128 x 4 tiles of 512 bytes; in a tile row m, column c at (m % 32) 16 + (m / 32) 4 + c;
+    tiles by row tile, then column tile; zero padding. Hand-placed entries and a bijection."""
+    n, kb = 300, 10                                   # 3 row tiles, 3 column tiles (padded)
+    s = (np.arange(n * kb) % 251 + 1).astype(np.uint8).reshape(n, kb)
+    out = orc.swizzle_scales(s)
+    assert out.size == 384 * 12
+    assert out[0] == s[0, 0] and out[1] == s[0, 1] and out[3] == s[0, 3]
+    assert out[16] == s[1, 0] and out[4] == s[32, 0] and out[15 * 16 + 3 * 4 + 2] == s[111, 2]
+    assert out[512] == s[0, 4]                        # next column tile
+    assert out[3 * 512 + 5 * 16] == s[133, 0]         # second row tile, row 5 of it
+    assert out[2 * 512 + 0 * 16 + 1] == s[0, 9]       # column 9 = tile 2, column 1
+    assert out[2 * 512 + 2] == 0                      # padded column 10
+    nz = out[out != 0]
+    assert sorted(nz.tolist()) == sorted(s.reshape(-1).tolist())
