@@ -61,7 +61,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block", type=int, default=0, help="block size (default: the workload's)")
-    ap.add_argument("--mode", default="", choices=["", "naive", "sse", "hopt"])
+    ap.add_argument("--mode", default="", choices=["", "naive", "sse", "hopt", "bhopt"],
+                    help="bhopt: the block-Hessian objective d^T G_b d (Gram pass on the "
+                         "tensor cores instead of the h pass)")
     ap.add_argument("--fmt", default="", choices=["", "nvfp4", "int4", "int8", "e4m3"],
                     help="element format (default: the workload's)")
     ap.add_argument("--scale-fmt", default="", choices=["", "e4m3", "ue4m4", "ue5m3", "ue8m0"],
@@ -197,10 +199,17 @@ def oracle_step_sample(X_bits, W_bits, h_np, n_threads, R_full, N_full, q):
     x_rows, K = X_bits.shape
     w_rows = W_bits.shape[0]
     t0 = time.perf_counter()
-    orc.act_sqmean(X_bits, n_threads=n_threads)
+    if mode == "bhopt":
+        G = orc.block_gram(X_bits, block)
+    else:
+        orc.act_sqmean(X_bits, n_threads=n_threads)
     t1 = time.perf_counter()
-    r = orc.quantize(W_bits, fmt, mode, block, h=h_np, window=window, n_threads=n_threads,
-                     sfmt=q.sfmt)
+    if mode == "bhopt":
+        r = orc.quantize_gram(W_bits, fmt, block, G, window=window, n_threads=n_threads,
+                              sfmt=q.sfmt)
+    else:
+        r = orc.quantize(W_bits, fmt, mode, block, h=h_np, window=window, n_threads=n_threads,
+                         sfmt=q.sfmt)
     What = orc.dequant(r.codes, r.scales, fmt, block, w_rows, K, sfmt=q.sfmt)
     orc.error_sums(W_bits, What, h_np)
     t2 = time.perf_counter()
@@ -274,12 +283,14 @@ def metric_for(q):
             f"% of roofline")
 
 
-def ops_per_weight(fmt, mode, window, sfmt="e4m3"):
+def ops_per_weight(fmt, mode, window, sfmt="e4m3", block=16):
     """Algorithmic lane-operations per weight of a scale search: C candidates x 6 (quotient,
     projection, dequantise, subtract, h-multiply, square-accumulate; 5 without h) + 4
     (amax, naive quotient, final projection, pack)."""
     full = 126 if sfmt == "e4m3" else 255
     C = 64 if fmt == "e4m3" else (full if window < 0 else 2 * window + 1)
+    if mode == "bhopt":      # quotient, round, dequantise, sign + B FMAs of the form
+        return C * (block + 4) + 4
     return C * (6 if mode == "hopt" else 5) + 4
 
 
@@ -306,19 +317,25 @@ def gpu_arm(args):
     wl = synth.WORKLOADS[args.workload]
     q = quantizer_for(wl, args)
     fmt, block, mode, window = q.fmt, q.block, q.mode, q.window
-    p = mxq.params(fmt, mode, block, window=window, scale_fmt=q.sfmt)
+    bh = mode == "bhopt"
+    if bh and world > 1:
+        raise SystemExit("--mode bhopt runs on one GPU")
+    p = mxq.params(fmt, "hopt" if bh else mode, block, window=window, scale_fmt=q.sfmt)
     # inputs: every rank draws its own shard (weak scaling)
     wl_r = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
     # activations and their h, one per activation width
-    Xs, hs, wss, cols = [], [], [], []
+    Xs, hs, wss, cols, Gs = [], [], [], [], []
     for xi, (R, k) in enumerate(wl.x_shapes):
         R = min(R, args.x_rows) if args.x_rows else R
         X = torch.empty(R, k, dtype=wl.w_dtype, device=dev)
         synth.workload_activations(wl_r, xi, device=dev, rows=R, out=X)
         Xs.append(X)
         hs.append(torch.empty(k, dtype=torch.float32, device=dev))
-        wss.append(torch.empty(mxq.mxq_act_sqmean_workspace(R, k), dtype=torch.uint8, device=dev))
+        wss.append(torch.empty(mxq.mxq_act_block_gram_workspace(R, k, block) if bh else
+                               mxq.mxq_act_sqmean_workspace(R, k), dtype=torch.uint8, device=dev))
         cols.append(torch.empty(k, dtype=torch.float64, device=dev))
+        Gs.append(torch.empty(k // block, block, block, dtype=torch.float32, device=dev)
+                  if bh else None)
     # weights and their outputs (codes, scales, error sums, error workspace, which h)
     Ws, outs = [], []
     for wi, (_, n, k) in enumerate(wl.weights):
@@ -331,14 +348,16 @@ def gpu_arm(args):
     stream = torch.cuda.current_stream(dev)
     # our kernels per step: h pass (2 per activation matrix; 3 with the sharded finalize),
     # search (+ exact fixup for NVFP4 searches), error sums + combine (2) per weight
-    fixup = 1 if fmt == "nvfp4" and mode != "naive" else 0
+    fixup = 1 if mode != "naive" and fmt != "e4m3" else 0
     launches_per_step = len(Xs) * (2 if world == 1 else 3) + len(Ws) * (1 + fixup + 2)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        for X, h, ws, colsum in zip(Xs, hs, wss, cols):
-            if world == 1:
+        for X, h, ws, colsum, G in zip(Xs, hs, wss, cols, Gs):
+            if bh:
+                mxq.mxq_act_block_gram(X, block, G, h, workspace=ws)
+            elif world == 1:
                 mxq.mxq_act_sqmean(X, h, workspace=ws)
             else:
                 # per-rank column sums -> rank-ordered all-gather -> fixed-order finalize
@@ -348,7 +367,10 @@ def gpu_arm(args):
         if ev is not None:
             ev[1].record(stream)
         for W, (codes, scales, _, _, xi) in zip(Ws, outs):
-            mxq.mxq_quantize(W, p, hs[xi], codes=codes, scales=scales)
+            if bh:
+                mxq.mxq_quantize_gram(W, p, Gs[xi], codes=codes, scales=scales)
+            else:
+                mxq.mxq_quantize(W, p, hs[xi], codes=codes, scales=scales)
         if ev is not None:
             ev[2].record(stream)
         for W, (codes, scales, sums, ews, xi) in zip(Ws, outs):
@@ -432,16 +454,27 @@ def gpu_arm(args):
     e2e_ms = t2.item() / args.e2e_steps
     e2e_value = world * weights / (e2e_ms * 1e-3) / 1e9
     metrics = mxq.mxq_metrics_from_sums(oh[0][2])
+    # The pages' output error ||X_s Wq^T - X_s W^T||_F / ||X_s W^T||_F on 512 sampled rows of
+    # X, for the first weight (tensor cores; outside the timed region).
+    out_rel = None
+    if fmt in ("nvfp4", "int4") and Xs[0].dtype == torch.bfloat16:
+        W0, (c0_, s0_, _, _, xi0) = Ws[0], outs[0]
+        rows = synth.sample_rows(Xs[xi0].shape[0], 512, wl.seed + 7).to(dev)
+        Xsmp = Xs[xi0].index_select(0, rows).contiguous()
+        osum = mxq.mxq_output_error(Xsmp, W0, c0_, s0_, p).cpu()
+        out_rel = float((osum[0] / osum[1]).sqrt())
 
     # ---- roofline ------------------------------------------------------------------------
     hbm, hbm_kind = measured_peaks()
     headline = args.workload == "nvfp4_full_calib" and q == HEADLINE_Q and not args.x_rows
-    x_bytes = sum(X.numel() * X.element_size() + 4 * X.shape[1] for X in Xs)
+    x_bytes = sum(X.numel() * X.element_size() + 4 * X.shape[1] * (block if bh else 1)
+                  for X in Xs)
     w_bytes = sum(W.numel() * W.element_size() for W in Ws)
     h_gbs = x_bytes / (k_h * 1e-3) / 1e9
-    kernels = {"act_sqmean": {"ms": k_h, "bound": "hbm", "achieved": h_gbs, "peak": hbm,
-                              "unit": "GB/s", "frac": h_gbs / hbm, "algorithmic_bytes": x_bytes,
-                              "traffic": traffic_for("act_sqmean") if headline else None}}
+    hname = "block_gram" if bh else "act_sqmean"
+    kernels = {hname: {"ms": k_h, "bound": "hbm", "achieved": h_gbs, "peak": hbm,
+                       "unit": "GB/s", "frac": h_gbs / hbm, "algorithmic_bytes": x_bytes,
+                       "traffic": traffic_for("act_sqmean") if headline else None}}
     if mode == "naive":
         q_bytes = w_bytes + weights * code_bytes(fmt, block)
         q_gbs = q_bytes / (k_q * 1e-3) / 1e9
@@ -449,7 +482,7 @@ def gpu_arm(args):
                                "unit": "GB/s", "frac": q_gbs / hbm, "algorithmic_bytes": q_bytes,
                                "traffic": None}
     else:
-        ops = ops_per_weight(fmt, mode, window, q.sfmt) * weights
+        ops = ops_per_weight(fmt, mode, window, q.sfmt, block) * weights
         q_tops = ops / (k_q * 1e-3) / 1e12
         kernels["quantize"] = {"ms": k_q, "bound": "alu", "achieved": q_tops,
                                "peak": ALU_PEAK_TOPS, "unit": "T lane-op/s",
@@ -490,13 +523,14 @@ def gpu_arm(args):
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(),
-            "result": {"weight_rel": metrics["weight_rel"], "h_rel": metrics["h_rel"]}}
+            "result": {"weight_rel": metrics["weight_rel"], "h_rel": metrics["h_rel"],
+                       "output_rel_512_rows": out_rel}}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         X0, W0 = Xs[0], Ws[0]
         R0, n0 = X0.shape[0], W0.shape[0]
         x_rows = min(CPU_X_ROWS, R0)
-        w_rows = min(CPU_W_ROWS // (8 if fmt == "e4m3" else 1), n0)
+        w_rows = min(CPU_W_ROWS // (8 if fmt == "e4m3" or mode == "bhopt" else 1), n0)
         Xb = bits_of(X0[:x_rows].cpu())
         Wb = bits_of(W0[:w_rows].cpu())
         from oracle import oracle as orc

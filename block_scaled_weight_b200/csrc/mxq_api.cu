@@ -202,6 +202,39 @@ mxq_status mxq_act_sqmean_finalize(const double* partials, int64_t parts, int64_
                      "h finalize");
 }
 
+size_t mxq_act_block_gram_workspace(int64_t rows, int64_t cols, int32_t block) {
+  if (rows <= 0 || cols <= 0 || (block != 16 && block != 32)) return 0;
+  return mxq::gram_workspace(rows, cols, block);
+}
+
+mxq_status mxq_act_block_gram(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+                              int64_t ld, int32_t block, float* G, float* h, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (dtype != MXQ_BF16) return fail(MXQ_ERR_DTYPE, "block Gram needs bf16 X (dtype %d)", dtype);
+  mxq_status s = check_matrix(X, dtype, rows, cols, ld, "X");
+  if (s != MXQ_OK) return s;
+  if (block != 16 && block != 32) return fail(MXQ_ERR_UNSUPPORTED, "block %d (16 or 32)", block);
+  if (cols % block != 0) return fail(MXQ_ERR_SHAPE, "cols %% block != 0");
+  if (cols == 0) return MXQ_OK;
+  if (!G) return fail(MXQ_ERR_INVALID_ARG, "G is NULL");
+  if (!aligned(G, 16) || (h && !aligned(h, 4)))
+    return fail(MXQ_ERR_ALIGN, "G not 16-byte or h not 4-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rows == 0) {
+    mxq_status z = cuda_status(cudaMemsetAsync(G, 0, (size_t)cols * block * sizeof(float), st),
+                               "memset G");
+    if (z != MXQ_OK || !h) return z;
+    return cuda_status(cudaMemsetAsync(h, 0, (size_t)cols * sizeof(float), st), "memset h");
+  }
+  if (rows > 0x7fffffff - 64) return fail(MXQ_ERR_SHAPE, "rows beyond 2^31 - 64");
+  const size_t need = mxq::gram_workspace(rows, cols, block);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(MXQ_ERR_ALIGN, "workspace not 16-byte aligned");
+  return cuda_status(mxq::launch_gram(X, rows, cols, ld, block, G, h, workspace, st),
+                     "block Gram");
+}
+
 mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
                         const float* h, const mxq_params* p, void* codes, void* scales,
                         void* stream) {
@@ -240,6 +273,37 @@ mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int6
   return cuda_status(mxq::launch_quantize(a, (cudaStream_t)stream), "quantize");
 }
 
+mxq_status mxq_quantize_gram(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                             const float* G, const mxq_params* p, void* codes, void* scales,
+                             void* stream) {
+  mxq_status s = check_matrix(W, dtype, n, k, ld, "W");
+  if (s != MXQ_OK) return s;
+  s = check_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (p->fmt != MXQ_FMT_NVFP4 && p->fmt != MXQ_FMT_INT4)
+    return fail(MXQ_ERR_UNSUPPORTED, "block-Hessian search: NVFP4 or INT4 elements");
+  if (p->mode != MXQ_HOPT) return fail(MXQ_ERR_INVALID_ARG, "block-Hessian search: mode MXQ_HOPT");
+  if (n == 0 || k == 0) return MXQ_OK;
+  if (!codes || !scales || !G) return fail(MXQ_ERR_INVALID_ARG, "codes, scales or G is NULL");
+  if (!aligned(codes, 16) || !aligned(G, 16))
+    return fail(MXQ_ERR_ALIGN, "codes or G not 16-byte aligned");
+  mxq::QuantArgs a{};
+  a.W = W;
+  a.dtype = dtype;
+  a.n = n;
+  a.k = k;
+  a.ld = ld;
+  a.G = G;
+  a.fmt = p->fmt;
+  a.mode = p->mode;
+  a.block = p->block;
+  a.window = p->window;
+  a.scale_fmt = p->scale_fmt;
+  a.codes = codes;
+  a.scales = scales;
+  return cuda_status(mxq::launch_quantize_gram(a, (cudaStream_t)stream), "quantize (block Hessian)");
+}
+
 mxq_status mxq_project(const float* w, int64_t count, int32_t fmt, int32_t scale_fmt,
                        float scale, uint8_t* q, void* stream) {
   if (count < 0) return fail(MXQ_ERR_SHAPE, "negative count");
@@ -272,6 +336,20 @@ mxq_status mxq_dequant(const void* codes, const void* scales, const mxq_params* 
   return cuda_status(mxq::launch_dequant(d, out, (cudaStream_t)stream), "dequant");
 }
 
+size_t mxq_swizzled_scales_bytes(int64_t n, int64_t kb) {
+  if (n <= 0 || kb <= 0) return 0;
+  return mxq::swizzled_scales_bytes(n, kb);
+}
+
+mxq_status mxq_swizzle_scales(const uint8_t* scales, int64_t n, int64_t kb, uint8_t* out,
+                              void* stream) {
+  if (n < 0 || kb < 0) return fail(MXQ_ERR_SHAPE, "negative shape");
+  if (n == 0 || kb == 0) return MXQ_OK;
+  if (!scales || !out) return fail(MXQ_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(mxq::launch_swizzle_scales(scales, n, kb, out, (cudaStream_t)stream),
+                     "swizzle scales");
+}
+
 size_t mxq_error_workspace(int64_t n, int64_t k) {
   if (n <= 0 || k <= 0) return 0;
   return (size_t)mxq::error_partials(n, k) * 4 * sizeof(double);
@@ -301,6 +379,41 @@ mxq_status mxq_error(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t
   return cuda_status(mxq::launch_error(d, W, dtype, ld, h, (double*)workspace,
                                        mxq::error_partials(n, k), sums, st),
                      "error");
+}
+
+size_t mxq_output_error_workspace(int64_t m, int64_t n) {
+  if (m <= 0 || n <= 0) return 0;
+  return mxq::outerr_workspace(m, n);
+}
+
+mxq_status mxq_output_error(const void* X, int64_t m, int64_t k, int64_t ldx, const void* W,
+                            int64_t n, int64_t ldw, const void* codes, const void* scales,
+                            const mxq_params* p, double* sums, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  mxq_status s = check_matrix(X, MXQ_BF16, m, k, ldx, "X");
+  if (s != MXQ_OK) return s;
+  s = check_matrix(W, MXQ_BF16, n, k, ldw, "W");
+  if (s != MXQ_OK) return s;
+  s = check_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (p->fmt != MXQ_FMT_NVFP4 && p->fmt != MXQ_FMT_INT4)
+    return fail(MXQ_ERR_UNSUPPORTED, "output error: NVFP4 or INT4 codes");
+  if (!sums) return fail(MXQ_ERR_INVALID_ARG, "sums is NULL");
+  if (!aligned(sums, 8)) return fail(MXQ_ERR_ALIGN, "sums not 8-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (m == 0 || n == 0 || k == 0)
+    return cuda_status(cudaMemsetAsync(sums, 0, 2 * sizeof(double), st), "memset");
+  if (!codes || !scales) return fail(MXQ_ERR_INVALID_ARG, "codes or scales is NULL");
+  if (!aligned(codes, 8)) return fail(MXQ_ERR_ALIGN, "codes not 8-byte aligned");
+  if (m > 0x7fffff00 || n > 0x7fffff00) return fail(MXQ_ERR_SHAPE, "rows beyond 2^31");
+  const size_t need = mxq::outerr_workspace(m, n);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(MXQ_ERR_ALIGN, "workspace not 16-byte aligned");
+  return cuda_status(mxq::launch_outerr(X, m, k, ldx, W, n, ldw, (const uint8_t*)codes,
+                                        (const uint8_t*)scales, p->fmt, p->scale_fmt, p->block,
+                                        sums, workspace, st),
+                     "output error");
 }
 
 mxq_status mxq_metrics_from_sums(const double* s, mxq_metrics* out) {

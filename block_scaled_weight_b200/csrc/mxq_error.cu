@@ -261,6 +261,34 @@ int error_partials(int64_t n, int64_t k) {
   return (int)(ctas < 1 ? 1 : ctas);
 }
 
+namespace {
+// One output byte per thread: the 128 x 4 tile layout of sm_100 block-scaled MMA.
+__global__ void k_swizzle_scales(const uint8_t* __restrict__ in, int64_t n, int64_t kb,
+                                 uint8_t* __restrict__ out, int64_t total) {
+  const int64_t ct = (kb + 3) / 4;
+  for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < total;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tile = o / 512, w = o % 512;
+    const int64_t m = (tile / ct) * 128 + (w % 16) / 4 * 32 + w / 16;
+    const int64_t c = (tile % ct) * 4 + (w % 4);
+    out[o] = (m < n && c < kb) ? in[m * kb + c] : (uint8_t)0;
+  }
+}
+}  // namespace
+
+size_t swizzled_scales_bytes(int64_t n, int64_t kb) {
+  return (size_t)((n + 127) / 128) * 128 * (size_t)((kb + 3) / 4) * 4;
+}
+
+cudaError_t launch_swizzle_scales(const uint8_t* in, int64_t n, int64_t kb, uint8_t* out,
+                                  cudaStream_t st) {
+  const int64_t total = (int64_t)swizzled_scales_bytes(n, kb);
+  int64_t grid = (total + 255) / 256;
+  if (grid > 4096) grid = 4096;
+  k_swizzle_scales<<<(unsigned)grid, 256, 0, st>>>(in, n, kb, out, total);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequant(const DecodeArgs& d, float* out, cudaStream_t st) {
   switch (decoder_of(d)) {
     case kDecFp4: return dequant_fmt<kDecFp4>(d, out, st);

@@ -20,12 +20,20 @@ cudaError_t launch_hpass_partial(const void* X, int dtype, int64_t rows, int64_t
 cudaError_t launch_hpass_finalize(const double* partial, int64_t parts, int64_t cols,
                                   int64_t total_rows, double* colsum, float* h, cudaStream_t st);
 
+// ---- Gram blocks (tensor cores) ---------------------------------------------------------
+// G [cols/B][B][B] = fl32(X_b^T X_b / rows) and optionally h = diag(G), for bf16 X.
+int gram_chunks(int64_t rows, int64_t cols);
+size_t gram_workspace(int64_t rows, int64_t cols, int B);
+cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, int B, float* G,
+                        float* h, void* workspace, cudaStream_t st);
+
 // ---- quantization ---------------------------------------------------------------------
 struct QuantArgs {
   const void* W;
   int dtype;
   int64_t n, k, ld;
   const float* h;      // null unless mode == HOPT
+  const float* G;      // Gram blocks [k/B][B][B] for the block-Hessian search
   int fmt, mode, block, window;
   int scale_fmt;       // block-scale grid of NVFP4 / INT4 elements (mxq_grids.h)
   void* codes;
@@ -36,6 +44,8 @@ struct QuantArgs {
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 // E2M1 on a scale grid other than E4M3, and INT4 on any grid (mxq_quant_grid.cu).
 cudaError_t launch_quantize_grid(const QuantArgs& a, cudaStream_t st);
+// Block-Hessian search (d^T G_b d) for E2M1 / INT4 elements on any scale grid.
+cudaError_t launch_quantize_gram(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, uint8_t* q,
                            cudaStream_t st);
 
@@ -48,10 +58,20 @@ struct DecodeArgs {
   int64_t n, k;
 };
 cudaError_t launch_dequant(const DecodeArgs& d, float* out, cudaStream_t st);
+size_t swizzled_scales_bytes(int64_t n, int64_t kb);
+cudaError_t launch_swizzle_scales(const uint8_t* in, int64_t n, int64_t kb, uint8_t* out,
+                                  cudaStream_t st);
 int error_partials(int64_t n, int64_t k);
 cudaError_t launch_error(const DecodeArgs& d, const void* W, int dtype, int64_t ld,
                          const float* h, double* partial, int parts, double* sums,
                          cudaStream_t st);
+
+// ---- output error on the tensor cores (mxq_outerr.cu) ------------------------------------
+size_t outerr_workspace(int64_t m, int64_t n);
+cudaError_t launch_outerr(const void* X, int64_t m, int64_t k, int64_t ldx, const void* W,
+                          int64_t n, int64_t ldw, const uint8_t* codes, const uint8_t* scales,
+                          int fmt, int scale_fmt, int block, double* sums, void* workspace,
+                          cudaStream_t st);
 
 int sm_count();
 // Sets the per-thread text that mxq_last_error() returns.

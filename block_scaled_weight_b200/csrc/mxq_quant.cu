@@ -530,19 +530,47 @@ k_int8_search(Int8Params P, Int8Table T) {
       const float inf = __int_as_float(0x7f800000);
       float m1 = inf, hi1 = inf, l1 = inf, l2 = inf;
       int i1 = lo, j1 = -1;
-      for (int t = 0; t < span; ++t) {
+      auto visit = [&](int cc, float e, float s) {
+        const float del = fmaf(kdel * s, Q, slack);
+        const float elo = fmaf(e, lo_f, -del);
+        if (e < m1) { m1 = e; i1 = cc; hi1 = fmaf(e, hi_f, del); }
+        if (elo < l1) { l2 = l1; l1 = elo; j1 = cc; }
+        else if (elo < l2) l2 = elo;
+      };
+      // Seed: the naive code (clipped to the range), evaluated first.
+      const int cs = min(max(c0, lo), hi);
+      {
+        float e = int8_eval<MODE == 2>(a, c, tab[cs]);
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) e += __shfl_xor_sync(kFull, e, o);
+        visit(cs, e, tab[cs].x);
+      }
+      // Saturation cut: for s <= a_j / 127 every level is at most 127 s, so the definition's
+      // error is at least c_j (a_j - 127 s)^2, which exceeds the seed's upper bound hi1 for
+      // every s below (a_j - sqrt(hi1 / c_j)) / 127; such candidates can neither win nor tie.
+      // The warp starts at the lowest cut among its blocks (candidate loop stays uniform).
+      float s_cut = 0.f;
+      {
+        const float sqt = sqrtf(hi1) * 1.00001f;
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float cx = MODE == 2 ? c[p].x : 1.f, cy = MODE == 2 ? c[p].y : 1.f;
+          if (cx > 0.f) s_cut = fmaxf(s_cut, (-a[p].x - sqt * rsqrtf(cx)) * (1.0f / 127.0f) * 0.99999f);
+          if (cy > 0.f) s_cut = fmaxf(s_cut, (-a[p].y - sqt * rsqrtf(cy)) * (1.0f / 127.0f) * 0.99999f);
+        }
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) s_cut = fmaxf(s_cut, __shfl_xor_sync(kFull, s_cut, o));
+      }
+      int cl = lo;
+      while (cl < hi && tab[cl].x < s_cut) ++cl;
+      const int t0 = __reduce_min_sync(kFull, (unsigned)(cl - lo));
+      for (int t = t0; t < span; ++t) {
         const int cc = lo + t;
         const float4 tb = tab[min(cc, 126)];
         float e = int8_eval<MODE == 2>(a, c, tb);
 #pragma unroll
         for (int o = 1; o < G; o <<= 1) e += __shfl_xor_sync(kFull, e, o);
-        if (cc <= hi) {
-          const float del = fmaf(kdel * tb.x, Q, slack);
-          const float elo = fmaf(e, lo_f, -del);
-          if (e < m1) { m1 = e; i1 = cc; hi1 = fmaf(e, hi_f, del); }
-          if (elo < l1) { l2 = l1; l1 = elo; j1 = cc; }
-          else if (elo < l2) l2 = elo;
-        }
+        if (cc <= hi && cc != cs) visit(cc, e, tb.x);
       }
       flag = !((j1 == i1 ? l2 : l1) > hi1);
       best = i1;
@@ -771,6 +799,7 @@ k_e4m3_tile(TileParams P, LogGrid G) {
         band[p] = sp > 0.0f && !fast;
       }
       __syncthreads();
+      const float del = fmaf(17.0f * 5.9604645e-8f, aw, slack);
       for (int p0 = 0; p0 < P.points; p0 += kTileChunk) {
         float part[kTileChunk];
 #pragma unroll
@@ -800,7 +829,6 @@ k_e4m3_tile(TileParams P, LogGrid G) {
         for (int p = lane; p < P.points; p += 32)
           if (errf[p] < v) { v = errf[p]; vi = p; }
         warp_argmin(v, vi);
-        const float del = fmaf(17.0f * 5.9604645e-8f, aw, slack);
         const float hi1 = fmaf(v, hi_f, del);
         int cnt = 0;
         for (int p = lane; p < P.points; p += 32) {

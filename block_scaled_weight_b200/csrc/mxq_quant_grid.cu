@@ -424,7 +424,307 @@ cudaError_t grid_dispatch(const QuantArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------------
+// Block-Hessian objective: candidate error d^T G_b d with the block's Gram matrix G_b
+// ("quantization_algorithms.txt", sec. 1: the exact output-error objective of a block).
+// A CTA owns one column block b (G_b staged in shared memory) and 256 consecutive rows;
+// thread t quantizes row t's block. Per candidate: signed differences d (as in the grid
+// search), t = G_b d with packed FMAs, e = d . t in float32.
+// Bracket: |e_f - e| <= (B + 4) u sum_ij |G_ij| |d_i| |d_j| (float32 roundings of d, of the
+// B-term products and of the final dot), and sum_ij |G_ij| |d_i||d_j| <= kappa
+// (sum_i sqrt(G_ii) |d_i|)^2 with kappa = max(1, max_ij |G_ij| / sqrt(G_ii G_jj)) computed
+// per block (1 for any Gram matrix; infinite when a diagonal entry is not positive, which
+// sends every block to the exact pass). Flagged blocks are re-scored exactly by
+// k_gram_fixup in the definition's order (e += G_ij * (d_i * d_j), i then j, in double).
+// ---------------------------------------------------------------------------------------
+struct GramSearchParams {
+  const char* W;
+  int64_t n, k, ld_bytes;
+  const float* G;  // [k/B][B][B]
+  int window;
+  uint8_t* codes;
+  uint8_t* scales;
+};
+
+// kappa of one B x B block (see above); +inf when some G_ii <= 0 or a value is not finite.
+template <int B>
+__device__ float gram_kappa(const float* g) {
+  float kap = 1.0f;
+  for (int i = 0; i < B; ++i) {
+    const float gi = g[i * B + i];
+    if (!(gi > 0.0f) || !(gi < __int_as_float(0x7f800000))) return __int_as_float(0x7f800000);
+    for (int j = 0; j < B; ++j) {
+      const float gj = g[j * B + j];
+      if (!(gj > 0.0f)) return __int_as_float(0x7f800000);
+      const float r = fabsf(g[i * B + j]) / sqrtf(gi * gj);
+      if (!(r <= 1e30f)) return __int_as_float(0x7f800000);
+      kap = fmaxf(kap, r);
+    }
+  }
+  return kap * 1.0001f;  // covers the roundings of this estimate
+}
+
+// Signed differences d_j = w_j - sign(w_j) fl32(s g_j) of one candidate, in pairs.
+template <int B, int ELEM>
+__device__ __forceinline__ void gram_diffs(const float2 (&a)[B / 2], uint32_t sgn, float4 t,
+                                           float2 (&d)[B / 2]) {
+  const float2 ns = make_float2(-t.x, -t.x);
+#pragma unroll
+  for (int p = 0; p < B / 2; ++p) {
+    const float2 dd = __ffma2_rn(elem_values<ELEM>(quot2(a[p], t)), ns, a[p]);
+    d[p].x = __uint_as_float(__float_as_uint(dd.x) ^ (((sgn >> (2 * p)) & 1u) << 31));
+    d[p].y = __uint_as_float(__float_as_uint(dd.y) ^ (((sgn >> (2 * p + 1)) & 1u) << 31));
+  }
+}
+
+// A 16-byte shared-memory load the compiler may not hoist out of the candidate loop (G
+// is loop-invariant; kept in registers it would not fit).
+__device__ __forceinline__ float4 lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// Float32 d^T G d and the bracket's sum_i sqrt(G_ii) |d_i| (g: G_b in shared memory,
+// sq: sqrt(G_ii)).
+template <int B>
+__device__ __forceinline__ float gram_form(const float2 (&d)[B / 2], const float* g,
+                                           const float* sq, float& sd) {
+  float e = 0.0f;
+  float2 s2 = make_float2(0.f, 0.f);
+  const uint32_t gbase = (uint32_t)__cvta_generic_to_shared(g);
+#pragma unroll
+  for (int i = 0; i < B; ++i) {
+    float2 t0 = make_float2(0.f, 0.f), t1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < B / 4; ++q) {
+      const float4 gv = lds4(gbase + (uint32_t)((i * B + 4 * q) * 4));
+      t0 = __ffma2_rn(make_float2(gv.x, gv.y), d[2 * q], t0);
+      t1 = __ffma2_rn(make_float2(gv.z, gv.w), d[2 * q + 1], t1);
+    }
+    const float ti = (t0.x + t0.y) + (t1.x + t1.y);
+    const float di = (i & 1) ? d[i / 2].y : d[i / 2].x;
+    e = fmaf(di, ti, e);
+  }
+#pragma unroll
+  for (int p = 0; p < B / 2; p += 2) {
+    const float4 q4 = lds4((uint32_t)__cvta_generic_to_shared(sq) + (uint32_t)(p * 8));
+    s2 = __ffma2_rn(make_float2(q4.x, q4.y), make_float2(fabsf(d[p].x), fabsf(d[p].y)), s2);
+    s2 = __ffma2_rn(make_float2(q4.z, q4.w), make_float2(fabsf(d[p + 1].x), fabsf(d[p + 1].y)), s2);
+  }
+  sd = s2.x + s2.y;
+  return e;
+}
+
+// Double d^T G d in the definition's order.
+template <int B, int ELEM>
+__device__ double gram_exact(const float2 (&a)[B / 2], uint32_t sgn, float4 t, const float* g) {
+  double d[B];
+#pragma unroll
+  for (int p = 0; p < B / 2; ++p) {
+    const float2 v = elem_values<ELEM>(quot2(a[p], t));
+    const float w0 = ((sgn >> (2 * p)) & 1u) ? -a[p].x : a[p].x;
+    const float w1 = ((sgn >> (2 * p + 1)) & 1u) ? -a[p].y : a[p].y;
+    const float q0 = __fmul_rn(t.x, v.x), q1 = __fmul_rn(t.x, v.y);
+    d[2 * p] = (double)w0 - (double)(((sgn >> (2 * p)) & 1u) ? -q0 : q0);
+    d[2 * p + 1] = (double)w1 - (double)(((sgn >> (2 * p + 1)) & 1u) ? -q1 : q1);
+  }
+  double e = 0.0;
+  for (int i = 0; i < B; ++i)
+#pragma unroll
+    for (int j = 0; j < B; ++j) e = __dadd_rn(e, __dmul_rn((double)g[i * B + j], __dmul_rn(d[i], d[j])));
+  return e;
+}
+
+// Pruning (as the diagonal searches, with per-element weights that bound the quadratic
+// form from below): d^T G d >= sum_i cg_i d_i^2 with the Gershgorin weights
+// cg_i = G_ii - sum_{j != i} (|G_ij| + |G_ji|) / 2 (|G_ij d_i d_j| <= |G_ij| (d_i^2 + d_j^2)
+// / 2). Bounds from a subset of elements (the range cuts, the two-element bound) need every
+// cg_i >= 0, i.e. a diagonally dominant G (weakly correlated inputs); otherwise all cg are
+// set to 0 and every candidate is evaluated. With U the smallest upper bracket seen (the
+// seed's first), the saturation and zero range cuts and the two-element bound of
+// k_grid_search apply with cg in place of c; a candidate whose bound exceeds U can neither
+// win nor tie.
+template <int B, bool BF16, int ELEM>
+__global__ void __launch_bounds__(kThreads, 2)
+k_gram_search(GramSearchParams P, GridTable T) {
+  __shared__ float4 tab[256];
+  __shared__ __align__(16) float g[B * B];
+  __shared__ __align__(16) float sq[B];
+  __shared__ float cg[B];
+  __shared__ float kap_s;
+  __shared__ int dominant;
+  for (int i = threadIdx.x; i < 256; i += kThreads) tab[i] = T.c[i];
+  const int64_t kb = P.k / B;
+  const int64_t jb = blockIdx.x;
+  for (int i = threadIdx.x; i < B * B; i += kThreads) g[i] = P.G[jb * B * B + i];
+  if (threadIdx.x == 0) dominant = 1;
+  __syncthreads();
+  if (threadIdx.x < B) {
+    const int i = threadIdx.x;
+    sq[i] = sqrtf(fmaxf(g[i * (B + 1)], 0.0f));
+    double off = 0.0;
+    for (int j = 0; j < B; ++j)
+      if (j != i) off += 0.5 * (fabs((double)g[i * B + j]) + fabs((double)g[j * B + i]));
+    const double w = (double)g[i * (B + 1)] - off;
+    const bool ok = w >= 0.0 && w < 1e38;
+    cg[i] = ok ? __double2float_rd(w * (1.0 - 1e-12)) : 0.0f;
+    if (!ok) dominant = 0;
+  }
+  if (threadIdx.x == 0) kap_s = gram_kappa<B>(g);
+  __syncthreads();
+  if (!dominant && threadIdx.x < B) cg[threadIdx.x] = 0.0f;
+  __syncthreads();
+  constexpr float kQmax = ELEM == kElemE2M1 ? 6.0f : 7.0f;
+  constexpr float kZero = ELEM == kElemE2M1 ? 4.0f : 2.0f;
+  const float kap = kap_s;
+  const int ncodes = T.ncodes, first = T.first, sfmt = T.sfmt;
+  const int elsz = BF16 ? 2 : 4;
+  const float gam = (float)(B + 4) * 5.9604645e-8f * kap;
+  const float slack = 7.3468396e-40f;
+  const float inf = __int_as_float(0x7f800000);
+  const float lb_f = 1.0f - 8.0f * 5.9604645e-8f;
+  for (int64_t row = (int64_t)blockIdx.y * kThreads + threadIdx.x; row < P.n;
+       row += (int64_t)gridDim.y * kThreads) {
+    float2 a[B / 2];
+    uint32_t sgn;
+    load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
+    const int c0 = naive_code<ELEM>(block_amax<B>(a), tab, ncodes, sfmt);
+    int lo, hi;
+    grid_window(tab, ncodes, first, c0, P.window, lo, hi);
+    float m1 = inf, h1 = inf, l1 = inf, l2 = inf, U = inf;
+    int i1 = lo, j1 = -1;
+    auto visit = [&](int cc) {
+      float2 d[B / 2];
+      gram_diffs<B, ELEM>(a, sgn, tab[cc], d);
+      float sd;
+      const float e = gram_form<B>(d, g, sq, sd);
+      const float w = fmaf(gam * sd, sd, slack);
+      const float elo = e - w;
+      if (e < m1) { m1 = e; i1 = cc; h1 = e + w; }
+      if (elo < l1) { l2 = l1; l1 = elo; j1 = cc; }
+      else if (elo < l2) l2 = elo;
+      U = fminf(U, e + w);
+    };
+    const int cs = min(max(c0, lo), hi);
+    visit(cs);
+    float2 at = make_float2(0.f, 0.f), ct = make_float2(0.f, 0.f);
+    if (U < inf) {
+      const float sqt = sqrtf(fmaxf(U, 0.0f)) * 1.00001f;
+      float s_cut = 0.f, s_hi = inf;
+      float v1 = -1.f, a1 = 0.f, c1 = 0.f, v2 = -1.f, a2 = 0.f, c2 = 0.f;
+#pragma unroll
+      for (int p = 0; p < B; ++p) {
+        const float aj = (p & 1) ? a[p / 2].y : a[p / 2].x, cj = cg[p];
+        const float v = cj * aj * aj;
+        if (v > v1) { v2 = v1; a2 = a1; c2 = c1; v1 = v; a1 = aj; c1 = cj; }
+        else if (v > v2) { v2 = v; a2 = aj; c2 = cj; }
+        if (cj > 0.f) {
+          s_cut = fmaxf(s_cut, (aj - sqt * rsqrtf(cj)) * (1.0f / kQmax) * 0.99999f);
+          if (v * 0.99999f - slack > U) s_hi = fminf(s_hi, kZero * aj);
+        }
+      }
+      at = make_float2(a1, a2);
+      ct = make_float2(c1, c2);
+      if (s_cut > 0.f) lo = max(lo, grid_ceil(tab, ncodes, s_cut));
+      if (s_hi < inf) hi = min(hi, grid_ceil(tab, ncodes, s_hi) - 1);
+    }
+    for (int cc = lo; cc <= hi; ++cc) {
+      if (cc == cs) continue;
+      if (grid_lb<ELEM>(at, ct, tab[cc]) * lb_f - slack > U) continue;
+      visit(cc);
+    }
+    const bool flag = !((j1 == i1 ? l2 : l1) > h1);
+    const int64_t b = row * kb + jb;
+    grid_emit<B, ELEM>(a, sgn, tab[i1], P.codes + row * (P.k / 2) + jb * (B / 2));
+    P.scales[b] = (uint8_t)(i1 | (flag ? 0x80 : 0));
+  }
+}
+
+// Exact pass over flagged blocks: one warp per flagged block, lane l scores candidates
+// lo + l + 32 t in double in the definition's order; lowest code on equal values.
+template <int B, bool BF16, int ELEM>
+__global__ void __launch_bounds__(kThreads)
+k_gram_fixup(GramSearchParams P, GridTable T) {
+  __shared__ float4 tab[256];
+  for (int i = threadIdx.x; i < 256; i += kThreads) tab[i] = T.c[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int ncodes = T.ncodes, first = T.first, sfmt = T.sfmt;
+  const int64_t kb = P.k / B, nblocks = P.n * kb;
+  const int elsz = BF16 ? 2 : 4;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t base = gw * 32; base < nblocks; base += nw * 32) {
+    const int64_t mine = base + lane;
+    const bool flagged = mine < nblocks && (P.scales[mine] & 0x80);
+    unsigned todo = __ballot_sync(kFull, flagged);
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int64_t b = base + src;
+      const int64_t row = b / kb, jb = b - row * kb;
+      float2 a[B / 2];
+      uint32_t sgn;
+      load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
+      const float* gb = P.G + jb * B * B;
+      const int c0 = naive_code<ELEM>(block_amax<B>(a), tab, ncodes, sfmt);
+      int lo, hi;
+      grid_window(tab, ncodes, first, c0, P.window, lo, hi);
+      double best = __longlong_as_double(0x7ff0000000000000ll);
+      int bi = 0x7fffffff;
+      for (int cc = lo + lane; cc <= hi; cc += 32) {
+        const double ed = gram_exact<B, ELEM>(a, sgn, tab[cc], gb);
+        if (ed < best) { best = ed; bi = cc; }
+      }
+      warp_argmin(best, bi);
+      if (bi > hi) bi = lo;  // every candidate NaN (non-finite input): keep the first
+      if (lane == 0) {
+        grid_emit<B, ELEM>(a, sgn, tab[bi], P.codes + row * (P.k / 2) + jb * (B / 2));
+        P.scales[b] = (uint8_t)bi;
+      }
+    }
+  }
+}
+
+template <int B, bool BF16, int ELEM>
+cudaError_t gram_dispatch(const QuantArgs& a, cudaStream_t st) {
+  static const GridTable tables[4] = {make_grid_table(0), make_grid_table(1),
+                                      make_grid_table(2), make_grid_table(3)};
+  const GridTable& T = tables[a.scale_fmt];
+  GramSearchParams P{(const char*)a.W, a.n, a.k, a.ld * (BF16 ? 2 : 4), a.G, a.window,
+                     (uint8_t*)a.codes, (uint8_t*)a.scales};
+  const int64_t kb = a.k / B;
+  int64_t ry = (a.n + kThreads - 1) / kThreads;
+  const int64_t target = (int64_t)sm_count() * 8;
+  if (ry * kb > target) ry = (target + kb - 1) / kb;
+  if (ry < 1) ry = 1;
+  if (ry > 65535) ry = 65535;
+  k_gram_search<B, BF16, ELEM><<<dim3((unsigned)kb, (unsigned)ry), kThreads, 0, st>>>(P, T);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t nblocks = a.n * kb;
+  const int64_t fwant = (nblocks + 32 * 8 - 1) / (32 * 8);
+  const int fgrid = (int)(fwant < (int64_t)sm_count() * 8 ? fwant : (int64_t)sm_count() * 8);
+  k_gram_fixup<B, BF16, ELEM><<<fgrid, kThreads, 0, st>>>(P, T);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_gram(const QuantArgs& a, cudaStream_t st) {
+  const bool bf = a.dtype == 1;
+  if (a.fmt == 0) {
+    if (a.block == 16)
+      return bf ? gram_dispatch<16, true, kElemE2M1>(a, st) : gram_dispatch<16, false, kElemE2M1>(a, st);
+    return bf ? gram_dispatch<32, true, kElemE2M1>(a, st) : gram_dispatch<32, false, kElemE2M1>(a, st);
+  }
+  if (a.block == 16)
+    return bf ? gram_dispatch<16, true, kElemInt4>(a, st) : gram_dispatch<16, false, kElemInt4>(a, st);
+  return bf ? gram_dispatch<32, true, kElemInt4>(a, st) : gram_dispatch<32, false, kElemInt4>(a, st);
+}
 
 cudaError_t launch_quantize_grid(const QuantArgs& a, cudaStream_t st) {
   const bool bf = a.dtype == 1;

@@ -31,8 +31,10 @@ MODE = {"naive": 0, "sse": 1, "hopt": 2}
 SCALE = {"e4m3": 0, "ue4m4": 1, "ue5m3": 2, "ue8m0": 3}
 
 EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc",
-           "mxq_act_sqsum",
-           "mxq_act_sqmean_finalize", "mxq_quantize", "mxq_project", "mxq_dequant", "mxq_error_workspace",
+           "mxq_act_sqsum", "mxq_act_block_gram_workspace", "mxq_act_block_gram",
+           "mxq_act_sqmean_finalize", "mxq_quantize", "mxq_quantize_gram", "mxq_project",
+           "mxq_swizzled_scales_bytes", "mxq_swizzle_scales", "mxq_output_error_workspace",
+           "mxq_output_error", "mxq_dequant", "mxq_error_workspace",
            "mxq_error", "mxq_metrics_from_sums", "mxq_status_string", "mxq_last_error")
 
 
@@ -55,9 +57,19 @@ _sig = {
     "mxq_act_sqmean_noalloc": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P]),
     "mxq_act_sqsum": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mxq_act_sqmean_finalize": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
+    "mxq_act_block_gram_workspace": (_SZ, [_I64, _I64, _I32]),
+    "mxq_act_block_gram": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _I32, _P, _P, _P, _SZ,
+                                          _P]),
     "mxq_quantize": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(MxqParams),
                                     _P, _P, _P]),
+    "mxq_quantize_gram": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P,
+                                         ctypes.POINTER(MxqParams), _P, _P, _P]),
     "mxq_project": (ctypes.c_int, [_P, _I64, _I32, _I32, ctypes.c_float, _P, _P]),
+    "mxq_swizzled_scales_bytes": (_SZ, [_I64, _I64]),
+    "mxq_output_error_workspace": (_SZ, [_I64, _I64]),
+    "mxq_output_error": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P,
+                                        ctypes.POINTER(MxqParams), _P, _P, _SZ, _P]),
+    "mxq_swizzle_scales": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "mxq_dequant": (ctypes.c_int, [_P, _P, ctypes.POINTER(MxqParams), _I64, _I64, _P, _P]),
     "mxq_error_workspace": (_SZ, [_I64, _I64]),
     "mxq_error": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
@@ -173,6 +185,27 @@ def mxq_act_sqsum(X: torch.Tensor, colsum: torch.Tensor | None = None, *, worksp
     return colsum
 
 
+def mxq_act_block_gram_workspace(rows: int, cols: int, block: int) -> int:
+    return int(_lib.mxq_act_block_gram_workspace(rows, cols, block))
+
+
+def mxq_act_block_gram(X: torch.Tensor, block: int = 16, G: torch.Tensor | None = None,
+                       h: torch.Tensor | None = None, *, with_h=False, workspace=None,
+                       stream=None):
+    """Gram blocks G [cols/B, B, B] = fl32(X_b^T X_b / R) of bf16 X (tensor cores); with
+    ``with_h`` (or ``h`` given) also h = diag(G). Returns G, or (G, h)."""
+    R, K = X.shape
+    if G is None:
+        G = torch.empty(K // block, block, block, dtype=torch.float32, device=X.device)
+    if with_h and h is None:
+        h = torch.empty(K, dtype=torch.float32, device=X.device)
+    ws = _workspace(mxq_act_block_gram_workspace(R, K, block), X.device, workspace)
+    _check(_lib.mxq_act_block_gram(_ptr(X), _dtype(X), R, K, _ld(X), block, _ptr(G), _ptr(h),
+                                   _ptr(ws), ws.numel(), _stream(stream, X.device)),
+           "mxq_act_block_gram")
+    return (G, h) if h is not None else G
+
+
 def mxq_act_sqmean_finalize(partials: torch.Tensor, total_rows: int,
                             h: torch.Tensor | None = None, *, stream=None) -> torch.Tensor:
     """h from gathered per-shard column sums ``partials`` [parts, cols] (float64)."""
@@ -209,6 +242,21 @@ def mxq_quantize(W: torch.Tensor, p: MxqParams, h: torch.Tensor | None = None, *
     return codes, scales
 
 
+def mxq_quantize_gram(W: torch.Tensor, p: MxqParams, G: torch.Tensor, *, codes=None,
+                      scales=None, stream=None):
+    """(codes, scales) of W [n, k] minimising d^T G_b d per block (G [k/B, B, B] float)."""
+    n, k = W.shape
+    cs, cd, ss, sd = output_shapes(p, n, k)
+    if codes is None:
+        codes = torch.empty(cs, dtype=cd, device=W.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sd, device=W.device)
+    _check(_lib.mxq_quantize_gram(_ptr(W), _dtype(W), n, k, _ld(W), _ptr(G), ctypes.byref(p),
+                                  _ptr(codes), _ptr(scales), _stream(stream, W.device)),
+           "mxq_quantize_gram")
+    return codes, scales
+
+
 def mxq_project(w: torch.Tensor, fmt: str, scale: float, *, scale_fmt="e4m3", q=None,
                 stream=None) -> torch.Tensor:
     """Magnitude codes of float32 ``w`` at one fixed scale (the search's element step);
@@ -219,6 +267,32 @@ def mxq_project(w: torch.Tensor, fmt: str, scale: float, *, scale_fmt="e4m3", q=
     _check(_lib.mxq_project(_ptr(w), w.numel(), FMT[fmt], SCALE[scale_fmt], float(scale),
                             _ptr(q), _stream(stream, w.device)), "mxq_project")
     return q
+
+
+def mxq_output_error(X: torch.Tensor, W: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                     p: MxqParams, *, sums=None, workspace=None, stream=None) -> torch.Tensor:
+    """[sum (X Wq^T - X W^T)^2, sum (X W^T)^2] (float64, device) for bf16 X [m, k], W [n, k]."""
+    m, k = X.shape
+    n = W.shape[0]
+    if sums is None:
+        sums = torch.empty(2, dtype=torch.float64, device=X.device)
+    ws = _workspace(int(_lib.mxq_output_error_workspace(m, n)), X.device, workspace)
+    _check(_lib.mxq_output_error(_ptr(X), m, k, _ld(X), _ptr(W), n, _ld(W), _ptr(codes),
+                                 _ptr(scales), ctypes.byref(p), _ptr(sums), _ptr(ws), ws.numel(),
+                                 _stream(stream, X.device)), "mxq_output_error")
+    return sums
+
+
+def mxq_swizzle_scales(scales: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:
+    """Row-major scale bytes [n, kb] -> the 128 x 4 tile layout of block-scaled MMA (flat)."""
+    scales = scales.contiguous()
+    n, kb = scales.shape
+    if out is None:
+        out = torch.empty(int(_lib.mxq_swizzled_scales_bytes(n, kb)), dtype=torch.uint8,
+                          device=scales.device)
+    _check(_lib.mxq_swizzle_scales(_ptr(scales), n, kb, _ptr(out), _stream(stream, scales.device)),
+           "mxq_swizzle_scales")
+    return out
 
 
 def mxq_dequant(codes: torch.Tensor, scales: torch.Tensor, p: MxqParams, n: int, k: int, *,

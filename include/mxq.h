@@ -171,6 +171,28 @@ MXQ_API mxq_status mxq_act_sqmean_finalize(const double* partials, int64_t parts
                                    int64_t total_rows, float* h, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * Gram blocks of the activations, for the block-Hessian objective: the page's exact
+ * output-error objective of a block, || X_b (W_b - s Q(W_b / s))^T ||_F^2 =
+ * R d^T G_b d per row, with G_b = X_b^T X_b / R ("quantization_algorithms.txt", sec. 1;
+ * h is its diagonal). Computed on the tensor cores from one read of X.
+ *
+ *  X          device bf16 [rows, cols] row-major, leading dimension ld (elements); 16-byte
+ *             aligned, ld * 2 % 16 == 0. (float32 X: MXQ_ERR_DTYPE.)
+ *  block      B = 16 or 32; cols % B == 0.
+ *  G          device float [cols/B][B][B], 16-byte aligned: G[b][i][j] =
+ *             fl32(sum_r x_r,bB+i x_r,bB+j / rows) (the sum: float32 over at most 512 rows
+ *             inside the tensor cores, then double); symmetric to within that rounding.
+ *  h          device float [cols] or NULL: h[c] = G[c/B][c%B][c%B].
+ *  workspace  device, at least mxq_act_block_gram_workspace(rows, cols, block) bytes,
+ *             16-byte aligned.
+ * A launch whose internal waits time out (none does on a working GPU) writes NaN to G and h.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API size_t mxq_act_block_gram_workspace(int64_t rows, int64_t cols, int32_t block);
+MXQ_API mxq_status mxq_act_block_gram(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+                                      int64_t ld, int32_t block, float* G, float* h,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * Scale search and quantization (naive / sse / hopt), fused in one kernel per format.
  *
  *  W       device, [n, k] row-major, leading dimension ld (elements), 16-byte aligned,
@@ -200,6 +222,24 @@ MXQ_API mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t
                         void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * Block-Hessian H-optimal search: the scale minimising d^T G_b d per block (d = w - w^,
+ * G_b the block's Gram matrix from mxq_act_block_gram, or any symmetric B x B matrices),
+ * i.e. the page's output-error objective || X_b d ||^2 / R instead of its diagonal
+ * approximation ("quantization_algorithms.txt", sec. 1).
+ *
+ *  W, codes, scales  as for mxq_quantize; p->fmt MXQ_FMT_NVFP4 or MXQ_FMT_INT4, any
+ *                    p->scale_fmt they accept, p->block 16 or 32, p->mode MXQ_HOPT,
+ *                    p->window as for mxq_quantize.
+ *  G                 device float [k/B][B][B], 16-byte aligned.
+ *  Result: identical to the definition e = sum_i sum_j G_ij (d_i d_j) (double, i then j,
+ *  d_i = (double)w_i - (double)fl32(s q_i) signed), lowest code on ties -- exactly,
+ *  including ties.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API mxq_status mxq_quantize_gram(const void* W, int32_t dtype, int64_t n, int64_t k,
+                                     int64_t ld, const float* G, const mxq_params* p,
+                                     void* codes, void* scales, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * Element projection at one fixed scale -- the per-element step of the search above,
  * exposed so that it can be verified exhaustively.
  *
@@ -227,6 +267,19 @@ MXQ_API mxq_status mxq_dequant(const void* codes, const void* scales, const mxq_
                        int64_t k, float* out, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * Scale bytes for sm_100 block-scaled tensor-core GEMMs. The quantizer writes scales
+ * row-major [n, kb] (kb = k / block); block-scaled MMA instructions (and the libraries
+ * built on them) read them in 128 x 4 tiles of 512 bytes: tiles ordered by row tile, then
+ * column tile; inside a tile, row m and column c at byte (m % 32) * 16 + (m / 32) * 4 + c;
+ * rows padded to a multiple of 128 and columns to a multiple of 4 with zeros. This layout
+ * is the hardware's, not the pages'.
+ *  scales  device uint8 [n, kb]; out  device uint8, mxq_swizzled_scales_bytes(n, kb) bytes.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API size_t mxq_swizzled_scales_bytes(int64_t n, int64_t kb);
+MXQ_API mxq_status mxq_swizzle_scales(const uint8_t* scales, int64_t n, int64_t kb,
+                                      uint8_t* out, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * Weight error (qwantize "Results": ||Q(W) - W||_F / ||W||_F) and the h-weighted error
  * (the diagonal objective, "quantization_algorithms.txt", sec. 1), without materialising
  * the dequantised matrix.
@@ -243,6 +296,25 @@ MXQ_API mxq_status mxq_error(const void* W, int32_t dtype, int64_t n, int64_t k,
                      const mxq_params* p, double* sums, void* workspace,
                      size_t workspace_bytes, void* stream);
 MXQ_API mxq_status mxq_metrics_from_sums(const double* host_sums, mxq_metrics* out);
+
+/* ------------------------------------------------------------------------------------
+ * Output error of a quantized weight (qwantize "Results": ||X_s Wq^T - X_s W^T||_F /
+ * ||X_s W^T||_F on sampled calibration rows X_s), on the tensor cores: both products with
+ * float32 accumulation (bf16 operands; the 4-bit codes are expanded to bf16 exactly), the
+ * squared Frobenius norms summed in double in a fixed order.
+ *  X       device bf16 [m, k], leading dimension ldx; W device bf16 [n, k], ldw; both
+ *          16-byte aligned with ld * 2 % 16 == 0.
+ *  codes, scales, p  the quantized W (p->fmt MXQ_FMT_NVFP4 or MXQ_FMT_INT4, any scale grid
+ *          and block they accept; row-major scales).
+ *  sums    device double [2]: sum (X Wq^T - X W^T)^2, sum (X W^T)^2 (NaN after an internal
+ *          wait timed out, which no working GPU does).
+ *  workspace  mxq_output_error_workspace(m, n) bytes, 16-byte aligned.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API size_t mxq_output_error_workspace(int64_t m, int64_t n);
+MXQ_API mxq_status mxq_output_error(const void* X, int64_t m, int64_t k, int64_t ldx,
+                                    const void* W, int64_t n, int64_t ldw, const void* codes,
+                                    const void* scales, const mxq_params* p, double* sums,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Human-readable text for a status; the last failure's detail on this host thread. */
 MXQ_API const char* mxq_status_string(mxq_status s);

@@ -129,3 +129,10 @@ def test_ue8m0_nan_scale_decodes_to_nan(mxq):
     scales = torch.tensor([[255]], dtype=torch.uint8, device=DEV)
     out = mxq.mxq_dequant(codes, scales, p, 1, 16).cpu()
     assert torch.isnan(out).all()
+
+
+@pytest.mark.parametrize("n,kb", [(300, 10), (128, 4), (2560, 608), (37, 2)])
+def test_swizzle_scales_matches_oracle(mxq, orc, n, kb):
+    s = torch.randint(0, 256, (n, kb), dtype=torch.uint8, device=DEV)
+    out = mxq.mxq_swizzle_scales(s).cpu().numpy()
+    assert np.array_equal(out, orc.swizzle_scales(s.cpu().numpy()))
