@@ -249,38 +249,48 @@ k_outerr_tc(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CU
     const int64_t row = n0 + r;
     const int64_t kb = P.k / P.block;
     bool ok = true;
+    // codes and scales of a stage: fetched one stage ahead, so that the global-load latency
+    // overlaps the expansion of the previous stage
+    auto fetch = [&](int it, uint32_t (&cw)[4], float (&sc)[4]) {
+      const int64_t kk0 = (int64_t)it * kOeK + 32 * hf;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { cw[q] = 0u; sc[q] = 0.0f; }
+      if (it < nk && row < P.n && kk0 < P.k) {
+        const uint2* cp = reinterpret_cast<const uint2*>(P.codes + row * (P.k / 2) + kk0 / 2);
+        const uint2 c0 = __ldg(cp), c1 = (kk0 + 16 < P.k) ? __ldg(cp + 1) : make_uint2(0u, 0u);
+        cw[0] = c0.x; cw[1] = c0.y; cw[2] = c1.x; cw[3] = c1.y;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int64_t e0 = kk0 + 8 * q;
+          sc[q] = e0 < P.k ? stab[__ldg(P.scales + row * kb + e0 / P.block)] : 0.0f;
+        }
+      }
+    };
+    uint32_t cw[4], cwn[4];
+    float sc[4], scn[4];
+    fetch(0, cw, sc);
     for (int it = 0; it < nk; ++it) {
       const int s = it % kOeStages;
+      fetch(it + 1, cwn, scn);
       ok = bar_wait(&empty[s], ((uint32_t)(it / kOeStages) & 1u) ^ 1u, abort_flag);
       if (!__all_sync(kFull, ok)) { ok = false; break; }
       uint32_t wd[16];
-      const int64_t kk0 = (int64_t)it * kOeK + 32 * hf;
-      if (row < P.n && kk0 < P.k) {
-        const uint2* cp = reinterpret_cast<const uint2*>(P.codes + row * (P.k / 2) + kk0 / 2);
-        const uint2 c0 = __ldg(cp), c1 = (kk0 + 16 < P.k) ? __ldg(cp + 1) : make_uint2(0u, 0u);
-        const uint32_t cw[4] = {c0.x, c0.y, c1.x, c1.y};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {         // 8 elements per word
-          const int64_t e0 = kk0 + 8 * q;
-          const float sc = e0 < P.k ? stab[P.scales[row * kb + e0 / P.block]] : 0.0f;
+      for (int q = 0; q < 4; ++q) {           // 8 elements per word
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t byte = (cw[q] >> (8 * u)) & 0xffu;
-            float v0, v1;
-            if (P.int4) {
-              v0 = (float)((int)(byte << 28) >> 28);
-              v1 = (float)((int)(byte << 24) >> 28);
-            } else {
-              const uint32_t h2 = e2m1x2_to_f16x2(byte);
-              v0 = __half2float(__ushort_as_half(lo16(h2)));
-              v1 = __half2float(__ushort_as_half(hi16(h2)));
-            }
-            wd[4 * q + u] = pack_bf16(__fmul_rn(v0, sc), __fmul_rn(v1, sc));
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t byte = (cw[q] >> (8 * u)) & 0xffu;
+          float v0, v1;
+          if (P.int4) {
+            v0 = (float)((int)(byte << 28) >> 28);
+            v1 = (float)((int)(byte << 24) >> 28);
+          } else {
+            const uint32_t h2 = e2m1x2_to_f16x2(byte);
+            v0 = __half2float(__ushort_as_half(lo16(h2)));
+            v1 = __half2float(__ushort_as_half(hi16(h2)));
           }
+          wd[4 * q + u] = pack_bf16(__fmul_rn(v0, sc[q]), __fmul_rn(v1, sc[q]));
         }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 16; ++q) wd[q] = 0u;
       }
       uint8_t* qt = smem + s * kOeStageBytes + kOeXBytes + kOeWBytes + r * 128;
 #pragma unroll
@@ -291,6 +301,8 @@ k_outerr_tc(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CU
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       bar_arrive(&qfull[s]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { cw[q] = cwn[q]; sc[q] = scn[q]; }
     }
     if (!ok && lane == 0) fail();
     // epilogue: this warp's tensor-memory lanes 32 (warp % 4) ..

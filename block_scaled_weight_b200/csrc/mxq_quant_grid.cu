@@ -643,18 +643,28 @@ k_gram_search(GramSearchParams P, GridTable T) {
   }
 }
 
-// Exact pass over flagged blocks: one warp per flagged block, lane l scores candidates
-// lo + l + 32 t in double in the definition's order; lowest code on equal values.
+// Exact pass over flagged blocks: one warp per flagged block. The block's G is staged in
+// the warp's slice of shared memory; lane l evaluates candidates lo + l + 32 t in float32
+// with their brackets (as the search), and only the candidates whose bracket reaches the
+// smallest upper end are scored in double in the definition's order (e += G_ij (d_i d_j),
+// i then j); the warp arg-min (lowest code on equal values) wins.
 template <int B, bool BF16, int ELEM>
 __global__ void __launch_bounds__(kThreads)
 k_gram_fixup(GramSearchParams P, GridTable T) {
+  constexpr int kWarps = kThreads / 32;
   __shared__ float4 tab[256];
+  __shared__ __align__(16) float gw_s[kWarps][B * B];
+  __shared__ __align__(16) float sq_s[kWarps][B];
   for (int i = threadIdx.x; i < 256; i += kThreads) tab[i] = T.c[i];
   __syncthreads();
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  float* g = gw_s[wid];
+  float* sq = sq_s[wid];
   const int ncodes = T.ncodes, first = T.first, sfmt = T.sfmt;
   const int64_t kb = P.k / B, nblocks = P.n * kb;
   const int elsz = BF16 ? 2 : 4;
+  const float slack = 7.3468396e-40f;
+  const float inf = __int_as_float(0x7f800000);
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
   for (int64_t base = gw * 32; base < nblocks; base += nw * 32) {
@@ -670,14 +680,53 @@ k_gram_fixup(GramSearchParams P, GridTable T) {
       uint32_t sgn;
       load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
       const float* gb = P.G + jb * B * B;
+      __syncwarp();
+      for (int i = lane; i < B * B; i += 32) g[i] = gb[i];
+      __syncwarp();
+      // kappa of the block (as gram_kappa), one row per lane
+      float kl = 1.0f;
+      if (lane < B) {
+        const float gi = g[lane * (B + 1)];
+        sq[lane] = sqrtf(fmaxf(gi, 0.0f));
+        if (!(gi > 0.0f) || !(gi < inf)) kl = inf;
+        for (int j = 0; j < B && kl < inf; ++j) {
+          const float gj = g[j * (B + 1)];
+          const float r = (gj > 0.0f) ? fabsf(g[lane * B + j]) / sqrtf(gi * gj) : inf;
+          kl = (r <= 1e30f) ? fmaxf(kl, r) : inf;
+        }
+      }
+      const float kap = warp_max(kl) * 1.0001f;
+      __syncwarp();
+      const float gam = (float)(B + 4) * 5.9604645e-8f * kap;
       const int c0 = naive_code<ELEM>(block_amax<B>(a), tab, ncodes, sfmt);
       int lo, hi;
       grid_window(tab, ncodes, first, c0, P.window, lo, hi);
+      float ef[8], wf[8];
+      float up = inf;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int cc = lo + lane + 32 * t;
+        ef[t] = inf;
+        wf[t] = 0.f;
+        if (cc <= hi) {
+          float2 d[B / 2];
+          gram_diffs<B, ELEM>(a, sgn, tab[cc], d);
+          float sd;
+          ef[t] = gram_form<B>(d, g, sq, sd);
+          wf[t] = fmaf(gam * sd, sd, slack);
+          up = fminf(up, ef[t] + wf[t]);
+        }
+      }
+      up = warp_min(up);
       double best = __longlong_as_double(0x7ff0000000000000ll);
       int bi = 0x7fffffff;
-      for (int cc = lo + lane; cc <= hi; cc += 32) {
-        const double ed = gram_exact<B, ELEM>(a, sgn, tab[cc], gb);
-        if (ed < best) { best = ed; bi = cc; }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int cc = lo + lane + 32 * t;
+        if (cc <= hi && !(ef[t] - wf[t] > up)) {
+          const double ed = gram_exact<B, ELEM>(a, sgn, tab[cc], gb);
+          if (ed < best || (ed == best && cc < bi)) { best = ed; bi = cc; }
+        }
       }
       warp_argmin(best, bi);
       if (bi > hi) bi = lo;  // every candidate NaN (non-finite input): keep the first

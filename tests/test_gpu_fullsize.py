@@ -33,14 +33,14 @@ def synth():
     return s
 
 
-def sampled_parity(mxq, orc, W, fmt, block, mode, h_np, window, rows, tag):
+def sampled_parity(mxq, orc, W, fmt, block, mode, h_np, window, rows, tag, sfmt="e4m3"):
     """Quantize all of W on the GPU; compare `rows` with the oracle; return near-tie count."""
-    p = mxq.params(fmt, mode, block, window=window)
+    p = mxq.params(fmt, mode, block, window=window, scale_fmt=sfmt)
     hd = None if h_np is None else torch.from_numpy(h_np).to(DEV)
     codes, scales = mxq.mxq_quantize(W, p, hd)
     torch.cuda.synchronize()
     Ws = oracle_view(W[torch.as_tensor(rows, device=W.device)])
-    r = orc.quantize(Ws, fmt, mode, block, h=h_np, window=window, n_threads=NT)
+    r = orc.quantize(Ws, fmt, mode, block, h=h_np, window=window, n_threads=NT, sfmt=sfmt)
     if fmt == "e4m3":
         raise AssertionError("use tile_parity for e4m3")
     g_codes = codes[torch.as_tensor(rows, device=W.device)].cpu().numpy().view(np.uint8)
@@ -154,3 +154,35 @@ def test_decoder_layer_back_to_back(mxq, orc, synth):
         ri = torch.as_tensor(rows, device=DEV)
         assert np.array_equal(scales[ri].cpu().numpy(), r.scales), name
         assert np.array_equal(codes[ri].cpu().numpy(), r.codes), name
+
+
+@pytest.mark.parametrize("fmt,sfmt,block", [("nvfp4", "ue8m0", 32), ("int4", "e4m3", 16),
+                                            ("nvfp4", "ue4m4", 16)])
+def test_scale_grids_full_size(mxq, orc, synth, fmt, sfmt, block):
+    """MXFP4, NVINT4 and E2M1-on-UE4M4 on the full-calibration weight (2560 x 9728), H-opt
+    over the whole grid, with h from 32768 rows of the full-calibration activations."""
+    wl = synth.WORKLOADS["nvfp4_full_calib"]
+    W = synth.workload_weight(wl, 0, device=DEV)
+    X = synth.workload_activations(wl, 0, device="cpu", rows=32768)
+    h = orc.act_sqmean(oracle_view(X), n_threads=NT)
+    rows = synth.sample_rows(W.shape[0], 24, wl.seed + 31).tolist()
+    near, tot = sampled_parity(mxq, orc, W, fmt, block, "hopt", h, -1, rows,
+                               f"{fmt}/{sfmt} bs{block}", sfmt=sfmt)
+    print(f"{fmt}/{sfmt} bs{block}: {tot} sampled blocks bit-exact, {near} near ties")
+
+
+def test_block_hessian_full_size(mxq, orc, synth):
+    """Block-Hessian NVFP4 bs16 on the full-calibration weight with the oracle's Gram blocks
+    of 16384 activation rows (uploaded): sampled rows bit-exact."""
+    wl = synth.WORKLOADS["nvfp4_full_calib"]
+    W = synth.workload_weight(wl, 0, device=DEV)
+    X = synth.workload_activations(wl, 0, device="cpu", rows=16384)
+    G = orc.block_gram(oracle_view(X), 16)
+    p = mxq.params("nvfp4", "hopt", 16)
+    codes, scales = mxq.mxq_quantize_gram(W, p, torch.from_numpy(G).to(DEV))
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(W.shape[0], 8, wl.seed + 41).tolist()
+    ri = torch.as_tensor(rows, device=DEV)
+    r = orc.quantize_gram(oracle_view(W[ri]), "nvfp4", 16, G, n_threads=NT)
+    assert np.array_equal(scales[ri].cpu().numpy(), r.scales)
+    assert np.array_equal(codes[ri].cpu().numpy(), r.codes)
