@@ -600,6 +600,53 @@ int orc_quantize_tiles(const void *W, int dtype, int64_t n, int64_t k, int64_t l
 }
 
 /* ----------------------------------------------------------------------------------
+ * FP8-GPTQ on 64 x 64 tiles ("quantization_algorithms.txt", section 1, "For a 64x64 tile
+ * scheme": fix or search the tile scale, H = X^T X + lambda I over the tile's 64 input
+ * dimensions, quantise the columns sequentially to E4M3, propagate each quantisation
+ * residual through H^-1). The propagation is GPTQ's (Frantar et al. 2022) in its Cholesky
+ * form: with U the upper Cholesky factor of H^-1 (H^-1 = U^T U), after column i
+ *     err_r = (w_ri - q_ri) / U_ii,   w_rj -= err_r * U_ij   for j > i,
+ * every step a separately rounded float32 operation (division, product, difference).
+ * U [k/64][64][64] (float32, upper triangular; computed by the Python front end from the
+ * Gram blocks) and the tile scales [n/64][k/64] are inputs. codes as orc_quantize_tiles;
+ * W_prop (optional) receives the propagated weights at the moment each column was
+ * quantised.
+ * ---------------------------------------------------------------------------------- */
+int orc_gptq_tiles(const void *W, int dtype, int64_t n, int64_t k, int64_t ld, const float *U,
+                   const float *scales, uint8_t *codes, float *W_prop)
+{
+    const int T = 64;
+    if (n % T != 0 || k % T != 0 || U == NULL || scales == NULL) return -1;
+    int64_t tn = n / T, tk = k / T;
+    float *w = (float *)malloc(sizeof(float) * T * T);
+    for (int64_t ti = 0; ti < tn; ++ti)
+        for (int64_t tj = 0; tj < tk; ++tj) {
+            const float *Ub = U + tj * T * T;
+            float s = scales[ti * tk + tj];
+            for (int i = 0; i < T; ++i)
+                for (int j = 0; j < T; ++j)
+                    w[i * T + j] = elem(W, dtype, ld, ti * T + i, tj * T + j);
+            for (int c = 0; c < T; ++c) {            /* column c, every row r of the tile */
+                for (int r = 0; r < T; ++r) {
+                    float wv = w[r * T + c];
+                    float wq_abs;
+                    int q = e4m3_elem_code(fabsf(wv), s, &wq_abs);
+                    float wq = copysignf(wq_abs, wv);
+                    codes[(ti * T + r) * k + tj * T + c] = (uint8_t)((signbit(wv) ? 0x80 : 0) | q);
+                    if (W_prop) W_prop[(ti * T + r) * k + tj * T + c] = wv;
+                    float err = (wv - wq) / Ub[c * T + c];
+                    for (int j = c + 1; j < T; ++j) {
+                        float prod = err * Ub[c * T + j];
+                        w[r * T + j] = w[r * T + j] - prod;
+                    }
+                }
+            }
+        }
+    free(w);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------------------
  * Dequantisation and error metrics (qwantize "Results": weight error
  * ||Q(W) - W||_F / ||W||_F; the h-weighted error is the diagonal objective itself).
  * ---------------------------------------------------------------------------------- */

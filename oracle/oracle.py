@@ -82,6 +82,8 @@ def lib():
             L.orc_quantize_blocks_gram.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I,
                                                    _I64, _I64, _P, _P, _P, _P, _P]
             L.orc_swizzle_scales.argtypes = [_P, _I64, _I64, _P]
+            L.orc_gptq_tiles.restype = _I
+            L.orc_gptq_tiles.argtypes = [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P]
             L.orc_log_grid.argtypes = [_I, _D, _D, _P]
             L.orc_quantize_tiles.restype = _I
             L.orc_quantize_tiles.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _D, _D,
@@ -340,6 +342,36 @@ def dequant(codes, scales, fmt: str, block: int, n: int, k: int,
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out
+
+
+def gptq_prepare(G, damp: float = 0.01) -> np.ndarray:
+    """U [k/64, 64, 64] float32 for FP8-GPTQ on 64 x 64 tiles ("quantization_algorithms.txt",
+    sec. 1): per column block H = G + lambda I with lambda = damp * mean(diag G) (1 when that
+    mean is 0 -- an all-zero block), H^-1, and U its upper Cholesky factor (H^-1 = U^T U),
+    all in float64, rounded to float32 once. G: the Gram blocks (block_gram(X, 64))."""
+    G = np.asarray(G, dtype=np.float64)
+    U = np.zeros(G.shape, np.float32)
+    for b in range(G.shape[0]):
+        lam = damp * float(np.mean(np.diag(G[b])))
+        H = G[b] + (lam if lam > 0 else 1.0) * np.eye(G.shape[1])
+        Hinv = np.linalg.inv(H)
+        U[b] = np.linalg.cholesky((Hinv + Hinv.T) / 2).T.astype(np.float32)
+    return U
+
+
+def gptq_tiles(W, U, scales, want_prop=False):
+    """E4M3 codes [n, k] of the tile GPTQ sweep with fixed tile scales; optionally the
+    propagated weights (float32 [n, k]) at the moment each column was quantised."""
+    W, dt = _as_input(W)
+    n, k = W.shape
+    U = np.ascontiguousarray(U, dtype=np.float32)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    codes = np.zeros((n, k), np.uint8)
+    prop = np.zeros((n, k), np.float32) if want_prop else None
+    if lib().orc_gptq_tiles(_ptr(W), dt, n, k, k, _ptr(U), _ptr(scales), _ptr(codes),
+                            _ptr(prop)) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return (codes, prop) if want_prop else codes
 
 
 def swizzle_scales(scales) -> np.ndarray:

@@ -50,6 +50,9 @@ MUTANTS = {
                            "            e += (i == j) ? (double)Gb[i * B + j] * (d[i] * d[j]) : 0.0;"),
     "gram_unsigned_difference": ("d[j] = (double)w[j] - (double)copysignf(wq_abs, w[j]);",
                                  "d[j] = (double)fabsf(w[j]) - (double)wq_abs;"),
+    "gptq_no_division": ("float err = (wv - wq) / Ub[c * T + c];", "float err = (wv - wq);"),
+    "gptq_wrong_sign": ("w[r * T + j] = w[r * T + j] - prod;", "w[r * T + j] = w[r * T + j] + prod;"),
+    "gptq_transposed_factor": ("float prod = err * Ub[c * T + j];", "float prod = err * Ub[j * T + c];"),
     "dequant_not_rounded": ("float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - (double)wq;",
                             "float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - 1.0000001 * (double)wq;"),
 }
@@ -69,6 +72,7 @@ def test_planted_mistake_is_caught(name, tmp_path):
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                           os.path.join(HERE, "test_oracle_pins.py"),
                           os.path.join(HERE, "test_oracle_pins_scales.py"),
-                          os.path.join(HERE, "test_oracle_pins_gram.py")], cwd=ROOT, env=env,
+                          os.path.join(HERE, "test_oracle_pins_gram.py"),
+                          os.path.join(HERE, "test_oracle_pins_gptq.py")], cwd=ROOT, env=env,
                          capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"pins did not catch planted mistake {name}:\n{res.stdout[-2000:]}"
