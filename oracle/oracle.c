@@ -350,6 +350,32 @@ static void emit_block(int fmt, int sfmt, int c, const float *w, int B, uint8_t 
     }
 }
 
+/* The quantizer's pick for one block of B weights w with error weights cw: the naive
+ * code in naive mode, else the candidate of smallest error, the lowest code on equal
+ * errors. e1 / e2: the smallest and second-smallest candidate errors (NaN in naive mode);
+ * naive: the naive code. */
+static int search_block(int fmt, int sfmt, int mode, int window, const scale_grid *g,
+                        const float *w, const float *cw, int B, double *e1, double *e2,
+                        int *naive)
+{
+    float amax = 0.0f;
+    for (int j = 0; j < B; ++j)
+        if (fabsf(w[j]) > amax) amax = fabsf(w[j]);
+    int c0 = naive_code(fmt, sfmt, amax);
+    int cbest = c0;
+    *e1 = NAN;
+    *e2 = NAN;
+    if (mode != ORC_NAIVE) {
+        int lo, hi;
+        candidate_range(g, c0, window, &lo, &hi);
+        *e1 = INFINITY; *e2 = INFINITY; cbest = lo;
+        for (int c = lo; c <= hi; ++c)
+            keep_best(block_error(fmt, sfmt, c, w, cw, B), c, e1, e2, &cbest);
+    }
+    *naive = c0;
+    return cbest;
+}
+
 /*
  * Quantize rows [row0, row1) of W [n, k] (leading dimension ld) in blocks of B along k.
  * fmt: ORC_NVFP4 (E2M1 elements), ORC_INT4 or ORC_INT8; sfmt: the scale grid
@@ -382,22 +408,13 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
     for (int64_t i = row0; i < row1 && i < n; ++i) {
         for (int64_t b = 0; b < kb; ++b) {
             int64_t j0 = b * B;
-            float amax = 0.0f;
             for (int j = 0; j < B; ++j) {
                 w[j] = elem(W, dtype, ld, i, j0 + j);
                 cw[j] = (mode == ORC_HOPT) ? h[j0 + j] : 1.0f;
-                if (fabsf(w[j]) > amax) amax = fabsf(w[j]);
             }
-            int c0 = naive_code(fmt, sfmt, amax);
-            int cbest = c0;
-            double e1 = NAN, e2 = NAN;
-            if (mode != ORC_NAIVE) {
-                int lo, hi;
-                candidate_range(&g, c0, window, &lo, &hi);
-                e1 = INFINITY; e2 = INFINITY; cbest = lo;
-                for (int c = lo; c <= hi; ++c)
-                    keep_best(block_error(fmt, sfmt, c, w, cw, B), c, &e1, &e2, &cbest);
-            }
+            double e1, e2;
+            int c0;
+            int cbest = search_block(fmt, sfmt, mode, window, &g, w, cw, B, &e1, &e2, &c0);
             scales[i * kb + b] = (uint8_t)cbest;
             if (best) best[i * kb + b] = e1;
             if (second) second[i * kb + b] = e2;
@@ -407,6 +424,74 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
     }
     free(w);
     free(cw);
+    return 0;
+}
+
+/* ----------------------------------------------------------------------------------
+ * GPTQ with the block quantizer as its inner step (qwantize "Results", "GPTQ
+ * Quantization": the GPTQ block is the quantization block, each block's quantization
+ * error is compensated in all later columns through the inverse Hessian; the algorithm is
+ * Frantar et al. 2022, Algorithm 1, in its Cholesky form). When the sweep reaches a block,
+ * its scale is the quantizer's pick (naive / SSE / H-optimal, as orc_quantize_blocks) for
+ * the block's CURRENT weights -- GPTQ fixes a group's quantization grid at the moment the
+ * group is reached -- and the block's columns are then quantised one after another at that
+ * scale, each residual propagated at once. Rows are independent; for row i, with the
+ * block visited at sweep position t being perm[t] (t itself when perm is NULL) and the
+ * sweep position of column col = b B + j being p = t B + j:
+ *     q = project(w_col at the block's scale), wq = +-fl32(s q) (the sign of w_col),
+ *     err = (w_col - wq) / U[p][p],
+ *     w at every later position p' -= err * U[p][p']
+ * every step a separately rounded float32 operation. U [k][k] (float32, upper triangular)
+ * is the upper Cholesky factor of the damped H^-1 with H's rows and columns in sweep order
+ * (positions). codes / scales: the layouts of orc_quantize_blocks; rows [row0, row1).
+ * ---------------------------------------------------------------------------------- */
+int orc_gptq_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
+                    const float *h, int fmt, int sfmt, int mode, int B, int window,
+                    const float *U, const int32_t *perm, int64_t row0, int64_t row1,
+                    uint8_t *codes, uint8_t *scales)
+{
+    scale_grid g;
+    if (B <= 0 || k % B != 0 || U == NULL || grid_of(sfmt, &g)) return -1;
+    if (fmt != ORC_NVFP4 && fmt != ORC_INT8 && fmt != ORC_INT4) return -1;
+    if (fmt == ORC_INT8 && sfmt != ORC_S_E4M3) return -1;
+    if (fmt == ORC_INT4 && sfmt == ORC_S_UE8M0) return -1;
+    if (mode == ORC_HOPT && h == NULL) return -1;
+    int64_t kb = k / B;
+    int64_t *col = (int64_t *)malloc(sizeof(int64_t) * (size_t)k);   /* position -> column */
+    for (int64_t t = 0; t < kb; ++t) {
+        int64_t b = perm ? perm[t] : t;
+        if (b < 0 || b >= kb) { free(col); return -1; }
+        for (int j = 0; j < B; ++j) col[t * B + j] = b * B + j;
+    }
+    float *w = (float *)malloc(sizeof(float) * (size_t)k);
+    float *cw = (float *)malloc(sizeof(float) * (size_t)B);
+    for (int64_t i = row0; i < row1 && i < n; ++i) {
+        for (int64_t j = 0; j < k; ++j) w[j] = elem(W, dtype, ld, i, j);
+        for (int64_t t = 0; t < kb; ++t) {
+            int64_t j0 = col[t * B];                 /* the block's first column */
+            for (int j = 0; j < B; ++j) cw[j] = (mode == ORC_HOPT) ? h[j0 + j] : 1.0f;
+            double e1, e2;
+            int c0;
+            int c = search_block(fmt, sfmt, mode, window, &g, &w[j0], cw, B, &e1, &e2, &c0);
+            scales[i * kb + j0 / B] = (uint8_t)c;
+            for (int j = 0; j < B; ++j) {
+                int64_t p = t * B + j;
+                float wv = w[j0 + j];
+                float wq_abs;
+                project(fmt, sfmt, c, wv, &wq_abs);
+                emit_block(fmt, sfmt, c, &w[j0 + j], 1, codes, i, j0 + j, k);
+                float wq = copysignf(wq_abs, wv);
+                float err = (wv - wq) / U[p * k + p];
+                for (int64_t p2 = p + 1; p2 < k; ++p2) {
+                    float prod = err * U[p * k + p2];
+                    w[col[p2]] = w[col[p2]] - prod;
+                }
+            }
+        }
+    }
+    free(w);
+    free(cw);
+    free(col);
     return 0;
 }
 

@@ -82,6 +82,9 @@ def lib():
             L.orc_quantize_blocks_gram.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I,
                                                    _I64, _I64, _P, _P, _P, _P, _P]
             L.orc_swizzle_scales.argtypes = [_P, _I64, _I64, _P]
+            L.orc_gptq_blocks.restype = _I
+            L.orc_gptq_blocks.argtypes = [_P, _I, _I64, _I64, _I64, _P, _I, _I, _I, _I, _I, _P,
+                                          _P, _I64, _I64, _P, _P]
             L.orc_gptq_tiles.restype = _I
             L.orc_gptq_tiles.argtypes = [_P, _I, _I64, _I64, _I64, _P, _P, _P, _P]
             L.orc_log_grid.argtypes = [_I, _D, _D, _P]
@@ -372,6 +375,84 @@ def gptq_tiles(W, U, scales, want_prop=False):
                             _ptr(prop)) != 0:
         raise ValueError("oracle rejected the arguments")
     return (codes, prop) if want_prop else codes
+
+
+def gram(X) -> np.ndarray:
+    """The full K x K Gram matrix H = fl32(X^T X / R) of X [R, K] (float64 product)."""
+    Xf = to_float(X).astype(np.float64)
+    R = Xf.shape[0]
+    return (Xf.T @ Xf / R).astype(np.float32) if R else np.zeros((Xf.shape[1],) * 2, np.float32)
+
+
+def block_losses(W, h, fmt: str, mode: str, block: int, *, sfmt: str = "e4m3",
+                 window: int = -1) -> np.ndarray:
+    """Hessian-weighted quantization loss of each column block: sum over rows and the
+    block's columns of h_j (w_ij - w^_ij)^2 (float64, rows ascending) for the block
+    quantizer's own (uncompensated) result."""
+    W, _ = _as_input(W)
+    n, k = W.shape
+    r = quantize(W, fmt, mode, block, h=h if mode == "hopt" else None, window=window,
+                 sfmt=sfmt)
+    What = dequant(r.codes, r.scales, fmt, block, n, k, sfmt=sfmt).astype(np.float64)
+    d = to_float(W).astype(np.float64) - What
+    e = (d * d) * np.asarray(h, np.float64)[None, :]
+    loss = np.zeros(k // block)
+    for b in range(k // block):
+        for i in range(n):
+            loss[b] += float(np.sum(e[i, b * block:(b + 1) * block]))
+    return loss
+
+
+def block_order(losses) -> np.ndarray:
+    """Ordered GPTQ's block sequence: descending loss, the lower block first on equal loss."""
+    losses = np.asarray(losses, np.float64)
+    return np.array(sorted(range(len(losses)), key=lambda b: (-losses[b], b)), np.int32)
+
+
+def gptq_blocks(W, U, h, fmt: str, mode: str, block: int, *, sfmt: str = "e4m3",
+                window: int = -1, perm=None, rows=None, n_threads=1) -> Result:
+    """GPTQ with the block quantizer as its inner step (orc_gptq_blocks): codes and scales
+    in the layouts of ``quantize``. U [k, k]: the factor of the damped H^-1 in sweep order;
+    perm: the block visited at each sweep position (None: natural order)."""
+    W, dt = _as_input(W)
+    n, k = W.shape
+    f, m = FMTS[fmt], MODES[mode]
+    if f == E4M3:
+        raise ValueError("E4M3 elements: gptq_tiles")
+    hp = None if h is None else np.ascontiguousarray(h, dtype=np.float32)
+    if m == HOPT and hp is None:
+        raise ValueError("H-optimal needs h")
+    U = np.ascontiguousarray(U, dtype=np.float32)
+    pp = None if perm is None else np.ascontiguousarray(perm, dtype=np.int32)
+    codes = np.zeros((n, k // 2) if f in (NVFP4, INT4) else (n, k), np.uint8)
+    scales = np.zeros((n, k // block), np.uint8)
+    r0, r1 = (0, n) if rows is None else rows
+
+    def run(a, b):
+        if lib().orc_gptq_blocks(_ptr(W), dt, n, k, k, _ptr(hp), f, SFMTS[sfmt], m, block,
+                                 window, _ptr(U), _ptr(pp), a, b, _ptr(codes),
+                                 _ptr(scales)) != 0:
+            raise ValueError("oracle rejected the arguments")
+    _run_ranges(run, r0, r1, _threads(n_threads))
+    return Result(codes=codes, scales=scales, best=None, second=None, naive=None)
+
+
+def gptq(W, H, h, fmt: str, mode: str, block: int, *, ordered: bool = False,
+         damp: float = 0.01, sfmt: str = "e4m3", window: int = -1, rows=None,
+         n_threads=1) -> Result:
+    """Sequential (natural block order) or ordered (descending block loss) GPTQ of W [n, k]
+    with Hessian H [k, k] (e.g. gram(X)) and h = diag(H) for the H-optimal search. Returns
+    codes and scales in the original column order; ``naive`` holds the block order used."""
+    k = np.asarray(H).shape[0]
+    perm = block_order(block_losses(W, h, fmt, mode, block, sfmt=sfmt, window=window)) \
+        if ordered else np.arange(k // block, dtype=np.int32)
+    cols = (perm[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+    Hp = np.asarray(H, np.float32)[np.ix_(cols, cols)]
+    U = gptq_prepare(Hp[None], damp)[0]
+    r = gptq_blocks(W, U, h, fmt, mode, block, sfmt=sfmt, window=window,
+                    perm=perm if ordered else None, rows=rows, n_threads=n_threads)
+    r["naive"] = perm
+    return r
 
 
 def swizzle_scales(scales) -> np.ndarray:

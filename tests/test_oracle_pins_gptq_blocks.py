@@ -1,0 +1,138 @@
+"""Pins of the oracle's GPTQ with the block quantizer as its inner step (qwantize "Results",
+"GPTQ Quantization": the GPTQ block is the quantization block; sequential and ordered
+variants; Frantar et al. 2022, Algorithm 1, in its Cholesky form).
+
+Checks: a hand-derived worked example in which the propagated residual changes the next
+block's scale, the reduction to the plain quantizer when nothing propagates, the ordered
+variant against a physical permutation of the columns, the block losses against their
+definition, and the output-error improvement GPTQ exists for.
+"""
+import numpy as np
+import pytest
+
+
+def worked(sign=1.0, u00=1.0):
+    k = 32
+    W = np.zeros((1, k), np.float32)
+    W[0, [0, 1, 2, 16]] = np.array([1.25, 5.0625, 6.0, 5.0], np.float32) * sign
+    U = np.eye(k, dtype=np.float32)
+    U[0, 0], U[0, 1], U[0, 16] = u00, 0.5, 4.0
+    return W, U, np.ones(k, np.float32)
+
+
+@pytest.mark.parametrize("u00,scale1", [(1.0, 0x33), (2.0, 0x34)])
+def test_worked_example(orc, u00, scale1):
+    """NVFP4 block 16, naive scales. Block 0: amax 6 gives scale E4M3(6 / 6) = 1.0 (0x38);
+    w0 = 1.25 is the midpoint of E2M1 1.0 (code 2) and 1.5 (code 3), ties to the even code
+    2; err = 0.25 / U_00.
+    U_00 = 1: err = 0.25 moves w1 to 5.0625 - 0.25 * 0.5 = 4.9375, below the E2M1 midpoint
+    5, so code 6 (4.0) where the plain quantizer gives code 7 (6.0); w16 becomes
+    5 - 0.25 * 4 = 4, and block 1 is reached with amax 4: scale E4M3(4 / 6 = 0.667) = 0.6875
+    (0x33), 4 / 0.6875 = 5.82 rounds to E2M1 6 (code 7).
+    U_00 = 2: err = 0.125; w1 = 5.0 exactly, the midpoint, ties to the even code 6; w16 =
+    4.5, scale E4M3(0.75) = 0x34, 4.5 / 0.75 = 6 (code 7).
+    Without GPTQ block 1's scale is E4M3(5 / 6 = 0.833) = 0.8125 (0x35)."""
+    W, U, h = worked(u00=u00)
+    r = orc.gptq_blocks(W, U, h, "nvfp4", "naive", 16)
+    assert r.scales[0].tolist() == [0x38, scale1]
+    assert r.codes[0, 0] == 0x62 and r.codes[0, 1] == 0x07 and r.codes[0, 8] == 0x07
+    assert np.all(np.delete(r.codes[0], [0, 1, 8]) == 0)
+    p = orc.quantize(W, "nvfp4", "naive", 16)
+    assert p.scales[0].tolist() == [0x38, 0x35] and p.codes[0, 0] == 0x72
+
+
+def test_worked_example_negative(orc):
+    """The mirror image: the same scales, sign bits set (nibbles 0xA, 0xE, 0xF)."""
+    W, U, h = worked(-1.0)
+    r = orc.gptq_blocks(W, U, h, "nvfp4", "naive", 16)
+    assert r.scales[0].tolist() == [0x38, 0x33]
+    assert r.codes[0, 0] == 0xEA and r.codes[0, 1] == 0x0F and r.codes[0, 8] == 0x0F
+
+
+@pytest.mark.parametrize("fmt,sfmt,block", [("nvfp4", "e4m3", 16), ("nvfp4", "ue8m0", 32),
+                                            ("int4", "e4m3", 16), ("int8", "e4m3", 32)])
+@pytest.mark.parametrize("mode", ["naive", "sse", "hopt"])
+def test_diagonal_factor_is_plain_quantization(orc, fmt, sfmt, block, mode):
+    """A diagonal U propagates nothing (products with +0 leave nonzero weights alone), so
+    every scale and code is the plain quantizer's (weights without exact zeros)."""
+    rng = np.random.default_rng(11)
+    n, k = 7, 4 * block
+    W = (rng.standard_t(4, (n, k)) * 0.05).astype(np.float32)
+    W[W == 0] = 1e-3
+    h = np.exp(rng.normal(0, 1, k)).astype(np.float32)
+    U = np.diag(rng.uniform(0.5, 2.0, k)).astype(np.float32)
+    r = orc.gptq_blocks(W, U, h, fmt, mode, block, sfmt=sfmt)
+    p = orc.quantize(W, fmt, mode, block, h=h if mode == "hopt" else None, sfmt=sfmt)
+    assert np.array_equal(r.scales, p.scales) and np.array_equal(r.codes, p.codes)
+
+
+def correlated(rng, R, k):
+    X = rng.standard_normal((R, k)).astype(np.float32)
+    X[:, 1::2] += 0.8 * X[:, 0::2]
+    X[:, 2::3] += 0.5 * X[:, 1::3][:, :X[:, 2::3].shape[1]]
+    return X
+
+
+def test_ordered_equals_physical_permutation(orc):
+    """The sweep in a permuted block order equals the natural-order sweep of the physically
+    permuted matrix (columns, h and H permuted block-wise), mapped back."""
+    rng = np.random.default_rng(12)
+    n, k, B = 9, 128, 16
+    X = correlated(rng, 800, k)
+    W = (rng.standard_t(4, (n, k)) * 0.05).astype(np.float32)
+    H = orc.gram(X)
+    h = np.diagonal(H).copy()
+    perm = rng.permutation(k // B).astype(np.int32)
+    cols = (perm[:, None] * B + np.arange(B)[None, :]).reshape(-1)
+    U = orc.gptq_prepare(H[np.ix_(cols, cols)][None])[0]
+    a = orc.gptq_blocks(W, U, h, "nvfp4", "hopt", B, perm=perm)
+    b = orc.gptq_blocks(np.ascontiguousarray(W[:, cols]), U, h[cols], "nvfp4", "hopt", B)
+    assert np.array_equal(a.scales[:, perm], b.scales)
+    qa = orc.dequant(a.codes, a.scales, "nvfp4", B, n, k)
+    qb = orc.dequant(b.codes, b.scales, "nvfp4", B, n, k)
+    assert np.array_equal(qa[:, cols], qb)
+
+
+def test_block_losses_and_order(orc):
+    rng = np.random.default_rng(13)
+    n, k, B = 6, 96, 16
+    W = (rng.standard_t(4, (n, k)) * 0.05).astype(np.float32)
+    W[:, 32:48] *= 4.0                                   # the costliest block
+    h = np.exp(rng.normal(0, 1, k)).astype(np.float32)
+    L = orc.block_losses(W, h, "nvfp4", "hopt", B)
+    r = orc.quantize(W, "nvfp4", "hopt", B, h=h)
+    np.testing.assert_allclose(L, r.best.sum(axis=0), rtol=1e-12)  # hopt's own objective
+    order = orc.block_order(L)
+    assert order[0] == 2 and sorted(order.tolist()) == list(range(k // B))
+    assert np.all(np.diff(L[order]) <= 0)
+    assert orc.block_order([1.0, 3.0, 3.0, 2.0]).tolist() == [1, 2, 3, 0]
+
+
+@pytest.mark.parametrize("ordered", [False, True])
+def test_gptq_lowers_output_error(orc, ordered):
+    """What GPTQ is for: a smaller output error ||X (W - Q)^T|| than the plain quantizer,
+    with correlated inputs (the weight error itself grows, as on the page's tables)."""
+    rng = np.random.default_rng(14)
+    R, n, k, B = 3000, 48, 256, 16
+    X = correlated(rng, R, k)
+    W = (rng.standard_t(4, (n, k)) * 0.05).astype(np.float32)
+    H = orc.gram(X)
+    h = np.diagonal(H).copy()
+    g = orc.gptq(W, H, h, "nvfp4", "hopt", B, ordered=ordered)
+    p = orc.quantize(W, "nvfp4", "hopt", B, h=h)
+    Xd, Wd = X.astype(np.float64), W.astype(np.float64)
+    out = {}
+    for nm, r in (("gptq", g), ("plain", p)):
+        Q = orc.dequant(r.codes, r.scales, "nvfp4", B, n, k).astype(np.float64)
+        out[nm] = (np.linalg.norm(Xd @ (Wd - Q).T), np.linalg.norm(Wd - Q))
+    assert out["gptq"][0] < 0.92 * out["plain"][0]
+    assert out["gptq"][1] > out["plain"][1]
+
+
+def test_gram_is_the_mean_outer_product(orc):
+    rng = np.random.default_rng(15)
+    X = rng.standard_normal((5, 4)).astype(np.float32)
+    H = orc.gram(X)
+    ref = sum(np.outer(x.astype(np.float64), x.astype(np.float64)) for x in X) / 5
+    np.testing.assert_allclose(H, ref.astype(np.float32), rtol=1e-7)
+    assert np.array_equal(np.diagonal(H), orc.act_sqmean(X))
