@@ -429,21 +429,26 @@ int orc_quantize_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t 
 
 /* ----------------------------------------------------------------------------------
  * GPTQ with the block quantizer as its inner step (qwantize "Results", "GPTQ
- * Quantization": the GPTQ block is the quantization block, each block's quantization
- * error is compensated in all later columns through the inverse Hessian; the algorithm is
- * Frantar et al. 2022, Algorithm 1, in its Cholesky form). When the sweep reaches a block,
- * its scale is the quantizer's pick (naive / SSE / H-optimal, as orc_quantize_blocks) for
- * the block's CURRENT weights -- GPTQ fixes a group's quantization grid at the moment the
- * group is reached -- and the block's columns are then quantised one after another at that
- * scale, each residual propagated at once. Rows are independent; for row i, with the
- * block visited at sweep position t being perm[t] (t itself when perm is NULL) and the
- * sweep position of column col = b B + j being p = t B + j:
- *     q = project(w_col at the block's scale), wq = +-fl32(s q) (the sign of w_col),
- *     err = (w_col - wq) / U[p][p],
- *     w at every later position p' -= err * U[p][p']
- * every step a separately rounded float32 operation. U [k][k] (float32, upper triangular)
- * is the upper Cholesky factor of the damped H^-1 with H's rows and columns in sweep order
- * (positions). codes / scales: the layouts of orc_quantize_blocks; rows [row0, row1).
+ * Quantization": the GPTQ block is the quantization block; after a block is quantised its
+ * error is compensated in all remaining columns by one product of the block's residuals
+ * with the block's rows of the inverse-Hessian factor). The algorithm is Frantar et al.
+ * 2022, Algorithm 1, in its Cholesky form. When the sweep reaches a block, its scale is the
+ * quantizer's pick (naive / SSE / H-optimal, as orc_quantize_blocks) for the block's
+ * CURRENT weights -- GPTQ fixes a group's quantization grid at the moment the group is
+ * reached -- and the block's columns are then quantised one after another at that scale.
+ * Rows are independent; for row i, with the block visited at sweep position t being
+ * perm[t] (t itself when perm is NULL) and p = t B + j the sweep position of column
+ * col = b B + j:
+ *   for j = 0 .. B-1:
+ *     q = project(w at p, the block's scale), wq = +-fl32(s q) (the sign of w),
+ *     err_j = (w - wq) / U[p][p],
+ *     w at position p' -= err_j * U[p][p'] for the block's later positions p'
+ *       (product, then difference: the in-block update of the algorithm);
+ *   then for every position p' after the block (the block's product "err @ U[block, rest]"):
+ *     acc = 0; for j = 0 .. B-1: acc = fma(err_j, U[t B + j][p'], acc);  w at p' -= acc.
+ * Every step is one IEEE float32 operation (fma rounded once). U [k][k] (float32, upper
+ * triangular) is the upper Cholesky factor of the damped H^-1 with H's rows and columns in
+ * sweep order. codes / scales: the layouts of orc_quantize_blocks; rows [row0, row1).
  * ---------------------------------------------------------------------------------- */
 int orc_gptq_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
                     const float *h, int fmt, int sfmt, int mode, int B, int window,
@@ -451,7 +456,7 @@ int orc_gptq_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
                     uint8_t *codes, uint8_t *scales)
 {
     scale_grid g;
-    if (B <= 0 || k % B != 0 || U == NULL || grid_of(sfmt, &g)) return -1;
+    if (B <= 0 || B > 256 || k % B != 0 || U == NULL || grid_of(sfmt, &g)) return -1;
     if (fmt != ORC_NVFP4 && fmt != ORC_INT8 && fmt != ORC_INT4) return -1;
     if (fmt == ORC_INT8 && sfmt != ORC_S_E4M3) return -1;
     if (fmt == ORC_INT4 && sfmt == ORC_S_UE8M0) return -1;
@@ -465,6 +470,7 @@ int orc_gptq_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
     }
     float *w = (float *)malloc(sizeof(float) * (size_t)k);
     float *cw = (float *)malloc(sizeof(float) * (size_t)B);
+    float *err = (float *)malloc(sizeof(float) * (size_t)B);
     for (int64_t i = row0; i < row1 && i < n; ++i) {
         for (int64_t j = 0; j < k; ++j) w[j] = elem(W, dtype, ld, i, j);
         for (int64_t t = 0; t < kb; ++t) {
@@ -474,23 +480,29 @@ int orc_gptq_blocks(const void *W, int dtype, int64_t n, int64_t k, int64_t ld,
             int c0;
             int c = search_block(fmt, sfmt, mode, window, &g, &w[j0], cw, B, &e1, &e2, &c0);
             scales[i * kb + j0 / B] = (uint8_t)c;
-            for (int j = 0; j < B; ++j) {
+            for (int j = 0; j < B; ++j) {            /* the block's columns, in order */
                 int64_t p = t * B + j;
                 float wv = w[j0 + j];
                 float wq_abs;
                 project(fmt, sfmt, c, wv, &wq_abs);
                 emit_block(fmt, sfmt, c, &w[j0 + j], 1, codes, i, j0 + j, k);
                 float wq = copysignf(wq_abs, wv);
-                float err = (wv - wq) / U[p * k + p];
-                for (int64_t p2 = p + 1; p2 < k; ++p2) {
-                    float prod = err * U[p * k + p2];
-                    w[col[p2]] = w[col[p2]] - prod;
+                err[j] = (wv - wq) / U[p * k + p];
+                for (int j2 = j + 1; j2 < B; ++j2) {
+                    float prod = err[j] * U[p * k + t * B + j2];
+                    w[j0 + j2] = w[j0 + j2] - prod;
                 }
+            }
+            for (int64_t p2 = (t + 1) * B; p2 < k; ++p2) {   /* the rest: one product */
+                float acc = 0.0f;
+                for (int j = 0; j < B; ++j) acc = fmaf(err[j], U[(t * B + j) * k + p2], acc);
+                w[col[p2]] = w[col[p2]] - acc;
             }
         }
     }
     free(w);
     free(cw);
+    free(err);
     free(col);
     return 0;
 }

@@ -53,17 +53,23 @@ MUTANTS = {
     "gptq_no_division": ("float err = (wv - wq) / Ub[c * T + c];", "float err = (wv - wq);"),
     "gptq_wrong_sign": ("w[r * T + j] = w[r * T + j] - prod;", "w[r * T + j] = w[r * T + j] + prod;"),
     "gptq_transposed_factor": ("float prod = err * Ub[c * T + j];", "float prod = err * Ub[j * T + c];"),
-    "gptq_blocks_no_division": ("float err = (wv - wq) / U[p * k + p];", "float err = (wv - wq);"),
-    "gptq_blocks_wrong_sign": ("w[col[p2]] = w[col[p2]] - prod;", "w[col[p2]] = w[col[p2]] + prod;"),
-    "gptq_blocks_transposed_factor": ("float prod = err * U[p * k + p2];",
-                                      "float prod = err * U[p2 * k + p];"),
-    "gptq_blocks_no_intrablock": ("for (int64_t p2 = p + 1; p2 < k; ++p2) {",
-                                  "for (int64_t p2 = (t + 1) * B; p2 < k; ++p2) {"),
+    "gptq_blocks_no_division": ("err[j] = (wv - wq) / U[p * k + p];", "err[j] = (wv - wq);"),
+    "gptq_blocks_wrong_sign": ("w[col[p2]] = w[col[p2]] - acc;", "w[col[p2]] = w[col[p2]] + acc;"),
+    "gptq_blocks_transposed_factor": (
+        "acc = fmaf(err[j], U[(t * B + j) * k + p2], acc);",
+        "acc = fmaf(err[j], U[p2 * k + t * B + j], acc);"),
+    "gptq_blocks_no_intrablock": ("w[j0 + j2] = w[j0 + j2] - prod;", "w[j0 + j2] = w[j0 + j2];"),
     "gptq_blocks_search_original": (
         "int c = search_block(fmt, sfmt, mode, window, &g, &w[j0], cw, B, &e1, &e2, &c0);",
-        "float w0[64];\n            for (int j = 0; j < B; ++j) w0[j] = elem(W, dtype, ld, i, j0 + j);\n"
+        "float w0[256];\n            for (int j = 0; j < B; ++j) w0[j] = elem(W, dtype, ld, i, j0 + j);\n"
         "            int c = search_block(fmt, sfmt, mode, window, &g, w0, cw, B, &e1, &e2, &c0);"),
     "gptq_blocks_perm_ignored": ("int64_t b = perm ? perm[t] : t;", "int64_t b = t;"),
+    "gptq_blocks_per_column_subtraction": (
+        "for (int j = 0; j < B; ++j) acc = fmaf(err[j], U[(t * B + j) * k + p2], acc);\n"
+        "                w[col[p2]] = w[col[p2]] - acc;",
+        "for (int j = 0; j < B; ++j) w[col[p2]] = w[col[p2]] - err[j] * U[(t * B + j) * k + p2];"),
+    "gptq_blocks_last_residual_only": ("for (int j = 0; j < B; ++j) acc = fmaf(",
+                                       "for (int j = B - 1; j < B; ++j) acc = fmaf("),
     "dequant_not_rounded": ("float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - (double)wq;",
                             "float wq = copysignf(wq_abs, w[j]);\n        double d = (double)w[j] - 1.0000001 * (double)wq;"),
 }

@@ -49,6 +49,25 @@ def test_worked_example_negative(orc):
     assert r.codes[0, 0] == 0xEA and r.codes[0, 1] == 0x0F and r.codes[0, 8] == 0x0F
 
 
+def test_block_product_subtracted_once(orc):
+    """Past its block a residual is applied as one product per block (the page's
+    w_rem -= err @ h_cross), not column by column, and the two differ in rounding: block 0
+    leaves residuals err_0 = err_1 = 0.25 (1.25 at scale 1 ties to E2M1 1.0), and
+    U[0][16] = U[1][16] = 2^-22, so column 16 (1.75) receives 2^-24 twice. One subtraction of
+    their sum gives 1.75 - 2^-23, which at block 1's scale 0.5 (amax 3) is 3.4999998: E2M1
+    3.0 (code 5). Two subtractions of 2^-24 each tie back to 1.75 (the even neighbour):
+    3.5, the E2M1 midpoint, ties to 4.0 (code 6). Column 17 (3.0) is E2M1 6.0 (code 7)."""
+    k = 32
+    W = np.zeros((1, k), np.float32)
+    W[0, [0, 1, 2, 16, 17]] = [1.25, 1.25, 6.0, 1.75, 3.0]
+    U = np.eye(k, dtype=np.float32)
+    U[0, 16] = U[1, 16] = 2.0 ** -22
+    r = orc.gptq_blocks(W, U, np.ones(k, np.float32), "nvfp4", "naive", 16)
+    assert r.scales[0].tolist() == [0x38, 0x30]
+    assert r.codes[0, 8] == 0x75 and r.codes[0, 0] == 0x22 and r.codes[0, 1] == 0x07
+    assert orc.quantize(W, "nvfp4", "naive", 16).codes[0, 8] == 0x76
+
+
 @pytest.mark.parametrize("fmt,sfmt,block", [("nvfp4", "e4m3", 16), ("nvfp4", "ue8m0", 32),
                                             ("int4", "e4m3", 16), ("int8", "e4m3", 32)])
 @pytest.mark.parametrize("mode", ["naive", "sse", "hopt"])
