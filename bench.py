@@ -46,6 +46,7 @@ ALU_PEAK_TOPS = 148 * 128 * 1.965e9 / 1e12
 # Oracle samples: the cpu_baseline leg (about 10-30 s of CPU work) and each step of the
 # reference arm (well under a second, so that a long --steps run stays short).
 CPU_X_ROWS, CPU_W_ROWS = 32768, 1024
+GPTQ_CPU_X_ROWS, GPTQ_CPU_W_ROWS = 4096, 16
 Quantizer = collections.namedtuple("Quantizer", "fmt block mode window sfmt")
 HEADLINE_Q = Quantizer("nvfp4", 16, "hopt", -1, "e4m3")
 REF_X_ROWS, REF_W_ROWS = 2048, 8
@@ -61,9 +62,12 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block", type=int, default=0, help="block size (default: the workload's)")
-    ap.add_argument("--mode", default="", choices=["", "naive", "sse", "hopt", "bhopt"],
+    ap.add_argument("--mode", default="",
+                    choices=["", "naive", "sse", "hopt", "bhopt", "gptq", "gptq-ord"],
                     help="bhopt: the block-Hessian objective d^T G_b d (Gram pass on the "
-                         "tensor cores instead of the h pass)")
+                         "tensor cores instead of the h pass); gptq: GPTQ with the H-optimal "
+                         "quantizer as its inner step (NVFP4 / INT4: full Hessian; E4M3: "
+                         "64 x 64 tiles); gptq-ord: ordered GPTQ (NVFP4 / INT4)")
     ap.add_argument("--fmt", default="", choices=["", "nvfp4", "int4", "int8", "e4m3"],
                     help="element format (default: the workload's)")
     ap.add_argument("--scale-fmt", default="", choices=["", "e4m3", "ue4m4", "ue5m3", "ue8m0"],
@@ -181,6 +185,10 @@ def workload_desc(wl, q, x_rows=None):
     ncand = {"e4m3": 126, "ue4m4": 255, "ue5m3": 255, "ue8m0": 255}[q.sfmt]
     grid = ("64-point log grid" if fmt == "e4m3" else
             f"all {ncand} {sg} scales" if window < 0 else f"{sg} scales within +-{window} codes")
+    if mode == "gptq":
+        return (f"{wl.name}: W {shapes} {dt}; X {xsh} {dt}; e4m3 64x64 tiles: Gram blocks of X "
+                f"(h = their diagonal), GPTQ factors (damp {GPTQ_DAMP}), tile scales by the "
+                f"hopt search on the {grid}, GPTQ sweep; then weight/h-weighted error sums")
     return (f"{wl.name}: W {shapes} {dt}; X {xsh} {dt}; {quant_name(q)} block {block}, {mode}, "
             f"{grid}; then weight/h-weighted error sums")
 
@@ -194,27 +202,55 @@ def oracle_step_sample(X_bits, W_bits, h_np, n_threads, R_full, N_full, q):
     rows of W, bf16 bits; q the quantizer) and scale each part to the full
     workload (R_full rows of X, N_full rows of W, in units of the sample's row widths).
     Returns (seconds for a full step, measured seconds per part)."""
+    import numpy as np
     from oracle import oracle as orc
     fmt, block, mode, window = q.fmt, q.block, q.mode, q.window
     x_rows, K = X_bits.shape
     w_rows = W_bits.shape[0]
+    if full_gptq(q):
+        t0 = time.perf_counter()
+        H = orc.gram(X_bits)
+        h = orc.act_sqmean(X_bits, n_threads=n_threads)
+        t1 = time.perf_counter()
+        if mode == "gptq-ord":
+            perm = orc.block_order(orc.block_losses(W_bits, h, fmt, "hopt", block, sfmt=q.sfmt,
+                                                    window=window))
+        else:
+            perm = np.arange(K // block, dtype=np.int32)
+        t2 = time.perf_counter()
+        cols = (perm[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+        U = orc.gptq_prepare(np.ascontiguousarray(H[np.ix_(cols, cols)])[None], GPTQ_DAMP)[0]
+        t3 = time.perf_counter()
+        r = orc.gptq_blocks(W_bits, U, h, fmt, "hopt", block, sfmt=q.sfmt, window=window,
+                            perm=perm, n_threads=n_threads)
+        What = orc.dequant(r.codes, r.scales, fmt, block, w_rows, K, sfmt=q.sfmt)
+        orc.error_sums(W_bits, What, h)
+        t4 = time.perf_counter()
+        full = ((t1 - t0) * (R_full / x_rows) + (t2 - t1) * (N_full / w_rows) + (t3 - t2)
+                + (t4 - t3) * (N_full / w_rows))
+        return full, {"h_s": t1 - t0 + t3 - t2, "quant_s": t2 - t1 + t4 - t3}
     t0 = time.perf_counter()
-    if mode == "bhopt":
+    if mode in ("bhopt", "gptq"):
         G = orc.block_gram(X_bits, block)
     else:
         orc.act_sqmean(X_bits, n_threads=n_threads)
     t1 = time.perf_counter()
+    if mode == "gptq":                     # per column block: independent of the rows
+        U = orc.gptq_prepare(G)
+        h_np = np.diagonal(G, axis1=1, axis2=2).reshape(-1).copy()
+    tp = time.perf_counter()
     if mode == "bhopt":
         r = orc.quantize_gram(W_bits, fmt, block, G, window=window, n_threads=n_threads,
                               sfmt=q.sfmt)
     else:
-        r = orc.quantize(W_bits, fmt, mode, block, h=h_np, window=window, n_threads=n_threads,
-                         sfmt=q.sfmt)
-    What = orc.dequant(r.codes, r.scales, fmt, block, w_rows, K, sfmt=q.sfmt)
+        r = orc.quantize(W_bits, fmt, "hopt" if mode == "gptq" else mode, block, h=h_np,
+                         window=window, n_threads=n_threads, sfmt=q.sfmt)
+    codes = orc.gptq_tiles(W_bits, U, r.scales) if mode == "gptq" else r.codes
+    What = orc.dequant(codes, r.scales, fmt, block, w_rows, K, sfmt=q.sfmt)
     orc.error_sums(W_bits, What, h_np)
     t2 = time.perf_counter()
-    full = (t1 - t0) * (R_full / x_rows) + (t2 - t1) * (N_full / w_rows)
-    return full, {"h_s": t1 - t0, "quant_s": t2 - t1}
+    full = (t1 - t0) * (R_full / x_rows) + (tp - t1) + (t2 - tp) * (N_full / w_rows)
+    return full, {"h_s": t1 - t0 + tp - t1, "quant_s": t2 - tp}
 
 
 def bits_of(t):
@@ -275,7 +311,28 @@ def quantizer_for(wl, args):
     """The quantizer the bench times for a workload (its own, or the command line's)."""
     block = args.block or wl.blocks[0]
     mode = args.mode or ("hopt" if "hopt" in wl.modes else wl.modes[-1])
-    return Quantizer(args.fmt or wl.fmt, block, mode, wl.window, args.scale_fmt or "e4m3")
+    fmt = args.fmt or wl.fmt
+    if mode == "gptq" and fmt == "e4m3" and block != 64:
+        raise SystemExit("--mode gptq on E4M3 elements uses 64 x 64 tiles")
+    if mode.startswith("gptq") and fmt not in ("e4m3", "nvfp4", "int4"):
+        raise SystemExit("--mode gptq: NVFP4 / INT4 blocks or E4M3 64 x 64 tiles")
+    if mode == "gptq-ord" and fmt == "e4m3":
+        raise SystemExit("--mode gptq-ord: NVFP4 / INT4 blocks")
+    return Quantizer(fmt, block, mode, wl.window, args.scale_fmt or "e4m3")
+
+
+def full_gptq(q):
+    """GPTQ over the whole input dimension (NVFP4 / INT4 blocks), not the E4M3 tiles."""
+    return q.mode in ("gptq", "gptq-ord") and q.fmt in ("nvfp4", "int4")
+
+
+def sweep_ops_per_weight(q, k):
+    """Algorithmic lane-operations per weight of the GPTQ sweep: the block's scale search
+    (C candidates x 6 + 4, as the plain search), its own quantisation, residual and division
+    (6), and the updates it receives from every earlier column -- one product and one
+    difference from each earlier column of its block, one fma from each column of every
+    earlier block plus one difference per earlier block: on average (k / 2)(1 + 1/B)."""
+    return ops_per_weight(q.fmt, "hopt", q.window, q.sfmt, q.block) + 6 + (k / 2) * (1 + 1 / q.block)
 
 
 def metric_for(q):
@@ -294,6 +351,13 @@ def ops_per_weight(fmt, mode, window, sfmt="e4m3", block=16):
     return C * (6 if mode == "hopt" else 5) + 4
 
 
+# The GPTQ sweep per weight: quotient, round, dequantise, residual, division by U_cc, pack
+# (6), and its residual's propagation into the 63 - c later columns of the tile row, one
+# product and one difference each (2 x 31.5 on average over c = 0 .. 63).
+GPTQ_SWEEP_OPS = 6 + 63
+GPTQ_DAMP = 0.01          # lambda = 0.01 x mean(diag G_b), GPTQ's customary damping
+
+
 def code_bytes(fmt, block):
     """Bytes of codes + scales per weight."""
     if fmt in ("nvfp4", "int4"):
@@ -308,34 +372,39 @@ def gpu_arm(args):
     from block_scaled_weight_b200 import mxq, synth
     from block_scaled_weight_b200.dist import distributed_h
     rank, world, local = dist_env()
+    wl = synth.WORKLOADS[args.workload]
+    q = quantizer_for(wl, args)
+    if full_gptq(q):
+        return gpu_arm_gptq(args, wl, q)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    wl = synth.WORKLOADS[args.workload]
-    q = quantizer_for(wl, args)
     fmt, block, mode, window = q.fmt, q.block, q.mode, q.window
-    bh = mode == "bhopt"
-    if bh and world > 1:
-        raise SystemExit("--mode bhopt runs on one GPU")
-    p = mxq.params(fmt, "hopt" if bh else mode, block, window=window, scale_fmt=q.sfmt)
+    bh, gq = mode == "bhopt", mode == "gptq"
+    gram = bh or gq                       # the Gram pass replaces the h pass
+    if gram and world > 1:
+        raise SystemExit(f"--mode {mode} runs on one GPU")
+    p = mxq.params(fmt, "hopt" if gram else mode, block, window=window, scale_fmt=q.sfmt)
     # inputs: every rank draws its own shard (weak scaling)
     wl_r = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
     # activations and their h, one per activation width
-    Xs, hs, wss, cols, Gs = [], [], [], [], []
+    Xs, hs, wss, cols, Gs, Us = [], [], [], [], [], []
     for xi, (R, k) in enumerate(wl.x_shapes):
         R = min(R, args.x_rows) if args.x_rows else R
         X = torch.empty(R, k, dtype=wl.w_dtype, device=dev)
         synth.workload_activations(wl_r, xi, device=dev, rows=R, out=X)
         Xs.append(X)
         hs.append(torch.empty(k, dtype=torch.float32, device=dev))
-        wss.append(torch.empty(mxq.mxq_act_block_gram_workspace(R, k, block) if bh else
+        wss.append(torch.empty(mxq.mxq_act_block_gram_workspace(R, k, block) if gram else
                                mxq.mxq_act_sqmean_workspace(R, k), dtype=torch.uint8, device=dev))
         cols.append(torch.empty(k, dtype=torch.float64, device=dev))
         Gs.append(torch.empty(k // block, block, block, dtype=torch.float32, device=dev)
-                  if bh else None)
+                  if gram else None)
+        Us.append(torch.empty(k // block, block, block, dtype=torch.float32, device=dev)
+                  if gq else None)
     # weights and their outputs (codes, scales, error sums, error workspace, which h)
     Ws, outs = [], []
     for wi, (_, n, k) in enumerate(wl.weights):
@@ -346,16 +415,17 @@ def gpu_arm(args):
                      torch.empty(mxq.mxq_error_workspace(n, k), dtype=torch.uint8, device=dev),
                      synth.x_index_for_weight(wl, wi)))
     stream = torch.cuda.current_stream(dev)
-    # our kernels per step: h pass (2 per activation matrix; 3 with the sharded finalize),
-    # search (+ exact fixup for NVFP4 searches), error sums + combine (2) per weight
+    # our kernels per step: h pass or Gram pass (2 per activation matrix; 3 with the sharded
+    # finalize), search (+ exact fixup for NVFP4 / INT8 searches), error sums + combine (2)
+    # per weight; GPTQ adds the factor (1 per activation matrix) and the sweep (1 per weight)
     fixup = 1 if mode != "naive" and fmt != "e4m3" else 0
     launches_per_step = len(Xs) * (2 if world == 1 else 3) + len(Ws) * (1 + fixup + 2)
+    if gq:
+        launches_per_step += len(Xs) + len(Ws)
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def h_phase():
         for X, h, ws, colsum, G in zip(Xs, hs, wss, cols, Gs):
-            if bh:
+            if gram:
                 mxq.mxq_act_block_gram(X, block, G, h, workspace=ws)
             elif world == 1:
                 mxq.mxq_act_sqmean(X, h, workspace=ws)
@@ -364,19 +434,42 @@ def gpu_arm(args):
                 distributed_h(X, lambda x, c=colsum, w=ws: mxq.mxq_act_sqsum(x, c, workspace=w),
                               lambda pp, r, hh=h: mxq.mxq_act_sqmean_finalize(pp, r, hh),
                               X.shape[0] * world)
-        if ev is not None:
-            ev[1].record(stream)
+
+    def prepare_phase():
+        for G, U in zip(Gs, Us):
+            mxq.mxq_gptq_prepare(G, GPTQ_DAMP, U=U)
+
+    def quantize_phase():
         for W, (codes, scales, _, _, xi) in zip(Ws, outs):
             if bh:
                 mxq.mxq_quantize_gram(W, p, Gs[xi], codes=codes, scales=scales)
             else:
                 mxq.mxq_quantize(W, p, hs[xi], codes=codes, scales=scales)
-        if ev is not None:
-            ev[2].record(stream)
+
+    def sweep_phase():
+        for W, (codes, scales, _, _, xi) in zip(Ws, outs):
+            mxq.mxq_gptq_tiles(W, Us[xi], scales, codes=codes)
+
+    def error_phase():
         for W, (codes, scales, sums, ews, xi) in zip(Ws, outs):
             mxq.mxq_error(W, codes, scales, p, hs[xi], sums=sums, workspace=ews)
+
+    hname = "block_gram" if gram else "act_sqmean"
+    phases = [(hname, h_phase)]
+    if gq:
+        phases.append(("gptq_prepare", prepare_phase))
+    phases.append(("quantize", quantize_phase))
+    if gq:
+        phases.append(("gptq_tiles", sweep_phase))
+    phases.append(("error", error_phase))
+
+    def step(ev=None):
+        for i, (_, fn) in enumerate(phases):
+            if ev is not None:
+                ev[i].record(stream)
+            fn()
         if ev is not None:
-            ev[3].record(stream)
+            ev[-1].record(stream)
 
     def barrier():
         if world > 1:
@@ -391,7 +484,8 @@ def gpu_arm(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)]
+           for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -407,14 +501,15 @@ def gpu_arm(args):
         torch.cuda.synchronize(dev)
     barrier()
     ms_total = t_start.elapsed_time(t_end) if flush is None else \
-        sum(e[0].elapsed_time(e[3]) for e in evs)
-    k_h = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    k_q = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    k_e = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-    t = torch.tensor([ms_total, k_h, k_q, k_e], dtype=torch.float64, device=dev)
+        sum(e[0].elapsed_time(e[-1]) for e in evs)
+    k_ph = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
+            for i in range(len(phases))]
+    t = torch.tensor([ms_total] + k_ph, dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total, k_h, k_q, k_e = t.tolist()
+    ms_total, *k_ph = t.tolist()
+    k_of = {nm: kk for (nm, _), kk in zip(phases, k_ph)}
+    k_h, k_q, k_e = k_of[hname], k_of["quantize"], k_of["error"]
     ms_step = ms_total / args.steps
     weights = sum(W.numel() for W in Ws)
     value = world * weights / (ms_step * 1e-3) / 1e9
@@ -467,11 +562,10 @@ def gpu_arm(args):
     # ---- roofline ------------------------------------------------------------------------
     hbm, hbm_kind = measured_peaks()
     headline = args.workload == "nvfp4_full_calib" and q == HEADLINE_Q and not args.x_rows
-    x_bytes = sum(X.numel() * X.element_size() + 4 * X.shape[1] * (block if bh else 1)
+    x_bytes = sum(X.numel() * X.element_size() + 4 * X.shape[1] * (block if gram else 1)
                   for X in Xs)
     w_bytes = sum(W.numel() * W.element_size() for W in Ws)
     h_gbs = x_bytes / (k_h * 1e-3) / 1e9
-    hname = "block_gram" if bh else "act_sqmean"
     kernels = {hname: {"ms": k_h, "bound": "hbm", "achieved": h_gbs, "peak": hbm,
                        "unit": "GB/s", "frac": h_gbs / hbm, "algorithmic_bytes": x_bytes,
                        "traffic": traffic_for("act_sqmean") if headline else None}}
@@ -488,6 +582,19 @@ def gpu_arm(args):
                                "peak": ALU_PEAK_TOPS, "unit": "T lane-op/s",
                                "frac": q_tops / ALU_PEAK_TOPS, "algorithmic_ops": ops,
                                "traffic": traffic_for("quantize") if headline else None}
+    if gq:
+        u_bytes = sum(2 * 4 * X.shape[1] * block for X in Xs)     # G read, U written
+        kernels["gptq_prepare"] = {
+            "ms": k_of["gptq_prepare"], "bound": "hbm",
+            "achieved": u_bytes / (k_of["gptq_prepare"] * 1e-3) / 1e9, "peak": hbm,
+            "unit": "GB/s", "frac": u_bytes / (k_of["gptq_prepare"] * 1e-3) / 1e9 / hbm,
+            "algorithmic_bytes": u_bytes, "traffic": None}
+        s_ops = GPTQ_SWEEP_OPS * weights
+        s_tops = s_ops / (k_of["gptq_tiles"] * 1e-3) / 1e12
+        kernels["gptq_tiles"] = {"ms": k_of["gptq_tiles"], "bound": "alu", "achieved": s_tops,
+                                 "peak": ALU_PEAK_TOPS, "unit": "T lane-op/s",
+                                 "frac": s_tops / ALU_PEAK_TOPS, "algorithmic_ops": s_ops,
+                                 "traffic": None}
     e_bytes = w_bytes + weights * code_bytes(fmt, block) + sum(4 * W.shape[1] for W in Ws)
     e_gbs = e_bytes / (k_e * 1e-3) / 1e9
     kernels["error"] = {"ms": k_e, "bound": "hbm", "achieved": e_gbs, "peak": hbm, "unit": "GB/s",
@@ -531,6 +638,8 @@ def gpu_arm(args):
         R0, n0 = X0.shape[0], W0.shape[0]
         x_rows = min(CPU_X_ROWS, R0)
         w_rows = min(CPU_W_ROWS // (8 if fmt == "e4m3" or mode == "bhopt" else 1), n0)
+        if fmt == "e4m3":
+            w_rows = max(w_rows - w_rows % block, block)
         Xb = bits_of(X0[:x_rows].cpu())
         Wb = bits_of(W0[:w_rows].cpu())
         from oracle import oracle as orc
@@ -548,6 +657,203 @@ def gpu_arm(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def bf16_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops_sustained"]), "measured, sustained"
+    except Exception:
+        return 1400.0, "fallback, sustained"
+
+
+# FP64 FMA peak of the factorisation kernels: 148 SMs x 64 FP64 lanes x 2 flops x 1965 MHz.
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
+
+
+def gpu_arm_gptq(args, wl, q):
+    """GPTQ over the whole input dimension with the H-optimal quantizer as its inner step
+    (sequential or ordered) on one GPU: h pass, Gram matrix, [block order], factor, sweep,
+    error sums."""
+    from block_scaled_weight_b200 import mxq, synth
+    rank, world, local = dist_env()
+    if world > 1:
+        raise SystemExit(f"--mode {q.mode} runs on one GPU")
+    if len(wl.weights) != 1:
+        raise SystemExit(f"--mode {q.mode}: workloads with one weight matrix")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ordered = q.mode == "gptq-ord"
+    B = q.block
+    p = mxq.params(q.fmt, "hopt", B, window=q.window, scale_fmt=q.sfmt)
+    (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
+    R = min(R, args.x_rows) if args.x_rows else R
+    X = torch.empty(R, k, dtype=wl.w_dtype, device=dev)
+    synth.workload_activations(wl, 0, device=dev, rows=R, out=X)
+    W = synth.workload_weight(wl, 0, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    u8 = dict(dtype=torch.uint8, device=dev)
+    h = torch.empty(k, **f32)
+    H = torch.empty(k, k, **f32)
+    U = torch.empty(k, k, **f32)
+    perm = torch.arange(k // B, dtype=torch.int32, device=dev)
+    hws = torch.empty(mxq.mxq_act_sqmean_workspace(R, k), **u8)
+    fws = torch.empty(mxq.mxq_gptq_factor_workspace(k), **u8)
+    ows = torch.empty(max(mxq.mxq_gptq_order_workspace(n, k, p), 8), **u8)
+    sws = torch.empty(mxq.mxq_gptq_workspace(n, k), **u8)
+    cs, cd, ss, sd = mxq.output_shapes(p, n, k)
+    codes, scales = torch.empty(cs, dtype=cd, device=dev), torch.empty(ss, dtype=sd, device=dev)
+    sums = torch.empty(4, dtype=torch.float64, device=dev)
+    ews = torch.empty(mxq.mxq_error_workspace(n, k), **u8)
+    pv = perm if ordered else None
+    phases = [("act_sqmean", lambda: mxq.mxq_act_sqmean(X, h, workspace=hws)),
+              ("gram", lambda: mxq.mxq_act_gram(X, H))]
+    if ordered:
+        phases.append(("gptq_order", lambda: mxq.mxq_gptq_order(W, h, p, perm=perm,
+                                                                workspace=ows)))
+    phases += [("gptq_factor", lambda: mxq.mxq_gptq_factor(H, B, pv, GPTQ_DAMP, U=U,
+                                                           workspace=fws)),
+               ("gptq_sweep", lambda: mxq.mxq_gptq(W, U, p, h, pv, codes=codes, scales=scales,
+                                                   workspace=sws)),
+               ("error", lambda: mxq.mxq_error(W, codes, scales, p, h, sums=sums,
+                                               workspace=ews))]
+    stream = torch.cuda.current_stream(dev)
+    nt = (k + 63) // 64
+    panels = (k + 63) // 64
+    launches_per_step = (2 + (4 if ordered else 0) + (4 * nt + 1) + 2 * panels + 2)
+
+    def step(ev=None):
+        for i, (_, fn) in enumerate(phases):
+            if ev is not None:
+                ev[i].record(stream)
+            fn()
+        if ev is not None:
+            ev[-1].record(stream)
+
+    in_bytes = X.numel() * X.element_size() + W.numel() * W.element_size()
+    flush = torch.empty(2 * L2_BYTES, **u8) if in_bytes < 4 * L2_BYTES else None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)]
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        t_start.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_total = t_start.elapsed_time(t_end) if flush is None else \
+        sum(e[0].elapsed_time(e[-1]) for e in evs)
+    k_of = {nm: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
+            for i, (nm, _) in enumerate(phases)}
+    ms_step = ms_total / args.steps
+    weights = W.numel()
+    value = weights / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API, host buffers -----------------------------
+    Xh = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+    Wh = torch.empty(W.shape, dtype=W.dtype, pin_memory=True)
+    Xh.copy_(X)
+    Wh.copy_(W)
+    oh = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (codes, scales, sums)]
+    h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in oh)
+
+    def e2e_step():
+        X.copy_(Xh, non_blocking=True)
+        W.copy_(Wh, non_blocking=True)
+        step()
+        for td, th in zip((codes, scales, sums), oh):
+            th.copy_(td, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a.elapsed_time(b) / args.e2e_steps
+    metrics = mxq.mxq_metrics_from_sums(oh[2])
+    rows = synth.sample_rows(R, 512, wl.seed + 7).to(dev)
+    Xsmp = X.index_select(0, rows).contiguous()
+    osum = mxq.mxq_output_error(Xsmp, W, codes, scales, p).cpu()
+    out_rel = float((osum[0] / osum[1]).sqrt())
+
+    # ---- roofline ------------------------------------------------------------------------
+    hbm, hbm_kind = measured_peaks()
+    bfp, bf_kind = bf16_peak()
+    x_bytes = X.numel() * X.element_size() + 4 * k
+    w_bytes = W.numel() * W.element_size()
+
+    def kern(nm, bound, amount, peak, unit):
+        ach = amount / (k_of[nm] * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+        return {"ms": k_of[nm], "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                "frac": ach / peak, ("algorithmic_bytes" if unit == "GB/s" else
+                                     "algorithmic_ops"): amount, "traffic": None}
+    kernels = {"act_sqmean": kern("act_sqmean", "hbm", x_bytes, hbm, "GB/s"),
+               "gram": kern("gram", "tensor", 2.0 * R * k * k, bfp, "TFLOP/s")}
+    if ordered:
+        kernels["gptq_order"] = kern("gptq_order", "alu",
+                                     ops_per_weight(q.fmt, "hopt", q.window, q.sfmt, B) * weights,
+                                     ALU_PEAK_TOPS, "T lane-op/s")
+    kernels["gptq_factor"] = kern("gptq_factor", "fp64", 2.0 / 3.0 * k ** 3, FP64_PEAK_TFLOPS,
+                                  "TFLOP/s")
+    kernels["gptq_sweep"] = kern("gptq_sweep", "alu", sweep_ops_per_weight(q, k) * weights,
+                                 ALU_PEAK_TOPS, "T lane-op/s")
+    kernels["error"] = kern("error", "hbm", w_bytes + weights * code_bytes(q.fmt, B) + 4 * k, hbm,
+                            "GB/s")
+    dom = max(kernels, key=lambda kk: kernels[kk]["ms"])
+    dk = kernels[dom]
+    src = {"hbm": "MEASURED_PEAKS.json hbm_gbs (" + hbm_kind + ")",
+           "tensor": "MEASURED_PEAKS.json bf16_tflops_sustained (" + bf_kind + ")",
+           "alu": "148 SM x 128 FP32 lanes x 1965 MHz",
+           "fp64": "148 SM x 64 FP64 lanes x 2 x 1965 MHz"}[dk["bound"]]
+    roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"],
+                "peak": dk["peak"], "unit": dk["unit"], "frac": dk["frac"],
+                "traffic": None, "peak_source": src}
+    line = {"metric": metric_for(q), "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(wl, q, [R]), "weights_per_gpu": weights,
+                       "x_rows_per_gpu": R, "parallelism": "dp1",
+                       "l2": ("inputs larger than L2: X (%.2f GB) is streamed every step"
+                              % (X.numel() * X.element_size() / 1e9)) if flush is None else
+                       ("L2 flushed between steps (a %d MB write, outside the step's events); "
+                        "inputs %.0f MB" % (2 * L2_BYTES >> 20, in_bytes / 1e6))},
+            "roofline": roofline, "kernels": kernels,
+            "e2e": {"value": weights / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "steps": args.e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary(),
+            "result": {"weight_rel": metrics["weight_rel"], "h_rel": metrics["h_rel"],
+                       "output_rel_512_rows": out_rel}}
+    if not args.no_cpu_baseline:
+        x_rows = min(GPTQ_CPU_X_ROWS, R)
+        w_rows = min(GPTQ_CPU_W_ROWS, n)
+        Xb = bits_of(X[:x_rows].cpu())
+        Wb = bits_of(W[:w_rows].cpu())
+        nt_cpu = os.cpu_count() or 1
+        full, d = oracle_step_sample(Xb, Wb, None, nt_cpu, R, n, q)
+        line["cpu_baseline"] = {
+            "value": weights / full / 1e9, "unit": UNIT, "cores": nt_cpu, "kind": "oracle",
+            "sample": (f"oracle on {x_rows} of {R} X rows (Gram, h) and {w_rows} of {n} W rows "
+                       f"({q.mode} sweep + error), the factor of the full {k} x {k} Hessian, "
+                       f"{nt_cpu} threads; times scaled to the full workload ({d['h_s']:.1f} s "
+                       f"+ {d['quant_s']:.1f} s measured)")}
+    print(json.dumps(line), flush=True)
 
 
 def main():

@@ -1,7 +1,8 @@
 """Build ``libmxq.so`` in-tree with nvcc for sm_100a (B200).
 
 The library is a plain C-ABI shared object (see ``include/mxq.h``); the CUDA runtime is
-linked statically so the object carries no dependency on any particular libcudart.
+linked statically so the object carries no dependency on any particular libcudart. cuBLAS
+(the one plain GEMM, GPTQ's Gram matrix) is linked dynamically from the CUDA toolkit.
 """
 from __future__ import annotations
 
@@ -14,8 +15,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmxq.so")
 SOURCES = ["mxq_api.cu", "mxq_hpass.cu", "mxq_gram.cu", "mxq_quant.cu", "mxq_quant_grid.cu",
-           "mxq_error.cu", "mxq_outerr.cu", "mxq_noalloc.cu"]
-HEADERS = ["mxq_common.cuh", "mxq_internal.h", "mxq_block.cuh", "mxq_grids.h"]
+           "mxq_error.cu", "mxq_outerr.cu", "mxq_gptq.cu", "mxq_gptq_full.cu",
+           "mxq_noalloc.cu"]
+HEADERS = ["mxq_common.cuh", "mxq_internal.h", "mxq_block.cuh", "mxq_grids.h", "mxq_gridk.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 
@@ -55,8 +57,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         subprocess.run(cmd, check=True)
         objs.append(obj)
     tmp = LIB + ".tmp"
+    cuda_lib = os.path.join(os.path.dirname(os.path.dirname(nvcc())), "lib64")
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
-           "-cudart", "static"]
+           "-cudart", "static", "-L" + cuda_lib, "-lcublas", "-Xlinker", "-rpath=" + cuda_lib]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)

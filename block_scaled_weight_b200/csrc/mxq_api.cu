@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <vector>
 
 namespace mxq {
 
@@ -203,7 +204,7 @@ mxq_status mxq_act_sqmean_finalize(const double* partials, int64_t parts, int64_
 }
 
 size_t mxq_act_block_gram_workspace(int64_t rows, int64_t cols, int32_t block) {
-  if (rows <= 0 || cols <= 0 || (block != 16 && block != 32)) return 0;
+  if (rows <= 0 || cols <= 0 || (block != 16 && block != 32 && block != 64)) return 0;
   return mxq::gram_workspace(rows, cols, block);
 }
 
@@ -213,7 +214,8 @@ mxq_status mxq_act_block_gram(const void* X, int32_t dtype, int64_t rows, int64_
   if (dtype != MXQ_BF16) return fail(MXQ_ERR_DTYPE, "block Gram needs bf16 X (dtype %d)", dtype);
   mxq_status s = check_matrix(X, dtype, rows, cols, ld, "X");
   if (s != MXQ_OK) return s;
-  if (block != 16 && block != 32) return fail(MXQ_ERR_UNSUPPORTED, "block %d (16 or 32)", block);
+  if (block != 16 && block != 32 && block != 64)
+    return fail(MXQ_ERR_UNSUPPORTED, "block %d (16, 32 or 64)", block);
   if (cols % block != 0) return fail(MXQ_ERR_SHAPE, "cols %% block != 0");
   if (cols == 0) return MXQ_OK;
   if (!G) return fail(MXQ_ERR_INVALID_ARG, "G is NULL");
@@ -379,6 +381,184 @@ mxq_status mxq_error(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t
   return cuda_status(mxq::launch_error(d, W, dtype, ld, h, (double*)workspace,
                                        mxq::error_partials(n, k), sums, st),
                      "error");
+}
+
+mxq_status mxq_gptq_prepare(const float* G, int64_t nblocks, double damp, float* U,
+                            void* stream) {
+  if (nblocks < 0) return fail(MXQ_ERR_SHAPE, "nblocks %lld", (long long)nblocks);
+  if (!std::isfinite(damp) || damp < 0) return fail(MXQ_ERR_INVALID_ARG, "damp %g", damp);
+  if (nblocks == 0) return MXQ_OK;
+  if (nblocks > 0x7fffffff) return fail(MXQ_ERR_SHAPE, "nblocks beyond 2^31 - 1");
+  if (!G || !U) return fail(MXQ_ERR_INVALID_ARG, "G or U is NULL");
+  if (!aligned(G, 16) || !aligned(U, 16)) return fail(MXQ_ERR_ALIGN, "G or U not 16-byte aligned");
+  return cuda_status(mxq::launch_gptq_prepare(G, nblocks, damp, U, (cudaStream_t)stream),
+                     "GPTQ prepare");
+}
+
+mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                          const float* U, const float* scales, uint8_t* codes, void* stream) {
+  mxq_status s = check_matrix(W, dtype, n, k, ld, "W");
+  if (s != MXQ_OK) return s;
+  if (n % 64 != 0 || k % 64 != 0) return fail(MXQ_ERR_SHAPE, "n and k must be multiples of 64");
+  if (n == 0 || k == 0) return MXQ_OK;
+  if (k / 64 > 65535) return fail(MXQ_ERR_SHAPE, "k beyond 64 * 65535");
+  if (!U || !scales || !codes) return fail(MXQ_ERR_INVALID_ARG, "U, scales or codes is NULL");
+  if (!aligned(U, 16) || !aligned(codes, 16) || !aligned(scales, 4))
+    return fail(MXQ_ERR_ALIGN, "U or codes not 16-byte, or scales not 4-byte aligned");
+  return cuda_status(mxq::launch_gptq_tiles(W, dtype, n, k, ld, U, scales, codes,
+                                            (cudaStream_t)stream),
+                     "GPTQ tiles");
+}
+
+mxq_status mxq_act_gram(const void* X, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                        float* H, void* stream) {
+  if (dtype != MXQ_BF16) return fail(MXQ_ERR_DTYPE, "Gram matrix needs bf16 X (dtype %d)", dtype);
+  mxq_status s = check_matrix(X, dtype, rows, cols, ld, "X");
+  if (s != MXQ_OK) return s;
+  if (cols == 0) return MXQ_OK;
+  if (!H) return fail(MXQ_ERR_INVALID_ARG, "H is NULL");
+  if (!aligned(H, 16)) return fail(MXQ_ERR_ALIGN, "H not 16-byte aligned");
+  if (rows > 0x7fffffff || cols > 0x7fffffff || ld > 0x7fffffff)
+    return fail(MXQ_ERR_SHAPE, "rows, cols and ld must be below 2^31");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (rows == 0)
+    return cuda_status(cudaMemsetAsync(H, 0, (size_t)cols * cols * sizeof(float), st), "memset H");
+  const char* why = "";
+  cudaError_t e = mxq::launch_gram_full(X, rows, cols, ld, H, st, &why);
+  if (e == cudaErrorUnknown && why[0]) return fail(MXQ_ERR_CUDA, "Gram matrix: %s", why);
+  return cuda_status(e, "Gram matrix");
+}
+
+size_t mxq_gptq_factor_workspace(int64_t k) {
+  return k > 0 ? mxq::gptq_factor_workspace(k) : 0;
+}
+
+mxq_status mxq_gptq_factor(const float* H, int64_t k, int32_t block, const int32_t* perm,
+                           double damp, float* U, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (k < 0) return fail(MXQ_ERR_SHAPE, "k %lld", (long long)k);
+  if (block != 16 && block != 32) return fail(MXQ_ERR_UNSUPPORTED, "block %d (16 or 32)", block);
+  if (k % block != 0) return fail(MXQ_ERR_SHAPE, "k %% block != 0");
+  if (!std::isfinite(damp) || damp < 0) return fail(MXQ_ERR_INVALID_ARG, "damp %g", damp);
+  if (k == 0) return MXQ_OK;
+  if (k > 65536) return fail(MXQ_ERR_SHAPE, "k beyond 65536");
+  if (!H || !U) return fail(MXQ_ERR_INVALID_ARG, "H or U is NULL");
+  if (!aligned(H, 16) || !aligned(U, 16) || (perm && !aligned(perm, 4)))
+    return fail(MXQ_ERR_ALIGN, "H or U not 16-byte, or perm not 4-byte aligned");
+  const size_t need = mxq::gptq_factor_workspace(k);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(MXQ_ERR_ALIGN, "workspace not 16-byte aligned");
+  return cuda_status(mxq::launch_gptq_factor(H, k, block, perm, damp, U, workspace,
+                                             (cudaStream_t)stream),
+                     "GPTQ factor");
+}
+
+namespace {
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+mxq_status check_gptq_params(const mxq_params* p, int64_t n, int64_t k) {
+  mxq_status s = check_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (p->fmt != MXQ_FMT_NVFP4 && p->fmt != MXQ_FMT_INT4)
+    return fail(MXQ_ERR_UNSUPPORTED, "GPTQ: NVFP4 or INT4 elements (E4M3 tiles: mxq_gptq_tiles)");
+  return MXQ_OK;
+}
+}  // namespace
+
+size_t mxq_gptq_order_workspace(int64_t n, int64_t k, const mxq_params* p) {
+  if (n <= 0 || k <= 0 || !p || p->block <= 0) return 0;
+  return round256((size_t)n * (size_t)(k / 2)) + round256((size_t)n * (size_t)(k / p->block)) +
+         round256((size_t)(k / p->block) * sizeof(double));
+}
+
+mxq_status mxq_gptq_order(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                          const float* h, const mxq_params* p, int32_t* perm, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  mxq_status s = check_matrix(W, dtype, n, k, ld, "W");
+  if (s != MXQ_OK) return s;
+  s = check_gptq_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (k == 0) return MXQ_OK;
+  if (k / p->block > mxq::gptq_sort_max())
+    return fail(MXQ_ERR_SHAPE, "more than %d blocks per row", mxq::gptq_sort_max());
+  if (!h || !perm) return fail(MXQ_ERR_INVALID_ARG, "h or perm is NULL");
+  if (!aligned(h, 16) || !aligned(perm, 4))
+    return fail(MXQ_ERR_ALIGN, "h not 16-byte or perm not 4-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (n == 0) {
+    std::vector<int32_t> id((size_t)(k / p->block));
+    for (size_t i = 0; i < id.size(); ++i) id[i] = (int32_t)i;
+    return cuda_status(cudaMemcpyAsync(perm, id.data(), id.size() * sizeof(int32_t),
+                                       cudaMemcpyHostToDevice, st),
+                       "perm copy");
+  }
+  const size_t need = mxq_gptq_order_workspace(n, k, p);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(MXQ_ERR_ALIGN, "workspace not 16-byte aligned");
+  char* ws = (char*)workspace;
+  uint8_t* codes = (uint8_t*)ws;
+  uint8_t* scales = codes + round256((size_t)n * (size_t)(k / 2));
+  double* loss = (double*)(scales + round256((size_t)n * (size_t)(k / p->block)));
+  s = mxq_quantize(W, dtype, n, k, ld, h, p, codes, scales, stream);
+  if (s != MXQ_OK) return s;
+  mxq::GptqArgs g{};
+  g.W = W;
+  g.dtype = dtype;
+  g.n = n;
+  g.k = k;
+  g.ld = ld;
+  g.h = h;
+  g.fmt = p->fmt;
+  g.block = p->block;
+  g.scale_fmt = p->scale_fmt;
+  return cuda_status(mxq::launch_gptq_order(g, codes, scales, loss, perm, st), "GPTQ order");
+}
+
+size_t mxq_gptq_workspace(int64_t n, int64_t k) {
+  return n > 0 && k > 0 ? mxq::gptq_sweep_workspace(n, k) : 0;
+}
+
+mxq_status mxq_gptq(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                    const float* h, const float* U, const int32_t* perm, const mxq_params* p,
+                    void* codes, void* scales, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  mxq_status s = check_matrix(W, dtype, n, k, ld, "W");
+  if (s != MXQ_OK) return s;
+  s = check_gptq_params(p, n, k);
+  if (s != MXQ_OK) return s;
+  if (n == 0 || k == 0) return MXQ_OK;
+  if (n > 0x7fffffff / 8) return fail(MXQ_ERR_SHAPE, "n beyond 2^28");
+  if (!U || !codes || !scales) return fail(MXQ_ERR_INVALID_ARG, "U, codes or scales is NULL");
+  if (!aligned(U, 16) || !aligned(codes, 16) || (perm && !aligned(perm, 4)))
+    return fail(MXQ_ERR_ALIGN, "U or codes not 16-byte, or perm not 4-byte aligned");
+  if (p->mode == MXQ_HOPT) {
+    if (!h) return fail(MXQ_ERR_INVALID_ARG, "H-optimal needs h");
+    if (!aligned(h, 16)) return fail(MXQ_ERR_ALIGN, "h not 16-byte aligned");
+  }
+  const size_t need = mxq::gptq_sweep_workspace(n, k);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(MXQ_ERR_ALIGN, "workspace not 16-byte aligned");
+  mxq::GptqArgs g{};
+  g.W = W;
+  g.dtype = dtype;
+  g.n = n;
+  g.k = k;
+  g.ld = ld;
+  g.h = p->mode == MXQ_HOPT ? h : nullptr;
+  g.U = U;
+  g.perm = perm;
+  g.fmt = p->fmt;
+  g.mode = p->mode;
+  g.block = p->block;
+  g.window = p->window;
+  g.scale_fmt = p->scale_fmt;
+  g.codes = codes;
+  g.scales = scales;
+  g.workspace = workspace;
+  return cuda_status(mxq::launch_gptq_sweep(g, (cudaStream_t)stream), "GPTQ sweep");
 }
 
 size_t mxq_output_error_workspace(int64_t m, int64_t n) {

@@ -1,0 +1,748 @@
+// mxq_gptq_full.cu -- GPTQ with the block quantizer as its inner step (qwantize "Results",
+// "GPTQ Quantization": the GPTQ block is the quantization block; sequential and ordered
+// variants; the algorithm is Frantar et al. 2022, Algorithm 1, in its Cholesky form).
+//
+// Three stages, each its own entry point:
+//   factor  U = upper Cholesky factor of the damped H^-1, H's rows and columns in sweep
+//           order (a block permutation for the ordered variant), in float64, rounded to
+//           float32 once. With J the order reversal, J H J = L L^T gives H^-1 = U^T U with
+//           U = J L^-1 J, so one blocked Cholesky and one blocked triangular inverse (64 x 64
+//           tiles, float64 on the CUDA cores) replace GPTQ's inverse-then-Cholesky.
+//   order   (ordered variant) the Hessian-weighted loss of every column block under the
+//           plain quantizer, and the blocks sorted by descending loss.
+//   sweep   rows are independent. Positions are processed in panels of up to 64: one warp
+//           per row searches each block's scale exactly on its current weights (every
+//           candidate's error in double, element order, lowest code on ties), quantises
+//           the block's columns one after another with the in-block updates, and applies
+//           each block's product to the panel's later blocks; a tiled kernel then applies
+//           the panel's block products to every later position of every row.
+// Every float32 step follows the definition's operation order: in-block updates
+// w -= fl32(err U), past the block acc = fma(err_j, U_j, acc) over the block's columns in
+// order, then one subtraction.
+#include "mxq_common.cuh"
+#include "mxq_gridk.cuh"
+#include "mxq_internal.h"
+
+#include <cublas_v2.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <mutex>
+
+namespace mxq {
+namespace {
+
+// ======================================================================================
+// factor
+// ======================================================================================
+constexpr int kNB = 64;                  // tile edge of the blocked factorisation
+constexpr int kTLd = kNB + 1;            // padded shared-memory row (doubles)
+constexpr int kFThreads = 256;
+constexpr size_t kTwoTiles = 2 * kNB * kTLd * sizeof(double);
+
+struct FactorArgs {
+  const float* H;        // [k][k]
+  int64_t k, kp;         // order, padded to a multiple of 64
+  int B;                 // block of the permutation
+  const int32_t* perm;   // [k / B] or null
+  double* A;             // [kp][kp]: J H J + lambda I, then L (lower tiles)
+  double* M;             // [kp][kp]: L^-1 (lower tiles)
+  double* scal;          // [0] lambda
+  float* U;              // [k][k]
+};
+
+// Column of sweep position pos; a block index outside 0 .. k/B - 1 is clamped into range
+// (an invalid permutation gives a meaningless result, never an out-of-bounds access).
+__device__ __forceinline__ int64_t perm_col(const FactorArgs& a, int64_t pos) {
+  if (!a.perm) return pos;
+  const int64_t b = min(max((int64_t)a.perm[pos / a.B], (int64_t)0), a.k / a.B - 1);
+  return b * a.B + pos % a.B;
+}
+
+// lambda = damp * mean(diag H), 1 when that is not positive; fixed-order reduction.
+__global__ void __launch_bounds__(kFThreads)
+k_factor_lambda(const float* __restrict__ H, int64_t k, double damp, double* scal) {
+  __shared__ double part[kFThreads];
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < k; i += kFThreads) s += (double)H[i * k + i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = kFThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double lam = damp * (part[0] / (double)k);
+    scal[0] = lam > 0.0 ? lam : 1.0;
+  }
+}
+
+// A_ij = H~_{k-1-i, k-1-j} (+ lambda on the diagonal), H~ = sym(H) in sweep order; the
+// padding beyond k is the identity.
+__global__ void k_factor_load(FactorArgs a) {
+  const double lam = a.scal[0];
+  const int64_t total = a.kp * a.kp;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / a.kp, j = e % a.kp;
+    double v;
+    if (i >= a.k || j >= a.k) {
+      v = i == j ? 1.0 : 0.0;
+    } else {
+      const int64_t p = perm_col(a, a.k - 1 - i), q = perm_col(a, a.k - 1 - j);
+      v = 0.5 * ((double)a.H[p * a.k + q] + (double)a.H[q * a.k + p]);
+      if (i == j) v += lam;
+    }
+    a.A[e] = v;
+  }
+}
+
+__device__ __forceinline__ void load_tile(double* s, const double* g, int64_t ld) {
+  for (int e = threadIdx.x; e < kNB * kNB; e += blockDim.x)
+    s[(e / kNB) * kTLd + e % kNB] = g[(int64_t)(e / kNB) * ld + e % kNB];
+}
+__device__ __forceinline__ void store_tile(double* g, const double* s, int64_t ld) {
+  for (int e = threadIdx.x; e < kNB * kNB; e += blockDim.x)
+    g[(int64_t)(e / kNB) * ld + e % kNB] = s[(e / kNB) * kTLd + e % kNB];
+}
+
+// Cholesky of the diagonal tile p, in place (lower; the upper part set to 0).
+__global__ void __launch_bounds__(kFThreads) k_potrf(double* A, int64_t kp, int p) {
+  __shared__ double T[kNB * kTLd];
+  double* g = A + (int64_t)p * kNB * kp + (int64_t)p * kNB;
+  load_tile(T, g, kp);
+  __syncthreads();
+  const int t = threadIdx.x;
+  for (int j = 0; j < kNB; ++j) {
+    const double d = sqrt(T[j * kTLd + j]);
+    __syncthreads();
+    if (t == 0) T[j * kTLd + j] = d;
+    for (int i = j + 1 + t; i < kNB; i += kFThreads) T[i * kTLd + j] /= d;
+    __syncthreads();
+    const int m = kNB - 1 - j;
+    for (int e = t; e < m * m; e += kFThreads) {
+      const int i = j + 1 + e / m, l = j + 1 + e % m;
+      if (l <= i) T[i * kTLd + l] -= T[i * kTLd + j] * T[l * kTLd + j];
+    }
+    __syncthreads();
+  }
+  for (int e = t; e < kNB * kNB; e += kFThreads)
+    if (e % kNB > e / kNB) T[(e / kNB) * kTLd + e % kNB] = 0.0;
+  __syncthreads();
+  store_tile(g, T, kp);
+}
+
+// Tiles below the diagonal tile p: A_ip <- A_ip L_pp^-T (one row per thread, forward
+// substitution).
+__global__ void __launch_bounds__(kFThreads) k_trsm(double* A, int64_t kp, int p) {
+  extern __shared__ double sm[];
+  double* L = sm;
+  double* X = sm + kNB * kTLd;
+  const int i = p + 1 + blockIdx.x;
+  load_tile(L, A + (int64_t)p * kNB * kp + (int64_t)p * kNB, kp);
+  double* g = A + (int64_t)i * kNB * kp + (int64_t)p * kNB;
+  load_tile(X, g, kp);
+  __syncthreads();
+  if (threadIdx.x < kNB) {
+    double* x = X + threadIdx.x * kTLd;
+    for (int c = 0; c < kNB; ++c) {
+      double v = x[c];
+      for (int c2 = 0; c2 < c; ++c2) v -= x[c2] * L[c * kTLd + c2];
+      x[c] = v / L[c * kTLd + c];
+    }
+  }
+  __syncthreads();
+  store_tile(g, X, kp);
+}
+
+// C (4 x 4 per thread) = S1 S2^T over 64 terms; thread (ty, tx) owns rows ty + 16 a and
+// columns tx + 16 b.
+__device__ __forceinline__ void tile_mul_nt(const double* S1, const double* S2, double (&c)[4][4]) {
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+#pragma unroll 4
+  for (int kk = 0; kk < kNB; ++kk) {
+    double x[4], y[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) x[a] = S1[(ty + 16 * a) * kTLd + kk];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) y[b] = S2[(tx + 16 * b) * kTLd + kk];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
+  }
+}
+
+// C = S1 S2 over 64 terms (S2 read by rows).
+__device__ __forceinline__ void tile_mul_nn(const double* S1, const double* S2, double (&c)[4][4]) {
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+#pragma unroll 4
+  for (int kk = 0; kk < kNB; ++kk) {
+    double x[4], y[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) x[a] = S1[(ty + 16 * a) * kTLd + kk];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) y[b] = S2[kk * kTLd + tx + 16 * b];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
+  }
+}
+
+// Trailing update after panel p: A_ij -= L_ip L_jp^T for p < j <= i (lower tiles).
+__global__ void __launch_bounds__(kFThreads) k_syrk(double* A, int64_t kp, int p) {
+  extern __shared__ double sm[];
+  double* Li = sm;
+  double* Lj = sm + kNB * kTLd;
+  // blockIdx.x -> (ii, jj), jj <= ii
+  const int64_t idx = blockIdx.x;
+  int64_t ii = (int64_t)((sqrt(8.0 * (double)idx + 1.0) - 1.0) / 2.0);
+  while (ii * (ii + 1) / 2 > idx) --ii;
+  while ((ii + 1) * (ii + 2) / 2 <= idx) ++ii;
+  const int64_t jj = idx - ii * (ii + 1) / 2;
+  const int64_t i = p + 1 + ii, j = p + 1 + jj;
+  load_tile(Li, A + i * kNB * kp + (int64_t)p * kNB, kp);
+  load_tile(Lj, A + j * kNB * kp + (int64_t)p * kNB, kp);
+  __syncthreads();
+  double c[4][4] = {};
+  tile_mul_nt(Li, Lj, c);
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  double* g = A + i * kNB * kp + j * kNB;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) g[(int64_t)(ty + 16 * a) * kp + tx + 16 * b] -= c[a][b];
+}
+
+// Diagonal tiles of M = L^-1: one column per thread, forward substitution.
+__global__ void __launch_bounds__(kFThreads) k_trtri_diag(const double* A, double* M, int64_t kp) {
+  extern __shared__ double sm[];
+  double* L = sm;
+  double* X = sm + kNB * kTLd;
+  const int64_t j = blockIdx.x;
+  load_tile(L, A + j * kNB * kp + j * kNB, kp);
+  __syncthreads();
+  if (threadIdx.x < kNB) {
+    const int c = threadIdx.x;
+    for (int i = 0; i < kNB; ++i) {
+      double v = 0.0;
+      if (i == c) {
+        v = 1.0 / L[i * kTLd + i];
+      } else if (i > c) {
+        double s = 0.0;
+        for (int r = c; r < i; ++r) s += L[i * kTLd + r] * X[r * kTLd + c];
+        v = -s / L[i * kTLd + i];
+      }
+      X[i * kTLd + c] = v;
+    }
+  }
+  __syncthreads();
+  store_tile(M + j * kNB * kp + j * kNB, X, kp);
+}
+
+// Sub-diagonal d: M_ij = -M_ii sum_{kk=j}^{i-1} L_i,kk M_kk,j for i = j + d.
+__global__ void __launch_bounds__(kFThreads)
+k_trtri_step(const double* A, double* M, int64_t kp, int d) {
+  extern __shared__ double sm[];
+  double* S1 = sm;
+  double* S2 = sm + kNB * kTLd;
+  const int64_t j = blockIdx.x, i = j + d;
+  double c[4][4] = {};
+  for (int64_t kk = j; kk < i; ++kk) {
+    __syncthreads();
+    load_tile(S1, A + i * kNB * kp + kk * kNB, kp);
+    load_tile(S2, M + kk * kNB * kp + j * kNB, kp);
+    __syncthreads();
+    tile_mul_nn(S1, S2, c);
+  }
+  __syncthreads();
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) S2[(ty + 16 * a) * kTLd + tx + 16 * b] = c[a][b];
+  load_tile(S1, M + i * kNB * kp + i * kNB, kp);
+  __syncthreads();
+  double r[4][4] = {};
+  tile_mul_nn(S1, S2, r);
+  double* g = M + i * kNB * kp + j * kNB;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) g[(int64_t)(ty + 16 * a) * kp + tx + 16 * b] = -r[a][b];
+}
+
+// U_pq = fl32(M_{k-1-p, k-1-q}) for q >= p, else 0.
+__global__ void k_factor_store(FactorArgs a) {
+  const int64_t total = a.k * a.k;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t p = e / a.k, q = e % a.k;
+    a.U[e] = q >= p ? (float)a.M[(a.k - 1 - p) * a.kp + (a.k - 1 - q)] : 0.0f;
+  }
+}
+
+}  // namespace
+
+size_t gptq_factor_workspace(int64_t k) {
+  const int64_t kp = (k + kNB - 1) / kNB * kNB;
+  return 256 + 2 * (size_t)kp * (size_t)kp * sizeof(double);
+}
+
+cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* perm,
+                               double damp, float* U, void* ws, cudaStream_t st) {
+  static const bool attrs = [] {
+    bool ok = true;
+    for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_trtri_diag,
+                          (const void*)k_trtri_step})
+      ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kTwoTiles) == cudaSuccess;
+    return ok;
+  }();
+  if (!attrs) return cudaErrorInvalidConfiguration;
+  const int64_t kp = (k + kNB - 1) / kNB * kNB, nt = kp / kNB;
+  char* w = (char*)ws;
+  FactorArgs a{H, k, kp, B, perm, (double*)(w + 256), (double*)(w + 256) + kp * kp,
+               (double*)w, U};
+  const int gs = sm_count() * 8;
+  k_factor_lambda<<<1, kFThreads, 0, st>>>(H, k, damp, a.scal);
+  k_factor_load<<<gs, 256, 0, st>>>(a);
+  for (int p = 0; p < nt; ++p) {
+    k_potrf<<<1, kFThreads, 0, st>>>(a.A, kp, p);
+    const int64_t m = nt - 1 - p;
+    if (m > 0) {
+      k_trsm<<<(unsigned)m, kFThreads, kTwoTiles, st>>>(a.A, kp, p);
+      k_syrk<<<(unsigned)(m * (m + 1) / 2), kFThreads, kTwoTiles, st>>>(a.A, kp, p);
+    }
+  }
+  k_trtri_diag<<<(unsigned)nt, kFThreads, kTwoTiles, st>>>(a.A, a.M, kp);
+  for (int d = 1; d < nt; ++d)
+    k_trtri_step<<<(unsigned)(nt - d), kFThreads, kTwoTiles, st>>>(a.A, a.M, kp, d);
+  k_factor_store<<<gs, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+// ======================================================================================
+// sweep
+// ======================================================================================
+namespace {
+
+constexpr int kPanel = 64;               // positions per panel
+constexpr int kPanelWarps = 8;           // rows per panel CTA (one warp each)
+constexpr int kTrailThreads = 256;       // 64 rows x 64 positions per trailing CTA
+
+struct SweepArgs {
+  const char* W;
+  int64_t n, k, ld_bytes;
+  int bf16;
+  const float* h;
+  const float* U;        // [k][k], sweep order
+  const int32_t* perm;   // [k / B] or null
+  int window;
+  float* Wc;             // [n][k] working weights, sweep order
+  float* Err;            // [n][kPanel] the panel's residuals
+  uint8_t* codes;        // [n][k / 2]
+  uint8_t* scales;       // [n][k / B]
+};
+
+template <int B>
+__device__ __forceinline__ int64_t pos_col(const SweepArgs& a, int64_t pos) {
+  if (!a.perm) return pos;
+  const int64_t b = min(max((int64_t)a.perm[pos / B], (int64_t)0), a.k / B - 1);
+  return b * B + pos % B;
+}
+
+template <int B>
+__global__ void k_sweep_init(SweepArgs a) {
+  const int64_t total = a.n * a.k;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / a.k, pos = e % a.k;
+    const int64_t c = pos_col<B>(a, pos);
+    const char* row = a.W + r * a.ld_bytes;
+    a.Wc[e] = a.bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[c])
+                     : reinterpret_cast<const float*>(row)[c];
+  }
+}
+
+// Element step of the definition at scale t = {s, r_hi, r_lo}: the magnitude code q and
+// fl32(s g(q)) for a = |w| (q = 0 for a zero scale).
+template <int ELEM>
+__device__ __forceinline__ int elem_project(float a, float4 t, float& wq_abs) {
+  if (t.x == 0.0f) {
+    wq_abs = 0.0f;
+    return 0;
+  }
+  const float2 z = quot2(make_float2(a, 0.0f), t);
+  const float g = elem_values<ELEM>(z).x;
+  wq_abs = __fmul_rn(t.x, g);
+  if constexpr (ELEM == kElemE2M1) return (int)(e2m1x2_rn(z.x, 0.0f) & 7u);
+  else return (int)g;
+}
+
+// The definition's candidate error sum_j c_j (w_j - wq_j)^2: double, element order,
+// each operation rounded once.
+template <int B, int ELEM, bool HOPT>
+__device__ __forceinline__ double exact_error(const float* wb, const float* cw, float4 t) {
+  double e = 0.0;
+#pragma unroll 4
+  for (int j = 0; j < B; ++j) {
+    float wq_abs;
+    elem_project<ELEM>(fabsf(wb[j]), t, wq_abs);
+    const double d = __dsub_rn((double)wb[j], (double)copysignf(wq_abs, wb[j]));
+    const double c = HOPT ? (double)cw[j] : 1.0;
+    e = __dadd_rn(e, __dmul_rn(c, __dmul_rn(d, d)));
+  }
+  return e;
+}
+
+// One warp per row; lane l holds panel positions 2l and 2l + 1.
+template <int B, int ELEM, int MODE>
+__global__ void __launch_bounds__(kPanelWarps * 32)
+k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S) {
+  __shared__ float4 tab[256];
+  __shared__ float Us[kPanel][kPanel + 1];
+  __shared__ float hs[kPanel];
+  __shared__ float wb[kPanelWarps][32];
+  __shared__ float errs[kPanelWarps][32];
+  for (int c = threadIdx.x; c < T.ncodes; c += blockDim.x) tab[c] = T.c[c];
+  for (int e = threadIdx.x; e < kPanel * kPanel; e += blockDim.x) {
+    const int i = e / kPanel, j = e % kPanel;
+    Us[i][j] = (i < S && j < S) ? a.U[(p0 + i) * a.k + p0 + j] : 0.0f;
+  }
+  for (int i = threadIdx.x; i < kPanel; i += blockDim.x)
+    hs[i] = (MODE == 2 && i < S) ? a.h[pos_col<B>(a, p0 + i)] : 1.0f;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t r = (int64_t)blockIdx.x * kPanelWarps + wid;
+  if (r >= a.n) return;
+  const int64_t kb = a.k / B;
+  float* wrow = a.Wc + r * a.k + p0;
+  const bool live = 2 * lane < S;
+  float2 w = live ? *reinterpret_cast<const float2*>(wrow + 2 * lane) : make_float2(0.f, 0.f);
+  float2 err2 = make_float2(0.f, 0.f);
+  uint32_t nib = 0;                       // the lane's two nibbles
+  for (int bb = 0; bb * B < S; ++bb) {
+    const int q0 = bb * B;                // the block's first panel position
+    const bool mine = 2 * lane >= q0 && 2 * lane < q0 + B;
+    if (mine) {
+      wb[wid][2 * lane - q0] = w.x;
+      wb[wid][2 * lane - q0 + 1] = w.y;
+    }
+    __syncwarp();
+    float amax = 0.0f;
+#pragma unroll 4
+    for (int j = 0; j < B; ++j) amax = fmaxf(amax, fabsf(wb[wid][j]));
+    const int c0 = naive_code<ELEM>(amax, tab, T.ncodes, T.sfmt);
+    int cbest = c0;
+    if (MODE != 0) {
+      int lo, hi;
+      grid_window(tab, T.ncodes, T.first, c0, a.window, lo, hi);
+      double be = __longlong_as_double(0x7ff0000000000000LL);   // +inf
+      int bc = 0x7fffffff;
+      for (int c = lo + lane; c <= hi; c += 32) {
+        const double e = exact_error<B, ELEM, MODE == 2>(wb[wid], hs + q0, tab[c]);
+        if (e < be) { be = e; bc = c; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double oe = __shfl_xor_sync(kFull, be, o);
+        const int oc = __shfl_xor_sync(kFull, bc, o);
+        if (oe < be || (oe == be && oc < bc)) { be = oe; bc = oc; }
+      }
+      cbest = bc == 0x7fffffff ? lo : bc;
+    }
+    const float4 t = tab[cbest];
+    const int64_t blk = pos_col<B>(a, p0 + q0) / B;   // the block's index in W
+    if (lane == 0) a.scales[r * kb + blk] = (uint8_t)cbest;
+    // the block's columns, one after another
+#pragma unroll 1
+    for (int j = 0; j < B; ++j) {
+      const int q = q0 + j;
+      const int owner = q >> 1;
+      float err = 0.0f;
+      if (lane == owner) {
+        const float wv = (q & 1) ? w.y : w.x;
+        float wq_abs;
+        const int code = elem_project<ELEM>(fabsf(wv), t, wq_abs);
+        const uint32_t neg = __float_as_uint(wv) >> 31;
+        const uint32_t nb = ELEM == kElemE2M1 ? ((neg << 3) | (uint32_t)code)
+                                              : ((uint32_t)(neg ? -code : code) & 15u);
+        nib |= nb << (4 * (q & 1));
+        err = __fdiv_rn(__fsub_rn(wv, copysignf(wq_abs, wv)), Us[q][q]);
+        if (q & 1) err2.y = err; else err2.x = err;
+        errs[wid][j] = err;
+      }
+      err = __shfl_sync(kFull, err, owner);
+      // in-block updates of the later columns: w -= fl32(err U)
+      if (mine) {
+        const int qa = 2 * lane, qb = 2 * lane + 1;
+        if (qa > q) w.x = __fsub_rn(w.x, __fmul_rn(err, Us[q][qa]));
+        if (qb > q) w.y = __fsub_rn(w.y, __fmul_rn(err, Us[q][qb]));
+      }
+    }
+    __syncwarp();
+    // the block's product into the panel's later blocks: acc = sum_j fma, one subtraction
+    if (live && 2 * lane >= q0 + B) {
+      float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll 4
+      for (int j = 0; j < B; ++j) {
+        const float e = errs[wid][j];
+        acc0 = __fmaf_rn(e, Us[q0 + j][2 * lane], acc0);
+        acc1 = __fmaf_rn(e, Us[q0 + j][2 * lane + 1], acc1);
+      }
+      w.x = __fsub_rn(w.x, acc0);
+      w.y = __fsub_rn(w.y, acc1);
+    }
+    __syncwarp();
+  }
+  if (live) {
+    const int64_t c = pos_col<B>(a, p0 + 2 * lane);    // even: both nibbles share a byte
+    a.codes[r * (a.k / 2) + c / 2] = (uint8_t)nib;
+    *reinterpret_cast<float2*>(a.Err + r * kPanel + 2 * lane) = err2;
+  }
+}
+
+// Later positions p >= p0 + S: for each block of the panel (in order)
+// acc = sum_j fma(err_j, U[j][p], acc) over the block's columns, then w -= acc.
+// CTA: 64 rows x 64 positions; thread: 4 rows x 4 consecutive positions.
+template <int B>
+__global__ void __launch_bounds__(kTrailThreads)
+k_gptq_trailing(SweepArgs a, int64_t p0, int S) {
+  __shared__ float Es[64][kPanel + 1];
+  __shared__ __align__(16) float Ut[kPanel][64];
+  const int64_t pstart = p0 + S;
+  const int64_t c0 = pstart + (int64_t)blockIdx.x * 64;
+  const int64_t r0 = (int64_t)blockIdx.y * 64;
+  for (int e = threadIdx.x; e < 64 * kPanel; e += kTrailThreads) {
+    const int i = e / kPanel, j = e % kPanel;
+    Es[i][j] = (r0 + i < a.n && j < S) ? a.Err[(r0 + i) * kPanel + j] : 0.0f;
+  }
+  for (int e = threadIdx.x; e < kPanel * 16; e += kTrailThreads) {
+    const int j = e / 16, g = e % 16;
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < S && c0 + 4 * g < a.k)
+      u = *reinterpret_cast<const float4*>(a.U + (p0 + j) * a.k + c0 + 4 * g);
+    *reinterpret_cast<float4*>(&Ut[j][4 * g]) = u;
+  }
+  __syncthreads();
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const int64_t col = c0 + 4 * tx;
+  if (col >= a.k) return;
+  float4 w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + 4 * ty + i;
+    w[i] = r < a.n ? *reinterpret_cast<const float4*>(a.Wc + r * a.k + col)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int q0 = 0; q0 < S; q0 += B) {
+    float4 acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int j = 0; j < B; ++j) {
+      const float4 u = *reinterpret_cast<const float4*>(&Ut[q0 + j][4 * tx]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float e = Es[4 * ty + i][q0 + j];
+        acc[i].x = __fmaf_rn(e, u.x, acc[i].x);
+        acc[i].y = __fmaf_rn(e, u.y, acc[i].y);
+        acc[i].z = __fmaf_rn(e, u.z, acc[i].z);
+        acc[i].w = __fmaf_rn(e, u.w, acc[i].w);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      w[i].x = __fsub_rn(w[i].x, acc[i].x);
+      w[i].y = __fsub_rn(w[i].y, acc[i].y);
+      w[i].z = __fsub_rn(w[i].z, acc[i].z);
+      w[i].w = __fsub_rn(w[i].w, acc[i].w);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + 4 * ty + i;
+    if (r < a.n) *reinterpret_cast<float4*>(a.Wc + r * a.k + col) = w[i];
+  }
+}
+
+template <int B, int ELEM>
+cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cudaStream_t st) {
+  k_sweep_init<B><<<sm_count() * 8, 256, 0, st>>>(a);
+  const unsigned prow = (unsigned)((a.n + kPanelWarps - 1) / kPanelWarps);
+  for (int64_t p0 = 0; p0 < a.k; p0 += kPanel) {
+    const int S = (int)(a.k - p0 < kPanel ? a.k - p0 : kPanel);
+    if (mode == 0) k_gptq_panel<B, ELEM, 0><<<prow, kPanelWarps * 32, 0, st>>>(a, T, p0, S);
+    else if (mode == 1) k_gptq_panel<B, ELEM, 1><<<prow, kPanelWarps * 32, 0, st>>>(a, T, p0, S);
+    else k_gptq_panel<B, ELEM, 2><<<prow, kPanelWarps * 32, 0, st>>>(a, T, p0, S);
+    const int64_t rest = a.k - p0 - S;
+    if (rest > 0) {
+      const dim3 grid((unsigned)((rest + 63) / 64), (unsigned)((a.n + 63) / 64));
+      k_gptq_trailing<B><<<grid, kTrailThreads, 0, st>>>(a, p0, S);
+    }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gptq_sweep_workspace(int64_t n, int64_t k) {
+  return (size_t)n * (size_t)k * sizeof(float) + (size_t)n * kPanel * sizeof(float) + 256;
+}
+
+cudaError_t launch_gptq_sweep(const GptqArgs& g, cudaStream_t st) {
+  static const GridTable tables[4] = {make_grid_table(0), make_grid_table(1),
+                                      make_grid_table(2), make_grid_table(3)};
+  char* ws = (char*)g.workspace;
+  SweepArgs a{(const char*)g.W, g.n, g.k, g.ld * (g.dtype == 1 ? 2 : 4), g.dtype == 1, g.h,
+              g.U, g.perm, g.window, (float*)ws, (float*)(ws + (size_t)g.n * g.k * sizeof(float)),
+              (uint8_t*)g.codes, (uint8_t*)g.scales};
+  const GridTable& T = tables[g.scale_fmt];
+  if (g.fmt == 0) {
+    return g.block == 16 ? sweep_dispatch<16, kElemE2M1>(a, T, g.mode, st)
+                         : sweep_dispatch<32, kElemE2M1>(a, T, g.mode, st);
+  }
+  return g.block == 16 ? sweep_dispatch<16, kElemInt4>(a, T, g.mode, st)
+                       : sweep_dispatch<32, kElemInt4>(a, T, g.mode, st);
+}
+
+// ======================================================================================
+// order (ordered variant)
+// ======================================================================================
+namespace {
+
+constexpr int kLossThreads = 256;
+constexpr int kSortMax = 2048;           // blocks a single-CTA sort handles
+
+struct LossArgs {
+  const char* W;
+  int64_t n, k, ld_bytes;
+  int bf16, fmt, block;
+  const float* h;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  GridTable T;
+  double* loss;          // [k / B]
+};
+
+// loss_b = sum over rows and the block's columns of h_j (w_ij - w^_ij)^2 (double), one CTA
+// per block: each thread sums its rows' blocks (columns in order), then a fixed tree.
+__global__ void __launch_bounds__(kLossThreads) k_block_loss(LossArgs a) {
+  __shared__ double part[kLossThreads];
+  const int64_t b = blockIdx.x, kb = a.k / a.block;
+  double acc = 0.0;
+  for (int64_t r = threadIdx.x; r < a.n; r += kLossThreads) {
+    const float s = a.T.c[a.scales[r * kb + b]].x;
+    const char* row = a.W + r * a.ld_bytes;
+    double e = 0.0;
+    for (int j = 0; j < a.block; ++j) {
+      const int64_t c = b * a.block + j;
+      const float w = a.bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(row)[c])
+                             : reinterpret_cast<const float*>(row)[c];
+      const uint32_t nib = (a.codes[r * (a.k / 2) + c / 2] >> (4 * (c & 1))) & 15u;
+      float g;
+      if (a.fmt == 0) {
+        g = __half2float(__ushort_as_half((uint16_t)(e2m1x2_to_f16x2(nib & 7u) & 0xffffu)));
+        if (nib & 8u) g = -g;
+      } else {
+        g = (float)((nib & 8u) ? (int)nib - 16 : (int)nib);
+      }
+      const double d = __dsub_rn((double)w, (double)__fmul_rn(s, g));
+      e = __dadd_rn(e, __dmul_rn(__dmul_rn(d, d), (double)a.h[c]));
+    }
+    acc = __dadd_rn(acc, e);
+  }
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = kLossThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) a.loss[b] = part[0];
+}
+
+// perm = blocks by descending loss, the lower block first on equal loss (bitonic sort).
+__global__ void __launch_bounds__(1024) k_block_sort(const double* loss, int kb, int32_t* perm) {
+  __shared__ double key[kSortMax];
+  __shared__ int32_t idx[kSortMax];
+  int m = 1;
+  while (m < kb) m <<= 1;
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    key[i] = i < kb ? loss[i] : -__longlong_as_double(0x7ff0000000000000LL);
+    idx[i] = i < kb ? i : 0x7fffffff;
+  }
+  __syncthreads();
+  // "before(x, y)": x sorts first (larger loss, then smaller index)
+  for (int size = 2; size <= m; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < m; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const bool before_j = key[j] > key[i] || (key[j] == key[i] && idx[j] < idx[i]);
+          if (before_j == up) {
+            const double tk = key[i]; key[i] = key[j]; key[j] = tk;
+            const int32_t ti = idx[i]; idx[i] = idx[j]; idx[j] = ti;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < kb; i += blockDim.x) perm[i] = idx[i];
+}
+
+}  // namespace
+
+cudaError_t launch_gptq_order(const GptqArgs& g, const uint8_t* codes, const uint8_t* scales,
+                              double* loss, int32_t* perm, cudaStream_t st) {
+  static const GridTable tables[4] = {make_grid_table(0), make_grid_table(1),
+                                      make_grid_table(2), make_grid_table(3)};
+  const int64_t kb = g.k / g.block;
+  LossArgs a{(const char*)g.W, g.n, g.k, g.ld * (g.dtype == 1 ? 2 : 4), g.dtype == 1, g.fmt,
+             g.block, g.h, codes, scales, tables[g.scale_fmt], loss};
+  k_block_loss<<<(unsigned)kb, kLossThreads, 0, st>>>(a);
+  k_block_sort<<<1, 1024, 0, st>>>(loss, (int)kb, perm);
+  return cudaGetLastError();
+}
+
+int gptq_sort_max() { return kSortMax; }
+
+// ======================================================================================
+// the full Gram matrix H = X^T X / R (a plain GEMM: cuBLAS, bf16 in, float32 out)
+// ======================================================================================
+namespace {
+std::mutex g_blas_mu;
+cublasHandle_t g_blas[64] = {};
+}  // namespace
+
+cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t ld, float* H,
+                             cudaStream_t st, const char** why) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  cublasHandle_t hd;
+  {
+    std::lock_guard<std::mutex> lk(g_blas_mu);
+    if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
+      *why = "cublasCreate failed";
+      return cudaErrorUnknown;
+    }
+    hd = g_blas[dev];
+  }
+  const float alpha = (float)(1.0 / (double)rows), beta = 0.0f;
+  // column-major view: X^T is [cols x rows] with leading dimension ld; H = X^T (X^T)^T
+  cublasStatus_t s = cublasSetStream(hd, st);
+  if (s == CUBLAS_STATUS_SUCCESS)
+    s = cublasGemmEx(hd, CUBLAS_OP_N, CUBLAS_OP_T, (int)cols, (int)cols, (int)rows, &alpha, X,
+                     CUDA_R_16BF, (int)ld, X, CUDA_R_16BF, (int)ld, &beta, H, CUDA_R_32F,
+                     (int)cols, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+  if (s != CUBLAS_STATUS_SUCCESS) {
+    *why = "cublasGemmEx failed";
+    return cudaErrorUnknown;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mxq

@@ -13,6 +13,7 @@
 // G = fl32(sum / R) and h = diag(G). Only the B x B diagonal blocks of each 128 x 128 tile
 // are kept: the kernel is bound by reading X, the discarded products are free.
 //
+// Blocks of B = 16, 32 or 64 columns (64: the E4M3 tile width).
 // Warp roles (192 threads): warps 0-3 epilogue (tensor-memory lanes 32 (w % 4) ..), warp 4
 // TMA producer, warp 5 MMA issuer. Every wait is bounded: on timeout the CTA sets
 // `*err`, stops issuing, lets its copies and MMAs finish (bounded) and frees its tensor
@@ -282,10 +283,22 @@ k_gram_tc(const __grid_constant__ CUtensorMap tmap, GramParams P) {
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      float v[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * kGramCols + warp * 32), v);
+      const uint32_t lanes = (uint32_t)(warp * 32) << 16;
+      if constexpr (B == 64) {
+        // lanes 32 w .. 32 w + 31 all lie in diagonal block w / 2: its 64 columns
 #pragma unroll
-      for (int j = 0; j < B; ++j) acc[j] += (double)(B == 16 ? (upper ? v[16 + j] : v[j]) : v[j]);
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          float v[32];
+          tmem_ld32(tmem + lanes + (uint32_t)(buf * kGramCols + (warp / 2) * 64 + hlf * 32), v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[hlf * 32 + j] += (double)v[j];
+        }
+      } else {
+        float v[32];
+        tmem_ld32(tmem + lanes + (uint32_t)(buf * kGramCols + warp * 32), v);
+#pragma unroll
+        for (int j = 0; j < B; ++j) acc[j] += (double)(B == 16 ? (upper ? v[16 + j] : v[j]) : v[j]);
+      }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       mbar_arrive(&accempty[buf]);
     }
@@ -380,6 +393,11 @@ cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, i
                                              kGramSmem) == cudaSuccess;
     if (!set16) return cudaErrorInvalidConfiguration;
     k_gram_tc<16><<<grid, kGramThreads, kGramSmem, st>>>(map, P);
+  } else if (B == 64) {
+    static bool set64 = cudaFuncSetAttribute(k_gram_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kGramSmem) == cudaSuccess;
+    if (!set64) return cudaErrorInvalidConfiguration;
+    k_gram_tc<64><<<grid, kGramThreads, kGramSmem, st>>>(map, P);
   } else {
     static bool set32 = cudaFuncSetAttribute(k_gram_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kGramSmem) == cudaSuccess;

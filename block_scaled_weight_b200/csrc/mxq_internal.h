@@ -73,6 +73,37 @@ cudaError_t launch_outerr(const void* X, int64_t m, int64_t k, int64_t ldx, cons
                           int fmt, int scale_fmt, int block, double* sums, void* workspace,
                           cudaStream_t st);
 
+// ---- FP8-GPTQ on 64 x 64 tiles (mxq_gptq.cu) ---------------------------------------------
+cudaError_t launch_gptq_prepare(const float* G, int64_t nblocks, double damp, float* U,
+                                cudaStream_t st);
+cudaError_t launch_gptq_tiles(const void* W, int dtype, int64_t n, int64_t k, int64_t ld,
+                              const float* U, const float* scales, uint8_t* codes,
+                              cudaStream_t st);
+
+// ---- GPTQ with the block quantizer (mxq_gptq_full.cu) ----------------------------------
+struct GptqArgs {
+  const void* W;
+  int dtype;
+  int64_t n, k, ld;
+  const float* h;          // HOPT search weights (and the ordered variant's loss weights)
+  const float* U;          // [k][k] factor in sweep order
+  const int32_t* perm;     // [k / block] block order, or null
+  int fmt, mode, block, window, scale_fmt;
+  void* codes;
+  void* scales;
+  void* workspace;         // gptq_sweep_workspace(n, k) bytes
+};
+size_t gptq_factor_workspace(int64_t k);
+cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* perm,
+                               double damp, float* U, void* ws, cudaStream_t st);
+size_t gptq_sweep_workspace(int64_t n, int64_t k);
+cudaError_t launch_gptq_sweep(const GptqArgs& g, cudaStream_t st);
+int gptq_sort_max();
+cudaError_t launch_gptq_order(const GptqArgs& g, const uint8_t* codes, const uint8_t* scales,
+                              double* loss, int32_t* perm, cudaStream_t st);
+cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t ld, float* H,
+                             cudaStream_t st, const char** why);
+
 int sm_count();
 // Sets the per-thread text that mxq_last_error() returns.
 void set_error_text(const char* fmt, ...) __attribute__((format(printf, 1, 2)));

@@ -34,7 +34,10 @@ EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc
            "mxq_act_sqsum", "mxq_act_block_gram_workspace", "mxq_act_block_gram",
            "mxq_act_sqmean_finalize", "mxq_quantize", "mxq_quantize_gram", "mxq_project",
            "mxq_swizzled_scales_bytes", "mxq_swizzle_scales", "mxq_output_error_workspace",
-           "mxq_output_error", "mxq_dequant", "mxq_error_workspace",
+           "mxq_output_error", "mxq_gptq_prepare", "mxq_gptq_tiles", "mxq_act_gram",
+           "mxq_gptq_factor_workspace", "mxq_gptq_factor", "mxq_gptq_order_workspace",
+           "mxq_gptq_order", "mxq_gptq_workspace", "mxq_gptq", "mxq_dequant",
+           "mxq_error_workspace",
            "mxq_error", "mxq_metrics_from_sums", "mxq_status_string", "mxq_last_error")
 
 
@@ -70,6 +73,17 @@ _sig = {
     "mxq_output_error": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P,
                                         ctypes.POINTER(MxqParams), _P, _P, _SZ, _P]),
     "mxq_swizzle_scales": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "mxq_gptq_prepare": (ctypes.c_int, [_P, _I64, ctypes.c_double, _P, _P]),
+    "mxq_gptq_tiles": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "mxq_act_gram": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P]),
+    "mxq_gptq_factor_workspace": (_SZ, [_I64]),
+    "mxq_gptq_factor": (ctypes.c_int, [_P, _I64, _I32, _P, ctypes.c_double, _P, _P, _SZ, _P]),
+    "mxq_gptq_order_workspace": (_SZ, [_I64, _I64, ctypes.POINTER(MxqParams)]),
+    "mxq_gptq_order": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(MxqParams),
+                                      _P, _P, _SZ, _P]),
+    "mxq_gptq_workspace": (_SZ, [_I64, _I64]),
+    "mxq_gptq": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
+                                ctypes.POINTER(MxqParams), _P, _P, _P, _SZ, _P]),
     "mxq_dequant": (ctypes.c_int, [_P, _P, ctypes.POINTER(MxqParams), _I64, _I64, _P, _P]),
     "mxq_error_workspace": (_SZ, [_I64, _I64]),
     "mxq_error": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
@@ -267,6 +281,93 @@ def mxq_project(w: torch.Tensor, fmt: str, scale: float, *, scale_fmt="e4m3", q=
     _check(_lib.mxq_project(_ptr(w), w.numel(), FMT[fmt], SCALE[scale_fmt], float(scale),
                             _ptr(q), _stream(stream, w.device)), "mxq_project")
     return q
+
+
+def mxq_gptq_prepare(G: torch.Tensor, damp: float = 0.01, *, U=None, stream=None) -> torch.Tensor:
+    """U [nb, 64, 64] float32: the upper Cholesky factor of the inverse of each damped Gram
+    block G [nb, 64, 64] (float32, from mxq_act_block_gram with block 64)."""
+    nb = G.shape[0]
+    if U is None:
+        U = torch.empty((nb, 64, 64), dtype=torch.float32, device=G.device)
+    _check(_lib.mxq_gptq_prepare(_ptr(G), nb, float(damp), _ptr(U), _stream(stream, G.device)),
+           "mxq_gptq_prepare")
+    return U
+
+
+def mxq_gptq_tiles(W: torch.Tensor, U: torch.Tensor, scales: torch.Tensor, *, codes=None,
+                   stream=None) -> torch.Tensor:
+    """E4M3 codes [n, k] (uint8, sign << 7 | code) of the tile GPTQ sweep of W [n, k] at the
+    tile scales [n/64, k/64] (float32) with the factors U [k/64, 64, 64]."""
+    n, k = W.shape
+    if codes is None:
+        codes = torch.empty((n, k), dtype=torch.uint8, device=W.device)
+    _check(_lib.mxq_gptq_tiles(_ptr(W), _dtype(W), n, k, _ld(W), _ptr(U), _ptr(scales),
+                               _ptr(codes), _stream(stream, W.device)), "mxq_gptq_tiles")
+    return codes
+
+
+def mxq_act_gram(X: torch.Tensor, H: torch.Tensor | None = None, *, stream=None) -> torch.Tensor:
+    """H = X^T X / R [K, K] float32 of bf16 X [R, K] (GPTQ's Hessian up to a factor)."""
+    R, K = X.shape
+    if H is None:
+        H = torch.empty(K, K, dtype=torch.float32, device=X.device)
+    _check(_lib.mxq_act_gram(_ptr(X), _dtype(X), R, K, _ld(X), _ptr(H), _stream(stream, X.device)),
+           "mxq_act_gram")
+    return H
+
+
+def mxq_gptq_factor_workspace(k: int) -> int:
+    return int(_lib.mxq_gptq_factor_workspace(k))
+
+
+def mxq_gptq_order_workspace(n: int, k: int, p: MxqParams) -> int:
+    return int(_lib.mxq_gptq_order_workspace(n, k, ctypes.byref(p)))
+
+
+def mxq_gptq_workspace(n: int, k: int) -> int:
+    return int(_lib.mxq_gptq_workspace(n, k))
+
+
+def mxq_gptq_factor(H: torch.Tensor, block: int, perm: torch.Tensor | None = None,
+                    damp: float = 0.01, *, U=None, workspace=None, stream=None) -> torch.Tensor:
+    """U [K, K] float32: the upper Cholesky factor of the damped H^-1 in sweep order."""
+    K = H.shape[0]
+    if U is None:
+        U = torch.empty(K, K, dtype=torch.float32, device=H.device)
+    ws = _workspace(mxq_gptq_factor_workspace(K), H.device, workspace)
+    _check(_lib.mxq_gptq_factor(_ptr(H), K, block, _ptr(perm), float(damp), _ptr(U), _ptr(ws),
+                                ws.numel(), _stream(stream, H.device)), "mxq_gptq_factor")
+    return U
+
+
+def mxq_gptq_order(W: torch.Tensor, h: torch.Tensor, p: MxqParams, *, perm=None,
+                   workspace=None, stream=None) -> torch.Tensor:
+    """Ordered GPTQ's block sequence (int32 [k / block]): descending Hessian-weighted loss."""
+    n, k = W.shape
+    if perm is None:
+        perm = torch.empty(k // p.block, dtype=torch.int32, device=W.device)
+    ws = _workspace(mxq_gptq_order_workspace(n, k, p), W.device, workspace)
+    _check(_lib.mxq_gptq_order(_ptr(W), _dtype(W), n, k, _ld(W), _ptr(h), ctypes.byref(p),
+                               _ptr(perm), _ptr(ws), ws.numel(), _stream(stream, W.device)),
+           "mxq_gptq_order")
+    return perm
+
+
+def mxq_gptq(W: torch.Tensor, U: torch.Tensor, p: MxqParams, h: torch.Tensor | None = None,
+             perm: torch.Tensor | None = None, *, codes=None, scales=None, workspace=None,
+             stream=None):
+    """(codes, scales) of the GPTQ sweep of W [n, k] (layouts of mxq_quantize)."""
+    n, k = W.shape
+    cs, cd, ss, sd = output_shapes(p, n, k)
+    if codes is None:
+        codes = torch.empty(cs, dtype=cd, device=W.device)
+    if scales is None:
+        scales = torch.empty(ss, dtype=sd, device=W.device)
+    ws = _workspace(mxq_gptq_workspace(n, k), W.device, workspace)
+    _check(_lib.mxq_gptq(_ptr(W), _dtype(W), n, k, _ld(W), _ptr(h), _ptr(U), _ptr(perm),
+                         ctypes.byref(p), _ptr(codes), _ptr(scales), _ptr(ws), ws.numel(),
+                         _stream(stream, W.device)), "mxq_gptq")
+    return codes, scales
 
 
 def mxq_output_error(X: torch.Tensor, W: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,

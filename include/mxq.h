@@ -178,7 +178,7 @@ MXQ_API mxq_status mxq_act_sqmean_finalize(const double* partials, int64_t parts
  *
  *  X          device bf16 [rows, cols] row-major, leading dimension ld (elements); 16-byte
  *             aligned, ld * 2 % 16 == 0. (float32 X: MXQ_ERR_DTYPE.)
- *  block      B = 16 or 32; cols % B == 0.
+ *  block      B = 16, 32 or 64 (64: the E4M3 tile width, for the tile GPTQ); cols % B == 0.
  *  G          device float [cols/B][B][B], 16-byte aligned: G[b][i][j] =
  *             fl32(sum_r x_r,bB+i x_r,bB+j / rows) (the sum: float32 over at most 512 rows
  *             inside the tensor cores, then double); symmetric to within that rounding.
@@ -315,6 +315,110 @@ MXQ_API mxq_status mxq_output_error(const void* X, int64_t m, int64_t k, int64_t
                                     const void* W, int64_t n, int64_t ldw, const void* codes,
                                     const void* scales, const mxq_params* p, double* sums,
                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * FP8-GPTQ on 64 x 64 tiles ("quantization_algorithms.txt", section 1, the 64x64 tile
+ * scheme): E4M3 elements at fixed tile scales, the columns of every tile quantised one
+ * after another with each residual propagated through the inverse of the damped Gram
+ * matrix of the tile's 64 input dimensions (GPTQ's update in its Cholesky form).
+ *
+ * mxq_gptq_prepare: per column block b, H = (G_b + G_b^T) / 2 + lambda I with
+ * lambda = damp * mean(diag G_b) (1 when that mean is 0), and U the upper Cholesky factor
+ * of H^-1 (H^-1 = U^T U), computed in float64 and rounded to float32 once.
+ *  G        device float [nblocks][64][64], 16-byte aligned: the Gram blocks of
+ *           mxq_act_block_gram with block 64 (any scaling of them gives the same codes).
+ *  damp     relative damping, finite and >= 0 (GPTQ's customary value is 0.01).
+ *  U        device float [nblocks][64][64], 16-byte aligned; the strict lower triangle is
+ *           written as 0. A block whose damped H is not positive definite (impossible for
+ *           a Gram matrix) yields NaN entries.
+ *
+ * mxq_gptq_tiles: for every row r of every 64 x 64 tile (rows independent), columns
+ * c = 0 .. 63 in order: q = RNE_E4M3(fl32(|w_c| / s)) (code 0..126, 0 when s == 0),
+ * wq = +-fl32(s E4M3(q)) with the sign of w_c, err = fl32(fl32(w_c - wq) / U_cc),
+ * w_j = fl32(w_j - fl32(err U_cj)) for j > c; w starts as the tile's weights.
+ *  W        as for mxq_quantize (bf16 or float32), n % 64 == 0, k % 64 == 0.
+ *  U        device float [k/64][64][64], 16-byte aligned (mxq_gptq_prepare's output).
+ *  scales   device float [n/64][k/64], 4-byte aligned: the tile scales (e.g. those of
+ *           mxq_quantize with MXQ_FMT_E4M3), finite and >= 0.
+ *  codes    device uint8 [n, k], 16-byte aligned: sign << 7 | e4m3 code (the layout of
+ *           mxq_quantize's E4M3 codes; mxq_dequant and mxq_error read them with the same
+ *           scales).
+ *  Result: identical to the definition above evaluated in that order (every step a
+ *  separately rounded IEEE float32 operation), given the same U.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API mxq_status mxq_gptq_prepare(const float* G, int64_t nblocks, double damp, float* U,
+                                    void* stream);
+MXQ_API mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64_t k,
+                                  int64_t ld, const float* U, const float* scales,
+                                  uint8_t* codes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * GPTQ with the block quantizer as its inner step (qwantize "Results", "GPTQ
+ * Quantization": the GPTQ block is the quantization block; after a block is quantised its
+ * error is compensated in all remaining columns through the inverse Hessian; sequential
+ * order, or "ordered" -- blocks sorted by descending Hessian-weighted quantization loss).
+ * The algorithm is Frantar et al. 2022, Algorithm 1, in its Cholesky form.
+ *
+ * mxq_act_gram: H = X^T X / R, the full cols x cols Gram matrix (the GPTQ Hessian up to a
+ *  factor) of bf16 X [rows, cols] (ld as for mxq_act_sqmean), float32, row-major, 16-byte
+ *  aligned. A plain GEMM (cuBLAS; bf16 products, float32 accumulation in the library's
+ *  order): each entry is within rows * 2^-24 * (|X|^T |X|)_ij / rows of the exact value.
+ *
+ * mxq_gptq_factor: U [k][k] float32 (upper, the strict lower triangle written as 0), the
+ *  upper Cholesky factor of (H~ + lambda I)^-1, H~ = (H + H^T) / 2 with rows and columns in
+ *  sweep order (position t*block + j is column perm[t]*block + j; natural order when perm
+ *  is NULL), lambda = damp * mean(diag H) (1 when that mean is 0); computed in float64,
+ *  rounded to float32 once.
+ *   H       device float [k][k], 16-byte aligned.
+ *   block   the quantization block (16 or 32); k % block == 0; perm device int32 [k/block]
+ *           (a permutation of 0 .. k/block - 1; other values are clamped into range and
+ *           give a meaningless result) or NULL.
+ *   damp    finite, >= 0 (GPTQ's customary 0.01).
+ *   workspace  mxq_gptq_factor_workspace(k) bytes (two float64 k x k matrices, k rounded
+ *           up to a multiple of 64), 16-byte aligned.
+ *
+ * mxq_gptq_order: the ordered variant's block sequence. loss_b = sum over rows and the
+ *  block's columns of h_j (w_ij - w^_ij)^2 (float64) for the plain quantizer's result
+ *  (mxq_quantize with p and h); perm = the blocks by descending loss, the lower block first
+ *  on equal loss. k / block <= 2048.
+ *   W, p    as for mxq_quantize (p->fmt MXQ_FMT_NVFP4 or MXQ_FMT_INT4, block 16 or 32).
+ *   h       device float [k] (required: the loss weights; also the H-optimal search's).
+ *   perm    device int32 [k / block].
+ *   workspace  mxq_gptq_order_workspace(n, k, p) bytes, 16-byte aligned.
+ *
+ * mxq_gptq: the sweep. Rows are independent; for each row and each block position
+ *  t = 0 .. k/block - 1 (block b = perm[t], or t): the block's scale is the quantizer's pick
+ *  (p->mode, p->window, p->scale_fmt as for mxq_quantize) for the block's CURRENT weights;
+ *  then for its columns j in order, at position q = t*block + j:
+ *    code = the element projection at that scale, wq = +-fl32(s g(code)),
+ *    err_j = fl32(fl32(w - wq) / U[q][q]), w at the block's later positions q' -=
+ *    fl32(err_j U[q][q']);
+ *  then at every later position q': acc = 0, acc = fma(err_j, U[t*block + j][q'], acc) for
+ *  j = 0 .. block-1, w -= acc. Every step one IEEE float32 operation.
+ *   W       as for mxq_quantize; h as for mxq_quantize (H-optimal); U mxq_gptq_factor's
+ *           output for the same perm; codes / scales: mxq_quantize's layouts (original
+ *           column order).
+ *   workspace  mxq_gptq_workspace(n, k) bytes (the working weights, n x k float32),
+ *           16-byte aligned.
+ *  Result: identical to the definition above, including ties (each scale search scores
+ *  every candidate exactly in float64, element order; lowest code on equal errors).
+ * ------------------------------------------------------------------------------------ */
+MXQ_API mxq_status mxq_act_gram(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+                                int64_t ld, float* H, void* stream);
+MXQ_API size_t mxq_gptq_factor_workspace(int64_t k);
+MXQ_API mxq_status mxq_gptq_factor(const float* H, int64_t k, int32_t block,
+                                   const int32_t* perm, double damp, float* U, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+MXQ_API size_t mxq_gptq_order_workspace(int64_t n, int64_t k, const mxq_params* p);
+MXQ_API mxq_status mxq_gptq_order(const void* W, int32_t dtype, int64_t n, int64_t k,
+                                  int64_t ld, const float* h, const mxq_params* p,
+                                  int32_t* perm, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+MXQ_API size_t mxq_gptq_workspace(int64_t n, int64_t k);
+MXQ_API mxq_status mxq_gptq(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                            const float* h, const float* U, const int32_t* perm,
+                            const mxq_params* p, void* codes, void* scales, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /* Human-readable text for a status; the last failure's detail on this host thread. */
 MXQ_API const char* mxq_status_string(mxq_status s);

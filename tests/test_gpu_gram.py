@@ -42,7 +42,9 @@ def check_gram(orc, X, G, B):
 
 
 @pytest.mark.parametrize("rows,cols,B", [(64, 128, 16), (1000, 384, 16), (1000, 384, 32),
-                                         (777, 336, 16), (20000, 1024, 16), (5, 256, 32)])
+                                         (777, 336, 16), (20000, 1024, 16), (5, 256, 32),
+                                         (1000, 384, 64), (777, 320, 64), (20000, 1024, 64),
+                                         (5, 192, 64)])
 def test_gram_matches_oracle(mxq, orc, synth, rows, cols, B):
     X = synth.activations(rows, cols, 81, dtype=torch.bfloat16, device=DEV)
     G, h = mxq.mxq_act_block_gram(X, B, with_h=True)
@@ -73,7 +75,9 @@ def test_gram_rejects_float32_and_bad_blocks(mxq):
     with pytest.raises(mxq.MxqError):
         mxq.mxq_act_block_gram(Xb, 16)
     with pytest.raises(mxq.MxqError):
-        mxq.mxq_act_block_gram(torch.zeros(64, 128, dtype=torch.bfloat16, device=DEV), 64)
+        mxq.mxq_act_block_gram(torch.zeros(64, 128, dtype=torch.bfloat16, device=DEV), 48)
+    with pytest.raises(mxq.MxqError):
+        mxq.mxq_act_block_gram(torch.zeros(64, 96, dtype=torch.bfloat16, device=DEV), 64)
 
 
 # ---------------------------------------------------------------------------------------
