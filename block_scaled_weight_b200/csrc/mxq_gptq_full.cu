@@ -39,6 +39,7 @@ constexpr int kNB = 64;                  // tile edge of the blocked factorisati
 constexpr int kTLd = kNB + 1;            // padded shared-memory row (doubles)
 constexpr int kFThreads = 256;
 constexpr size_t kTwoTiles = 2 * kNB * kTLd * sizeof(double);
+constexpr int kPanelTiles = 4;           // tile columns per trailing update of the Cholesky
 
 struct FactorArgs {
   const float* H;        // [k][k]
@@ -106,171 +107,233 @@ __device__ __forceinline__ void store_tile(double* g, const double* s, int64_t l
     g[(int64_t)(e / kNB) * ld + e % kNB] = s[(e / kNB) * kTLd + e % kNB];
 }
 
-// Cholesky of the diagonal tile p, in place (lower; the upper part set to 0).
-__global__ void __launch_bounds__(kFThreads) k_potrf(double* A, int64_t kp, int p) {
-  __shared__ double T[kNB * kTLd];
+// Diagonal tile p: its Cholesky factor L_pp (lower, the upper part 0) into A and its
+// inverse M_pp into M. The elimination keeps the columns unscaled (step j: T_il -= T_ij T_lj
+// / T_jj over the trailing triangle, one barrier per step), and scales every column by
+// 1/sqrt of its pivot at the end. The inverse: four threads per column of M (consecutive
+// lanes), each summing every fourth term of the forward substitution, then two shuffles.
+__global__ void __launch_bounds__(kFThreads) k_potrf_inv(double* A, double* M, int64_t kp, int p) {
+  extern __shared__ double sm[];
+  __shared__ double dg[kNB], rdiag[kNB];
+  double* T = sm;
+  double* X = sm + kNB * kTLd;
   double* g = A + (int64_t)p * kNB * kp + (int64_t)p * kNB;
   load_tile(T, g, kp);
   __syncthreads();
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, tx = t % 16, ty = t / 16;
   for (int j = 0; j < kNB; ++j) {
-    const double d = sqrt(T[j * kTLd + j]);
-    __syncthreads();
-    if (t == 0) T[j * kTLd + j] = d;
-    for (int i = j + 1 + t; i < kNB; i += kFThreads) T[i * kTLd + j] /= d;
-    __syncthreads();
-    const int m = kNB - 1 - j;
-    for (int e = t; e < m * m; e += kFThreads) {
-      const int i = j + 1 + e / m, l = j + 1 + e % m;
-      if (l <= i) T[i * kTLd + l] -= T[i * kTLd + j] * T[l * kTLd + j];
+    const double rr = 1.0 / T[j * kTLd + j];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = j + 1 + ty + 16 * a;
+      if (i < kNB) {
+        const double tij = T[i * kTLd + j] * rr;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int l = j + 1 + tx + 16 * b;
+          if (l <= i) T[i * kTLd + l] -= tij * T[l * kTLd + j];
+        }
+      }
     }
     __syncthreads();
   }
-  for (int e = t; e < kNB * kNB; e += kFThreads)
-    if (e % kNB > e / kNB) T[(e / kNB) * kTLd + e % kNB] = 0.0;
+  if (t < kNB) {
+    const double d = sqrt(T[t * kTLd + t]);
+    dg[t] = d;
+    rdiag[t] = 1.0 / d;
+  }
+  __syncthreads();
+  for (int e = t; e < kNB * kNB; e += kFThreads) {
+    const int r = e / kNB, c = e % kNB;
+    double& v = T[r * kTLd + c];
+    v = c > r ? 0.0 : (c == r ? dg[r] : v * rdiag[c]);
+  }
+  __syncthreads();
+  if (t < kNB) rdiag[t] = 1.0 / T[t * kTLd + t];
+  __syncthreads();
+  const int c = t >> 2, part = t & 3;
+  for (int i = 0; i < kNB; ++i) {
+    double acc = 0.0;
+    for (int r = c + part; r < i; r += 4) acc += T[i * kTLd + r] * X[r * kTLd + c];
+    acc += __shfl_xor_sync(kFull, acc, 1);
+    acc += __shfl_xor_sync(kFull, acc, 2);
+    if (part == 0) X[i * kTLd + c] = i == c ? rdiag[i] : (i > c ? -acc * rdiag[i] : 0.0);
+    __syncwarp();
+  }
   __syncthreads();
   store_tile(g, T, kp);
+  store_tile(M + (int64_t)p * kNB * kp + (int64_t)p * kNB, X, kp);
 }
 
-// Tiles below the diagonal tile p: A_ip <- A_ip L_pp^-T (one row per thread, forward
-// substitution).
-__global__ void __launch_bounds__(kFThreads) k_trsm(double* A, int64_t kp, int p) {
-  extern __shared__ double sm[];
-  double* L = sm;
-  double* X = sm + kNB * kTLd;
-  const int i = p + 1 + blockIdx.x;
-  load_tile(L, A + (int64_t)p * kNB * kp + (int64_t)p * kNB, kp);
-  double* g = A + (int64_t)i * kNB * kp + (int64_t)p * kNB;
-  load_tile(X, g, kp);
-  __syncthreads();
-  if (threadIdx.x < kNB) {
-    double* x = X + threadIdx.x * kTLd;
-    for (int c = 0; c < kNB; ++c) {
-      double v = x[c];
-      for (int c2 = 0; c2 < c; ++c2) v -= x[c2] * L[c * kTLd + c2];
-      x[c] = v / L[c * kTLd + c];
+// ---- 64 x 64 x 64 float64 tile products --------------------------------------------------
+// 256 threads, thread (ty, tx) = (t / 16, t % 16) owns rows ty + 16 a and columns tx + 16 b
+// (a, b < 4). Operand tiles sit row-major in shared memory (rows of kTLd doubles); the tiles
+// of the next inner step are fetched with cp.async while the current ones are multiplied
+// (two buffers of two tiles: 133 KB).
+constexpr int kPThreads = 256;
+constexpr size_t kTileBytes = kNB * kTLd * sizeof(double);
+constexpr size_t kProdSmem = 4 * kTileBytes;   // NBUF = 2
+constexpr size_t kProdSmem1 = 2 * kTileBytes;  // NBUF = 1
+
+__device__ __forceinline__ void cp_async8(double* s, const double* g) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(s);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(a), "l"(g) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void stage_async(double* s, const double* g, int64_t ld) {
+  for (int e = threadIdx.x; e < kNB * kNB; e += kPThreads)
+    cp_async8(s + (e / kNB) * kTLd + e % kNB, g + (int64_t)(e / kNB) * ld + e % kNB);
+}
+
+// c += S1 S2^T (NT = true) or S1 S2 (NT = false) over 64 terms.
+template <bool NT>
+__device__ __forceinline__ void tile_mul(const double* S1, const double* S2, double (&c)[4][4]) {
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+#pragma unroll 4
+  for (int kk = 0; kk < kNB; ++kk) {
+    double x[4], y[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) x[a] = S1[(ty + 16 * a) * kTLd + kk];
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      y[b] = NT ? S2[(tx + 16 * b) * kTLd + kk] : S2[kk * kTLd + tx + 16 * b];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
+  }
+}
+
+// c = sum over n steps of tile(G1(q)) x tile(G2(q)) (x: NT or NN), q = 0 .. n-1. NBUF = 2:
+// the fetch of step q + 1 overlaps the product of step q (4 tiles of shared memory, one CTA
+// per SM); NBUF = 1: fetch, then multiply (2 tiles, three CTAs per SM overlap each other).
+template <bool NT, int NBUF, class F1, class F2>
+__device__ __forceinline__ void tile_sum(double* sm, int n, F1 g1, F2 g2, int64_t ld,
+                                         double (&c)[4][4]) {
+  if (n <= 0) return;
+  if constexpr (NBUF == 1) {
+    for (int q = 0; q < n; ++q) {
+      stage_async(sm, g1(q), ld);
+      stage_async(sm + kNB * kTLd, g2(q), ld);
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncthreads();
+      tile_mul<NT>(sm, sm + kNB * kTLd, c);
+      __syncthreads();
     }
+    return;
   }
-  __syncthreads();
-  store_tile(g, X, kp);
+  stage_async(sm, g1(0), ld);
+  stage_async(sm + kNB * kTLd, g2(0), ld);
+  cp_async_commit();
+  for (int q = 0; q < n; ++q) {
+    double* cur = sm + (q & 1) * 2 * kNB * kTLd;
+    if (q + 1 < n) {
+      double* nxt = sm + ((q + 1) & 1) * 2 * kNB * kTLd;
+      stage_async(nxt, g1(q + 1), ld);
+      stage_async(nxt + kNB * kTLd, g2(q + 1), ld);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    tile_mul<NT>(cur, cur + kNB * kTLd, c);
+    __syncthreads();
+  }
 }
 
-// C (4 x 4 per thread) = S1 S2^T over 64 terms; thread (ty, tx) owns rows ty + 16 a and
-// columns tx + 16 b.
-__device__ __forceinline__ void tile_mul_nt(const double* S1, const double* S2, double (&c)[4][4]) {
+// g = c (MODE 0), -c (1) or g - c (2); row-major tile, leading dimension ld.
+template <int MODE>
+__device__ __forceinline__ void put_tile(double* g, int64_t ld, const double (&c)[4][4]) {
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-#pragma unroll 4
-  for (int kk = 0; kk < kNB; ++kk) {
-    double x[4], y[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) x[a] = S1[(ty + 16 * a) * kTLd + kk];
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) y[b] = S2[(tx + 16 * b) * kTLd + kk];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
-  }
+    for (int b = 0; b < 4; ++b) {
+      double& o = g[(int64_t)(ty + 16 * a) * ld + tx + 16 * b];
+      o = MODE == 0 ? c[a][b] : (MODE == 1 ? -c[a][b] : o - c[a][b]);
+    }
 }
 
-// C = S1 S2 over 64 terms (S2 read by rows).
-__device__ __forceinline__ void tile_mul_nn(const double* S1, const double* S2, double (&c)[4][4]) {
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-#pragma unroll 4
-  for (int kk = 0; kk < kNB; ++kk) {
-    double x[4], y[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) x[a] = S1[(ty + 16 * a) * kTLd + kk];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) y[b] = S2[kk * kTLd + tx + 16 * b];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
-  }
-}
-
-// Trailing update after panel p: A_ij -= L_ip L_jp^T for p < j <= i (lower tiles).
-__global__ void __launch_bounds__(kFThreads) k_syrk(double* A, int64_t kp, int p) {
+// Tiles below the diagonal tile p: L_ip = A_ip L_pp^-T = A_ip M_pp^T.
+__global__ void __launch_bounds__(kPThreads) k_trsm(double* A, const double* M, int64_t kp, int p) {
   extern __shared__ double sm[];
-  double* Li = sm;
-  double* Lj = sm + kNB * kTLd;
+  const int64_t i = p + 1 + blockIdx.x;
+  double* g = A + i * kNB * kp + (int64_t)p * kNB;
+  const double* mpp = M + (int64_t)p * kNB * kp + (int64_t)p * kNB;
+  double c[4][4] = {};
+  tile_sum<true, 1>(sm, 1, [&](int) { return (const double*)g; }, [&](int) { return mpp; }, kp, c);
+  put_tile<0>(g, kp, c);
+}
+
+// Inside a panel of tile columns [p0, pe): before column p is factored, its tiles i >= p
+// receive the panel's earlier columns: A_ip -= sum_{t=p0}^{p-1} L_it L_pt^T.
+__global__ void __launch_bounds__(kPThreads)
+k_panel_update(double* A, int64_t kp, int p0, int p) {
+  extern __shared__ double sm[];
+  const int64_t i = p + blockIdx.x;
+  double c[4][4] = {};
+  tile_sum<true, 1>(sm, p - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
+                 [&](int q) { return (const double*)(A + (int64_t)p * kNB * kp + (int64_t)(p0 + q) * kNB); },
+                 kp, c);
+  put_tile<2>(A + i * kNB * kp + (int64_t)p * kNB, kp, c);
+}
+
+// Trailing update after the panel [p0, pe): A_ij -= sum_{t=p0}^{pe-1} L_it L_jt^T for
+// pe <= j <= i (lower tiles), one read-modify-write per tile.
+__global__ void __launch_bounds__(kPThreads) k_syrk(double* A, int64_t kp, int p0, int pe) {
+  extern __shared__ double sm[];
   // blockIdx.x -> (ii, jj), jj <= ii
   const int64_t idx = blockIdx.x;
   int64_t ii = (int64_t)((sqrt(8.0 * (double)idx + 1.0) - 1.0) / 2.0);
   while (ii * (ii + 1) / 2 > idx) --ii;
   while ((ii + 1) * (ii + 2) / 2 <= idx) ++ii;
   const int64_t jj = idx - ii * (ii + 1) / 2;
-  const int64_t i = p + 1 + ii, j = p + 1 + jj;
-  load_tile(Li, A + i * kNB * kp + (int64_t)p * kNB, kp);
-  load_tile(Lj, A + j * kNB * kp + (int64_t)p * kNB, kp);
-  __syncthreads();
+  const int64_t i = pe + ii, j = pe + jj;
   double c[4][4] = {};
-  tile_mul_nt(Li, Lj, c);
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  double* g = A + i * kNB * kp + j * kNB;
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) g[(int64_t)(ty + 16 * a) * kp + tx + 16 * b] -= c[a][b];
+  tile_sum<true, 1>(sm, pe - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
+                 [&](int q) { return (const double*)(A + j * kNB * kp + (int64_t)(p0 + q) * kNB); },
+                 kp, c);
+  put_tile<2>(A + i * kNB * kp + j * kNB, kp, c);
 }
 
-// Diagonal tiles of M = L^-1: one column per thread, forward substitution.
-__global__ void __launch_bounds__(kFThreads) k_trtri_diag(const double* A, double* M, int64_t kp) {
+// Off-diagonal blocks of M = L^-1 by doubling: segments of s tiles [a, a + s) and
+// [a + s, a + 2s) (the second cut at nt), both already inverted, merge as
+//   M_21 = -M_22 L_21 M_11,
+// in two launches over every pair of the level: T = L_21 M_11 (kept in A's unused upper
+// tiles, T_ij at tile (j, i)), then M_21 = -M_22 T. One CTA per output tile, blockIdx.y the
+// pair.
+__global__ void __launch_bounds__(kPThreads)
+k_inv_a(double* A, const double* M, int64_t kp, int nt, int s) {
   extern __shared__ double sm[];
-  double* L = sm;
-  double* X = sm + kNB * kTLd;
-  const int64_t j = blockIdx.x;
-  load_tile(L, A + j * kNB * kp + j * kNB, kp);
-  __syncthreads();
-  if (threadIdx.x < kNB) {
-    const int c = threadIdx.x;
-    for (int i = 0; i < kNB; ++i) {
-      double v = 0.0;
-      if (i == c) {
-        v = 1.0 / L[i * kTLd + i];
-      } else if (i > c) {
-        double s = 0.0;
-        for (int r = c; r < i; ++r) s += L[i * kTLd + r] * X[r * kTLd + c];
-        v = -s / L[i * kTLd + i];
-      }
-      X[i * kTLd + c] = v;
-    }
-  }
-  __syncthreads();
-  store_tile(M + j * kNB * kp + j * kNB, X, kp);
+  const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
+  const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
+  if (i >= nt) return;
+  double c[4][4] = {};
+  // T_ij = sum_{kk = j}^{a0 + s - 1} L_i,kk M_kk,j  (M_kk,j = 0 for kk < j)
+  tile_sum<false, 2>(sm, (int)(a0 + s - j),
+                  [&](int q) { return (const double*)(A + i * kNB * kp + (j + q) * kNB); },
+                  [&](int q) { return M + (j + q) * kNB * kp + j * kNB; }, kp, c);
+  put_tile<0>(A + j * kNB * kp + i * kNB, kp, c);          // upper tile (j, i)
 }
 
-// Sub-diagonal d: M_ij = -M_ii sum_{kk=j}^{i-1} L_i,kk M_kk,j for i = j + d.
-__global__ void __launch_bounds__(kFThreads)
-k_trtri_step(const double* A, double* M, int64_t kp, int d) {
+__global__ void __launch_bounds__(kPThreads)
+k_inv_b(const double* A, double* M, int64_t kp, int nt, int s) {
   extern __shared__ double sm[];
-  double* S1 = sm;
-  double* S2 = sm + kNB * kTLd;
-  const int64_t j = blockIdx.x, i = j + d;
+  const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
+  const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
+  if (i >= nt) return;
   double c[4][4] = {};
-  for (int64_t kk = j; kk < i; ++kk) {
-    __syncthreads();
-    load_tile(S1, A + i * kNB * kp + kk * kNB, kp);
-    load_tile(S2, M + kk * kNB * kp + j * kNB, kp);
-    __syncthreads();
-    tile_mul_nn(S1, S2, c);
-  }
-  __syncthreads();
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) S2[(ty + 16 * a) * kTLd + tx + 16 * b] = c[a][b];
-  load_tile(S1, M + i * kNB * kp + i * kNB, kp);
-  __syncthreads();
-  double r[4][4] = {};
-  tile_mul_nn(S1, S2, r);
-  double* g = M + i * kNB * kp + j * kNB;
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) g[(int64_t)(ty + 16 * a) * kp + tx + 16 * b] = -r[a][b];
+  // M_ij = -sum_{kk = a0 + s}^{i} M_i,kk T_kk,j  (T_kk,j kept at tile (j, kk))
+  tile_sum<false, 2>(sm, (int)(i - a0 - s + 1),
+                  [&](int q) { return (const double*)(M + i * kNB * kp + (a0 + s + q) * kNB); },
+                  [&](int q) { return A + j * kNB * kp + (a0 + s + q) * kNB; }, kp, c);
+  put_tile<1>(M + i * kNB * kp + j * kNB, kp, c);
 }
 
 // U_pq = fl32(M_{k-1-p, k-1-q}) for q >= p, else 0.
@@ -294,10 +357,14 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
                                double damp, float* U, void* ws, cudaStream_t st) {
   static const bool attrs = [] {
     bool ok = true;
-    for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_trtri_diag,
-                          (const void*)k_trtri_step})
+    ok = cudaFuncSetAttribute(k_potrf_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kTwoTiles) == cudaSuccess;
+    for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update})
       ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kTwoTiles) == cudaSuccess;
+                                      (int)kProdSmem1) == cudaSuccess;
+    for (const void* f : {(const void*)k_inv_a, (const void*)k_inv_b})
+      ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kProdSmem) == cudaSuccess;
     return ok;
   }();
   if (!attrs) return cudaErrorInvalidConfiguration;
@@ -308,17 +375,23 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   const int gs = sm_count() * 8;
   k_factor_lambda<<<1, kFThreads, 0, st>>>(H, k, damp, a.scal);
   k_factor_load<<<gs, 256, 0, st>>>(a);
-  for (int p = 0; p < nt; ++p) {
-    k_potrf<<<1, kFThreads, 0, st>>>(a.A, kp, p);
-    const int64_t m = nt - 1 - p;
-    if (m > 0) {
-      k_trsm<<<(unsigned)m, kFThreads, kTwoTiles, st>>>(a.A, kp, p);
-      k_syrk<<<(unsigned)(m * (m + 1) / 2), kFThreads, kTwoTiles, st>>>(a.A, kp, p);
+  // right-looking over panels of kPanelTiles tile columns, left-looking inside a panel
+  for (int p0 = 0; p0 < nt; p0 += kPanelTiles) {
+    const int pe = (int)(p0 + kPanelTiles < nt ? p0 + kPanelTiles : nt);
+    for (int p = p0; p < pe; ++p) {
+      if (p > p0) k_panel_update<<<(unsigned)(nt - p), kPThreads, kProdSmem1, st>>>(a.A, kp, p0, p);
+      k_potrf_inv<<<1, kFThreads, kTwoTiles, st>>>(a.A, a.M, kp, p);
+      if (nt - 1 - p > 0)
+        k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem1, st>>>(a.A, a.M, kp, p);
     }
+    const int64_t m = nt - pe;
+    if (m > 0) k_syrk<<<(unsigned)(m * (m + 1) / 2), kPThreads, kProdSmem1, st>>>(a.A, kp, p0, pe);
   }
-  k_trtri_diag<<<(unsigned)nt, kFThreads, kTwoTiles, st>>>(a.A, a.M, kp);
-  for (int d = 1; d < nt; ++d)
-    k_trtri_step<<<(unsigned)(nt - d), kFThreads, kTwoTiles, st>>>(a.A, a.M, kp, d);
+  for (int s = 1; s < nt; s *= 2) {
+    const dim3 grid((unsigned)(s * s), (unsigned)((nt + 2 * s - 1) / (2 * s)));
+    k_inv_a<<<grid, kPThreads, kProdSmem, st>>>(a.A, a.M, kp, (int)nt, s);
+    k_inv_b<<<grid, kPThreads, kProdSmem, st>>>(a.A, a.M, kp, (int)nt, s);
+  }
   k_factor_store<<<gs, 256, 0, st>>>(a);
   return cudaGetLastError();
 }

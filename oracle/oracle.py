@@ -385,21 +385,21 @@ def gram(X) -> np.ndarray:
 
 
 def block_losses(W, h, fmt: str, mode: str, block: int, *, sfmt: str = "e4m3",
-                 window: int = -1) -> np.ndarray:
+                 window: int = -1, n_threads=1) -> np.ndarray:
     """Hessian-weighted quantization loss of each column block: sum over rows and the
-    block's columns of h_j (w_ij - w^_ij)^2 (float64, rows ascending) for the block
-    quantizer's own (uncompensated) result."""
+    block's columns of h_j (w_ij - w^_ij)^2 (float64; each row's block summed, then the rows
+    in ascending order) for the block quantizer's own (uncompensated) result."""
     W, _ = _as_input(W)
     n, k = W.shape
     r = quantize(W, fmt, mode, block, h=h if mode == "hopt" else None, window=window,
-                 sfmt=sfmt)
+                 sfmt=sfmt, n_threads=n_threads)
     What = dequant(r.codes, r.scales, fmt, block, n, k, sfmt=sfmt).astype(np.float64)
     d = to_float(W).astype(np.float64) - What
     e = (d * d) * np.asarray(h, np.float64)[None, :]
+    per_row = e.reshape(n, k // block, block).sum(axis=2)
     loss = np.zeros(k // block)
-    for b in range(k // block):
-        for i in range(n):
-            loss[b] += float(np.sum(e[i, b * block:(b + 1) * block]))
+    for i in range(n):
+        loss += per_row[i]
     return loss
 
 

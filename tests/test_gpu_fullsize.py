@@ -186,3 +186,38 @@ def test_block_hessian_full_size(mxq, orc, synth):
     r = orc.quantize_gram(oracle_view(W[ri]), "nvfp4", 16, G, n_threads=NT)
     assert np.array_equal(scales[ri].cpu().numpy(), r.scales)
     assert np.array_equal(codes[ri].cpu().numpy(), r.codes)
+
+
+def test_gptq_ordered_full_size(mxq, orc, synth):
+    """Ordered GPTQ with the NVFP4 bs16 H-optimal quantizer on the full-calibration weight
+    (2560 x 9728), the Hessian of 8192 activation rows (the oracle's, uploaded): the block
+    order exactly, the factor of the full 9728 x 9728 Hessian within one float32 rounding of
+    the oracle's, and sampled rows of the sweep bit-exact given the oracle's factor."""
+    wl = synth.WORKLOADS["nvfp4_full_calib"]
+    W = synth.workload_weight(wl, 0, device=DEV)
+    n, k = W.shape
+    X = oracle_view(synth.workload_activations(wl, 0, device="cpu", rows=8192))
+    H = orc.gram(X)
+    h = orc.act_sqmean(X, n_threads=NT)
+    p = mxq.params("nvfp4", "hopt", 16)
+    hd = torch.from_numpy(h).to(DEV)
+    perm = mxq.mxq_gptq_order(W, hd, p)
+    Wo = oracle_view(W)
+    perm_ref = orc.block_order(orc.block_losses(Wo, h, "nvfp4", "hopt", 16, n_threads=NT))
+    assert np.array_equal(perm.cpu().numpy(), perm_ref)
+    cols = (perm_ref[:, None] * 16 + np.arange(16)[None, :]).reshape(-1)
+    U_ref = orc.gptq_prepare(np.ascontiguousarray(H[np.ix_(cols, cols)])[None])[0]
+    U = mxq.mxq_gptq_factor(torch.from_numpy(H).to(DEV), 16, perm).cpu().numpy()
+    ref = U_ref.astype(np.float64)
+    tol = 2.0 ** -23 * np.abs(ref) + 2.0 ** -28 * np.abs(ref).max()
+    err = np.abs(U.astype(np.float64) - ref)
+    assert np.all(err <= tol), float((err / tol).max())
+    del U, ref, err
+    codes, scales = mxq.mxq_gptq(W, torch.from_numpy(U_ref).to(DEV), p, hd, perm)
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(n, 8, wl.seed + 51).tolist()
+    ri = torch.as_tensor(rows, device=DEV)
+    r = orc.gptq_blocks(oracle_view(W[ri]), U_ref, h, "nvfp4", "hopt", 16, perm=perm_ref,
+                        n_threads=NT)
+    assert np.array_equal(scales[ri].cpu().numpy(), r.scales)
+    assert np.array_equal(codes[ri].cpu().numpy(), r.codes)
