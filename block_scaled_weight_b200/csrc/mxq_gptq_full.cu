@@ -166,14 +166,14 @@ __global__ void __launch_bounds__(kFThreads) k_potrf_inv(double* A, double* M, i
 }
 
 // ---- 64 x 64 x 64 float64 tile products --------------------------------------------------
-// 256 threads, thread (ty, tx) = (t / 16, t % 16) owns rows ty + 16 a and columns tx + 16 b
-// (a, b < 4). Operand tiles sit row-major in shared memory (rows of kTLd doubles); the tiles
-// of the next inner step are fetched with cp.async while the current ones are multiplied
-// (two buffers of two tiles: 133 KB).
-constexpr int kPThreads = 256;
+// 128 threads, thread (ty, tx) = (t / 16, t % 16) owns rows ty + 8 a (a < 8) and columns
+// tx + 16 b (b < 4): per inner step 8 broadcast loads and 4 row-of-16 loads feed 32 FMAs,
+// enough to keep the FP64 pipe, not shared memory, the limit. Operand tiles sit row-major in
+// shared memory (rows of kTLd doubles), fetched with cp.async.
+constexpr int kPThreads = 128;
+constexpr int kRows = 8, kCols = 4;       // outputs per thread
 constexpr size_t kTileBytes = kNB * kTLd * sizeof(double);
-constexpr size_t kProdSmem = 4 * kTileBytes;   // NBUF = 2
-constexpr size_t kProdSmem1 = 2 * kTileBytes;  // NBUF = 1
+constexpr size_t kProdSmem1 = 2 * kTileBytes;
 
 __device__ __forceinline__ void cp_async8(double* s, const double* g) {
   const uint32_t a = (uint32_t)__cvta_generic_to_shared(s);
@@ -193,69 +193,50 @@ __device__ __forceinline__ void stage_async(double* s, const double* g, int64_t 
 
 // c += S1 S2^T (NT = true) or S1 S2 (NT = false) over 64 terms.
 template <bool NT>
-__device__ __forceinline__ void tile_mul(const double* S1, const double* S2, double (&c)[4][4]) {
+__device__ __forceinline__ void tile_mul(const double* S1, const double* S2,
+                                         double (&c)[kRows][kCols]) {
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-#pragma unroll 4
+#pragma unroll 2
   for (int kk = 0; kk < kNB; ++kk) {
-    double x[4], y[4];
+    double x[kRows], y[kCols];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) x[a] = S1[(ty + 16 * a) * kTLd + kk];
+    for (int a = 0; a < kRows; ++a) x[a] = S1[(ty + 8 * a) * kTLd + kk];
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
+    for (int b = 0; b < kCols; ++b)
       y[b] = NT ? S2[(tx + 16 * b) * kTLd + kk] : S2[kk * kTLd + tx + 16 * b];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < kRows; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
+      for (int b = 0; b < kCols; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
   }
 }
 
-// c = sum over n steps of tile(G1(q)) x tile(G2(q)) (x: NT or NN), q = 0 .. n-1. NBUF = 2:
-// the fetch of step q + 1 overlaps the product of step q (4 tiles of shared memory, one CTA
-// per SM); NBUF = 1: fetch, then multiply (2 tiles, three CTAs per SM overlap each other).
-template <bool NT, int NBUF, class F1, class F2>
+// c = sum over n steps of tile(G1(q)) x tile(G2(q)) (x: NT or NN), q = 0 .. n-1: fetch both
+// tiles, multiply (two tiles of shared memory; three CTAs per SM overlap one another's
+// fetches and products).
+template <bool NT, class F1, class F2>
 __device__ __forceinline__ void tile_sum(double* sm, int n, F1 g1, F2 g2, int64_t ld,
-                                         double (&c)[4][4]) {
-  if (n <= 0) return;
-  if constexpr (NBUF == 1) {
-    for (int q = 0; q < n; ++q) {
-      stage_async(sm, g1(q), ld);
-      stage_async(sm + kNB * kTLd, g2(q), ld);
-      cp_async_commit();
-      cp_async_wait<0>();
-      __syncthreads();
-      tile_mul<NT>(sm, sm + kNB * kTLd, c);
-      __syncthreads();
-    }
-    return;
-  }
-  stage_async(sm, g1(0), ld);
-  stage_async(sm + kNB * kTLd, g2(0), ld);
-  cp_async_commit();
+                                         double (&c)[kRows][kCols]) {
   for (int q = 0; q < n; ++q) {
-    double* cur = sm + (q & 1) * 2 * kNB * kTLd;
-    if (q + 1 < n) {
-      double* nxt = sm + ((q + 1) & 1) * 2 * kNB * kTLd;
-      stage_async(nxt, g1(q + 1), ld);
-      stage_async(nxt + kNB * kTLd, g2(q + 1), ld);
-    }
+    stage_async(sm, g1(q), ld);
+    stage_async(sm + kNB * kTLd, g2(q), ld);
     cp_async_commit();
-    cp_async_wait<1>();
+    cp_async_wait<0>();
     __syncthreads();
-    tile_mul<NT>(cur, cur + kNB * kTLd, c);
+    tile_mul<NT>(sm, sm + kNB * kTLd, c);
     __syncthreads();
   }
 }
 
 // g = c (MODE 0), -c (1) or g - c (2); row-major tile, leading dimension ld.
 template <int MODE>
-__device__ __forceinline__ void put_tile(double* g, int64_t ld, const double (&c)[4][4]) {
+__device__ __forceinline__ void put_tile(double* g, int64_t ld, const double (&c)[kRows][kCols]) {
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < kRows; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      double& o = g[(int64_t)(ty + 16 * a) * ld + tx + 16 * b];
+    for (int b = 0; b < kCols; ++b) {
+      double& o = g[(int64_t)(ty + 8 * a) * ld + tx + 16 * b];
       o = MODE == 0 ? c[a][b] : (MODE == 1 ? -c[a][b] : o - c[a][b]);
     }
 }
@@ -266,8 +247,8 @@ __global__ void __launch_bounds__(kPThreads) k_trsm(double* A, const double* M, 
   const int64_t i = p + 1 + blockIdx.x;
   double* g = A + i * kNB * kp + (int64_t)p * kNB;
   const double* mpp = M + (int64_t)p * kNB * kp + (int64_t)p * kNB;
-  double c[4][4] = {};
-  tile_sum<true, 1>(sm, 1, [&](int) { return (const double*)g; }, [&](int) { return mpp; }, kp, c);
+  double c[kRows][kCols] = {};
+  tile_sum<true>(sm, 1, [&](int) { return (const double*)g; }, [&](int) { return mpp; }, kp, c);
   put_tile<0>(g, kp, c);
 }
 
@@ -277,8 +258,8 @@ __global__ void __launch_bounds__(kPThreads)
 k_panel_update(double* A, int64_t kp, int p0, int p) {
   extern __shared__ double sm[];
   const int64_t i = p + blockIdx.x;
-  double c[4][4] = {};
-  tile_sum<true, 1>(sm, p - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
+  double c[kRows][kCols] = {};
+  tile_sum<true>(sm, p - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  [&](int q) { return (const double*)(A + (int64_t)p * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  kp, c);
   put_tile<2>(A + i * kNB * kp + (int64_t)p * kNB, kp, c);
@@ -295,8 +276,8 @@ __global__ void __launch_bounds__(kPThreads) k_syrk(double* A, int64_t kp, int p
   while ((ii + 1) * (ii + 2) / 2 <= idx) ++ii;
   const int64_t jj = idx - ii * (ii + 1) / 2;
   const int64_t i = pe + ii, j = pe + jj;
-  double c[4][4] = {};
-  tile_sum<true, 1>(sm, pe - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
+  double c[kRows][kCols] = {};
+  tile_sum<true>(sm, pe - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  [&](int q) { return (const double*)(A + j * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  kp, c);
   put_tile<2>(A + i * kNB * kp + j * kNB, kp, c);
@@ -314,9 +295,9 @@ k_inv_a(double* A, const double* M, int64_t kp, int nt, int s) {
   const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
   const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
   if (i >= nt) return;
-  double c[4][4] = {};
+  double c[kRows][kCols] = {};
   // T_ij = sum_{kk = j}^{a0 + s - 1} L_i,kk M_kk,j  (M_kk,j = 0 for kk < j)
-  tile_sum<false, 2>(sm, (int)(a0 + s - j),
+  tile_sum<false>(sm, (int)(a0 + s - j),
                   [&](int q) { return (const double*)(A + i * kNB * kp + (j + q) * kNB); },
                   [&](int q) { return M + (j + q) * kNB * kp + j * kNB; }, kp, c);
   put_tile<0>(A + j * kNB * kp + i * kNB, kp, c);          // upper tile (j, i)
@@ -328,9 +309,9 @@ k_inv_b(const double* A, double* M, int64_t kp, int nt, int s) {
   const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
   const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
   if (i >= nt) return;
-  double c[4][4] = {};
+  double c[kRows][kCols] = {};
   // M_ij = -sum_{kk = a0 + s}^{i} M_i,kk T_kk,j  (T_kk,j kept at tile (j, kk))
-  tile_sum<false, 2>(sm, (int)(i - a0 - s + 1),
+  tile_sum<false>(sm, (int)(i - a0 - s + 1),
                   [&](int q) { return (const double*)(M + i * kNB * kp + (a0 + s + q) * kNB); },
                   [&](int q) { return A + j * kNB * kp + (a0 + s + q) * kNB; }, kp, c);
   put_tile<1>(M + i * kNB * kp + j * kNB, kp, c);
@@ -359,12 +340,10 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
     bool ok = true;
     ok = cudaFuncSetAttribute(k_potrf_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)kTwoTiles) == cudaSuccess;
-    for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update})
+    for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update,
+                          (const void*)k_inv_a, (const void*)k_inv_b})
       ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kProdSmem1) == cudaSuccess;
-    for (const void* f : {(const void*)k_inv_a, (const void*)k_inv_b})
-      ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kProdSmem) == cudaSuccess;
     return ok;
   }();
   if (!attrs) return cudaErrorInvalidConfiguration;
@@ -389,8 +368,8 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   }
   for (int s = 1; s < nt; s *= 2) {
     const dim3 grid((unsigned)(s * s), (unsigned)((nt + 2 * s - 1) / (2 * s)));
-    k_inv_a<<<grid, kPThreads, kProdSmem, st>>>(a.A, a.M, kp, (int)nt, s);
-    k_inv_b<<<grid, kPThreads, kProdSmem, st>>>(a.A, a.M, kp, (int)nt, s);
+    k_inv_a<<<grid, kPThreads, kProdSmem1, st>>>(a.A, a.M, kp, (int)nt, s);
+    k_inv_b<<<grid, kPThreads, kProdSmem1, st>>>(a.A, a.M, kp, (int)nt, s);
   }
   k_factor_store<<<gs, 256, 0, st>>>(a);
   return cudaGetLastError();
@@ -579,19 +558,35 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S) {
 
 // Later positions p >= p0 + S: for each block of the panel (in order)
 // acc = sum_j fma(err_j, U[j][p], acc) over the block's columns, then w -= acc.
-// CTA: 64 rows x 64 positions; thread: 4 rows x 4 consecutive positions.
+// CTA: 64 positions x rg groups of 64 rows; thread: 4 rows x 4 consecutive positions. The
+// CTA's rows of U are staged once; the residuals of the next row group are fetched with
+// cp.async while the current group is updated.
+constexpr int kEsLd = kPanel + 4;        // padded residual row (16-byte aligned)
+constexpr size_t kTrailSmem = (2 * 64 * kEsLd + kPanel * 64) * sizeof(float);
+
+__device__ __forceinline__ void cp_async16(float* s, const float* g) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(s);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(g) : "memory");
+}
+
 template <int B>
 __global__ void __launch_bounds__(kTrailThreads)
-k_gptq_trailing(SweepArgs a, int64_t p0, int S) {
-  __shared__ float Es[64][kPanel + 1];
-  __shared__ __align__(16) float Ut[kPanel][64];
-  const int64_t pstart = p0 + S;
-  const int64_t c0 = pstart + (int64_t)blockIdx.x * 64;
-  const int64_t r0 = (int64_t)blockIdx.y * 64;
-  for (int e = threadIdx.x; e < 64 * kPanel; e += kTrailThreads) {
-    const int i = e / kPanel, j = e % kPanel;
-    Es[i][j] = (r0 + i < a.n && j < S) ? a.Err[(r0 + i) * kPanel + j] : 0.0f;
-  }
+k_gptq_trailing(SweepArgs a, int64_t p0, int S, int rg) {
+  extern __shared__ __align__(16) float tsm[];
+  float (*Es)[64 * kEsLd] = reinterpret_cast<float (*)[64 * kEsLd]>(tsm);
+  float (*Ut)[64] = reinterpret_cast<float (*)[64]>(tsm + 2 * 64 * kEsLd);
+  const int64_t c0 = p0 + S + (int64_t)blockIdx.x * 64;
+  const int64_t groups = (a.n + 63) / 64;
+  const int64_t g0 = (int64_t)blockIdx.y * rg;
+  const int ng = (int)(groups - g0 < rg ? groups - g0 : rg);
+  auto stage_es = [&](int buf, int64_t r0) {
+    for (int e = threadIdx.x; e < 64 * (kPanel / 4); e += kTrailThreads) {
+      const int i = e / (kPanel / 4), q = e % (kPanel / 4);
+      if (r0 + i < a.n) cp_async16(&Es[buf][i * kEsLd + 4 * q], a.Err + (r0 + i) * kPanel + 4 * q);
+    }
+  };
+  stage_es(0, g0 * 64);
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
   for (int e = threadIdx.x; e < kPanel * 16; e += kTrailThreads) {
     const int j = e / 16, g = e % 16;
     float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -599,50 +594,62 @@ k_gptq_trailing(SweepArgs a, int64_t p0, int S) {
       u = *reinterpret_cast<const float4*>(a.U + (p0 + j) * a.k + c0 + 4 * g);
     *reinterpret_cast<float4*>(&Ut[j][4 * g]) = u;
   }
-  __syncthreads();
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const int64_t col = c0 + 4 * tx;
-  if (col >= a.k) return;
-  float4 w[4];
+  const bool on = col < a.k;
+  for (int g = 0; g < ng; ++g) {
+    const int64_t r0 = (g0 + g) * 64;
+    if (g + 1 < ng) stage_es((g + 1) & 1, r0 + 64);
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    float4 w[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t r = r0 + 4 * ty + i;
-    w[i] = r < a.n ? *reinterpret_cast<const float4*>(a.Wc + r * a.k + col)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int q0 = 0; q0 < S; q0 += B) {
-    float4 acc[4];
+    for (int i = 0; i < 4; ++i) {
+      const int64_t r = r0 + 4 * ty + i;
+      w[i] = (on && r < a.n) ? *reinterpret_cast<const float4*>(a.Wc + r * a.k + col)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+    __syncthreads();
+    const float* E = Es[g & 1];
+    for (int q0 = 0; q0 < S; q0 += B) {
+      float4 acc[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-    for (int j = 0; j < B; ++j) {
-      const float4 u = *reinterpret_cast<const float4*>(&Ut[q0 + j][4 * tx]);
+      for (int j = 0; j < B; ++j) {
+        const float4 u = *reinterpret_cast<const float4*>(&Ut[q0 + j][4 * tx]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float e = E[(4 * ty + i) * kEsLd + q0 + j];
+          acc[i].x = __fmaf_rn(e, u.x, acc[i].x);
+          acc[i].y = __fmaf_rn(e, u.y, acc[i].y);
+          acc[i].z = __fmaf_rn(e, u.z, acc[i].z);
+          acc[i].w = __fmaf_rn(e, u.w, acc[i].w);
+        }
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float e = Es[4 * ty + i][q0 + j];
-        acc[i].x = __fmaf_rn(e, u.x, acc[i].x);
-        acc[i].y = __fmaf_rn(e, u.y, acc[i].y);
-        acc[i].z = __fmaf_rn(e, u.z, acc[i].z);
-        acc[i].w = __fmaf_rn(e, u.w, acc[i].w);
+        w[i].x = __fsub_rn(w[i].x, acc[i].x);
+        w[i].y = __fsub_rn(w[i].y, acc[i].y);
+        w[i].z = __fsub_rn(w[i].z, acc[i].z);
+        w[i].w = __fsub_rn(w[i].w, acc[i].w);
       }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      w[i].x = __fsub_rn(w[i].x, acc[i].x);
-      w[i].y = __fsub_rn(w[i].y, acc[i].y);
-      w[i].z = __fsub_rn(w[i].z, acc[i].z);
-      w[i].w = __fsub_rn(w[i].w, acc[i].w);
+      const int64_t r = r0 + 4 * ty + i;
+      if (on && r < a.n) *reinterpret_cast<float4*>(a.Wc + r * a.k + col) = w[i];
     }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t r = r0 + 4 * ty + i;
-    if (r < a.n) *reinterpret_cast<float4*>(a.Wc + r * a.k + col) = w[i];
+    __syncthreads();                      // Es[g & 1] is refilled two groups later
   }
 }
 
 template <int B, int ELEM>
 cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cudaStream_t st) {
+  static const bool attr = cudaFuncSetAttribute(k_gptq_trailing<B>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)kTrailSmem) == cudaSuccess;
+  if (!attr) return cudaErrorInvalidConfiguration;
   k_sweep_init<B><<<sm_count() * 8, 256, 0, st>>>(a);
   const unsigned prow = (unsigned)((a.n + kPanelWarps - 1) / kPanelWarps);
   for (int64_t p0 = 0; p0 < a.k; p0 += kPanel) {
@@ -652,8 +659,12 @@ cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cud
     else k_gptq_panel<B, ELEM, 2><<<prow, kPanelWarps * 32, 0, st>>>(a, T, p0, S);
     const int64_t rest = a.k - p0 - S;
     if (rest > 0) {
-      const dim3 grid((unsigned)((rest + 63) / 64), (unsigned)((a.n + 63) / 64));
-      k_gptq_trailing<B><<<grid, kTrailThreads, 0, st>>>(a, p0, S);
+      // row groups per CTA: as many as keep at least ~4 CTAs per SM
+      const int64_t ctiles = (rest + 63) / 64, groups = (a.n + 63) / 64;
+      int64_t rg = ctiles * groups / ((int64_t)sm_count() * 4);
+      rg = rg < 1 ? 1 : (rg > 8 ? 8 : rg);
+      const dim3 grid((unsigned)ctiles, (unsigned)((groups + rg - 1) / rg));
+      k_gptq_trailing<B><<<grid, kTrailThreads, kTrailSmem, st>>>(a, p0, S, (int)rg);
     }
   }
   return cudaGetLastError();
