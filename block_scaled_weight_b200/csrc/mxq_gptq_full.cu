@@ -107,6 +107,18 @@ __device__ __forceinline__ void store_tile(double* g, const double* s, int64_t l
     g[(int64_t)(e / kNB) * ld + e % kNB] = s[(e / kNB) * kTLd + e % kNB];
 }
 
+// 1 / x for the elimination's pivots, off the division unit: a float32 reciprocal as the seed,
+// then two Newton-Raphson steps r <- r + r (1 - x r) (quadratic convergence: 2^-24 -> 2^-48
+// -> below the float64 rounding); x outside float32's normal range takes the division.
+__device__ __forceinline__ double recip(double x) {
+  const float xf = (float)x;
+  if (!(fabsf(xf) >= 1.2e-38f && fabsf(xf) <= 3.0e38f)) return 1.0 / x;
+  double r = (double)__frcp_rn(xf);
+  r = fma(r, fma(-x, r, 1.0), r);
+  r = fma(r, fma(-x, r, 1.0), r);
+  return r;
+}
+
 // Diagonal tile p: its Cholesky factor L_pp (lower, the upper part 0) into A and its
 // inverse M_pp into M. The elimination keeps the columns unscaled (step j: T_il -= T_ij T_lj
 // / T_jj over the trailing triangle, one barrier per step), and scales every column by
@@ -122,7 +134,7 @@ __global__ void __launch_bounds__(kFThreads) k_potrf_inv(double* A, double* M, i
   __syncthreads();
   const int t = threadIdx.x, tx = t % 16, ty = t / 16;
   for (int j = 0; j < kNB; ++j) {
-    const double rr = 1.0 / T[j * kTLd + j];
+    const double rr = recip(T[j * kTLd + j]);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int i = j + 1 + ty + 16 * a;
@@ -165,19 +177,20 @@ __global__ void __launch_bounds__(kFThreads) k_potrf_inv(double* A, double* M, i
   store_tile(M + (int64_t)p * kNB * kp + (int64_t)p * kNB, X, kp);
 }
 
-// ---- 64 x 64 x 64 float64 tile products --------------------------------------------------
-// 128 threads, thread (ty, tx) = (t / 16, t % 16) owns rows ty + 8 a (a < 8) and columns
-// tx + 16 b (b < 4): per inner step 8 broadcast loads and 4 row-of-16 loads feed 32 FMAs,
-// enough to keep the FP64 pipe, not shared memory, the limit. Operand tiles sit row-major in
-// shared memory (rows of kTLd doubles), fetched with cp.async.
+// ---- 64 x 64 x 64 float64 tile products (FP64 tensor cores) -----------------------------
+// 128 threads = 4 warps; warp w computes the 32 x 32 quadrant (rows 32 (w / 2), columns
+// 32 (w % 2)) as 4 x 4 fragments of mma.sync m8n8k4 f64 (A row-major 8 x 4, B 4 x 8, C 8 x 8
+// in two doubles per lane). Operand tiles sit row-major in shared memory with rows of kPLd
+// doubles (68: every fragment load -- 8 rows x 4 columns of A, or of B either way round --
+// touches each bank pair exactly twice), fetched with 16-byte cp.async.
 constexpr int kPThreads = 128;
-constexpr int kRows = 8, kCols = 4;       // outputs per thread
-constexpr size_t kTileBytes = kNB * kTLd * sizeof(double);
-constexpr size_t kProdSmem1 = 2 * kTileBytes;
+constexpr int kPLd = kNB + 4;
+constexpr size_t kProdSmem1 = 2 * kNB * kPLd * sizeof(double);
+using Frag = double[4][4][2];            // [m tile][n tile][c0, c1]
 
-__device__ __forceinline__ void cp_async8(double* s, const double* g) {
+__device__ __forceinline__ void cp_async16d(double* s, const double* g) {
   const uint32_t a = (uint32_t)__cvta_generic_to_shared(s);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(a), "l"(g) : "memory");
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(g) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
@@ -187,57 +200,68 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void stage_async(double* s, const double* g, int64_t ld) {
-  for (int e = threadIdx.x; e < kNB * kNB; e += kPThreads)
-    cp_async8(s + (e / kNB) * kTLd + e % kNB, g + (int64_t)(e / kNB) * ld + e % kNB);
+  for (int e = threadIdx.x * 2; e < kNB * kNB; e += kPThreads * 2)
+    cp_async16d(s + (e / kNB) * kPLd + e % kNB, g + (int64_t)(e / kNB) * ld + e % kNB);
 }
 
-// c += S1 S2^T (NT = true) or S1 S2 (NT = false) over 64 terms.
+__device__ __forceinline__ void dmma(double a, double b, double (&c)[2]) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
+}
+
+// c += S1 S2^T (NT = true: S2 holds B^T, [n][k]) or S1 S2 (NT = false: S2 is [k][n]).
 template <bool NT>
-__device__ __forceinline__ void tile_mul(const double* S1, const double* S2,
-                                         double (&c)[kRows][kCols]) {
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+__device__ __forceinline__ void tile_mul(const double* S1, const double* S2, Frag& c) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int mb = 32 * (w >> 1), nb = 32 * (w & 1);
+  const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll 2
-  for (int kk = 0; kk < kNB; ++kk) {
-    double x[kRows], y[kCols];
+  for (int k0 = 0; k0 < kNB; k0 += 4) {
+    double a[4], b[4];
 #pragma unroll
-    for (int a = 0; a < kRows; ++a) x[a] = S1[(ty + 8 * a) * kTLd + kk];
+    for (int m = 0; m < 4; ++m) a[m] = S1[(mb + 8 * m + g) * kPLd + k0 + t4];
 #pragma unroll
-    for (int b = 0; b < kCols; ++b)
-      y[b] = NT ? S2[(tx + 16 * b) * kTLd + kk] : S2[kk * kTLd + tx + 16 * b];
+    for (int n = 0; n < 4; ++n)
+      b[n] = NT ? S2[(nb + 8 * n + g) * kPLd + k0 + t4] : S2[(k0 + t4) * kPLd + nb + 8 * n + g];
 #pragma unroll
-    for (int a = 0; a < kRows; ++a)
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int b = 0; b < kCols; ++b) c[a][b] = fma(x[a], y[b], c[a][b]);
+      for (int n = 0; n < 4; ++n) dmma(a[m], b[n], c[m][n]);
   }
 }
 
 // c = sum over n steps of tile(G1(q)) x tile(G2(q)) (x: NT or NN), q = 0 .. n-1: fetch both
-// tiles, multiply (two tiles of shared memory; three CTAs per SM overlap one another's
+// tiles, multiply (two tiles of shared memory; several CTAs per SM overlap one another's
 // fetches and products).
 template <bool NT, class F1, class F2>
-__device__ __forceinline__ void tile_sum(double* sm, int n, F1 g1, F2 g2, int64_t ld,
-                                         double (&c)[kRows][kCols]) {
+__device__ __forceinline__ void tile_sum(double* sm, int n, F1 g1, F2 g2, int64_t ld, Frag& c) {
   for (int q = 0; q < n; ++q) {
     stage_async(sm, g1(q), ld);
-    stage_async(sm + kNB * kTLd, g2(q), ld);
+    stage_async(sm + kNB * kPLd, g2(q), ld);
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
-    tile_mul<NT>(sm, sm + kNB * kTLd, c);
+    tile_mul<NT>(sm, sm + kNB * kPLd, c);
     __syncthreads();
   }
 }
 
 // g = c (MODE 0), -c (1) or g - c (2); row-major tile, leading dimension ld.
 template <int MODE>
-__device__ __forceinline__ void put_tile(double* g, int64_t ld, const double (&c)[kRows][kCols]) {
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+__device__ __forceinline__ void put_tile(double* g, int64_t ld, const Frag& c) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int mb = 32 * (w >> 1), nb = 32 * (w & 1);
 #pragma unroll
-  for (int a = 0; a < kRows; ++a)
+  for (int m = 0; m < 4; ++m)
 #pragma unroll
-    for (int b = 0; b < kCols; ++b) {
-      double& o = g[(int64_t)(ty + 8 * a) * ld + tx + 16 * b];
-      o = MODE == 0 ? c[a][b] : (MODE == 1 ? -c[a][b] : o - c[a][b]);
+    for (int n = 0; n < 4; ++n) {
+      double2* q = reinterpret_cast<double2*>(
+          g + (int64_t)(mb + 8 * m + (lane >> 2)) * ld + nb + 8 * n + 2 * (lane & 3));
+      const double2 o = MODE == 2 ? *q : make_double2(0.0, 0.0);
+      if (MODE == 0) *q = make_double2(c[m][n][0], c[m][n][1]);
+      else if (MODE == 1) *q = make_double2(-c[m][n][0], -c[m][n][1]);
+      else *q = make_double2(o.x - c[m][n][0], o.y - c[m][n][1]);
     }
 }
 
@@ -247,7 +271,7 @@ __global__ void __launch_bounds__(kPThreads) k_trsm(double* A, const double* M, 
   const int64_t i = p + 1 + blockIdx.x;
   double* g = A + i * kNB * kp + (int64_t)p * kNB;
   const double* mpp = M + (int64_t)p * kNB * kp + (int64_t)p * kNB;
-  double c[kRows][kCols] = {};
+  Frag c = {};
   tile_sum<true>(sm, 1, [&](int) { return (const double*)g; }, [&](int) { return mpp; }, kp, c);
   put_tile<0>(g, kp, c);
 }
@@ -258,25 +282,36 @@ __global__ void __launch_bounds__(kPThreads)
 k_panel_update(double* A, int64_t kp, int p0, int p) {
   extern __shared__ double sm[];
   const int64_t i = p + blockIdx.x;
-  double c[kRows][kCols] = {};
+  Frag c = {};
   tile_sum<true>(sm, p - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  [&](int q) { return (const double*)(A + (int64_t)p * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  kp, c);
   put_tile<2>(A + i * kNB * kp + (int64_t)p * kNB, kp, c);
 }
 
-// Trailing update after the panel [p0, pe): A_ij -= sum_{t=p0}^{pe-1} L_it L_jt^T for
-// pe <= j <= i (lower tiles), one read-modify-write per tile.
-__global__ void __launch_bounds__(kPThreads) k_syrk(double* A, int64_t kp, int p0, int pe) {
+// Trailing update after the panel [p0, pe): A_ij -= sum_{t=p0}^{pe-1} L_it L_jt^T for the
+// lower tiles j <= i < nt with j0 <= j < j1, one read-modify-write per tile. tri: the grid
+// enumerates the triangle j0 <= j <= i < nt itself ((nt - j0)(nt - j0 + 1) / 2 CTAs; j1 = nt);
+// otherwise rows [j0, nt) by columns [j0, j1) ((nt - j0)(j1 - j0) CTAs, those above the
+// diagonal return).
+__global__ void __launch_bounds__(kPThreads)
+k_syrk(double* A, int64_t kp, int p0, int pe, int j0, int j1, bool tri) {
   extern __shared__ double sm[];
-  // blockIdx.x -> (ii, jj), jj <= ii
-  const int64_t idx = blockIdx.x;
-  int64_t ii = (int64_t)((sqrt(8.0 * (double)idx + 1.0) - 1.0) / 2.0);
-  while (ii * (ii + 1) / 2 > idx) --ii;
-  while ((ii + 1) * (ii + 2) / 2 <= idx) ++ii;
-  const int64_t jj = idx - ii * (ii + 1) / 2;
-  const int64_t i = pe + ii, j = pe + jj;
-  double c[kRows][kCols] = {};
+  int64_t i, j;
+  if (tri) {                               // blockIdx.x -> (ii, jj), jj <= ii
+    const int64_t idx = blockIdx.x;
+    int64_t ii = (int64_t)((sqrt(8.0 * (double)idx + 1.0) - 1.0) / 2.0);
+    while (ii * (ii + 1) / 2 > idx) --ii;
+    while ((ii + 1) * (ii + 2) / 2 <= idx) ++ii;
+    i = j0 + ii;
+    j = j0 + (idx - ii * (ii + 1) / 2);
+  } else {                                 // band of columns: rows x columns
+    const int w = j1 - j0;
+    i = j0 + blockIdx.x / w;
+    j = j0 + blockIdx.x % w;
+    if (j > i) return;
+  }
+  Frag c = {};
   tile_sum<true>(sm, pe - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  [&](int q) { return (const double*)(A + j * kNB * kp + (int64_t)(p0 + q) * kNB); },
                  kp, c);
@@ -295,7 +330,7 @@ k_inv_a(double* A, const double* M, int64_t kp, int nt, int s) {
   const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
   const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
   if (i >= nt) return;
-  double c[kRows][kCols] = {};
+  Frag c = {};
   // T_ij = sum_{kk = j}^{a0 + s - 1} L_i,kk M_kk,j  (M_kk,j = 0 for kk < j)
   tile_sum<false>(sm, (int)(a0 + s - j),
                   [&](int q) { return (const double*)(A + i * kNB * kp + (j + q) * kNB); },
@@ -309,7 +344,7 @@ k_inv_b(const double* A, double* M, int64_t kp, int nt, int s) {
   const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
   const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
   if (i >= nt) return;
-  double c[kRows][kCols] = {};
+  Frag c = {};
   // M_ij = -sum_{kk = a0 + s}^{i} M_i,kk T_kk,j  (T_kk,j kept at tile (j, kk))
   tile_sum<false>(sm, (int)(i - a0 - s + 1),
                   [&](int q) { return (const double*)(M + i * kNB * kp + (a0 + s + q) * kNB); },
@@ -327,6 +362,36 @@ __global__ void k_factor_store(FactorArgs a) {
   }
 }
 
+}  // namespace
+
+namespace {
+// Two streams and events for the factor's look-ahead, one set per device, created on first
+// use; calls on one device enqueue under its mutex. chain (the highest priority) carries the
+// panel factorisations, side (the lowest) the bulk trailing updates, so the block scheduler
+// serves the serial chain first whenever both have CTAs waiting.
+struct FactorStreams {
+  std::mutex mu;
+  cudaStream_t chain = nullptr, side = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_panel = nullptr, ev_rest = nullptr, ev_end = nullptr,
+              ev_done = nullptr;
+};
+FactorStreams& factor_streams() {
+  static FactorStreams fs[64];
+  static std::mutex init_mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  FactorStreams& f = fs[dev < 0 || dev >= 64 ? 0 : dev];
+  std::lock_guard<std::mutex> lk(init_mu);
+  if (!f.side) {
+    int least = 0, greatest = 0;
+    cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    cudaStreamCreateWithPriority(&f.chain, cudaStreamNonBlocking, greatest);
+    cudaStreamCreateWithPriority(&f.side, cudaStreamNonBlocking, least);
+    for (cudaEvent_t* e : {&f.ev_start, &f.ev_panel, &f.ev_rest, &f.ev_end, &f.ev_done})
+      cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+  }
+  return f;
+}
 }  // namespace
 
 size_t gptq_factor_workspace(int64_t k) {
@@ -352,26 +417,55 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   FactorArgs a{H, k, kp, B, perm, (double*)(w + 256), (double*)(w + 256) + kp * kp,
                (double*)w, U};
   const int gs = sm_count() * 8;
-  k_factor_lambda<<<1, kFThreads, 0, st>>>(H, k, damp, a.scal);
-  k_factor_load<<<gs, 256, 0, st>>>(a);
-  // right-looking over panels of kPanelTiles tile columns, left-looking inside a panel
+  // Right-looking over panels of kPanelTiles tile columns, left-looking inside a panel, with
+  // a look-ahead of one panel: after panel P is factored (stream chain), its update of the
+  // next panel's columns runs on chain, its update of everything beyond on side while chain
+  // factors panel P + 1; panel P + 1's column update waits for the previous panel's update
+  // of everything beyond (both write those tiles). The two streams fork from and join the
+  // caller's stream.
+  FactorStreams& fs = factor_streams();
+  std::lock_guard<std::mutex> lk(fs.mu);
+  cudaStream_t cs = fs.chain;
+  cudaEventRecord(fs.ev_start, st);
+  cudaStreamWaitEvent(cs, fs.ev_start, 0);
+  cudaStreamWaitEvent(fs.side, fs.ev_start, 0);
+  k_factor_lambda<<<1, kFThreads, 0, cs>>>(H, k, damp, a.scal);
+  k_factor_load<<<gs, 256, 0, cs>>>(a);
+  bool rest_pending = false;
   for (int p0 = 0; p0 < nt; p0 += kPanelTiles) {
     const int pe = (int)(p0 + kPanelTiles < nt ? p0 + kPanelTiles : nt);
     for (int p = p0; p < pe; ++p) {
-      if (p > p0) k_panel_update<<<(unsigned)(nt - p), kPThreads, kProdSmem1, st>>>(a.A, kp, p0, p);
-      k_potrf_inv<<<1, kFThreads, kTwoTiles, st>>>(a.A, a.M, kp, p);
+      if (p > p0) k_panel_update<<<(unsigned)(nt - p), kPThreads, kProdSmem1, cs>>>(a.A, kp, p0, p);
+      k_potrf_inv<<<1, kFThreads, kTwoTiles, cs>>>(a.A, a.M, kp, p);
       if (nt - 1 - p > 0)
-        k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem1, st>>>(a.A, a.M, kp, p);
+        k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, p);
     }
-    const int64_t m = nt - pe;
-    if (m > 0) k_syrk<<<(unsigned)(m * (m + 1) / 2), kPThreads, kProdSmem1, st>>>(a.A, kp, p0, pe);
+    if (pe >= nt) break;
+    const int pn = (int)(pe + kPanelTiles < nt ? pe + kPanelTiles : nt);   // next panel's end
+    if (rest_pending) cudaStreamWaitEvent(cs, fs.ev_rest, 0);
+    k_syrk<<<(unsigned)((nt - pe) * (pn - pe)), kPThreads, kProdSmem1, cs>>>(a.A, kp, p0, pe, pe,
+                                                                            pn, false);
+    rest_pending = false;
+    if (pn < nt) {
+      cudaEventRecord(fs.ev_panel, cs);
+      cudaStreamWaitEvent(fs.side, fs.ev_panel, 0);
+      const int64_t m = nt - pn;
+      k_syrk<<<(unsigned)(m * (m + 1) / 2), kPThreads, kProdSmem1, fs.side>>>(a.A, kp, p0, pe, pn,
+                                                                              (int)nt, true);
+      cudaEventRecord(fs.ev_rest, fs.side);
+      rest_pending = true;
+    }
   }
+  cudaEventRecord(fs.ev_end, fs.side);
+  cudaStreamWaitEvent(cs, fs.ev_end, 0);
   for (int s = 1; s < nt; s *= 2) {
     const dim3 grid((unsigned)(s * s), (unsigned)((nt + 2 * s - 1) / (2 * s)));
-    k_inv_a<<<grid, kPThreads, kProdSmem1, st>>>(a.A, a.M, kp, (int)nt, s);
-    k_inv_b<<<grid, kPThreads, kProdSmem1, st>>>(a.A, a.M, kp, (int)nt, s);
+    k_inv_a<<<grid, kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, (int)nt, s);
+    k_inv_b<<<grid, kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, (int)nt, s);
   }
-  k_factor_store<<<gs, 256, 0, st>>>(a);
+  k_factor_store<<<gs, 256, 0, cs>>>(a);
+  cudaEventRecord(fs.ev_done, cs);
+  cudaStreamWaitEvent(st, fs.ev_done, 0);
   return cudaGetLastError();
 }
 

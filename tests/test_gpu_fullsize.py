@@ -221,3 +221,31 @@ def test_gptq_ordered_full_size(mxq, orc, synth):
                         n_threads=NT)
     assert np.array_equal(scales[ri].cpu().numpy(), r.scales)
     assert np.array_equal(codes[ri].cpu().numpy(), r.codes)
+
+
+def test_gptq_tiles_full_size(mxq, orc, synth):
+    """FP8-GPTQ on the 64 x 64 tiles of the 4096 x 4096 weight: the oracle's Gram blocks of
+    all 8192 activation rows, its factors and its tile scales (two sampled tile rows,
+    uploaded); those tile rows of the GPU sweep bit-exact, the factors within one float32
+    rounding."""
+    wl = synth.WORKLOADS["e4m3_tiles"]
+    W = synth.workload_weight(wl, 0, device=DEV)
+    n, k = W.shape
+    X = oracle_view(synth.workload_activations(wl, 0, device="cpu"))
+    G = orc.block_gram(X, 64)
+    U = orc.gptq_prepare(G)
+    Ug = mxq.mxq_gptq_prepare(torch.from_numpy(G).to(DEV)).cpu().numpy()
+    tol = 2.0 ** -23 * np.abs(U) + 2.0 ** -30 * np.abs(U).max(axis=(1, 2), keepdims=True)
+    assert np.all(np.abs(Ug.astype(np.float64) - U) <= tol)
+    h = orc.act_sqmean(X, n_threads=NT)
+    scales = np.zeros((n // 64, k // 64), np.float32)
+    tile_rows = synth.sample_rows(n // 64, 2, wl.seed + 61).numpy()
+    for tr in tile_rows:
+        r = orc.quantize(oracle_view(W[tr * 64:(tr + 1) * 64]), "e4m3", "hopt", 64, h=h,
+                         n_threads=NT)
+        scales[tr] = r.scales[0]
+    codes = mxq.mxq_gptq_tiles(W, torch.from_numpy(U).to(DEV),
+                               torch.from_numpy(scales).to(DEV)).cpu().numpy()
+    for tr in tile_rows:
+        ref = orc.gptq_tiles(oracle_view(W[tr * 64:(tr + 1) * 64]), U, scales[tr:tr + 1])
+        assert np.array_equal(codes[tr * 64:(tr + 1) * 64], ref), f"tile row {tr}"
