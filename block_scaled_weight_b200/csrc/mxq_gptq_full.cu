@@ -527,20 +527,26 @@ __device__ __forceinline__ int elem_project(float a, float4 t, float& wq_abs) {
   else return (int)g;
 }
 
-// The definition's candidate error sum_j c_j (w_j - wq_j)^2: double, element order,
-// each operation rounded once.
+// The definition's candidate errors sum_j c_j (w_j - wq_j)^2 for four candidates at once
+// (independent accumulation chains): double, element order, each operation rounded once.
 template <int B, int ELEM, bool HOPT>
-__device__ __forceinline__ double exact_error(const float* wb, const float* cw, float4 t) {
-  double e = 0.0;
-#pragma unroll 4
+__device__ __forceinline__ void exact_error4(const float* wb, const float* cw,
+                                             const float4 (&t)[4], double (&e)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) e[q] = 0.0;
+#pragma unroll 2
   for (int j = 0; j < B; ++j) {
-    float wq_abs;
-    elem_project<ELEM>(fabsf(wb[j]), t, wq_abs);
-    const double d = __dsub_rn((double)wb[j], (double)copysignf(wq_abs, wb[j]));
+    const float w = wb[j];
+    const double wd = (double)w;
     const double c = HOPT ? (double)cw[j] : 1.0;
-    e = __dadd_rn(e, __dmul_rn(c, __dmul_rn(d, d)));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float wq_abs;
+      elem_project<ELEM>(fabsf(w), t[q], wq_abs);
+      const double d = __dsub_rn(wd, (double)copysignf(wq_abs, w));
+      e[q] = __dadd_rn(e[q], __dmul_rn(c, __dmul_rn(d, d)));
+    }
   }
-  return e;
 }
 
 // One warp per row; lane l holds panel positions 2l and 2l + 1.
@@ -587,9 +593,16 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S) {
       grid_window(tab, T.ncodes, T.first, c0, a.window, lo, hi);
       double be = __longlong_as_double(0x7ff0000000000000LL);   // +inf
       int bc = 0x7fffffff;
-      for (int c = lo + lane; c <= hi; c += 32) {
-        const double e = exact_error<B, ELEM, MODE == 2>(wb[wid], hs + q0, tab[c]);
-        if (e < be) { be = e; bc = c; }
+      // candidates lo + lane + 32 (4 g + q), four per pass (ascending within the lane)
+      for (int cb = lo + lane; cb <= hi; cb += 128) {
+        float4 tq[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tq[q] = tab[min(cb + 32 * q, hi)];
+        double e[4];
+        exact_error4<B, ELEM, MODE == 2>(wb[wid], hs + q0, tq, e);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (cb + 32 * q <= hi && e[q] < be) { be = e[q]; bc = cb + 32 * q; }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {

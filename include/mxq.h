@@ -376,6 +376,9 @@ MXQ_API mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64
  *   damp    finite, >= 0 (GPTQ's customary 0.01).
  *   workspace  mxq_gptq_factor_workspace(k) bytes (two float64 k x k matrices, k rounded
  *           up to a multiple of 64), 16-byte aligned.
+ *   The call is asynchronous like the others: its kernels run on two streams of the library
+ *   (one per device, created on first use) that wait for `stream` and that `stream` waits
+ *   for before its next work; concurrent calls on one device are ordered on the host.
  *
  * mxq_gptq_order: the ordered variant's block sequence. loss_b = sum over rows and the
  *  block's columns of h_j (w_ij - w^_ij)^2 (float64) for the plain quantizer's result
