@@ -659,6 +659,28 @@ def gpu_arm(args):
         dist.destroy_process_group()
 
 
+def gptq_launches(k, ordered, panel_tiles=4):
+    """Our kernels per GPTQ step (the Hessian GEMM is cuBLAS's): h pass 2, [order: search,
+    fixup, block losses, sort], factor (lambda, load, per tile column: panel update (not the
+    panel's first), diagonal tile, tiles below (not the last); per panel but the last: the
+    next panel's columns and, while any remain, everything beyond; 2 per doubling level;
+    store), sweep (init, 64-position panels, trailing updates), error 2."""
+    nt = (k + 63) // 64
+    f = 2 + 1
+    for p0 in range(0, nt, panel_tiles):
+        pe = min(p0 + panel_tiles, nt)
+        for p in range(p0, pe):
+            f += (p > p0) + 1 + (p < nt - 1)
+        if pe < nt:
+            f += 1 + (min(pe + panel_tiles, nt) < nt)
+    s = 1
+    while s < nt:
+        f += 2
+        s *= 2
+    panels = (k + 63) // 64
+    return 2 + (4 if ordered else 0) + f + 1 + panels + (panels - 1) + 2
+
+
 def bf16_peak():
     try:
         with open(PEAKS_FILE) as f:
@@ -719,9 +741,7 @@ def gpu_arm_gptq(args, wl, q):
                ("error", lambda: mxq.mxq_error(W, codes, scales, p, h, sums=sums,
                                                workspace=ews))]
     stream = torch.cuda.current_stream(dev)
-    nt = (k + 63) // 64
-    panels = (k + 63) // 64
-    launches_per_step = (2 + (4 if ordered else 0) + (4 * nt + 1) + 2 * panels + 2)
+    launches_per_step = gptq_launches(k, ordered)
 
     def step(ev=None):
         for i, (_, fn) in enumerate(phases):

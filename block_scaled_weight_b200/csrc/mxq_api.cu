@@ -529,7 +529,7 @@ mxq_status mxq_gptq(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t 
   s = check_gptq_params(p, n, k);
   if (s != MXQ_OK) return s;
   if (n == 0 || k == 0) return MXQ_OK;
-  if (n > 0x7fffffff / 8) return fail(MXQ_ERR_SHAPE, "n beyond 2^28");
+  if (n > (int64_t)65535 * 64) return fail(MXQ_ERR_SHAPE, "n beyond 65535 x 64 rows");
   if (!U || !codes || !scales) return fail(MXQ_ERR_INVALID_ARG, "U, codes or scales is NULL");
   if (!aligned(U, 16) || !aligned(codes, 16) || (perm && !aligned(perm, 4)))
     return fail(MXQ_ERR_ALIGN, "U or codes not 16-byte, or perm not 4-byte aligned");

@@ -353,16 +353,20 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-int gram_chunks(int64_t rows, int64_t cols) {
+int gram_chunks(int64_t rows, int64_t cols, int B) {
   const int64_t strips = (cols + kGramCols - 1) / kGramCols;
   const int64_t stages = (rows + kGramRows - 1) / kGramRows;
   int64_t want = (8 * 2 * (int64_t)sm_count() + strips - 1) / strips;  // ~8 waves of 2 CTAs/SM
+  // the partial sums (chunks x cols x B doubles, written and read back) stay within a quarter
+  // of X's bytes: chunks <= rows / (16 B)
+  const int64_t cap = rows / (16 * (int64_t)B);
+  if (want > cap) want = cap;
   if (want > stages) want = stages;
   return (int)(want < 1 ? 1 : want);
 }
 
 size_t gram_workspace(int64_t rows, int64_t cols, int B) {
-  return 256 + (size_t)gram_chunks(rows, cols) * (size_t)cols * (size_t)B * sizeof(double);
+  return 256 + (size_t)gram_chunks(rows, cols, B) * (size_t)cols * (size_t)B * sizeof(double);
 }
 
 cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, int B, float* G,
@@ -379,7 +383,7 @@ cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, i
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const int chunks = gram_chunks(rows, cols);
+  const int chunks = gram_chunks(rows, cols, B);
   const int64_t stages = (rows + kGramRows - 1) / kGramRows;
   const int64_t per_chunk = (stages + chunks - 1) / chunks * kGramRows;
   int* err = (int*)workspace;

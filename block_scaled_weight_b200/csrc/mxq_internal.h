@@ -22,7 +22,7 @@ cudaError_t launch_hpass_finalize(const double* partial, int64_t parts, int64_t 
 
 // ---- Gram blocks (tensor cores) ---------------------------------------------------------
 // G [cols/B][B][B] = fl32(X_b^T X_b / rows) and optionally h = diag(G), for bf16 X.
-int gram_chunks(int64_t rows, int64_t cols);
+int gram_chunks(int64_t rows, int64_t cols, int B);
 size_t gram_workspace(int64_t rows, int64_t cols, int B);
 cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, int B, float* G,
                         float* h, void* workspace, cudaStream_t st);

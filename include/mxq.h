@@ -402,7 +402,7 @@ MXQ_API mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64
  *           output for the same perm; codes / scales: mxq_quantize's layouts (original
  *           column order).
  *   workspace  mxq_gptq_workspace(n, k) bytes (the working weights, n x k float32),
- *           16-byte aligned.
+ *           16-byte aligned. n <= 65535 x 64.
  *  Result: identical to the definition above, including ties (each scale search scores
  *  every candidate exactly in float64, element order; lowest code on equal errors).
  * ------------------------------------------------------------------------------------ */
