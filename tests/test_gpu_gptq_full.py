@@ -222,3 +222,35 @@ def test_rejections(mxq):
         mxq.mxq_gptq_factor(torch.zeros(64, 64, device=DEV), 16, damp=float("inf"))
     with pytest.raises(mxq.MxqError):
         mxq.mxq_act_gram(torch.zeros(8, 64, device=DEV))              # float32 X
+
+
+@pytest.mark.parametrize("fmt,sfmt,B,mode", [("nvfp4", "e4m3", 16, "hopt"), ("nvfp4", "ue8m0", 32, "sse"),
+                                             ("int4", "e4m3", 16, "naive"),
+                                             ("nvfp4", "ue5m3", 16, "hopt")])
+def test_sweep_special_values(mxq, orc, fmt, sfmt, B, mode):
+    """All-zero and negative-zero blocks (every candidate ties at zero error), saturating and
+    subnormal-scale blocks, a dead input channel (h = 0), and a factor with negative and
+    zero couplings -- bit-exact with the oracle on the same factor."""
+    rng = np.random.default_rng(17)
+    n, k = 12, 128
+    W = (rng.standard_t(4, (n, k)) * 0.05).astype(np.float32)
+    W[0, :] = 0.0
+    W[1, :] = -0.0
+    W[2, :B] = 1e30                                    # far above every scale's range
+    W[3, :] *= 1e-30                                   # scales in the subnormal corner
+    W[4, ::7] = 0.0
+    W[5, B:2 * B] = -W[5, :B]
+    h = np.exp(rng.normal(0, 1, k)).astype(np.float32)
+    h[5] = 0.0
+    A = rng.standard_normal((300, k)).astype(np.float32)
+    A[:, 1::2] -= 0.7 * A[:, 0::2]
+    H = (A.T @ A / 300).astype(np.float32)
+    U = orc.gptq_prepare(H[None])[0]
+    U[0, 1:5] = 0.0
+    p = mxq.params(fmt, mode, B, scale_fmt=sfmt)
+    Wt = torch.from_numpy(W).to(DEV)
+    codes, scales = mxq.mxq_gptq(Wt, torch.from_numpy(U).to(DEV), p, torch.from_numpy(h).to(DEV))
+    torch.cuda.synchronize()
+    r = orc.gptq_blocks(W, U, h, fmt, mode, B, sfmt=sfmt)
+    assert np.array_equal(scales.cpu().numpy(), r.scales)
+    assert np.array_equal(codes.cpu().numpy(), r.codes)
