@@ -45,7 +45,7 @@ L2_BYTES = 126 * 1024 * 1024
 ALU_PEAK_TOPS = 148 * 128 * 1.965e9 / 1e12
 # Oracle samples: the cpu_baseline leg (about 10-30 s of CPU work) and each step of the
 # reference arm (well under a second, so that a long --steps run stays short).
-CPU_X_ROWS, CPU_W_ROWS = 32768, 1024
+CPU_X_ROWS, CPU_W_ROWS = 65536, 4096
 GPTQ_CPU_X_ROWS, GPTQ_CPU_W_ROWS = 4096, 16
 Quantizer = collections.namedtuple("Quantizer", "fmt block mode window sfmt")
 HEADLINE_Q = Quantizer("nvfp4", 16, "hopt", -1, "e4m3")

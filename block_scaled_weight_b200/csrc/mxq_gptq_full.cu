@@ -487,7 +487,7 @@ struct SweepArgs {
   const int32_t* perm;   // [k / B] or null
   int window;
   float* Wc;             // [n][k] working weights, sweep order
-  float* Err;            // [n][kPanel] the panel's residuals
+  float* Err;            // 2 x [n][kPanel]: the residuals of alternate panels
   uint8_t* codes;        // [n][k / 2]
   uint8_t* scales;       // [n][k / B]
 };
@@ -552,7 +552,7 @@ __device__ __forceinline__ void exact_error4(const float* wb, const float* cw,
 // One warp per row; lane l holds panel positions 2l and 2l + 1.
 template <int B, int ELEM, int MODE>
 __global__ void __launch_bounds__(kPanelWarps * 32)
-k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S) {
+k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Err) {
   __shared__ float4 tab[256];
   __shared__ float Us[kPanel][kPanel + 1];
   __shared__ float hs[kPanel];
@@ -659,13 +659,13 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S) {
   if (live) {
     const int64_t c = pos_col<B>(a, p0 + 2 * lane);    // even: both nibbles share a byte
     a.codes[r * (a.k / 2) + c / 2] = (uint8_t)nib;
-    *reinterpret_cast<float2*>(a.Err + r * kPanel + 2 * lane) = err2;
+    *reinterpret_cast<float2*>(Err + r * kPanel + 2 * lane) = err2;
   }
 }
 
-// Later positions p >= p0 + S: for each block of the panel (in order)
-// acc = sum_j fma(err_j, U[j][p], acc) over the block's columns, then w -= acc.
-// CTA: 64 positions x rg groups of 64 rows; thread: 4 rows x 4 consecutive positions. The
+// Later positions p in [cbeg, cend) (after the panel [p0, p0 + S)): for each block of the
+// panel (in order) acc = sum_j fma(err_j, U[j][p], acc) over the block's columns, then
+// w -= acc. CTA: 64 positions x rg groups of 64 rows; thread: 4 rows x 4 consecutive positions. The
 // CTA's rows of U are staged once; the residuals of the next row group are fetched with
 // cp.async while the current group is updated.
 constexpr int kEsLd = kPanel + 4;        // padded residual row (16-byte aligned)
@@ -678,18 +678,19 @@ __device__ __forceinline__ void cp_async16(float* s, const float* g) {
 
 template <int B>
 __global__ void __launch_bounds__(kTrailThreads)
-k_gptq_trailing(SweepArgs a, int64_t p0, int S, int rg) {
+k_gptq_trailing(SweepArgs a, const float* __restrict__ Err, int64_t p0, int S, int64_t cbeg,
+                int64_t cend, int rg) {
   extern __shared__ __align__(16) float tsm[];
   float (*Es)[64 * kEsLd] = reinterpret_cast<float (*)[64 * kEsLd]>(tsm);
   float (*Ut)[64] = reinterpret_cast<float (*)[64]>(tsm + 2 * 64 * kEsLd);
-  const int64_t c0 = p0 + S + (int64_t)blockIdx.x * 64;
+  const int64_t c0 = cbeg + (int64_t)blockIdx.x * 64;
   const int64_t groups = (a.n + 63) / 64;
   const int64_t g0 = (int64_t)blockIdx.y * rg;
   const int ng = (int)(groups - g0 < rg ? groups - g0 : rg);
   auto stage_es = [&](int buf, int64_t r0) {
     for (int e = threadIdx.x; e < 64 * (kPanel / 4); e += kTrailThreads) {
       const int i = e / (kPanel / 4), q = e % (kPanel / 4);
-      if (r0 + i < a.n) cp_async16(&Es[buf][i * kEsLd + 4 * q], a.Err + (r0 + i) * kPanel + 4 * q);
+      if (r0 + i < a.n) cp_async16(&Es[buf][i * kEsLd + 4 * q], Err + (r0 + i) * kPanel + 4 * q);
     }
   };
   stage_es(0, g0 * 64);
@@ -697,13 +698,13 @@ k_gptq_trailing(SweepArgs a, int64_t p0, int S, int rg) {
   for (int e = threadIdx.x; e < kPanel * 16; e += kTrailThreads) {
     const int j = e / 16, g = e % 16;
     float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < S && c0 + 4 * g < a.k)
+    if (j < S && c0 + 4 * g < cend)
       u = *reinterpret_cast<const float4*>(a.U + (p0 + j) * a.k + c0 + 4 * g);
     *reinterpret_cast<float4*>(&Ut[j][4 * g]) = u;
   }
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const int64_t col = c0 + 4 * tx;
-  const bool on = col < a.k;
+  const bool on = col < cend;
   for (int g = 0; g < ng; ++g) {
     const int64_t r0 = (g0 + g) * 64;
     if (g + 1 < ng) stage_es((g + 1) & 1, r0 + 64);
@@ -751,36 +752,68 @@ k_gptq_trailing(SweepArgs a, int64_t p0, int S, int rg) {
   }
 }
 
+template <int B>
+void launch_trailing(const SweepArgs& a, const float* Err, int64_t p0, int S, int64_t cbeg,
+                     int64_t cend, cudaStream_t st) {
+  // row groups per CTA: as many as keep at least ~4 CTAs per SM
+  const int64_t ctiles = (cend - cbeg + 63) / 64, groups = (a.n + 63) / 64;
+  int64_t rg = ctiles * groups / ((int64_t)sm_count() * 4);
+  rg = rg < 1 ? 1 : (rg > 8 ? 8 : rg);
+  const dim3 grid((unsigned)ctiles, (unsigned)((groups + rg - 1) / rg));
+  k_gptq_trailing<B><<<grid, kTrailThreads, kTrailSmem, st>>>(a, Err, p0, S, cbeg, cend, (int)rg);
+}
+
+// Panels of 64 positions with a look-ahead of one panel, as the factor: panel t's update of
+// the next 64 positions runs on the chain stream (the next panel needs only those), its
+// update of everything beyond on the side stream while the chain runs panel t + 1; the
+// residuals alternate between two buffers, and the next-64 update of panel t + 1 waits for
+// panel t's update beyond (both write those positions).
 template <int B, int ELEM>
 cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cudaStream_t st) {
   static const bool attr = cudaFuncSetAttribute(k_gptq_trailing<B>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 (int)kTrailSmem) == cudaSuccess;
   if (!attr) return cudaErrorInvalidConfiguration;
-  k_sweep_init<B><<<sm_count() * 8, 256, 0, st>>>(a);
+  FactorStreams& fs = factor_streams();
+  std::lock_guard<std::mutex> lk(fs.mu);
+  cudaStream_t cs = fs.chain;
+  cudaEventRecord(fs.ev_start, st);
+  cudaStreamWaitEvent(cs, fs.ev_start, 0);
+  cudaStreamWaitEvent(fs.side, fs.ev_start, 0);
+  k_sweep_init<B><<<sm_count() * 8, 256, 0, cs>>>(a);
   const unsigned prow = (unsigned)((a.n + kPanelWarps - 1) / kPanelWarps);
-  for (int64_t p0 = 0; p0 < a.k; p0 += kPanel) {
+  bool rest_pending = false;
+  int t = 0;
+  for (int64_t p0 = 0; p0 < a.k; p0 += kPanel, ++t) {
     const int S = (int)(a.k - p0 < kPanel ? a.k - p0 : kPanel);
-    if (mode == 0) k_gptq_panel<B, ELEM, 0><<<prow, kPanelWarps * 32, 0, st>>>(a, T, p0, S);
-    else if (mode == 1) k_gptq_panel<B, ELEM, 1><<<prow, kPanelWarps * 32, 0, st>>>(a, T, p0, S);
-    else k_gptq_panel<B, ELEM, 2><<<prow, kPanelWarps * 32, 0, st>>>(a, T, p0, S);
-    const int64_t rest = a.k - p0 - S;
-    if (rest > 0) {
-      // row groups per CTA: as many as keep at least ~4 CTAs per SM
-      const int64_t ctiles = (rest + 63) / 64, groups = (a.n + 63) / 64;
-      int64_t rg = ctiles * groups / ((int64_t)sm_count() * 4);
-      rg = rg < 1 ? 1 : (rg > 8 ? 8 : rg);
-      const dim3 grid((unsigned)ctiles, (unsigned)((groups + rg - 1) / rg));
-      k_gptq_trailing<B><<<grid, kTrailThreads, kTrailSmem, st>>>(a, p0, S, (int)rg);
+    float* err = a.Err + (t & 1) * a.n * kPanel;
+    if (mode == 0) k_gptq_panel<B, ELEM, 0><<<prow, kPanelWarps * 32, 0, cs>>>(a, T, p0, S, err);
+    else if (mode == 1) k_gptq_panel<B, ELEM, 1><<<prow, kPanelWarps * 32, 0, cs>>>(a, T, p0, S, err);
+    else k_gptq_panel<B, ELEM, 2><<<prow, kPanelWarps * 32, 0, cs>>>(a, T, p0, S, err);
+    const int64_t c1 = p0 + S, c2 = c1 + kPanel < a.k ? c1 + kPanel : a.k;
+    if (c1 >= a.k) break;
+    if (rest_pending) cudaStreamWaitEvent(cs, fs.ev_rest, 0);
+    launch_trailing<B>(a, err, p0, S, c1, c2, cs);
+    rest_pending = false;
+    if (c2 < a.k) {
+      cudaEventRecord(fs.ev_panel, cs);
+      cudaStreamWaitEvent(fs.side, fs.ev_panel, 0);
+      launch_trailing<B>(a, err, p0, S, c2, a.k, fs.side);
+      cudaEventRecord(fs.ev_rest, fs.side);
+      rest_pending = true;
     }
   }
+  cudaEventRecord(fs.ev_end, fs.side);
+  cudaStreamWaitEvent(cs, fs.ev_end, 0);
+  cudaEventRecord(fs.ev_done, cs);
+  cudaStreamWaitEvent(st, fs.ev_done, 0);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t gptq_sweep_workspace(int64_t n, int64_t k) {
-  return (size_t)n * (size_t)k * sizeof(float) + (size_t)n * kPanel * sizeof(float) + 256;
+  return (size_t)n * (size_t)k * sizeof(float) + 2 * (size_t)n * kPanel * sizeof(float) + 256;
 }
 
 cudaError_t launch_gptq_sweep(const GptqArgs& g, cudaStream_t st) {
