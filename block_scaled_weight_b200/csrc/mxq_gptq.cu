@@ -172,7 +172,8 @@ k_gptq_tiles(SweepParams P) {
     }
     uint4* dst = reinterpret_cast<uint4*>(P.codes + row * P.k + (int64_t)tj * kT);
 #pragma unroll
-    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(cw[4 * v], cw[4 * v + 1], cw[4 * v + 2], cw[4 * v + 3]);
+    for (int v = 0; v < 4; ++v)
+      dst[v] = make_uint4(cw[4 * v], cw[4 * v + 1], cw[4 * v + 2], cw[4 * v + 3]);
   }
 }
 
@@ -183,7 +184,8 @@ constexpr size_t kPrepSmem = 2 * kT * kLd * sizeof(double);
 cudaError_t launch_gptq_prepare(const float* G, int64_t nblocks, double damp, float* U,
                                 cudaStream_t st) {
   if (nblocks <= 0) return cudaSuccess;
-  static bool set = cudaFuncSetAttribute(k_gptq_prepare, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static bool set = cudaFuncSetAttribute(k_gptq_prepare,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kPrepSmem) == cudaSuccess;
   if (!set) return cudaErrorInvalidConfiguration;
   k_gptq_prepare<<<(unsigned)nblocks, kPrepThreads, kPrepSmem, st>>>(G, damp, U);

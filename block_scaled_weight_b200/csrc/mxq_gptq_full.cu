@@ -7,7 +7,8 @@
 //           order (a block permutation for the ordered variant), in float64, rounded to
 //           float32 once. With J the order reversal, J H J = L L^T gives H^-1 = U^T U with
 //           U = J L^-1 J, so one blocked Cholesky and one blocked triangular inverse (64 x 64
-//           tiles, float64 on the CUDA cores) replace GPTQ's inverse-then-Cholesky.
+//           tiles, float64 products on the tensor cores) replace GPTQ's
+//           inverse-then-Cholesky.
 //   order   (ordered variant) the Hessian-weighted loss of every column block under the
 //           plain quantizer, and the blocks sorted by descending loss.
 //   sweep   rows are independent. Positions are processed in panels of up to 64: one warp
@@ -15,7 +16,8 @@
 //           candidate's error in double, element order, lowest code on ties), quantises
 //           the block's columns one after another with the in-block updates, and applies
 //           each block's product to the panel's later blocks; a tiled kernel then applies
-//           the panel's block products to every later position of every row.
+//           the panel's block products to every later position of every row (the next
+//           panel's positions first, the rest overlapping the next panel).
 // Every float32 step follows the definition's operation order: in-block updates
 // w -= fl32(err U), past the block acc = fma(err_j, U_j, acc) over the block's columns in
 // order, then one subtraction.
@@ -283,9 +285,10 @@ k_panel_update(double* A, int64_t kp, int p0, int p) {
   extern __shared__ double sm[];
   const int64_t i = p + blockIdx.x;
   Frag c = {};
-  tile_sum<true>(sm, p - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
-                 [&](int q) { return (const double*)(A + (int64_t)p * kNB * kp + (int64_t)(p0 + q) * kNB); },
-                 kp, c);
+  const double* rowi = A + i * kNB * kp + (int64_t)p0 * kNB;
+  const double* rowp = A + (int64_t)p * kNB * kp + (int64_t)p0 * kNB;
+  tile_sum<true>(sm, p - p0, [&](int q) { return rowi + (int64_t)q * kNB; },
+                 [&](int q) { return rowp + (int64_t)q * kNB; }, kp, c);
   put_tile<2>(A + i * kNB * kp + (int64_t)p * kNB, kp, c);
 }
 
@@ -312,9 +315,10 @@ k_syrk(double* A, int64_t kp, int p0, int pe, int j0, int j1, bool tri) {
     if (j > i) return;
   }
   Frag c = {};
-  tile_sum<true>(sm, pe - p0, [&](int q) { return (const double*)(A + i * kNB * kp + (int64_t)(p0 + q) * kNB); },
-                 [&](int q) { return (const double*)(A + j * kNB * kp + (int64_t)(p0 + q) * kNB); },
-                 kp, c);
+  const double* rowi = A + i * kNB * kp + (int64_t)p0 * kNB;
+  const double* rowj = A + j * kNB * kp + (int64_t)p0 * kNB;
+  tile_sum<true>(sm, pe - p0, [&](int q) { return rowi + (int64_t)q * kNB; },
+                 [&](int q) { return rowj + (int64_t)q * kNB; }, kp, c);
   put_tile<2>(A + i * kNB * kp + j * kNB, kp, c);
 }
 
@@ -665,9 +669,9 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Er
 
 // Later positions p in [cbeg, cend) (after the panel [p0, p0 + S)): for each block of the
 // panel (in order) acc = sum_j fma(err_j, U[j][p], acc) over the block's columns, then
-// w -= acc. CTA: 64 positions x rg groups of 64 rows; thread: 4 rows x 4 consecutive positions. The
-// CTA's rows of U are staged once; the residuals of the next row group are fetched with
-// cp.async while the current group is updated.
+// w -= acc. CTA: 64 positions x rg groups of 64 rows; thread: 4 rows x 4 consecutive
+// positions. The CTA's rows of U are staged once; the residuals of the next row group are
+// fetched with cp.async while the current group is updated.
 constexpr int kEsLd = kPanel + 4;        // padded residual row (16-byte aligned)
 constexpr size_t kTrailSmem = (2 * 64 * kEsLd + kPanel * 64) * sizeof(float);
 
