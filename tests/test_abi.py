@@ -154,3 +154,71 @@ def test_project_and_error_rejections(mxq):
              None) == S["MXQ_ERR_WORKSPACE"]
     assert e(FAKE, 1, 64, 256, 256, ODD, FAKE, None, ctypes.byref(p), FAKE, FAKE, need,
              None) == S["MXQ_ERR_ALIGN"]
+
+
+def test_gptq_rejections(mxq):
+    S = {v: k for k, v in mxq.STATUS.items()}
+    L = mxq._lib
+    # 64 x 64 E4M3 tiles
+    tiles = L.mxq_gptq_tiles
+    assert tiles(FAKE, 1, 64, 96, 96, FAKE, FAKE, FAKE, None) == S["MXQ_ERR_SHAPE"]     # k % 64
+    assert tiles(FAKE, 1, 100, 128, 128, FAKE, FAKE, FAKE, None) == S["MXQ_ERR_SHAPE"]  # n % 64
+    assert tiles(FAKE, 5, 64, 128, 128, FAKE, FAKE, FAKE, None) == S["MXQ_ERR_DTYPE"]
+    assert tiles(FAKE, 1, 64, 128, 128, None, FAKE, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert tiles(FAKE, 1, 64, 128, 128, ODD, FAKE, FAKE, None) == S["MXQ_ERR_ALIGN"]
+    assert tiles(FAKE, 1, 64, 128, 128, FAKE, FAKE + 2, FAKE, None) == S["MXQ_ERR_ALIGN"]
+    prep = L.mxq_gptq_prepare
+    assert prep(FAKE, -1, 0.01, FAKE, None) == S["MXQ_ERR_SHAPE"]
+    assert prep(FAKE, 2, float("nan"), FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert prep(FAKE, 2, -0.1, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert prep(None, 2, 0.01, FAKE, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert prep(FAKE, 2, 0.01, ODD, None) == S["MXQ_ERR_ALIGN"]
+    assert prep(None, 0, 0.01, None, None) == 0                                        # empty
+    # Hessian, factor, order, sweep
+    gram = L.mxq_act_gram
+    assert gram(FAKE, 0, 100, 64, 64, FAKE, None) == S["MXQ_ERR_DTYPE"]                 # float32 X
+    assert gram(FAKE, 1, 100, 64, 64, None, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert gram(FAKE, 1, 100, 64, 64, ODD, None) == S["MXQ_ERR_ALIGN"]
+    assert gram(None, 1, 100, 0, 0, None, None) == 0                                   # no columns
+    fac = L.mxq_gptq_factor
+    need = mxq.mxq_gptq_factor_workspace(256)
+    assert need == 256 + 2 * 256 * 256 * 8
+    assert fac(FAKE, 256, 64, None, 0.01, FAKE, FAKE, need, None) == S["MXQ_ERR_UNSUPPORTED"]
+    assert fac(FAKE, 250, 16, None, 0.01, FAKE, FAKE, need, None) == S["MXQ_ERR_SHAPE"]
+    assert fac(FAKE, 256, 16, None, float("inf"), FAKE, FAKE, need, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert fac(FAKE, 256, 16, None, 0.01, FAKE, None, need, None) == S["MXQ_ERR_WORKSPACE"]
+    assert fac(FAKE, 256, 16, None, 0.01, FAKE, FAKE, need - 8, None) == S["MXQ_ERR_WORKSPACE"]
+    assert fac(ODD, 256, 16, None, 0.01, FAKE, FAKE, need, None) == S["MXQ_ERR_ALIGN"]
+    assert fac(FAKE, 256, 16, FAKE + 2, 0.01, FAKE, FAKE, need, None) == S["MXQ_ERR_ALIGN"]
+    assert fac(FAKE, 65552, 16, None, 0.01, FAKE, FAKE, need, None) == S["MXQ_ERR_SHAPE"]
+    assert fac(None, 0, 16, None, 0.01, None, None, 0, None) == 0                       # empty
+    p4 = mxq.params("nvfp4", "hopt", 16)
+    p8 = mxq.params("int8", "hopt", 32)
+    order = L.mxq_gptq_order
+    ows = mxq.mxq_gptq_order_workspace(64, 256, p4)
+    assert order(FAKE, 1, 64, 256, 256, FAKE, ctypes.byref(p8), FAKE, FAKE, ows,
+                 None) == S["MXQ_ERR_UNSUPPORTED"]
+    assert order(FAKE, 1, 64, 256, 256, None, ctypes.byref(p4), FAKE, FAKE, ows,
+                 None) == S["MXQ_ERR_INVALID_ARG"]
+    assert order(FAKE, 1, 64, 256, 256, FAKE, ctypes.byref(p4), None, FAKE, ows,
+                 None) == S["MXQ_ERR_INVALID_ARG"]
+    assert order(FAKE, 1, 64, 16 * 2049, 16 * 2049, FAKE, ctypes.byref(p4), FAKE, FAKE, ows,
+                 None) == S["MXQ_ERR_SHAPE"]                                            # > 2048 blocks
+    assert order(FAKE, 1, 64, 256, 256, FAKE, ctypes.byref(p4), FAKE, FAKE, ows - 8,
+                 None) == S["MXQ_ERR_WORKSPACE"]
+    sweep = L.mxq_gptq
+    sws = mxq.mxq_gptq_workspace(64, 256)
+    assert sws == 64 * 256 * 4 + 2 * 64 * 64 * 4 + 256
+    pe = mxq.params("e4m3", "hopt", 64)
+    assert sweep(FAKE, 1, 64, 256, 256, FAKE, FAKE, None, ctypes.byref(pe), FAKE, FAKE, FAKE,
+                 sws, None) == S["MXQ_ERR_UNSUPPORTED"]
+    assert sweep(FAKE, 1, 64, 256, 256, FAKE, None, None, ctypes.byref(p4), FAKE, FAKE, FAKE,
+                 sws, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert sweep(FAKE, 1, 64, 256, 256, None, FAKE, None, ctypes.byref(p4), FAKE, FAKE, FAKE,
+                 sws, None) == S["MXQ_ERR_INVALID_ARG"]                                 # hopt, no h
+    assert sweep(FAKE, 1, 64, 256, 256, FAKE, FAKE, None, ctypes.byref(p4), FAKE, FAKE, FAKE,
+                 sws - 8, None) == S["MXQ_ERR_WORKSPACE"]
+    assert sweep(FAKE, 1, 65535 * 64 + 64, 256, 256, FAKE, FAKE, None, ctypes.byref(p4), FAKE,
+                 FAKE, FAKE, sws, None) == S["MXQ_ERR_SHAPE"]
+    assert sweep(None, 1, 0, 256, 256, None, None, None, ctypes.byref(p4), None, None, None, 0,
+                 None) == 0                                                              # empty
