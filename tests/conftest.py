@@ -14,6 +14,8 @@ def pytest_configure(config):
 
 
 def pytest_collection_modifyitems(config, items):
+    if not any("gpu" in item.keywords for item in items):
+        return                                    # nothing to skip: no need to import torch
     try:
         import torch
         have_gpu = torch.cuda.is_available()

@@ -86,11 +86,16 @@ def test_planted_mistake_is_caught(name, tmp_path):
     subprocess.run(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-o",
                     str(so), str(mut), "-lm"], check=True)
     env = dict(os.environ, MXQ_ORACLE_LIB=str(so))
+    # every pin file runs; the one the mutant's area belongs to first, so that -x stops early
+    pins = ["test_oracle_pins.py", "test_oracle_pins_scales.py", "test_oracle_pins_gram.py",
+            "test_oracle_pins_gptq.py", "test_oracle_pins_gptq_blocks.py"]
+    first = ("test_oracle_pins_gptq_blocks.py" if name.startswith("gptq_blocks") else
+             "test_oracle_pins_gptq.py" if name.startswith("gptq") else
+             "test_oracle_pins_gram.py" if name.startswith("gram") else
+             "test_oracle_pins_scales.py" if name.startswith(("ue", "int4", "mx")) else
+             "test_oracle_pins.py")
+    pins.remove(first)
     res = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                          os.path.join(HERE, "test_oracle_pins.py"),
-                          os.path.join(HERE, "test_oracle_pins_scales.py"),
-                          os.path.join(HERE, "test_oracle_pins_gram.py"),
-                          os.path.join(HERE, "test_oracle_pins_gptq.py"),
-                          os.path.join(HERE, "test_oracle_pins_gptq_blocks.py")], cwd=ROOT, env=env,
+                          *[os.path.join(HERE, f) for f in [first] + pins]], cwd=ROOT, env=env,
                          capture_output=True, text=True, timeout=600)
     assert res.returncode != 0, f"pins did not catch planted mistake {name}:\n{res.stdout[-2000:]}"
