@@ -38,9 +38,7 @@ namespace {
 // factor
 // ======================================================================================
 constexpr int kNB = 64;                  // tile edge of the blocked factorisation
-constexpr int kTLd = kNB + 1;            // padded shared-memory row (doubles)
 constexpr int kFThreads = 256;
-constexpr size_t kTwoTiles = 2 * kNB * kTLd * sizeof(double);
 constexpr int kPanelTiles = 4;           // tile columns per trailing update of the Cholesky
 
 struct FactorArgs {
@@ -100,15 +98,6 @@ __global__ void k_factor_load(FactorArgs a) {
   }
 }
 
-__device__ __forceinline__ void load_tile(double* s, const double* g, int64_t ld) {
-  for (int e = threadIdx.x; e < kNB * kNB; e += blockDim.x)
-    s[(e / kNB) * kTLd + e % kNB] = g[(int64_t)(e / kNB) * ld + e % kNB];
-}
-__device__ __forceinline__ void store_tile(double* g, const double* s, int64_t ld) {
-  for (int e = threadIdx.x; e < kNB * kNB; e += blockDim.x)
-    g[(int64_t)(e / kNB) * ld + e % kNB] = s[(e / kNB) * kTLd + e % kNB];
-}
-
 // 1 / x for the elimination's pivots, off the division unit: a float32 reciprocal as the seed,
 // then two Newton-Raphson steps r <- r + r (1 - x r) (quadratic convergence: 2^-24 -> 2^-48
 // -> below the float64 rounding); x outside float32's normal range takes the division.
@@ -122,61 +111,75 @@ __device__ __forceinline__ double recip(double x) {
 }
 
 // Diagonal tile p: its Cholesky factor L_pp (lower, the upper part 0) into A and its
-// inverse M_pp into M. The elimination keeps the columns unscaled (step j: T_il -= T_ij T_lj
-// / T_jj over the trailing triangle, one barrier per step), and scales every column by
-// 1/sqrt of its pivot at the end. The inverse: four threads per column of M (consecutive
-// lanes), each summing every fourth term of the forward substitution, then two shuffles.
+// inverse M_pp into M, in one 64-step elimination held in registers: thread (ty, tx) keeps
+// the 16 elements (ty + 16a, tx + 16b) of the tile T and of B (B = I at the start). Step j
+// publishes column j of T and row j of B through shared memory (double-buffered, one
+// barrier per step); with f_i = T_ij / T_jj every thread then updates its elements,
+//     T_il -= f_i T_lj   (l > j: the unscaled elimination, T = L_unit D L_unit^T),
+//     B_ic -= f_i B_jc   (i > j: the same row operations on I, so B -> L_unit^-1).
+// With d = sqrt(diag D): L_il = T_il / d_l, L_ll = d_l, and M = L^-1 = D^-1/2 B, M_ic = B_ic / d_i.
 __global__ void __launch_bounds__(kFThreads) k_potrf_inv(double* A, double* M, int64_t kp, int p) {
-  extern __shared__ double sm[];
-  __shared__ double dg[kNB], rdiag[kNB];
-  double* T = sm;
-  double* X = sm + kNB * kTLd;
-  double* g = A + (int64_t)p * kNB * kp + (int64_t)p * kNB;
-  load_tile(T, g, kp);
-  __syncthreads();
+  __shared__ double colT[2][kNB], rowB[2][kNB], piv[kNB], dg[kNB], rdg[kNB];
   const int t = threadIdx.x, tx = t % 16, ty = t / 16;
-  for (int j = 0; j < kNB; ++j) {
-    const double rr = recip(T[j * kTLd + j]);
+  double* g = A + (int64_t)p * kNB * kp + (int64_t)p * kNB;
+  double* gm = M + (int64_t)p * kNB * kp + (int64_t)p * kNB;
+  double a[4][4], bm[4][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int i = j + 1 + ty + 16 * a;
-      if (i < kNB) {
-        const double tij = T[i * kTLd + j] * rr;
+  for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int l = j + 1 + tx + 16 * b;
-          if (l <= i) T[i * kTLd + l] -= tij * T[l * kTLd + j];
-        }
-      }
+    for (int c = 0; c < 4; ++c) {
+      a[r][c] = g[(int64_t)(ty + 16 * r) * kp + tx + 16 * c];
+      bm[r][c] = ty + 16 * r == tx + 16 * c ? 1.0 : 0.0;
     }
-    __syncthreads();
+#pragma unroll
+  for (int jb = 0; jb < 4; ++jb) {
+#pragma unroll 1
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = 16 * jb + jj, buf = j & 1;
+      if (tx == jj) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) colT[buf][ty + 16 * r] = a[r][jb];
+      }
+      if (ty == jj) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) rowB[buf][tx + 16 * c] = bm[jb][c];
+      }
+      __syncthreads();
+      const double pv = colT[buf][j];
+      if (t == 0) piv[j] = pv;
+      const double rr = recip(pv);
+      double f[4], tl[4], bj[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        f[q] = colT[buf][ty + 16 * q] * rr;
+        tl[q] = colT[buf][tx + 16 * q];
+        bj[q] = rowB[buf][tx + 16 * q];
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int i = ty + 16 * r, l = tx + 16 * c;
+          if (l > j && i >= l) a[r][c] -= f[r] * tl[c];
+          if (i > j) bm[r][c] -= f[r] * bj[c];
+        }
+    }
   }
+  __syncthreads();
   if (t < kNB) {
-    const double d = sqrt(T[t * kTLd + t]);
+    const double d = sqrt(piv[t]);
     dg[t] = d;
-    rdiag[t] = 1.0 / d;
+    rdg[t] = 1.0 / d;
   }
   __syncthreads();
-  for (int e = t; e < kNB * kNB; e += kFThreads) {
-    const int r = e / kNB, c = e % kNB;
-    double& v = T[r * kTLd + c];
-    v = c > r ? 0.0 : (c == r ? dg[r] : v * rdiag[c]);
-  }
-  __syncthreads();
-  if (t < kNB) rdiag[t] = 1.0 / T[t * kTLd + t];
-  __syncthreads();
-  const int c = t >> 2, part = t & 3;
-  for (int i = 0; i < kNB; ++i) {
-    double acc = 0.0;
-    for (int r = c + part; r < i; r += 4) acc += T[i * kTLd + r] * X[r * kTLd + c];
-    acc += __shfl_xor_sync(kFull, acc, 1);
-    acc += __shfl_xor_sync(kFull, acc, 2);
-    if (part == 0) X[i * kTLd + c] = i == c ? rdiag[i] : (i > c ? -acc * rdiag[i] : 0.0);
-    __syncwarp();
-  }
-  __syncthreads();
-  store_tile(g, T, kp);
-  store_tile(M + (int64_t)p * kNB * kp + (int64_t)p * kNB, X, kp);
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = ty + 16 * r, l = tx + 16 * c;
+      g[(int64_t)i * kp + l] = i > l ? a[r][c] * rdg[l] : (i == l ? dg[i] : 0.0);
+      gm[(int64_t)i * kp + l] = i >= l ? bm[r][c] * rdg[i] : 0.0;
+    }
 }
 
 // ---- 64 x 64 x 64 float64 tile products (FP64 tensor cores) -----------------------------
@@ -407,8 +410,6 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
                                double damp, float* U, void* ws, cudaStream_t st) {
   static const bool attrs = [] {
     bool ok = true;
-    ok = cudaFuncSetAttribute(k_potrf_inv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)kTwoTiles) == cudaSuccess;
     for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update,
                           (const void*)k_inv_a, (const void*)k_inv_b})
       ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -440,7 +441,7 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
     const int pe = (int)(p0 + kPanelTiles < nt ? p0 + kPanelTiles : nt);
     for (int p = p0; p < pe; ++p) {
       if (p > p0) k_panel_update<<<(unsigned)(nt - p), kPThreads, kProdSmem1, cs>>>(a.A, kp, p0, p);
-      k_potrf_inv<<<1, kFThreads, kTwoTiles, cs>>>(a.A, a.M, kp, p);
+      k_potrf_inv<<<1, kFThreads, 0, cs>>>(a.A, a.M, kp, p);
       if (nt - 1 - p > 0)
         k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, p);
     }
