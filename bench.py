@@ -711,7 +711,8 @@ def gpu_arm(args):
 
 
 def gptq_launches(k, ordered, panel_tiles=4):
-    """Our kernels per GPTQ step (the Hessian GEMM is cuBLAS's): h pass 2, [order: search,
+    """Our kernels per GPTQ step (the Hessian's GEMMs are cuBLAS's): h pass 2, the Hessian's
+    mirrored triangle 1, [order: search,
     fixup, block losses, sort], factor (lambda, load, per tile column: panel update (not the
     panel's first), diagonal tile, tiles below (not the last); per panel but the last: the
     next panel's columns and, while any remain, everything beyond; 2 per doubling level;
@@ -729,7 +730,7 @@ def gptq_launches(k, ordered, panel_tiles=4):
         f += 2
         s *= 2
     panels = (k + 63) // 64
-    return 2 + (4 if ordered else 0) + f + 1 + panels + (panels - 1) + 2
+    return 2 + 1 + (4 if ordered else 0) + f + 1 + panels + (panels - 1) + 2
 
 
 def bf16_peak():
@@ -873,7 +874,8 @@ def gpu_arm_gptq(args, wl, q):
                 "frac": ach / peak, ("algorithmic_bytes" if unit == "GB/s" else
                                      "algorithmic_ops"): amount, "traffic": None}
     kernels = {"act_sqmean": kern("act_sqmean", "hbm", x_bytes, hbm, "GB/s"),
-               "gram": kern("gram", "tensor", 2.0 * R * k * k, bfp, "TFLOP/s")}
+               # H is symmetric: the work that defines it is one triangle, diagonal included
+               "gram": kern("gram", "tensor", 1.0 * R * k * (k + 1), bfp, "TFLOP/s")}
     if ordered:
         kernels["gptq_order"] = kern("gptq_order", "alu",
                                      ops_per_weight(q.fmt, "hopt", q.window, q.sfmt, B) * weights,

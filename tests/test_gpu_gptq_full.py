@@ -47,10 +47,14 @@ def correlated_x(synth, rows, k, seed, device):
     return X.to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("rows,k", [(3000, 256), (777, 208), (20000, 512)])
+# k = 2048 and 4096 take one and two levels of the triangle's halving (strided-batched
+# rectangles plus diagonal blocks); the smaller ones a single product
+@pytest.mark.parametrize("rows,k", [(3000, 256), (777, 208), (20000, 512), (3000, 2048),
+                                    (600, 4096)])
 def test_gram_matches_oracle(mxq, orc, synth, rows, k):
     X = correlated_x(synth, rows, k, 121, DEV)
     H = mxq.mxq_act_gram(X).cpu().numpy()
+    assert np.array_equal(H, H.T)
     Xo = oracle_view(X)
     ref = orc.gram(Xo).astype(np.float64)
     A = np.abs(orc.to_float(Xo).astype(np.float64))
