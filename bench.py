@@ -189,6 +189,12 @@ def workload_desc(wl, q, x_rows=None):
     ncand = {"e4m3": 126, "ue4m4": 255, "ue5m3": 255, "ue8m0": 255}[q.sfmt]
     grid = ("64-point log grid" if fmt == "e4m3" else
             f"all {ncand} {sg} scales" if window < 0 else f"{sg} scales within +-{window} codes")
+    if full_gptq(q):
+        kind = "ordered" if mode == "gptq-ord" else "sequential"
+        return (f"{wl.name}: W {shapes} {dt}; X {xsh} {dt}; {quant_name(q)} block {block}, "
+                f"{kind} GPTQ over the full input dimension: h = mean of X^2, H = X^T X / R, "
+                f"float64 factor of (H + lambda I)^-1 (damp {GPTQ_DAMP}), sweep with the hopt "
+                f"block search on the {grid}; then weight/h-weighted error sums")
     if mode == "gptq":
         return (f"{wl.name}: W {shapes} {dt}; X {xsh} {dt}; e4m3 64x64 tiles: Gram blocks of X "
                 f"(h = their diagonal), GPTQ factors (damp {GPTQ_DAMP}), tile scales by the "
