@@ -17,7 +17,8 @@ LIB = os.path.join(PKG, "libmxq.so")
 SOURCES = ["mxq_api.cu", "mxq_hpass.cu", "mxq_gram.cu", "mxq_quant.cu", "mxq_quant_grid.cu",
            "mxq_error.cu", "mxq_outerr.cu", "mxq_gptq.cu", "mxq_gptq_full.cu",
            "mxq_noalloc.cu"]
-HEADERS = ["mxq_common.cuh", "mxq_internal.h", "mxq_block.cuh", "mxq_grids.h", "mxq_gridk.cuh"]
+HEADERS = ["mxq_common.cuh", "mxq_internal.h", "mxq_block.cuh", "mxq_grids.h", "mxq_gridk.cuh",
+           "mxq_chol64.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 

@@ -8,7 +8,8 @@
 //                   the mean of diag G_b, 1 when that mean is 0), U the upper Cholesky factor
 //                   of H^-1 (H^-1 = U^T U), all in float64, rounded to float32 once. U is
 //                   reached without forming H^-1: with J the order reversal, J H J = L L^T
-//                   (lower Cholesky) gives H^-1 = (J L^-1 J)^T (J L^-1 J), so U = J L^-1 J.
+//                   (lower Cholesky) gives H^-1 = (J L^-1 J)^T (J L^-1 J), so U = J L^-1 J;
+//                   L and L^-1 come from one register-resident elimination (mxq_chol64.cuh).
 //   k_gptq_tiles    one thread per (row, column block): the row's 64 weights live in
 //                   registers and are swept column by column,
 //                       q = E4M3(RNE(fl32(|w_c| / s))),  wq = +-fl32(s q),
@@ -16,6 +17,7 @@
 //                   every step a separately rounded float32 operation, as in the definition.
 //                   Rows are independent; U (16 KB) is staged once per CTA in shared memory
 //                   and read as warp-wide broadcasts.
+#include "mxq_chol64.cuh"
 #include "mxq_common.cuh"
 #include "mxq_internal.h"
 
@@ -25,19 +27,16 @@ namespace mxq {
 namespace {
 
 constexpr int kT = 64;                 // tile edge
-constexpr int kPrepThreads = 256;
+constexpr int kPrepThreads = kCholThreads;
 constexpr int kSweepThreads = 128;     // rows per CTA pass
-constexpr int kLd = kT + 1;            // padded row of the float64 work matrices
 
 __global__ void __launch_bounds__(kPrepThreads)
 k_gptq_prepare(const float* __restrict__ G, double damp, float* __restrict__ U) {
-  extern __shared__ double sm[];
-  double* A = sm;                 // J H J, then its lower Cholesky factor L
-  double* M = sm + kT * kLd;      // L^-1 (lower)
+  __shared__ Chol64Smem s;
   __shared__ double lam_s;
   const float* Gb = G + (int64_t)blockIdx.x * kT * kT;
   float* Ub = U + (int64_t)blockIdx.x * kT * kT;
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, tx = t % 16, ty = t / 16;
 
   if (t < 32) {                   // lambda = damp * mean(diag G_b)
     double d = (double)Gb[t * (kT + 1)] + (double)Gb[(t + 32) * (kT + 1)];
@@ -48,51 +47,27 @@ k_gptq_prepare(const float* __restrict__ G, double damp, float* __restrict__ U) 
     }
   }
   __syncthreads();
-  // A_ij = H_{63-i, 63-j}, H = (G + G^T) / 2 + lambda I; lower triangle only
-  for (int e = t; e < kT * kT; e += kPrepThreads) {
-    const int i = e / kT, j = e % kT;
-    if (j > i) continue;
-    const int p = kT - 1 - i, q = kT - 1 - j;
-    double v = 0.5 * ((double)Gb[p * kT + q] + (double)Gb[q * kT + p]);
-    if (i == j) v += lam_s;
-    A[i * kLd + j] = v;
-  }
-  __syncthreads();
-  // right-looking Cholesky, column by column
-  for (int j = 0; j < kT; ++j) {
-    const double d = sqrt(A[j * kLd + j]);
-    __syncthreads();                       // every thread has read the pivot
-    if (t == 0) A[j * kLd + j] = d;
-    for (int i = j + 1 + t; i < kT; i += kPrepThreads) A[i * kLd + j] /= d;
-    __syncthreads();
-    const int m = kT - 1 - j;              // trailing block rows j+1 .. 63
-    for (int e = t; e < m * m; e += kPrepThreads) {
-      const int i = j + 1 + e / m, l = j + 1 + e % m;
-      if (l <= i) A[i * kLd + l] -= A[i * kLd + j] * A[l * kLd + j];
+  // A_il = H_{63-i, 63-l}, H = (G + G^T) / 2 + lambda I, this thread's 16 elements
+  double a[4][4], bm[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = ty + 16 * r, l = tx + 16 * c, p = kT - 1 - i, q = kT - 1 - l;
+      double v = 0.5 * ((double)Gb[p * kT + q] + (double)Gb[q * kT + p]);
+      if (i == l) v += lam_s;
+      a[r][c] = v;
     }
-    __syncthreads();
-  }
-  // M = L^-1, one column per thread (forward substitution over the rows, broadcast reads of L)
-  if (t < kT) {
-    const int c = t;
-    for (int i = 0; i < kT; ++i) {
-      double v = 0.0;
-      if (i == c) {
-        v = 1.0 / A[i * kLd + i];
-      } else if (i > c) {
-        double s = 0.0;
-        for (int r = c; r < i; ++r) s += A[i * kLd + r] * M[r * kLd + c];
-        v = -s / A[i * kLd + i];
-      }
-      M[i * kLd + c] = v;
+  // L (A = L L^T) and L^-1 = D^-1/2 B
+  chol64_regs(a, bm, s);
+  // U_pq = (L^-1)_{63-p, 63-q} (upper), rounded to float32 once
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = ty + 16 * r, l = tx + 16 * c;
+      Ub[(kT - 1 - i) * kT + (kT - 1 - l)] = i >= l ? (float)(bm[r][c] * s.rdg[i]) : 0.0f;
     }
-  }
-  __syncthreads();
-  // U_pq = M_{63-p, 63-q} (upper), rounded to float32 once
-  for (int e = t; e < kT * kT; e += kPrepThreads) {
-    const int p = e / kT, q = e % kT;
-    Ub[e] = q >= p ? (float)M[(kT - 1 - p) * kLd + (kT - 1 - q)] : 0.0f;
-  }
 }
 
 template <bool BF16>
@@ -179,16 +154,10 @@ k_gptq_tiles(SweepParams P) {
 
 }  // namespace
 
-constexpr size_t kPrepSmem = 2 * kT * kLd * sizeof(double);
-
 cudaError_t launch_gptq_prepare(const float* G, int64_t nblocks, double damp, float* U,
                                 cudaStream_t st) {
   if (nblocks <= 0) return cudaSuccess;
-  static bool set = cudaFuncSetAttribute(k_gptq_prepare,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kPrepSmem) == cudaSuccess;
-  if (!set) return cudaErrorInvalidConfiguration;
-  k_gptq_prepare<<<(unsigned)nblocks, kPrepThreads, kPrepSmem, st>>>(G, damp, U);
+  k_gptq_prepare<<<(unsigned)nblocks, kPrepThreads, 0, st>>>(G, damp, U);
   return cudaGetLastError();
 }
 

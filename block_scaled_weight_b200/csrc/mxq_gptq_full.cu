@@ -21,6 +21,7 @@
 // Every float32 step follows the definition's operation order: in-block updates
 // w -= fl32(err U), past the block acc = fma(err_j, U_j, acc) over the block's columns in
 // order, then one subtraction.
+#include "mxq_chol64.cuh"
 #include "mxq_common.cuh"
 #include "mxq_gridk.cuh"
 #include "mxq_internal.h"
@@ -98,28 +99,10 @@ __global__ void k_factor_load(FactorArgs a) {
   }
 }
 
-// 1 / x for the elimination's pivots, off the division unit: a float32 reciprocal as the seed,
-// then two Newton-Raphson steps r <- r + r (1 - x r) (quadratic convergence: 2^-24 -> 2^-48
-// -> below the float64 rounding); x outside float32's normal range takes the division.
-__device__ __forceinline__ double recip(double x) {
-  const float xf = (float)x;
-  if (!(fabsf(xf) >= 1.2e-38f && fabsf(xf) <= 3.0e38f)) return 1.0 / x;
-  double r = (double)__frcp_rn(xf);
-  r = fma(r, fma(-x, r, 1.0), r);
-  r = fma(r, fma(-x, r, 1.0), r);
-  return r;
-}
-
 // Diagonal tile p: its Cholesky factor L_pp (lower, the upper part 0) into A and its
-// inverse M_pp into M, in one 64-step elimination held in registers: thread (ty, tx) keeps
-// the 16 elements (ty + 16a, tx + 16b) of the tile T and of B (B = I at the start). Step j
-// publishes column j of T and row j of B through shared memory (double-buffered, one
-// barrier per step); with f_i = T_ij / T_jj every thread then updates its elements,
-//     T_il -= f_i T_lj   (l > j: the unscaled elimination, T = L_unit D L_unit^T),
-//     B_ic -= f_i B_jc   (i > j: the same row operations on I, so B -> L_unit^-1).
-// With d = sqrt(diag D): L_il = T_il / d_l, L_ll = d_l, and M = L^-1 = D^-1/2 B, M_ic = B_ic / d_i.
+// inverse M_pp into M (the register-resident elimination of mxq_chol64.cuh).
 __global__ void __launch_bounds__(kFThreads) k_potrf_inv(double* A, double* M, int64_t kp, int p) {
-  __shared__ double colT[2][kNB], rowB[2][kNB], piv[kNB], dg[kNB], rdg[kNB];
+  __shared__ Chol64Smem s;
   const int t = threadIdx.x, tx = t % 16, ty = t / 16;
   double* g = A + (int64_t)p * kNB * kp + (int64_t)p * kNB;
   double* gm = M + (int64_t)p * kNB * kp + (int64_t)p * kNB;
@@ -127,62 +110,15 @@ __global__ void __launch_bounds__(kFThreads) k_potrf_inv(double* A, double* M, i
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      a[r][c] = g[(int64_t)(ty + 16 * r) * kp + tx + 16 * c];
-      bm[r][c] = ty + 16 * r == tx + 16 * c ? 1.0 : 0.0;
-    }
-#pragma unroll
-  for (int jb = 0; jb < 4; ++jb) {
-#pragma unroll 1
-    for (int jj = 0; jj < 16; ++jj) {
-      const int j = 16 * jb + jj, buf = j & 1;
-      // jb is a compile-time constant here, so the register blocks a step cannot touch
-      // (T: block columns before jb or above the diagonal; B: block rows before jb, block
-      // columns after jb, where row j of B is 0) drop out of the code
-      if (tx == jj) {
-#pragma unroll
-        for (int r = jb; r < 4; ++r) colT[buf][ty + 16 * r] = a[r][jb];
-      }
-      if (ty == jj) {
-#pragma unroll
-        for (int c = 0; c <= jb; ++c) rowB[buf][tx + 16 * c] = bm[jb][c];
-      }
-      __syncthreads();
-      const double pv = colT[buf][j];
-      if (t == 0) piv[j] = pv;
-      const double rr = recip(pv);
-      double f[4], tl[4], bj[4];
-#pragma unroll
-      for (int q = jb; q < 4; ++q) {
-        f[q] = colT[buf][ty + 16 * q] * rr;
-        tl[q] = colT[buf][tx + 16 * q];
-      }
-#pragma unroll
-      for (int q = 0; q <= jb; ++q) bj[q] = rowB[buf][tx + 16 * q];
-#pragma unroll
-      for (int r = jb; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c <= r; ++c) {
-          const int i = ty + 16 * r, l = tx + 16 * c;
-          if (c >= jb && l > j && i >= l) a[r][c] -= f[r] * tl[c];
-          if (c <= jb && i > j) bm[r][c] -= f[r] * bj[c];
-        }
-    }
-  }
-  __syncthreads();
-  if (t < kNB) {
-    const double d = sqrt(piv[t]);
-    dg[t] = d;
-    rdg[t] = 1.0 / d;
-  }
-  __syncthreads();
+    for (int c = 0; c < 4; ++c) a[r][c] = g[(int64_t)(ty + 16 * r) * kp + tx + 16 * c];
+  chol64_regs(a, bm, s);
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int i = ty + 16 * r, l = tx + 16 * c;
-      g[(int64_t)i * kp + l] = i > l ? a[r][c] * rdg[l] : (i == l ? dg[i] : 0.0);
-      gm[(int64_t)i * kp + l] = i >= l ? bm[r][c] * rdg[i] : 0.0;
+      g[(int64_t)i * kp + l] = i > l ? a[r][c] * s.rdg[l] : (i == l ? s.dg[i] : 0.0);
+      gm[(int64_t)i * kp + l] = i >= l ? bm[r][c] * s.rdg[i] : 0.0;
     }
 }
 
