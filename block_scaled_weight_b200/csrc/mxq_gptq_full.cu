@@ -40,6 +40,7 @@ namespace {
 // ======================================================================================
 constexpr int kNB = 64;                  // tile edge of the blocked factorisation
 constexpr int kFThreads = 256;
+static_assert(kFThreads == kCholThreads && kNB == kCholN, "the diagonal tile is one chol64 CTA");
 constexpr int kPanelTiles = 4;           // tile columns per trailing update of the Cholesky
 
 struct FactorArgs {
