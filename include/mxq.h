@@ -361,8 +361,11 @@ MXQ_API mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64
  *
  * mxq_act_gram: H = X^T X / R, the full cols x cols Gram matrix (the GPTQ Hessian up to a
  *  factor) of bf16 X [rows, cols] (ld as for mxq_act_sqmean), float32, row-major, 16-byte
- *  aligned. A plain GEMM (cuBLAS; bf16 products, float32 accumulation in the library's
- *  order): each entry is within rows * 2^-24 * (|X|^T |X|)_ij / rows of the exact value.
+ *  aligned. Plain GEMMs (cuBLAS; bf16 products, float32 accumulation in the library's
+ *  order) over one triangle only -- the matrix halved up to four times, each level's
+ *  off-diagonal blocks and the last level's diagonal blocks as strided-batched products --
+ *  then the upper triangle copied onto the lower one: H is exactly symmetric, and each
+ *  entry is within rows * 2^-24 * (|X|^T |X|)_ij / rows of the exact value.
  *
  * mxq_gptq_factor: U [k][k] float32 (upper, the strict lower triangle written as 0), the
  *  upper Cholesky factor of (H~ + lambda I)^-1, H~ = (H + H^T) / 2 with rows and columns in

@@ -77,3 +77,20 @@ def test_algorithmic_counts(bench):
     assert bench.gptq_launches(9728, True) == 822
     assert bench.code_bytes("nvfp4", 16) == 0.5 + 1 / 16
     assert bench.code_bytes("e4m3", 64) == 1 + 4 / 4096
+
+
+def test_workload_descriptions(bench):
+    """The config line says which GPTQ runs: the full-Hessian one (sequential or ordered) on
+    the 4-bit blocks, the tile one on E4M3."""
+    from block_scaled_weight_b200 import synth
+    full = synth.WORKLOADS["nvfp4_full_calib"]
+    for mode, kind in (("gptq", "sequential"), ("gptq-ord", "ordered")):
+        d = bench.workload_desc(full, bench.quantizer_for(full, args(mode=mode)))
+        assert f"{kind} GPTQ over the full input dimension" in d and "H = X^T X / R" in d
+        assert "64x64 tiles" not in d
+    tiles = synth.WORKLOADS["e4m3_tiles"]
+    d = bench.workload_desc(tiles, bench.quantizer_for(tiles, args(mode="gptq")))
+    assert "e4m3 64x64 tiles" in d and "GPTQ sweep" in d
+    d = bench.workload_desc(full, bench.quantizer_for(full, args()))
+    assert "GPTQ" not in d and "hopt" in d
+
