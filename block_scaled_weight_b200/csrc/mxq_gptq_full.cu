@@ -929,6 +929,11 @@ cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t 
                              cudaStream_t st, const char** why) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const int64_t tiles = (cols + kMirror - 1) / kMirror;
+  if (tiles > 65535) {                  // the mirror's grid; H would hold over 4e12 entries
+    *why = "cols beyond 65535 * 32";
+    return cudaErrorUnknown;
+  }
   cublasHandle_t hd;
   {
     std::lock_guard<std::mutex> lk(g_blas_mu);
@@ -965,8 +970,7 @@ cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t 
     *why = "cublasGemmStridedBatchedEx failed";
     return cudaErrorUnknown;
   }
-  const unsigned tiles = (unsigned)((cols + kMirror - 1) / kMirror);
-  k_mirror_lower<<<dim3(tiles, tiles), 256, 0, st>>>(H, cols);
+  k_mirror_lower<<<dim3((unsigned)tiles, (unsigned)tiles), 256, 0, st>>>(H, cols);
   return cudaGetLastError();
 }
 
