@@ -155,3 +155,60 @@ def test_gram_is_the_mean_outer_product(orc):
     ref = sum(np.outer(x.astype(np.float64), x.astype(np.float64)) for x in X) / 5
     np.testing.assert_allclose(H, ref.astype(np.float32), rtol=1e-7)
     assert np.array_equal(np.diagonal(H), orc.act_sqmean(X))
+
+
+GRIDS = {"nvfp4": [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0],
+         "int4": [0.0, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 7.0]}
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("mode", ["naive", "hopt"])
+@pytest.mark.parametrize("ordered", [False, True])
+def test_residual_relation_and_nearest_codes(orc, fmt, mode, ordered):
+    """GPTQ's residual relation, checked from the outside: after the sweep W - Q = E U in
+    sweep order, with E_c the residual err_c of column c (Frantar et al. 2022, Algorithm 1:
+    every update adds -err_c U_c,: to the later columns, and w_c - q_c = err_c U_cc at column
+    c's turn). So E is recovered from W, Q and U alone by a float64 triangular solve; the value
+    column c had when the sweep reached it is q_c + E_c U_cc, and q_c must be the grid point
+    nearest to it at its block's scale (a saturated top code: anything beyond the last
+    midpoint); and each block's scale must be the plain quantizer's pick on the block's
+    weights as they stood when the sweep reached the block. A dropped or misplaced update, a
+    wrong sign, a transposed U, a missing division by U_cc, a scale searched on the original
+    weights or a block order ignored breaks this for many elements."""
+    from scipy.linalg import solve_triangular
+    rng = np.random.default_rng(16)
+    R, n, k, B = 2000, 48, 256, 16
+    X = correlated(rng, R, k)
+    W = (rng.standard_t(4, (n, k)) * 0.05).astype(np.float32)
+    H = orc.gram(X)
+    h = np.diagonal(H).copy()
+    perm = rng.permutation(k // B).astype(np.int32) if ordered else np.arange(k // B, dtype=np.int32)
+    cols = (perm[:, None] * B + np.arange(B)[None, :]).reshape(-1)   # sweep position -> column
+    U = orc.gptq_prepare(H[np.ix_(cols, cols)][None])[0].astype(np.float64)
+    r = orc.gptq_blocks(W, U.astype(np.float32), h, fmt, mode, B, perm=perm if ordered else None)
+    # everything below in sweep order
+    Q = orc.dequant(r.codes, r.scales, fmt, B, n, k).astype(np.float64)[:, cols]
+    # every nibble the value 1 (E2M1 code 2, INT4 code 1): dequantizes to the block scale
+    ones = np.full_like(r.codes, 0x22 if fmt == "nvfp4" else 0x11)
+    S = orc.dequant(ones, r.scales, fmt, B, n, k).astype(np.float64)[:, cols]
+    Wp, hp, scales = W[:, cols].astype(np.float64), h[cols], r.scales[:, perm]
+    E = solve_triangular(U, (Wp - Q).T, trans="T", lower=False).T
+    seen = Q + E * np.diagonal(U)[None, :]              # column c's value at its turn
+    v, q = np.abs(seen / S), np.abs(Q / S)
+    g = np.asarray(GRIDS[fmt])
+    i = np.searchsorted(g, q)
+    assert np.array_equal(g[i], q)                      # Q is on the grid
+    lo = np.where(i > 0, (g[np.maximum(i - 1, 0)] + g[i]) / 2, 0.0)
+    hi = np.where(i < len(g) - 1, (g[i] + g[np.minimum(i + 1, len(g) - 1)]) / 2, np.inf)
+    same_sign = (np.sign(seen) == np.sign(Q)) | (Q == 0)
+    ok = (v >= lo - 1e-4) & (v <= hi + 1e-4) & same_sign
+    assert ok.all(), (int((~ok).sum()), np.argwhere(~ok)[:3].tolist())
+    start = np.empty_like(seen)
+    for b in range(k // B):
+        c0 = b * B
+        start[:, c0:c0 + B] = Wp[:, c0:c0 + B] - E[:, :c0] @ U[:c0, c0:c0 + B]
+    hq = hp if mode == "hopt" else None
+    plain_start = orc.quantize(start.astype(np.float32), fmt, mode, B, h=hq)
+    assert np.sum(plain_start.scales != scales) <= 2         # float32 vs float64 near-ties
+    plain = orc.quantize(Wp.astype(np.float32), fmt, mode, B, h=hq)   # before the sweep:
+    assert np.sum(plain.scales != scales) >= 20              # the propagation moves many scales
