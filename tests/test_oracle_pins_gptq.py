@@ -4,7 +4,8 @@
 through H^-1 -- GPTQ's update in Cholesky form, err = (w - q) / U_ii, w_j -= err U_ij).
 
 Checks: hand-derived worked examples, the reduction to plain projection when U is diagonal,
-closed forms of the prepared factor, and the output-error improvement GPTQ exists for.
+closed forms of the prepared factor, the output-error improvement GPTQ exists for, and the
+residual relation W - Q = E U with every code nearest to its column's value at its turn.
 """
 import numpy as np
 import pytest
@@ -94,3 +95,48 @@ def test_gptq_lowers_output_error(orc):
     e_plain = np.sum((Xd @ (W - plain).T) ** 2)
     e_gptq = np.sum((Xd @ (W - gptq).T) ** 2)
     assert e_gptq < 0.9 * e_plain
+
+
+def e4m3_magnitudes():
+    """The 127 finite E4M3 magnitudes (OCP FP8: bias 7, 3 mantissa bits, subnormals below
+    2^-6, S.1111.111 the only NaN), ascending."""
+    v = [m / 8 * 2.0 ** -6 for m in range(8)]
+    v += [(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8) if (e, m) != (15, 7)]
+    return np.array(v)
+
+
+def test_residual_relation_and_nearest_codes(orc):
+    """GPTQ's residual relation per tile, checked from the outside: after the sweep of a tile
+    row, W - Q = E U_b with E_c the residual of column c (every update adds -err_c U_c,: to
+    the tile's later columns; w_c - q_c = err_c U_cc at column c's turn). E is recovered from
+    W, Q and U by a float64 triangular solve, so the value column c had at its turn is
+    q_c + E_c U_cc, and its code must be the E4M3 value nearest to that value over the tile's
+    scale (the top value 448 takes everything beyond the last midpoint)."""
+    from scipy.linalg import solve_triangular
+    rng = np.random.default_rng(17)
+    n, k = 128, 192
+    X = rng.standard_normal((1500, k)).astype(np.float32)
+    X[:, 1::2] += 0.8 * X[:, 0::2]
+    U = orc.gptq_prepare(orc.block_gram(X, T)).astype(np.float64)
+    W = (rng.standard_t(4, (n, k)) * 0.05).astype(np.float32)
+    scales = (np.abs(W).reshape(n // T, T, k // T, T).max(axis=(1, 3)) / 400).astype(np.float32)
+    codes = orc.gptq_tiles(W, U.astype(np.float32), scales)
+    g = e4m3_magnitudes()
+    mag = g[codes & 0x7F]
+    sign = np.where(codes & 0x80, -1.0, 1.0)
+    S = np.repeat(np.repeat(scales.astype(np.float64), T, 0), T, 1)
+    Q = sign * (mag * S).astype(np.float32)               # fl32(s q), as dequantized
+    seen = np.empty_like(Q)
+    for tj in range(k // T):
+        c = slice(tj * T, (tj + 1) * T)
+        E = solve_triangular(U[tj], (W[:, c].astype(np.float64) - Q[:, c]).T, trans="T",
+                             lower=False).T
+        seen[:, c] = Q[:, c] + E * np.diagonal(U[tj])[None, :]
+    v = np.abs(seen) / S
+    i = codes & 0x7F
+    lo = np.where(i > 0, (g[np.maximum(i - 1, 0)] + g[i]) / 2, 0.0)
+    hi = np.where(i < len(g) - 1, (g[i] + g[np.minimum(i + 1, len(g) - 1)]) / 2, np.inf)
+    ok = (v >= lo * (1 - 1e-5)) & (v <= hi * (1 + 1e-5)) & ((np.sign(seen) == sign) | (mag == 0))
+    assert ok.all(), (int((~ok).sum()), np.argwhere(~ok)[:3].tolist())
+    plain = orc.gptq_tiles(W, np.stack([np.diag(np.diag(u)) for u in U]).astype(np.float32), scales)
+    assert np.mean(codes != plain) > 0.05                 # the propagation changed many codes
