@@ -934,15 +934,14 @@ cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t 
     *why = "cols beyond 65535 * 32";
     return cudaErrorUnknown;
   }
-  cublasHandle_t hd;
-  {
-    std::lock_guard<std::mutex> lk(g_blas_mu);
-    if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
-      *why = "cublasCreate failed";
-      return cudaErrorUnknown;
-    }
-    hd = g_blas[dev];
+  // the handle is shared by the device's callers: the lock covers binding it to this call's
+  // stream and every launch on it (all asynchronous)
+  std::lock_guard<std::mutex> lk(g_blas_mu);
+  if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
+    *why = "cublasCreate failed";
+    return cudaErrorUnknown;
   }
+  cublasHandle_t hd = g_blas[dev];
   const float alpha = (float)(1.0 / (double)rows), beta = 0.0f;
   const __nv_bfloat16* x = (const __nv_bfloat16*)X;
   // column-major view: X^T is [cols x rows] with leading dimension ld, and the column-major
