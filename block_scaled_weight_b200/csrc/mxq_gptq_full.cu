@@ -323,20 +323,40 @@ struct FactorStreams {
   cudaEvent_t ev_start = nullptr, ev_panel = nullptr, ev_rest = nullptr, ev_end = nullptr,
               ev_done = nullptr;
 };
-FactorStreams& factor_streams() {
+// The current device's two streams and five events, created on first use; *err is set (and
+// nothing kept, so that a later call tries again) when any of them cannot be created.
+FactorStreams& factor_streams(cudaError_t* err) {
   static FactorStreams fs[64];
   static std::mutex init_mu;
   int dev = 0;
   cudaGetDevice(&dev);
   FactorStreams& f = fs[dev < 0 || dev >= 64 ? 0 : dev];
   std::lock_guard<std::mutex> lk(init_mu);
+  *err = cudaSuccess;
   if (!f.side) {
     int least = 0, greatest = 0;
-    cudaDeviceGetStreamPriorityRange(&least, &greatest);
-    cudaStreamCreateWithPriority(&f.chain, cudaStreamNonBlocking, greatest);
-    cudaStreamCreateWithPriority(&f.side, cudaStreamNonBlocking, least);
-    for (cudaEvent_t* e : {&f.ev_start, &f.ev_panel, &f.ev_rest, &f.ev_end, &f.ev_done})
-      cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+    cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    cudaStream_t chain = nullptr, side = nullptr;
+    cudaEvent_t ev[5] = {};
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, least);
+    for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+      e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      for (cudaEvent_t x : ev)
+        if (x) cudaEventDestroy(x);
+      if (side) cudaStreamDestroy(side);
+      if (chain) cudaStreamDestroy(chain);
+      *err = e;
+      return f;
+    }
+    f.chain = chain;
+    f.ev_start = ev[0];
+    f.ev_panel = ev[1];
+    f.ev_rest = ev[2];
+    f.ev_end = ev[3];
+    f.ev_done = ev[4];
+    f.side = side;                          // last: marks the set complete
   }
   return f;
 }
@@ -369,7 +389,9 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   // factors panel P + 1; panel P + 1's column update waits for the previous panel's update
   // of everything beyond (both write those tiles). The two streams fork from and join the
   // caller's stream.
-  FactorStreams& fs = factor_streams();
+  cudaError_t serr = cudaSuccess;
+  FactorStreams& fs = factor_streams(&serr);
+  if (serr != cudaSuccess) return serr;
   std::lock_guard<std::mutex> lk(fs.mu);
   cudaStream_t cs = fs.chain;
   cudaEventRecord(fs.ev_start, st);
@@ -720,7 +742,9 @@ cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cud
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 (int)kTrailSmem) == cudaSuccess;
   if (!attr) return cudaErrorInvalidConfiguration;
-  FactorStreams& fs = factor_streams();
+  cudaError_t serr = cudaSuccess;
+  FactorStreams& fs = factor_streams(&serr);
+  if (serr != cudaSuccess) return serr;
   std::lock_guard<std::mutex> lk(fs.mu);
   cudaStream_t cs = fs.chain;
   cudaEventRecord(fs.ev_start, st);
