@@ -94,3 +94,18 @@ def test_workload_descriptions(bench):
     d = bench.workload_desc(full, bench.quantizer_for(full, args()))
     assert "GPTQ" not in d and "hopt" in d
 
+
+
+@pytest.mark.parametrize("mode,kind", [("gptq", "sequential"), ("gptq-ord", "ordered")])
+def test_reference_arm_gptq_line(mode, kind):
+    """The reference arm times the oracle's full-Hessian GPTQ (h, H, factor, [order], sweep)
+    on the smallest workload and prints the same contract line."""
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_nvfp4", "--mode", mode, "--steps", "1",
+                          "--warmup", "0"], cwd=ROOT, capture_output=True, text=True,
+                         timeout=600, env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "G weights/s"
+    assert f"{kind} GPTQ over the full input dimension" in line["config"]["workload"]
+    assert line["cpu_baseline"]["kind"] == "oracle"
