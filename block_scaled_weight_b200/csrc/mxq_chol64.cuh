@@ -9,7 +9,7 @@
 //     T_il -= f_i T_lj   (l > j, i >= l: the unscaled elimination, T = L_unit D L_unit^T),
 //     B_ic -= f_i B_jc   (i > j: the same row operations applied to I, so B -> L_unit^-1).
 // With d = sqrt(diag D): L_il = T_il / d_l, L_ll = d_l, and L^-1 = D^-1/2 B, (L^-1)_ic = B_ic / d_i.
-// Only the lower triangle of the input is read.
+// Only the lower triangle of the input affects the result (the upper one may hold anything finite).
 #pragma once
 
 #include <cuda_runtime.h>
