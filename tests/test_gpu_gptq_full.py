@@ -11,8 +11,9 @@ Bars:
 - the factor (mxq_gptq_factor): float64 on both sides by different stable routes, rounded
   to float32 once: |dU| <= 2^-23 |U| + 2^-28 max|U| (the float64 difference is a small
   multiple of cond(H) 2^-53 of the largest entry, cond(H) <= 1 + 100 k with the damping);
-- the Gram matrix (mxq_act_gram, a cuBLAS GEMM accumulating bf16 products in float32 in an
-  unspecified order, times fl32(1/R)): |dH| <= (R + 2) 2^-24 (|X|^T |X|)_ij / R;
+- the Gram matrix (mxq_act_gram: cuBLAS GEMMs over one triangle, accumulating bf16 products
+  in float32 in an unspecified order, times fl32(1/R), then mirrored):
+  |dH| <= (R + 2) 2^-24 (|X|^T |X|)_ij / R, and H exactly symmetric;
 - end to end (Gram, order, factor and sweep on the GPU against the oracle's pipeline on the
   same X and W): the Gram matrices differ within that bound, which moves U, so codes are
   compared by what is unique: the output error within 1% and below the plain quantizer's.
@@ -72,6 +73,21 @@ def check_factor(U, ref):
 
 def block_cols(perm, B):
     return (np.asarray(perm)[:, None] * B + np.arange(B)[None, :]).reshape(-1)
+
+
+def test_gram_strided_columns(mxq, orc, synth):
+    """X a column slice of a wider matrix (ld 2304, 2048 columns: one level of halving): the
+    products' operand offsets are columns of the slice."""
+    rows = 1500
+    big = correlated_x(synth, rows, 2304, 123, DEV)
+    X = big[:, 128:2176]
+    H = mxq.mxq_act_gram(X).cpu().numpy()
+    assert np.array_equal(H, H.T)
+    Xo = oracle_view(X)
+    ref = orc.gram(Xo).astype(np.float64)
+    A = np.abs(orc.to_float(Xo).astype(np.float64))
+    tol = (rows + 2) * 2.0 ** -24 * (A.T @ A) / rows + 1e-38
+    assert np.all(np.abs(H - ref) <= tol), float((np.abs(H - ref) / tol).max())
 
 
 @pytest.mark.parametrize("k,B,ordered", [(64, 16, False), (256, 16, True), (1024, 32, True),
