@@ -43,13 +43,14 @@ L2_BYTES = 126 * 1024 * 1024
 # Plain-ALU peak of the search kernel: 148 SMs x 4 sub-partitions x 32 FP32 lanes x
 # 1965 MHz (max SM clock) = lane-operations per second, an FMA counted as one operation.
 ALU_PEAK_TOPS = 148 * 128 * 1.965e9 / 1e12
-# Oracle samples: the cpu_baseline leg (about 10-30 s of CPU work) and each step of the
-# reference arm (well under a second, so that a long --steps run stays short).
-CPU_X_ROWS, CPU_W_ROWS = 65536, 4096
+# Oracle samples, in weight rows of the first weight (with the matching share of activation
+# rows): the cpu_baseline leg (about 10-30 s of CPU work) and each step of the reference arm
+# (a fraction of a second, so that a long --steps run stays short).
+CPU_W_ROWS = 1024
 GPTQ_CPU_X_ROWS, GPTQ_CPU_W_ROWS = 4096, 16
 Quantizer = collections.namedtuple("Quantizer", "fmt block mode window sfmt")
 HEADLINE_Q = Quantizer("nvfp4", 16, "hopt", -1, "e4m3")
-REF_X_ROWS, REF_W_ROWS = 2048, 8
+REF_X_ROWS, REF_W_ROWS = 2048, 64
 
 
 def parse():
@@ -271,9 +272,25 @@ def bits_of(t):
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+def proportional_rows(wl, w_rows):
+    """Rows of the first activation matrix and of the first weight that make the same
+    fraction of the workload: w_rows of the weights' rows (in units of the first weight's
+    width) and the matching share of the activation rows (in units of the first activation
+    matrix's width), so that a sample's time is that fraction of a full step's."""
+    (_, n, k), (R, kx) = wl.weights[0], wl.x_shapes[0]
+    n_equiv = sum(nn * kk for _, nn, kk in wl.weights) / k
+    r_equiv = sum(r * kk for r, kk in wl.x_shapes) / kx
+    w_rows = min(w_rows, n)
+    x_rows = max(1, min(R, round(w_rows * r_equiv / n_equiv)))
+    return x_rows, w_rows, w_rows / n_equiv
+
+
 def reference_arm(args):
-    """The CPU oracle, as it stands, timed on the host cores: each step is a bounded sample
-    of the workload (the first X and W matrices), its time scaled to the full workload."""
+    """The CPU oracle, as it stands, timed on the host cores. Each step is the whole path on
+    a proportional sample of the workload -- REF_W_ROWS weight rows and the matching share of
+    the activation rows (h pass, search, error sums) -- so ms_per_step is the step's own
+    measured time and the throughput is the sample's weights over it. GPTQ modes (whose
+    factor does not shrink with the rows) time a smaller sample and scale it."""
     rank, world, _ = dist_env()
     if world > 1 and rank != 0:
         return
@@ -282,28 +299,45 @@ def reference_arm(args):
     wl = synth.WORKLOADS[args.workload]
     q = quantizer_for(wl, args)
     (_, n, k), (R, _) = wl.weights[0], wl.x_shapes[0]
-    x_rows = min(REF_X_ROWS, R)
-    w_rows = min(max(REF_W_ROWS, q.block if q.fmt == "e4m3" else 1), n)
-    X = bits_of(synth.workload_activations(wl, 0, rows=x_rows))
-    W = bits_of(synth.workload_weight(wl, 0, rows=w_rows))
-    h = orc.act_sqmean(X)
     nt = os.cpu_count() or 1
     weights = sum(nn * kk for _, nn, kk in wl.weights)
-    R_full = sum(r * kk for r, kk in wl.x_shapes) / k
-    times = []
-    for i in range(args.warmup + args.steps):
-        full, _ = oracle_step_sample(X, W, h, nt, R_full, weights / k, q)
-        if i >= args.warmup:
-            times.append(full)
-    full_step = statistics.mean(times)
-    value = weights / full_step / 1e9
-    sample = (f"oracle on {x_rows} of {R} X rows (h) and {w_rows} of {n} W rows ({q.mode} "
-              f"search + error) per step, {nt} threads; times scaled to the full workload")
     headline = args.workload == "nvfp4_full_calib" and q == HEADLINE_Q
     metric = METRIC if headline else metric_for(q)
+    times = []
+    if full_gptq(q):
+        x_rows, w_rows = min(REF_X_ROWS, R), min(GPTQ_CPU_W_ROWS, n)
+        X = bits_of(synth.workload_activations(wl, 0, rows=x_rows))
+        W = bits_of(synth.workload_weight(wl, 0, rows=w_rows))
+        h = orc.act_sqmean(X)
+        R_full = sum(r * kk for r, kk in wl.x_shapes) / k
+        for i in range(args.warmup + args.steps):
+            full, _ = oracle_step_sample(X, W, h, nt, R_full, weights / k, q)
+            if i >= args.warmup:
+                times.append(full)
+        step_s = statistics.mean(times)
+        value = weights / step_s / 1e9
+        sample = (f"oracle on {x_rows} of {R} X rows and {w_rows} of {n} W rows per step, "
+                  f"{nt} threads; times scaled to the full workload")
+    else:
+        w_rows = REF_W_ROWS
+        if q.fmt == "e4m3":
+            w_rows = max(w_rows - w_rows % q.block, q.block)
+        x_rows, w_rows, frac = proportional_rows(wl, w_rows)
+        X = bits_of(synth.workload_activations(wl, 0, rows=x_rows))
+        W = bits_of(synth.workload_weight(wl, 0, rows=w_rows))
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            oracle_path(X, W, nt, q)
+            if i >= args.warmup:
+                times.append(time.perf_counter() - t0)
+        step_s = statistics.mean(times)
+        value = frac * weights / step_s / 1e9
+        sample = (f"oracle, whole path per step on {x_rows} of {R} X rows and {w_rows} of "
+                  f"{n} W rows (the same {frac:.2%} share of the activations and of the "
+                  f"weights), {nt} threads; per-step time measured, not scaled")
     line = {"impl": "reference", "metric": metric, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": workload_desc(wl, q)},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": nt, "kind": "oracle",
@@ -311,6 +345,34 @@ def reference_arm(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def oracle_path(X_bits, W_bits, n_threads, q):
+    """One pass of the whole path through the oracle on host inputs: h pass (or Gram blocks),
+    search (or tile GPTQ), dequantisation and the error sums."""
+    import numpy as np
+    from oracle import oracle as orc
+    fmt, block, mode, window = q.fmt, q.block, q.mode, q.window
+    w_rows, K = W_bits.shape
+    if mode in ("bhopt", "gptq"):
+        G = orc.block_gram(X_bits, block)
+        h = np.diagonal(G, axis1=1, axis2=2).reshape(-1).copy()
+    else:
+        h = orc.act_sqmean(X_bits, n_threads=n_threads)
+    if mode == "bhopt":
+        r = orc.quantize_gram(W_bits, fmt, block, G, window=window, n_threads=n_threads,
+                              sfmt=q.sfmt)
+        codes = r.codes
+    elif mode == "gptq":
+        r = orc.quantize(W_bits, fmt, "hopt", block, h=h, window=window, n_threads=n_threads,
+                         sfmt=q.sfmt)
+        codes = orc.gptq_tiles(W_bits, orc.gptq_prepare(G), r.scales)
+    else:
+        r = orc.quantize(W_bits, fmt, mode, block, h=h if mode == "hopt" else None,
+                         window=window, n_threads=n_threads, sfmt=q.sfmt)
+        codes = r.codes
+    What = orc.dequant(codes, r.scales, fmt, block, w_rows, K, sfmt=q.sfmt)
+    return orc.error_sums(W_bits, What, h)
 
 
 # ---------------------------------------------------------------------------------------
@@ -693,27 +755,60 @@ def gpu_arm(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         X0, W0 = Xs[0], Ws[0]
         R0, n0 = X0.shape[0], W0.shape[0]
-        x_rows = min(CPU_X_ROWS, R0)
-        w_rows = min(CPU_W_ROWS // (8 if fmt == "e4m3" or mode == "bhopt" else 1), n0)
+        # the whole path on a proportional sample: the same share of X's rows and W's rows
+        w_rows = CPU_W_ROWS // (8 if fmt == "e4m3" or mode == "bhopt" else 1)
         if fmt == "e4m3":
             w_rows = max(w_rows - w_rows % block, block)
+        x_rows, w_rows, frac = proportional_rows(wl, w_rows)
+        x_rows = min(x_rows, R0)
         Xb = bits_of(X0[:x_rows].cpu())
         Wb = bits_of(W0[:w_rows].cpu())
         from oracle import oracle as orc
         nt = os.cpu_count() or 1
-        h_np = orc.act_sqmean(Xb, n_threads=nt)
-        # the sample's per-row times scaled to every X row and every W row of the step
-        full, d = oracle_step_sample(Xb, Wb, h_np, nt, sum(X.numel() for X in Xs) / X0.shape[1],
-                                     weights / W0.shape[1], q)
+        t0 = time.perf_counter()
+        oracle_path(Xb, Wb, nt, q)
+        t_cpu = time.perf_counter() - t0
         line["cpu_baseline"] = {
-            "value": weights / full / 1e9, "unit": UNIT, "cores": nt, "kind": "oracle",
-            "sample": (f"oracle on {x_rows} of {R0} X rows (h) and {w_rows} of {n0} W rows "
-                       f"({mode} search + error), {nt} threads; times scaled to the full "
-                       f"workload ({d['h_s']:.1f} s + {d['quant_s']:.1f} s measured)")}
+            "value": frac * weights / t_cpu / 1e9, "unit": UNIT, "cores": nt, "kind": "oracle",
+            "sample": (f"oracle, whole path on {x_rows} of {R0} X rows and {w_rows} of {n0} W "
+                       f"rows (the same {frac:.2%} share of the activations and the weights), "
+                       f"{nt} threads, {t_cpu:.1f} s measured")}
+        line["result"]["parity_sample"] = sampled_parity(orc, synth, wl, q, p, Ws[0], outs[0],
+                                                         hs[outs[0][4]], nt)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def sampled_parity(orc, synth, wl, q, p, W, out, h, nt, n_rows=32):
+    """The timed step's own outputs for sampled rows of the first weight against the oracle
+    run on the same bytes (the same weight rows, the GPU's h): blocks compared, blocks whose
+    scale or codes differ, and near ties -- blocks whose two best candidate errors differ by
+    less than 1e-6 relative, which the acceptance rule counts and excludes. 1-D block
+    quantizers with a diagonal objective only (null otherwise)."""
+    import numpy as np
+    if q.fmt == "e4m3" or q.mode not in ("naive", "sse", "hopt"):
+        return None
+    codes, scales = out[0], out[1]
+    n = W.shape[0]
+    rows = synth.sample_rows(n, min(n_rows, n), wl.seed + 11)
+    ri = rows.to(W.device)
+    r = orc.quantize(bits_of(W.index_select(0, ri).cpu()), q.fmt, q.mode, q.block,
+                     h=h.cpu().numpy() if q.mode == "hopt" else None, window=q.window,
+                     sfmt=q.sfmt, n_threads=nt)
+    g_s = scales.index_select(0, ri).cpu().numpy()
+    g_c = codes.index_select(0, ri).cpu().numpy().view(np.uint8)
+    bpr = g_s.shape[1]
+    cpb = g_c.shape[1] // bpr                        # code bytes per block
+    code_bad = (g_c.reshape(len(rows), bpr, cpb) !=
+                r.codes.view(np.uint8).reshape(len(rows), bpr, cpb)).any(axis=2)
+    bad = (g_s != r.scales) | code_bad
+    near = orc.near_tie(r.best, r.second) if q.mode != "naive" else np.zeros_like(bad)
+    return {"rows": int(len(rows)), "blocks": int(bad.size),
+            "differing_blocks": int(bad.sum()), "near_tie_blocks": int(near.sum()),
+            "differing_outside_near_ties": int((bad & ~near).sum()),
+            "h": "the GPU's h of the timed step (the oracle gets the same bytes)"}
 
 
 def gptq_launches(k, ordered, panel_tiles=4):

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 namespace mxq {
@@ -18,6 +19,23 @@ int sm_count() {
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
+}
+
+cudaError_t ensure_dynamic_smem(const void* func, int bytes) {
+  // The attribute belongs to the (device, kernel) pair: remember each pair raised so far.
+  struct Done { int dev; const void* func; int bytes; };
+  static std::mutex mu;
+  static std::vector<Done> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Done& d : done)
+    if (d.dev == dev && d.func == func && d.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  done.push_back(Done{dev, func, bytes});
+  return cudaSuccess;
 }
 
 }  // namespace mxq

@@ -369,15 +369,11 @@ size_t gptq_factor_workspace(int64_t k) {
 
 cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* perm,
                                double damp, float* U, void* ws, cudaStream_t st) {
-  static const bool attrs = [] {
-    bool ok = true;
-    for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update,
-                          (const void*)k_inv_a, (const void*)k_inv_b})
-      ok = ok && cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kProdSmem1) == cudaSuccess;
-    return ok;
-  }();
-  if (!attrs) return cudaErrorInvalidConfiguration;
+  for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update,
+                        (const void*)k_inv_a, (const void*)k_inv_b}) {
+    const cudaError_t ae = ensure_dynamic_smem(f, (int)kProdSmem1);
+    if (ae != cudaSuccess) return ae;
+  }
   const int64_t kp = (k + kNB - 1) / kNB * kNB, nt = kp / kNB;
   char* w = (char*)ws;
   FactorArgs a{H, k, kp, B, perm, (double*)(w + 256), (double*)(w + 256) + kp * kp,
@@ -738,10 +734,8 @@ void launch_trailing(const SweepArgs& a, const float* Err, int64_t p0, int S, in
 // panel t's update beyond (both write those positions).
 template <int B, int ELEM>
 cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cudaStream_t st) {
-  static const bool attr = cudaFuncSetAttribute(k_gptq_trailing<B>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                (int)kTrailSmem) == cudaSuccess;
-  if (!attr) return cudaErrorInvalidConfiguration;
+  const cudaError_t ae = ensure_dynamic_smem((const void*)k_gptq_trailing<B>, (int)kTrailSmem);
+  if (ae != cudaSuccess) return ae;
   cudaError_t serr = cudaSuccess;
   FactorStreams& fs = factor_streams(&serr);
   if (serr != cudaSuccess) return serr;

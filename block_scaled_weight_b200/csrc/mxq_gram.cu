@@ -393,19 +393,16 @@ cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, i
   GramParams P{rows, cols, per_chunk, partial, err};
   const dim3 grid((unsigned)((cols + kGramCols - 1) / kGramCols), (unsigned)chunks);
   if (B == 16) {
-    static bool set16 = cudaFuncSetAttribute(k_gram_tc<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kGramSmem) == cudaSuccess;
-    if (!set16) return cudaErrorInvalidConfiguration;
+    e = ensure_dynamic_smem((const void*)k_gram_tc<16>, (int)kGramSmem);
+    if (e != cudaSuccess) return e;
     k_gram_tc<16><<<grid, kGramThreads, kGramSmem, st>>>(map, P);
   } else if (B == 64) {
-    static bool set64 = cudaFuncSetAttribute(k_gram_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kGramSmem) == cudaSuccess;
-    if (!set64) return cudaErrorInvalidConfiguration;
+    e = ensure_dynamic_smem((const void*)k_gram_tc<64>, (int)kGramSmem);
+    if (e != cudaSuccess) return e;
     k_gram_tc<64><<<grid, kGramThreads, kGramSmem, st>>>(map, P);
   } else {
-    static bool set32 = cudaFuncSetAttribute(k_gram_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kGramSmem) == cudaSuccess;
-    if (!set32) return cudaErrorInvalidConfiguration;
+    e = ensure_dynamic_smem((const void*)k_gram_tc<32>, (int)kGramSmem);
+    if (e != cudaSuccess) return e;
     k_gram_tc<32><<<grid, kGramThreads, kGramSmem, st>>>(map, P);
   }
   e = cudaGetLastError();

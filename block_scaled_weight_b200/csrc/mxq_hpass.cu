@@ -18,8 +18,8 @@ namespace {
 
 constexpr int kWarps = kHpassThreads / 32;
 constexpr int kRowsPerStep = 8;
-constexpr int kCtasPerSm = 3;          // resident 256-thread CTAs per SM (launch bounds)
-constexpr int kTargetCtas = 148 * kCtasPerSm;   // one wave on a 148-SM B200
+constexpr int kCtasPerSm = kHpassCtasPerSm;    // resident CTAs per SM (launch bounds)
+constexpr int kTargetCtas = kHpassTargetCtas;   // one wave on a 148-SM B200
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;

@@ -12,6 +12,11 @@ namespace mxq {
 // partial[chunk][cols]. The chunk count depends only on (rows, cols), so the reduction
 // order (and the result) is the same on every run and every device.
 constexpr int kHpassThreads = 256;
+// Resident 256-thread CTAs per SM and the one-wave target grid on a 148-SM B200; strips x
+// chunks never exceeds kHpassTargetCtas, so the workspace is at most
+// max(kHpassTargetCtas x 256, cols) doubles.
+constexpr int kHpassCtasPerSm = 3;
+constexpr int kHpassTargetCtas = 148 * kHpassCtasPerSm;
 int hpass_chunks(int64_t rows, int64_t cols, int dtype);
 cudaError_t launch_hpass_partial(const void* X, int dtype, int64_t rows, int64_t cols,
                                  int64_t ld, int chunks, double* partial, cudaStream_t st);
@@ -105,6 +110,9 @@ cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t 
                              cudaStream_t st, const char** why);
 
 int sm_count();
+// Raises func's dynamic shared-memory limit to `bytes` on the current device, once per
+// (device, kernel): the attribute is per device, so each GPU a process uses needs its own.
+cudaError_t ensure_dynamic_smem(const void* func, int bytes);
 // Sets the per-thread text that mxq_last_error() returns.
 void set_error_text(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
 

@@ -19,7 +19,9 @@
 //
 // Set-up: the first call on each device, with that device current, looks the array's
 // device address up (cudaGetSymbolAddress) and caches it; make that first call before any
-// stream capture begins.
+// stream capture begins. The cache lives as long as the process and does not survive a
+// cudaDeviceReset (which unloads the module and may move the array): a caller that resets
+// a device must not call this entry point on it afterwards.
 #include "../../include/mxq.h"
 #include "mxq_internal.h"
 
@@ -30,6 +32,13 @@
 namespace {
 
 constexpr size_t kScratchBytes = size_t(1) << 20;
+// The h pass needs at most max(kHpassTargetCtas x 256, cols) doubles of scratch (strips x
+// row chunks never exceeds one wave of kHpassTargetCtas CTAs; a strip is at most 256
+// columns wide): within 1 MiB for every width up to 131072 columns, whatever the rows.
+static_assert(size_t(mxq::kHpassTargetCtas) * 256 * sizeof(double) <= kScratchBytes,
+              "a one-wave h pass grid must fit the static scratch");
+static_assert(size_t(131072) * sizeof(double) <= kScratchBytes,
+              "the documented width limit must fit the static scratch");
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;

@@ -424,9 +424,8 @@ cudaError_t launch_outerr(const void* X, int64_t m, int64_t k, int64_t ldx, cons
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((m + kOeM - 1) / kOeM), (unsigned)((n + kOeN - 1) / kOeN));
   OeParams P{m, n, k, codes, scales, block, fmt == 3 ? 1 : 0, partial, err};
-  static bool attr = cudaFuncSetAttribute(k_outerr_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          kOeSmem) == cudaSuccess;
-  if (!attr) return cudaErrorInvalidConfiguration;
+  e = ensure_dynamic_smem((const void*)k_outerr_tc, (int)kOeSmem);
+  if (e != cudaSuccess) return e;
   k_outerr_tc<<<grid, kOeThreads, kOeSmem, st>>>(xmap, wmap, P, T);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -155,7 +155,9 @@ MXQ_API mxq_status mxq_act_sqmean(const void* X, int32_t dtype, int64_t rows, in
  * rejected with MXQ_ERR_SHAPE, launching nothing). No cudaMalloc, cudaFree or other
  * allocation happens. All calls share the array: calls that overlap on the GPU race, so
  * order them (e.g. one stream). The first call on each device, with that device current,
- * looks up the array's device address; make it before any stream capture begins.
+ * looks up the array's device address and caches it for the life of the process; make it
+ * before any stream capture begins. The cached address does not survive a cudaDeviceReset:
+ * after resetting a device, do not call this entry point on it again.
  * Arguments and result as for mxq_act_sqmean. */
 MXQ_API mxq_status mxq_act_sqmean_noalloc(const void* X, int32_t dtype, int64_t rows,
                                           int64_t cols, int64_t ld, float* h, void* stream);

@@ -388,7 +388,12 @@ def block_losses(W, h, fmt: str, mode: str, block: int, *, sfmt: str = "e4m3",
                  window: int = -1, n_threads=1) -> np.ndarray:
     """Hessian-weighted quantization loss of each column block: sum over rows and the
     block's columns of h_j (w_ij - w^_ij)^2 (float64; each row's block summed, then the rows
-    in ascending order) for the block quantizer's own (uncompensated) result."""
+    in ascending order) for the block quantizer's own (uncompensated) result.
+
+    The qwantize "GPTQ Quantization" section orders blocks by this loss but fixes no
+    summation order; rows outer, a block's columns inner, is the reading taken here. A
+    device that sums in another order can swap two blocks whose losses agree to ~1e-15, so
+    block orders are compared under a 1e-12 relative tie rule."""
     W, _ = _as_input(W)
     n, k = W.shape
     r = quantize(W, fmt, mode, block, h=h if mode == "hopt" else None, window=window,

@@ -26,3 +26,21 @@ def near_tie_mask(best, second, rel=1e-6):
 def sample_oracle_rows(W_np, rows):
     """Rows of W (oracle form) gathered into a dense matrix."""
     return np.ascontiguousarray(W_np[np.asarray(rows)])
+
+
+def order_with_ties(perm, perm_ref, losses, rel=1e-12):
+    """Check a block order against the oracle's under the tie rule: perm must be a
+    permutation, and at every position its block's oracle loss must equal that of the
+    oracle's block there to within `rel` relative (the two sides sum each block's float64
+    loss in different orders, so blocks whose losses agree to ~1e-15 may swap; the lower
+    block first on exactly equal losses is the oracle's own rule). Returns the number of
+    adjacent pairs in the oracle order whose losses are that close (the near ties)."""
+    perm = np.asarray(perm)
+    perm_ref = np.asarray(perm_ref)
+    L = np.asarray(losses, np.float64)
+    assert np.array_equal(np.sort(perm), np.arange(len(L))), "not a permutation"
+    a, b = L[perm], L[perm_ref]
+    bad = np.abs(a - b) > rel * np.maximum(np.abs(a), np.abs(b))
+    assert not bad.any(), f"{int(bad.sum())} positions differ beyond the tie rule"
+    s = L[perm_ref]
+    return int((np.abs(s[1:] - s[:-1]) <= rel * np.abs(s[:-1])).sum())

@@ -5,9 +5,12 @@ allocator or a fixed arena, or they must not allocate after start-up because an 
 can synchronise the device. For them the library offers an h pass that takes no workspace
 and uses a 1 MiB static device array inside the library instead. This test calls it through
 the C-ABI, twice in a row (the second call reuses the array the first one wrote), and
-checks each result against the workspace version, mxq_act_sqmean, within the h tolerance
-used everywhere else (1e-5 relative); it also checks that a width beyond the array's limit
-is rejected before any launch. It must pass alone in a fresh process and after the rest of
+checks each result against the workspace version, mxq_act_sqmean. Both run the same two
+kernels with the same row chunks in the same fixed order, so the results must be equal bit
+for bit (a wrong offset or leading dimension in the scratch path would show up even where
+it moves h only slightly); the shapes include the widest scratch use (a one-wave grid of
+256-column strips) and the widest accepted input. It also checks that a width beyond the
+array's limit is rejected before any launch. It must pass alone in a fresh process and after the rest of
 the suite, so it lives in a file that is collected last.
 """
 import ctypes
@@ -39,7 +42,11 @@ def call_noalloc(mxq, X, h):
 
 @pytest.mark.parametrize("rows,cols,dtype", [(244449 // 8, 9728, torch.bfloat16),
                                              (1000, 264, torch.bfloat16),
-                                             (512, 256, torch.float32)])
+                                             (512, 256, torch.float32),
+                                             # 4 strips x 111 chunks: ~0.9 MB of scratch
+                                             (65536, 1024, torch.bfloat16),
+                                             # the widest accepted input, many rows
+                                             (2048, 131072, torch.bfloat16)])
 def test_noalloc_matches_workspace_version_twice(mxq, rows, cols, dtype):
     from block_scaled_weight_b200 import synth
     for call in range(2):
@@ -48,7 +55,8 @@ def test_noalloc_matches_workspace_version_twice(mxq, rows, cols, dtype):
         h = torch.full((cols,), float("nan"), dtype=torch.float32, device=DEV)
         assert call_noalloc(mxq, X, h) == 0, mxq._lib.mxq_last_error()
         torch.cuda.synchronize()
-        np.testing.assert_allclose(h.cpu().numpy(), ref.cpu().numpy(), rtol=1e-5, atol=0)
+        assert np.array_equal(h.cpu().numpy(), ref.cpu().numpy())
+        del X
 
 
 def test_noalloc_rejects_widths_beyond_the_static_scratch(mxq):
