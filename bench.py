@@ -812,8 +812,8 @@ def sampled_parity(orc, synth, wl, q, p, W, out, h, nt, n_rows=32):
 
 
 def gptq_launches(k, ordered, panel_tiles=4):
-    """Our kernels per GPTQ step (the Hessian's GEMMs are cuBLAS's): h pass 2, the Hessian's
-    mirrored triangle 1, [order: search,
+    """Our kernels per GPTQ step: h pass 2, the Hessian 3 (the tensor-core product, the sums
+    of the last wave's row chunks, the transpose onto the lower triangle), [order: search,
     fixup, block losses, sort], factor (lambda, load, per tile column: panel update (not the
     panel's first), diagonal tile, tiles below (not the last); per panel but the last: the
     next panel's columns and, while any remain, everything beyond; 2 per doubling level;
@@ -831,7 +831,7 @@ def gptq_launches(k, ordered, panel_tiles=4):
         f += 2
         s *= 2
     panels = (k + 63) // 64
-    return 2 + 1 + (4 if ordered else 0) + f + 1 + panels + (panels - 1) + 2
+    return 2 + 3 + (4 if ordered else 0) + f + 1 + panels + (panels - 1) + 2
 
 
 def bf16_peak():
@@ -871,6 +871,7 @@ def gpu_arm_gptq(args, wl, q):
     u8 = dict(dtype=torch.uint8, device=dev)
     h = torch.empty(k, **f32)
     H = torch.empty(k, k, **f32)
+    gws = torch.empty(max(mxq.mxq_act_gram_workspace(R, k), 8), **u8)
     U = torch.empty(k, k, **f32)
     perm = torch.arange(k // B, dtype=torch.int32, device=dev)
     hws = torch.empty(mxq.mxq_act_sqmean_workspace(R, k), **u8)
@@ -883,7 +884,7 @@ def gpu_arm_gptq(args, wl, q):
     ews = torch.empty(mxq.mxq_error_workspace(n, k), **u8)
     pv = perm if ordered else None
     phases = [("act_sqmean", lambda: mxq.mxq_act_sqmean(X, h, workspace=hws)),
-              ("gram", lambda: mxq.mxq_act_gram(X, H))]
+              ("gram", lambda: mxq.mxq_act_gram(X, H, workspace=gws))]
     if ordered:
         phases.append(("gptq_order", lambda: mxq.mxq_gptq_order(W, h, p, perm=perm,
                                                                 workspace=ows)))

@@ -1,8 +1,8 @@
 """Build ``libmxq.so`` in-tree with nvcc for sm_100a (B200).
 
 The library is a plain C-ABI shared object (see ``include/mxq.h``); the CUDA runtime is
-linked statically so the object carries no dependency on any particular libcudart. cuBLAS
-(the one plain GEMM, GPTQ's Gram matrix) is linked dynamically from the CUDA toolkit.
+linked statically so the object carries no dependency on any particular libcudart. Every
+kernel is the library's own; no CUDA math library is linked.
 """
 from __future__ import annotations
 
@@ -16,10 +16,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmxq.so")
 SOURCES = ["mxq_api.cu", "mxq_hpass.cu", "mxq_gram.cu", "mxq_quant.cu", "mxq_quant_grid.cu",
-           "mxq_error.cu", "mxq_outerr.cu", "mxq_gptq.cu", "mxq_gptq_full.cu",
+           "mxq_error.cu", "mxq_outerr.cu", "mxq_gptq.cu", "mxq_gptq_full.cu", "mxq_gram_full.cu",
            "mxq_noalloc.cu"]
 HEADERS = ["mxq_common.cuh", "mxq_internal.h", "mxq_block.cuh", "mxq_grids.h", "mxq_gridk.cuh",
-           "mxq_chol64.cuh"]
+           "mxq_chol64.cuh", "mxq_tc.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 
@@ -64,9 +64,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         for f in [pool.submit(compile_one, s, o) for s, o in zip(SOURCES, objs)]:
             f.result()
     tmp = LIB + ".tmp"
-    cuda_lib = os.path.join(os.path.dirname(os.path.dirname(nvcc())), "lib64")
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
-           "-cudart", "static", "-L" + cuda_lib, "-lcublas", "-Xlinker", "-rpath=" + cuda_lib]
+           "-cudart", "static"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)

@@ -428,8 +428,13 @@ mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64_t k, in
                      "GPTQ tiles");
 }
 
+size_t mxq_act_gram_workspace(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0) return 0;
+  return mxq::gram_full_workspace(rows, cols);
+}
+
 mxq_status mxq_act_gram(const void* X, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
-                        float* H, void* stream) {
+                        float* H, void* workspace, size_t workspace_bytes, void* stream) {
   if (dtype != MXQ_BF16) return fail(MXQ_ERR_DTYPE, "Gram matrix needs bf16 X (dtype %d)", dtype);
   mxq_status s = check_matrix(X, dtype, rows, cols, ld, "X");
   if (s != MXQ_OK) return s;
@@ -441,8 +446,12 @@ mxq_status mxq_act_gram(const void* X, int32_t dtype, int64_t rows, int64_t cols
   cudaStream_t st = (cudaStream_t)stream;
   if (rows == 0)
     return cuda_status(cudaMemsetAsync(H, 0, (size_t)cols * cols * sizeof(float), st), "memset H");
+  const size_t need = mxq_act_gram_workspace(rows, cols);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(MXQ_ERR_ALIGN, "workspace not 16-byte aligned");
   const char* why = "";
-  cudaError_t e = mxq::launch_gram_full(X, rows, cols, ld, H, st, &why);
+  cudaError_t e = mxq::launch_gram_full(X, rows, cols, ld, H, workspace, st, &why);
   if (e == cudaErrorUnknown && why[0]) return fail(MXQ_ERR_CUDA, "Gram matrix: %s", why);
   return cuda_status(e, "Gram matrix");
 }

@@ -26,7 +26,6 @@
 #include "mxq_gridk.cuh"
 #include "mxq_internal.h"
 
-#include <cublas_v2.h>
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -897,98 +896,5 @@ cudaError_t launch_gptq_order(const GptqArgs& g, const uint8_t* codes, const uin
 }
 
 int gptq_sort_max() { return kSortMax; }
-
-// ======================================================================================
-// the full Gram matrix H = X^T X / R (plain GEMMs: cuBLAS, bf16 in, float32 out)
-// ======================================================================================
-// H is symmetric, so only one triangle is multiplied out, by recursive halving: at level
-// l = 1 .. d the k x k matrix is cut into 2^l diagonal blocks of s = k / 2^l, and each pair of
-// sibling blocks contributes its off-diagonal s x s rectangle (one strided-batched GEMM of
-// 2^(l-1) rectangles per level); the 2^d diagonal blocks of the last level are multiplied out
-// whole (one more strided-batched GEMM). That is (1/2 + 1/2^(d+1)) of the full product's
-// tensor work. A transpose then copies the upper triangle onto the lower one, so H comes out
-// exactly symmetric.
-namespace {
-std::mutex g_blas_mu;
-cublasHandle_t g_blas[64] = {};
-
-constexpr int kMirror = 32;
-
-// H[p][q] = H[q][p] for q < p; one 32 x 32 tile of the lower triangle per CTA (32 x 8 threads)
-__global__ void __launch_bounds__(256) k_mirror_lower(float* H, int64_t k) {
-  __shared__ float tile[kMirror][kMirror + 1];
-  const int tq = blockIdx.x, tp = blockIdx.y;
-  if (tq > tp) return;
-  const int tx = threadIdx.x % kMirror, ty = threadIdx.x / kMirror;
-#pragma unroll
-  for (int r = 0; r < kMirror; r += 8) {
-    const int64_t q = (int64_t)tq * kMirror + ty + r, pc = (int64_t)tp * kMirror + tx;
-    if (q < k && pc < k) tile[ty + r][tx] = H[q * k + pc];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < kMirror; r += 8) {
-    const int64_t pr = (int64_t)tp * kMirror + ty + r, q = (int64_t)tq * kMirror + tx;
-    if (pr < k && q < pr) H[pr * k + q] = tile[tx][ty + r];
-  }
-}
-}  // namespace
-
-// levels of halving for a k-wide Gram matrix: each half stays a multiple of 8 columns (16-byte
-// aligned operands) and at least kGramMinBlock wide; at most 4
-constexpr int64_t kGramMinBlock = 1024;
-int gram_levels(int64_t k) {
-  int d = 0;
-  while (d < 4 && k % ((int64_t)16 << d) == 0 && (k >> (d + 1)) >= kGramMinBlock) ++d;
-  return d;
-}
-
-cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t ld, float* H,
-                             cudaStream_t st, const char** why) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  const int64_t tiles = (cols + kMirror - 1) / kMirror;
-  if (tiles > 65535) {                  // the mirror's grid; H would hold over 4e12 entries
-    *why = "cols beyond 65535 * 32";
-    return cudaErrorUnknown;
-  }
-  // the handle is shared by the device's callers: the lock covers binding it to this call's
-  // stream and every launch on it (all asynchronous)
-  std::lock_guard<std::mutex> lk(g_blas_mu);
-  if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
-    *why = "cublasCreate failed";
-    return cudaErrorUnknown;
-  }
-  cublasHandle_t hd = g_blas[dev];
-  const float alpha = (float)(1.0 / (double)rows), beta = 0.0f;
-  const __nv_bfloat16* x = (const __nv_bfloat16*)X;
-  // column-major view: X^T is [cols x rows] with leading dimension ld, and the column-major
-  // cols x cols result C(i, j) = sum_r X[r][i] X[r][j] is H read row-major (C(i, j) = H[j][i]);
-  // the rectangles below have i > j, the upper triangle of H
-  cublasStatus_t s = cublasSetStream(hd, st);
-  const int d = gram_levels(cols);
-  for (int l = 1; l <= d && s == CUBLAS_STATUS_SUCCESS; ++l) {
-    const int64_t b = cols >> l, pairs = (int64_t)1 << (l - 1);
-    s = cublasGemmStridedBatchedEx(hd, CUBLAS_OP_N, CUBLAS_OP_T, (int)b, (int)b, (int)rows,
-                                   &alpha, x + b, CUDA_R_16BF, (int)ld, 2 * b, x, CUDA_R_16BF,
-                                   (int)ld, 2 * b, &beta, H + b, CUDA_R_32F, (int)cols,
-                                   2 * b * (cols + 1), (int)pairs, CUBLAS_COMPUTE_32F,
-                                   CUBLAS_GEMM_DEFAULT);
-  }
-  if (s == CUBLAS_STATUS_SUCCESS) {
-    const int64_t b = cols >> d;
-    s = cublasGemmStridedBatchedEx(hd, CUBLAS_OP_N, CUBLAS_OP_T, (int)b, (int)b, (int)rows,
-                                   &alpha, x, CUDA_R_16BF, (int)ld, b, x, CUDA_R_16BF, (int)ld,
-                                   b, &beta, H, CUDA_R_32F, (int)cols, b * (cols + 1),
-                                   (int)((int64_t)1 << d), CUBLAS_COMPUTE_32F,
-                                   CUBLAS_GEMM_DEFAULT);
-  }
-  if (s != CUBLAS_STATUS_SUCCESS) {
-    *why = "cublasGemmStridedBatchedEx failed";
-    return cudaErrorUnknown;
-  }
-  k_mirror_lower<<<dim3((unsigned)tiles, (unsigned)tiles), 256, 0, st>>>(H, cols);
-  return cudaGetLastError();
-}
 
 }  // namespace mxq

@@ -20,6 +20,7 @@
 // memory before returning.
 #include "mxq_common.cuh"
 #include "mxq_internal.h"
+#include "mxq_tc.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -334,12 +335,15 @@ __global__ void k_gram_finalize(const double* __restrict__ partial, int chunks, 
   }
 }
 
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+bool encode_bf16_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                    uint32_t box_cols, uint32_t box_rows) {
   static EncodeTiledFn fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -348,10 +352,16 @@ EncodeTiledFn encode_fn() {
       p = nullptr;
     return (EncodeTiledFn)p;
   }();
-  return fn;
+  if (!fn) return false;
+  std::memset(map, 0, sizeof *map);
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 int gram_chunks(int64_t rows, int64_t cols, int B) {
   const int64_t strips = (cols + kGramCols - 1) / kGramCols;
@@ -371,18 +381,8 @@ size_t gram_workspace(int64_t rows, int64_t cols, int B) {
 
 cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, int B, float* G,
                         float* h, void* workspace, cudaStream_t st) {
-  EncodeTiledFn encode = encode_fn();
-  if (!encode) return cudaErrorNotSupported;
   CUtensorMap map;
-  std::memset(&map, 0, sizeof map);
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  const cuuint32_t box[2] = {64, 64};
-  const cuuint32_t estr[2] = {1, 1};
-  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  if (!encode_bf16_2d(&map, X, rows, cols, ld, 64, kGramRows)) return cudaErrorInvalidValue;
   const int chunks = gram_chunks(rows, cols, B);
   const int64_t stages = (rows + kGramRows - 1) / kGramRows;
   const int64_t per_chunk = (stages + chunks - 1) / chunks * kGramRows;

@@ -106,8 +106,10 @@ cudaError_t launch_gptq_sweep(const GptqArgs& g, cudaStream_t st);
 int gptq_sort_max();
 cudaError_t launch_gptq_order(const GptqArgs& g, const uint8_t* codes, const uint8_t* scales,
                               double* loss, int32_t* perm, cudaStream_t st);
+// ---- the full Gram matrix on the tensor cores (mxq_gram_full.cu) ---------------------------
+size_t gram_full_workspace(int64_t rows, int64_t cols);
 cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t ld, float* H,
-                             cudaStream_t st, const char** why);
+                             void* workspace, cudaStream_t st, const char** why);
 
 int sm_count();
 // Raises func's dynamic shared-memory limit to `bytes` on the current device, once per

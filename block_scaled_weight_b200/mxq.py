@@ -34,7 +34,8 @@ EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc
            "mxq_act_sqsum", "mxq_act_block_gram_workspace", "mxq_act_block_gram",
            "mxq_act_sqmean_finalize", "mxq_quantize", "mxq_quantize_gram", "mxq_project",
            "mxq_swizzled_scales_bytes", "mxq_swizzle_scales", "mxq_output_error_workspace",
-           "mxq_output_error", "mxq_gptq_prepare", "mxq_gptq_tiles", "mxq_act_gram",
+           "mxq_output_error", "mxq_gptq_prepare", "mxq_gptq_tiles", "mxq_act_gram_workspace",
+           "mxq_act_gram",
            "mxq_gptq_factor_workspace", "mxq_gptq_factor", "mxq_gptq_order_workspace",
            "mxq_gptq_order", "mxq_gptq_workspace", "mxq_gptq", "mxq_dequant",
            "mxq_error_workspace",
@@ -75,7 +76,8 @@ _sig = {
     "mxq_swizzle_scales": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
     "mxq_gptq_prepare": (ctypes.c_int, [_P, _I64, ctypes.c_double, _P, _P]),
     "mxq_gptq_tiles": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]),
-    "mxq_act_gram": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P]),
+    "mxq_act_gram_workspace": (_SZ, [_I64, _I64]),
+    "mxq_act_gram": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mxq_gptq_factor_workspace": (_SZ, [_I64]),
     "mxq_gptq_factor": (ctypes.c_int, [_P, _I64, _I32, _P, ctypes.c_double, _P, _P, _SZ, _P]),
     "mxq_gptq_order_workspace": (_SZ, [_I64, _I64, ctypes.POINTER(MxqParams)]),
@@ -306,13 +308,19 @@ def mxq_gptq_tiles(W: torch.Tensor, U: torch.Tensor, scales: torch.Tensor, *, co
     return codes
 
 
-def mxq_act_gram(X: torch.Tensor, H: torch.Tensor | None = None, *, stream=None) -> torch.Tensor:
+def mxq_act_gram_workspace(rows: int, cols: int) -> int:
+    return int(_lib.mxq_act_gram_workspace(rows, cols))
+
+
+def mxq_act_gram(X: torch.Tensor, H: torch.Tensor | None = None, *, workspace=None,
+                 stream=None) -> torch.Tensor:
     """H = X^T X / R [K, K] float32 of bf16 X [R, K] (GPTQ's Hessian up to a factor)."""
     R, K = X.shape
     if H is None:
         H = torch.empty(K, K, dtype=torch.float32, device=X.device)
-    _check(_lib.mxq_act_gram(_ptr(X), _dtype(X), R, K, _ld(X), _ptr(H), _stream(stream, X.device)),
-           "mxq_act_gram")
+    ws = _workspace(mxq_act_gram_workspace(R, K), X.device, workspace)
+    _check(_lib.mxq_act_gram(_ptr(X), _dtype(X), R, K, _ld(X), _ptr(H), _ptr(ws), ws.numel(),
+                             _stream(stream, X.device)), "mxq_act_gram")
     return H
 
 

@@ -363,11 +363,14 @@ MXQ_API mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64
  *
  * mxq_act_gram: H = X^T X / R, the full cols x cols Gram matrix (the GPTQ Hessian up to a
  *  factor) of bf16 X [rows, cols] (ld as for mxq_act_sqmean), float32, row-major, 16-byte
- *  aligned. Plain GEMMs (cuBLAS; bf16 products, float32 accumulation in the library's
- *  order) over one triangle only -- the matrix halved up to four times, each level's
- *  off-diagonal blocks and the last level's diagonal blocks as strided-batched products --
- *  then the upper triangle copied onto the lower one: H is exactly symmetric, and each
- *  entry is within rows * 2^-24 * (|X|^T |X|)_ij / rows of the exact value.
+ *  aligned. Computed on the tensor cores (tcgen05, pairs of SMs, 256 x 512 tiles of H) over
+ *  the tiles that reach the upper triangle: bf16 products (exact), float32 accumulation
+ *  over the rows in order (the last wave's tiles in row chunks added in double in a fixed
+ *  order), then the upper triangle copied onto the lower one: H is exactly symmetric,
+ *  deterministic, and each entry is within rows * 2^-24 * (|X|^T |X|)_ij / rows of the
+ *  exact value. workspace: mxq_act_gram_workspace(rows, cols) bytes, 16-byte aligned (at
+ *  most one 256 x 512 float32 partial tile per pair of SMs). A launch whose internal waits
+ *  time out (none does on a working GPU) writes NaN over all of H.
  *
  * mxq_gptq_factor: U [k][k] float32 (upper, the strict lower triangle written as 0), the
  *  upper Cholesky factor of (H~ + lambda I)^-1, H~ = (H + H^T) / 2 with rows and columns in
@@ -411,8 +414,10 @@ MXQ_API mxq_status mxq_gptq_tiles(const void* W, int32_t dtype, int64_t n, int64
  *  Result: identical to the definition above, including ties (each scale search scores
  *  every candidate exactly in float64, element order; lowest code on equal errors).
  * ------------------------------------------------------------------------------------ */
+MXQ_API size_t mxq_act_gram_workspace(int64_t rows, int64_t cols);
 MXQ_API mxq_status mxq_act_gram(const void* X, int32_t dtype, int64_t rows, int64_t cols,
-                                int64_t ld, float* H, void* stream);
+                                int64_t ld, float* H, void* workspace, size_t workspace_bytes,
+                                void* stream);
 MXQ_API size_t mxq_gptq_factor_workspace(int64_t k);
 MXQ_API mxq_status mxq_gptq_factor(const float* H, int64_t k, int32_t block,
                                    const int32_t* perm, double damp, float* U, void* workspace,

@@ -384,6 +384,22 @@ def gram(X) -> np.ndarray:
     return (Xf.T @ Xf / R).astype(np.float32) if R else np.zeros((Xf.shape[1],) * 2, np.float32)
 
 
+def gram_entries(X, pairs, chunk_rows: int = 16384) -> np.ndarray:
+    """Entries (i, j) of the Gram matrix H = X^T X / R of X [R, K] (float64 sums of the exact
+    products, then / R; float64 result) for pairs [P, 2] of column indices -- the same
+    definition as ``gram`` for matrices too large to multiply out on the host."""
+    Xin, _ = _as_input(X)
+    R = Xin.shape[0]
+    pairs = np.asarray(pairs, np.int64)
+    cols, inv = np.unique(pairs.reshape(-1), return_inverse=True)
+    a, b = inv.reshape(-1, 2).T
+    acc = np.zeros(len(pairs))
+    for r0 in range(0, R, chunk_rows):
+        Xc = to_float(Xin[r0:r0 + chunk_rows])[:, cols].astype(np.float64)
+        acc += (Xc[:, a] * Xc[:, b]).sum(axis=0)
+    return acc / R if R else acc
+
+
 def block_losses(W, h, fmt: str, mode: str, block: int, *, sfmt: str = "e4m3",
                  window: int = -1, n_threads=1) -> np.ndarray:
     """Hessian-weighted quantization loss of each column block: sum over rows and the

@@ -176,10 +176,15 @@ def test_gptq_rejections(mxq):
     assert prep(None, 0, 0.01, None, None) == 0                                        # empty
     # Hessian, factor, order, sweep
     gram = L.mxq_act_gram
-    assert gram(FAKE, 0, 100, 64, 64, FAKE, None) == S["MXQ_ERR_DTYPE"]                 # float32 X
-    assert gram(FAKE, 1, 100, 64, 64, None, None) == S["MXQ_ERR_INVALID_ARG"]
-    assert gram(FAKE, 1, 100, 64, 64, ODD, None) == S["MXQ_ERR_ALIGN"]
-    assert gram(None, 1, 100, 0, 0, None, None) == 0                                   # no columns
+    gws = mxq.mxq_act_gram_workspace(100, 64)
+    assert gws >= 256 and mxq.mxq_act_gram_workspace(0, 64) == 0
+    assert gram(FAKE, 0, 100, 64, 64, FAKE, FAKE, gws, None) == S["MXQ_ERR_DTYPE"]      # float32 X
+    assert gram(FAKE, 1, 100, 64, 64, None, FAKE, gws, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert gram(FAKE, 1, 100, 64, 64, ODD, FAKE, gws, None) == S["MXQ_ERR_ALIGN"]
+    assert gram(FAKE, 1, 100, 64, 64, FAKE, None, gws, None) == S["MXQ_ERR_WORKSPACE"]
+    assert gram(FAKE, 1, 100, 64, 64, FAKE, FAKE, gws - 8, None) == S["MXQ_ERR_WORKSPACE"]
+    assert gram(FAKE, 1, 100, 64, 64, FAKE, FAKE + 8, gws, None) == S["MXQ_ERR_ALIGN"]
+    assert gram(None, 1, 100, 0, 0, None, None, 0, None) == 0                          # no columns
     fac = L.mxq_gptq_factor
     need = mxq.mxq_gptq_factor_workspace(256)
     assert need == 256 + 2 * 256 * 256 * 8

@@ -287,3 +287,40 @@ def test_error_sums_full_size(mxq, orc, synth, wl_name, wi, fmt, block):
     assert m["h_rel"] == pytest.approx(mo["h_rel"], rel=1e-5)
     print(f"{wl_name}[{wi}] {fmt} bs{block}: weight error {m['weight_rel']:.4%}, "
           f"h-weighted {m['h_rel']:.4%} (oracle {mo['weight_rel']:.4%}, {mo['h_rel']:.4%})")
+
+
+def test_gram_full_size_sampled(mxq, orc, synth):
+    """The GPTQ Hessian H = X^T X / R of the full-calibration activations (244449 x 9728, the
+    launch the GPTQ benchmark times: 380 tiles of 256 x 512 over 74 pairs of SMs, five whole
+    waves and ten tiles cut into row chunks), checked entry by entry against the oracle's
+    float64 sums on sampled entries: every diagonal entry of a sampled set, random pairs,
+    and pairs at the tile edges (rows 255 / 256, columns 511 / 512, the last column)."""
+    wl = synth.WORKLOADS["nvfp4_full_calib"]
+    X = synth.workload_activations(wl, 0, device=DEV)
+    R, K = X.shape
+    H = mxq.mxq_act_gram(X)
+    torch.cuda.synchronize()
+    Xh = oracle_view(X)
+    del X
+    torch.cuda.empty_cache()
+    rng = np.random.default_rng(7)
+    edges = [0, 255, 256, 511, 512, 4607, 4608, 9215, 9216, K - 1]
+    pairs = np.concatenate([
+        np.stack([d := rng.choice(K, 256, replace=False), d], axis=1),
+        rng.integers(0, K, (768, 2)),
+        np.array([(i, j) for i in edges for j in edges])])
+    got = H[torch.as_tensor(pairs[:, 0], device=DEV),
+            torch.as_tensor(pairs[:, 1], device=DEV)].cpu().numpy().astype(np.float64)
+    sym = H[torch.as_tensor(pairs[:, 1], device=DEV),
+            torch.as_tensor(pairs[:, 0], device=DEV)].cpu().numpy().astype(np.float64)
+    assert np.array_equal(got, sym)
+    ref = orc.gram_entries(Xh, pairs)
+    absref = np.zeros(len(pairs))                # (|X|^T |X|)_ij for the bound
+    for r0 in range(0, R, 16384):
+        c = np.abs(orc.to_float(Xh[r0:r0 + 16384])).astype(np.float64)
+        absref += (c[:, pairs[:, 0]] * c[:, pairs[:, 1]]).sum(axis=0)
+    tol = (R + 2) * 2.0 ** -24 * absref / R + 1e-38
+    err = np.abs(got - ref)
+    assert np.all(err <= tol), float((err / tol).max())
+    print(f"Gram 244449 x 9728: {len(pairs)} sampled entries within the float32 bound; "
+          f"largest error / bound {float((err / tol).max()):.3g}")

@@ -5,15 +5,16 @@ Bars:
 - the sweep (mxq_gptq) is bit-exact: given the oracle's factor U (and block order), every
   scale and code equals the oracle's -- both evaluate the definition's float32 steps in its
   order, and every scale search scores its candidates exactly;
-- the block order (mxq_gptq_order) equals the oracle's: the losses are float64 sums of the
-  same float32 terms in different orders, so only blocks whose losses agree to ~1e-12
-  relative could swap (none do on these inputs);
+- the block order (mxq_gptq_order) equals the oracle's except where two blocks' losses
+  agree to 1e-12 relative: the losses are float64 sums of the same float32 terms in
+  different orders, so only such blocks can swap;
 - the factor (mxq_gptq_factor): float64 on both sides by different stable routes, rounded
   to float32 once: |dU| <= 2^-23 |U| + 2^-28 max|U| (the float64 difference is a small
   multiple of cond(H) 2^-53 of the largest entry, cond(H) <= 1 + 100 k with the damping);
-- the Gram matrix (mxq_act_gram: cuBLAS GEMMs over one triangle, accumulating bf16 products
-  in float32 in an unspecified order, times fl32(1/R), then mirrored):
-  |dH| <= (R + 2) 2^-24 (|X|^T |X|)_ij / R, and H exactly symmetric;
+- the Gram matrix (mxq_act_gram: tensor-core tiles over the upper triangle, accumulating
+  bf16 products in float32 over the rows in order -- the last wave's tiles in row chunks
+  added in double --, times 1/R, then mirrored):
+  |dH| <= (R + 2) 2^-24 (|X|^T |X|)_ij / R, H exactly symmetric and the same on every run;
 - end to end (Gram, order, factor and sweep on the GPU against the oracle's pipeline on the
   same X and W): the Gram matrices differ within that bound, which moves U, so codes are
   compared by what is unique: the output error within 1% and below the plain quantizer's.
@@ -48,14 +49,17 @@ def correlated_x(synth, rows, k, seed, device):
     return X.to(torch.bfloat16)
 
 
-# k = 2048 and 4096 take one and two levels of the triangle's halving (strided-batched
-# rectangles plus diagonal blocks); the smaller ones a single product
+# Tiles of H are 256 x 512 per pair of SMs, 74 pairs on a B200: k <= 4096 gives fewer tiles
+# than pairs (every tile cut into row chunks, added in a fixed order); k = 6144 gives 156
+# tiles (two whole waves, then 8 tiles in chunks); 208 and 777 rows leave ragged edges in
+# both dimensions
 @pytest.mark.parametrize("rows,k", [(3000, 256), (777, 208), (20000, 512), (3000, 2048),
-                                    (600, 4096)])
+                                    (600, 4096), (1000, 6144), (65, 8)])
 def test_gram_matches_oracle(mxq, orc, synth, rows, k):
     X = correlated_x(synth, rows, k, 121, DEV)
     H = mxq.mxq_act_gram(X).cpu().numpy()
     assert np.array_equal(H, H.T)
+    assert np.array_equal(H, mxq.mxq_act_gram(X).cpu().numpy())       # deterministic
     Xo = oracle_view(X)
     ref = orc.gram(Xo).astype(np.float64)
     A = np.abs(orc.to_float(Xo).astype(np.float64))
@@ -75,9 +79,23 @@ def block_cols(perm, B):
     return (np.asarray(perm)[:, None] * B + np.arange(B)[None, :]).reshape(-1)
 
 
+def test_gram_odd_width(mxq, orc, synth):
+    """102 columns of a 104-wide matrix: rows of H are not 16-byte multiples, and the last
+    column group of every TMA box lies partly beyond the matrix (zero fill)."""
+    rows = 1234
+    X = correlated_x(synth, rows, 104, 125, DEV)[:, :102]
+    H = mxq.mxq_act_gram(X).cpu().numpy()
+    assert H.shape == (102, 102) and np.array_equal(H, H.T)
+    Xo = oracle_view(X)
+    ref = orc.gram(Xo).astype(np.float64)
+    A = np.abs(orc.to_float(Xo).astype(np.float64))
+    tol = (rows + 2) * 2.0 ** -24 * (A.T @ A) / rows + 1e-38
+    assert np.all(np.abs(H - ref) <= tol), float((np.abs(H - ref) / tol).max())
+
+
 def test_gram_strided_columns(mxq, orc, synth):
-    """X a column slice of a wider matrix (ld 2304, 2048 columns: one level of halving): the
-    products' operand offsets are columns of the slice."""
+    """X a column slice of a wider matrix (ld 2304, 2048 columns starting at column 128): the
+    tiles' operand offsets are columns of the slice."""
     rows = 1500
     big = correlated_x(synth, rows, 2304, 123, DEV)
     X = big[:, 128:2176]

@@ -157,6 +157,24 @@ def test_gram_is_the_mean_outer_product(orc):
     assert np.array_equal(np.diagonal(H), orc.act_sqmean(X))
 
 
+def test_gram_entries_exact_sums(orc):
+    """Sampled Gram entries on small-integer bf16 inputs: every product and every partial sum
+    is an integer below 2^53, so the float64 sums are exact and must equal Python's integer
+    sums over the rows, divided by R once; chunking the rows (3 rows a chunk here) must not
+    change the result. The diagonal equals the h pass."""
+    rng = np.random.default_rng(16)
+    R, K = 11, 9
+    Xi = rng.integers(-40, 41, (R, K))
+    X = (np.asarray(Xi, np.float32).view(np.uint32) >> 16).astype(np.uint16)   # exact bf16
+    pairs = np.array([(0, 0), (0, 8), (8, 0), (3, 5), (5, 3), (7, 7), (2, 6)])
+    got = orc.gram_entries(X, pairs, chunk_rows=3)
+    ref = [sum(int(Xi[r, i]) * int(Xi[r, j]) for r in range(R)) / R for i, j in pairs]
+    assert got.tolist() == ref
+    d = np.arange(K)
+    diag = orc.gram_entries(X, np.stack([d, d], axis=1))
+    assert np.array_equal(diag.astype(np.float32), orc.act_sqmean(X))
+
+
 GRIDS = {"nvfp4": [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0],
          "int4": [0.0, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 7.0]}
 
