@@ -17,6 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmxq.so")
 SOURCES = ["mxq_api.cu", "mxq_hpass.cu", "mxq_gram.cu", "mxq_quant.cu", "mxq_quant_grid.cu",
            "mxq_error.cu", "mxq_outerr.cu", "mxq_gptq.cu", "mxq_gptq_full.cu", "mxq_gram_full.cu",
+           "mxq_nvfp4_mm.cu",
            "mxq_noalloc.cu"]
 HEADERS = ["mxq_common.cuh", "mxq_internal.h", "mxq_block.cuh", "mxq_grids.h", "mxq_gridk.cuh",
            "mxq_chol64.cuh", "mxq_tc.cuh"]

@@ -370,6 +370,35 @@ mxq_status mxq_swizzle_scales(const uint8_t* scales, int64_t n, int64_t kb, uint
                      "swizzle scales");
 }
 
+size_t mxq_nvfp4_gemm_workspace(void) { return mxq::nvfp4_mm_workspace(); }
+
+mxq_status mxq_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
+                          const uint8_t* b_codes, const uint8_t* b_scales, int64_t m, int64_t n,
+                          int64_t k, float* D, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  if (m < 0 || n < 0 || k < 0) return fail(MXQ_ERR_SHAPE, "negative shape");
+  if (m > 0x7fffffff || n > 0x7fffffff || k > 0x7fffffff)
+    return fail(MXQ_ERR_SHAPE, "m, n and k must be below 2^31");
+  if (k % 64 != 0) return fail(MXQ_ERR_SHAPE, "k %% 64 != 0");
+  if (m == 0 || n == 0) return MXQ_OK;
+  if (!D) return fail(MXQ_ERR_INVALID_ARG, "D is NULL");
+  if (!aligned(D, 16)) return fail(MXQ_ERR_ALIGN, "D not 16-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (k == 0) return cuda_status(cudaMemsetAsync(D, 0, (size_t)m * n * sizeof(float), st), "memset D");
+  if (!a_codes || !a_scales || !b_codes || !b_scales)
+    return fail(MXQ_ERR_INVALID_ARG, "NULL operand");
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_scales, 16) ||
+      !aligned(b_scales, 16))
+    return fail(MXQ_ERR_ALIGN, "operands must be 16-byte aligned");
+  if (!workspace || workspace_bytes < mxq::nvfp4_mm_workspace())
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes,
+                mxq::nvfp4_mm_workspace());
+  if (!aligned(workspace, 16)) return fail(MXQ_ERR_ALIGN, "workspace not 16-byte aligned");
+  return cuda_status(mxq::launch_nvfp4_mm(a_codes, a_scales, b_codes, b_scales, m, n, k, D,
+                                          workspace, st),
+                     "NVFP4 product");
+}
+
 size_t mxq_error_workspace(int64_t n, int64_t k) {
   if (n <= 0 || k <= 0) return 0;
   return (size_t)mxq::error_partials(n, k) * 4 * sizeof(double);

@@ -78,6 +78,12 @@ cudaError_t launch_outerr(const void* X, int64_t m, int64_t k, int64_t ldx, cons
                           int fmt, int scale_fmt, int block, double* sums, void* workspace,
                           cudaStream_t st);
 
+// ---- NVFP4 x NVFP4 product on the block-scaled tensor cores (mxq_nvfp4_mm.cu) -----------
+size_t nvfp4_mm_workspace();
+cudaError_t launch_nvfp4_mm(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* b_codes,
+                            const uint8_t* b_sf, int64_t m, int64_t n, int64_t k, float* D,
+                            void* workspace, cudaStream_t st);
+
 // ---- FP8-GPTQ on 64 x 64 tiles (mxq_gptq.cu) ---------------------------------------------
 cudaError_t launch_gptq_prepare(const float* G, int64_t nblocks, double damp, float* U,
                                 cudaStream_t st);

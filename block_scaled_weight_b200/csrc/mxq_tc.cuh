@@ -15,6 +15,9 @@ namespace mxq {
 // (elements), boxes of box_cols x box_rows, 128-byte swizzle, zero fill out of range.
 bool encode_bf16_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
                     uint32_t box_cols, uint32_t box_rows);
+// The same for any element type of `elsize` bytes (ld in elements).
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, int elsize, const void* base,
+               int64_t rows, int64_t cols, int64_t ld, uint32_t box_cols, uint32_t box_rows);
 
 namespace tc {
 
@@ -151,6 +154,82 @@ __device__ __forceinline__ void commit_pair(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar)
                : "memory");
+}
+
+// K-major operand with 128-byte swizzle: rows of 128 bytes, 8-row groups 1 KB apart (stride
+// byte offset); the leading byte offset is unused for swizzled K-major layouts.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)((1024u >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Unswizzled matrix of 16-byte rows stored contiguously (8-row core matrices 128 bytes apart):
+// the source of a 32-row x 128-bit tensor-memory copy.
+__device__ __forceinline__ uint64_t desc_rows16(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((128u >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((128u >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (packed, K-major), UE4M3 scale
+// vectors (scale-factor IDs 0), float32 D.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global memory
+// into this CTA's shared memory, completing on an mbarrier of this CTA.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// D (+)= (A x scale_A) (B x scale_B)^T over K = 64 E2M1 elements, one UE4M3 scale per 16
+// elements of a row, scales read from tensor memory; one thread of the CTA issues it.
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], "
+      "[%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate));
+}
+
+// Copy a 32-row x 128-bit shared-memory matrix into tensor memory at column `taddr`, the same
+// rows into each of the four 32-lane quarters (4 columns of 32 bits per lane).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc));
+}
+
+__device__ __forceinline__ void commit_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(cols));
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
 }
 
 // Tensor memory of a pair: one warp of each CTA executes these together.

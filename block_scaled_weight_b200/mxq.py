@@ -33,7 +33,8 @@ SCALE = {"e4m3": 0, "ue4m4": 1, "ue5m3": 2, "ue8m0": 3}
 EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc",
            "mxq_act_sqsum", "mxq_act_block_gram_workspace", "mxq_act_block_gram",
            "mxq_act_sqmean_finalize", "mxq_quantize", "mxq_quantize_gram", "mxq_project",
-           "mxq_swizzled_scales_bytes", "mxq_swizzle_scales", "mxq_output_error_workspace",
+           "mxq_swizzled_scales_bytes", "mxq_swizzle_scales", "mxq_nvfp4_gemm_workspace",
+           "mxq_nvfp4_gemm", "mxq_output_error_workspace",
            "mxq_output_error", "mxq_gptq_prepare", "mxq_gptq_tiles", "mxq_act_gram_workspace",
            "mxq_act_gram",
            "mxq_gptq_factor_workspace", "mxq_gptq_factor", "mxq_gptq_order_workspace",
@@ -74,6 +75,8 @@ _sig = {
     "mxq_output_error": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _P,
                                         ctypes.POINTER(MxqParams), _P, _P, _SZ, _P]),
     "mxq_swizzle_scales": (ctypes.c_int, [_P, _I64, _I64, _P, _P]),
+    "mxq_nvfp4_gemm_workspace": (_SZ, []),
+    "mxq_nvfp4_gemm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "mxq_gptq_prepare": (ctypes.c_int, [_P, _I64, ctypes.c_double, _P, _P]),
     "mxq_gptq_tiles": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P, _P]),
     "mxq_act_gram_workspace": (_SZ, [_I64, _I64]),
@@ -402,6 +405,20 @@ def mxq_swizzle_scales(scales: torch.Tensor, *, out=None, stream=None) -> torch.
     _check(_lib.mxq_swizzle_scales(_ptr(scales), n, kb, _ptr(out), _stream(stream, scales.device)),
            "mxq_swizzle_scales")
     return out
+
+
+def mxq_nvfp4_gemm(a_codes: torch.Tensor, a_scales_sw: torch.Tensor, b_codes: torch.Tensor,
+                   b_scales_sw: torch.Tensor, m: int, n: int, k: int, *, D=None, workspace=None,
+                   stream=None) -> torch.Tensor:
+    """D = dequant(A) dequant(B)^T [m, n] float32 on the block-scaled tensor cores, from NVFP4
+    codes [rows, k/2] and scales already in the swizzled layout (mxq_swizzle_scales)."""
+    if D is None:
+        D = torch.empty(m, n, dtype=torch.float32, device=a_codes.device)
+    ws = _workspace(int(_lib.mxq_nvfp4_gemm_workspace()), a_codes.device, workspace)
+    _check(_lib.mxq_nvfp4_gemm(_ptr(a_codes), _ptr(a_scales_sw), _ptr(b_codes), _ptr(b_scales_sw),
+                               m, n, k, _ptr(D), _ptr(ws), ws.numel(),
+                               _stream(stream, a_codes.device)), "mxq_nvfp4_gemm")
+    return D
 
 
 def mxq_dequant(codes: torch.Tensor, scales: torch.Tensor, p: MxqParams, n: int, k: int, *,

@@ -282,6 +282,32 @@ MXQ_API mxq_status mxq_swizzle_scales(const uint8_t* scales, int64_t n, int64_t 
                                       uint8_t* out, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * The product of two NVFP4 operands in this library's output format, on the block-scaled
+ * tensor cores: D = A^ B^T with A^ = dequant(A) [m, k] and B^ = dequant(B) [n, k], each an
+ * NVFP4 matrix of 16-element blocks along k -- E2M1 codes and one E4M3 scale per block
+ * ("Is Finer Better? The Limits of Microscaling Formats in LLMs", sec. 2.1: x^ = s q). The
+ * hardware (tcgen05.mma kind::mxf4nvf4, scale_vec::4X) reads the codes as mxq_quantize packs
+ * them and the scales in the layout mxq_swizzle_scales writes, so quantized weights feed a
+ * block-scaled GEMM as they are; e.g. Y = X_q W_q^T with X quantized along its rows.
+ *
+ *  a_codes    device uint8 [m, k/2] (NVFP4 codes, element 2i in the low nibble), 16-byte
+ *             aligned; b_codes likewise [n, k/2].
+ *  a_scales   device, the E4M3 block scales of A [m, k/16] rewritten by mxq_swizzle_scales
+ *             (mxq_swizzled_scales_bytes(m, k/16) bytes), 16-byte aligned; b_scales likewise.
+ *  k          a multiple of 64; m, n, k below 2^31.
+ *  D          device float [m, n] row-major, 16-byte aligned: D[i][j] = sum_c A^[i][c] B^[j][c],
+ *             float32 accumulation in the tensor cores (each product of two scaled E2M1
+ *             values is exact), within (k + 2) 2^-24 (|A^| |B^|^T)_ij of the exact sum.
+ *  workspace  device, mxq_nvfp4_gemm_workspace() bytes, 16-byte aligned. A launch whose
+ *             internal waits time out (none does on a working GPU) writes NaN over D.
+ * ------------------------------------------------------------------------------------ */
+MXQ_API size_t mxq_nvfp4_gemm_workspace(void);
+MXQ_API mxq_status mxq_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
+                                  const uint8_t* b_codes, const uint8_t* b_scales, int64_t m,
+                                  int64_t n, int64_t k, float* D, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * Weight error (qwantize "Results": ||Q(W) - W||_F / ||W||_F) and the h-weighted error
  * (the diagonal objective, "quantization_algorithms.txt", sec. 1), without materialising
  * the dequantised matrix.

@@ -44,3 +44,13 @@ def order_with_ties(perm, perm_ref, losses, rel=1e-12):
     assert not bad.any(), f"{int(bad.sum())} positions differ beyond the tie rule"
     s = L[perm_ref]
     return int((np.abs(s[1:] - s[:-1]) <= rel * np.abs(s[:-1])).sum())
+
+
+def output_error_np(Xs, W, What) -> float:
+    """||X_s What^T - X_s W^T||_F / ||X_s W^T||_F in float64 with plain numpy (a measurement
+    of a GPU result in the test itself, so that no GPU output becomes an oracle input)."""
+    Xs = np.asarray(Xs, np.float64)
+    Y = Xs @ np.asarray(W, np.float64).T
+    Yq = Xs @ np.asarray(What, np.float64).T
+    den = np.linalg.norm(Y)
+    return float(np.linalg.norm(Yq - Y) / den) if den > 0 else 0.0

@@ -185,6 +185,18 @@ def test_gptq_rejections(mxq):
     assert gram(FAKE, 1, 100, 64, 64, FAKE, FAKE, gws - 8, None) == S["MXQ_ERR_WORKSPACE"]
     assert gram(FAKE, 1, 100, 64, 64, FAKE, FAKE + 8, gws, None) == S["MXQ_ERR_ALIGN"]
     assert gram(None, 1, 100, 0, 0, None, None, 0, None) == 0                          # no columns
+    mm = L.mxq_nvfp4_gemm
+    mws = mxq.mxq_nvfp4_gemm_workspace() if hasattr(mxq, "mxq_nvfp4_gemm_workspace") else \
+        L.mxq_nvfp4_gemm_workspace()
+    assert mm(FAKE, FAKE, FAKE, FAKE, 128, 128, 96, FAKE, FAKE, mws, None) == S["MXQ_ERR_SHAPE"]
+    assert mm(FAKE, FAKE, FAKE, FAKE, -1, 128, 64, FAKE, FAKE, mws, None) == S["MXQ_ERR_SHAPE"]
+    assert mm(FAKE, FAKE, FAKE, FAKE, 128, 128, 64, None, FAKE, mws, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert mm(None, FAKE, FAKE, FAKE, 128, 128, 64, FAKE, FAKE, mws, None) == S["MXQ_ERR_INVALID_ARG"]
+    assert mm(FAKE + 8, FAKE, FAKE, FAKE, 128, 128, 64, FAKE, FAKE, mws, None) == S["MXQ_ERR_ALIGN"]
+    assert mm(FAKE, FAKE, FAKE, FAKE + 4, 128, 128, 64, FAKE, FAKE, mws, None) == S["MXQ_ERR_ALIGN"]
+    assert mm(FAKE, FAKE, FAKE, FAKE, 128, 128, 64, FAKE, None, mws, None) == S["MXQ_ERR_WORKSPACE"]
+    assert mm(FAKE, FAKE, FAKE, FAKE, 128, 128, 64, FAKE, FAKE, mws - 8, None) == S["MXQ_ERR_WORKSPACE"]
+    assert mm(None, None, None, None, 0, 128, 64, None, None, 0, None) == 0            # empty
     fac = L.mxq_gptq_factor
     need = mxq.mxq_gptq_factor_workspace(256)
     assert need == 256 + 2 * 256 * 256 * 8

@@ -264,7 +264,8 @@ def test_error_sums_full_size(mxq, orc, synth, wl_name, wi, fmt, block):
     whole weight at its full shape -- the launch configuration the benchmark times (the
     headline 2560 x 9728 weight, the decoder layer's 14336 x 4096 gate projection, the INT8
     workload's weight) -- against the oracle's float64 sums of the same codes, 1e-5
-    relative. h from 8192 rows of the workload's activations (the oracle's, uploaded)."""
+    relative. h from 8192 rows of the workload's activations, and the codes and scales, are
+    the oracle's (uploaded), so both sides measure the same quantization."""
     wl = synth.WORKLOADS[wl_name]
     W = synth.workload_weight(wl, wi, device=DEV)
     n, k = W.shape
@@ -274,11 +275,13 @@ def test_error_sums_full_size(mxq, orc, synth, wl_name, wi, fmt, block):
     del X
     hd = torch.from_numpy(h).to(DEV)
     p = mxq.params(fmt, "hopt", block, window=wl.window)
-    codes, scales = mxq.mxq_quantize(W, p, hd)
+    Wo = oracle_view(W)
+    r = orc.quantize(Wo, fmt, "hopt", block, h=h, window=wl.window, n_threads=NT)
+    codes, scales = torch.from_numpy(r.codes).to(DEV), torch.from_numpy(r.scales).to(DEV)
     sums = mxq.mxq_error(W, codes, scales, p, hd).cpu().numpy()
     sums0 = mxq.mxq_error(W, codes, scales, p, None).cpu().numpy()
-    What = orc.dequant(codes.cpu().numpy(), scales.cpu().numpy(), fmt, block, n, k)
-    ref = orc.error_sums(oracle_view(W), What, h)
+    What = orc.dequant(r.codes, r.scales, fmt, block, n, k)
+    ref = orc.error_sums(Wo, What, h)
     np.testing.assert_allclose(sums, ref, rtol=1e-5)
     np.testing.assert_allclose(sums0[:2], ref[:2], rtol=1e-5)
     assert sums0[2] == 0 and sums0[3] == 0

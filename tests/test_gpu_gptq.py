@@ -20,7 +20,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import oracle_view
+from gpu_util import output_error_np, oracle_view
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -196,7 +196,11 @@ def test_end_to_end_against_oracle_pipeline(mxq, orc, synth):
     assert np.mean(cg[mask] != ref[mask]) <= 1e-4
     idx = synth.sample_rows(rows, 512, 99).to(DEV)
     Xs = oracle_view(X[idx])
-    e_gpu = orc.output_error(Xs, Wo, orc.dequant(cg, sg, "e4m3", T, n, k))
+    # the GPU result measured with its own dequant and plain numpy (no GPU output enters the
+    # oracle); the oracle's pipeline and the plain tile search measured by the oracle
+    pg = mxq.params("e4m3", "hopt", T)
+    What_gpu = mxq.mxq_dequant(codes, scales, pg, n, k).cpu().numpy()
+    e_gpu = output_error_np(orc.to_float(Xs), orc.to_float(Wo), What_gpu)
     e_ref = orc.output_error(Xs, Wo, orc.dequant(ref, r.scales, "e4m3", T, n, k))
     e_plain = orc.output_error(Xs, Wo, orc.dequant(r.codes, r.scales, "e4m3", T, n, k))
     assert e_gpu == pytest.approx(e_ref, rel=1e-3)

@@ -23,7 +23,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import oracle_view, order_with_ties
+from gpu_util import oracle_view, order_with_ties, output_error_np
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -241,7 +241,10 @@ def test_end_to_end_against_oracle_pipeline(mxq, orc, synth):
 
     def out_err(c, s):
         return orc.output_error(Xs, Wo, orc.dequant(c, s, "nvfp4", B, n, k))
-    e_gpu = out_err(codes.cpu().numpy(), scales.cpu().numpy())
+    # the GPU result measured with its own dequant and plain numpy (no GPU output enters the
+    # oracle)
+    What_gpu = mxq.mxq_dequant(codes, scales, p, n, k).cpu().numpy()
+    e_gpu = output_error_np(orc.to_float(Xs), orc.to_float(Wo), What_gpu)
     e_ref = out_err(r.codes, r.scales)
     assert e_gpu == pytest.approx(e_ref, rel=1e-2)
     assert e_gpu < 0.95 * out_err(plain.codes, plain.scales)

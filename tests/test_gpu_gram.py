@@ -164,11 +164,9 @@ def test_gpu_gram_feeds_search(mxq, orc, synth):
     r = orc.quantize_gram(oracle_view(W), "nvfp4", B, Go)
     Wf = orc.to_float(oracle_view(W)).astype(np.float64)
 
-    def diffs(c, s):
-        return (Wf - orc.dequant(c, s, "nvfp4", B, n, k)).reshape(n, k // B, B)
-
-    dg = diffs(codes.cpu().numpy(), scales.cpu().numpy())
-    do = diffs(r.codes, r.scales)
+    # the GPU picks decoded by the GPU's own dequant (no GPU output enters the oracle)
+    dg = (Wf - mxq.mxq_dequant(codes, scales, p, n, k).cpu().numpy()).reshape(n, k // B, B)
+    do = (Wf - orc.dequant(r.codes, r.scales, "nvfp4", B, n, k)).reshape(n, k // B, B)
     A = np.abs(Gg - Go.astype(np.float64))
     e_g = np.einsum("nbi,bij,nbj->nb", dg, Go.astype(np.float64), dg)
     slack = (np.einsum("nbi,bij,nbj->nb", np.abs(dg), A, np.abs(dg)) +

@@ -113,11 +113,13 @@ def test_dequant_and_error_parity(mxq, orc, synth, fmt, sfmt):
     h = orc.act_sqmean(oracle_view(X))
     hd = torch.from_numpy(h).to(DEV)
     p = mxq.params(fmt, "hopt", 16, scale_fmt=sfmt)
-    codes, scales = mxq.mxq_quantize(W, p, hd)
+    # the oracle's quantization, uploaded: both sides decode and measure the same codes
+    r = orc.quantize(oracle_view(W), fmt, "hopt", 16, h=h, sfmt=sfmt)
+    codes, scales = torch.from_numpy(r.codes).to(DEV), torch.from_numpy(r.scales).to(DEV)
     What = mxq.mxq_dequant(codes, scales, p, n, k)
     sums = mxq.mxq_error(W, codes, scales, p, hd)
     torch.cuda.synchronize()
-    ref = orc.dequant(codes.cpu().numpy(), scales.cpu().numpy(), fmt, 16, n, k, sfmt=sfmt)
+    ref = orc.dequant(r.codes, r.scales, fmt, 16, n, k, sfmt=sfmt)
     assert np.array_equal(What.cpu().numpy(), ref)
     rs = orc.error_sums(oracle_view(W), ref, h)
     np.testing.assert_allclose(sums.cpu().numpy(), rs, rtol=1e-5)

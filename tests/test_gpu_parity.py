@@ -279,12 +279,13 @@ def test_dequant_and_error_parity(mxq, orc, synth, fmt, block, mode):
     h = orc.act_sqmean(oracle_view(X))
     hd = torch.from_numpy(h).to(DEV)
     p = mxq.params(fmt, mode, block)
-    codes, scales = mxq.mxq_quantize(W, p, hd if mode == "hopt" else None)
+    # the oracle's quantization, uploaded: both sides decode and measure the same codes
+    r = orc.quantize(oracle_view(W), fmt, mode, block, h=h if mode == "hopt" else None)
+    c_np, s_np = r.codes, r.scales
+    codes, scales = torch.from_numpy(c_np).to(DEV), torch.from_numpy(s_np).to(DEV)
     What = mxq.mxq_dequant(codes, scales, p, n, k)
     sums = mxq.mxq_error(W, codes, scales, p, hd)
     torch.cuda.synchronize()
-    c_np = codes.cpu().numpy()
-    s_np = scales.cpu().numpy()
     ref = orc.dequant(c_np, s_np, fmt, block, n, k)
     assert np.array_equal(What.cpu().numpy(), ref)
     rs = orc.error_sums(oracle_view(W), ref, h)
