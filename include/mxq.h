@@ -29,15 +29,19 @@
  *
  * Conventions for every call below:
  *  - Pointers named as device pointers are device memory (any allocator) owned by the
- *    caller; the library allocates nothing. Workspace sizes come from the *_workspace
- *    queries.
+ *    caller; the library allocates no device memory for data. Workspace sizes come from the
+ *    *_workspace queries.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
  *    stream) unless stated otherwise. Results are valid after the stream synchronises.
  *  - Arguments are validated on the host before any launch; a rejected call launches
  *    nothing and returns a status. A CUDA launch failure returns MXQ_ERR_CUDA and
  *    mxq_last_error() (per host thread) describes it. No exception crosses the boundary.
- *  - Calls are reentrant: the library keeps no mutable state besides the per-thread
- *    error text.
+ *  - Calls are reentrant. Mutable state, all of it set up on first use and guarded by
+ *    locks: the per-thread error text; per device, the raised shared-memory limit of each
+ *    tensor-core kernel; per device, the two library streams and their events that
+ *    mxq_gptq_factor and mxq_gptq create on first use (their calls on one device are
+ *    ordered on the host); and per device the address of the static scratch of
+ *    mxq_act_sqmean_noalloc.
  *  - Empty problems (n, k or rows == 0) return MXQ_OK without launching.
  *  - Weights and activations may not contain NaN or infinities (the result is then
  *    unspecified, but no launch faults).
