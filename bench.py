@@ -102,6 +102,21 @@ def source_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def executed_for(kernel):
+    """Executed thread instructions per launch (and active lanes per warp instruction) from a
+    committed ncu capture, if the kernel source is unchanged."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, rec["source"])
+        if source_sha(src) != rec["source_sha"] or "thread_inst_per_launch" not in rec:
+            return None
+        return {"thread_inst": rec["thread_inst_per_launch"], "lanes": rec.get("lanes_per_inst"),
+                "candidates_per_block": rec.get("candidates_per_block")}
+    except Exception:
+        return None
+
+
 def traffic_for(kernel):
     """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged."""
     try:
@@ -482,16 +497,22 @@ def gpu_arm(args):
     for wi, (_, n, k) in enumerate(wl.weights):
         Ws.append(synth.workload_weight(wl_r, wi, device=dev))
         cs, cd, ss, sd = mxq.output_shapes(p, n, k)
+        ews = max(mxq.mxq_error_workspace(n, k), mxq.mxq_quantize_err_workspace(n, k, p))
         outs.append((torch.empty(cs, dtype=cd, device=dev), torch.empty(ss, dtype=sd, device=dev),
                      torch.empty(4, dtype=torch.float64, device=dev),
-                     torch.empty(mxq.mxq_error_workspace(n, k), dtype=torch.uint8, device=dev),
+                     torch.empty(ews, dtype=torch.uint8, device=dev),
                      synth.x_index_for_weight(wl, wi)))
     stream = torch.cuda.current_stream(dev)
+    # The NVFP4 search with E4M3 scales adds the error sums itself (mxq_quantize_err: search,
+    # exact pass, combine); every other quantizer runs the error pass after it.
+    fused = fmt == "nvfp4" and q.sfmt == "e4m3" and mode in ("sse", "hopt")
     # our kernels per step: h pass or Gram pass (2 per activation matrix; 3 with the sharded
     # finalize), search (+ exact fixup for NVFP4 / INT8 searches), error sums + combine (2)
-    # per weight; GPTQ adds the factor (1 per activation matrix) and the sweep (1 per weight)
+    # per weight (fused: the combine only); GPTQ adds the factor (1 per activation matrix)
+    # and the sweep (1 per weight)
     fixup = 1 if mode != "naive" and fmt != "e4m3" else 0
-    launches_per_step = len(Xs) * (2 if world == 1 else 3) + len(Ws) * (1 + fixup + 2)
+    launches_per_step = len(Xs) * (2 if world == 1 else 3) + len(Ws) * (
+        1 + fixup + (1 if fused else 2))
     if gq:
         launches_per_step += len(Xs) + len(Ws)
 
@@ -512,8 +533,11 @@ def gpu_arm(args):
             mxq.mxq_gptq_prepare(G, GPTQ_DAMP, U=U)
 
     def quantize_phase():
-        for W, (codes, scales, _, _, xi) in zip(Ws, outs):
-            if bh:
+        for W, (codes, scales, sums, ews, xi) in zip(Ws, outs):
+            if fused:
+                mxq.mxq_quantize_err(W, p, hs[xi], codes=codes, scales=scales, sums=sums,
+                                     workspace=ews)
+            elif bh:
                 mxq.mxq_quantize_gram(W, p, Gs[xi], codes=codes, scales=scales)
             else:
                 mxq.mxq_quantize(W, p, hs[xi], codes=codes, scales=scales)
@@ -533,7 +557,8 @@ def gpu_arm(args):
     phases.append(("quantize", quantize_phase))
     if gq:
         phases.append(("gptq_tiles", sweep_phase))
-    phases.append(("error", error_phase))
+    if not fused:
+        phases.append(("error", error_phase))
 
     def step(ev=None):
         for i, (_, fn) in enumerate(phases):
@@ -581,7 +606,7 @@ def gpu_arm(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_total, *k_ph = t.tolist()
     k_of = {nm: kk for (nm, _), kk in zip(phases, k_ph)}
-    k_h, k_q, k_e = k_of[hname], k_of["quantize"], k_of["error"]
+    k_h, k_q, k_e = k_of[hname], k_of["quantize"], k_of.get("error")
     ms_step = ms_total / args.steps
     ms_step_serial = ms_step
     weights = sum(W.numel() for W in Ws)
@@ -609,8 +634,12 @@ def gpu_arm(args):
             with torch.cuda.stream(s_q):
                 s_q.wait_event(ev_h[b])
                 for W, (codes, scales, sums, ews, xi) in zip(Ws, outs):
-                    mxq.mxq_quantize(W, p, hb[b][xi], codes=codes, scales=scales)
-                    mxq.mxq_error(W, codes, scales, p, hb[b][xi], sums=sums, workspace=ews)
+                    if fused:
+                        mxq.mxq_quantize_err(W, p, hb[b][xi], codes=codes, scales=scales,
+                                             sums=sums, workspace=ews)
+                    else:
+                        mxq.mxq_quantize(W, p, hb[b][xi], codes=codes, scales=scales)
+                        mxq.mxq_error(W, codes, scales, p, hb[b][xi], sums=sums, workspace=ews)
                 ev_q[b].record(s_q)
 
         for i in range(args.warmup):
@@ -697,6 +726,19 @@ def gpu_arm(args):
                                "peak": ALU_PEAK_TOPS, "unit": "T lane-op/s",
                                "frac": q_tops / ALU_PEAK_TOPS, "algorithmic_ops": ops,
                                "traffic": traffic_for("quantize") if headline else None}
+        if fused:
+            kernels["quantize"]["includes"] = ("the error sums at the winning scales (added "
+                                               "inside the search and its exact pass)")
+        ex = executed_for("quantize") if headline else None
+        if ex:
+            # the hardware's view: thread instructions the search kernels executed per launch
+            # (an ncu capture of this build) over the launch time, against the lane peak
+            kernels["quantize"]["executed"] = {
+                "thread_inst_per_launch": ex["thread_inst"],
+                "achieved": ex["thread_inst"] / (k_q * 1e-3) / 1e12,
+                "frac_executed": ex["thread_inst"] / (k_q * 1e-3) / 1e12 / ALU_PEAK_TOPS,
+                "active_lanes_per_inst": ex["lanes"],
+                "candidates_scored_per_block": ex.get("candidates_per_block")}
     if gq:
         u_bytes = sum(2 * 4 * X.shape[1] * block for X in Xs)     # G read, U written
         kernels["gptq_prepare"] = {
@@ -710,11 +752,12 @@ def gpu_arm(args):
                                  "peak": ALU_PEAK_TOPS, "unit": "T lane-op/s",
                                  "frac": s_tops / ALU_PEAK_TOPS, "algorithmic_ops": s_ops,
                                  "traffic": None}
-    e_bytes = w_bytes + weights * code_bytes(fmt, block) + sum(4 * W.shape[1] for W in Ws)
-    e_gbs = e_bytes / (k_e * 1e-3) / 1e9
-    kernels["error"] = {"ms": k_e, "bound": "hbm", "achieved": e_gbs, "peak": hbm, "unit": "GB/s",
-                        "frac": e_gbs / hbm, "algorithmic_bytes": e_bytes,
-                        "traffic": traffic_for("error") if headline else None}
+    if k_e is not None:
+        e_bytes = w_bytes + weights * code_bytes(fmt, block) + sum(4 * W.shape[1] for W in Ws)
+        e_gbs = e_bytes / (k_e * 1e-3) / 1e9
+        kernels["error"] = {"ms": k_e, "bound": "hbm", "achieved": e_gbs, "peak": hbm,
+                            "unit": "GB/s", "frac": e_gbs / hbm, "algorithmic_bytes": e_bytes,
+                            "traffic": traffic_for("error") if headline else None}
     dom = max(kernels, key=lambda kk: kernels[kk]["ms"])
     dk = kernels[dom]
     roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"],

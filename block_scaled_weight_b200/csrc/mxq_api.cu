@@ -255,13 +255,16 @@ mxq_status mxq_act_block_gram(const void* X, int32_t dtype, int64_t rows, int64_
                      "block Gram");
 }
 
-mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
-                        const float* h, const mxq_params* p, void* codes, void* scales,
-                        void* stream) {
+// Validation shared by mxq_quantize and mxq_quantize_err; fills `a` for a non-empty
+// problem (a->n == 0 when there is nothing to launch).
+static mxq_status prepare_quantize(const void* W, int32_t dtype, int64_t n, int64_t k,
+                                   int64_t ld, const float* h, const mxq_params* p, void* codes,
+                                   void* scales, mxq::QuantArgs* a) {
   mxq_status s = check_matrix(W, dtype, n, k, ld, "W");
   if (s != MXQ_OK) return s;
   s = check_params(p, n, k);
   if (s != MXQ_OK) return s;
+  a->n = 0;
   if (n == 0 || k == 0) return MXQ_OK;
   if (!codes || !scales) return fail(MXQ_ERR_INVALID_ARG, "codes or scales is NULL");
   if (!aligned(codes, 16)) return fail(MXQ_ERR_ALIGN, "codes not 16-byte aligned");
@@ -271,26 +274,78 @@ mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int6
     if (!h) return fail(MXQ_ERR_INVALID_ARG, "H-optimal needs h");
     if (!aligned(h, 16)) return fail(MXQ_ERR_ALIGN, "h not 16-byte aligned");
   }
-  mxq::QuantArgs a{};
-  a.W = W;
-  a.dtype = dtype;
-  a.n = n;
-  a.k = k;
-  a.ld = ld;
-  a.h = p->mode == MXQ_HOPT ? h : nullptr;
-  a.fmt = p->fmt;
-  a.mode = p->mode;
-  a.block = p->block;
-  a.window = p->window;
-  a.scale_fmt = p->scale_fmt;
-  a.codes = codes;
-  a.scales = scales;
-  a.log_points = p->fmt == MXQ_FMT_E4M3 && p->mode != MXQ_NAIVE ? p->log_points : 0;
-  for (int i = 0; i < a.log_points; ++i) {
+  a->W = W;
+  a->dtype = dtype;
+  a->n = n;
+  a->k = k;
+  a->ld = ld;
+  a->h = p->mode == MXQ_HOPT ? h : nullptr;
+  a->fmt = p->fmt;
+  a->mode = p->mode;
+  a->block = p->block;
+  a->window = p->window;
+  a->scale_fmt = p->scale_fmt;
+  a->codes = codes;
+  a->scales = scales;
+  a->log_points = p->fmt == MXQ_FMT_E4M3 && p->mode != MXQ_NAIVE ? p->log_points : 0;
+  for (int i = 0; i < a->log_points; ++i) {
     const double lo = p->log_lo_exp2, hi = p->log_hi_exp2;
-    a.log_grid[i] = (float)std::exp2(lo + (hi - lo) * (double)i / (double)(a.log_points - 1));
+    a->log_grid[i] = (float)std::exp2(lo + (hi - lo) * (double)i / (double)(a->log_points - 1));
   }
+  return MXQ_OK;
+}
+
+mxq_status mxq_quantize(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                        const float* h, const mxq_params* p, void* codes, void* scales,
+                        void* stream) {
+  mxq::QuantArgs a{};
+  mxq_status s = prepare_quantize(W, dtype, n, k, ld, h, p, codes, scales, &a);
+  if (s != MXQ_OK || a.n == 0) return s;
   return cuda_status(mxq::launch_quantize(a, (cudaStream_t)stream), "quantize");
+}
+
+// The NVFP4 search with E4M3 scales adds the error sums itself; every other quantizer is
+// followed by the error pass.
+static bool fused_error(const mxq_params* p) {
+  return p->fmt == MXQ_FMT_NVFP4 && p->scale_fmt == 0 && p->mode != MXQ_NAIVE;
+}
+
+size_t mxq_quantize_err_workspace(int64_t n, int64_t k, const mxq_params* p) {
+  if (n <= 0 || k <= 0 || !p) return 0;
+  const int64_t parts = fused_error(p) && (p->block == 16 || p->block == 32)
+                            ? mxq::fp4_error_parts(n, k, p->block)
+                            : mxq::error_partials(n, k);
+  return (size_t)parts * 4 * sizeof(double);
+}
+
+mxq_status mxq_quantize_err(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,
+                            const float* h, const mxq_params* p, void* codes, void* scales,
+                            double* sums, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  mxq::QuantArgs a{};
+  mxq_status s = prepare_quantize(W, dtype, n, k, ld, h, p, codes, scales, &a);
+  if (s != MXQ_OK) return s;
+  if (!sums) return fail(MXQ_ERR_INVALID_ARG, "sums is NULL");
+  if (!aligned(sums, 8)) return fail(MXQ_ERR_ALIGN, "sums not 8-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (a.n == 0) return cuda_status(cudaMemsetAsync(sums, 0, 4 * sizeof(double), st), "memset");
+  if (h && !aligned(h, 16)) return fail(MXQ_ERR_ALIGN, "h not 16-byte aligned");
+  const size_t need = mxq_quantize_err_workspace(n, k, p);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXQ_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!aligned(workspace, 8)) return fail(MXQ_ERR_ALIGN, "workspace not 8-byte aligned");
+  if (fused_error(p)) {
+    a.err_partial = (double*)workspace;
+    a.err_sums = sums;
+    a.h_err = p->mode == MXQ_HOPT ? nullptr : h;
+    return cuda_status(mxq::launch_quantize(a, st), "quantize with error sums");
+  }
+  cudaError_t e = mxq::launch_quantize(a, st);
+  if (e != cudaSuccess) return cuda_status(e, "quantize");
+  mxq::DecodeArgs d{codes, scales, p->fmt, p->block, p->scale_fmt, n, k};
+  return cuda_status(mxq::launch_error(d, W, dtype, ld, h, (double*)workspace,
+                                       mxq::error_partials(n, k), sums, st),
+                     "error");
 }
 
 mxq_status mxq_quantize_gram(const void* W, int32_t dtype, int64_t n, int64_t k, int64_t ld,

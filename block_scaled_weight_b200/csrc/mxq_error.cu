@@ -254,6 +254,11 @@ cudaError_t error_fmt(const DecodeArgs& d, const void* W, int dtype, int64_t ld,
 
 }  // namespace
 
+cudaError_t launch_error_final(const double* partial, int parts, double* sums, cudaStream_t st) {
+  k_error_final<<<1, kThreads, 0, st>>>(partial, parts, sums);
+  return cudaGetLastError();
+}
+
 int error_partials(int64_t n, int64_t k) {
   const int64_t units = n * (k / 16);
   int64_t ctas = (units + kThreads - 1) / kThreads;

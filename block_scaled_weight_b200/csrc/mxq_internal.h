@@ -45,8 +45,15 @@ struct QuantArgs {
   void* scales;
   int log_points;
   float log_grid[256];  // E4M3 tiles: g_p
+  // fused error sums (NVFP4 searches with E4M3 scales): per-CTA partials, the four sums, and
+  // h for the h-weighted sums of an SSE search (HOPT uses h)
+  double* err_partial = nullptr;
+  double* err_sums = nullptr;
+  const float* h_err = nullptr;
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
+// Partial slots the fused error sums of an NVFP4 search need (search CTAs + exact-pass CTAs).
+int fp4_error_parts(int64_t n, int64_t k, int B);
 // E2M1 on a scale grid other than E4M3, and INT4 on any grid (mxq_quant_grid.cu).
 cudaError_t launch_quantize_grid(const QuantArgs& a, cudaStream_t st);
 // Block-Hessian search (d^T G_b d) for E2M1 / INT4 elements on any scale grid.
@@ -67,6 +74,8 @@ size_t swizzled_scales_bytes(int64_t n, int64_t kb);
 cudaError_t launch_swizzle_scales(const uint8_t* in, int64_t n, int64_t kb, uint8_t* out,
                                   cudaStream_t st);
 int error_partials(int64_t n, int64_t k);
+// sums[i] = sum over p < parts of partial[p][i], in a fixed order.
+cudaError_t launch_error_final(const double* partial, int parts, double* sums, cudaStream_t st);
 cudaError_t launch_error(const DecodeArgs& d, const void* W, int dtype, int64_t ld,
                          const float* h, double* partial, int parts, double* sums,
                          cudaStream_t st);

@@ -56,6 +56,9 @@ struct Fp4Params {
   int window;
   uint8_t* codes;
   uint8_t* scales;
+  double* err_partial;     // per-CTA error sums (search CTAs, then fixup CTAs), or null
+  const float* h_err;      // h for the h-weighted sums of an SSE search, or null
+  int fix_slot0;           // first partial slot of the fixup CTAs
 };
 
 // fl32(|w| / s) for an E4M3 scale s, from the split reciprocal (see the file header).
@@ -170,26 +173,6 @@ k_fp4_naive(Fp4Params P, Fp4Table T) {
   }
 }
 
-// Float32 error of one candidate from precomputed exact quotients x (pairs):
-// sum_j c_j (a_j - s g_j)^2 with g = RNE_E2M1(x).
-template <int B, bool HOPT>
-__device__ __forceinline__ float fp4_eval_x(const float2 (&a)[B / 2], const float2 (&c)[B / 2],
-                                            const float2 (&xs)[B / 2], float2 pow2,
-                                            uint32_t s_neg_h) {
-  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int p = 0; p < B / 2; ++p) {
-    const float2 d = fp4_pair_diff(a[p], __fmul2_rn(xs[p], pow2), s_neg_h);
-    float2& acc = (p & 1) ? acc1 : acc0;
-    if constexpr (HOPT) {
-      acc = __ffma2_rn(__fmul2_rn(c[p], d), d, acc);
-    } else {
-      acc = __ffma2_rn(d, d, acc);
-    }
-  }
-  return (acc0.x + acc0.y) + (acc1.x + acc1.y);
-}
-
 // Float32 error of the two bound elements (at, with weights ct) at one candidate.
 __device__ __forceinline__ float fp4_lb(float2 at, float2 ct, float2 x, uint32_t s_neg_h) {
   const float2 d = fp4_pair_diff(at, x, s_neg_h);
@@ -198,28 +181,112 @@ __device__ __forceinline__ float fp4_lb(float2 at, float2 ct, float2 x, uint32_t
 }
 
 
-// NVFP4, SSE / H-optimal search: one thread per block walks every candidate, grouped by
-// significand. Blocks whose float32 winner is not separated from the runner-up by the
-// error bound are flagged (bit 7 of the scale byte) for k_fp4_fixup.
+// NVFP4, SSE / H-optimal search, compacted. A warp owns 32 blocks: one column block jb
+// (so h is the same for every lane and stays in registers) in 32 consecutive rows, one block
+// per lane. Every lane first scores, in full, its naive code and the codes on either side
+// (the winner is usually within a few codes of the naive snap), then filters the rest of its
+// range with exact lower bounds, writing the codes that survive into its own list in shared
+// memory. The warp then scores the surviving (block, code) pairs 32 at a time -- every lane
+// takes the next pair, whoever's block it is, reading that block's magnitudes from shared
+// memory -- and each lane folds its own results back in code order. Blocks whose float32
+// winner is not separated from the runner-up by the error bound are flagged (bit 7 of the
+// scale byte) for k_fp4_fixup. With P.err_partial set, the kernel also adds each unflagged
+// block's error sums at its winning scale (float32 over the block, double beyond) into
+// per-CTA partials.
+constexpr int kFp4Queue = 128;       // scored pairs held per warp before the owners fold them
+constexpr int kFp4List = 132;        // bytes per lane's code list (126 codes; rows offset by a bank)
+
+template <int B>
+struct Fp4WarpSmem {
+  float a[32][B];                    // each lane's block magnitudes
+  float res[kFp4Queue];              // scores of the current window of pairs
+  int off[32];                       // first pair of each lane (exclusive prefix of counts)
+  uint8_t list[32 * kFp4List];       // surviving codes of each lane, ascending
+};
+
+template <int B>
+constexpr size_t fp4_search_smem() {
+  return (size_t)(kThreads / 32) * sizeof(Fp4WarpSmem<B>);
+}
+
+// Error sums of one block at table entry t: sum d^2, sum a^2, sum c d^2, sum c a^2 (float32
+// over the block, as the error pass does) added to acc in double.
+template <int B, bool HAS_C>
+__device__ __forceinline__ void fp4_block_sums(const float2 (&a)[B / 2], const float2 (&c)[B / 2],
+                                               float4 t, double (&acc)[4]) {
+  const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
+  const uint32_t sn = __float_as_uint(t.w) ^ 0x8000u;
+  float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
+#pragma unroll
+  for (int p = 0; p < B / 2; ++p) {
+    const float2 d = fp4_pair_diff(a[p], fp4_quot(a[p], rhi, rlo), sn);
+    const float2 d2 = __fmul2_rn(d, d), w2 = __fmul2_rn(a[p], a[p]);
+    s0 = __fadd2_rn(s0, d2);
+    s1 = __fadd2_rn(s1, w2);
+    if constexpr (HAS_C) {
+      s2 = __ffma2_rn(c[p], d2, s2);
+      s3 = __ffma2_rn(c[p], w2, s3);
+    }
+  }
+  acc[0] += (double)s0.x + (double)s0.y;
+  acc[1] += (double)s1.x + (double)s1.y;
+  if constexpr (HAS_C) {
+    acc[2] += (double)s2.x + (double)s2.y;
+    acc[3] += (double)s3.x + (double)s3.y;
+  }
+}
+
+// Fixed-order sum of the CTA's per-thread sums into partial[slot][4].
+__device__ void cta_sums(const double (&acc)[4], double* partial, int slot) {
+  __shared__ double red[kThreads / 32][4];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double r = warp_sum(acc[i]);
+    if (lane == 0) red[wid][i] = r;
+  }
+  __syncthreads();
+  if (threadIdx.x < 4) {
+    double s = 0.0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) s += red[w][threadIdx.x];
+    partial[(int64_t)slot * 4 + threadIdx.x] = s;
+  }
+}
+
 template <int B, bool BF16, bool HOPT>
 __global__ void __launch_bounds__(kThreads, B == 16 ? 3 : 2)
 k_fp4_search(Fp4Params P, Fp4Table T) {
   __shared__ float4 tab[128];
-  __shared__ float2 sig[8];
+  extern __shared__ __align__(16) unsigned char fp4_dyn[];
+  Fp4WarpSmem<B>& S = reinterpret_cast<Fp4WarpSmem<B>*>(fp4_dyn)[threadIdx.x >> 5];
   for (int i = threadIdx.x; i < 128; i += kThreads) tab[i] = T.c[i];
-  for (int i = threadIdx.x; i < 8; i += kThreads) sig[i] = T.sig[i];
   __syncthreads();
-  const int64_t kb = P.k / B, nblocks = P.n * kb;
+  const int lane = threadIdx.x & 31;
+  const int64_t kb = P.k / B, ntiles = (P.n + 31) / 32 * kb;
   const int elsz = BF16 ? 2 : 4;
   const float gam = (float)(B + 8) * 5.9604645e-8f;  // (B + 8) 2^-24
   const float lo_f = 1.0f - gam, hi_f = 1.0f + 2.0f * gam;
   const float slack = 7.3468396e-40f;                // 2^-130: underflow slack
-  for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks;
-       b += (int64_t)gridDim.x * kThreads) {
-    const int64_t row = b / kb, jb = b - row * kb;
+  const float lb_f = 1.0f - 8.0f * 5.9604645e-8f;
+  const bool want_err = P.err_partial != nullptr;
+  const bool err_h = HOPT || P.h_err != nullptr;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  uint8_t* my_list = S.list + lane * kFp4List;
+  const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  for (int64_t tile = gw; tile < ntiles; tile += nw) {
+    const int64_t rg = tile / kb, jb = tile - rg * kb;
+    const int64_t row = rg * 32 + lane;
+    const bool valid = row < P.n;
     float2 a[B / 2], c[B / 2];
-    uint32_t sgn;
-    load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
+    uint32_t sgn = 0;
+    if (valid) {
+      load_block<B, BF16>(P.W + row * P.ld_bytes + jb * B * elsz, a, sgn);
+    } else {
+#pragma unroll
+      for (int p = 0; p < B / 2; ++p) a[p] = make_float2(0.f, 0.f);
+    }
     if constexpr (HOPT) load_h<B>(P.h + jb * B, c);
     const int c0 = e4m3_rn_code(__fdiv_rn(block_amax<B>(a), 6.0f));
     int lo = 1, hi = 126;
@@ -228,126 +295,148 @@ k_fp4_search(Fp4Params P, Fp4Table T) {
       hi = min(126, c0 + P.window);
       if (c0 == 0) { lo = 1; hi = max(1, P.window); }
     }
+    if (!valid) hi = 0;                                // no candidates
     float m1 = __int_as_float(0x7f800000), m2 = m1;
     int i1 = lo;
-    // Seed: the naive code (clipped to the candidate range), evaluated in full.
-    const int cs = min(max(c0, lo), hi);
-    {
-      const float4 t = tab[cs];
-      const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
-      float2 xs[B / 2];
-#pragma unroll
-      for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
-      track(fp4_eval_x<B, HOPT>(a, c, xs, make_float2(1.f, 1.f), __float_as_uint(t.w) ^ 0x8000u),
-            cs, m1, m2, i1);
+    // the naive code (clipped to the candidate range) and its two neighbours, in full
+    const int cs = min(max(c0, lo), max(hi, lo));
+#pragma unroll 1
+    for (int d = -1; d <= 1; ++d) {
+      const int cc = cs + d;
+      if (cc >= lo && cc <= hi) track(fp4_eval<B, HOPT>(a, c, tab[cc]), cc, m1, m2, i1);
     }
-    // Lower bounds. A candidate's error is at least the error of any subset of elements;
-    // the subset here is the two elements with the largest c w^2 (t1, t2). A candidate
-    // whose bound, minus its float32 rounding margin, exceeds the current winner's upper
-    // bound can neither win nor tie, nor fall in the band that decides flagging: it is
-    // skipped without a full evaluation.
-    //
-    // Range cuts, from single elements j (T: the seed's upper bound, which only shrinks):
-    //  * for s < a_j / 6, element j maps to 6 s, so the error is at least
-    //    c_j (a_j - 6 s)^2, growing as s shrinks: every s below
-    //    max_j (a_j - sqrt(T / c_j)) / 6 is out;
-    //  * for s >= 4 a_j, element j's quotient is at most 0.25 and it maps to 0,
-    //    contributing exactly c_j a_j^2: every s >= min {4 a_j : c_j a_j^2 > T} is out.
-    // The candidate range shrinks to the codes in between. The margins (1e-5 relative)
-    // cover the float32 roundings of the approximate reciprocal square root and products.
-    float upper = fmaf(m1, hi_f, slack);
-    float2 at, ct;
-    float s_cut = 0.f, s_hi = __int_as_float(0x7f800000);
-    {
-      const float sqt = sqrtf(upper) * 1.00001f;
-      float v1 = -1.f, a1 = 0.f, c1 = 0.f, v2 = -1.f, a2 = 0.f, c2 = 0.f;
-      auto visit = [&](float aj, float cj) {
-        const float v = cj * aj * aj;
-        if (v > v1) { v2 = v1; a2 = a1; c2 = c1; v1 = v; a1 = aj; c1 = cj; }
-        else if (v > v2) { v2 = v; a2 = aj; c2 = cj; }
-        if (cj > 0.f) {
-          s_cut = fmaxf(s_cut, (aj - sqt * rsqrtf(cj)) * (1.0f / 6.0f) * 0.99999f);
-          if (v * 0.99999f - slack > upper) s_hi = fminf(s_hi, 4.0f * aj);
+    int cnt = 0;
+    if (valid) {
+      // Lower bounds. A candidate's error is at least the error of any subset of elements;
+      // the subset here is the two elements with the largest c w^2 (t1, t2). A candidate
+      // whose bound, minus its float32 rounding margin, exceeds the upper bound T of the
+      // best error so far can neither win nor tie, nor fall in the band that decides
+      // flagging: it is never scored.
+      //
+      // Range cuts, from single elements j:
+      //  * for s < a_j / 6, element j maps to 6 s, so the error is at least
+      //    c_j (a_j - 6 s)^2, growing as s shrinks: every s below
+      //    max_j (a_j - sqrt(T / c_j)) / 6 is out;
+      //  * for s >= 4 a_j, element j's quotient is at most 0.25 and it maps to 0,
+      //    contributing exactly c_j a_j^2: every s >= min {4 a_j : c_j a_j^2 > T} is out.
+      // The margins (1e-5 relative) cover the float32 roundings of the approximate
+      // reciprocal square root and products.
+      const float upper = fmaf(m1, hi_f, slack);
+      float2 at, ct;
+      float s_cut = 0.f, s_hi = __int_as_float(0x7f800000);
+      {
+        const float sqt = sqrtf(upper) * 1.00001f;
+        float v1 = -1.f, a1 = 0.f, c1 = 0.f, v2 = -1.f, a2 = 0.f, c2 = 0.f;
+        auto visit = [&](float aj, float cj) {
+          const float v = cj * aj * aj;
+          if (v > v1) { v2 = v1; a2 = a1; c2 = c1; v1 = v; a1 = aj; c1 = cj; }
+          else if (v > v2) { v2 = v; a2 = aj; c2 = cj; }
+          if (cj > 0.f) {
+            s_cut = fmaxf(s_cut, (aj - sqt * rsqrtf(cj)) * (1.0f / 6.0f) * 0.99999f);
+            if (v * 0.99999f - slack > upper) s_hi = fminf(s_hi, 4.0f * aj);
+          }
+        };
+#pragma unroll
+        for (int p = 0; p < B / 2; ++p) {
+          visit(a[p].x, HOPT ? c[p].x : 1.f);
+          visit(a[p].y, HOPT ? c[p].y : 1.f);
         }
-      };
-#pragma unroll
-      for (int p = 0; p < B / 2; ++p) {
-        visit(a[p].x, HOPT ? c[p].x : 1.f);
-        visit(a[p].y, HOPT ? c[p].y : 1.f);
+        at = make_float2(a1, a2);
+        ct = make_float2(c1, c2);
       }
-      at = make_float2(a1, a2);
-      ct = make_float2(c1, c2);
-    }
-    if (s_cut > 0.f) {
-      int cl = e4m3_rn_code(s_cut);
-      if (e4m3_pos(cl) < s_cut) ++cl;                 // smallest code with value >= s_cut
-      lo = max(lo, cl);
-    }
-    if (s_hi < 1e30f) {
-      int ch = e4m3_rn_code(s_hi);
-      if (!(e4m3_pos(ch) < s_hi)) --ch;               // largest code with value < s_hi
-      hi = min(hi, ch);
-    }
-    const float lb_f = 1.0f - 8.0f * 5.9604645e-8f;
-    // subnormal scales (codes 1..7): the split-reciprocal quotient per candidate
-    for (int cc = lo; cc <= min(hi, 7); ++cc) {
-      if (cc == cs) continue;
-      const float4 t = tab[cc];
-      const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
-      const uint32_t sn = __float_as_uint(t.w) ^ 0x8000u;
-      if (fp4_lb(at, ct, fp4_quot(at, rhi, rlo), sn) * lb_f - slack > upper) continue;
-      float2 xs[B / 2];
-#pragma unroll
-      for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
-      track(fp4_eval_x<B, HOPT>(a, c, xs, make_float2(1.f, 1.f), sn), cc, m1, m2, i1);
-      upper = fmaf(m1, hi_f, slack);
-    }
-    // Normal scales, grouped by mantissa field m: codes (e << 3) | m, e = 1..15. Their
-    // quotients are fl32(|w| 8/S) 2^(7-e) (S = 8 + m): exact power-of-two rescalings of
-    // one split-reciprocal quotient per significand (the result is a normal float
-    // whenever it can reach an E2M1 decision boundary).
-    for (int m = 0; m < 8; ++m) {
-      const int e_lo = max(1, (lo - m + 7) >> 3);
-      const int e_hi = min(m == 7 ? 14 : 15, (hi - m) >> 3);
-      if (e_lo > e_hi) continue;
-      const float2 r = sig[m];
-      const float2 rhi = make_float2(r.x, r.x), rlo = make_float2(r.y, r.y);
-      const float2 xt = fp4_quot(at, rhi, rlo);
-      float2 xs[B / 2];
-      bool have_xs = false;
-      for (int e = e_lo; e <= e_hi; ++e) {
-        const int cc = (e << 3) | m;
-        if (cc == cs) continue;
+      int lo2 = lo, hi2 = hi;
+      if (s_cut > 0.f) {
+        int cl = e4m3_rn_code(s_cut);
+        if (e4m3_pos(cl) < s_cut) ++cl;                 // smallest code with value >= s_cut
+        lo2 = max(lo2, cl);
+      }
+      if (s_hi < 1e30f) {
+        int ch = e4m3_rn_code(s_hi);
+        if (!(e4m3_pos(ch) < s_hi)) --ch;               // largest code with value < s_hi
+        hi2 = min(hi2, ch);
+      }
+      for (int cc = lo2; cc <= hi2; ++cc) {
+        if (cc >= cs - 1 && cc <= cs + 1) continue;    // scored above
         const float4 t = tab[cc];
-        const float pw = __int_as_float((134 - e) << 23);  // 2^(7 - e)
-        const float2 pw2 = make_float2(pw, pw);
-        const uint32_t sn = __float_as_uint(t.w) ^ 0x8000u;
-        if (fp4_lb(at, ct, __fmul2_rn(xt, pw2), sn) * lb_f - slack > upper) continue;
-        if (!have_xs) {
-#pragma unroll
-          for (int p = 0; p < B / 2; ++p) xs[p] = fp4_quot(a[p], rhi, rlo);
-          have_xs = true;
-        }
-        track(fp4_eval_x<B, HOPT>(a, c, xs, pw2, sn), cc, m1, m2, i1);
-        upper = fmaf(m1, hi_f, slack);
+        const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
+        if (fp4_lb(at, ct, fp4_quot(at, rhi, rlo), __float_as_uint(t.w) ^ 0x8000u) * lb_f -
+                slack > upper)
+          continue;
+        my_list[cnt++] = (uint8_t)cc;
       }
     }
-    if (!(m2 * lo_f - slack > upper)) {
-      // A second candidate may tie or beat the float32 winner: flag the block (bit 7 of
-      // the scale byte) for the exact pass, k_fp4_fixup.
-      P.scales[b] = (uint8_t)(0x80 | i1);
-    } else {
-      fp4_emit<B>(a, sgn, tab[i1], false, P.codes + row * (P.k / 2) + jb * (B / 2));
-      P.scales[b] = (uint8_t)i1;
+    // the block's magnitudes for the lanes that score its pairs
+#pragma unroll
+    for (int p = 0; p < B / 4; ++p)
+      *reinterpret_cast<float4*>(&S.a[lane][4 * p]) =
+          make_float4(a[2 * p].x, a[2 * p].y, a[2 * p + 1].x, a[2 * p + 1].y);
+    int off = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(kFull, off, o);
+      if (lane >= o) off += v;
     }
+    const int total = __shfl_sync(kFull, off, 31);
+    off -= cnt;
+    S.off[lane] = off;
+    __syncwarp();
+    for (int wbase = 0; wbase < total; wbase += kFp4Queue) {
+      const int wend = min(total, wbase + kFp4Queue);
+      for (int g = wbase + lane; g < wend; g += 32) {
+        int o = 0;                                      // the lane whose pairs include g
+#pragma unroll
+        for (int step = 16; step > 0; step >>= 1)
+          if (S.off[o + step] <= g) o += step;
+        const int cc = S.list[o * kFp4List + (g - S.off[o])];
+        float2 ao[B / 2];
+#pragma unroll
+        for (int p = 0; p < B / 4; ++p) {
+          const float4 v = *reinterpret_cast<const float4*>(&S.a[o][4 * p]);
+          ao[2 * p] = make_float2(v.x, v.y);
+          ao[2 * p + 1] = make_float2(v.z, v.w);
+        }
+        S.res[g - wbase] = fp4_eval<B, HOPT>(ao, c, tab[cc]);
+      }
+      __syncwarp();
+      const int j1 = min(off + cnt, wend);
+      for (int j = max(off, wbase); j < j1; ++j) track(S.res[j - wbase], my_list[j - off], m1, m2, i1);
+      __syncwarp();
+    }
+    if (valid) {
+      const float upper = fmaf(m1, hi_f, slack);
+      const int64_t b = row * kb + jb;
+      if (!(m2 * lo_f - slack > upper)) {
+        // A second candidate may tie or beat the float32 winner: flag the block (bit 7 of
+        // the scale byte) for the exact pass, k_fp4_fixup.
+        P.scales[b] = (uint8_t)(0x80 | i1);
+      } else {
+        const float4 t = tab[i1];
+        fp4_emit<B>(a, sgn, t, false, P.codes + row * (P.k / 2) + jb * (B / 2));
+        P.scales[b] = (uint8_t)i1;
+        if (want_err) {
+          if constexpr (HOPT) {
+            fp4_block_sums<B, true>(a, c, t, acc);
+          } else if (err_h) {
+            float2 ce[B / 2];
+            load_h<B>(P.h_err + jb * B, ce);
+            fp4_block_sums<B, true>(a, ce, t, acc);
+          } else {
+            fp4_block_sums<B, false>(a, c, t, acc);
+          }
+        }
+      }
+    }
+    __syncwarp();                                       // S is refilled by the next tile
   }
+  if (want_err) cta_sums(acc, P.err_partial, blockIdx.x);
 }
 
 // Exact pass over the blocks the search flagged. Each warp scans 32 scale bytes at a time;
 // every flagged block is handled by the whole warp: lanes evaluate candidates lo + lane +
 // 32 t in float32, the warp minimum bounds the band, candidates inside it are re-scored in
 // double in the definition's order, and the warp arg-min (lowest code on equal doubles)
-// is emitted.
+// is emitted. With P.err_partial set, the emitted blocks' error sums go into this CTA's
+// partial (after the search CTAs' partials).
 template <int B, bool BF16, bool HOPT>
 __global__ void __launch_bounds__(kThreads)
 k_fp4_fixup(Fp4Params P, Fp4Table T) {
@@ -362,6 +451,7 @@ k_fp4_fixup(Fp4Params P, Fp4Table T) {
   const float slack = 7.3468396e-40f;
   const int64_t gw = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
   for (int64_t base = gw * 32; base < nblocks; base += nw * 32) {
     const int64_t mine = base + lane;
     const bool flagged = mine < nblocks && (P.scales[mine] & 0x80);
@@ -406,9 +496,21 @@ k_fp4_fixup(Fp4Params P, Fp4Table T) {
       if (lane == 0) {
         fp4_emit<B>(a, sgn, tab[bi], false, P.codes + row * (P.k / 2) + jb * (B / 2));
         P.scales[b] = (uint8_t)bi;
+        if (P.err_partial) {
+          if constexpr (HOPT) {
+            fp4_block_sums<B, true>(a, c, tab[bi], acc);
+          } else if (P.h_err) {
+            float2 ce[B / 2];
+            load_h<B>(P.h_err + jb * B, ce);
+            fp4_block_sums<B, true>(a, ce, tab[bi], acc);
+          } else {
+            fp4_block_sums<B, false>(a, c, tab[bi], acc);
+          }
+        }
       }
     }
   }
+  if (P.err_partial) cta_sums(acc, P.err_partial, P.fix_slot0 + blockIdx.x);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -942,27 +1044,47 @@ int grid_for(int64_t work_threads) {
   return (int)(want < 1 ? 1 : (want > cap ? cap : want));
 }
 
+// Grids of the NVFP4 search and its exact pass (fixed by the shape and the device's SM
+// count, so the order of the fused error sums is too).
+template <int B>
+void fp4_grids(int64_t n, int64_t k, int& gs, int& gf) {
+  const int64_t ntiles = (n + 31) / 32 * (k / B);
+  const int64_t cap = (int64_t)sm_count() * (B == 16 ? 3 : 2);
+  const int64_t want = (ntiles + kThreads / 32 - 1) / (kThreads / 32);
+  gs = (int)(want < 1 ? 1 : (want > cap ? cap : want));
+  const int64_t fwant = (n * (k / B) + 32 * 8 - 1) / (32 * 8);   // one 32-block tile per warp
+  gf = (int)(fwant < 1 ? 1 : (fwant < (int64_t)sm_count() * 8 ? fwant : (int64_t)sm_count() * 8));
+}
+
 template <int B, bool BF16>
 cudaError_t fp4_dispatch(const QuantArgs& a, cudaStream_t st) {
   static const Fp4Table T = make_fp4_table();
   Fp4Params P{(const char*)a.W, a.n, a.k, a.ld * (BF16 ? 2 : 4), a.h, a.window,
-              (uint8_t*)a.codes, (uint8_t*)a.scales};
+              (uint8_t*)a.codes, (uint8_t*)a.scales, a.err_partial, a.h_err, 0};
   const int64_t nblocks = a.n * (a.k / B);
-  const int grid = grid_for(nblocks);
   if (a.mode == 0) {
-    k_fp4_naive<B, BF16><<<grid, kThreads, 0, st>>>(P, T);
+    k_fp4_naive<B, BF16><<<grid_for(nblocks), kThreads, 0, st>>>(P, T);
     return cudaGetLastError();
   }
-  if (a.mode == 1) k_fp4_search<B, BF16, false><<<grid, kThreads, 0, st>>>(P, T);
-  else k_fp4_search<B, BF16, true><<<grid, kThreads, 0, st>>>(P, T);
-  cudaError_t e = cudaGetLastError();
+  int gs, gf;
+  fp4_grids<B>(a.n, a.k, gs, gf);
+  P.fix_slot0 = gs;
+  const size_t smem = fp4_search_smem<B>();
+  const void* kern = a.mode == 1 ? (const void*)k_fp4_search<B, BF16, false>
+                                 : (const void*)k_fp4_search<B, BF16, true>;
+  cudaError_t e = ensure_dynamic_smem(kern, (int)smem);
   if (e != cudaSuccess) return e;
-  const int64_t fwant = (nblocks + 32 * 8 - 1) / (32 * 8);   // one 32-block tile per warp
-  const int fgrid = (int)(fwant < (int64_t)sm_count() * 8 ? fwant : (int64_t)sm_count() * 8);
-  if (a.mode == 1) k_fp4_fixup<B, BF16, false><<<fgrid, kThreads, 0, st>>>(P, T);
-  else k_fp4_fixup<B, BF16, true><<<fgrid, kThreads, 0, st>>>(P, T);
-  return cudaGetLastError();
+  if (a.mode == 1) k_fp4_search<B, BF16, false><<<gs, kThreads, smem, st>>>(P, T);
+  else k_fp4_search<B, BF16, true><<<gs, kThreads, smem, st>>>(P, T);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.mode == 1) k_fp4_fixup<B, BF16, false><<<gf, kThreads, 0, st>>>(P, T);
+  else k_fp4_fixup<B, BF16, true><<<gf, kThreads, 0, st>>>(P, T);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !a.err_partial) return e;
+  return launch_error_final(a.err_partial, gs + gf, a.err_sums, st);
 }
+
 
 Int8Table make_int8_table() {
   Int8Table t;
@@ -1038,6 +1160,13 @@ cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, 
   if (grid > 4096) grid = 4096;
   k_project<<<(unsigned)grid, kThreads, 0, st>>>(w, count, fmt, scale, rhi, rlo, q);
   return cudaGetLastError();
+}
+
+int fp4_error_parts(int64_t n, int64_t k, int B) {
+  int gs, gf;
+  if (B == 16) fp4_grids<16>(n, k, gs, gf);
+  else fp4_grids<32>(n, k, gs, gf);
+  return gs + gf;
 }
 
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st) {

@@ -39,7 +39,7 @@ EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc
            "mxq_act_gram",
            "mxq_gptq_factor_workspace", "mxq_gptq_factor", "mxq_gptq_order_workspace",
            "mxq_gptq_order", "mxq_gptq_workspace", "mxq_gptq", "mxq_dequant",
-           "mxq_error_workspace",
+           "mxq_error_workspace", "mxq_quantize_err_workspace", "mxq_quantize_err",
            "mxq_error", "mxq_metrics_from_sums", "mxq_status_string", "mxq_last_error")
 
 
@@ -91,6 +91,9 @@ _sig = {
                                 ctypes.POINTER(MxqParams), _P, _P, _P, _SZ, _P]),
     "mxq_dequant": (ctypes.c_int, [_P, _P, ctypes.POINTER(MxqParams), _I64, _I64, _P, _P]),
     "mxq_error_workspace": (_SZ, [_I64, _I64]),
+    "mxq_quantize_err_workspace": (_SZ, [_I64, _I64, ctypes.POINTER(MxqParams)]),
+    "mxq_quantize_err": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, ctypes.POINTER(MxqParams),
+                                        _P, _P, _P, _P, _SZ, _P]),
     "mxq_error": (ctypes.c_int, [_P, _I32, _I64, _I64, _I64, _P, _P, _P,
                                  ctypes.POINTER(MxqParams), _P, _P, _SZ, _P]),
     "mxq_metrics_from_sums": (ctypes.c_int, [_P, ctypes.POINTER(MxqMetrics)]),
@@ -442,6 +445,27 @@ def mxq_error(W: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, p: Mxq
                           ctypes.byref(p), _ptr(sums), _ptr(ws), ws.numel(),
                           _stream(stream, W.device)), "mxq_error")
     return sums
+
+
+def mxq_quantize_err_workspace(n: int, k: int, p: MxqParams) -> int:
+    return int(_lib.mxq_quantize_err_workspace(n, k, ctypes.byref(p)))
+
+
+def mxq_quantize_err(W: torch.Tensor, p: MxqParams, h: torch.Tensor | None = None, *,
+                     codes=None, scales=None, sums=None, workspace=None, stream=None):
+    """mxq_quantize and mxq_error in one call: (codes, scales, device float64 [4] sums)."""
+    n, k = W.shape
+    if codes is None or scales is None:
+        cs, cd, ss, sd = output_shapes(p, n, k)
+        codes = torch.empty(cs, dtype=cd, device=W.device) if codes is None else codes
+        scales = torch.empty(ss, dtype=sd, device=W.device) if scales is None else scales
+    if sums is None:
+        sums = torch.empty(4, dtype=torch.float64, device=W.device)
+    ws = _workspace(mxq_quantize_err_workspace(n, k, p), W.device, workspace)
+    _check(_lib.mxq_quantize_err(_ptr(W), _dtype(W), n, k, _ld(W), _ptr(h), ctypes.byref(p),
+                                 _ptr(codes), _ptr(scales), _ptr(sums), _ptr(ws), ws.numel(),
+                                 _stream(stream, W.device)), "mxq_quantize_err")
+    return codes, scales, sums
 
 
 def mxq_metrics_from_sums(sums) -> dict:

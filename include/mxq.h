@@ -329,6 +329,20 @@ MXQ_API mxq_status mxq_error(const void* W, int32_t dtype, int64_t n, int64_t k,
                      size_t workspace_bytes, void* stream);
 MXQ_API mxq_status mxq_metrics_from_sums(const double* host_sums, mxq_metrics* out);
 
+/* mxq_quantize followed by mxq_error on its result, in one call: codes and scales as
+ * mxq_quantize writes them (identical bytes), sums as mxq_error defines them, h-weighted
+ * with h when h is not NULL (H-optimal uses the same h for the search). The NVFP4 search
+ * with E4M3 scales (mode SSE or H-optimal) adds each block's sums at its winning scale as
+ * it emits the block, so the weights are read once; every other quantizer runs the error
+ * pass after the search. The sums group the blocks differently from mxq_error's, so the two
+ * can differ in the last bits (each is deterministic). workspace:
+ * mxq_quantize_err_workspace(n, k, p) bytes, 8-byte aligned. */
+MXQ_API size_t mxq_quantize_err_workspace(int64_t n, int64_t k, const mxq_params* p);
+MXQ_API mxq_status mxq_quantize_err(const void* W, int32_t dtype, int64_t n, int64_t k,
+                                    int64_t ld, const float* h, const mxq_params* p,
+                                    void* codes, void* scales, double* sums, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------------------
  * Output error of a quantized weight (qwantize "Results": ||X_s Wq^T - X_s W^T||_F /
  * ||X_s W^T||_F on sampled calibration rows X_s), on the tensor cores: both products with

@@ -71,10 +71,10 @@ def test_algorithmic_counts(bench):
     # GPTQ sweep: the search + 6 + (k/2)(1 + 1/B) updates received
     q = bench.Quantizer("nvfp4", 16, "gptq", -1, "e4m3")
     assert bench.sweep_ops_per_weight(q, 9728) == 760 + 6 + 4864 * (1 + 1 / 16)
-    # our launches per GPTQ step on the 9728-wide workload: 818 (ncu's launch list of one
-    # step shows the same count), 822 ordered
-    assert bench.gptq_launches(9728, False) == 818
-    assert bench.gptq_launches(9728, True) == 822
+    # our launches per GPTQ step on the 9728-wide workload: 820, 824 ordered (the Hessian is
+    # three of them: the tensor-core product, the last wave's chunk sums, the transpose)
+    assert bench.gptq_launches(9728, False) == 820
+    assert bench.gptq_launches(9728, True) == 824
     assert bench.code_bytes("nvfp4", 16) == 0.5 + 1 / 16
     assert bench.code_bytes("e4m3", 64) == 1 + 4 / 4096
 

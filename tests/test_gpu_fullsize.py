@@ -285,6 +285,14 @@ def test_error_sums_full_size(mxq, orc, synth, wl_name, wi, fmt, block):
     np.testing.assert_allclose(sums, ref, rtol=1e-5)
     np.testing.assert_allclose(sums0[:2], ref[:2], rtol=1e-5)
     assert sums0[2] == 0 and sums0[3] == 0
+    if fmt == "nvfp4":
+        # the fused call (error sums added inside the search) on the whole weight: every
+        # block's codes and scale equal the oracle's, and the sums agree
+        cf, sf, sumsf = mxq.mxq_quantize_err(W, p, hd)
+        torch.cuda.synchronize()
+        assert np.array_equal(sf.cpu().numpy(), r.scales)
+        assert np.array_equal(cf.cpu().numpy(), r.codes)
+        np.testing.assert_allclose(sumsf.cpu().numpy(), ref, rtol=1e-5)
     m, mo = mxq.mxq_metrics_from_sums(sums), orc.metrics(ref)
     assert m["weight_rel"] == pytest.approx(mo["weight_rel"], rel=1e-5)
     assert m["h_rel"] == pytest.approx(mo["h_rel"], rel=1e-5)

@@ -299,6 +299,38 @@ def test_dequant_and_error_parity(mxq, orc, synth, fmt, block, mode):
     np.testing.assert_allclose(sums0[:2], rs[:2], rtol=1e-5)
 
 
+@pytest.mark.parametrize("fmt,block,mode,with_h", [("nvfp4", 16, "hopt", True),
+                                                   ("nvfp4", 32, "hopt", True),
+                                                   ("nvfp4", 16, "sse", True),
+                                                   ("nvfp4", 32, "sse", False),
+                                                   ("nvfp4", 16, "naive", True),
+                                                   ("int8", 64, "hopt", True),
+                                                   ("e4m3", 64, "hopt", True)])
+def test_quantize_with_error_sums(mxq, orc, synth, fmt, block, mode, with_h):
+    """mxq_quantize_err: the same codes and scales as mxq_quantize, bit for bit, and the
+    error sums of the oracle's quantization (equal to the GPU's, checked first) at 1e-5; the
+    NVFP4 searches add the sums inside the search (ragged row count: 77 rows)."""
+    n, k = (128, 512) if fmt == "e4m3" else (77, 1024)
+    W = synth.gaussian_weight(n, k, 81, dtype=torch.bfloat16, device=DEV)
+    X = synth.activations(256, k, 82, dtype=torch.bfloat16, device="cpu")
+    h = orc.act_sqmean(oracle_view(X))
+    hd = torch.from_numpy(h).to(DEV) if with_h else None
+    p = mxq.params(fmt, mode, block)
+    c1, s1 = mxq.mxq_quantize(W, p, hd)
+    c2, s2, sums = mxq.mxq_quantize_err(W, p, hd)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2) and torch.equal(s1, s2)
+    r = orc.quantize(oracle_view(W), fmt, mode, block, h=h if mode == "hopt" else None)
+    if fmt != "e4m3":              # (tiles are bit-exact outside near ties: tested elsewhere)
+        assert np.array_equal(c2.cpu().numpy().view(np.uint8), r.codes.view(np.uint8))
+        assert np.array_equal(s2.cpu().numpy(), r.scales)
+    What = orc.dequant(r.codes, r.scales, fmt, block, n, k)
+    ref = orc.error_sums(oracle_view(W), What, h if with_h else None)
+    np.testing.assert_allclose(sums.cpu().numpy(), ref, rtol=1e-5, atol=0)
+    again = mxq.mxq_quantize_err(W, p, hd)[2]
+    assert torch.equal(sums, again)                     # deterministic
+
+
 def test_error_deterministic(mxq, synth):
     W = synth.gaussian_weight(512, 4096, 61, dtype=torch.bfloat16, device=DEV)
     p = mxq.params("nvfp4", "naive", 16)
