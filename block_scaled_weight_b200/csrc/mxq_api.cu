@@ -5,6 +5,7 @@
 #include "mxq_internal.h"
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -19,6 +20,15 @@ int sm_count() {
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
+}
+
+namespace {
+std::atomic<uint32_t> g_wait_polls{0};
+}
+
+uint32_t wait_polls() {
+  const uint32_t p = g_wait_polls.load(std::memory_order_relaxed);
+  return p ? p : (1u << 26);
 }
 
 cudaError_t ensure_dynamic_smem(const void* func, int bytes) {
@@ -146,6 +156,8 @@ const char* mxq_status_string(mxq_status s) {
 }
 
 const char* mxq_last_error(void) { return g_err; }
+
+void mxq_set_wait_polls(uint32_t polls) { mxq::g_wait_polls.store(polls, std::memory_order_relaxed); }
 
 size_t mxq_act_sqmean_workspace(int64_t rows, int64_t cols) {
   if (rows <= 0 || cols <= 0) return 0;

@@ -69,10 +69,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity; false on timeout or abort.
+// Bounded wait for the phase with the given parity (at most `polls` polls); false on
+// timeout or abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag) {
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+                                          volatile int* abort_flag, uint32_t polls) {
+  for (uint32_t it = 0; it < polls; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 1023u) == 1023u && *abort_flag) return false;
   }
@@ -151,6 +152,7 @@ struct GramParams {
   int64_t rows_per_chunk;  // a multiple of kGramRows: chunk boundaries fall on stage edges
   double* partial;         // [chunks][cols][B]: column c's row of its diagonal block
   int* err;
+  uint32_t polls;          // bound of every pipeline wait (the drains keep kSpinLimit)
 };
 
 // Shared-memory layout (dynamic, 1024-byte aligned for the swizzle atoms).
@@ -219,7 +221,7 @@ k_gram_tc(const __grid_constant__ CUtensorMap tmap, GramParams P) {
       for (int it = 0; it < nst; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { fail(); break; }
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, P.polls)) { fail(); break; }
         mbar_expect_tx(&full[s], kStageBytes);
         const int y = (int)(row_begin + (int64_t)it * kGramRows);
         uint8_t* dst = smem + s * kStageBytes;
@@ -230,7 +232,7 @@ k_gram_tc(const __grid_constant__ CUtensorMap tmap, GramParams P) {
       // every copy this thread started has landed before the CTA can exit
 #pragma unroll
       for (int s = 0; s < kStages; ++s)
-        if (issued[s] > 0 && !mbar_wait(&full[s], (uint32_t)(issued[s] - 1) & 1u, abort_flag)) {
+        if (issued[s] > 0 && !mbar_wait(&full[s], (uint32_t)(issued[s] - 1) & 1u, abort_flag, P.polls)) {
           for (uint32_t it = 0; it < kSpinLimit && !mbar_try_wait(&full[s], (uint32_t)(issued[s] - 1) & 1u); ++it) {
           }
         }
@@ -241,7 +243,7 @@ k_gram_tc(const __grid_constant__ CUtensorMap tmap, GramParams P) {
       int it = 0;
       for (int per = 0; per < nper; ++per) {
         const int buf = per & 1;
-        if (!mbar_wait(&accempty[buf], ((uint32_t)(per >> 1) & 1u) ^ 1u, abort_flag)) {
+        if (!mbar_wait(&accempty[buf], ((uint32_t)(per >> 1) & 1u) ^ 1u, abort_flag, P.polls)) {
           fail();
           break;
         }
@@ -251,7 +253,7 @@ k_gram_tc(const __grid_constant__ CUtensorMap tmap, GramParams P) {
         bool ok = true;
         for (; it < end; ++it) {
           const int s = it % kStages;
-          if (!mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, abort_flag, P.polls)) { ok = false; break; }
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
           const uint32_t base = smem_u32(smem + s * kStageBytes);
 #pragma unroll
@@ -278,7 +280,7 @@ k_gram_tc(const __grid_constant__ CUtensorMap tmap, GramParams P) {
     const bool upper = B == 16 && lane >= 16;  // B = 16: lanes 16-31 own the second block
     for (int per = 0; per < nper; ++per) {
       const int buf = per & 1;
-      const bool ok = mbar_wait(&accfull[buf], (uint32_t)(per >> 1) & 1u, abort_flag);
+      const bool ok = mbar_wait(&accfull[buf], (uint32_t)(per >> 1) & 1u, abort_flag, P.polls);
       if (!__all_sync(kFull, ok)) {
         if (lane == 0) fail();
         break;
@@ -396,7 +398,7 @@ cudaError_t launch_gram(const void* X, int64_t rows, int64_t cols, int64_t ld, i
   double* partial = (double*)((char*)workspace + 256);
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
-  GramParams P{rows, cols, per_chunk, partial, err};
+  GramParams P{rows, cols, per_chunk, partial, err, wait_polls()};
   const dim3 grid((unsigned)((cols + kGramCols - 1) / kGramCols), (unsigned)chunks);
   if (B == 16) {
     e = ensure_dynamic_smem((const void*)k_gram_tc<16>, (int)kGramSmem);

@@ -188,12 +188,6 @@ k_gram_full(const __grid_constant__ CUtensorMap tmap, GfParams P) {
           tc::tma_load_2d_pair(dst + kGfA + kGfB + kGfBox, &tmap, xb1 + 64, y, bar);
         }
       }
-      // Copies complete on the even CTA's barriers, which this thread cannot watch. On the
-      // normal path every copy was consumed by an MMA that the accumulator hand-off waited
-      // for; after an abort, give copies still in flight time to land before the shared
-      // memory can be released (a copy takes microseconds).
-      if (aborted)
-        for (int i = 0; i < 1000; ++i) __nanosleep(1000);
     }
   } else if (warp == 5) {
     // ---- MMA issuer (even CTA) ---------------------------------------------------------
@@ -286,6 +280,16 @@ k_gram_full(const __grid_constant__ CUtensorMap tmap, GfParams P) {
     }
   }
   __syncthreads();
+  // Copies complete on the even CTA's barriers, which the odd CTA cannot watch. On the normal
+  // path every copy was consumed by an MMA that the accumulator hand-off waited for; after
+  // an abort (either CTA sets both flags), give copies still in flight time to land before
+  // shared memory can be released: a copy takes microseconds, this waits about a
+  // millisecond, and the cluster barrier keeps the other CTA until then too.
+  if (*abort_flag) {
+    if (threadIdx.x == 0)
+      for (int i = 0; i < 1000; ++i) __nanosleep(1000);
+    __syncthreads();
+  }
   tc::cluster_sync();       // neither CTA leaves while the other may still signal it
   if (warp == 5) {
     tc::fence_after_sync();
@@ -399,7 +403,7 @@ cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t 
   if (e != cudaSuccess) return e;
   e = ensure_dynamic_smem((const void*)k_gram_full, kGfSmem);
   if (e != cudaSuccess) return e;
-  GfParams p{S, H, partial, err, tc::kDefaultPolls, 1.0 / (double)rows};
+  GfParams p{S, H, partial, err, wait_polls(), 1.0 / (double)rows};
   k_gram_full<<<2 * S.pairs, kGfThreads, kGfSmem, st>>>(map, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

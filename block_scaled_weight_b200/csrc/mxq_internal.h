@@ -127,6 +127,9 @@ cudaError_t launch_gram_full(const void* X, int64_t rows, int64_t cols, int64_t 
                              void* workspace, cudaStream_t st, const char** why);
 
 int sm_count();
+// Bound (in polls) of every pipeline wait of the tensor-core kernels: 2^26 unless a caller
+// lowered it with mxq_set_wait_polls (to exercise the timeout path).
+uint32_t wait_polls();
 // Raises func's dynamic shared-memory limit to `bytes` on the current device, once per
 // (device, kernel): the attribute is per device, so each GPU a process uses needs its own.
 cudaError_t ensure_dynamic_smem(const void* func, int bytes);

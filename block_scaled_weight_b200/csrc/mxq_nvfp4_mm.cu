@@ -209,7 +209,7 @@ cudaError_t launch_nvfp4_mm(const uint8_t* a_codes, const uint8_t* a_sf, const u
   if (e != cudaSuccess) return e;
   e = ensure_dynamic_smem((const void*)k_nvfp4_mm, kMmSmem);
   if (e != cudaSuccess) return e;
-  MmParams P{m, n, k, a_sf, b_sf, (k + 63) / 64, D, err, tc::kDefaultPolls};
+  MmParams P{m, n, k, a_sf, b_sf, (k + 63) / 64, D, err, wait_polls()};
   const dim3 grid((unsigned)((n + kMmN - 1) / kMmN), (unsigned)((m + kMmM - 1) / kMmM));
   k_nvfp4_mm<<<grid, kMmThreads, kMmSmem, st>>>(amap, bmap, P);
   e = cudaGetLastError();

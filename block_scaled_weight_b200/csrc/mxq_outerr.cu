@@ -54,8 +54,9 @@ __device__ __forceinline__ bool bar_try(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
-  for (uint32_t it = 0; it < kOeSpin; ++it) {
+__device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                         uint32_t polls) {
+  for (uint32_t it = 0; it < polls; ++it) {
     if (bar_try(b, parity)) return true;
     if ((it & 1023u) == 1023u && *abort_flag) return false;
   }
@@ -122,6 +123,7 @@ struct OeParams {
   int int4;                // 0: E2M1 nibbles, 1: two's-complement INT4 nibbles
   double* partial;         // [ctas][2]
   int* err;
+  uint32_t polls;          // bound of every pipeline wait (the drains keep kOeSpin)
 };
 
 struct OeScaleTab {
@@ -201,7 +203,7 @@ k_outerr_tc(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CU
       for (int s = 0; s < kOeStages; ++s) issued[s] = 0;
       for (int it = 0; it < nk; ++it) {
         const int s = it % kOeStages;
-        if (!bar_wait(&empty[s], ((uint32_t)(it / kOeStages) & 1u) ^ 1u, abort_flag)) { fail(); break; }
+        if (!bar_wait(&empty[s], ((uint32_t)(it / kOeStages) & 1u) ^ 1u, abort_flag, P.polls)) { fail(); break; }
         bar_expect(&full[s], kOeXBytes + kOeWBytes);
         uint8_t* st = smem + s * kOeStageBytes;
         tma2d(st, &xmap, it * kOeK, (int)m0, &full[s]);
@@ -222,7 +224,7 @@ k_outerr_tc(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CU
       for (int it = 0; it < nk && ok; ++it) {
         const int s = it % kOeStages;
         const uint32_t ph = (uint32_t)(it / kOeStages) & 1u;
-        ok = bar_wait(&full[s], ph, abort_flag) && bar_wait(&qfull[s], ph, abort_flag);
+        ok = bar_wait(&full[s], ph, abort_flag, P.polls) && bar_wait(&qfull[s], ph, abort_flag, P.polls);
         if (!ok) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t xs = s_u32(smem + s * kOeStageBytes);
@@ -272,7 +274,7 @@ k_outerr_tc(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CU
     for (int it = 0; it < nk; ++it) {
       const int s = it % kOeStages;
       fetch(it + 1, cwn, scn);
-      ok = bar_wait(&empty[s], ((uint32_t)(it / kOeStages) & 1u) ^ 1u, abort_flag);
+      ok = bar_wait(&empty[s], ((uint32_t)(it / kOeStages) & 1u) ^ 1u, abort_flag, P.polls);
       if (!__all_sync(kFull, ok)) { ok = false; break; }
       uint32_t wd[16];
 #pragma unroll
@@ -307,7 +309,7 @@ k_outerr_tc(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CU
     if (!ok && lane == 0) fail();
     // epilogue: this warp's tensor-memory lanes 32 (warp % 4) ..
     double sdd = 0.0, syy = 0.0;
-    const bool got = __all_sync(kFull, ok && bar_wait(accfull, 0, abort_flag));
+    const bool got = __all_sync(kFull, ok && bar_wait(accfull, 0, abort_flag, P.polls));
     if (got) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
@@ -423,7 +425,7 @@ cudaError_t launch_outerr(const void* X, int64_t m, int64_t k, int64_t ldx, cons
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((m + kOeM - 1) / kOeM), (unsigned)((n + kOeN - 1) / kOeN));
-  OeParams P{m, n, k, codes, scales, block, fmt == 3 ? 1 : 0, partial, err};
+  OeParams P{m, n, k, codes, scales, block, fmt == 3 ? 1 : 0, partial, err, wait_polls()};
   e = ensure_dynamic_smem((const void*)k_outerr_tc, (int)kOeSmem);
   if (e != cudaSuccess) return e;
   k_outerr_tc<<<grid, kOeThreads, kOeSmem, st>>>(xmap, wmap, P, T);

@@ -40,7 +40,8 @@ EXPORTS = ("mxq_act_sqmean_workspace", "mxq_act_sqmean", "mxq_act_sqmean_noalloc
            "mxq_gptq_factor_workspace", "mxq_gptq_factor", "mxq_gptq_order_workspace",
            "mxq_gptq_order", "mxq_gptq_workspace", "mxq_gptq", "mxq_dequant",
            "mxq_error_workspace", "mxq_quantize_err_workspace", "mxq_quantize_err",
-           "mxq_error", "mxq_metrics_from_sums", "mxq_status_string", "mxq_last_error")
+           "mxq_error", "mxq_metrics_from_sums", "mxq_status_string", "mxq_last_error",
+           "mxq_set_wait_polls")
 
 
 class MxqParams(ctypes.Structure):
@@ -99,6 +100,7 @@ _sig = {
     "mxq_metrics_from_sums": (ctypes.c_int, [_P, ctypes.POINTER(MxqMetrics)]),
     "mxq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mxq_last_error": (ctypes.c_char_p, []),
+    "mxq_set_wait_polls": (None, [ctypes.c_uint32]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -475,3 +477,8 @@ def mxq_metrics_from_sums(sums) -> dict:
     _check(_lib.mxq_metrics_from_sums(ctypes.cast(arr, ctypes.c_void_p), ctypes.byref(m)),
            "mxq_metrics_from_sums")
     return {name: getattr(m, name) for name, _ in MxqMetrics._fields_}
+
+
+def mxq_set_wait_polls(polls: int) -> None:
+    """Bound of the tensor-core kernels' pipeline waits for later launches (0: the default)."""
+    _lib.mxq_set_wait_polls(int(polls))

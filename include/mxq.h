@@ -477,6 +477,15 @@ MXQ_API mxq_status mxq_gptq(const void* W, int32_t dtype, int64_t n, int64_t k, 
                             const mxq_params* p, void* codes, void* scales, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* The tensor-core kernels (mxq_act_block_gram, mxq_act_gram, mxq_output_error,
+ * mxq_nvfp4_gemm) bound every wait of their pipelines (a poll of an mbarrier); a wait that
+ * runs out sets an error word, the kernel lets its copies and MMAs finish and frees its
+ * tensor memory, and the call's outputs become NaN. mxq_set_wait_polls sets that bound for
+ * the launches that follow, process-wide (0 restores the default, 2^26 polls: seconds). A
+ * small bound makes the waits run out on purpose, to test that path; the library stays
+ * usable afterwards. No page counterpart: this is the library's own failure handling. */
+MXQ_API void mxq_set_wait_polls(uint32_t polls);
+
 /* Human-readable text for a status; the last failure's detail on this host thread. */
 MXQ_API const char* mxq_status_string(mxq_status s);
 MXQ_API const char* mxq_last_error(void);
