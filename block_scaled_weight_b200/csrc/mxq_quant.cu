@@ -183,16 +183,17 @@ __device__ __forceinline__ float fp4_lb(float2 at, float2 ct, float2 x, uint32_t
 
 // NVFP4, SSE / H-optimal search, compacted. A warp owns 32 blocks: one column block jb
 // (so h is the same for every lane and stays in registers) in 32 consecutive rows, one block
-// per lane. Every lane first scores, in full, its naive code and the codes on either side
-// (the winner is usually within a few codes of the naive snap), then filters the rest of its
-// range with exact lower bounds, writing the codes that survive into its own list in shared
-// memory. The warp then scores the surviving (block, code) pairs 32 at a time -- every lane
+// per lane. Every lane first scores, in full and in step with the other lanes, a window of
+// codes around its naive code (naive - 1 .. naive + 5: the winner is usually there), then
+// filters the codes the range cuts leave outside the window with exact lower bounds, writing
+// the codes that survive into its own list in shared memory. The warp then scores the surviving (block, code) pairs 32 at a time -- every lane
 // takes the next pair, whoever's block it is, reading that block's magnitudes from shared
 // memory -- and each lane folds its own results back in code order. Blocks whose float32
 // winner is not separated from the runner-up by the error bound are flagged (bit 7 of the
 // scale byte) for k_fp4_fixup. With P.err_partial set, the kernel also adds each unflagged
 // block's error sums at its winning scale (float32 over the block, double beyond) into
 // per-CTA partials.
+constexpr int kFp4WinLo = -1, kFp4WinHi = 5;   // codes every lane scores in full
 constexpr int kFp4Queue = 128;       // scored pairs held per warp before the owners fold them
 constexpr int kFp4List = 132;        // bytes per lane's code list (126 codes; rows offset by a bank)
 
@@ -298,10 +299,10 @@ k_fp4_search(Fp4Params P, Fp4Table T) {
     if (!valid) hi = 0;                                // no candidates
     float m1 = __int_as_float(0x7f800000), m2 = m1;
     int i1 = lo;
-    // the naive code (clipped to the candidate range) and its two neighbours, in full
+    // a window of codes around the naive code (clipped to the candidate range), in full
     const int cs = min(max(c0, lo), max(hi, lo));
-#pragma unroll 1
-    for (int d = -1; d <= 1; ++d) {
+#pragma unroll
+    for (int d = kFp4WinLo; d <= kFp4WinHi; ++d) {
       const int cc = cs + d;
       if (cc >= lo && cc <= hi) track(fp4_eval<B, HOPT>(a, c, tab[cc]), cc, m1, m2, i1);
     }
@@ -355,15 +356,23 @@ k_fp4_search(Fp4Params P, Fp4Table T) {
         if (!(e4m3_pos(ch) < s_hi)) --ch;               // largest code with value < s_hi
         hi2 = min(hi2, ch);
       }
-      for (int cc = lo2; cc <= hi2; ++cc) {
-        if (cc >= cs - 1 && cc <= cs + 1) continue;    // scored above
-        const float4 t = tab[cc];
-        const float2 rhi = make_float2(t.y, t.y), rlo = make_float2(t.z, t.z);
-        if (fp4_lb(at, ct, fp4_quot(at, rhi, rlo), __float_as_uint(t.w) ^ 0x8000u) * lb_f -
-                slack > upper)
-          continue;
-        my_list[cnt++] = (uint8_t)cc;
-      }
+      // the codes the cuts leave below and above the window, two at a time (independent)
+      auto bound_range = [&](int c_lo, int c_hi) {
+        for (int cc = c_lo; cc <= c_hi; cc += 2) {
+          const int cd = min(cc + 1, c_hi);
+          const float4 t0 = tab[cc], t1 = tab[cd];
+          const float l0 = fp4_lb(at, ct, fp4_quot(at, make_float2(t0.y, t0.y),
+                                                   make_float2(t0.z, t0.z)),
+                                  __float_as_uint(t0.w) ^ 0x8000u);
+          const float l1 = fp4_lb(at, ct, fp4_quot(at, make_float2(t1.y, t1.y),
+                                                   make_float2(t1.z, t1.z)),
+                                  __float_as_uint(t1.w) ^ 0x8000u);
+          if (!(l0 * lb_f - slack > upper)) my_list[cnt++] = (uint8_t)cc;
+          if (cd > cc && !(l1 * lb_f - slack > upper)) my_list[cnt++] = (uint8_t)cd;
+        }
+      };
+      bound_range(lo2, min(hi2, cs + kFp4WinLo - 1));
+      bound_range(max(lo2, cs + kFp4WinHi + 1), hi2);
     }
     // the block's magnitudes for the lanes that score its pairs
 #pragma unroll
