@@ -23,8 +23,8 @@
 //
 // Warp roles (192 threads per CTA): warps 0-3 drain the accumulators (tensor-memory lanes
 // 32 w .. 32 w + 31 = H rows) and store H; warp 4 issues the TMA copies; warp 5 issues the
-// MMAs (even CTA) and owns the tensor-memory allocation (both CTAs). No TMA load uses
-// cluster multicast; operands come from this GPU's memory only. Every wait is bounded: on
+// MMAs (even CTA) and owns the tensor-memory allocation (both CTAs). Each CTA loads only
+// its own tiles, into its own shared memory, from this GPU's memory. Every wait is bounded: on
 // timeout a CTA sets the error word and its peer's abort flag, and the final transpose then
 // writes NaN over all of H.
 #include "mxq_common.cuh"

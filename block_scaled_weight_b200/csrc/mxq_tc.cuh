@@ -2,7 +2,7 @@
 // waits), thread-block-cluster addressing, 2-D TMA tile loads, tcgen05 MMA / commit /
 // tensor-memory allocation and loads, and the shared-memory operand descriptor of a
 // 128-byte-swizzled MN-major bf16 tile. Each is one PTX instruction (or a bounded loop of
-// one); no TMA load here uses cluster multicast.
+// one); every TMA load here fills only the issuing CTA's shared memory.
 #pragma once
 
 #include <cstdint>
