@@ -475,6 +475,10 @@ def gpu_arm(args):
     if gram and world > 1:
         raise SystemExit(f"--mode {mode} runs on one GPU")
     p = mxq.params(fmt, "hopt" if gram else mode, block, window=window, scale_fmt=q.sfmt)
+    # for the overlapped steps below, when the h pass is long enough to hide it: the search
+    # holds one CTA per SM, leaving the other SM slots to the next batch's h pass beside it
+    p_overlap = mxq.params(fmt, "hopt" if gram else mode, block, window=window,
+                           scale_fmt=q.sfmt, ctas_per_sm=1)
     # inputs: every rank draws its own shard (weak scaling)
     wl_r = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
     # activations and their h, one per activation width
@@ -497,7 +501,8 @@ def gpu_arm(args):
     for wi, (_, n, k) in enumerate(wl.weights):
         Ws.append(synth.workload_weight(wl_r, wi, device=dev))
         cs, cd, ss, sd = mxq.output_shapes(p, n, k)
-        ews = max(mxq.mxq_error_workspace(n, k), mxq.mxq_quantize_err_workspace(n, k, p))
+        ews = max(mxq.mxq_error_workspace(n, k), mxq.mxq_quantize_err_workspace(n, k, p),
+                  mxq.mxq_quantize_err_workspace(n, k, p_overlap))
         outs.append((torch.empty(cs, dtype=cd, device=dev), torch.empty(ss, dtype=sd, device=dev),
                      torch.empty(4, dtype=torch.float64, device=dev),
                      torch.empty(ews, dtype=torch.uint8, device=dev),
@@ -615,6 +620,9 @@ def gpu_arm(args):
     # pass (another stream; h in two alternating buffers). The h pass is HBM-bound, the search
     # ALU-bound. Every step still does all of its work; only consecutive steps overlap.
     pipelined = world == 1 and not gram and flush is None and not args.serial
+    # a search held to one CTA per SM runs about 1.7 x longer alone: worth it only when the
+    # h pass it runs beside is longer still
+    p_pipe = p_overlap if k_h >= 1.8 * k_q else p
     if pipelined:
         # the search stream at the higher priority: its CTAs take SM slots first as the h
         # pass's free up
@@ -635,8 +643,8 @@ def gpu_arm(args):
                 s_q.wait_event(ev_h[b])
                 for W, (codes, scales, sums, ews, xi) in zip(Ws, outs):
                     if fused:
-                        mxq.mxq_quantize_err(W, p, hb[b][xi], codes=codes, scales=scales,
-                                             sums=sums, workspace=ews)
+                        mxq.mxq_quantize_err(W, p_pipe, hb[b][xi], codes=codes,
+                                             scales=scales, sums=sums, workspace=ews)
                     else:
                         mxq.mxq_quantize(W, p, hb[b][xi], codes=codes, scales=scales)
                         mxq.mxq_error(W, codes, scales, p, hb[b][xi], sums=sums, workspace=ews)
@@ -771,8 +779,11 @@ def gpu_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "ms_per_step_serial": ms_step_serial,
             "pipelined": ("step i's search and error sums overlap step i+1's h pass (two "
-                          "streams, h double-buffered); kernel times below are from the "
-                          "serial timed region") if pipelined else None,
+                          "streams, h double-buffered; search occupancy: "
+                          + ("one CTA per SM beside the h pass's two, mxq_params.ctas_per_sm "
+                             "= 1" if p_pipe is p_overlap else "all SM slots") +
+                          "); kernel times below are from the serial timed region")
+            if pipelined else None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": workload_desc(wl, q, [X.shape[0] for X in Xs]),

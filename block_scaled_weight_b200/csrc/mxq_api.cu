@@ -88,6 +88,7 @@ mxq_status check_matrix(const void* X, int32_t dt, int64_t rows, int64_t cols, i
 mxq_status check_params(const mxq_params* p, int64_t n, int64_t k) {
   if (!p) return fail(MXQ_ERR_INVALID_ARG, "params is NULL");
   if (p->mode < MXQ_NAIVE || p->mode > MXQ_HOPT) return fail(MXQ_ERR_INVALID_ARG, "mode %d", p->mode);
+  if (p->ctas_per_sm < 0) return fail(MXQ_ERR_INVALID_ARG, "ctas_per_sm %d", p->ctas_per_sm);
   switch (p->fmt) {
     case MXQ_FMT_NVFP4:
     case MXQ_FMT_INT4:
@@ -297,6 +298,7 @@ static mxq_status prepare_quantize(const void* W, int32_t dtype, int64_t n, int6
   a->block = p->block;
   a->window = p->window;
   a->scale_fmt = p->scale_fmt;
+  a->ctas_per_sm = p->ctas_per_sm;
   a->codes = codes;
   a->scales = scales;
   a->log_points = p->fmt == MXQ_FMT_E4M3 && p->mode != MXQ_NAIVE ? p->log_points : 0;
@@ -325,7 +327,7 @@ static bool fused_error(const mxq_params* p) {
 size_t mxq_quantize_err_workspace(int64_t n, int64_t k, const mxq_params* p) {
   if (n <= 0 || k <= 0 || !p) return 0;
   const int64_t parts = fused_error(p) && (p->block == 16 || p->block == 32)
-                            ? mxq::fp4_error_parts(n, k, p->block)
+                            ? mxq::fp4_error_parts(n, k, p->block, p->ctas_per_sm)
                             : mxq::error_partials(n, k);
   return (size_t)parts * 4 * sizeof(double);
 }

@@ -14,8 +14,10 @@ namespace mxq {
 constexpr int kHpassThreads = 256;
 // Resident 256-thread CTAs per SM and the one-wave target grid on a 148-SM B200; strips x
 // chunks never exceeds kHpassTargetCtas, so the workspace is at most
-// max(kHpassTargetCtas x 256, cols) doubles.
-constexpr int kHpassCtasPerSm = 3;
+// max(kHpassTargetCtas x 256, cols) doubles. Two of the three register-bound slots of an SM:
+// the third stays free for a search CTA of the previous batch running beside the h pass
+// (3 per SM streamed 3 % faster alone, but left no room).
+constexpr int kHpassCtasPerSm = 2;
 constexpr int kHpassTargetCtas = 148 * kHpassCtasPerSm;
 int hpass_chunks(int64_t rows, int64_t cols, int dtype);
 cudaError_t launch_hpass_partial(const void* X, int dtype, int64_t rows, int64_t cols,
@@ -50,10 +52,11 @@ struct QuantArgs {
   double* err_partial = nullptr;
   double* err_sums = nullptr;
   const float* h_err = nullptr;
+  int ctas_per_sm = 0;  // NVFP4 search: CTAs per SM of its persistent grid (0: all that fit)
 };
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 // Partial slots the fused error sums of an NVFP4 search need (search CTAs + exact-pass CTAs).
-int fp4_error_parts(int64_t n, int64_t k, int B);
+int fp4_error_parts(int64_t n, int64_t k, int B, int ctas_per_sm);
 // E2M1 on a scale grid other than E4M3, and INT4 on any grid (mxq_quant_grid.cu).
 cudaError_t launch_quantize_grid(const QuantArgs& a, cudaStream_t st);
 // Block-Hessian search (d^T G_b d) for E2M1 / INT4 elements on any scale grid.

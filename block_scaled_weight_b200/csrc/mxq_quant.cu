@@ -1056,9 +1056,10 @@ int grid_for(int64_t work_threads) {
 // Grids of the NVFP4 search and its exact pass (fixed by the shape and the device's SM
 // count, so the order of the fused error sums is too).
 template <int B>
-void fp4_grids(int64_t n, int64_t k, int& gs, int& gf) {
+void fp4_grids(int64_t n, int64_t k, int ctas_per_sm, int& gs, int& gf) {
   const int64_t ntiles = (n + 31) / 32 * (k / B);
-  const int64_t cap = (int64_t)sm_count() * (B == 16 ? 3 : 2);
+  const int fit = B == 16 ? 3 : 2;                 // resident CTAs per SM (registers)
+  const int64_t cap = (int64_t)sm_count() * (ctas_per_sm > 0 && ctas_per_sm < fit ? ctas_per_sm : fit);
   const int64_t want = (ntiles + kThreads / 32 - 1) / (kThreads / 32);
   gs = (int)(want < 1 ? 1 : (want > cap ? cap : want));
   const int64_t fwant = (n * (k / B) + 32 * 8 - 1) / (32 * 8);   // one 32-block tile per warp
@@ -1076,7 +1077,7 @@ cudaError_t fp4_dispatch(const QuantArgs& a, cudaStream_t st) {
     return cudaGetLastError();
   }
   int gs, gf;
-  fp4_grids<B>(a.n, a.k, gs, gf);
+  fp4_grids<B>(a.n, a.k, a.ctas_per_sm, gs, gf);
   P.fix_slot0 = gs;
   const size_t smem = fp4_search_smem<B>();
   const void* kern = a.mode == 1 ? (const void*)k_fp4_search<B, BF16, false>
@@ -1171,10 +1172,10 @@ cudaError_t launch_project(const float* w, int64_t count, int fmt, float scale, 
   return cudaGetLastError();
 }
 
-int fp4_error_parts(int64_t n, int64_t k, int B) {
+int fp4_error_parts(int64_t n, int64_t k, int B, int ctas_per_sm) {
   int gs, gf;
-  if (B == 16) fp4_grids<16>(n, k, gs, gf);
-  else fp4_grids<32>(n, k, gs, gf);
+  if (B == 16) fp4_grids<16>(n, k, ctas_per_sm, gs, gf);
+  else fp4_grids<32>(n, k, ctas_per_sm, gs, gf);
   return gs + gf;
 }
 

@@ -48,7 +48,8 @@ class MxqParams(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("mode", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("tile_rows", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("log_points", ctypes.c_int32), ("log_lo_exp2", ctypes.c_float),
-                ("log_hi_exp2", ctypes.c_float), ("scale_fmt", ctypes.c_int32)]
+                ("log_hi_exp2", ctypes.c_float), ("scale_fmt", ctypes.c_int32),
+                ("ctas_per_sm", ctypes.c_int32)]
 
 
 class MxqMetrics(ctypes.Structure):
@@ -125,13 +126,14 @@ def lib_path() -> str:
 
 
 def params(fmt="nvfp4", mode="hopt", block=16, *, window=-1, tile_rows=None, log_points=64,
-           log_lo_exp2=-2.0, log_hi_exp2=2.0, scale_fmt="e4m3") -> MxqParams:
+           log_lo_exp2=-2.0, log_hi_exp2=2.0, scale_fmt="e4m3", ctas_per_sm=0) -> MxqParams:
     f = FMT[fmt] if isinstance(fmt, str) else int(fmt)
     sf = SCALE[scale_fmt] if isinstance(scale_fmt, str) else int(scale_fmt)
     m = MODE[mode] if isinstance(mode, str) else int(mode)
     if tile_rows is None:
         tile_rows = block if f == FMT["e4m3"] else 1
-    return MxqParams(f, m, block, tile_rows, window, log_points, log_lo_exp2, log_hi_exp2, sf)
+    return MxqParams(f, m, block, tile_rows, window, log_points, log_lo_exp2, log_hi_exp2, sf,
+                     ctas_per_sm)
 
 
 def _ptr(t):

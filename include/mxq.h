@@ -112,6 +112,12 @@ typedef enum { MXQ_SCALE_E4M3 = 0, MXQ_SCALE_UE4M4 = 1, MXQ_SCALE_UE5M3 = 2,
  *             Naive scale: UE8M0 2^(floor(log2 amax) - 2) (the OCP rule, 2 = the largest
  *             E2M1 exponent), clamped to codes 0..254 (0 for amax = 0); every other grid
  *             its nearest value (RNE, saturating) to fl32(amax / qmax).
+ *  ctas_per_sm  how many CTAs per SM the NVFP4 (E4M3-scale) search may occupy: 0 = as many
+ *             as fit (fastest alone); 1 leaves room beside it for a streaming kernel on
+ *             another stream, e.g. the next batch's h pass, which then overlaps the search.
+ *             Results are the same for every value (the fused error sums of
+ *             mxq_quantize_err group blocks by CTA, so they can differ in the last bits).
+ *             Other quantizers ignore it.
  */
 typedef struct mxq_params {
     int32_t fmt;
@@ -123,6 +129,7 @@ typedef struct mxq_params {
     float log_lo_exp2;
     float log_hi_exp2;
     int32_t scale_fmt;
+    int32_t ctas_per_sm;
 } mxq_params;
 
 /* Weight error metrics from the four sums that mxq_error produces. */

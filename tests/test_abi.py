@@ -89,6 +89,7 @@ def test_quantize_rejections(mxq):
     assert q(mxq, fmt="e4m3", mode="hopt", block=64, log_points=1) == S["MXQ_ERR_INVALID_ARG"]
     assert q(mxq, fmt="e4m3", mode="hopt", block=64, log_lo_exp2=3.0) == S["MXQ_ERR_INVALID_ARG"]
     assert q(mxq, fmt="nvfp4", mode="sse", block=16, window=-2) == S["MXQ_ERR_INVALID_ARG"]
+    assert q(mxq, fmt="nvfp4", mode="sse", block=16, ctas_per_sm=-1) == S["MXQ_ERR_INVALID_ARG"]
     assert q(mxq, fmt="int4", mode="sse", block=64) == S["MXQ_ERR_UNSUPPORTED"]
     assert q(mxq, fmt="int4", mode="sse", block=16, scale_fmt="ue8m0") == S["MXQ_ERR_UNSUPPORTED"]
     assert q(mxq, fmt="nvfp4", mode="sse", block=16, scale_fmt=7) == S["MXQ_ERR_INVALID_ARG"]
