@@ -8,7 +8,7 @@
 //           float32 once. With J the order reversal, J H J = L L^T gives H^-1 = U^T U with
 //           U = J L^-1 J, so one blocked Cholesky and one blocked triangular inverse (64 x 64
 //           tiles, float64 products on the tensor cores) replace GPTQ's
-//           inverse-then-Cholesky.
+//           inverse-then-Cholesky; the inverse follows the Cholesky panel by panel.
 //   order   (ordered variant) the Hessian-weighted loss of every column block under the
 //           plain quantizer, and the blocks sorted by descending loss.
 //   sweep   rows are independent. Positions are processed in panels of up to 64: one warp
@@ -192,7 +192,7 @@ __device__ __forceinline__ void tile_sum(double* sm, int n, F1 g1, F2 g2, int64_
   }
 }
 
-// g = c (MODE 0), -c (1) or g - c (2); row-major tile, leading dimension ld.
+// g = c (MODE 0), -c (1), g - c (2) or g + c (3); row-major tile, leading dimension ld.
 template <int MODE>
 __device__ __forceinline__ void put_tile(double* g, int64_t ld, const Frag& c) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -203,10 +203,11 @@ __device__ __forceinline__ void put_tile(double* g, int64_t ld, const Frag& c) {
     for (int n = 0; n < 4; ++n) {
       double2* q = reinterpret_cast<double2*>(
           g + (int64_t)(mb + 8 * m + (lane >> 2)) * ld + nb + 8 * n + 2 * (lane & 3));
-      const double2 o = MODE == 2 ? *q : make_double2(0.0, 0.0);
+      const double2 o = MODE >= 2 ? *q : make_double2(0.0, 0.0);
       if (MODE == 0) *q = make_double2(c[m][n][0], c[m][n][1]);
       else if (MODE == 1) *q = make_double2(-c[m][n][0], -c[m][n][1]);
-      else *q = make_double2(o.x - c[m][n][0], o.y - c[m][n][1]);
+      else if (MODE == 2) *q = make_double2(o.x - c[m][n][0], o.y - c[m][n][1]);
+      else *q = make_double2(o.x + c[m][n][0], o.y + c[m][n][1]);
     }
 }
 
@@ -265,38 +266,73 @@ k_syrk(double* A, int64_t kp, int p0, int pe, int j0, int j1, bool tri) {
   put_tile<2>(A + i * kNB * kp + j * kNB, kp, c);
 }
 
-// Off-diagonal blocks of M = L^-1 by doubling: segments of s tiles [a, a + s) and
-// [a + s, a + 2s) (the second cut at nt), both already inverted, merge as
-//   M_21 = -M_22 L_21 M_11,
-// in two launches over every pair of the level: T = L_21 M_11 (kept in A's unused upper
-// tiles, T_ij at tile (j, i)), then M_21 = -M_22 T. One CTA per output tile, blockIdx.y the
-// pair.
+// Off-diagonal tiles of M = L^-1, one row panel [p0, pe) at a time, right after the
+// Cholesky has finished that panel. Row i of L M = I gives, for j < i,
+//   M_ij = -M_ii sum_{t=j}^{i-1} L_it M_tj.
+// The terms with t below the panel arrive early: when panel P is final, k_minv_update adds
+// sum_{t in P} L_it M_tj into M_ij for every later row i >= pe and column j < pe (M's lower
+// tiles hold these partial sums S_ij until their row is finished); k_minv_row then finishes
+// row i of panel P from S_ij and the panel's own earlier rows. The work of the update is
+// largest when the Cholesky's trailing update has become small, so the two share the GPU.
+
+// Row i of the panel that starts at p0: M_ij for every j < i (one CTA per j).
 __global__ void __launch_bounds__(kPThreads)
-k_inv_a(double* A, const double* M, int64_t kp, int nt, int s) {
+k_minv_row(const double* A, double* M, int64_t kp, int p0, int i) {
   extern __shared__ double sm[];
-  const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
-  const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
-  if (i >= nt) return;
-  Frag c = {};
-  // T_ij = sum_{kk = j}^{a0 + s - 1} L_i,kk M_kk,j  (M_kk,j = 0 for kk < j)
-  tile_sum<false>(sm, (int)(a0 + s - j),
-                  [&](int q) { return (const double*)(A + i * kNB * kp + (j + q) * kNB); },
-                  [&](int q) { return M + (j + q) * kNB * kp + j * kNB; }, kp, c);
-  put_tile<0>(A + j * kNB * kp + i * kNB, kp, c);          // upper tile (j, i)
+  const int64_t j = blockIdx.x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int mb = 32 * (w >> 1), nb = 32 * (w & 1);
+  Frag c;
+  double* g = M + (int64_t)i * kNB * kp + j * kNB;
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      double2 v = make_double2(0.0, 0.0);    // S_ij from the earlier panels (none for j >= p0)
+      if (j < p0)
+        v = *reinterpret_cast<const double2*>(
+            g + (int64_t)(mb + 8 * m + (lane >> 2)) * kp + nb + 8 * n + 2 * (lane & 3));
+      c[m][n][0] = v.x;
+      c[m][n][1] = v.y;
+    }
+  const int64_t t0 = j > p0 ? j : p0;      // this panel's rows t in [max(j, p0), i)
+  tile_sum<false>(sm, (int)(i - t0),
+                  [&](int q) { return A + (int64_t)i * kNB * kp + (t0 + q) * kNB; },
+                  [&](int q) { return (const double*)(M + (t0 + q) * kNB * kp + j * kNB); }, kp,
+                  c);
+  // M_ij = -M_ii X, X = c: X through shared memory, M_ii staged beside it
+  double* xs = sm + kNB * kPLd;
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+      *reinterpret_cast<double2*>(xs + (mb + 8 * m + (lane >> 2)) * kPLd + nb + 8 * n +
+                                  2 * (lane & 3)) = make_double2(c[m][n][0], c[m][n][1]);
+  stage_async(sm, M + (int64_t)i * kNB * kp + (int64_t)i * kNB, kp);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  Frag d = {};
+  tile_mul<false>(sm, xs, d);
+  put_tile<1>(g, kp, d);
 }
 
+// After the rows of panel [p0, pe) are final: S_ij += sum_{t = max(j, p0)}^{pe-1} L_it M_tj
+// for rows pe <= i < nt and columns j < pe (the first contribution to a tile, j >= p0,
+// writes it).
 __global__ void __launch_bounds__(kPThreads)
-k_inv_b(const double* A, double* M, int64_t kp, int nt, int s) {
+k_minv_update(const double* A, double* M, int64_t kp, int p0, int pe) {
   extern __shared__ double sm[];
-  const int64_t a0 = (int64_t)blockIdx.y * 2 * s;
-  const int64_t i = a0 + s + blockIdx.x / s, j = a0 + blockIdx.x % s;
-  if (i >= nt) return;
+  const int64_t i = pe + blockIdx.x / pe, j = blockIdx.x % pe;
+  const int64_t t0 = j > p0 ? j : p0;
   Frag c = {};
-  // M_ij = -sum_{kk = a0 + s}^{i} M_i,kk T_kk,j  (T_kk,j kept at tile (j, kk))
-  tile_sum<false>(sm, (int)(i - a0 - s + 1),
-                  [&](int q) { return (const double*)(M + i * kNB * kp + (a0 + s + q) * kNB); },
-                  [&](int q) { return A + j * kNB * kp + (a0 + s + q) * kNB; }, kp, c);
-  put_tile<1>(M + i * kNB * kp + j * kNB, kp, c);
+  tile_sum<false>(sm, (int)(pe - t0),
+                  [&](int q) { return A + i * kNB * kp + (t0 + q) * kNB; },
+                  [&](int q) { return (const double*)(M + (t0 + q) * kNB * kp + j * kNB); }, kp,
+                  c);
+  double* g = M + i * kNB * kp + j * kNB;
+  if (j >= p0) put_tile<0>(g, kp, c);
+  else put_tile<3>(g, kp, c);
 }
 
 // U_pq = fl32(M_{k-1-p, k-1-q}) for q >= p, else 0.
@@ -312,17 +348,18 @@ __global__ void k_factor_store(FactorArgs a) {
 }  // namespace
 
 namespace {
-// Two streams and events for the factor's look-ahead, one set per device, created on first
-// use; calls on one device enqueue under its mutex. chain (the highest priority) carries the
-// panel factorisations, side (the lowest) the bulk trailing updates, so the block scheduler
-// serves the serial chain first whenever both have CTAs waiting.
+// Three streams and events for the factor's and the sweep's look-ahead, one set per device,
+// created on first use; calls on one device enqueue under its mutex. chain (the highest
+// priority) carries the panel factorisations, side the bulk trailing updates, inv (the
+// lowest) the factor's row panels of L^-1, so the block scheduler serves the serial chain
+// first, then the updates the chain waits for, and fills the rest with the inverse.
 struct FactorStreams {
   std::mutex mu;
-  cudaStream_t chain = nullptr, side = nullptr;
+  cudaStream_t chain = nullptr, side = nullptr, inv = nullptr;
   cudaEvent_t ev_start = nullptr, ev_panel = nullptr, ev_rest = nullptr, ev_end = nullptr,
-              ev_done = nullptr;
+              ev_done = nullptr, ev_chain = nullptr, ev_inv = nullptr;
 };
-// The current device's two streams and five events, created on first use; *err is set (and
+// The current device's three streams and seven events, created on first use; *err is set (and
 // nothing kept, so that a later call tries again) when any of them cannot be created.
 FactorStreams& factor_streams(cudaError_t* err) {
   static FactorStreams fs[64];
@@ -335,26 +372,33 @@ FactorStreams& factor_streams(cudaError_t* err) {
   if (!f.side) {
     int least = 0, greatest = 0;
     cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
-    cudaStream_t chain = nullptr, side = nullptr;
-    cudaEvent_t ev[5] = {};
+    // greatest is the numerically smallest; side sits between the two when the range allows
+    const int mid = least - greatest >= 2 ? (least + greatest) / 2 : least;
+    cudaStream_t chain = nullptr, side = nullptr, inv = nullptr;
+    cudaEvent_t ev[7] = {};
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, greatest);
-    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, least);
-    for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, mid);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&inv, cudaStreamNonBlocking, least);
+    for (int i = 0; i < 7 && e == cudaSuccess; ++i)
       e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
       for (cudaEvent_t x : ev)
         if (x) cudaEventDestroy(x);
+      if (inv) cudaStreamDestroy(inv);
       if (side) cudaStreamDestroy(side);
       if (chain) cudaStreamDestroy(chain);
       *err = e;
       return f;
     }
     f.chain = chain;
+    f.inv = inv;
     f.ev_start = ev[0];
     f.ev_panel = ev[1];
     f.ev_rest = ev[2];
     f.ev_end = ev[3];
     f.ev_done = ev[4];
+    f.ev_chain = ev[5];
+    f.ev_inv = ev[6];
     f.side = side;                          // last: marks the set complete
   }
   return f;
@@ -369,7 +413,7 @@ size_t gptq_factor_workspace(int64_t k) {
 cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* perm,
                                double damp, float* U, void* ws, cudaStream_t st) {
   for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update,
-                        (const void*)k_inv_a, (const void*)k_inv_b}) {
+                        (const void*)k_minv_row, (const void*)k_minv_update}) {
     const cudaError_t ae = ensure_dynamic_smem(f, (int)kProdSmem1);
     if (ae != cudaSuccess) return ae;
   }
@@ -382,7 +426,9 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   // a look-ahead of one panel: after panel P is factored (stream chain), its update of the
   // next panel's columns runs on chain, its update of everything beyond on side while chain
   // factors panel P + 1; panel P + 1's column update waits for the previous panel's update
-  // of everything beyond (both write those tiles). The two streams fork from and join the
+  // of everything beyond (both write those tiles). Panel P's rows of L^-1 and their
+  // contributions to the later rows run on inv as soon as chain has factored it (they read
+  // only final tiles of L and write only M). The three streams fork from and join the
   // caller's stream.
   cudaError_t serr = cudaSuccess;
   FactorStreams& fs = factor_streams(&serr);
@@ -392,6 +438,7 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   cudaEventRecord(fs.ev_start, st);
   cudaStreamWaitEvent(cs, fs.ev_start, 0);
   cudaStreamWaitEvent(fs.side, fs.ev_start, 0);
+  cudaStreamWaitEvent(fs.inv, fs.ev_start, 0);
   k_factor_lambda<<<1, kFThreads, 0, cs>>>(H, k, damp, a.scal);
   k_factor_load<<<gs, 256, 0, cs>>>(a);
   bool rest_pending = false;
@@ -403,6 +450,13 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
       if (nt - 1 - p > 0)
         k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, p);
     }
+    cudaEventRecord(fs.ev_chain, cs);
+    cudaStreamWaitEvent(fs.inv, fs.ev_chain, 0);
+    for (int i = (p0 > 1 ? p0 : 1); i < pe; ++i)
+      k_minv_row<<<(unsigned)i, kPThreads, kProdSmem1, fs.inv>>>(a.A, a.M, kp, p0, i);
+    if (pe < nt)
+      k_minv_update<<<(unsigned)((nt - pe) * pe), kPThreads, kProdSmem1, fs.inv>>>(a.A, a.M, kp,
+                                                                                 p0, pe);
     if (pe >= nt) break;
     const int pn = (int)(pe + kPanelTiles < nt ? pe + kPanelTiles : nt);   // next panel's end
     if (rest_pending) cudaStreamWaitEvent(cs, fs.ev_rest, 0);
@@ -420,12 +474,9 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
     }
   }
   cudaEventRecord(fs.ev_end, fs.side);
+  cudaEventRecord(fs.ev_inv, fs.inv);
   cudaStreamWaitEvent(cs, fs.ev_end, 0);
-  for (int s = 1; s < nt; s *= 2) {
-    const dim3 grid((unsigned)(s * s), (unsigned)((nt + 2 * s - 1) / (2 * s)));
-    k_inv_a<<<grid, kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, (int)nt, s);
-    k_inv_b<<<grid, kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, (int)nt, s);
-  }
+  cudaStreamWaitEvent(cs, fs.ev_inv, 0);
   k_factor_store<<<gs, 256, 0, cs>>>(a);
   cudaEventRecord(fs.ev_done, cs);
   cudaStreamWaitEvent(st, fs.ev_done, 0);
@@ -490,27 +541,68 @@ __device__ __forceinline__ int elem_project(float a, float4 t, float& wq_abs) {
   else return (int)g;
 }
 
+// fl32(s g(q)) of two magnitudes at scale t = {s, r_hi, r_lo} (0 for a zero scale): the
+// element step of the definition for a pair of elements at once.
+template <int ELEM>
+__device__ __forceinline__ float2 pair_project(float2 a, float4 t) {
+  const float2 g = elem_values<ELEM>(quot2(a, t));
+  const float2 wq = __fmul2_rn(make_float2(t.x, t.x), g);
+  return t.x == 0.0f ? make_float2(0.0f, 0.0f) : wq;
+}
+
 // The definition's candidate errors sum_j c_j (w_j - wq_j)^2 for four candidates at once
 // (independent accumulation chains): double, element order, each operation rounded once.
+// |w| - wq is the negation of w - copysign(wq, w) for a negative w, so its square is the
+// same double.
 template <int B, int ELEM, bool HOPT>
 __device__ __forceinline__ void exact_error4(const float* wb, const float* cw,
                                              const float4 (&t)[4], double (&e)[4]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) e[q] = 0.0;
 #pragma unroll 2
-  for (int j = 0; j < B; ++j) {
-    const float w = wb[j];
-    const double wd = (double)w;
-    const double c = HOPT ? (double)cw[j] : 1.0;
+  for (int j = 0; j < B; j += 2) {
+    const float2 av = make_float2(fabsf(wb[j]), fabsf(wb[j + 1]));
+    const double a0 = (double)av.x, a1 = (double)av.y;
+    const double c0 = HOPT ? (double)cw[j] : 1.0, c1 = HOPT ? (double)cw[j + 1] : 1.0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float wq_abs;
-      elem_project<ELEM>(fabsf(w), t[q], wq_abs);
-      const double d = __dsub_rn(wd, (double)copysignf(wq_abs, w));
-      e[q] = __dadd_rn(e[q], __dmul_rn(c, __dmul_rn(d, d)));
+      const float2 wq = pair_project<ELEM>(av, t[q]);
+      const double d0 = __dsub_rn(a0, (double)wq.x), d1 = __dsub_rn(a1, (double)wq.y);
+      const double s0 = __dmul_rn(d0, d0), s1 = __dmul_rn(d1, d1);
+      e[q] = __dadd_rn(e[q], HOPT ? __dmul_rn(c0, s0) : s0);
+      e[q] = __dadd_rn(e[q], HOPT ? __dmul_rn(c1, s1) : s1);
     }
   }
 }
+
+// The same sum for one candidate.
+template <int B, int ELEM, bool HOPT>
+__device__ __forceinline__ double exact_error1(const float* wb, const float* cw, float4 t) {
+  double e = 0.0;
+#pragma unroll 4
+  for (int j = 0; j < B; j += 2) {
+    const float2 av = make_float2(fabsf(wb[j]), fabsf(wb[j + 1]));
+    const float2 wq = pair_project<ELEM>(av, t);
+    const double d0 = __dsub_rn((double)av.x, (double)wq.x);
+    const double d1 = __dsub_rn((double)av.y, (double)wq.y);
+    const double s0 = __dmul_rn(d0, d0), s1 = __dmul_rn(d1, d1);
+    e = __dadd_rn(e, HOPT ? __dmul_rn((double)cw[j], s0) : s0);
+    e = __dadd_rn(e, HOPT ? __dmul_rn((double)cw[j + 1], s1) : s1);
+  }
+  return e;
+}
+
+// Smallest error over the warp, the lowest code among equal errors; every lane gets it.
+__device__ __forceinline__ void warp_argmin(double& be, int& bc) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double oe = __shfl_xor_sync(kFull, be, o);
+    const int oc = __shfl_xor_sync(kFull, bc, o);
+    if (oe < be || (oe == be && oc < bc)) { be = oe; bc = oc; }
+  }
+}
+
+constexpr int kPanWinBelow = 8;          // the full-scored window starts this far below naive
 
 // One warp per row; lane l holds panel positions 2l and 2l + 1.
 template <int B, int ELEM, int MODE>
@@ -521,6 +613,7 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Er
   __shared__ float hs[kPanel];
   __shared__ float wb[kPanelWarps][32];
   __shared__ float errs[kPanelWarps][32];
+  __shared__ uint8_t surv[kPanelWarps][256];   // codes left after the bounds, ascending
   for (int c = threadIdx.x; c < T.ncodes; c += blockDim.x) tab[c] = T.c[c];
   for (int e = threadIdx.x; e < kPanel * kPanel; e += blockDim.x) {
     const int i = e / kPanel, j = e % kPanel;
@@ -554,24 +647,58 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Er
     if (MODE != 0) {
       int lo, hi;
       grid_window(tab, T.ncodes, T.first, c0, a.window, lo, hi);
+      // (1) a window of 32 codes from just below the naive code, one per lane, in full
+      const int ws = max(lo, min(c0 - kPanWinBelow, hi - 31)), we = min(hi, ws + 31);
       double be = __longlong_as_double(0x7ff0000000000000LL);   // +inf
       int bc = 0x7fffffff;
-      // candidates lo + lane + 32 (4 g + q), four per pass (ascending within the lane)
-      for (int cb = lo + lane; cb <= hi; cb += 128) {
-        float4 tq[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tq[q] = tab[min(cb + 32 * q, hi)];
-        double e[4];
-        exact_error4<B, ELEM, MODE == 2>(wb[wid], hs + q0, tq, e);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (cb + 32 * q <= hi && e[q] < be) { be = e[q]; bc = cb + 32 * q; }
+      if (ws + lane <= we) {
+        be = exact_error1<B, ELEM, MODE == 2>(wb[wid], hs + q0, tab[ws + lane]);
+        bc = ws + lane;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const double oe = __shfl_xor_sync(kFull, be, o);
-        const int oc = __shfl_xor_sync(kFull, bc, o);
-        if (oe < be || (oe == be && oc < bc)) { be = oe; bc = oc; }
+      warp_argmin(be, bc);
+      // (2) the codes outside the window: a candidate's error is at least that of its two
+      // elements with the largest c a^2 (the same double terms the full sum adds, so the
+      // bound minus 2^-45 relative lies below its full sum); those whose bound exceeds the
+      // best error so far can neither win nor tie and are dropped, the rest are listed
+      if (lo < ws || we < hi) {
+        float2 top = make_float2(0.f, 0.f), ctop = make_float2(0.f, 0.f);
+        {
+          float v1 = -1.f, v2 = -1.f;
+          for (int j = 0; j < B; ++j) {
+            const float aj = fabsf(wb[wid][j]), cj = MODE == 2 ? hs[q0 + j] : 1.f;
+            const float v = cj * aj * aj;
+            if (v > v1) { v2 = v1; top.y = top.x; ctop.y = ctop.x; v1 = v; top.x = aj; ctop.x = cj; }
+            else if (v > v2) { v2 = v; top.y = aj; ctop.y = cj; }
+          }
+        }
+        const double bound_cut = be;
+        int total = 0;
+        for (int cb = lo; cb <= hi; cb += 32) {
+          const int c = cb + lane;
+          const bool in = c <= hi && (c < ws || c > we);
+          bool keep = false;
+          if (in) {
+            const float2 wq = pair_project<ELEM>(top, tab[c]);
+            const double d0 = __dsub_rn((double)top.x, (double)wq.x);
+            const double d1 = __dsub_rn((double)top.y, (double)wq.y);
+            const double s0 = __dmul_rn(d0, d0), s1 = __dmul_rn(d1, d1);
+            const double lb = __dadd_rn(MODE == 2 ? __dmul_rn((double)ctop.x, s0) : s0,
+                                        MODE == 2 ? __dmul_rn((double)ctop.y, s1) : s1);
+            keep = !(lb * (1.0 - 0x1p-45) > bound_cut);
+          }
+          const unsigned m = __ballot_sync(kFull, keep);
+          if (keep) surv[wid][total + __popc(m & ((1u << lane) - 1u))] = (uint8_t)c;
+          total += __popc(m);
+        }
+        __syncwarp();
+        // (3) the survivors in full, 32 at a time
+        for (int i = lane; i < total; i += 32) {
+          const int c = surv[wid][i];
+          const double e = exact_error1<B, ELEM, MODE == 2>(wb[wid], hs + q0, tab[c]);
+          if (e < be || (e == be && c < bc)) { be = e; bc = c; }
+        }
+        warp_argmin(be, bc);
+        __syncwarp();
       }
       cbest = bc == 0x7fffffff ? lo : bc;
     }
@@ -629,89 +756,104 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Er
 // Later positions p in [cbeg, cend) (after the panel [p0, p0 + S)): for each block of the
 // panel (in order) acc = sum_j fma(err_j, U[j][p], acc) over the block's columns, then
 // w -= acc. CTA: 64 positions x rg groups of 64 rows; thread: 4 rows x 4 consecutive
-// positions. The CTA's rows of U are staged once; the residuals of the next row group are
-// fetched with cp.async while the current group is updated.
-constexpr int kEsLd = kPanel + 4;        // padded residual row (16-byte aligned)
-constexpr size_t kTrailSmem = (2 * 64 * kEsLd + kPanel * 64) * sizeof(float);
-
-__device__ __forceinline__ void cp_async16(float* s, const float* g) {
-  const uint32_t a = (uint32_t)__cvta_generic_to_shared(s);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(g) : "memory");
-}
+// positions, as paired float32 FMAs (fma.rn.f32x2: two FMAs per instruction, each rounded
+// on its own). The CTA's rows of U are staged once; each group's residuals are staged
+// transposed (one 16-byte load gives a column's residuals of a thread's four rows), the
+// next group's fetched into registers while the current group is updated.
+constexpr int kEtLd = 64 + 4;            // transposed residual row: 64 rows + pad (16-byte aligned)
+constexpr size_t kTrailSmem = (2 * kPanel * kEtLd + kPanel * 64) * sizeof(float);
 
 template <int B>
 __global__ void __launch_bounds__(kTrailThreads)
 k_gptq_trailing(SweepArgs a, const float* __restrict__ Err, int64_t p0, int S, int64_t cbeg,
                 int64_t cend, int rg) {
   extern __shared__ __align__(16) float tsm[];
-  float (*Es)[64 * kEsLd] = reinterpret_cast<float (*)[64 * kEsLd]>(tsm);
-  float (*Ut)[64] = reinterpret_cast<float (*)[64]>(tsm + 2 * 64 * kEsLd);
+  float (*Et)[kPanel * kEtLd] = reinterpret_cast<float (*)[kPanel * kEtLd]>(tsm);
+  float (*Ut)[64] = reinterpret_cast<float (*)[64]>(tsm + 2 * kPanel * kEtLd);
   const int64_t c0 = cbeg + (int64_t)blockIdx.x * 64;
   const int64_t groups = (a.n + 63) / 64;
   const int64_t g0 = (int64_t)blockIdx.y * rg;
   const int ng = (int)(groups - g0 < rg ? groups - g0 : rg);
-  auto stage_es = [&](int buf, int64_t r0) {
-    for (int e = threadIdx.x; e < 64 * (kPanel / 4); e += kTrailThreads) {
-      const int i = e / (kPanel / 4), q = e % (kPanel / 4);
-      if (r0 + i < a.n) cp_async16(&Es[buf][i * kEsLd + 4 * q], Err + (r0 + i) * kPanel + 4 * q);
+  const int t = threadIdx.x;
+  // staging: thread t moves row t % 64 of the group, residual quads jq = t / 64 + 4 m
+  auto fetch = [&](int64_t r0, float4 (&v)[4]) {
+    const int64_t r = r0 + (t & 63);
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      v[m] = r < a.n ? *reinterpret_cast<const float4*>(Err + r * kPanel + 4 * ((t >> 6) + 4 * m))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  auto put = [&](int buf, const float4 (&v)[4]) {
+    float* e = Et[buf] + (t & 63);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int j = 4 * ((t >> 6) + 4 * m);
+      e[(j + 0) * kEtLd] = v[m].x;
+      e[(j + 1) * kEtLd] = v[m].y;
+      e[(j + 2) * kEtLd] = v[m].z;
+      e[(j + 3) * kEtLd] = v[m].w;
     }
   };
-  stage_es(0, g0 * 64);
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-  for (int e = threadIdx.x; e < kPanel * 16; e += kTrailThreads) {
+  float4 nxt[4];
+  fetch(g0 * 64, nxt);
+  put(0, nxt);
+  for (int e = t; e < kPanel * 16; e += kTrailThreads) {
     const int j = e / 16, g = e % 16;
     float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
     if (j < S && c0 + 4 * g < cend)
       u = *reinterpret_cast<const float4*>(a.U + (p0 + j) * a.k + c0 + 4 * g);
     *reinterpret_cast<float4*>(&Ut[j][4 * g]) = u;
   }
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  __syncthreads();
+  const int tx = t % 16, ty = t / 16;
   const int64_t col = c0 + 4 * tx;
   const bool on = col < cend;
   for (int g = 0; g < ng; ++g) {
     const int64_t r0 = (g0 + g) * 64;
-    if (g + 1 < ng) stage_es((g + 1) & 1, r0 + 64);
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-    float4 w[4];
+    const bool more = g + 1 < ng;
+    if (more) fetch(r0 + 64, nxt);
+    float2 w[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t r = r0 + 4 * ty + i;
-      w[i] = (on && r < a.n) ? *reinterpret_cast<const float4*>(a.Wc + r * a.k + col)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 v = (on && r < a.n) ? *reinterpret_cast<const float4*>(a.Wc + r * a.k + col)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[i][0] = make_float2(v.x, v.y);
+      w[i][1] = make_float2(v.z, v.w);
     }
-    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-    __syncthreads();
-    const float* E = Es[g & 1];
+    const float* E = Et[g & 1] + 4 * ty;
     for (int q0 = 0; q0 < S; q0 += B) {
-      float4 acc[4];
+      float2 acc[4][2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
 #pragma unroll 4
       for (int j = 0; j < B; ++j) {
+        const float4 e = *reinterpret_cast<const float4*>(E + (q0 + j) * kEtLd);
         const float4 u = *reinterpret_cast<const float4*>(&Ut[q0 + j][4 * tx]);
+        const float2 ua = make_float2(u.x, u.y), ub = make_float2(u.z, u.w);
+        const float ev[4] = {e.x, e.y, e.z, e.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float e = E[(4 * ty + i) * kEsLd + q0 + j];
-          acc[i].x = __fmaf_rn(e, u.x, acc[i].x);
-          acc[i].y = __fmaf_rn(e, u.y, acc[i].y);
-          acc[i].z = __fmaf_rn(e, u.z, acc[i].z);
-          acc[i].w = __fmaf_rn(e, u.w, acc[i].w);
+          const float2 e2 = make_float2(ev[i], ev[i]);
+          acc[i][0] = __ffma2_rn(e2, ua, acc[i][0]);
+          acc[i][1] = __ffma2_rn(e2, ub, acc[i][1]);
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        w[i].x = __fsub_rn(w[i].x, acc[i].x);
-        w[i].y = __fsub_rn(w[i].y, acc[i].y);
-        w[i].z = __fsub_rn(w[i].z, acc[i].z);
-        w[i].w = __fsub_rn(w[i].w, acc[i].w);
+      for (int i = 0; i < 4; ++i) {         // w - acc, as w + (-acc): the same rounding
+        w[i][0] = __fadd2_rn(w[i][0], make_float2(-acc[i][0].x, -acc[i][0].y));
+        w[i][1] = __fadd2_rn(w[i][1], make_float2(-acc[i][1].x, -acc[i][1].y));
       }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t r = r0 + 4 * ty + i;
-      if (on && r < a.n) *reinterpret_cast<float4*>(a.Wc + r * a.k + col) = w[i];
+      if (on && r < a.n)
+        *reinterpret_cast<float4*>(a.Wc + r * a.k + col) =
+            make_float4(w[i][0].x, w[i][0].y, w[i][1].x, w[i][1].y);
     }
-    __syncthreads();                      // Es[g & 1] is refilled two groups later
+    if (more) put((g + 1) & 1, nxt);
+    __syncthreads();                      // the next group's residuals are in place
   }
 }
 
