@@ -176,18 +176,71 @@ __device__ __forceinline__ void tile_mul(const double* S1, const double* S2, Fra
   }
 }
 
-// c = sum over n steps of tile(G1(q)) x tile(G2(q)) (x: NT or NN), q = 0 .. n-1: fetch both
-// tiles, multiply (two tiles of shared memory; several CTAs per SM overlap one another's
-// fetches and products).
+// c = sum over n steps of tile(G1(q)) x tile(G2(q)) (x: NT or NN), q = 0 .. n-1, in k-chunks
+// of 32: each chunk's operand halves are fetched into one of two stages while the other
+// stage is multiplied (A half [64][32] and B^T half [64][32] in rows of kHLd doubles, or B
+// half [32][64] in rows of kPLd; both keep every fragment load at two wavefronts).
+constexpr int kHLd = kNB / 2 + 4;
+constexpr int kStageD = kNB * kHLd + (kNB * kHLd > (kNB / 2) * kPLd ? kNB * kHLd : (kNB / 2) * kPLd);
+constexpr size_t kProdSmem = 2 * kStageD * sizeof(double);
+static_assert(kProdSmem >= kProdSmem1, "the last product of k_minv_row reuses the stages");
+
+template <bool NT>
+__device__ __forceinline__ void half_mul(const double* S1, const double* S2, Frag& c) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int mb = 32 * (w >> 1), nb = 32 * (w & 1);
+  const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll 2
+  for (int k0 = 0; k0 < kNB / 2; k0 += 4) {
+    double a[4], b[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) a[m] = S1[(mb + 8 * m + g) * kHLd + k0 + t4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+      b[n] = NT ? S2[(nb + 8 * n + g) * kHLd + k0 + t4] : S2[(k0 + t4) * kPLd + nb + 8 * n + g];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int n = 0; n < 4; ++n) dmma(a[m], b[n], c[m][n]);
+  }
+}
+
 template <bool NT, class F1, class F2>
 __device__ __forceinline__ void tile_sum(double* sm, int n, F1 g1, F2 g2, int64_t ld, Frag& c) {
-  for (int q = 0; q < n; ++q) {
-    stage_async(sm, g1(q), ld);
-    stage_async(sm + kNB * kPLd, g2(q), ld);
+  if (n <= 0) return;
+  auto stage = [&](int buf, int ch) {
+    const int q = ch >> 1, h = ch & 1;
+    double* sa = sm + buf * kStageD;
+    double* sb = sa + kNB * kHLd;
+    const double* ga = g1(q) + 32 * h;
+    for (int e = threadIdx.x; e < kNB * 16; e += kPThreads) {
+      const int r = e >> 4, c2 = 2 * (e & 15);
+      cp_async16d(sa + r * kHLd + c2, ga + (int64_t)r * ld + c2);
+    }
+    if (NT) {
+      const double* gb = g2(q) + 32 * h;
+      for (int e = threadIdx.x; e < kNB * 16; e += kPThreads) {
+        const int r = e >> 4, c2 = 2 * (e & 15);
+        cp_async16d(sb + r * kHLd + c2, gb + (int64_t)r * ld + c2);
+      }
+    } else {
+      const double* gb = g2(q) + (int64_t)(32 * h) * ld;
+      for (int e = threadIdx.x; e < (kNB / 2) * 32; e += kPThreads) {
+        const int r = e >> 5, c2 = 2 * (e & 31);
+        cp_async16d(sb + r * kPLd + c2, gb + (int64_t)r * ld + c2);
+      }
+    }
+  };
+  const int chunks = 2 * n;
+  stage(0, 0);
+  cp_async_commit();
+  for (int ch = 0; ch < chunks; ++ch) {
+    if (ch + 1 < chunks) stage((ch + 1) & 1, ch + 1);
     cp_async_commit();
-    cp_async_wait<0>();
+    cp_async_wait<1>();
     __syncthreads();
-    tile_mul<NT>(sm, sm + kNB * kPLd, c);
+    const double* sa = sm + (ch & 1) * kStageD;
+    half_mul<NT>(sa, sa + kNB * kHLd, c);
     __syncthreads();
   }
 }
@@ -414,7 +467,7 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
                                double damp, float* U, void* ws, cudaStream_t st) {
   for (const void* f : {(const void*)k_trsm, (const void*)k_syrk, (const void*)k_panel_update,
                         (const void*)k_minv_row, (const void*)k_minv_update}) {
-    const cudaError_t ae = ensure_dynamic_smem(f, (int)kProdSmem1);
+    const cudaError_t ae = ensure_dynamic_smem(f, (int)kProdSmem);
     if (ae != cudaSuccess) return ae;
   }
   const int64_t kp = (k + kNB - 1) / kNB * kNB, nt = kp / kNB;
@@ -445,29 +498,29 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   for (int p0 = 0; p0 < nt; p0 += kPanelTiles) {
     const int pe = (int)(p0 + kPanelTiles < nt ? p0 + kPanelTiles : nt);
     for (int p = p0; p < pe; ++p) {
-      if (p > p0) k_panel_update<<<(unsigned)(nt - p), kPThreads, kProdSmem1, cs>>>(a.A, kp, p0, p);
+      if (p > p0) k_panel_update<<<(unsigned)(nt - p), kPThreads, kProdSmem, cs>>>(a.A, kp, p0, p);
       k_potrf_inv<<<1, kFThreads, 0, cs>>>(a.A, a.M, kp, p);
       if (nt - 1 - p > 0)
-        k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem1, cs>>>(a.A, a.M, kp, p);
+        k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem, cs>>>(a.A, a.M, kp, p);
     }
     cudaEventRecord(fs.ev_chain, cs);
     cudaStreamWaitEvent(fs.inv, fs.ev_chain, 0);
     for (int i = (p0 > 1 ? p0 : 1); i < pe; ++i)
-      k_minv_row<<<(unsigned)i, kPThreads, kProdSmem1, fs.inv>>>(a.A, a.M, kp, p0, i);
+      k_minv_row<<<(unsigned)i, kPThreads, kProdSmem, fs.inv>>>(a.A, a.M, kp, p0, i);
     if (pe < nt)
-      k_minv_update<<<(unsigned)((nt - pe) * pe), kPThreads, kProdSmem1, fs.inv>>>(a.A, a.M, kp,
+      k_minv_update<<<(unsigned)((nt - pe) * pe), kPThreads, kProdSmem, fs.inv>>>(a.A, a.M, kp,
                                                                                  p0, pe);
     if (pe >= nt) break;
     const int pn = (int)(pe + kPanelTiles < nt ? pe + kPanelTiles : nt);   // next panel's end
     if (rest_pending) cudaStreamWaitEvent(cs, fs.ev_rest, 0);
-    k_syrk<<<(unsigned)((nt - pe) * (pn - pe)), kPThreads, kProdSmem1, cs>>>(a.A, kp, p0, pe, pe,
+    k_syrk<<<(unsigned)((nt - pe) * (pn - pe)), kPThreads, kProdSmem, cs>>>(a.A, kp, p0, pe, pe,
                                                                             pn, false);
     rest_pending = false;
     if (pn < nt) {
       cudaEventRecord(fs.ev_panel, cs);
       cudaStreamWaitEvent(fs.side, fs.ev_panel, 0);
       const int64_t m = nt - pn;
-      k_syrk<<<(unsigned)(m * (m + 1) / 2), kPThreads, kProdSmem1, fs.side>>>(a.A, kp, p0, pe, pn,
+      k_syrk<<<(unsigned)(m * (m + 1) / 2), kPThreads, kProdSmem, fs.side>>>(a.A, kp, p0, pe, pn,
                                                                               (int)nt, true);
       cudaEventRecord(fs.ev_rest, fs.side);
       rest_pending = true;
@@ -489,8 +542,9 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
 namespace {
 
 constexpr int kPanel = 64;               // positions per panel
-constexpr int kPanelWarps = 8;           // rows per panel CTA (one warp each)
-constexpr int kTrailThreads = 256;       // 64 rows x 64 positions per trailing CTA
+constexpr int kPanelWarps = 4;           // rows per panel CTA (one warp each)
+constexpr int kTrRows = 8;               // rows per thread of the trailing update
+constexpr int kTrailThreads = 16 * (64 / kTrRows);   // 64 rows x 64 positions per CTA
 
 struct SweepArgs {
   const char* W;
@@ -550,32 +604,9 @@ __device__ __forceinline__ float2 pair_project(float2 a, float4 t) {
   return t.x == 0.0f ? make_float2(0.0f, 0.0f) : wq;
 }
 
-// The definition's candidate errors sum_j c_j (w_j - wq_j)^2 for four candidates at once
-// (independent accumulation chains): double, element order, each operation rounded once.
-// |w| - wq is the negation of w - copysign(wq, w) for a negative w, so its square is the
-// same double.
-template <int B, int ELEM, bool HOPT>
-__device__ __forceinline__ void exact_error4(const float* wb, const float* cw,
-                                             const float4 (&t)[4], double (&e)[4]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) e[q] = 0.0;
-#pragma unroll 2
-  for (int j = 0; j < B; j += 2) {
-    const float2 av = make_float2(fabsf(wb[j]), fabsf(wb[j + 1]));
-    const double a0 = (double)av.x, a1 = (double)av.y;
-    const double c0 = HOPT ? (double)cw[j] : 1.0, c1 = HOPT ? (double)cw[j + 1] : 1.0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 wq = pair_project<ELEM>(av, t[q]);
-      const double d0 = __dsub_rn(a0, (double)wq.x), d1 = __dsub_rn(a1, (double)wq.y);
-      const double s0 = __dmul_rn(d0, d0), s1 = __dmul_rn(d1, d1);
-      e[q] = __dadd_rn(e[q], HOPT ? __dmul_rn(c0, s0) : s0);
-      e[q] = __dadd_rn(e[q], HOPT ? __dmul_rn(c1, s1) : s1);
-    }
-  }
-}
-
-// The same sum for one candidate.
+// The definition's candidate error sum_j c_j (w_j - wq_j)^2 of one block (magnitudes in wb,
+// h weights in cw): double, element order, each operation rounded once. |w| - wq is the
+// negation of w - copysign(wq, w) for a negative w, so its square is the same double.
 template <int B, int ELEM, bool HOPT>
 __device__ __forceinline__ double exact_error1(const float* wb, const float* cw, float4 t) {
   double e = 0.0;
@@ -755,105 +786,103 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Er
 
 // Later positions p in [cbeg, cend) (after the panel [p0, p0 + S)): for each block of the
 // panel (in order) acc = sum_j fma(err_j, U[j][p], acc) over the block's columns, then
-// w -= acc. CTA: 64 positions x rg groups of 64 rows; thread: 4 rows x 4 consecutive
+// w -= acc. CTA: 64 positions x rg groups of 64 rows; thread: kTrRows rows (ty, ty + 64 /
+// kTrRows, ...: the rows a warp reads at once sit in different banks) x 4 consecutive
 // positions, as paired float32 FMAs (fma.rn.f32x2: two FMAs per instruction, each rounded
-// on its own). The CTA's rows of U are staged once; each group's residuals are staged
-// transposed (one 16-byte load gives a column's residuals of a thread's four rows), the
-// next group's fetched into registers while the current group is updated.
-constexpr int kEtLd = 64 + 4;            // transposed residual row: 64 rows + pad (16-byte aligned)
-constexpr size_t kTrailSmem = (2 * kPanel * kEtLd + kPanel * 64) * sizeof(float);
+// on its own). The CTA's rows of U are staged once; the residuals of the next row group are
+// fetched with cp.async while the current group is updated, and read four columns at a
+// time (one 16-byte load per row feeds 8 FMAs per position pair).
+constexpr int kEsLd = kPanel + 4;        // padded residual row (16-byte aligned)
+constexpr size_t kTrailSmem = (2 * 64 * kEsLd + kPanel * 64) * sizeof(float);
+
+__device__ __forceinline__ void cp_async16f(float* s, const float* g) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(s);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(a), "l"(g) : "memory");
+}
 
 template <int B>
 __global__ void __launch_bounds__(kTrailThreads)
 k_gptq_trailing(SweepArgs a, const float* __restrict__ Err, int64_t p0, int S, int64_t cbeg,
                 int64_t cend, int rg) {
   extern __shared__ __align__(16) float tsm[];
-  float (*Et)[kPanel * kEtLd] = reinterpret_cast<float (*)[kPanel * kEtLd]>(tsm);
-  float (*Ut)[64] = reinterpret_cast<float (*)[64]>(tsm + 2 * kPanel * kEtLd);
+  float (*Es)[64 * kEsLd] = reinterpret_cast<float (*)[64 * kEsLd]>(tsm);
+  float (*Ut)[64] = reinterpret_cast<float (*)[64]>(tsm + 2 * 64 * kEsLd);
+  constexpr int kRs = 64 / kTrRows;      // row stride of a thread's rows
   const int64_t c0 = cbeg + (int64_t)blockIdx.x * 64;
   const int64_t groups = (a.n + 63) / 64;
   const int64_t g0 = (int64_t)blockIdx.y * rg;
   const int ng = (int)(groups - g0 < rg ? groups - g0 : rg);
-  const int t = threadIdx.x;
-  // staging: thread t moves row t % 64 of the group, residual quads jq = t / 64 + 4 m
-  auto fetch = [&](int64_t r0, float4 (&v)[4]) {
-    const int64_t r = r0 + (t & 63);
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-      v[m] = r < a.n ? *reinterpret_cast<const float4*>(Err + r * kPanel + 4 * ((t >> 6) + 4 * m))
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-  };
-  auto put = [&](int buf, const float4 (&v)[4]) {
-    float* e = Et[buf] + (t & 63);
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int j = 4 * ((t >> 6) + 4 * m);
-      e[(j + 0) * kEtLd] = v[m].x;
-      e[(j + 1) * kEtLd] = v[m].y;
-      e[(j + 2) * kEtLd] = v[m].z;
-      e[(j + 3) * kEtLd] = v[m].w;
+  auto stage_es = [&](int buf, int64_t r0) {
+    for (int e = threadIdx.x; e < 64 * (kPanel / 4); e += kTrailThreads) {
+      const int i = e / (kPanel / 4), q = e % (kPanel / 4);
+      if (r0 + i < a.n) cp_async16f(&Es[buf][i * kEsLd + 4 * q], Err + (r0 + i) * kPanel + 4 * q);
     }
   };
-  float4 nxt[4];
-  fetch(g0 * 64, nxt);
-  put(0, nxt);
-  for (int e = t; e < kPanel * 16; e += kTrailThreads) {
+  stage_es(0, g0 * 64);
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+  for (int e = threadIdx.x; e < kPanel * 16; e += kTrailThreads) {
     const int j = e / 16, g = e % 16;
     float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
     if (j < S && c0 + 4 * g < cend)
       u = *reinterpret_cast<const float4*>(a.U + (p0 + j) * a.k + c0 + 4 * g);
     *reinterpret_cast<float4*>(&Ut[j][4 * g]) = u;
   }
-  __syncthreads();
-  const int tx = t % 16, ty = t / 16;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const int64_t col = c0 + 4 * tx;
   const bool on = col < cend;
   for (int g = 0; g < ng; ++g) {
     const int64_t r0 = (g0 + g) * 64;
-    const bool more = g + 1 < ng;
-    if (more) fetch(r0 + 64, nxt);
-    float2 w[4][2];
+    if (g + 1 < ng) stage_es((g + 1) & 1, r0 + 64);
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    float2 w[kTrRows][2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t r = r0 + 4 * ty + i;
+    for (int i = 0; i < kTrRows; ++i) {
+      const int64_t r = r0 + ty + kRs * i;
       const float4 v = (on && r < a.n) ? *reinterpret_cast<const float4*>(a.Wc + r * a.k + col)
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
       w[i][0] = make_float2(v.x, v.y);
       w[i][1] = make_float2(v.z, v.w);
     }
-    const float* E = Et[g & 1] + 4 * ty;
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+    __syncthreads();
+    const float* E = Es[g & 1] + ty * kEsLd;
     for (int q0 = 0; q0 < S; q0 += B) {
-      float2 acc[4][2];
+      float2 acc[kTrRows][2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
-#pragma unroll 4
-      for (int j = 0; j < B; ++j) {
-        const float4 e = *reinterpret_cast<const float4*>(E + (q0 + j) * kEtLd);
-        const float4 u = *reinterpret_cast<const float4*>(&Ut[q0 + j][4 * tx]);
-        const float2 ua = make_float2(u.x, u.y), ub = make_float2(u.z, u.w);
-        const float ev[4] = {e.x, e.y, e.z, e.w};
+      for (int i = 0; i < kTrRows; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 e2 = make_float2(ev[i], ev[i]);
-          acc[i][0] = __ffma2_rn(e2, ua, acc[i][0]);
-          acc[i][1] = __ffma2_rn(e2, ub, acc[i][1]);
+      for (int j4 = 0; j4 < B; j4 += 4) {
+        float4 e[kTrRows];
+#pragma unroll
+        for (int i = 0; i < kTrRows; ++i)
+          e[i] = *reinterpret_cast<const float4*>(E + kRs * i * kEsLd + q0 + j4);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float4 u = *reinterpret_cast<const float4*>(&Ut[q0 + j4 + jj][4 * tx]);
+          const float2 ua = make_float2(u.x, u.y), ub = make_float2(u.z, u.w);
+#pragma unroll
+          for (int i = 0; i < kTrRows; ++i) {
+            const float ev = jj == 0 ? e[i].x : jj == 1 ? e[i].y : jj == 2 ? e[i].z : e[i].w;
+            const float2 e2 = make_float2(ev, ev);
+            acc[i][0] = __ffma2_rn(e2, ua, acc[i][0]);
+            acc[i][1] = __ffma2_rn(e2, ub, acc[i][1]);
+          }
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {         // w - acc, as w + (-acc): the same rounding
+      for (int i = 0; i < kTrRows; ++i) {   // w - acc, as w + (-acc): the same rounding
         w[i][0] = __fadd2_rn(w[i][0], make_float2(-acc[i][0].x, -acc[i][0].y));
         w[i][1] = __fadd2_rn(w[i][1], make_float2(-acc[i][1].x, -acc[i][1].y));
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t r = r0 + 4 * ty + i;
+    for (int i = 0; i < kTrRows; ++i) {
+      const int64_t r = r0 + ty + kRs * i;
       if (on && r < a.n)
         *reinterpret_cast<float4*>(a.Wc + r * a.k + col) =
             make_float4(w[i][0].x, w[i][0].y, w[i][1].x, w[i][1].y);
     }
-    if (more) put((g + 1) & 1, nxt);
-    __syncthreads();                      // the next group's residuals are in place
+    __syncthreads();                      // Es[g & 1] is refilled two groups later
   }
 }
 
