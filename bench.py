@@ -628,19 +628,21 @@ def gpu_arm(args):
         # pass's free up
         s_h, s_q = torch.cuda.Stream(dev), torch.cuda.Stream(dev, priority=-1)
         hb = [hs, [torch.empty_like(h) for h in hs]]
-        ev_h = [torch.cuda.Event() for _ in range(2)]
-        ev_q = [torch.cuda.Event() for _ in range(2)]
+        # a fresh pair of events per step, so that no event is recorded again while a wait
+        # on its earlier record may still be queued (the host runs many steps ahead)
+        ev_h = [torch.cuda.Event() for _ in range(max(args.warmup, args.steps))]
+        ev_q = [torch.cuda.Event() for _ in range(max(args.warmup, args.steps))]
 
         def pstep(i, wait_free):
             b = i & 1
             with torch.cuda.stream(s_h):
                 if wait_free:
-                    s_h.wait_event(ev_q[b])
+                    s_h.wait_event(ev_q[i - 2])
                 for X, h, ws in zip(Xs, hb[b], wss):
                     mxq.mxq_act_sqmean(X, h, workspace=ws)
-                ev_h[b].record(s_h)
+                ev_h[i].record(s_h)
             with torch.cuda.stream(s_q):
-                s_q.wait_event(ev_h[b])
+                s_q.wait_event(ev_h[i])
                 for W, (codes, scales, sums, ews, xi) in zip(Ws, outs):
                     if fused:
                         mxq.mxq_quantize_err(W, p_pipe, hb[b][xi], codes=codes,
@@ -648,7 +650,7 @@ def gpu_arm(args):
                     else:
                         mxq.mxq_quantize(W, p, hb[b][xi], codes=codes, scales=scales)
                         mxq.mxq_error(W, codes, scales, p, hb[b][xi], sums=sums, workspace=ews)
-                ev_q[b].record(s_q)
+                ev_q[i].record(s_q)
 
         for i in range(args.warmup):
             pstep(i, i >= 2)

@@ -406,11 +406,19 @@ namespace {
 // priority) carries the panel factorisations, side the bulk trailing updates, inv (the
 // lowest) the factor's row panels of L^-1, so the block scheduler serves the serial chain
 // first, then the updates the chain waits for, and fills the rest with the inverse.
+constexpr int kEvRing = 1024;
 struct FactorStreams {
   std::mutex mu;
   cudaStream_t chain = nullptr, side = nullptr, inv = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_panel = nullptr, ev_rest = nullptr, ev_end = nullptr,
-              ev_done = nullptr, ev_chain = nullptr, ev_inv = nullptr;
+  cudaEvent_t ring[kEvRing] = {};
+  int next = 0;
+  // a fresh event for each record, so that no event is recorded again while an earlier wait
+  // on it may still be queued
+  cudaEvent_t take() {
+    cudaEvent_t e = ring[next];
+    next = (next + 1) % kEvRing;
+    return e;
+  }
 };
 // The current device's three streams and seven events, created on first use; *err is set (and
 // nothing kept, so that a later call tries again) when any of them cannot be created.
@@ -428,11 +436,11 @@ FactorStreams& factor_streams(cudaError_t* err) {
     // greatest is the numerically smallest; side sits between the two when the range allows
     const int mid = least - greatest >= 2 ? (least + greatest) / 2 : least;
     cudaStream_t chain = nullptr, side = nullptr, inv = nullptr;
-    cudaEvent_t ev[7] = {};
+    cudaEvent_t ev[kEvRing] = {};
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, greatest);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, mid);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&inv, cudaStreamNonBlocking, least);
-    for (int i = 0; i < 7 && e == cudaSuccess; ++i)
+    for (int i = 0; i < kEvRing && e == cudaSuccess; ++i)
       e = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
     if (e != cudaSuccess) {
       for (cudaEvent_t x : ev)
@@ -445,13 +453,7 @@ FactorStreams& factor_streams(cudaError_t* err) {
     }
     f.chain = chain;
     f.inv = inv;
-    f.ev_start = ev[0];
-    f.ev_panel = ev[1];
-    f.ev_rest = ev[2];
-    f.ev_end = ev[3];
-    f.ev_done = ev[4];
-    f.ev_chain = ev[5];
-    f.ev_inv = ev[6];
+    for (int i = 0; i < kEvRing; ++i) f.ring[i] = ev[i];
     f.side = side;                          // last: marks the set complete
   }
   return f;
@@ -488,10 +490,12 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
   if (serr != cudaSuccess) return serr;
   std::lock_guard<std::mutex> lk(fs.mu);
   cudaStream_t cs = fs.chain;
-  cudaEventRecord(fs.ev_start, st);
-  cudaStreamWaitEvent(cs, fs.ev_start, 0);
-  cudaStreamWaitEvent(fs.side, fs.ev_start, 0);
-  cudaStreamWaitEvent(fs.inv, fs.ev_start, 0);
+  cudaEvent_t e0 = fs.take();
+  cudaEventRecord(e0, st);
+  cudaStreamWaitEvent(cs, e0, 0);
+  cudaStreamWaitEvent(fs.side, e0, 0);
+  cudaStreamWaitEvent(fs.inv, e0, 0);
+  cudaEvent_t ev_rest = nullptr;
   k_factor_lambda<<<1, kFThreads, 0, cs>>>(H, k, damp, a.scal);
   k_factor_load<<<gs, 256, 0, cs>>>(a);
   bool rest_pending = false;
@@ -503,8 +507,11 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
       if (nt - 1 - p > 0)
         k_trsm<<<(unsigned)(nt - 1 - p), kPThreads, kProdSmem, cs>>>(a.A, a.M, kp, p);
     }
-    cudaEventRecord(fs.ev_chain, cs);
-    cudaStreamWaitEvent(fs.inv, fs.ev_chain, 0);
+    {
+      cudaEvent_t ec = fs.take();
+      cudaEventRecord(ec, cs);
+      cudaStreamWaitEvent(fs.inv, ec, 0);
+    }
     for (int i = (p0 > 1 ? p0 : 1); i < pe; ++i)
       k_minv_row<<<(unsigned)i, kPThreads, kProdSmem, fs.inv>>>(a.A, a.M, kp, p0, i);
     if (pe < nt)
@@ -512,27 +519,31 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
                                                                                  p0, pe);
     if (pe >= nt) break;
     const int pn = (int)(pe + kPanelTiles < nt ? pe + kPanelTiles : nt);   // next panel's end
-    if (rest_pending) cudaStreamWaitEvent(cs, fs.ev_rest, 0);
+    if (rest_pending) cudaStreamWaitEvent(cs, ev_rest, 0);
     k_syrk<<<(unsigned)((nt - pe) * (pn - pe)), kPThreads, kProdSmem, cs>>>(a.A, kp, p0, pe, pe,
                                                                             pn, false);
     rest_pending = false;
     if (pn < nt) {
-      cudaEventRecord(fs.ev_panel, cs);
-      cudaStreamWaitEvent(fs.side, fs.ev_panel, 0);
+      cudaEvent_t ep = fs.take();
+      cudaEventRecord(ep, cs);
+      cudaStreamWaitEvent(fs.side, ep, 0);
       const int64_t m = nt - pn;
       k_syrk<<<(unsigned)(m * (m + 1) / 2), kPThreads, kProdSmem, fs.side>>>(a.A, kp, p0, pe, pn,
                                                                               (int)nt, true);
-      cudaEventRecord(fs.ev_rest, fs.side);
+      ev_rest = fs.take();
+      cudaEventRecord(ev_rest, fs.side);
       rest_pending = true;
     }
   }
-  cudaEventRecord(fs.ev_end, fs.side);
-  cudaEventRecord(fs.ev_inv, fs.inv);
-  cudaStreamWaitEvent(cs, fs.ev_end, 0);
-  cudaStreamWaitEvent(cs, fs.ev_inv, 0);
+  cudaEvent_t e_end = fs.take(), e_inv = fs.take();
+  cudaEventRecord(e_end, fs.side);
+  cudaEventRecord(e_inv, fs.inv);
+  cudaStreamWaitEvent(cs, e_end, 0);
+  cudaStreamWaitEvent(cs, e_inv, 0);
   k_factor_store<<<gs, 256, 0, cs>>>(a);
-  cudaEventRecord(fs.ev_done, cs);
-  cudaStreamWaitEvent(st, fs.ev_done, 0);
+  cudaEvent_t e_done = fs.take();
+  cudaEventRecord(e_done, cs);
+  cudaStreamWaitEvent(st, e_done, 0);
   return cudaGetLastError();
 }
 
@@ -911,9 +922,11 @@ cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cud
   if (serr != cudaSuccess) return serr;
   std::lock_guard<std::mutex> lk(fs.mu);
   cudaStream_t cs = fs.chain;
-  cudaEventRecord(fs.ev_start, st);
-  cudaStreamWaitEvent(cs, fs.ev_start, 0);
-  cudaStreamWaitEvent(fs.side, fs.ev_start, 0);
+  cudaEvent_t e0 = fs.take();
+  cudaEventRecord(e0, st);
+  cudaStreamWaitEvent(cs, e0, 0);
+  cudaStreamWaitEvent(fs.side, e0, 0);
+  cudaEvent_t ev_rest = nullptr;
   k_sweep_init<B><<<sm_count() * 8, 256, 0, cs>>>(a);
   const unsigned prow = (unsigned)((a.n + kPanelWarps - 1) / kPanelWarps);
   bool rest_pending = false;
@@ -926,21 +939,24 @@ cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cud
     else k_gptq_panel<B, ELEM, 2><<<prow, kPanelWarps * 32, 0, cs>>>(a, T, p0, S, err);
     const int64_t c1 = p0 + S, c2 = c1 + kPanel < a.k ? c1 + kPanel : a.k;
     if (c1 >= a.k) break;
-    if (rest_pending) cudaStreamWaitEvent(cs, fs.ev_rest, 0);
+    if (rest_pending) cudaStreamWaitEvent(cs, ev_rest, 0);
     launch_trailing<B>(a, err, p0, S, c1, c2, cs);
     rest_pending = false;
     if (c2 < a.k) {
-      cudaEventRecord(fs.ev_panel, cs);
-      cudaStreamWaitEvent(fs.side, fs.ev_panel, 0);
+      cudaEvent_t ep = fs.take();
+      cudaEventRecord(ep, cs);
+      cudaStreamWaitEvent(fs.side, ep, 0);
       launch_trailing<B>(a, err, p0, S, c2, a.k, fs.side);
-      cudaEventRecord(fs.ev_rest, fs.side);
+      ev_rest = fs.take();
+      cudaEventRecord(ev_rest, fs.side);
       rest_pending = true;
     }
   }
-  cudaEventRecord(fs.ev_end, fs.side);
-  cudaStreamWaitEvent(cs, fs.ev_end, 0);
-  cudaEventRecord(fs.ev_done, cs);
-  cudaStreamWaitEvent(st, fs.ev_done, 0);
+  cudaEvent_t e_end = fs.take(), e_done = fs.take();
+  cudaEventRecord(e_end, fs.side);
+  cudaStreamWaitEvent(cs, e_end, 0);
+  cudaEventRecord(e_done, cs);
+  cudaStreamWaitEvent(st, e_done, 0);
   return cudaGetLastError();
 }
 

@@ -38,8 +38,8 @@
  *    mxq_last_error() (per host thread) describes it. No exception crosses the boundary.
  *  - Calls are reentrant. Mutable state, all of it set up on first use and guarded by
  *    locks: the per-thread error text; per device, the raised shared-memory limit of each
- *    tensor-core kernel; per device, the two library streams and their events that
- *    mxq_gptq_factor and mxq_gptq create on first use (their calls on one device are
+ *    tensor-core kernel; per device, the three library streams and the ring of events
+ *    that mxq_gptq_factor and mxq_gptq create on first use (their calls on one device are
  *    ordered on the host); and per device the address of the static scratch of
  *    mxq_act_sqmean_noalloc.
  *  - Empty problems (n, k or rows == 0) return MXQ_OK without launching.
