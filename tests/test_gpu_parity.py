@@ -331,7 +331,8 @@ def test_quantize_with_error_sums(mxq, orc, synth, fmt, block, mode, with_h):
     assert torch.equal(sums, again)                     # deterministic
 
 
-def test_search_occupancy_setting(mxq, orc, synth):
+@pytest.mark.parametrize("B,mode", [(16, "hopt"), (32, "hopt"), (32, "sse")])
+def test_search_occupancy_setting(mxq, orc, synth, B, mode):
     """ctas_per_sm limits the NVFP4 search's persistent grid (room for a concurrent h pass):
     the codes and scales are the same for every setting, and the fused error sums agree with
     the oracle's (they group the blocks by CTA, so only the last bits may move)."""
@@ -340,11 +341,12 @@ def test_search_occupancy_setting(mxq, orc, synth):
     X = synth.activations(256, k, 92, dtype=torch.bfloat16, device="cpu")
     h = orc.act_sqmean(oracle_view(X))
     hd = torch.from_numpy(h).to(DEV)
-    r = orc.quantize(oracle_view(W), "nvfp4", "hopt", 16, h=h)
-    ref = orc.error_sums(oracle_view(W), orc.dequant(r.codes, r.scales, "nvfp4", 16, n, k), h)
+    r = orc.quantize(oracle_view(W), "nvfp4", mode, B, h=h if mode == "hopt" else None)
+    ref = orc.error_sums(oracle_view(W), orc.dequant(r.codes, r.scales, "nvfp4", B, n, k),
+                         h if mode == "hopt" else None)
     for cps in (0, 1, 2, 3, 9):
-        p = mxq.params("nvfp4", "hopt", 16, ctas_per_sm=cps)
-        c, s, sums = mxq.mxq_quantize_err(W, p, hd)
+        p = mxq.params("nvfp4", mode, B, ctas_per_sm=cps)
+        c, s, sums = mxq.mxq_quantize_err(W, p, hd if mode == "hopt" else None)
         assert np.array_equal(c.cpu().numpy(), r.codes) and np.array_equal(s.cpu().numpy(), r.scales)
         np.testing.assert_allclose(sums.cpu().numpy(), ref, rtol=1e-5)
 
