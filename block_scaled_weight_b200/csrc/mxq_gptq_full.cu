@@ -11,9 +11,9 @@
 //           inverse-then-Cholesky; the inverse follows the Cholesky panel by panel.
 //   order   (ordered variant) the Hessian-weighted loss of every column block under the
 //           plain quantizer, and the blocks sorted by descending loss.
-//   sweep   rows are independent. Positions are processed in panels of up to 64: one warp
-//           per row searches each block's scale exactly on its current weights (every
-//           candidate's error in double, element order, lowest code on ties), quantises
+//   sweep   rows are independent. Positions are processed in panels of up to 64: one
+//           half-warp per row searches each block's scale exactly on its current weights
+//           (candidate errors in double, element order, lowest code on ties), quantises
 //           the block's columns one after another with the in-block updates, and applies
 //           each block's product to the panel's later blocks; a tiled kernel then applies
 //           the panel's block products to every later position of every row (the next
@@ -553,7 +553,6 @@ cudaError_t launch_gptq_factor(const float* H, int64_t k, int B, const int32_t* 
 namespace {
 
 constexpr int kPanel = 64;               // positions per panel
-constexpr int kPanelWarps = 4;           // rows per panel CTA (one warp each)
 constexpr int kTrRows = 8;               // rows per thread of the trailing update
 constexpr int kTrailThreads = 16 * (64 / kTrRows);   // 64 rows x 64 positions per CTA
 
@@ -634,28 +633,38 @@ __device__ __forceinline__ double exact_error1(const float* wb, const float* cw,
   return e;
 }
 
-// Smallest error over the warp, the lowest code among equal errors; every lane gets it.
-__device__ __forceinline__ void warp_argmin(double& be, int& bc) {
+constexpr int kPanWinBelow = 8;          // the full-scored window starts this far below naive
+
+// Two rows per warp, one per half-warp: lane l of half f (l = lane & 15) holds panel
+// positions 4l .. 4l + 3 of row 2 w + f, so that the per-column chain (projection, division,
+// broadcast), which leaves all but one lane of a row waiting, serves two rows per
+// instruction. Each block's scale search is exact (float64, element order, the split-
+// reciprocal quotient that equals the IEEE one; the lowest code on ties) but scores in full
+// only a window of 32 codes from 8 below the naive code (two per lane); every other code gets
+// a lower bound from the block's two elements with the largest c a^2 -- the same double terms
+// its full sum would add, so the bound less 2^-45 relative lies below that sum -- and only
+// codes whose bound does not exceed the best error so far are listed and scored in full.
+constexpr int kPanelWarpsH = 2;          // warps per CTA (four rows)
+
+// Smallest error within each half-warp, the lowest code among equal errors.
+__device__ __forceinline__ void half_argmin(double& be, int& bc) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int o = 8; o > 0; o >>= 1) {
     const double oe = __shfl_xor_sync(kFull, be, o);
     const int oc = __shfl_xor_sync(kFull, bc, o);
     if (oe < be || (oe == be && oc < bc)) { be = oe; bc = oc; }
   }
 }
 
-constexpr int kPanWinBelow = 8;          // the full-scored window starts this far below naive
-
-// One warp per row; lane l holds panel positions 2l and 2l + 1.
 template <int B, int ELEM, int MODE>
-__global__ void __launch_bounds__(kPanelWarps * 32)
+__global__ void __launch_bounds__(kPanelWarpsH * 32)
 k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Err) {
   __shared__ float4 tab[256];
   __shared__ float Us[kPanel][kPanel + 1];
   __shared__ float hs[kPanel];
-  __shared__ float wb[kPanelWarps][32];
-  __shared__ float errs[kPanelWarps][32];
-  __shared__ uint8_t surv[kPanelWarps][256];   // codes left after the bounds, ascending
+  __shared__ float wb[kPanelWarpsH][2][32];
+  __shared__ float errs[kPanelWarpsH][2][32];
+  __shared__ uint8_t surv[kPanelWarpsH][2][256];   // codes left after the bounds, ascending
   for (int c = threadIdx.x; c < T.ncodes; c += blockDim.x) tab[c] = T.c[c];
   for (int e = threadIdx.x; e < kPanel * kPanel; e += blockDim.x) {
     const int i = e / kPanel, j = e % kPanel;
@@ -665,59 +674,75 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Er
     hs[i] = (MODE == 2 && i < S) ? a.h[pos_col<B>(a, p0 + i)] : 1.0f;
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t r = (int64_t)blockIdx.x * kPanelWarps + wid;
-  if (r >= a.n) return;
+  const int hf = lane >> 4, sl = lane & 15;
+  const int64_t r = (int64_t)blockIdx.x * (2 * kPanelWarpsH) + 2 * wid + hf;
+  const bool row_ok = r < a.n;
+  if (__ballot_sync(kFull, row_ok) == 0) return;   // both of the warp's rows past the end
   const int64_t kb = a.k / B;
-  float* wrow = a.Wc + r * a.k + p0;
-  const bool live = 2 * lane < S;
-  float2 w = live ? *reinterpret_cast<const float2*>(wrow + 2 * lane) : make_float2(0.f, 0.f);
-  float2 err2 = make_float2(0.f, 0.f);
-  uint32_t nib = 0;                       // the lane's two nibbles
+  const bool live = row_ok && 4 * sl < S;
+  float w[4] = {0.f, 0.f, 0.f, 0.f};
+  if (live) {
+    const float4 v = *reinterpret_cast<const float4*>(a.Wc + r * a.k + p0 + 4 * sl);
+    w[0] = v.x;
+    w[1] = v.y;
+    w[2] = v.z;
+    w[3] = v.w;
+  }
+  float errv[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t nib = 0;                       // the lane's four nibbles
+  float* wbh = wb[wid][hf];
+  float* erh = errs[wid][hf];
+  uint8_t* svh = surv[wid][hf];
   for (int bb = 0; bb * B < S; ++bb) {
     const int q0 = bb * B;                // the block's first panel position
-    const bool mine = 2 * lane >= q0 && 2 * lane < q0 + B;
+    const bool mine = 4 * sl >= q0 && 4 * sl < q0 + B;
     if (mine) {
-      wb[wid][2 * lane - q0] = w.x;
-      wb[wid][2 * lane - q0 + 1] = w.y;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) wbh[4 * sl - q0 + c] = w[c];
     }
     __syncwarp();
     float amax = 0.0f;
 #pragma unroll 4
-    for (int j = 0; j < B; ++j) amax = fmaxf(amax, fabsf(wb[wid][j]));
+    for (int j = 0; j < B; ++j) amax = fmaxf(amax, fabsf(wbh[j]));
     const int c0 = naive_code<ELEM>(amax, tab, T.ncodes, T.sfmt);
     int cbest = c0;
     if (MODE != 0) {
       int lo, hi;
       grid_window(tab, T.ncodes, T.first, c0, a.window, lo, hi);
-      // (1) a window of 32 codes from just below the naive code, one per lane, in full
+      // (1) a window of 32 codes from just below the naive code, two per lane, in full
       const int ws = max(lo, min(c0 - kPanWinBelow, hi - 31)), we = min(hi, ws + 31);
       double be = __longlong_as_double(0x7ff0000000000000LL);   // +inf
       int bc = 0x7fffffff;
-      if (ws + lane <= we) {
-        be = exact_error1<B, ELEM, MODE == 2>(wb[wid], hs + q0, tab[ws + lane]);
-        bc = ws + lane;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int c = ws + sl + 16 * t;
+        if (c <= we) {
+          const double e = exact_error1<B, ELEM, MODE == 2>(wbh, hs + q0, tab[c]);
+          if (e < be) { be = e; bc = c; }
+        }
       }
-      warp_argmin(be, bc);
-      // (2) the codes outside the window: a candidate's error is at least that of its two
-      // elements with the largest c a^2 (the same double terms the full sum adds, so the
-      // bound minus 2^-45 relative lies below its full sum); those whose bound exceeds the
-      // best error so far can neither win nor tie and are dropped, the rest are listed
-      if (lo < ws || we < hi) {
+      half_argmin(be, bc);
+      // (2) the codes outside the window, by the two-element bounds; the loop runs over the
+      // union of both halves' ranges so that every lane takes part in the ballots
+      const bool need = lo < ws || we < hi;
+      if (__any_sync(kFull, need)) {
         float2 top = make_float2(0.f, 0.f), ctop = make_float2(0.f, 0.f);
         {
           float v1 = -1.f, v2 = -1.f;
           for (int j = 0; j < B; ++j) {
-            const float aj = fabsf(wb[wid][j]), cj = MODE == 2 ? hs[q0 + j] : 1.f;
+            const float aj = fabsf(wbh[j]), cj = MODE == 2 ? hs[q0 + j] : 1.f;
             const float v = cj * aj * aj;
             if (v > v1) { v2 = v1; top.y = top.x; ctop.y = ctop.x; v1 = v; top.x = aj; ctop.x = cj; }
             else if (v > v2) { v2 = v; top.y = aj; ctop.y = cj; }
           }
         }
         const double bound_cut = be;
+        const int lo_u = min(lo, __shfl_xor_sync(kFull, lo, 16));
+        const int hi_u = max(hi, __shfl_xor_sync(kFull, hi, 16));
         int total = 0;
-        for (int cb = lo; cb <= hi; cb += 32) {
-          const int c = cb + lane;
-          const bool in = c <= hi && (c < ws || c > we);
+        for (int cb = lo_u; cb <= hi_u; cb += 16) {
+          const int c = cb + sl;
+          const bool in = need && c >= lo && c <= hi && (c < ws || c > we);
           bool keep = false;
           if (in) {
             const float2 wq = pair_project<ELEM>(top, tab[c]);
@@ -728,70 +753,73 @@ k_gptq_panel(SweepArgs a, GridTable T, int64_t p0, int S, float* __restrict__ Er
                                         MODE == 2 ? __dmul_rn((double)ctop.y, s1) : s1);
             keep = !(lb * (1.0 - 0x1p-45) > bound_cut);
           }
-          const unsigned m = __ballot_sync(kFull, keep);
-          if (keep) surv[wid][total + __popc(m & ((1u << lane) - 1u))] = (uint8_t)c;
+          const unsigned m = (__ballot_sync(kFull, keep) >> (16 * hf)) & 0xffffu;
+          if (keep) svh[total + __popc(m & ((1u << sl) - 1u))] = (uint8_t)c;
           total += __popc(m);
         }
         __syncwarp();
-        // (3) the survivors in full, 32 at a time
-        for (int i = lane; i < total; i += 32) {
-          const int c = surv[wid][i];
-          const double e = exact_error1<B, ELEM, MODE == 2>(wb[wid], hs + q0, tab[c]);
+        // (3) the survivors in full, 16 at a time per row
+        for (int i = sl; i < total; i += 16) {
+          const int c = svh[i];
+          const double e = exact_error1<B, ELEM, MODE == 2>(wbh, hs + q0, tab[c]);
           if (e < be || (e == be && c < bc)) { be = e; bc = c; }
         }
-        warp_argmin(be, bc);
+        half_argmin(be, bc);
         __syncwarp();
       }
       cbest = bc == 0x7fffffff ? lo : bc;
     }
     const float4 t = tab[cbest];
     const int64_t blk = pos_col<B>(a, p0 + q0) / B;   // the block's index in W
-    if (lane == 0) a.scales[r * kb + blk] = (uint8_t)cbest;
-    // the block's columns, one after another
-#pragma unroll 1
+    if (row_ok && sl == 0) a.scales[r * kb + blk] = (uint8_t)cbest;
+    // the block's columns, one after another (the owner lane of each row divides, the
+    // residual is broadcast within the half)
+#pragma unroll
     for (int j = 0; j < B; ++j) {
       const int q = q0 + j;
-      const int owner = q >> 1;
+      const int owner = q >> 2;
+      const int comp = j & 3;             // q0 is a multiple of 4: q & 3 == j & 3
       float err = 0.0f;
-      if (lane == owner) {
-        const float wv = (q & 1) ? w.y : w.x;
+      if (sl == owner) {
+        const float wv = w[comp];
         float wq_abs;
         const int code = elem_project<ELEM>(fabsf(wv), t, wq_abs);
         const uint32_t neg = __float_as_uint(wv) >> 31;
         const uint32_t nb = ELEM == kElemE2M1 ? ((neg << 3) | (uint32_t)code)
                                               : ((uint32_t)(neg ? -code : code) & 15u);
-        nib |= nb << (4 * (q & 1));
+        nib |= nb << (4 * comp);
         err = __fdiv_rn(__fsub_rn(wv, copysignf(wq_abs, wv)), Us[q][q]);
-        if (q & 1) err2.y = err; else err2.x = err;
-        errs[wid][j] = err;
+        errv[comp] = err;
+        erh[j] = err;
       }
-      err = __shfl_sync(kFull, err, owner);
+      err = __shfl_sync(kFull, err, (lane & 16) | owner);
       // in-block updates of the later columns: w -= fl32(err U)
       if (mine) {
-        const int qa = 2 * lane, qb = 2 * lane + 1;
-        if (qa > q) w.x = __fsub_rn(w.x, __fmul_rn(err, Us[q][qa]));
-        if (qb > q) w.y = __fsub_rn(w.y, __fmul_rn(err, Us[q][qb]));
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (4 * sl + c > q) w[c] = __fsub_rn(w[c], __fmul_rn(err, Us[q][4 * sl + c]));
       }
     }
     __syncwarp();
     // the block's product into the panel's later blocks: acc = sum_j fma, one subtraction
-    if (live && 2 * lane >= q0 + B) {
-      float acc0 = 0.0f, acc1 = 0.0f;
+    if (live && 4 * sl >= q0 + B) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
       for (int j = 0; j < B; ++j) {
-        const float e = errs[wid][j];
-        acc0 = __fmaf_rn(e, Us[q0 + j][2 * lane], acc0);
-        acc1 = __fmaf_rn(e, Us[q0 + j][2 * lane + 1], acc1);
+        const float e = erh[j];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[c] = __fmaf_rn(e, Us[q0 + j][4 * sl + c], acc[c]);
       }
-      w.x = __fsub_rn(w.x, acc0);
-      w.y = __fsub_rn(w.y, acc1);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) w[c] = __fsub_rn(w[c], acc[c]);
     }
     __syncwarp();
   }
   if (live) {
-    const int64_t c = pos_col<B>(a, p0 + 2 * lane);    // even: both nibbles share a byte
-    a.codes[r * (a.k / 2) + c / 2] = (uint8_t)nib;
-    *reinterpret_cast<float2*>(Err + r * kPanel + 2 * lane) = err2;
+    const int64_t c = pos_col<B>(a, p0 + 4 * sl);     // four positions of one block
+    *reinterpret_cast<uint16_t*>(a.codes + r * (a.k / 2) + c / 2) = (uint16_t)nib;
+    *reinterpret_cast<float4*>(Err + r * kPanel + 4 * sl) =
+        make_float4(errv[0], errv[1], errv[2], errv[3]);
   }
 }
 
@@ -928,15 +956,15 @@ cudaError_t sweep_dispatch(const SweepArgs& a, const GridTable& T, int mode, cud
   cudaStreamWaitEvent(fs.side, e0, 0);
   cudaEvent_t ev_rest = nullptr;
   k_sweep_init<B><<<sm_count() * 8, 256, 0, cs>>>(a);
-  const unsigned prow = (unsigned)((a.n + kPanelWarps - 1) / kPanelWarps);
+  const unsigned prow = (unsigned)((a.n + 2 * kPanelWarpsH - 1) / (2 * kPanelWarpsH));
   bool rest_pending = false;
   int t = 0;
   for (int64_t p0 = 0; p0 < a.k; p0 += kPanel, ++t) {
     const int S = (int)(a.k - p0 < kPanel ? a.k - p0 : kPanel);
     float* err = a.Err + (t & 1) * a.n * kPanel;
-    if (mode == 0) k_gptq_panel<B, ELEM, 0><<<prow, kPanelWarps * 32, 0, cs>>>(a, T, p0, S, err);
-    else if (mode == 1) k_gptq_panel<B, ELEM, 1><<<prow, kPanelWarps * 32, 0, cs>>>(a, T, p0, S, err);
-    else k_gptq_panel<B, ELEM, 2><<<prow, kPanelWarps * 32, 0, cs>>>(a, T, p0, S, err);
+    if (mode == 0) k_gptq_panel<B, ELEM, 0><<<prow, kPanelWarpsH * 32, 0, cs>>>(a, T, p0, S, err);
+    else if (mode == 1) k_gptq_panel<B, ELEM, 1><<<prow, kPanelWarpsH * 32, 0, cs>>>(a, T, p0, S, err);
+    else k_gptq_panel<B, ELEM, 2><<<prow, kPanelWarpsH * 32, 0, cs>>>(a, T, p0, S, err);
     const int64_t c1 = p0 + S, c2 = c1 + kPanel < a.k ? c1 + kPanel : a.k;
     if (c1 >= a.k) break;
     if (rest_pending) cudaStreamWaitEvent(cs, ev_rest, 0);
