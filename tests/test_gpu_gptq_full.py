@@ -184,6 +184,21 @@ def test_sweep_bit_exact_larger(mxq, orc, synth, n, k, B, dtype):
     assert np.array_equal(codes.cpu().numpy(), r.codes)
 
 
+@pytest.mark.parametrize("n,k,B,mode", [(1, 16, 16, "hopt"), (2, 32, 32, "sse"), (3, 48, 16, "hopt"),
+                                        (5, 96, 32, "hopt"), (6, 16, 16, "naive")])
+def test_sweep_small_shapes(mxq, orc, synth, n, k, B, mode):
+    """Rows that leave half-warps and whole warps of the panel kernel without a row (the
+    kernel takes one half-warp per row, four rows per CTA), and inputs narrower than one
+    panel of 64 positions (a single partial panel, no trailing update)."""
+    W, h, U, perm = sweep_case(orc, synth, n, k, B, 133 + n, torch.bfloat16, False)
+    p = mxq.params("nvfp4", mode, B)
+    codes, scales = mxq.mxq_gptq(W, torch.from_numpy(U).to(DEV), p, torch.from_numpy(h).to(DEV))
+    torch.cuda.synchronize()
+    r = orc.gptq_blocks(oracle_view(W), U, h, "nvfp4", mode, B)
+    assert np.array_equal(scales.cpu().numpy(), r.scales)
+    assert np.array_equal(codes.cpu().numpy(), r.codes)
+
+
 def test_sweep_worked_examples(mxq):
     """The oracle's hand-derived cases: the residual changes the next block's scale
     (0x33, not 0x35) and an in-block code; one product per block past the block."""
