@@ -109,7 +109,8 @@ def test_gram_strided_columns(mxq, orc, synth):
 
 
 @pytest.mark.parametrize("k,B,ordered", [(64, 16, False), (256, 16, True), (1024, 32, True),
-                                         (208, 16, False), (1008, 16, True)])
+                                         (208, 16, False), (1008, 16, True), (1088, 16, False),
+                                         (1280, 32, True)])
 def test_factor_matches_oracle(mxq, orc, synth, k, B, ordered):
     X = correlated_x(synth, 4 * k, k, 122, "cpu")
     H = orc.gram(oracle_view(X))
@@ -119,6 +120,29 @@ def test_factor_matches_oracle(mxq, orc, synth, k, B, ordered):
     pd = None if perm is None else torch.from_numpy(perm).to(DEV)
     U = mxq.mxq_gptq_factor(torch.from_numpy(H).to(DEV), B, pd).cpu().numpy()
     check_factor(U, ref)
+
+
+def test_factor_and_sweep_enqueued_ahead(mxq, orc, synth):
+    """Several factor + sweep calls enqueued back to back with no synchronisation (the host
+    runs far ahead of the GPU, and the library's ring of events wraps around more than
+    once): every call's outputs equal those of a call made alone."""
+    n, k, B = 40, 1024, 16
+    W, h, U0, _ = sweep_case(orc, synth, n, k, B, 141, torch.bfloat16, False)
+    X = correlated_x(synth, 4 * k, k, 142, "cpu")
+    H = torch.from_numpy(orc.gram(oracle_view(X))).to(DEV)
+    hd = torch.from_numpy(h).to(DEV)
+    p = mxq.params("nvfp4", "hopt", B)
+    U_ref = mxq.mxq_gptq_factor(H, B)
+    c_ref, s_ref = mxq.mxq_gptq(W, U_ref, p, hd)
+    torch.cuda.synchronize()
+    outs = []
+    for _ in range(6):
+        U = mxq.mxq_gptq_factor(H, B)
+        outs.append((U,) + tuple(mxq.mxq_gptq(W, U, p, hd)))
+    torch.cuda.synchronize()
+    for U, c, s in outs:
+        assert torch.equal(U, U_ref)
+        assert torch.equal(c, c_ref) and torch.equal(s, s_ref)
 
 
 def test_factor_degenerate(mxq, orc):
